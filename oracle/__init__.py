@@ -1,0 +1,356 @@
+"""CPU oracle for the ZeRO stage-1/2 data-parallel step (TEST INFRASTRUCTURE ONLY).
+
+Only tests/, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
+this package. It never imports the CUDA library and the library never imports it; they share
+only the seeded input generators, which hold none of the method's arithmetic.
+
+The element arithmetic is plain C (``oracle.c``, built by ``oracle/build.py``); this module
+adds the partitioning that ZeRO-DP performs around it, written with numpy slicing:
+
+* ``dp_step``      -- plain data parallelism: every replica all-reduces the full gradient and
+                      updates the full model ("ZeRO: particionar estados do treino entre GPUs",
+                      section "Como funciona": the baseline DP keeps a full replica).
+* ``zero1_step``   -- stage 1 (Pos): full local gradients, one reduce-scatter at the step, each
+                      owner updates its 1/Nd shard, an all-gather writes every updated fp16
+                      shard back ("Como funciona"; "ZeRO-2" card, "ZeRO-1에서 남은 낭비").
+* ``zero2_step``   -- stage 2 (Pos+g): buckets in backward order, each reduce-scattered as soon
+                      as it is produced, the owner keeps its slice and the rest is released;
+                      then the owner update and the all-gather ("ZeRO-2" card, "Gradient
+                      생명주기" and "왜 all-gather는 그대로 필요한가").
+
+All three produce the same numbers ("ZeRO" (lastdictionary), "Usage note": ZeRO changes where
+state is stored, not how updates are computed); the pins in tests/test_oracle_pins.py check it.
+
+Parity status: every function here is pinned (see tests/test_oracle_pins.py).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import dataclasses
+import os
+from typing import Callable, List, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+SKIPPED = 1
+
+
+def lib():
+    """Load (building first if needed) the oracle's shared library."""
+    global _lib
+    if _lib is None:
+        _lib = bind(_build.build())
+    return _lib
+
+
+def bind(path: str):
+    """Open a build of oracle.c and declare its C signatures."""
+    L = C.CDLL(path)
+    u64, i64, f32p, u16p = C.c_uint64, C.c_int64, C.POINTER(C.c_float), C.POINTER(C.c_uint16)
+    L.orc_h2f.argtypes, L.orc_h2f.restype = [C.c_uint16], C.c_float
+    L.orc_f2h.argtypes, L.orc_f2h.restype = [C.c_float], C.c_uint16
+    L.orc_h2f_array.argtypes = [u64, u16p, f32p]
+    L.orc_f2h_array.argtypes = [u64, f32p, u16p]
+    L.orc_state_bytes.argtypes = [u64, C.c_int, C.c_int, C.POINTER(u64), C.POINTER(u64)]
+    L.orc_plan.argtypes = [C.POINTER(u64), C.c_int, C.c_int, u64, C.POINTER(u64),
+                           C.POINTER(u64), C.POINTER(u64), C.POINTER(u64), C.POINTER(i64)]
+    L.orc_bucket.argtypes = [u64, u64, i64, C.POINTER(u64), C.POINTER(u64)]
+    L.orc_adam_scalars.argtypes = [C.c_void_p, i64, C.c_void_p]
+    L.orc_reduce_mean.argtypes = [u64, C.c_int, C.POINTER(u16p), f32p]
+    L.orc_all_finite.argtypes, L.orc_all_finite.restype = [u64, f32p], C.c_int
+    L.orc_adam.argtypes = [u64, f32p, f32p, f32p, f32p, u16p, C.c_void_p]
+    L.orc_step.argtypes = [u64, C.c_int, C.POINTER(u16p), f32p, f32p, f32p, u16p,
+                           C.c_void_p, i64, f32p]
+    return L
+
+
+class _HP(C.Structure):
+    _fields_ = [("lr", C.c_double), ("beta1", C.c_double), ("beta2", C.c_double),
+                ("eps", C.c_double), ("loss_scale", C.c_double)]
+
+
+class _Scalars(C.Structure):
+    _fields_ = [(k, C.c_float) for k in
+                ("b1", "omb1", "b2", "omb2", "step_size", "bc2s", "eps", "loss_scale")]
+
+
+@dataclasses.dataclass(frozen=True)
+class AdamHP:
+    """Adam hyperparameters and the static loss scale (defaults: the tiny stage-1 workload)."""
+    lr: float = 1e-3
+    beta1: float = 0.9
+    beta2: float = 0.999
+    eps: float = 1e-8
+    loss_scale: float = 1024.0
+
+    def _c(self) -> _HP:
+        return _HP(self.lr, self.beta1, self.beta2, self.eps, self.loss_scale)
+
+
+def _f32p(a):
+    return a.ctypes.data_as(C.POINTER(C.c_float))
+
+
+def _u16p(a):
+    return a.ctypes.data_as(C.POINTER(C.c_uint16))
+
+
+def _as_u16(a) -> np.ndarray:
+    a = np.asarray(a)
+    if a.dtype == np.float16:
+        a = a.view(np.uint16)
+    assert a.dtype == np.uint16, a.dtype
+    return np.ascontiguousarray(a)
+
+
+# ---------------------------------------------------------------------------------------------
+# binary16 conversion
+# ---------------------------------------------------------------------------------------------
+def h2f(h) -> np.ndarray:
+    h = _as_u16(h)
+    out = np.empty(h.shape, np.float32)
+    lib().orc_h2f_array(h.size, _u16p(h), _f32p(out))
+    return out
+
+
+def f2h(x) -> np.ndarray:
+    """binary32 -> binary16 bits (uint16), round to nearest even."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, np.uint16)
+    lib().orc_f2h_array(x.size, _f32p(x), _u16p(out))
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
+# accounting and plan
+# ---------------------------------------------------------------------------------------------
+STAGES = ("dp", "pos", "pos_g", "pos_g_p")
+
+
+def state_bytes(psi: int, nd: int, K: int = 12) -> dict:
+    """Per-device bytes of each stage and the per-step communication volume (elements)."""
+    b = (C.c_uint64 * 16)()
+    c = (C.c_uint64 * 4)()
+    rc = lib().orc_state_bytes(psi, nd, K, b, c)
+    if rc:
+        raise ValueError("orc_state_bytes: invalid arguments")
+    out = {}
+    for s, name in enumerate(STAGES):
+        out[name] = dict(params=b[4 * s], grads=b[4 * s + 1], optim=b[4 * s + 2],
+                         total=b[4 * s + 3], comm_elems=c[s])
+    return out
+
+
+@dataclasses.dataclass
+class Plan:
+    numels: List[int]
+    nd: int
+    bucket_elems: int
+    tensor_off: List[int]
+    psi: int
+    psi_p: int
+    shard: int
+    buckets: List[tuple]   # (lo, len) in backward order: bucket 0 is produced first
+
+    def owners(self, k: int) -> tuple:
+        lo, ln = self.buckets[k]
+        return lo // self.shard, (lo + ln - 1) // self.shard
+
+
+def plan(numels: Sequence[int], nd: int, bucket_elems: int = 0) -> Plan:
+    n = len(numels)
+    arr = (C.c_uint64 * max(n, 1))(*numels)
+    off = (C.c_uint64 * max(n, 1))()
+    psi, psi_p, shard = C.c_uint64(), C.c_uint64(), C.c_uint64()
+    nb = C.c_int64()
+    rc = lib().orc_plan(arr, n, nd, bucket_elems, off, C.byref(psi), C.byref(psi_p),
+                        C.byref(shard), C.byref(nb))
+    if rc:
+        raise ValueError("orc_plan: invalid arguments")
+    buckets = []
+    for k in range(nb.value):
+        lo, ln = C.c_uint64(), C.c_uint64()
+        if lib().orc_bucket(psi_p.value, bucket_elems, k, C.byref(lo), C.byref(ln)):
+            raise ValueError("orc_bucket failed")
+        buckets.append((lo.value, ln.value))
+    return Plan(list(numels), nd, bucket_elems, list(off[:n]), psi.value, psi_p.value,
+                shard.value, buckets)
+
+
+# ---------------------------------------------------------------------------------------------
+# element arithmetic
+# ---------------------------------------------------------------------------------------------
+def adam_scalars(hp: AdamHP, t: int) -> dict:
+    s = _Scalars()
+    h = hp._c()
+    if lib().orc_adam_scalars(C.byref(h), t, C.byref(s)):
+        raise ValueError("step t must be >= 1")
+    return {k: getattr(s, k) for k, _ in _Scalars._fields_}
+
+
+def reduce_mean(grads: Sequence[np.ndarray]) -> np.ndarray:
+    """Rank-ordered binary32 mean of Nd fp16 gradients (given as float16 or uint16 arrays)."""
+    gs = [_as_u16(g) for g in grads]
+    n = gs[0].size
+    assert all(g.size == n for g in gs)
+    ptrs = (C.POINTER(C.c_uint16) * len(gs))(*[_u16p(g) for g in gs])
+    red = np.empty(n, np.float32)
+    lib().orc_reduce_mean(n, len(gs), ptrs, _f32p(red))
+    return red
+
+
+def all_finite(x: np.ndarray) -> bool:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    return bool(lib().orc_all_finite(x.size, _f32p(x)))
+
+
+def adam(red, master, m, v, hp: AdamHP, t: int):
+    """Owner update from reduced gradients; returns new (master, m, v, p16) copies."""
+    s = _Scalars()
+    h = hp._c()
+    if lib().orc_adam_scalars(C.byref(h), t, C.byref(s)):
+        raise ValueError("step t must be >= 1")
+    red = np.ascontiguousarray(red, np.float32)
+    w, mm, vv = (np.array(a, dtype=np.float32, copy=True) for a in (master, m, v))
+    p16 = np.empty(red.size, np.uint16)
+    lib().orc_adam(red.size, _f32p(red), _f32p(w), _f32p(mm), _f32p(vv), _u16p(p16),
+                   C.byref(s))
+    return w, mm, vv, p16
+
+
+def step(grads, master, m, v, hp: AdamHP, t: int):
+    """One owner step on a range: returns (skipped, master, m, v, p16 or None)."""
+    gs = [_as_u16(g) for g in grads]
+    n = gs[0].size
+    ptrs = (C.POINTER(C.c_uint16) * len(gs))(*[_u16p(g) for g in gs])
+    w, mm, vv = (np.array(a, dtype=np.float32, copy=True) for a in (master, m, v))
+    p16 = np.empty(n, np.uint16)
+    scratch = np.empty(n, np.float32)
+    h = _HP(hp.lr, hp.beta1, hp.beta2, hp.eps, hp.loss_scale)
+    rc = lib().orc_step(n, len(gs), ptrs, _f32p(w), _f32p(mm), _f32p(vv), _u16p(p16),
+                        C.byref(h), t, _f32p(scratch))
+    if rc < 0:
+        raise ValueError("step t must be >= 1")
+    if rc == SKIPPED:
+        return True, np.array(master, np.float32), np.array(m, np.float32), \
+            np.array(v, np.float32), None
+    return False, w, mm, vv, p16
+
+
+# ---------------------------------------------------------------------------------------------
+# whole-model steps: plain DP and the two ZeRO-DP stages
+# ---------------------------------------------------------------------------------------------
+@dataclasses.dataclass
+class Result:
+    skipped: bool
+    master: np.ndarray
+    m: np.ndarray
+    v: np.ndarray
+    params16: np.ndarray                 # the full fp16 parameter buffer every replica holds
+    reduced: np.ndarray = None           # reduced gradient as kept by its owner (psi_p floats)
+
+
+def dp_step(local_grads, master, m, v, params16, hp: AdamHP, t: int) -> Result:
+    """Plain DP: all-reduce (mean) the full gradient, then every replica updates everything.
+
+    local_grads: Nd arrays of psi_p fp16 values (one full local gradient per rank).
+    """
+    red = reduce_mean(local_grads)
+    if not all_finite(red):
+        return Result(True, np.array(master, np.float32), np.array(m, np.float32),
+                      np.array(v, np.float32), np.array(params16, np.uint16), red)
+    w, mm, vv, p16 = adam(red, master, m, v, hp, t)
+    return Result(False, w, mm, vv, p16, red)
+
+
+def zero1_step(pl: Plan, local_grads, master, m, v, params16, hp: AdamHP, t: int) -> Result:
+    """Stage 1: one reduce-scatter of the full local gradients at the step.
+
+    The state arrays hold the Nd owners' shards end to end (owner r: [r*S, (r+1)*S)).
+    """
+    S, nd = pl.shard, pl.nd
+    gs = [_as_u16(g) for g in local_grads]
+    assert len(gs) == nd and all(g.size == pl.psi_p for g in gs)
+    # reduce-scatter: owner r receives rank j's slice r of the local gradient, for every j
+    shards = []
+    for r in range(nd):
+        shards.append(reduce_mean([g[r * S:(r + 1) * S] for g in gs]))
+    # one verdict for the whole step, over every owner's shard
+    if not all(all_finite(sh) for sh in shards):
+        return Result(True, np.array(master, np.float32), np.array(m, np.float32),
+                      np.array(v, np.float32), np.array(params16, np.uint16),
+                      np.concatenate(shards))
+    w_out = np.array(master, np.float32)
+    m_out = np.array(m, np.float32)
+    v_out = np.array(v, np.float32)
+    p_out = np.array(params16, np.uint16)
+    for r in range(nd):
+        sl = slice(r * S, (r + 1) * S)
+        w, mm, vv, p16 = adam(shards[r], master[sl], m[sl], v[sl], hp, t)
+        w_out[sl], m_out[sl], v_out[sl] = w, mm, vv
+        p_out[sl] = p16           # all-gather: owner r's updated fp16 shard into the full buffer
+    return Result(False, w_out, m_out, v_out, p_out, np.concatenate(shards))
+
+
+def zero2_step(pl: Plan, bucket_grad: Callable[[int, int], np.ndarray], master, m, v, params16,
+               hp: AdamHP, t: int) -> Result:
+    """Stage 2: buckets in backward order; each is reduce-scattered when produced.
+
+    bucket_grad(k, rank) returns rank's local fp16 gradient for bucket k (pl.buckets[k][1]
+    values). After the reduce-scatter of bucket k only the owners' reduced slices are kept;
+    the local bucket gradients are dropped before the next bucket is produced.
+    """
+    S, nd = pl.shard, pl.nd
+    grad_shard = [np.zeros(S, np.float32) for _ in range(nd)]    # owner r's reduced grad shard
+    for k, (lo, ln) in enumerate(pl.buckets):
+        local = [_as_u16(bucket_grad(k, j)) for j in range(nd)]
+        assert all(g.size == ln for g in local)
+        o_lo, o_hi = lo // S, (lo + ln - 1) // S
+        for r in range(o_lo, o_hi + 1):
+            a, b = max(lo, r * S), min(lo + ln, (r + 1) * S)
+            grad_shard[r][a - r * S:b - r * S] = reduce_mean([g[a - lo:b - lo] for g in local])
+        del local                                                 # release
+    if not all(all_finite(sh) for sh in grad_shard):
+        return Result(True, np.array(master, np.float32), np.array(m, np.float32),
+                      np.array(v, np.float32), np.array(params16, np.uint16),
+                      np.concatenate(grad_shard))
+    w_out = np.array(master, np.float32)
+    m_out = np.array(m, np.float32)
+    v_out = np.array(v, np.float32)
+    p_out = np.array(params16, np.uint16)
+    for r in range(nd):
+        sl = slice(r * S, (r + 1) * S)
+        w, mm, vv, p16 = adam(grad_shard[r], master[sl], m[sl], v[sl], hp, t)
+        w_out[sl], m_out[sl], v_out[sl] = w, mm, vv
+        p_out[sl] = p16
+    return Result(False, w_out, m_out, v_out, p_out, np.concatenate(grad_shard))
+
+
+def ulp_diff_f32(a, b) -> np.ndarray:
+    """Distance in units in the last place between binary32 arrays (ordered-integer metric;
+    two NaNs are 0 apart, NaN vs a number is 2**32)."""
+    a = np.ascontiguousarray(a, np.float32).view(np.int32).astype(np.int64)
+    b = np.ascontiguousarray(b, np.float32).view(np.int32).astype(np.int64)
+    oa = np.where(a < 0, -(a & 0x7fffffff), a)
+    ob = np.where(b < 0, -(b & 0x7fffffff), b)
+    d = np.abs(oa - ob)
+    na = ((a & 0x7f800000) == 0x7f800000) & ((a & 0x7fffff) != 0)
+    nb = ((b & 0x7f800000) == 0x7f800000) & ((b & 0x7fffff) != 0)
+    d = np.where(na & nb, 0, np.where(na ^ nb, 1 << 32, d))
+    return d
+
+
+def ulp_diff_f16(a, b) -> np.ndarray:
+    """Same metric for binary16 bit patterns (uint16 or float16 arrays)."""
+    a = _as_u16(a).astype(np.int64)
+    b = _as_u16(b).astype(np.int64)
+    oa = np.where(a & 0x8000, -(a & 0x7fff), a)
+    ob = np.where(b & 0x8000, -(b & 0x7fff), b)
+    d = np.abs(oa - ob)
+    na = ((a & 0x7c00) == 0x7c00) & ((a & 0x3ff) != 0)
+    nb = ((b & 0x7c00) == 0x7c00) & ((b & 0x3ff) != 0)
+    return np.where(na & nb, 0, np.where(na ^ nb, 1 << 32, d))
