@@ -1,0 +1,455 @@
+#!/usr/bin/env python
+"""Throughput of the fused ZeRO shard step on B200: params/s, HBM GB/s and the fraction of
+the measured HBM roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gpt2_small|shard_7p5b|flat] [--nd ND] [--bucket B]
+
+One step is one pass of the whole hot path over one batch of synthetic input: the
+reduce-scatter of the Nd simulated ranks' fp16 gradients, the unscale, the fp32 Adam update of
+every owner's shard, the fp16 cast and the all-gather write-back into the full parameter buffer
+(zero_step_fused over the step's range(s), then zero_step_commit), all resident in HBM.
+
+Workloads (synthetic, seeded):
+  gpt2_small  GPT-2-small parameter list (psi = 123,653,376), Nd = 8, stage 1 (full local
+              gradients, one fused call per step); grads N(0, 1e-3^2) with 1% x100; master
+              N(0, 0.02^2), m = v = 0 at the start.               (default)
+  shard_7p5b  one owner's view of 7.5e9 parameters at Nd = 64: a 117,187,500-element shard,
+              64 separate fp16 gradient slices, written into a 7.5e9-element fp16 buffer at
+              r*S (r = 31); master U(-0.05, 0.05), m N(0, 1e-4^2), v |N(0, 1e-6^2)|.
+  flat        psi = 2^29 flat buffer, one fused call per bucket of B elements in backward
+              order, Nd in {2, 4, 8, 16, 64}; state as shard_7p5b.
+
+Every step reads and writes far more than the 126 MB L2 (5.2 GB for gpt2_small), so no L2 flush
+is needed between steps. With N > 1 (torchrun), every rank runs its own replica of the
+simulated Nd-rank step on its own GPU (the Nd ranks are simulated on one device; no data
+crosses GPUs), and the time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SRC = os.path.join(ROOT, "zero_partitioned_optimizer_plan_b200", "csrc", "zero_kernels.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+METRIC = "fused ZeRO shard step params/sec"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["gpt2_small", "shard_7p5b", "flat"],
+                    default="gpt2_small")
+    ap.add_argument("--nd", type=int, default=None)
+    ap.add_argument("--bucket", type=int, default=None)
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return a
+
+
+# ---------------------------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------------------------
+class Workload:
+    """Device buffers and the per-step call sequence of one workload."""
+
+    def __init__(self, args, dev):
+        import torch
+        from zero_partitioned_optimizer_plan_b200 import libzero as lz
+        from zero_partitioned_optimizer_plan_b200 import synth
+        self.torch, self.lz, self.dev = torch, lz, dev
+        self.hp = lz.AdamHP()
+        kind = args.workload
+        self.kind = kind
+        if kind == "gpt2_small":
+            nd = args.nd or 8
+            numels = synth.gpt2_small_list()
+            pl = lz.zero_plan_create(numels, nd, 1, 0)
+            psi, psi_p, S, nb = lz.zero_plan_info(pl)
+            self.nd, self.n, self.psi = nd, psi_p, psi
+            self.ranges = [(0, psi_p)]
+            self.grads = []
+            for r in range(nd):
+                g = torch.zeros(psi_p, dtype=torch.float16, device=dev)
+                synth.grad_f16(psi, 1e-3, seed=0, rank=r, step=1, spike_frac=0.01,
+                               spike_scale=100.0, out=g[:psi])
+                self.grads.append(g)
+            master, m, v = synth.state_small(psi_p, seed=0, device=dev)
+            self.params = torch.empty(psi_p, dtype=torch.float16, device=dev)
+            self.param_base = 0
+            self.config = {"workload": "gpt2_small_stage1", "psi": psi, "nd": nd, "stage": 1,
+                           "calls_per_step": 1, "tensors": len(numels)}
+        elif kind == "shard_7p5b":
+            nd = args.nd or 64
+            total = 7_500_000_000
+            S = total // nd
+            r = 31
+            self.nd, self.n, self.psi = nd, S, S
+            self.ranges = [(0, S)]
+            self.grads = [synth.grad_f16(S, 1e-3, seed=0, rank=j, step=1, device=dev)
+                          for j in range(nd)]
+            master, m, v = synth.state_warm(S, seed=0, device=dev)
+            self.full = torch.zeros(total, dtype=torch.float16, device=dev)
+            self.params = self.full[r * S:(r + 1) * S]
+            self.param_base = r * S
+            self.config = {"workload": "shard_7p5b_rank31", "psi_total": total, "shard": S,
+                           "nd": nd, "owner": r, "calls_per_step": 1}
+        else:
+            nd = args.nd or 16
+            psi = 1 << 29
+            B = args.bucket or (1 << 26)
+            self.nd, self.n, self.psi = nd, psi, psi
+            self.ranges = []
+            hi = psi
+            while hi > 0:
+                lo = max(0, hi - B)
+                self.ranges.append((lo, hi))
+                hi = lo
+            self.grads = [synth.grad_f16(psi, 1e-3, seed=0, rank=j, step=1, device=dev)
+                          for j in range(nd)]
+            master, m, v = synth.state_warm(psi, seed=0, device=dev)
+            self.params = torch.empty(psi, dtype=torch.float16, device=dev)
+            self.param_base = 0
+            self.config = {"workload": "flat_2p29", "psi": psi, "nd": nd, "bucket": B,
+                           "calls_per_step": len(self.ranges)}
+        self.cur = [master, m, v]
+        self.nxt = [torch.empty_like(x) for x in self.cur]
+        self.bytes_per_step = (2 * self.nd + 26) * self.n     # algorithmic HBM bytes
+        self.launches_per_step = len(self.ranges) + 1
+
+    def step(self, t, status, ev=None, grads=None):
+        """Enqueue one step on the current stream; ev = (start, end) events around the fused
+        launches."""
+        lz = self.lz
+        grads = grads or self.grads
+        if ev is not None:
+            ev[0].record()
+        for lo, hi in self.ranges:
+            lz.zero_step_fused(hi - lo, self.nd, [g[lo:hi] for g in grads],
+                               *[x[lo:hi] for x in self.cur], *[x[lo:hi] for x in self.nxt],
+                               self.params[lo:hi], self.hp, t, status)
+        if ev is not None:
+            ev[1].record()
+        lz.zero_step_commit(self.n, *self.cur, *self.nxt, self.params, status)
+        self.cur, self.nxt = self.nxt, self.cur
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks during the timed region (NVML, the data nvidia-smi reports)
+# ---------------------------------------------------------------------------------------------
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+           0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, dev_index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(dev_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # clocks are reported as unavailable, the run still counts
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                bits = get_r(self.h)
+                for b, name in REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def report(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.err}
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------------------------
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_per_launch(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
+    kernel source; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            tab = json.load(f)
+        with open(KERNEL_SRC, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        ent = tab.get(workload, {}).get(kernel)
+        if ent and ent.get("kernel_src_sha256") == sha:
+            return ent["dram_bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+def cpu_oracle_rate(nd: int, n_sample: int, target_s: float, seed=0):
+    """Time the oracle (single-threaded C, as it stands) on n_sample elements of the workload's
+    distribution; repeat until target_s seconds have passed. Returns (params/s, reps, secs)."""
+    import oracle
+    from zero_partitioned_optimizer_plan_b200 import synth
+    g = [synth.grad_f16(n_sample, 1e-3, seed=seed, rank=r, step=1, spike_frac=0.01,
+                        spike_scale=100.0).numpy() for r in range(nd)]
+    master, m, v = (x.numpy() for x in synth.state_small(n_sample, seed=seed))
+    hp = oracle.AdamHP()
+    reps, total = 0, 0.0
+    while total < target_s and reps < 50:
+        t0 = time.perf_counter()
+        skipped, master, m, v, _ = oracle.step(g, master, m, v, hp, reps + 1)
+        total += time.perf_counter() - t0
+        reps += 1
+    return n_sample * reps / total, reps, total
+
+
+def dist_setup(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ---------------------------------------------------------------------------------------------
+# reference arm: the CPU oracle, on the host cores, on a bounded sample per step
+# ---------------------------------------------------------------------------------------------
+def run_reference(args):
+    ws, rank, _ = dist_setup(args)
+    if rank != 0:
+        return 0
+    nd = args.nd or {"gpt2_small": 8, "shard_7p5b": 64, "flat": 16}[args.workload]
+    # calibrate, then size each step so that the whole run takes about two minutes
+    rate, _, _ = cpu_oracle_rate(nd, 200_000, 0.2)
+    per_step_s = max(0.05, 120.0 / (args.steps + args.warmup))
+    n_sample = int(min(16_000_000, max(100_000, rate * per_step_s)))
+    import oracle
+    from zero_partitioned_optimizer_plan_b200 import synth
+    g = [synth.grad_f16(n_sample, 1e-3, seed=0, rank=r, step=1, spike_frac=0.01,
+                        spike_scale=100.0).numpy() for r in range(nd)]
+    master, m, v = (x.numpy() for x in synth.state_small(n_sample, seed=0))
+    hp = oracle.AdamHP()
+    for t in range(1, args.warmup + 1):
+        _, master, m, v, _ = oracle.step(g, master, m, v, hp, t)
+    t0 = time.perf_counter()
+    for t in range(args.warmup + 1, args.warmup + args.steps + 1):
+        _, master, m, v, _ = oracle.step(g, master, m, v, hp, t)
+    dt = time.perf_counter() - t0
+    value = n_sample * args.steps / dt
+    sample = (f"first {n_sample} elements of the {args.workload} workload's distribution, "
+              f"Nd={nd}, one oracle step per timed step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "params/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": args.workload, "nd": nd, "sample_elems": n_sample},
+        "cpu_baseline": {"value": value, "unit": "params/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "params/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    ws, rank, local = dist_setup(args)
+    if ws > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from zero_partitioned_optimizer_plan_b200 import build as zbuild
+    zbuild.build()
+    from zero_partitioned_optimizer_plan_b200 import libzero as lz
+
+    wl = Workload(args, dev)
+    K, W = args.steps, args.warmup
+    status = torch.zeros(K + W, dtype=torch.int32, device=dev)   # one status word per step
+    torch.cuda.synchronize()
+
+    def barrier():
+        if ws > 1:
+            dist.barrier(device_ids=[local])
+
+    # warm-up
+    for i in range(W):
+        wl.step(i + 1, status[i:i + 1])
+    torch.cuda.synchronize()
+
+    # timed region: K steps on torch's current stream
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = lz.zero_kernel_launches()
+    with sampler:
+        start.record()
+        for i in range(K):
+            wl.step(W + i + 1, status[W + i:W + i + 1], ev=evs[i])
+        end.record()
+        torch.cuda.synchronize()
+    launches = lz.zero_kernel_launches() - launches0
+    barrier()
+    ms = start.elapsed_time(end)
+    kernel_ms = [a.elapsed_time(b) for a, b in evs]
+    flags = status.cpu()
+    if int((flags != 0).sum()):
+        raise RuntimeError(f"unexpected status flags in the timed steps: {set(flags.tolist())}")
+    if ws > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / K
+    value = ws * wl.n * K / (ms / 1e3)
+
+    # roofline of the dominant kernel: algorithmic bytes per launch / mean launch time
+    calls = len(wl.ranges)
+    launch_s = statistics.mean(kernel_ms) / 1e3 / calls
+    bytes_per_launch = wl.bytes_per_step / calls
+    peak, peak_kind = measured_peak()
+    achieved = bytes_per_launch / launch_s / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_source": peak_kind,
+                "traffic": traffic_per_launch("fused_tma_kernel", wl.config["workload"]),
+                "kernel": "fused_tma_kernel", "bytes_per_launch": bytes_per_launch,
+                "kernel_ms_mean": launch_s * 1e3}
+
+    # end to end through the public API with host buffers: H2D of the step's gradients from
+    # pinned memory, the step, D2H of the updated fp16 parameters and the status word
+    e2e = None
+    if not args.no_e2e:
+        E = args.e2e_steps or max(3, min(K, 10))
+        h_grads = [torch.empty(g.numel(), dtype=torch.float16, pin_memory=True)
+                   for g in wl.grads]
+        for h, g in zip(h_grads, wl.grads):
+            h.copy_(g)
+        h_params = torch.empty(wl.params.numel(), dtype=torch.float16, pin_memory=True)
+        h_status = torch.empty(1, dtype=torch.int32, pin_memory=True)
+        d_grads = [torch.empty_like(g) for g in wl.grads]
+        st = torch.zeros(E, dtype=torch.int32, device=dev)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(E):
+            for d, h in zip(d_grads, h_grads):
+                d.copy_(h, non_blocking=True)
+            wl.step(W + K + i + 1, st[i:i + 1], grads=d_grads)
+            h_params.copy_(wl.params, non_blocking=True)
+            h_status.copy_(st[i:i + 1], non_blocking=True)
+            torch.cuda.current_stream().synchronize()      # the caller reads the result
+            if int(h_status.item()) != 0:
+                raise RuntimeError("unexpected status in the end-to-end steps")
+        e1.record()
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if ws > 1:
+            t = torch.tensor([ems], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": ws * wl.n * E / (ems / 1e3), "unit": "params/s",
+               "h2d_bytes_per_step": 2 * wl.nd * wl.n, "d2h_bytes_per_step": 2 * wl.n + 4,
+               "steps": E}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        n_sample = 8_000_000
+        rate, reps, secs = cpu_oracle_rate(wl.nd, n_sample, 10.0)
+        cpu = {"value": rate, "unit": "params/s", "cores": 1, "kind": "oracle",
+               "sample": f"{n_sample} elements with the workload's gradient distribution, "
+                         f"Nd={wl.nd}, {reps} oracle steps, {secs:.1f} s"}
+
+    if rank == 0:
+        cfg = dict(wl.config)
+        cfg.update({"l2": "no flush: every step streams (2*Nd+26)*psi bytes, far above L2",
+                    "bytes_per_step": wl.bytes_per_step, "parallelism": f"replicas{ws}",
+                    "hbm_gbs": wl.bytes_per_step / (ms_per_step / 1e3) / 1e9})
+        line = {
+            "metric": METRIC, "value": value, "unit": "params/s", "n_gpus": ws, "steps": K,
+            "warmup": W, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded fp16 gradients and fp32 optimizer state)",
+            "config": cfg, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches, "clocks": sampler.report(),
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

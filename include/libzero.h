@@ -1,0 +1,253 @@
+/*
+ * libzero -- the data-parallel hot path of ZeRO stages 1 and 2 on one NVIDIA B200 (sm_100a).
+ *
+ * ZeRO-DP keeps, per parameter, 2 bytes of fp16 weights, 2 bytes of fp16 gradients and
+ * K = 12 bytes of fp32 optimizer state (master copy, momentum, variance), and partitions that
+ * state among the Nd data-parallel processes: stage 1 (Pos) splits the optimizer state, stage 2
+ * (Pos+g) also the gradients. Each gradient is reduced only on the owner of its partition by a
+ * reduce-scatter, the owner updates its own 1/Nd of the parameters with mixed-precision Adam,
+ * and an all-gather distributes the updated parameters.
+ *   Sources: "ZeRO: particionar estados do treino entre GPUs" (upskillscore.com), section
+ *   "Como funciona"; "ZeRO" (lastdictionary.com), main definition; "ZeRO-2" card
+ *   (llm-engineer.pages.dev), sections "Gradient 생명주기" and "왜 all-gather는 그대로 필요한가".
+ *
+ * In this library the Nd ranks are separate buffers in the memory of ONE GPU: the
+ * reduce-scatter is each owner reading its slice of every rank's gradient, and the all-gather
+ * is each owner writing its updated fp16 shard into one full parameter buffer that stands for
+ * every replica's copy.
+ *
+ * Conventions shared by every call:
+ *   - fp16 values travel as uint16_t bit patterns (IEEE binary16); fp32 as float.
+ *   - Every device pointer is caller-owned device memory of the current CUDA device. The
+ *     library allocates no device memory; the plan and the scheduler are its only objects
+ *     (host memory, plus CUDA events for the scheduler).
+ *   - zero_stream_t is a cudaStream_t (NULL = the legacy default stream). Data-path calls are
+ *     asynchronous and stream-ordered; only zero_step_status waits for the device.
+ *   - Every call returns a zero_status and never aborts or throws. Host-detectable argument
+ *     errors return at once and launch nothing. A failed CUDA launch returns ZERO_ECUDA.
+ *   - Outcomes known only on the device go to a caller-owned 32-bit status word in device
+ *     memory (d_status, the ZERO_FLAG_* bits). Zero it before the first call of each step.
+ *   - Sizes and offsets are element counts (uint64_t) unless named *_bytes.
+ *   - Thread safety: calls on different plans/schedulers may run concurrently; a plan is
+ *     read-only after creation; a scheduler is used by one host thread at a time.
+ */
+#ifndef LIBZERO_H
+#define LIBZERO_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* zero_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    ZERO_OK = 0,
+    ZERO_EINVAL = 1,        /* bad argument: null pointer, size, range, Nd, aliasing */
+    ZERO_EALIGN = 2,        /* a pointer is not aligned to its element size */
+    ZERO_ECUDA = 3,         /* a CUDA runtime call or kernel launch failed */
+    ZERO_ENOMEM = 4,        /* host allocation failed, or a caller buffer is too small */
+    ZERO_STEP_SKIPPED = 5   /* zero_step_status: the step was skipped on overflow */
+} zero_status;
+
+/* Bits of the device status word d_status. */
+#define ZERO_FLAG_OVERFLOW 0x1u /* some reduced gradient of this step was inf or NaN */
+#define ZERO_FLAG_SKIPPED 0x2u  /* the step was not applied (state and params unchanged) */
+#define ZERO_FLAG_TIMEOUT 0x4u  /* a kernel's bounded wait gave up; its outputs are invalid */
+
+#define ZERO_MAX_RANKS 64       /* largest Nd a call accepts */
+
+/* Human-readable name of a status code (static string). */
+const char* zero_status_string(zero_status s);
+
+/* Kernels this library has launched in this process so far (all entry points). */
+uint64_t zero_kernel_launches(void);
+
+/* ------------------------------------------------------------------------------------------
+ * Partition plan.
+ * "Como funciona": the model states are divided into Nd parts, one per data-parallel process;
+ * "ZeRO-2" card, "ZeRO-1에서 남은 낭비": every GPU's local gradient is [g_A, g_B, g_C], one
+ * slice per owner; diagram and "Gradient 생명주기": the backward pass hands over buckets in
+ * reverse layer order (B2, B1, B0), each reduce-scattered at once.
+ *
+ * The n_tensors tensors (numels[i] elements each, in forward order) are laid end to end into
+ * one flat list of psi elements, padded with zeros to psi_padded = ceil(psi/nd)*nd. Owner r
+ * holds shard [r*S, (r+1)*S) with S = psi_padded/nd. Bucket k (k = 0 is produced first) is
+ * [max(0, psi_padded - (k+1)*B), psi_padded - k*B) with B = bucket_elems (0: one bucket of
+ * everything). stage is 1 or 2 (recorded; the map is the same).
+ * Errors: ZERO_EINVAL for out == NULL, numels == NULL with n_tensors > 0, n_tensors < 0,
+ * nd outside [1, ZERO_MAX_RANKS], stage outside {1, 2}, or psi == 0; ZERO_ENOMEM if the host
+ * allocation fails. On success *out owns host memory released by zero_plan_destroy.
+ * ---------------------------------------------------------------------------------------- */
+typedef struct zero_plan zero_plan;
+
+zero_status zero_plan_create(const uint64_t* numels, int n_tensors, int nd, int stage,
+                             uint64_t bucket_elems, zero_plan** out);
+void zero_plan_destroy(zero_plan* plan);
+
+/* psi, psi_padded, shard length S and the bucket count; any output may be NULL. */
+zero_status zero_plan_info(const zero_plan* plan, uint64_t* psi, uint64_t* psi_padded,
+                           uint64_t* shard_elems, int* n_buckets);
+/* Flat offset of each tensor (n_tensors values written to out). */
+zero_status zero_plan_tensor_offsets(const zero_plan* plan, uint64_t* out);
+/* Bucket k: its flat range [flat_lo, flat_lo + len) and the owners it touches,
+ * owner_lo..owner_hi inclusive. ZERO_EINVAL if k is out of range. */
+zero_status zero_plan_bucket(const zero_plan* plan, int k, uint64_t* flat_lo, uint64_t* len,
+                             int* owner_lo, int* owner_hi);
+
+/* ------------------------------------------------------------------------------------------
+ * Model-state accounting, bytes held by one device ("Como funciona"; "ZeRO" (lastdictionary)):
+ *   stage[0] plain DP  : params 2psi, grads 2psi,   optim K psi      (16 psi for K = 12)
+ *   stage[1] Pos       : params 2psi, grads 2psi,   optim K psi/Nd   (4psi + 12psi/Nd)
+ *   stage[2] Pos+g     : params 2psi, grads 2psi/Nd, optim K psi/Nd  (2psi + 14psi/Nd)
+ *   stage[3] Pos+g+p   : params 2psi/Nd, grads 2psi/Nd, optim K psi/Nd (16psi/Nd)
+ * A partitioned quantity counts ceil(psi/Nd) elements. Communication per step in elements:
+ * 2psi (DP, Pos, Pos+g: reduce-scatter + all-gather), 3psi (Pos+g+p: two parameter
+ * all-gathers + the reduce-scatter); comm_bytes_fp16 is twice that.
+ * Errors: ZERO_EINVAL for out == NULL, nd < 1 or K < 0.
+ * ---------------------------------------------------------------------------------------- */
+typedef struct {
+    uint64_t params, grads, optim, total;
+} zero_bytes;
+
+typedef struct {
+    zero_bytes stage[4];
+    uint64_t comm_elems[4];
+    uint64_t comm_bytes_fp16[4];
+} zero_state_report;
+
+zero_status zero_state_bytes(uint64_t psi, int nd, int K, zero_state_report* out);
+
+/* ------------------------------------------------------------------------------------------
+ * Adam hyperparameters (host memory, read during the call only). Host-side constants are
+ * computed from them in double and rounded once to fp32: beta1, 1-beta1, beta2, 1-beta2,
+ * step_size = lr/(1-beta1^t), sqrt(1-beta2^t), eps, loss_scale.
+ * Requirements: lr finite; 0 <= beta1, beta2 < 1; eps >= 0; loss_scale finite and > 0.
+ * ---------------------------------------------------------------------------------------- */
+typedef struct {
+    double lr, beta1, beta2, eps, loss_scale;
+} zero_adam_hparams;
+
+/* ------------------------------------------------------------------------------------------
+ * Bucketed reduce-scatter (stage 2). "ZeRO-2" card, "Gradient 생명주기": as soon as a bucket's
+ * local gradient exists it is reduce-scattered; each GPU keeps only its reduced shard.
+ *
+ * For every element i of bucket k (flat index f = flat_lo + i):
+ *   red = (sum over r = 0..nd-1, in that order, of fp32(rank_grads[r][i])) / nd   (fp32)
+ *   owner_grad_shards[f / S][f % S] = red
+ * and ZERO_FLAG_OVERFLOW is ORed into *d_status if any red is inf or NaN.
+ *   rank_grads        : nd device pointers (host array), each to `len` fp16 values: rank r's
+ *                       local gradient of bucket k. 2-byte aligned; 16-byte alignment takes
+ *                       the fast path.
+ *   owner_grad_shards : nd device pointers (host array), each to S fp32 values (4-byte
+ *                       aligned): owner r's reduced-gradient shard. Only the part covered by
+ *                       bucket k is written.
+ * Errors: ZERO_EINVAL (null plan/pointers, k out of range, overlap between an output shard and
+ * an input); ZERO_EALIGN; ZERO_ECUDA.
+ * ---------------------------------------------------------------------------------------- */
+zero_status zero_reduce_scatter_bucket(const zero_plan* plan, int k,
+                                       const uint16_t* const* rank_grads,
+                                       float* const* owner_grad_shards, uint32_t* d_status,
+                                       zero_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Owner update of a shard (stages 1 and 2, unfused). "Como funciona": each process updates
+ * only its part of the optimizer state; "ZeRO-2" card, "Gradient 생명주기": GPU r updates
+ * parameter shard r from reduced-gradient shard r; "왜 all-gather는 그대로 필요한가": the
+ * updated shards are gathered into every GPU's full parameters.
+ *
+ * If ZERO_FLAG_OVERFLOW is set in *d_status when the kernel runs, nothing is written except
+ * ZERO_FLAG_SKIPPED into *d_status. Otherwise, in place, for i in [0, n):
+ *   g = grad[i] / loss_scale
+ *   m = beta1*m + (1-beta1)*g ;  v = beta2*v + (1-beta2)*(g*g)
+ *   master = master - step_size * (m / (sqrt(v)/sqrt(1-beta2^t) + eps))
+ *   param_out[i] = fp16(master), round to nearest even
+ * every operation an IEEE fp32 operation rounded to nearest even, no fused multiply-add.
+ *   grad, master, m, v : n fp32 each (device, 4-byte aligned; 16 bytes for the fast path)
+ *   param_out          : n fp16 (device, 2-byte aligned), e.g. full_params + owner*S
+ *   step               : t >= 1, the caller's counter (do not advance it on a skipped step)
+ * Errors: ZERO_EINVAL (null pointers, t < 1, bad hyperparameters, overlapping arrays);
+ * ZERO_EALIGN; ZERO_ECUDA. n == 0 launches nothing.
+ * ---------------------------------------------------------------------------------------- */
+zero_status zero_adam_shard(uint64_t n, const float* grad, float* master, float* m, float* v,
+                            uint16_t* param_out, const zero_adam_hparams* hp, int64_t step,
+                            uint32_t* d_status, zero_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Fused step: reduce-scatter + unscale + Adam + fp16 cast + all-gather write-back in one
+ * pass, so the reduced gradient never reaches memory. Same arithmetic as the two calls above:
+ *   red = (sum_{r=0..nd-1} fp32(rank_grads[r][i])) / nd, then the update of zero_adam_shard
+ *   from (master_in, m_in, v_in)[i] into (master_out, m_out, v_out)[i], param_out[i] = fp16.
+ * Inputs are never written, so a step with an inf/NaN anywhere can still be skipped after
+ * the fact: call zero_step_commit once after the last zero_step_fused call of the step.
+ * A step may be split into several calls (e.g. one per bucket) on disjoint ranges.
+ * ZERO_FLAG_OVERFLOW is ORed into *d_status if any red is inf or NaN.
+ *   n                 : elements in this call's range
+ *   rank_grads        : nd device pointers (host array), each to n fp16 values of this range
+ *   *_in / *_out      : n fp32 each; outputs must not overlap any input or each other
+ *   param_out         : n fp16, e.g. full_params + flat offset of the range
+ * Pointers must be aligned to their element size; when every gradient and state pointer is
+ * 16-byte aligned the TMA-pipelined kernel runs, else a plain-load kernel.
+ * Errors: ZERO_EINVAL (nd outside [1, 64], null pointers, t < 1, bad hyperparameters,
+ * overlapping outputs); ZERO_EALIGN; ZERO_ECUDA. n == 0 launches nothing.
+ * ---------------------------------------------------------------------------------------- */
+zero_status zero_step_fused(uint64_t n, int nd, const uint16_t* const* rank_grads,
+                            const float* master_in, const float* m_in, const float* v_in,
+                            float* master_out, float* m_out, float* v_out, uint16_t* param_out,
+                            const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
+                            zero_stream_t stream);
+
+/* Close a step made of zero_step_fused calls, on the same stream, over the same range(s).
+ * If ZERO_FLAG_OVERFLOW is set: (master_out, m_out, v_out) = (master_in, m_in, v_in),
+ * param_out = fp16(master_in), and ZERO_FLAG_SKIPPED is set -- the step did not happen.
+ * Otherwise nothing is written. Either way the caller may then swap the in/out buffers.
+ * Errors: as zero_step_fused. */
+zero_status zero_step_commit(uint64_t n, const float* master_in, const float* m_in,
+                             const float* v_in, float* master_out, float* m_out, float* v_out,
+                             uint16_t* param_out, uint32_t* d_status, zero_stream_t stream);
+
+/* Wait for `stream`, read *d_status into *flags_out (may be NULL) and map it to a status:
+ * ZERO_STEP_SKIPPED if ZERO_FLAG_SKIPPED is set, ZERO_ECUDA if ZERO_FLAG_TIMEOUT is set or the
+ * copy fails, else ZERO_OK. This is the only call that blocks the host. */
+zero_status zero_step_status(const uint32_t* d_status, zero_stream_t stream, uint32_t* flags_out);
+
+/* ------------------------------------------------------------------------------------------
+ * Stream-ordered bucket scheduler for stage 2. "ZeRO-2" card, "Gradient 생명주기": after a
+ * bucket's reduce-scatter the GPU keeps its own reduced shard and releases the rest of the
+ * local gradient. The local gradients of a bucket live in a staging slot (nd regions of
+ * slot_stride fp16 values, slot_stride = the longest bucket rounded up to 8 elements); the
+ * reduce-scatter runs on rs_stream once the producer has filled the slot, and the slot is
+ * released (reused by a later bucket) when that reduce-scatter has finished -- all ordered by
+ * CUDA events, without blocking the host.
+ *   slot_mem          : n_slots*nd*slot_stride fp16 values of caller device memory, 16-byte
+ *                       aligned (zero_sched_slot_elems gives the count)
+ *   owner_grad_shards : nd device pointers (copied), as for zero_reduce_scatter_bucket
+ *   d_status          : the step's status word
+ * Errors: ZERO_EINVAL, ZERO_EALIGN, ZERO_ENOMEM (slot_mem too small or host allocation),
+ * ZERO_ECUDA (event creation).
+ * ---------------------------------------------------------------------------------------- */
+typedef struct zero_sched zero_sched;
+
+zero_status zero_sched_slot_elems(const zero_plan* plan, int n_slots, uint64_t* elems);
+zero_status zero_sched_create(const zero_plan* plan, uint16_t* slot_mem, uint64_t slot_mem_elems,
+                              int n_slots, float* const* owner_grad_shards, uint32_t* d_status,
+                              zero_stream_t rs_stream, zero_sched** out);
+/* Choose the slot for bucket k, make `producer` wait until that slot is released, and write
+ * the nd device pointers (rank r's region, bucket k's len values) the producer must fill. */
+zero_status zero_sched_begin_bucket(zero_sched* s, int k, zero_stream_t producer,
+                                    uint16_t** rank_ptrs);
+/* The producer has enqueued the fill of bucket k on `producer`: the reduce-scatter of
+ * bucket k is enqueued on rs_stream after it, followed by the release of its slot. */
+zero_status zero_sched_end_bucket(zero_sched* s, int k, zero_stream_t producer);
+/* Make `stream` wait for every reduce-scatter enqueued so far (e.g. before zero_adam_shard). */
+zero_status zero_sched_wait(zero_sched* s, zero_stream_t stream);
+/* Number of reduce-scatter kernels the scheduler has launched since creation. */
+zero_status zero_sched_launches(const zero_sched* s, uint64_t* count);
+void zero_sched_destroy(zero_sched* s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBZERO_H */

@@ -1,0 +1,217 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol include/*.h
+declares, its planner and accounting agree bit-exactly with the oracle's independent ones, and
+host-detectable argument errors return their status codes without launching anything."""
+import glob
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from zero_partitioned_optimizer_plan_b200 import build as zbuild
+from zero_partitioned_optimizer_plan_b200 import synth
+
+zbuild.build()
+from zero_partitioned_optimizer_plan_b200 import libzero as lz  # noqa: E402
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(zero_\w+)\s*\(", src, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for must in ("zero_plan_create", "zero_state_bytes", "zero_reduce_scatter_bucket",
+                 "zero_adam_shard", "zero_step_fused"):
+        assert must in names
+    assert names == set(lz.SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", lz.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = _declared_functions() - exported
+    assert not missing, missing
+    for name in _declared_functions():
+        assert hasattr(lz._lib, name)
+
+
+def test_library_is_built_for_sm100a():
+    assert "arch=compute_100a,code=sm_100a" in " ".join(zbuild.NVCC_FLAGS)
+    log = open(os.path.join(zbuild.BUILD, "ptxas.log")).read()
+    assert "for 'sm_100a'" in log and "spill stores" in log
+    # no kernel spills registers to local memory
+    assert all(" 0 bytes spill stores" in ln for ln in log.splitlines() if "spill stores" in ln)
+
+
+# ---------------------------------------------------------------------------------------------
+# planner and accounting: two independent implementations agree exactly
+# ---------------------------------------------------------------------------------------------
+def _compare_plans(numels, nd, bucket):
+    ref = oracle.plan(numels, nd, bucket)
+    pl = lz.zero_plan_create(numels, nd, 2, bucket)
+    psi, psi_p, shard, nb = lz.zero_plan_info(pl)
+    assert (psi, psi_p, shard, nb) == (ref.psi, ref.psi_p, ref.shard, len(ref.buckets))
+    assert lz.zero_plan_tensor_offsets(pl) == ref.tensor_off
+    for k, (lo, ln) in enumerate(ref.buckets):
+        assert lz.zero_plan_bucket(pl, k) == (lo, ln, *ref.owners(k))
+    with pytest.raises(lz.ZeroError):
+        lz.zero_plan_bucket(pl, nb)
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_plan_matches_oracle_random(seed):
+    rng = np.random.default_rng(seed)
+    n = int(rng.integers(1, 12))
+    numels = [int(x) for x in rng.integers(0, 10 ** int(rng.integers(1, 7)), n)]
+    if sum(numels) == 0:
+        numels[0] = 1
+    nd = int(rng.integers(1, 65))
+    total = sum(numels)
+    # at most ~300 buckets: the oracle walks them one by one
+    small = max(1, -(-total // 300))
+    bucket = int(rng.choice([0, small, small + 7, 8 * small, int(rng.integers(small, total + 10))]))
+    _compare_plans(numels, nd, bucket)
+
+
+def test_plan_matches_oracle_workloads():
+    _compare_plans(synth.TINY_LIST, 4, 0)
+    _compare_plans(synth.gpt2_small_list(), 8, 0)
+    _compare_plans(synth.gpt_1p3b_list(), 16, 50_000_000)
+    _compare_plans([7_500_000_000], 64, 0)
+    _compare_plans([1 << 29], 64, 1 << 19)
+    _compare_plans([7], 4, 3)
+
+
+@pytest.mark.parametrize("psi,nd,K", [(7_500_000_000, 64, 12), (123_653_376, 8, 12),
+                                      (1_311_528_960, 16, 12), (1, 64, 12), (7, 4, 12),
+                                      (1000, 3, 8), (0, 5, 12)])
+def test_state_bytes_matches_oracle(psi, nd, K):
+    a = lz.zero_state_bytes(psi, nd, K)
+    b = oracle.state_bytes(psi, nd, K)
+    for s in lz.STAGES:
+        for key in ("params", "grads", "optim", "total", "comm_elems"):
+            assert a[s][key] == b[s][key], (s, key)
+        assert a[s]["comm_bytes_fp16"] == 2 * b[s]["comm_elems"]
+
+
+def test_plan_rejects_bad_arguments():
+    for args in [([], 4, 1, 0), ([5], 0, 1, 0), ([5], 65, 1, 0), ([5], 4, 3, 0), ([0, 0], 2, 1, 0)]:
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_plan_create(*args)
+        assert e.value.code == lz.ZERO_EINVAL
+    with pytest.raises(lz.ZeroError):
+        lz.zero_state_bytes(10, 0)
+
+
+# ---------------------------------------------------------------------------------------------
+# data-path argument errors (all caught on the host before any CUDA call)
+# ---------------------------------------------------------------------------------------------
+HP = lz.AdamHP()
+A = 1 << 32          # fake, 256-byte aligned device addresses far apart
+MB = 1 << 24
+
+
+def _fused(n=1000, nd=2, grads=None, ins=None, outs=None, p=None, hp=HP, step=1, st=None):
+    grads = grads if grads is not None else [A + i * MB for i in range(nd)]
+    ins = ins or [A + 100 * MB, A + 101 * MB, A + 102 * MB]
+    outs = outs or [A + 110 * MB, A + 111 * MB, A + 112 * MB]
+    p = p if p is not None else A + 120 * MB
+    st = st if st is not None else A + 130 * MB
+    lz.zero_step_fused(n, nd, grads, *ins, *outs, p, hp, step, st, 0)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(nd=0), lz.ZERO_EINVAL),
+    (dict(nd=65), lz.ZERO_EINVAL),
+    (dict(step=0), lz.ZERO_EINVAL),
+    (dict(st=0), lz.ZERO_EINVAL),
+    (dict(hp=lz.AdamHP(beta1=1.0)), lz.ZERO_EINVAL),
+    (dict(hp=lz.AdamHP(loss_scale=0.0)), lz.ZERO_EINVAL),
+    (dict(hp=lz.AdamHP(lr=float("nan"))), lz.ZERO_EINVAL),
+    (dict(hp=lz.AdamHP(eps=-1.0)), lz.ZERO_EINVAL),
+    (dict(grads=[A, 0]), lz.ZERO_EINVAL),
+    (dict(grads=[A, A + 1]), lz.ZERO_EALIGN),
+    (dict(p=A + 120 * MB + 1), lz.ZERO_EALIGN),
+    (dict(ins=[A + 100 * MB + 2, A + 101 * MB, A + 102 * MB]), lz.ZERO_EALIGN),
+    (dict(outs=[A + 100 * MB, A + 111 * MB, A + 112 * MB]), lz.ZERO_EINVAL),      # out == in
+    (dict(outs=[A + 110 * MB, A + 110 * MB + 400, A + 112 * MB]), lz.ZERO_EINVAL),  # outs overlap
+    (dict(p=A), lz.ZERO_EINVAL),                                                    # param over grads
+    (dict(st=A + 110 * MB + 8), lz.ZERO_EINVAL),                                    # status in out
+])
+def test_fused_rejects(kw, code):
+    with pytest.raises(lz.ZeroError) as e:
+        _fused(**kw)
+    assert e.value.code == code
+
+
+def test_zero_length_launches_nothing():
+    before = lz.zero_kernel_launches()
+    _fused(n=0)
+    lz.zero_adam_shard(0, A, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, HP, 1, A + 5 * MB, 0)
+    lz.zero_step_commit(0, A, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, A + 5 * MB,
+                        A + 6 * MB, A + 7 * MB, 0)
+    assert lz.zero_kernel_launches() == before
+
+
+@pytest.mark.parametrize("args,code", [
+    ((10, 0, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB), lz.ZERO_EINVAL),        # null grad
+    ((10, A, A + MB + 2, A + 2 * MB, A + 3 * MB, A + 4 * MB), lz.ZERO_EALIGN),
+    ((10, A, A + MB, A + MB + 20, A + 3 * MB, A + 4 * MB), lz.ZERO_EINVAL),        # m over master
+    ((10, A, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB + 1), lz.ZERO_EALIGN),
+])
+def test_adam_rejects(args, code):
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_adam_shard(*args, HP, 1, A + 9 * MB, 0)
+    assert e.value.code == code
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_adam_shard(10, A, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, HP, 0, A + 9 * MB, 0)
+    assert e.value.code == lz.ZERO_EINVAL
+
+
+def test_reduce_scatter_rejects():
+    pl = lz.zero_plan_create([100, 28], 4, 2, 32)
+    grads = [A + i * MB for i in range(4)]
+    shards = [A + (10 + i) * MB for i in range(4)]
+    st = A + 50 * MB
+    for k, g, s, code in [(4, grads, shards, lz.ZERO_EINVAL),       # bucket out of range
+                          (-1, grads, shards, lz.ZERO_EINVAL),
+                          (0, grads[:3] + [0], shards, lz.ZERO_EINVAL),
+                          (0, grads, shards[:3] + [A + 10 * MB + 2], lz.ZERO_EALIGN),
+                          (0, grads, shards[:3] + [A + 10 * MB + 8], lz.ZERO_EINVAL),  # overlap
+                          (0, grads, shards[:3] + [A + 4], lz.ZERO_EINVAL)]:            # over grads
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_reduce_scatter_bucket(pl, k, g, s, st, 0)
+        assert e.value.code == code
+
+
+def test_scheduler_rejects():
+    pl = lz.zero_plan_create([100, 28], 4, 2, 32)
+    need = lz.zero_sched_slot_elems(pl, 2)
+    assert need == 2 * 4 * 32
+    shards = [A + (10 + i) * MB for i in range(4)]
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_sched_create(pl, A, need - 1, 2, shards, A + 50 * MB, 0)
+    assert e.value.code == lz.ZERO_ENOMEM
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_sched_create(pl, A + 8, need, 2, shards, A + 50 * MB, 0)
+    assert e.value.code == lz.ZERO_EALIGN
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_sched_create(pl, A, need, 0, shards, A + 50 * MB, 0)
+    assert e.value.code == lz.ZERO_EINVAL
+
+
+def test_status_strings():
+    for code in range(6):
+        assert lz.zero_status_string(code).startswith("ZERO_")

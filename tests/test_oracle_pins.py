@@ -57,11 +57,22 @@ def test_f2h_strided_vs_numpy():
         _f2h_chunk_check(lo, lo + (1 << 24))
 
 
-@pytest.mark.slow
+def _f2h_chunk_worker(lo_hi):
+    _f2h_chunk_check(*lo_hi)
+    return lo_hi
+
+
 def test_f2h_exhaustive_vs_numpy():
-    step = 1 << 26
-    for lo in range(0, 1 << 32, step):
-        _f2h_chunk_check(lo, lo + step)
+    # all 2^32 binary32 bit patterns, spread over the host's cores (spawned workers, each
+    # loading its own copy of the oracle)
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    step = 1 << 25
+    chunks = [(lo, lo + step) for lo in range(0, 1 << 32, step)]
+    workers = max(1, min(16, os.cpu_count() or 1))
+    with cf.ProcessPoolExecutor(workers, mp_context=mp.get_context("spawn")) as ex:
+        done = list(ex.map(_f2h_chunk_worker, chunks))
+    assert len(done) == len(chunks)
 
 
 def test_f2h_vs_exact_rounding_at_midpoints():

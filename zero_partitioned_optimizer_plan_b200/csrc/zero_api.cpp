@@ -1,0 +1,224 @@
+// C ABI of the libzero data path: argument checks, the host-side Adam constants, and the
+// launches. Every function returns a zero_status and never throws.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "../../include/libzero.h"
+#include "zero_internal.h"
+
+namespace zk {
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Do the byte ranges [a, a+na) and [b, b+nb) intersect?
+bool overlap(const void* a, uint64_t na, const void* b, uint64_t nb) {
+    if (na == 0 || nb == 0) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+bool finite(double x) { return std::isfinite(x); }
+
+// 2^k with 1/2^k a normal binary32 number: then x * (1/2^k) rounds exactly like x / 2^k.
+bool pow2_with_normal_reciprocal(double x, float* inv) {
+    if (!(x > 0.0) || !finite(x)) return false;
+    int e = 0;
+    const double mant = std::frexp(x, &e);   // x = mant * 2^e, mant in [0.5, 1)
+    if (mant != 0.5) return false;
+    const int k = e - 1;                     // x = 2^k
+    if (k < -126 || k > 126) return false;
+    *inv = (float)std::ldexp(1.0, -k);
+    return true;
+}
+
+bool hparams_ok(const zero_adam_hparams* hp) {
+    return hp && finite(hp->lr) && hp->beta1 >= 0.0 && hp->beta1 < 1.0 && hp->beta2 >= 0.0 &&
+           hp->beta2 < 1.0 && finite(hp->eps) && hp->eps >= 0.0 && finite(hp->loss_scale) &&
+           hp->loss_scale > 0.0;
+}
+
+// The fp32 constants of step t: computed in double, each rounded once to binary32.
+AdamConsts make_adam(const zero_adam_hparams* hp, int64_t t) {
+    AdamConsts a;
+    const double c1 = 1.0 - std::pow(hp->beta1, (double)t);
+    const double c2 = 1.0 - std::pow(hp->beta2, (double)t);
+    a.b1 = (float)hp->beta1;
+    a.omb1 = (float)(1.0 - hp->beta1);
+    a.b2 = (float)hp->beta2;
+    a.omb2 = (float)(1.0 - hp->beta2);
+    a.step_size = (float)(hp->lr / c1);
+    a.bc2s = (float)std::sqrt(c2);
+    a.eps = (float)hp->eps;
+    a.loss_scale = (float)hp->loss_scale;
+    a.inv_ls = 0.0f;
+    a.ls_pow2 = pow2_with_normal_reciprocal((double)a.loss_scale, &a.inv_ls) ? 1 : 0;
+    return a;
+}
+
+zero_status from_cuda(cudaError_t e) { return e == cudaSuccess ? ZERO_OK : ZERO_ECUDA; }
+
+}  // namespace
+
+MeanConsts make_mean(int nd) {
+    MeanConsts mc;
+    mc.fnd = (float)nd;
+    mc.nd_pow2 = (nd & (nd - 1)) == 0 ? 1 : 0;
+    mc.inv_nd = 1.0f / (float)nd;   // exact when nd is a power of two
+    return mc;
+}
+
+cudaError_t rs_bucket_launch(const zero_plan* plan, int k, const uint16_t* const* rank_grads,
+                             float* const* shards, uint32_t* status, cudaStream_t stream) {
+    int nd = 0;
+    uint64_t psi_p = 0, S = 0, lo = 0, len = 0;
+    plan_geometry(plan, &nd, &psi_p, &S);
+    plan_bucket_range(plan, k, &lo, &len);
+    return launch_reduce_scatter(len, nd, rank_grads, shards, lo, S, make_mean(nd), status, stream);
+}
+
+}  // namespace zk
+
+extern "C" {
+
+const char* zero_status_string(zero_status s) {
+    switch (s) {
+        case ZERO_OK: return "ZERO_OK";
+        case ZERO_EINVAL: return "ZERO_EINVAL: invalid argument";
+        case ZERO_EALIGN: return "ZERO_EALIGN: pointer not aligned to its element size";
+        case ZERO_ECUDA: return "ZERO_ECUDA: CUDA error";
+        case ZERO_ENOMEM: return "ZERO_ENOMEM: out of memory or buffer too small";
+        case ZERO_STEP_SKIPPED: return "ZERO_STEP_SKIPPED: step skipped on gradient overflow";
+    }
+    return "unknown zero_status";
+}
+
+uint64_t zero_kernel_launches(void) { return zk::launches(); }
+
+zero_status zero_reduce_scatter_bucket(const zero_plan* plan, int k,
+                                       const uint16_t* const* rank_grads,
+                                       float* const* owner_grad_shards, uint32_t* d_status,
+                                       zero_stream_t stream) {
+    int nd = 0;
+    uint64_t psi_p = 0, S = 0, lo = 0, len = 0;
+    if (!zk::plan_geometry(plan, &nd, &psi_p, &S)) return ZERO_EINVAL;
+    if (!zk::plan_bucket_range(plan, k, &lo, &len)) return ZERO_EINVAL;
+    if (!rank_grads || !owner_grad_shards || !d_status) return ZERO_EINVAL;
+    if (!zk::aligned(d_status, 4)) return ZERO_EALIGN;
+    for (int r = 0; r < nd; ++r) {
+        if (!rank_grads[r] || !owner_grad_shards[r]) return ZERO_EINVAL;
+        if (!zk::aligned(rank_grads[r], 2) || !zk::aligned(owner_grad_shards[r], 4))
+            return ZERO_EALIGN;
+    }
+    // outputs may not overlap inputs, each other or the status word
+    for (int o = 0; o < nd; ++o) {
+        if (zk::overlap(owner_grad_shards[o], S * 4, d_status, 4)) return ZERO_EINVAL;
+        for (int r = 0; r < nd; ++r) {
+            if (zk::overlap(owner_grad_shards[o], S * 4, rank_grads[r], len * 2)) return ZERO_EINVAL;
+            if (r != o && zk::overlap(owner_grad_shards[o], S * 4, owner_grad_shards[r], S * 4))
+                return ZERO_EINVAL;
+        }
+    }
+    return zk::from_cuda(zk::rs_bucket_launch(plan, k, rank_grads, owner_grad_shards, d_status,
+                                              (cudaStream_t)stream));
+}
+
+zero_status zero_adam_shard(uint64_t n, const float* grad, float* master, float* m, float* v,
+                            uint16_t* param_out, const zero_adam_hparams* hp, int64_t step,
+                            uint32_t* d_status, zero_stream_t stream) {
+    if (!zk::hparams_ok(hp) || step < 1 || !d_status) return ZERO_EINVAL;
+    if (n == 0) return ZERO_OK;
+    if (!grad || !master || !m || !v || !param_out) return ZERO_EINVAL;
+    if (n > (UINT64_MAX / 8)) return ZERO_EINVAL;
+    if (!zk::aligned(grad, 4) || !zk::aligned(master, 4) || !zk::aligned(m, 4) ||
+        !zk::aligned(v, 4) || !zk::aligned(param_out, 2) || !zk::aligned(d_status, 4))
+        return ZERO_EALIGN;
+    const void* arr[6] = {grad, master, m, v, param_out, d_status};
+    const uint64_t len[6] = {n * 4, n * 4, n * 4, n * 4, n * 2, 4};
+    for (int i = 0; i < 6; ++i)
+        for (int j = i + 1; j < 6; ++j)
+            if (zk::overlap(arr[i], len[i], arr[j], len[j])) return ZERO_EINVAL;
+    return zk::from_cuda(zk::launch_adam(n, grad, master, m, v, param_out,
+                                         zk::make_adam(hp, step), d_status,
+                                         (cudaStream_t)stream));
+}
+
+static zero_status check_fused_state(uint64_t n, const float* master_in, const float* m_in,
+                                     const float* v_in, float* master_out, float* m_out,
+                                     float* v_out, uint16_t* param_out, uint32_t* d_status) {
+    if (!master_in || !m_in || !v_in || !master_out || !m_out || !v_out || !param_out ||
+        !d_status)
+        return ZERO_EINVAL;
+    if (n > (UINT64_MAX / 8)) return ZERO_EINVAL;
+    if (!zk::aligned(master_in, 4) || !zk::aligned(m_in, 4) || !zk::aligned(v_in, 4) ||
+        !zk::aligned(master_out, 4) || !zk::aligned(m_out, 4) || !zk::aligned(v_out, 4) ||
+        !zk::aligned(param_out, 2) || !zk::aligned(d_status, 4))
+        return ZERO_EALIGN;
+    const void* outs[5] = {master_out, m_out, v_out, param_out, d_status};
+    const uint64_t olen[5] = {n * 4, n * 4, n * 4, n * 2, 4};
+    const void* ins[3] = {master_in, m_in, v_in};
+    for (int i = 0; i < 5; ++i) {
+        for (int j = 0; j < 3; ++j)
+            if (zk::overlap(outs[i], olen[i], ins[j], n * 4)) return ZERO_EINVAL;
+        for (int j = i + 1; j < 5; ++j)
+            if (zk::overlap(outs[i], olen[i], outs[j], olen[j])) return ZERO_EINVAL;
+    }
+    return ZERO_OK;
+}
+
+zero_status zero_step_fused(uint64_t n, int nd, const uint16_t* const* rank_grads,
+                            const float* master_in, const float* m_in, const float* v_in,
+                            float* master_out, float* m_out, float* v_out, uint16_t* param_out,
+                            const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
+                            zero_stream_t stream) {
+    if (nd < 1 || nd > ZERO_MAX_RANKS || !zk::hparams_ok(hp) || step < 1 || !d_status)
+        return ZERO_EINVAL;
+    if (n == 0) return ZERO_OK;
+    if (!rank_grads) return ZERO_EINVAL;
+    zero_status st = check_fused_state(n, master_in, m_in, v_in, master_out, m_out, v_out,
+                                       param_out, d_status);
+    if (st != ZERO_OK) return st;
+    const void* outs[5] = {master_out, m_out, v_out, param_out, d_status};
+    const uint64_t olen[5] = {n * 4, n * 4, n * 4, n * 2, 4};
+    for (int r = 0; r < nd; ++r) {
+        if (!rank_grads[r]) return ZERO_EINVAL;
+        if (!zk::aligned(rank_grads[r], 2)) return ZERO_EALIGN;
+        for (int i = 0; i < 5; ++i)
+            if (zk::overlap(outs[i], olen[i], rank_grads[r], n * 2)) return ZERO_EINVAL;
+    }
+    return zk::from_cuda(zk::launch_fused(n, nd, rank_grads, master_in, m_in, v_in, master_out,
+                                          m_out, v_out, param_out, zk::make_adam(hp, step),
+                                          zk::make_mean(nd), d_status, (cudaStream_t)stream));
+}
+
+zero_status zero_step_commit(uint64_t n, const float* master_in, const float* m_in,
+                             const float* v_in, float* master_out, float* m_out, float* v_out,
+                             uint16_t* param_out, uint32_t* d_status, zero_stream_t stream) {
+    if (!d_status) return ZERO_EINVAL;
+    if (n == 0) return ZERO_OK;
+    zero_status st = check_fused_state(n, master_in, m_in, v_in, master_out, m_out, v_out,
+                                       param_out, d_status);
+    if (st != ZERO_OK) return st;
+    return zk::from_cuda(zk::launch_commit(n, master_in, m_in, v_in, master_out, m_out, v_out,
+                                           param_out, d_status, (cudaStream_t)stream));
+}
+
+zero_status zero_step_status(const uint32_t* d_status, zero_stream_t stream, uint32_t* flags_out) {
+    if (!d_status) return ZERO_EINVAL;
+    if (!zk::aligned(d_status, 4)) return ZERO_EALIGN;
+    uint32_t flags = 0;
+    cudaError_t e = cudaMemcpyAsync(&flags, d_status, sizeof(flags), cudaMemcpyDeviceToHost,
+                                    (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return ZERO_ECUDA;
+    if (flags_out) *flags_out = flags;
+    if (flags & ZERO_FLAG_TIMEOUT) return ZERO_ECUDA;
+    if (flags & ZERO_FLAG_SKIPPED) return ZERO_STEP_SKIPPED;
+    return ZERO_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,61 @@
+// Internal declarations shared by the libzero translation units (not part of the C ABI).
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "../../include/libzero.h"
+
+namespace zk {
+
+// fp32 constants of one Adam step, computed on the host (see zero_api.cpp).
+struct AdamConsts {
+    float b1, omb1, b2, omb2;
+    float step_size;   // lr / (1 - beta1^t)
+    float bc2s;        // sqrt(1 - beta2^t)
+    float eps;
+    float loss_scale;  // the divisor of the unscale
+    float inv_ls;      // 1/loss_scale when loss_scale is a power of two (then x*inv_ls == x/ls)
+    int ls_pow2;
+};
+
+// The division of the rank sum by nd.
+struct MeanConsts {
+    float fnd;
+    float inv_nd;      // 1/nd when nd is a power of two (then x*inv_nd == x/nd exactly)
+    int nd_pow2;
+};
+
+// Plan accessors used by the data path and the scheduler (zero_plan.cpp).
+bool plan_geometry(const zero_plan* p, int* nd, uint64_t* psi_p, uint64_t* shard);
+bool plan_bucket_range(const zero_plan* p, int k, uint64_t* lo, uint64_t* len);
+uint64_t plan_max_bucket(const zero_plan* p);
+uint64_t plan_n_buckets(const zero_plan* p);
+
+// Launchers (zero_kernels.cu). They validate nothing: the C ABI layer has done that.
+cudaError_t launch_fused(uint64_t n, int nd, const uint16_t* const* grads, const float* master_in,
+                         const float* m_in, const float* v_in, float* master_out, float* m_out,
+                         float* v_out, uint16_t* param_out, const AdamConsts& a,
+                         const MeanConsts& mc, uint32_t* status, cudaStream_t stream);
+cudaError_t launch_commit(uint64_t n, const float* master_in, const float* m_in,
+                          const float* v_in, float* master_out, float* m_out, float* v_out,
+                          uint16_t* param_out, uint32_t* status, cudaStream_t stream);
+cudaError_t launch_reduce_scatter(uint64_t n, int nd, const uint16_t* const* grads,
+                                  float* const* shards, uint64_t flat_lo, uint64_t shard,
+                                  const MeanConsts& mc, uint32_t* status, cudaStream_t stream);
+cudaError_t launch_adam(uint64_t n, const float* grad, float* master, float* m, float* v,
+                        uint16_t* param_out, const AdamConsts& a, uint32_t* status,
+                        cudaStream_t stream);
+
+// Count of kernels this library has launched in this process.
+void count_launch();
+uint64_t launches();
+
+// Launch the reduce-scatter of bucket k of a plan (arguments already validated).
+cudaError_t rs_bucket_launch(const zero_plan* plan, int k, const uint16_t* const* rank_grads,
+                             float* const* shards, uint32_t* status, cudaStream_t stream);
+
+MeanConsts make_mean(int nd);
+
+}  // namespace zk

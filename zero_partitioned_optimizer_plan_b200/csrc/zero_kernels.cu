@@ -1,0 +1,893 @@
+// libzero kernels for sm_100a (B200).
+//
+// The path is a streaming reduction plus an elementwise update: per parameter it reads Nd fp16
+// gradients (2*Nd bytes), 12 bytes of fp32 optimizer state and writes 12 + 2 bytes back, at
+// about one flop per byte. Nothing is a dense contraction, so no tensor cores; the bound is
+// HBM bandwidth, and the design is about keeping enough bytes in flight:
+//
+//   * persistent grid, one CTA per SM, tiles of T elements taken round-robin;
+//   * one elected producer thread per CTA streams each tile's Nd gradient rows and three state
+//     rows into a ring of shared-memory stages with 1-D bulk async copies
+//     (cp.async.bulk ... mbarrier::complete_tx, no multicast), so 100-200 KB per SM are in
+//     flight without spending registers on it;
+//   * eight consumer warps sum the Nd rows in rank order in fp32, release the stage, then
+//     run Adam and store fp32 state and fp16 parameters straight from registers;
+//   * a warp vote collects the overflow (inf/NaN) check, one atomicOr per warp at the end.
+//
+// Every wait on an mbarrier is bounded (1 s); on expiry the kernel sets ZERO_FLAG_TIMEOUT,
+// lets its own copies in flight land, and returns.
+//
+// Arithmetic (identical in every kernel here; see include/libzero.h):
+//   red = (sum_{r=0..nd-1} fp32(g_r)) / nd, the sum strictly in rank order;
+//   g = red / loss_scale; m = b1*m + (1-b1)*g; v = b2*v + (1-b2)*(g*g);
+//   w = w - step_size * (m / (sqrt(v)/bc2s + eps)); p = fp16_rn(w)
+// with every operation a separately rounded IEEE fp32 operation (no FMA contraction; this file
+// is also compiled with -fmad=false). A division by a power of two is done as the product with
+// its exact reciprocal, which is the same correctly rounded real number.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "zero_internal.h"
+
+namespace zk {
+
+namespace {
+
+constexpr int kMaxRanks = ZERO_MAX_RANKS;
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kThreads = kConsumerThreads + 32;  // + one producer warp
+constexpr int kMaxStages = 8;
+constexpr int kDataOffset = 128;                 // full[8] and empty[8] mbarriers first
+constexpr size_t kSmemBudget = 220 * 1024;       // pipeline stages per CTA
+constexpr uint64_t kWaitLimitNs = 1000000000ull; // bounded waits: 1 s
+
+struct FusedArgs {
+    const uint16_t* grads[kMaxRanks];
+    const float* master_in;
+    const float* m_in;
+    const float* v_in;
+    float* master_out;
+    float* m_out;
+    float* v_out;
+    uint16_t* param_out;
+    uint32_t* status;
+    uint64_t n;          // elements of the range
+    uint64_t n_tiled;    // elements covered by tiles (multiple of 8); [n_tiled, n) is the tail
+    uint64_t num_tiles;
+    uint32_t tile;       // elements per tile
+    uint32_t stage_bytes;
+    int nd;
+    int stages;
+    int param_vec;       // widest param store the pointer's alignment allows: 16, 8, 4, 2
+    AdamConsts a;
+    MeanConsts mc;
+};
+
+struct RsArgs {
+    const uint16_t* grads[kMaxRanks];
+    float* shards[kMaxRanks];
+    uint32_t* status;
+    uint64_t n;
+    uint64_t n_tiled;
+    uint64_t num_tiles;
+    uint64_t flat_lo;    // flat index of element 0 of the bucket
+    uint64_t shard;      // S
+    double inv_shard;    // 1/S, for the owner estimate
+    uint32_t tile;
+    uint32_t stage_bytes;
+    int nd;
+    int stages;
+    MeanConsts mc;
+};
+
+struct CommitArgs {
+    const float* master_in;
+    const float* m_in;
+    const float* v_in;
+    float* master_out;
+    float* m_out;
+    float* v_out;
+    uint16_t* param_out;
+    uint32_t* status;
+    uint64_t n;
+};
+
+struct AdamArgs {
+    const float* grad;
+    float* master;
+    float* m;
+    float* v;
+    uint16_t* param_out;
+    uint32_t* status;
+    uint64_t n;
+    int vec;             // 1: every fp32 pointer 16-byte aligned (float4 path)
+    int param_vec;       // 8, 4 or 2
+    AdamConsts a;
+};
+
+// ---------------------------------------------------------------------------------------------
+// element arithmetic
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ float h2f(uint16_t u) { return __half2float(__ushort_as_half(u)); }
+
+__device__ __forceinline__ uint16_t f2h(float x) { return __half_as_ushort(__float2half_rn(x)); }
+
+__device__ __forceinline__ float2 h2x2_to_f2(uint32_t u) {
+    __half2 h;
+    memcpy(&h, &u, 4);
+    return __half22float2(h);
+}
+
+__device__ __forceinline__ float mean_of(float s, const MeanConsts& mc) {
+    return mc.nd_pow2 ? __fmul_rn(s, mc.inv_nd) : __fdiv_rn(s, mc.fnd);
+}
+
+__device__ __forceinline__ bool non_finite(float x) {
+    return (__float_as_uint(x) & 0x7f800000u) == 0x7f800000u;
+}
+
+// Adam on one element from its reduced (still loss-scaled) gradient; w, m, v updated in place.
+__device__ __forceinline__ void adam_elem(float red, float& w, float& m, float& v,
+                                          const AdamConsts& a) {
+    const float g = a.ls_pow2 ? __fmul_rn(red, a.inv_ls) : __fdiv_rn(red, a.loss_scale);
+    const float mt = __fadd_rn(__fmul_rn(a.b1, m), __fmul_rn(a.omb1, g));
+    const float vt = __fadd_rn(__fmul_rn(a.b2, v), __fmul_rn(a.omb2, __fmul_rn(g, g)));
+    const float denom = __fadd_rn(__fdiv_rn(__fsqrt_rn(vt), a.bc2s), a.eps);
+    const float delta = __fmul_rn(a.step_size, __fdiv_rn(mt, denom));
+    w = __fsub_rn(w, delta);
+    m = mt;
+    v = vt;
+}
+
+// ---------------------------------------------------------------------------------------------
+// mbarrier and bulk-copy primitives (PTX)
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase with the given parity to complete; false after kWaitLimitNs.
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completion counted on `bar` in bytes.
+// Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// ---------------------------------------------------------------------------------------------
+// vector helpers
+// ---------------------------------------------------------------------------------------------
+template <int E>
+__device__ __forceinline__ void lds_f16(const uint8_t* p, float (&x)[E]) {
+    if constexpr (E == 8) {
+        const uint4 q = *reinterpret_cast<const uint4*>(p);
+        float2 a = h2x2_to_f2(q.x), b = h2x2_to_f2(q.y), c = h2x2_to_f2(q.z), d = h2x2_to_f2(q.w);
+        x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+        x[4] = c.x; x[5] = c.y; x[6] = d.x; x[7] = d.y;
+    } else if constexpr (E == 4) {
+        const uint2 q = *reinterpret_cast<const uint2*>(p);
+        float2 a = h2x2_to_f2(q.x), b = h2x2_to_f2(q.y);
+        x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+    } else {
+        static_assert(E == 2, "E");
+        const float2 a = h2x2_to_f2(*reinterpret_cast<const uint32_t*>(p));
+        x[0] = a.x; x[1] = a.y;
+    }
+}
+
+template <int E>
+__device__ __forceinline__ void lds_f32(const uint8_t* p, float (&x)[E]) {
+    if constexpr (E == 8) {
+        const float4 a = reinterpret_cast<const float4*>(p)[0];
+        const float4 b = reinterpret_cast<const float4*>(p)[1];
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    } else if constexpr (E == 4) {
+        const float4 a = *reinterpret_cast<const float4*>(p);
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    } else {
+        const float2 a = *reinterpret_cast<const float2*>(p);
+        x[0] = a.x; x[1] = a.y;
+    }
+}
+
+// Store E floats to global memory whose address is a multiple of 4*E bytes (E <= 4 needs
+// 4*E-byte alignment, E == 8 needs 16). Streaming (evict-first) stores.
+template <int E>
+__device__ __forceinline__ void stg_f32(float* p, const float (&x)[E]) {
+    if constexpr (E == 8) {
+        __stcs(reinterpret_cast<float4*>(p), make_float4(x[0], x[1], x[2], x[3]));
+        __stcs(reinterpret_cast<float4*>(p) + 1, make_float4(x[4], x[5], x[6], x[7]));
+    } else if constexpr (E == 4) {
+        __stcs(reinterpret_cast<float4*>(p), make_float4(x[0], x[1], x[2], x[3]));
+    } else {
+        __stcs(reinterpret_cast<float2*>(p), make_float2(x[0], x[1]));
+    }
+}
+
+// Store E floats at any 4-byte aligned address, with the widest stores the address allows.
+template <int E>
+__device__ __forceinline__ void stg_f32_any(float* p, const float (&x)[E]) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    if ((a & 15u) == 0 && (E % 4) == 0) {
+#pragma unroll
+        for (int j = 0; j < E; j += 4)
+            __stcs(reinterpret_cast<float4*>(p + j), make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]));
+    } else if ((a & 7u) == 0) {
+#pragma unroll
+        for (int j = 0; j < E; j += 2) __stcs(reinterpret_cast<float2*>(p + j), make_float2(x[j], x[j + 1]));
+    } else {
+#pragma unroll
+        for (int j = 0; j < E; ++j) __stcs(p + j, x[j]);
+    }
+}
+
+// Store E fp16 values (given as floats, rounded here) with stores of at most `vec` bytes;
+// `vec` is the widest store the destination's alignment allows.
+template <int E>
+__device__ __forceinline__ void stg_f16(uint16_t* p, const float (&x)[E], int vec) {
+    constexpr int H = E / 2;
+    uint32_t h[H];
+#pragma unroll
+    for (int j = 0; j < H; ++j)
+        h[j] = (uint32_t)f2h(x[2 * j]) | ((uint32_t)f2h(x[2 * j + 1]) << 16);
+    if constexpr (E == 8) {
+        if (vec >= 16) {
+            __stcs(reinterpret_cast<uint4*>(p), make_uint4(h[0], h[1], h[2], h[3]));
+            return;
+        }
+    }
+    if constexpr (E >= 4) {
+        if (vec >= 8) {
+#pragma unroll
+            for (int j = 0; j < H; j += 2)
+                __stcs(reinterpret_cast<uint2*>(p + 2 * j), make_uint2(h[j], h[j + 1]));
+            return;
+        }
+    }
+    if (vec >= 4) {
+#pragma unroll
+        for (int j = 0; j < H; ++j) __stcs(reinterpret_cast<unsigned int*>(p + 2 * j), h[j]);
+        return;
+    }
+#pragma unroll
+    for (int j = 0; j < H; ++j) {
+        __stcs(reinterpret_cast<unsigned short*>(p + 2 * j), (unsigned short)(h[j] & 0xffffu));
+        __stcs(reinterpret_cast<unsigned short*>(p + 2 * j + 1), (unsigned short)(h[j] >> 16));
+    }
+}
+
+__device__ __forceinline__ void flag_overflow(bool bad, uint32_t* status) {
+    const unsigned any = __ballot_sync(0xffffffffu, bad);
+    if (any && (threadIdx.x & 31) == 0) atomicOr(status, ZERO_FLAG_OVERFLOW);
+}
+
+// ---------------------------------------------------------------------------------------------
+// the producer: one thread per CTA fills the stages of the CTA's tiles
+// ---------------------------------------------------------------------------------------------
+template <typename IssueTile>
+__device__ void produce(uint64_t num_tiles, int stages, uint64_t* full, uint64_t* empty,
+                        uint32_t* status, IssueTile issue) {
+    uint32_t it = 0;
+    bool ok = true;
+    for (uint64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+        const int s = (int)(it % (uint32_t)stages);
+        const uint32_t use = it / (uint32_t)stages;
+        // the stage's previous tile must have been read by all consumer warps
+        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1u)) {
+            ok = false;
+            break;
+        }
+        issue(tile, s, &full[s]);
+    }
+    if (!ok) {
+        atomicOr(status, ZERO_FLAG_TIMEOUT);
+        // let every copy this thread started land before the CTA can exit
+        const uint32_t issued = it;
+        for (int s = 0; s < stages && (uint32_t)s < issued; ++s) {
+            const uint32_t last = (uint32_t)s + ((issued - 1u - (uint32_t)s) / (uint32_t)stages) * (uint32_t)stages;
+            (void)mbar_wait(&full[s], (last / (uint32_t)stages) & 1u);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// fused step: reduce-scatter + unscale + Adam + fp16 cast + write-back, TMA-pipelined
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void fused_element(const FusedArgs& p, uint64_t i, bool& bad) {
+    float s = 0.0f;
+    for (int r = 0; r < p.nd; ++r) s = __fadd_rn(s, h2f(p.grads[r][i]));
+    const float red = mean_of(s, p.mc);
+    bad |= non_finite(red);
+    float w = p.master_in[i], m = p.m_in[i], v = p.v_in[i];
+    adam_elem(red, w, m, v, p.a);
+    p.master_out[i] = w;
+    p.m_out[i] = m;
+    p.v_out[i] = v;
+    p.param_out[i] = f2h(w);
+}
+
+template <int E>
+__global__ void __launch_bounds__(kThreads, 1) fused_tma_kernel(const __grid_constant__ FusedArgs p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + kMaxStages;
+    uint8_t* data = smem + kDataOffset;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t T = p.tile;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == kConsumerWarps) {
+        if (lane == 0) {
+            produce(p.num_tiles, p.stages, full, empty, p.status,
+                    [&](uint64_t tile, int s, uint64_t* bar) {
+                        const uint64_t base = tile * T;
+                        const uint64_t left = p.n_tiled - base;
+                        const uint32_t cnt = left < T ? (uint32_t)left : T;
+                        uint8_t* st = data + (size_t)s * p.stage_bytes;
+                        const uint32_t gb = cnt * 2u, fb = cnt * 4u;
+                        mbar_arrive_expect_tx(bar, gb * (uint32_t)p.nd + 3u * fb);
+                        for (int r = 0; r < p.nd; ++r)
+                            bulk_g2s(st + (size_t)r * T * 2u, p.grads[r] + base, gb, bar);
+                        uint8_t* sf = st + (size_t)p.nd * T * 2u;
+                        bulk_g2s(sf, p.master_in + base, fb, bar);
+                        bulk_g2s(sf + (size_t)T * 4u, p.m_in + base, fb, bar);
+                        bulk_g2s(sf + (size_t)T * 8u, p.v_in + base, fb, bar);
+                    });
+        }
+        return;
+    }
+
+    // consumers: thread t owns elements [t*E, t*E + E) of every tile
+    bool bad = false;
+    const uint32_t e0 = (uint32_t)threadIdx.x * E;
+    uint32_t it = 0;
+    for (uint64_t tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
+        const int s = (int)(it % (uint32_t)p.stages);
+        const uint32_t use = it / (uint32_t)p.stages;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], use & 1u));
+        if (!ok) {
+            if (lane == 0) atomicOr(p.status, ZERO_FLAG_TIMEOUT);
+            break;
+        }
+        const uint64_t base = tile * T;
+        const uint64_t left = p.n_tiled - base;
+        const uint32_t cnt = left < T ? (uint32_t)left : T;
+        const bool active = e0 < cnt;   // cnt is a multiple of 8, E divides 8
+        const uint8_t* st = data + (size_t)s * p.stage_bytes;
+        float acc[E], w[E], m[E], v[E];
+        if (active) {
+#pragma unroll
+            for (int j = 0; j < E; ++j) acc[j] = 0.0f;
+            const uint8_t* row = st + (size_t)e0 * 2u;
+#pragma unroll 4
+            for (int r = 0; r < p.nd; ++r) {
+                float x[E];
+                lds_f16<E>(row + (size_t)r * T * 2u, x);
+#pragma unroll
+                for (int j = 0; j < E; ++j) acc[j] = __fadd_rn(acc[j], x[j]);
+            }
+            const uint8_t* sf = st + (size_t)p.nd * T * 2u + (size_t)e0 * 4u;
+            lds_f32<E>(sf, w);
+            lds_f32<E>(sf + (size_t)T * 4u, m);
+            lds_f32<E>(sf + (size_t)T * 8u, v);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);   // stage s may be refilled
+        if (active) {
+#pragma unroll
+            for (int j = 0; j < E; ++j) {
+                const float red = mean_of(acc[j], p.mc);
+                bad |= non_finite(red);
+                adam_elem(red, w[j], m[j], v[j], p.a);
+            }
+            const uint64_t g0 = base + e0;
+            stg_f32<E>(p.master_out + g0, w);
+            stg_f32<E>(p.m_out + g0, m);
+            stg_f32<E>(p.v_out + g0, v);
+            stg_f16<E>(p.param_out + g0, w, p.param_vec);
+        }
+    }
+    // the < 8 elements past the last tile
+    if (blockIdx.x == 0 && (uint64_t)threadIdx.x < p.n - p.n_tiled)
+        fused_element(p, p.n_tiled + threadIdx.x, bad);
+    flag_overflow(bad, p.status);
+}
+
+// plain-load variant for ranges whose pointers are not 16-byte aligned (or tiny ranges)
+__global__ void __launch_bounds__(256) fused_plain_kernel(const __grid_constant__ FusedArgs p) {
+    bool bad = false;
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n; i += stride)
+        fused_element(p, i, bad);
+    flag_overflow(bad, p.status);
+}
+
+// ---------------------------------------------------------------------------------------------
+// bucketed reduce-scatter: red -> owner shard, TMA-pipelined
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t owner_of(uint64_t f, const RsArgs& p) {
+    uint64_t o = (uint64_t)((double)f * p.inv_shard);
+    while (o > 0 && o * p.shard > f) --o;
+    while ((o + 1) * p.shard <= f) ++o;
+    return (uint32_t)o;
+}
+
+__device__ __forceinline__ void rs_store_one(const RsArgs& p, uint64_t local, float red) {
+    const uint64_t f = p.flat_lo + local;
+    const uint32_t o = owner_of(f, p);
+    __stcs(p.shards[o] + (f - (uint64_t)o * p.shard), red);
+}
+
+__device__ __forceinline__ void rs_element(const RsArgs& p, uint64_t i, bool& bad) {
+    float s = 0.0f;
+    for (int r = 0; r < p.nd; ++r) s = __fadd_rn(s, h2f(p.grads[r][i]));
+    const float red = mean_of(s, p.mc);
+    bad |= non_finite(red);
+    rs_store_one(p, i, red);
+}
+
+template <int E>
+__global__ void __launch_bounds__(kThreads, 1) rs_tma_kernel(const __grid_constant__ RsArgs p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + kMaxStages;
+    uint8_t* data = smem + kDataOffset;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t T = p.tile;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == kConsumerWarps) {
+        if (lane == 0) {
+            produce(p.num_tiles, p.stages, full, empty, p.status,
+                    [&](uint64_t tile, int s, uint64_t* bar) {
+                        const uint64_t base = tile * T;
+                        const uint64_t left = p.n_tiled - base;
+                        const uint32_t cnt = left < T ? (uint32_t)left : T;
+                        uint8_t* st = data + (size_t)s * p.stage_bytes;
+                        const uint32_t gb = cnt * 2u;
+                        mbar_arrive_expect_tx(bar, gb * (uint32_t)p.nd);
+                        for (int r = 0; r < p.nd; ++r)
+                            bulk_g2s(st + (size_t)r * T * 2u, p.grads[r] + base, gb, bar);
+                    });
+        }
+        return;
+    }
+
+    bool bad = false;
+    const uint32_t e0 = (uint32_t)threadIdx.x * E;
+    uint32_t it = 0;
+    for (uint64_t tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
+        const int s = (int)(it % (uint32_t)p.stages);
+        const uint32_t use = it / (uint32_t)p.stages;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], use & 1u));
+        if (!ok) {
+            if (lane == 0) atomicOr(p.status, ZERO_FLAG_TIMEOUT);
+            break;
+        }
+        const uint64_t base = tile * T;
+        const uint64_t left = p.n_tiled - base;
+        const uint32_t cnt = left < T ? (uint32_t)left : T;
+        const bool active = e0 < cnt;
+        const uint8_t* st = data + (size_t)s * p.stage_bytes;
+        float acc[E];
+        if (active) {
+#pragma unroll
+            for (int j = 0; j < E; ++j) acc[j] = 0.0f;
+            const uint8_t* row = st + (size_t)e0 * 2u;
+#pragma unroll 4
+            for (int r = 0; r < p.nd; ++r) {
+                float x[E];
+                lds_f16<E>(row + (size_t)r * T * 2u, x);
+#pragma unroll
+                for (int j = 0; j < E; ++j) acc[j] = __fadd_rn(acc[j], x[j]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (active) {
+#pragma unroll
+            for (int j = 0; j < E; ++j) {
+                acc[j] = mean_of(acc[j], p.mc);
+                bad |= non_finite(acc[j]);
+            }
+            const uint64_t l0 = base + e0;
+            const uint64_t f0 = p.flat_lo + l0;
+            const uint32_t o0 = owner_of(f0, p);
+            const uint32_t o1 = owner_of(f0 + E - 1, p);
+            if (o0 == o1) {
+                stg_f32_any<E>(p.shards[o0] + (f0 - (uint64_t)o0 * p.shard), acc);
+            } else {
+#pragma unroll
+                for (int j = 0; j < E; ++j) rs_store_one(p, l0 + j, acc[j]);
+            }
+        }
+    }
+    if (blockIdx.x == 0 && (uint64_t)threadIdx.x < p.n - p.n_tiled)
+        rs_element(p, p.n_tiled + threadIdx.x, bad);
+    flag_overflow(bad, p.status);
+}
+
+__global__ void __launch_bounds__(256) rs_plain_kernel(const __grid_constant__ RsArgs p) {
+    bool bad = false;
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n; i += stride)
+        rs_element(p, i, bad);
+    flag_overflow(bad, p.status);
+}
+
+// ---------------------------------------------------------------------------------------------
+// owner update of a shard from its reduced gradient (unfused path), in place
+// ---------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) adam_kernel(const __grid_constant__ AdamArgs p) {
+    // skip the whole step if any reduce-scatter of it saw inf/NaN
+    if (*reinterpret_cast<volatile uint32_t*>(p.status) & ZERO_FLAG_OVERFLOW) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.status, ZERO_FLAG_SKIPPED);
+        return;
+    }
+    const uint64_t tid = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    uint64_t done = 0;
+    if (p.vec) {
+        const uint64_t n4 = p.n / 4;
+        for (uint64_t q = tid; q < n4; q += stride) {
+            const float4 g = __ldcs(reinterpret_cast<const float4*>(p.grad) + q);
+            float4 w = __ldcs(reinterpret_cast<const float4*>(p.master) + q);
+            float4 m = __ldcs(reinterpret_cast<const float4*>(p.m) + q);
+            float4 v = __ldcs(reinterpret_cast<const float4*>(p.v) + q);
+            adam_elem(g.x, w.x, m.x, v.x, p.a);
+            adam_elem(g.y, w.y, m.y, v.y, p.a);
+            adam_elem(g.z, w.z, m.z, v.z, p.a);
+            adam_elem(g.w, w.w, m.w, v.w, p.a);
+            __stcs(reinterpret_cast<float4*>(p.master) + q, w);
+            __stcs(reinterpret_cast<float4*>(p.m) + q, m);
+            __stcs(reinterpret_cast<float4*>(p.v) + q, v);
+            const float x[4] = {w.x, w.y, w.z, w.w};
+            stg_f16<4>(p.param_out + 4 * q, x, p.param_vec);
+        }
+        done = n4 * 4;
+    }
+    for (uint64_t i = done + tid; i < p.n; i += stride) {
+        float w = p.master[i], m = p.m[i], v = p.v[i];
+        adam_elem(p.grad[i], w, m, v, p.a);
+        p.master[i] = w;
+        p.m[i] = m;
+        p.v[i] = v;
+        p.param_out[i] = f2h(w);
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// commit / skip of a fused step
+// ---------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) commit_kernel(const __grid_constant__ CommitArgs p) {
+    if (!(*reinterpret_cast<volatile uint32_t*>(p.status) & ZERO_FLAG_OVERFLOW)) return;
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.status, ZERO_FLAG_SKIPPED);
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n; i += stride) {
+        const float w = p.master_in[i];
+        p.master_out[i] = w;
+        p.m_out[i] = p.m_in[i];
+        p.v_out[i] = p.v_in[i];
+        p.param_out[i] = f2h(w);
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------------------
+std::atomic<uint64_t> g_launches{0};
+std::mutex g_mu;
+
+struct DevInfo {
+    int sms = 0;
+};
+
+cudaError_t dev_info(DevInfo* out) {
+    static DevInfo cache[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (cache[dev].sms == 0) {
+        int sms = 0;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        cache[dev].sms = sms;
+    }
+    *out = cache[dev];
+    return cudaSuccess;
+}
+
+// Resident CTAs per SM of a pipeline kernel with `smem` dynamic bytes (cached per device).
+template <typename K>
+cudaError_t pipe_blocks_per_sm(K kernel, size_t smem, int* out) {
+    static std::map<std::tuple<int, const void*, size_t>, int> cache;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto key = std::make_tuple(dev, (const void*)kernel, smem);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+        *out = it->second;
+        return cudaSuccess;
+    }
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int b = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (b < 1) return cudaErrorInvalidConfiguration;
+    cache[key] = b;
+    *out = b;
+    return cudaSuccess;
+}
+
+struct PipeShape {
+    int E;
+    uint32_t tile;
+    uint32_t stage_bytes;
+    int stages;
+    size_t smem;
+};
+
+PipeShape pipe_shape(int nd, uint32_t state_bytes_per_elem) {
+    PipeShape s;
+    s.E = nd <= 8 ? 8 : (nd <= 24 ? 4 : 2);
+    s.tile = (uint32_t)(kConsumerThreads * s.E);
+    s.stage_bytes = s.tile * (2u * (uint32_t)nd + state_bytes_per_elem);
+    size_t st = kSmemBudget / s.stage_bytes;
+    if (st < 2) st = 2;
+    if (st > kMaxStages) st = kMaxStages;
+    s.stages = (int)st;
+    s.smem = (size_t)kDataOffset + st * s.stage_bytes;
+    return s;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int store_vec(const void* p) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return (a & 15u) == 0 ? 16 : (a & 7u) == 0 ? 8 : (a & 3u) == 0 ? 4 : 2;
+}
+
+constexpr uint64_t kMinTiledElems = 4096;
+
+template <typename K, typename A>
+cudaError_t launch_pipe(K kernel, const A& args, const PipeShape& sh, cudaStream_t stream) {
+    DevInfo di;
+    cudaError_t e = dev_info(&di);
+    if (e != cudaSuccess) return e;
+    int bps = 1;
+    e = pipe_blocks_per_sm(kernel, sh.smem, &bps);
+    if (e != cudaSuccess) return e;
+    uint64_t grid = (uint64_t)di.sms * (uint64_t)bps;
+    if (args.num_tiles < grid) grid = args.num_tiles;
+    if (grid < 1) grid = 1;
+    kernel<<<(unsigned)grid, kThreads, sh.smem, stream>>>(args);
+    count_launch();
+    return cudaGetLastError();
+}
+
+unsigned plain_grid(uint64_t n, int sms) {
+    uint64_t blocks = (n + 255) / 256;
+    const uint64_t cap = (uint64_t)sms * 8;
+    if (blocks > cap) blocks = cap;
+    return (unsigned)(blocks ? blocks : 1);
+}
+
+}  // namespace
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+uint64_t launches() { return g_launches.load(std::memory_order_relaxed); }
+
+cudaError_t launch_fused(uint64_t n, int nd, const uint16_t* const* grads, const float* master_in,
+                         const float* m_in, const float* v_in, float* master_out, float* m_out,
+                         float* v_out, uint16_t* param_out, const AdamConsts& a,
+                         const MeanConsts& mc, uint32_t* status, cudaStream_t stream) {
+    FusedArgs p;
+    memset(&p, 0, sizeof(p));
+    bool all16 = aligned16(master_in) && aligned16(m_in) && aligned16(v_in) &&
+                 aligned16(master_out) && aligned16(m_out) && aligned16(v_out);
+    for (int r = 0; r < nd; ++r) {
+        p.grads[r] = grads[r];
+        all16 = all16 && aligned16(grads[r]);
+    }
+    p.master_in = master_in;
+    p.m_in = m_in;
+    p.v_in = v_in;
+    p.master_out = master_out;
+    p.m_out = m_out;
+    p.v_out = v_out;
+    p.param_out = param_out;
+    p.status = status;
+    p.n = n;
+    p.nd = nd;
+    p.param_vec = store_vec(param_out);
+    p.a = a;
+    p.mc = mc;
+    DevInfo di;
+    cudaError_t e = dev_info(&di);
+    if (e != cudaSuccess) return e;
+    if (!all16 || n < kMinTiledElems) {
+        fused_plain_kernel<<<plain_grid(n, di.sms), 256, 0, stream>>>(p);
+        count_launch();
+        return cudaGetLastError();
+    }
+    const PipeShape sh = pipe_shape(nd, 12);
+    p.tile = sh.tile;
+    p.stage_bytes = sh.stage_bytes;
+    p.stages = sh.stages;
+    p.n_tiled = n & ~(uint64_t)7;
+    p.num_tiles = (p.n_tiled + sh.tile - 1) / sh.tile;
+    switch (sh.E) {
+        case 8: return launch_pipe(fused_tma_kernel<8>, p, sh, stream);
+        case 4: return launch_pipe(fused_tma_kernel<4>, p, sh, stream);
+        default: return launch_pipe(fused_tma_kernel<2>, p, sh, stream);
+    }
+}
+
+cudaError_t launch_reduce_scatter(uint64_t n, int nd, const uint16_t* const* grads,
+                                  float* const* shards, uint64_t flat_lo, uint64_t shard,
+                                  const MeanConsts& mc, uint32_t* status, cudaStream_t stream) {
+    RsArgs p;
+    memset(&p, 0, sizeof(p));
+    bool all16 = true;
+    for (int r = 0; r < nd; ++r) {
+        p.grads[r] = grads[r];
+        p.shards[r] = shards[r];
+        all16 = all16 && aligned16(grads[r]);
+    }
+    p.status = status;
+    p.n = n;
+    p.flat_lo = flat_lo;
+    p.shard = shard;
+    p.inv_shard = 1.0 / (double)shard;
+    p.nd = nd;
+    p.mc = mc;
+    DevInfo di;
+    cudaError_t e = dev_info(&di);
+    if (e != cudaSuccess) return e;
+    if (!all16 || n < kMinTiledElems) {
+        rs_plain_kernel<<<plain_grid(n, di.sms), 256, 0, stream>>>(p);
+        count_launch();
+        return cudaGetLastError();
+    }
+    const PipeShape sh = pipe_shape(nd, 0);
+    p.tile = sh.tile;
+    p.stage_bytes = sh.stage_bytes;
+    p.stages = sh.stages;
+    p.n_tiled = n & ~(uint64_t)7;
+    p.num_tiles = (p.n_tiled + sh.tile - 1) / sh.tile;
+    switch (sh.E) {
+        case 8: return launch_pipe(rs_tma_kernel<8>, p, sh, stream);
+        case 4: return launch_pipe(rs_tma_kernel<4>, p, sh, stream);
+        default: return launch_pipe(rs_tma_kernel<2>, p, sh, stream);
+    }
+}
+
+cudaError_t launch_adam(uint64_t n, const float* grad, float* master, float* m, float* v,
+                        uint16_t* param_out, const AdamConsts& a, uint32_t* status,
+                        cudaStream_t stream) {
+    AdamArgs p;
+    memset(&p, 0, sizeof(p));
+    p.grad = grad;
+    p.master = master;
+    p.m = m;
+    p.v = v;
+    p.param_out = param_out;
+    p.status = status;
+    p.n = n;
+    p.vec = aligned16(grad) && aligned16(master) && aligned16(m) && aligned16(v);
+    const int pv = store_vec(param_out);
+    p.param_vec = pv > 8 ? 8 : pv;
+    p.a = a;
+    DevInfo di;
+    cudaError_t e = dev_info(&di);
+    if (e != cudaSuccess) return e;
+    uint64_t work = p.vec ? (n + 3) / 4 : n;
+    adam_kernel<<<plain_grid(work, di.sms), 256, 0, stream>>>(p);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_commit(uint64_t n, const float* master_in, const float* m_in,
+                          const float* v_in, float* master_out, float* m_out, float* v_out,
+                          uint16_t* param_out, uint32_t* status, cudaStream_t stream) {
+    CommitArgs p;
+    p.master_in = master_in;
+    p.m_in = m_in;
+    p.v_in = v_in;
+    p.master_out = master_out;
+    p.m_out = m_out;
+    p.v_out = v_out;
+    p.param_out = param_out;
+    p.status = status;
+    p.n = n;
+    DevInfo di;
+    cudaError_t e = dev_info(&di);
+    if (e != cudaSuccess) return e;
+    commit_kernel<<<plain_grid(n, di.sms), 256, 0, stream>>>(p);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace zk

@@ -1,0 +1,176 @@
+// Stream-ordered bucket scheduler for ZeRO stage 2.
+//
+// "ZeRO-2" card (llm-engineer.pages.dev), section "Gradient 생명주기": during the backward pass
+// each layer's (bucket's) local gradient is reduce-scattered as soon as it exists; the GPU keeps
+// only its own reduced shard and releases the rest of the local gradient; this repeats for
+// every bucket. Diagram: buckets B2, B1, B0 are produced and reduce-scattered in that order.
+//
+// Here the local gradients of a bucket (all Nd simulated ranks) live in a staging slot. The
+// producer (the backward pass, or whatever stands for it) fills the slot on its own stream; the
+// reduce-scatter runs on the scheduler's stream after a CUDA event says the fill is done; when
+// the reduce-scatter has read the slot, another event releases the slot, and the producer's
+// stream waits on that event before it fills the slot with a later bucket. The host never
+// blocks: all ordering is carried by events, so the fill of bucket k+1 overlaps the
+// reduce-scatter of bucket k whenever more than one slot exists.
+#include <cstdint>
+#include <new>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "../../include/libzero.h"
+#include "zero_internal.h"
+
+struct zero_sched {
+    const zero_plan* plan = nullptr;
+    int nd = 0;
+    int n_slots = 0;
+    uint64_t stride = 0;                 // fp16 elements per rank region of a slot
+    uint16_t* slot_mem = nullptr;
+    float* shards[ZERO_MAX_RANKS] = {};
+    uint32_t* status = nullptr;
+    cudaStream_t rs = nullptr;
+    std::vector<cudaEvent_t> produced;   // per slot: the producer finished filling it
+    std::vector<cudaEvent_t> released;   // per slot: its last reduce-scatter finished
+    std::vector<int> filled;             // per slot: released[] has been recorded once
+    std::vector<int> bucket_of_slot;     // per slot: the bucket begun in it (-1: none)
+    cudaEvent_t tail = nullptr;          // scratch event for zero_sched_wait
+    uint64_t launches = 0;
+};
+
+namespace {
+
+uint64_t round8(uint64_t x) { return (x + 7) & ~(uint64_t)7; }
+
+void destroy_events(zero_sched* s) {
+    for (cudaEvent_t e : s->produced)
+        if (e) cudaEventDestroy(e);
+    for (cudaEvent_t e : s->released)
+        if (e) cudaEventDestroy(e);
+    if (s->tail) cudaEventDestroy(s->tail);
+    s->produced.clear();
+    s->released.clear();
+    s->tail = nullptr;
+}
+
+}  // namespace
+
+extern "C" {
+
+zero_status zero_sched_slot_elems(const zero_plan* plan, int n_slots, uint64_t* elems) {
+    int nd = 0;
+    uint64_t psi_p = 0, S = 0;
+    if (!elems || n_slots < 1 || !zk::plan_geometry(plan, &nd, &psi_p, &S)) return ZERO_EINVAL;
+    *elems = (uint64_t)n_slots * (uint64_t)nd * round8(zk::plan_max_bucket(plan));
+    return ZERO_OK;
+}
+
+zero_status zero_sched_create(const zero_plan* plan, uint16_t* slot_mem, uint64_t slot_mem_elems,
+                              int n_slots, float* const* owner_grad_shards, uint32_t* d_status,
+                              zero_stream_t rs_stream, zero_sched** out) {
+    if (!out) return ZERO_EINVAL;
+    *out = nullptr;
+    int nd = 0;
+    uint64_t psi_p = 0, S = 0;
+    if (!zk::plan_geometry(plan, &nd, &psi_p, &S) || n_slots < 1 || !slot_mem ||
+        !owner_grad_shards || !d_status)
+        return ZERO_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(slot_mem) & 15u) || (reinterpret_cast<uintptr_t>(d_status) & 3u))
+        return ZERO_EALIGN;
+    uint64_t need = 0;
+    zero_sched_slot_elems(plan, n_slots, &need);
+    if (slot_mem_elems < need) return ZERO_ENOMEM;
+    for (int r = 0; r < nd; ++r) {
+        if (!owner_grad_shards[r]) return ZERO_EINVAL;
+        if (reinterpret_cast<uintptr_t>(owner_grad_shards[r]) & 3u) return ZERO_EALIGN;
+    }
+    zero_sched* s = new (std::nothrow) zero_sched();
+    if (!s) return ZERO_ENOMEM;
+    s->plan = plan;
+    s->nd = nd;
+    s->n_slots = n_slots;
+    s->stride = round8(zk::plan_max_bucket(plan));
+    s->slot_mem = slot_mem;
+    for (int r = 0; r < nd; ++r) s->shards[r] = owner_grad_shards[r];
+    s->status = d_status;
+    s->rs = (cudaStream_t)rs_stream;
+    try {
+        s->produced.assign((size_t)n_slots, nullptr);
+        s->released.assign((size_t)n_slots, nullptr);
+        s->filled.assign((size_t)n_slots, 0);
+        s->bucket_of_slot.assign((size_t)n_slots, -1);
+    } catch (...) {
+        delete s;
+        return ZERO_ENOMEM;
+    }
+    bool ok = cudaEventCreateWithFlags(&s->tail, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; ok && i < n_slots; ++i) {
+        ok = cudaEventCreateWithFlags(&s->produced[(size_t)i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&s->released[(size_t)i], cudaEventDisableTiming) == cudaSuccess;
+    }
+    if (!ok) {
+        destroy_events(s);
+        delete s;
+        return ZERO_ECUDA;
+    }
+    *out = s;
+    return ZERO_OK;
+}
+
+zero_status zero_sched_begin_bucket(zero_sched* s, int k, zero_stream_t producer,
+                                    uint16_t** rank_ptrs) {
+    uint64_t lo = 0, len = 0;
+    if (!s || !rank_ptrs || !zk::plan_bucket_range(s->plan, k, &lo, &len)) return ZERO_EINVAL;
+    const int slot = k % s->n_slots;
+    if (s->filled[(size_t)slot]) {
+        // the slot still holds an earlier bucket until its reduce-scatter has finished
+        if (cudaStreamWaitEvent((cudaStream_t)producer, s->released[(size_t)slot], 0) != cudaSuccess)
+            return ZERO_ECUDA;
+    }
+    s->bucket_of_slot[(size_t)slot] = k;
+    for (int r = 0; r < s->nd; ++r)
+        rank_ptrs[r] = s->slot_mem + ((uint64_t)slot * (uint64_t)s->nd + (uint64_t)r) * s->stride;
+    return ZERO_OK;
+}
+
+zero_status zero_sched_end_bucket(zero_sched* s, int k, zero_stream_t producer) {
+    uint64_t lo = 0, len = 0;
+    if (!s || !zk::plan_bucket_range(s->plan, k, &lo, &len)) return ZERO_EINVAL;
+    const int slot = k % s->n_slots;
+    if (s->bucket_of_slot[(size_t)slot] != k) return ZERO_EINVAL;   // not begun
+    const uint16_t* ptrs[ZERO_MAX_RANKS];
+    for (int r = 0; r < s->nd; ++r)
+        ptrs[r] = s->slot_mem + ((uint64_t)slot * (uint64_t)s->nd + (uint64_t)r) * s->stride;
+    cudaEvent_t prod = s->produced[(size_t)slot];
+    if (cudaEventRecord(prod, (cudaStream_t)producer) != cudaSuccess) return ZERO_ECUDA;
+    if (cudaStreamWaitEvent(s->rs, prod, 0) != cudaSuccess) return ZERO_ECUDA;
+    if (zk::rs_bucket_launch(s->plan, k, ptrs, s->shards, s->status, s->rs) != cudaSuccess)
+        return ZERO_ECUDA;
+    ++s->launches;
+    // release: the slot may be refilled once this reduce-scatter is done with it
+    if (cudaEventRecord(s->released[(size_t)slot], s->rs) != cudaSuccess) return ZERO_ECUDA;
+    s->filled[(size_t)slot] = 1;
+    s->bucket_of_slot[(size_t)slot] = -1;
+    return ZERO_OK;
+}
+
+zero_status zero_sched_wait(zero_sched* s, zero_stream_t stream) {
+    if (!s) return ZERO_EINVAL;
+    if (cudaEventRecord(s->tail, s->rs) != cudaSuccess) return ZERO_ECUDA;
+    if (cudaStreamWaitEvent((cudaStream_t)stream, s->tail, 0) != cudaSuccess) return ZERO_ECUDA;
+    return ZERO_OK;
+}
+
+zero_status zero_sched_launches(const zero_sched* s, uint64_t* count) {
+    if (!s || !count) return ZERO_EINVAL;
+    *count = s->launches;
+    return ZERO_OK;
+}
+
+void zero_sched_destroy(zero_sched* s) {
+    if (!s) return;
+    destroy_events(s);
+    delete s;
+}
+
+}  // extern "C"

@@ -1,0 +1,318 @@
+"""Python binding of libzero.so (argument marshalling only).
+
+Every function has the name of the C entry point it calls (include/libzero.h) and does no
+arithmetic of its own. Device buffers are given as torch tensors (their data_ptr() is passed)
+or as raw integer addresses; streams as torch.cuda.Stream, a raw cudaStream_t integer, or None
+for torch's current stream. A non-OK status raises ZeroError, except zero_step_status, which
+returns it.
+
+Importing this module loads the in-tree libzero.so and fails loudly if it has not been built
+(``python -m zero_partitioned_optimizer_plan_b200.build``): there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import dataclasses
+import os
+from typing import List, Sequence
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libzero.so")
+
+ZERO_OK = 0
+ZERO_EINVAL = 1
+ZERO_EALIGN = 2
+ZERO_ECUDA = 3
+ZERO_ENOMEM = 4
+ZERO_STEP_SKIPPED = 5
+
+ZERO_FLAG_OVERFLOW = 0x1
+ZERO_FLAG_SKIPPED = 0x2
+ZERO_FLAG_TIMEOUT = 0x4
+
+ZERO_MAX_RANKS = 64
+
+# every symbol include/libzero.h declares
+SYMBOLS = (
+    "zero_status_string", "zero_kernel_launches",
+    "zero_plan_create", "zero_plan_destroy", "zero_plan_info", "zero_plan_tensor_offsets",
+    "zero_plan_bucket", "zero_state_bytes",
+    "zero_reduce_scatter_bucket", "zero_adam_shard", "zero_step_fused", "zero_step_commit",
+    "zero_step_status",
+    "zero_sched_slot_elems", "zero_sched_create", "zero_sched_begin_bucket",
+    "zero_sched_end_bucket", "zero_sched_wait", "zero_sched_launches", "zero_sched_destroy",
+)
+
+
+class ZeroError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {zero_status_string(code)}")
+
+
+class _Bytes(C.Structure):
+    _fields_ = [("params", C.c_uint64), ("grads", C.c_uint64), ("optim", C.c_uint64),
+                ("total", C.c_uint64)]
+
+
+class _Report(C.Structure):
+    _fields_ = [("stage", _Bytes * 4), ("comm_elems", C.c_uint64 * 4),
+                ("comm_bytes_fp16", C.c_uint64 * 4)]
+
+
+class _HP(C.Structure):
+    _fields_ = [("lr", C.c_double), ("beta1", C.c_double), ("beta2", C.c_double),
+                ("eps", C.c_double), ("loss_scale", C.c_double)]
+
+
+@dataclasses.dataclass(frozen=True)
+class AdamHP:
+    lr: float = 1e-3
+    beta1: float = 0.9
+    beta2: float = 0.999
+    eps: float = 1e-8
+    loss_scale: float = 1024.0
+
+    def _c(self):
+        return _HP(self.lr, self.beta1, self.beta2, self.eps, self.loss_scale)
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libzero.so is not built ({LIB_PATH}); run "
+            "`python -m zero_partitioned_optimizer_plan_b200.build` (needs nvcc)")
+    L = C.CDLL(LIB_PATH)
+    u64, i64, vp, i32 = C.c_uint64, C.c_int64, C.c_void_p, C.c_int
+    P = C.POINTER
+    L.zero_status_string.argtypes, L.zero_status_string.restype = [i32], C.c_char_p
+    L.zero_kernel_launches.argtypes, L.zero_kernel_launches.restype = [], u64
+    L.zero_plan_create.argtypes = [P(u64), i32, i32, i32, u64, P(vp)]
+    L.zero_plan_destroy.argtypes, L.zero_plan_destroy.restype = [vp], None
+    L.zero_plan_info.argtypes = [vp, P(u64), P(u64), P(u64), P(i32)]
+    L.zero_plan_tensor_offsets.argtypes = [vp, P(u64)]
+    L.zero_plan_bucket.argtypes = [vp, i32, P(u64), P(u64), P(i32), P(i32)]
+    L.zero_state_bytes.argtypes = [u64, i32, i32, P(_Report)]
+    L.zero_reduce_scatter_bucket.argtypes = [vp, i32, P(vp), P(vp), vp, vp]
+    L.zero_adam_shard.argtypes = [u64, vp, vp, vp, vp, vp, P(_HP), i64, vp, vp]
+    L.zero_step_fused.argtypes = [u64, i32, P(vp), vp, vp, vp, vp, vp, vp, vp, P(_HP), i64,
+                                  vp, vp]
+    L.zero_step_commit.argtypes = [u64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.zero_step_status.argtypes = [vp, vp, P(C.c_uint32)]
+    L.zero_sched_slot_elems.argtypes = [vp, i32, P(u64)]
+    L.zero_sched_create.argtypes = [vp, vp, u64, i32, P(vp), vp, vp, P(vp)]
+    L.zero_sched_begin_bucket.argtypes = [vp, i32, vp, P(vp)]
+    L.zero_sched_end_bucket.argtypes = [vp, i32, vp]
+    L.zero_sched_wait.argtypes = [vp, vp]
+    L.zero_sched_launches.argtypes = [vp, P(u64)]
+    L.zero_sched_destroy.argtypes, L.zero_sched_destroy.restype = [vp], None
+    # every other entry point returns a zero_status: ctypes' default int restype
+    return L
+
+
+_lib = _load()
+
+
+# ---------------------------------------------------------------------------------------------
+# marshalling helpers
+# ---------------------------------------------------------------------------------------------
+def _ptr(x, elem_size: int | None = None) -> int:
+    if x is None:
+        return 0
+    if hasattr(x, "data_ptr"):
+        if elem_size is not None and x.element_size() != elem_size:
+            raise TypeError(f"expected a tensor of {elem_size}-byte elements, got {x.dtype}")
+        if not x.is_contiguous():
+            raise TypeError("tensor must be contiguous")
+        return int(x.data_ptr())
+    return int(x)
+
+
+def _stream(s) -> int:
+    if s is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    if hasattr(s, "cuda_stream"):
+        return int(s.cuda_stream)
+    return int(s)
+
+
+def _ptr_array(xs, elem_size=None):
+    return (C.c_void_p * max(len(xs), 1))(*[_ptr(x, elem_size) for x in xs])
+
+
+def _check(code: int, where: str):
+    if code != ZERO_OK:
+        raise ZeroError(code, where)
+
+
+def zero_status_string(code: int) -> str:
+    return _lib.zero_status_string(int(code)).decode()
+
+
+def zero_kernel_launches() -> int:
+    return int(_lib.zero_kernel_launches())
+
+
+# ---------------------------------------------------------------------------------------------
+# plan and accounting
+# ---------------------------------------------------------------------------------------------
+class Plan:
+    """Owns a zero_plan handle (host memory)."""
+
+    def __init__(self, handle: int, n_tensors: int):
+        self.handle = handle
+        self.n_tensors = n_tensors
+
+    def __del__(self):
+        if getattr(self, "handle", None):
+            _lib.zero_plan_destroy(self.handle)
+            self.handle = None
+
+
+def zero_plan_create(numels: Sequence[int], nd: int, stage: int = 1, bucket_elems: int = 0) -> Plan:
+    arr = (C.c_uint64 * max(len(numels), 1))(*[int(x) for x in numels])
+    h = C.c_void_p()
+    _check(_lib.zero_plan_create(arr, len(numels), nd, stage, bucket_elems, C.byref(h)),
+           "zero_plan_create")
+    return Plan(h.value, len(numels))
+
+
+def zero_plan_destroy(plan: Plan):
+    if plan.handle:
+        _lib.zero_plan_destroy(plan.handle)
+        plan.handle = None
+
+
+def zero_plan_info(plan: Plan):
+    psi, psi_p, shard = C.c_uint64(), C.c_uint64(), C.c_uint64()
+    nb = C.c_int()
+    _check(_lib.zero_plan_info(plan.handle, C.byref(psi), C.byref(psi_p), C.byref(shard),
+                               C.byref(nb)), "zero_plan_info")
+    return psi.value, psi_p.value, shard.value, nb.value
+
+
+def zero_plan_tensor_offsets(plan: Plan) -> List[int]:
+    out = (C.c_uint64 * max(plan.n_tensors, 1))()
+    _check(_lib.zero_plan_tensor_offsets(plan.handle, out), "zero_plan_tensor_offsets")
+    return list(out[:plan.n_tensors])
+
+
+def zero_plan_bucket(plan: Plan, k: int):
+    lo, ln = C.c_uint64(), C.c_uint64()
+    olo, ohi = C.c_int(), C.c_int()
+    _check(_lib.zero_plan_bucket(plan.handle, k, C.byref(lo), C.byref(ln), C.byref(olo),
+                                 C.byref(ohi)), "zero_plan_bucket")
+    return lo.value, ln.value, olo.value, ohi.value
+
+
+STAGES = ("dp", "pos", "pos_g", "pos_g_p")
+
+
+def zero_state_bytes(psi: int, nd: int, K: int = 12) -> dict:
+    rep = _Report()
+    _check(_lib.zero_state_bytes(psi, nd, K, C.byref(rep)), "zero_state_bytes")
+    out = {}
+    for s, name in enumerate(STAGES):
+        b = rep.stage[s]
+        out[name] = dict(params=b.params, grads=b.grads, optim=b.optim, total=b.total,
+                         comm_elems=rep.comm_elems[s], comm_bytes_fp16=rep.comm_bytes_fp16[s])
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
+# data path
+# ---------------------------------------------------------------------------------------------
+def zero_reduce_scatter_bucket(plan: Plan, k: int, rank_grads, owner_grad_shards, d_status,
+                               stream=None):
+    _check(_lib.zero_reduce_scatter_bucket(plan.handle, k, _ptr_array(rank_grads, 2),
+                                           _ptr_array(owner_grad_shards, 4), _ptr(d_status, 4),
+                                           _stream(stream)), "zero_reduce_scatter_bucket")
+
+
+def zero_adam_shard(n: int, grad, master, m, v, param_out, hp: AdamHP, step: int, d_status,
+                    stream=None):
+    h = hp._c()
+    _check(_lib.zero_adam_shard(n, _ptr(grad, 4), _ptr(master, 4), _ptr(m, 4), _ptr(v, 4),
+                                _ptr(param_out, 2), C.byref(h), step, _ptr(d_status, 4),
+                                _stream(stream)), "zero_adam_shard")
+
+
+def zero_step_fused(n: int, nd: int, rank_grads, master_in, m_in, v_in, master_out, m_out,
+                    v_out, param_out, hp: AdamHP, step: int, d_status, stream=None):
+    h = hp._c()
+    _check(_lib.zero_step_fused(n, nd, _ptr_array(rank_grads, 2), _ptr(master_in, 4),
+                                _ptr(m_in, 4), _ptr(v_in, 4), _ptr(master_out, 4),
+                                _ptr(m_out, 4), _ptr(v_out, 4), _ptr(param_out, 2), C.byref(h),
+                                step, _ptr(d_status, 4), _stream(stream)), "zero_step_fused")
+
+
+def zero_step_commit(n: int, master_in, m_in, v_in, master_out, m_out, v_out, param_out,
+                     d_status, stream=None):
+    _check(_lib.zero_step_commit(n, _ptr(master_in, 4), _ptr(m_in, 4), _ptr(v_in, 4),
+                                 _ptr(master_out, 4), _ptr(m_out, 4), _ptr(v_out, 4),
+                                 _ptr(param_out, 2), _ptr(d_status, 4), _stream(stream)),
+           "zero_step_commit")
+
+
+def zero_step_status(d_status, stream=None):
+    """Blocks until `stream` is done; returns (zero_status code, flags)."""
+    flags = C.c_uint32()
+    code = _lib.zero_step_status(_ptr(d_status, 4), _stream(stream), C.byref(flags))
+    return int(code), int(flags.value)
+
+
+# ---------------------------------------------------------------------------------------------
+# stage-2 bucket scheduler
+# ---------------------------------------------------------------------------------------------
+class Sched:
+    def __init__(self, handle: int, nd: int):
+        self.handle = handle
+        self.nd = nd
+
+    def __del__(self):
+        if getattr(self, "handle", None):
+            _lib.zero_sched_destroy(self.handle)
+            self.handle = None
+
+
+def zero_sched_slot_elems(plan: Plan, n_slots: int) -> int:
+    out = C.c_uint64()
+    _check(_lib.zero_sched_slot_elems(plan.handle, n_slots, C.byref(out)),
+           "zero_sched_slot_elems")
+    return out.value
+
+
+def zero_sched_create(plan: Plan, slot_mem, slot_mem_elems: int, n_slots: int,
+                      owner_grad_shards, d_status, rs_stream=None) -> Sched:
+    h = C.c_void_p()
+    _check(_lib.zero_sched_create(plan.handle, _ptr(slot_mem, 2), slot_mem_elems, n_slots,
+                                  _ptr_array(owner_grad_shards, 4), _ptr(d_status, 4),
+                                  _stream(rs_stream), C.byref(h)), "zero_sched_create")
+    return Sched(h.value, len(owner_grad_shards))
+
+
+def zero_sched_begin_bucket(s: Sched, k: int, producer=None) -> List[int]:
+    out = (C.c_void_p * s.nd)()
+    _check(_lib.zero_sched_begin_bucket(s.handle, k, _stream(producer), out),
+           "zero_sched_begin_bucket")
+    return [int(p) for p in out]
+
+
+def zero_sched_end_bucket(s: Sched, k: int, producer=None):
+    _check(_lib.zero_sched_end_bucket(s.handle, k, _stream(producer)), "zero_sched_end_bucket")
+
+
+def zero_sched_wait(s: Sched, stream=None):
+    _check(_lib.zero_sched_wait(s.handle, _stream(stream)), "zero_sched_wait")
+
+
+def zero_sched_launches(s: Sched) -> int:
+    out = C.c_uint64()
+    _check(_lib.zero_sched_launches(s.handle, C.byref(out)), "zero_sched_launches")
+    return out.value
+
+
+def zero_sched_destroy(s: Sched):
+    if s.handle:
+        _lib.zero_sched_destroy(s.handle)
+        s.handle = None
