@@ -55,6 +55,8 @@ typedef enum {
 #define ZERO_FLAG_OVERFLOW 0x1u /* some reduced gradient of this step was inf or NaN */
 #define ZERO_FLAG_SKIPPED 0x2u  /* the step was not applied (state and params unchanged) */
 #define ZERO_FLAG_TIMEOUT 0x4u  /* a kernel's bounded wait gave up; its outputs are invalid */
+#define ZERO_FLAG_BOUNDS 0x8u   /* a kernel's internal bounds self-check failed (a library bug):
+                                   the access was skipped; outputs are invalid */
 
 #define ZERO_MAX_RANKS 64       /* largest Nd a call accepts */
 
@@ -63,6 +65,10 @@ const char* zero_status_string(zero_status s);
 
 /* Kernels this library has launched in this process so far (all entry points). */
 uint64_t zero_kernel_launches(void);
+
+/* Text of the last CUDA error behind a ZERO_ECUDA returned to this host thread ("" if none);
+ * valid until the next libzero call on the thread. */
+const char* zero_last_error(void);
 
 /* ------------------------------------------------------------------------------------------
  * Partition plan.
@@ -208,8 +214,8 @@ zero_status zero_step_commit(uint64_t n, const float* master_in, const float* m_
                              uint16_t* param_out, uint32_t* d_status, zero_stream_t stream);
 
 /* Wait for `stream`, read *d_status into *flags_out (may be NULL) and map it to a status:
- * ZERO_STEP_SKIPPED if ZERO_FLAG_SKIPPED is set, ZERO_ECUDA if ZERO_FLAG_TIMEOUT is set or the
- * copy fails, else ZERO_OK. This is the only call that blocks the host. */
+ * ZERO_STEP_SKIPPED if ZERO_FLAG_SKIPPED is set, ZERO_ECUDA if ZERO_FLAG_TIMEOUT or ZERO_FLAG_BOUNDS is
+ * set or the copy fails, else ZERO_OK. This is the only call that blocks the host. */
 zero_status zero_step_status(const uint32_t* d_status, zero_stream_t stream, uint32_t* flags_out);
 
 /* ------------------------------------------------------------------------------------------

@@ -328,3 +328,22 @@ def test_step_split_into_bucket_calls():
     for a, b in zip(pp.cur, pp.nxt):
         assert torch.equal(a, b)
     assert np.array_equal(f16np(params), oracle.f2h(master.numpy()))
+
+
+def test_launch_sizes_in_any_order():
+    """Nd changes the pipeline's shared-memory size; alternating sizes on the same kernel
+    must keep launching (each size within the device's opt-in limit)."""
+    n = 2048 * 9 + 5
+    for nd in (1, 2, 1, 7, 6, 1, 64, 33, 64, 25):
+        master, m, v = synth.state_warm(n, seed=nd)
+        pp = PingPong(master, m, v)
+        g_cpu = _rank_grads_cpu(n, nd, 41, 1)
+        params = torch.empty(n, dtype=torch.float16, device=DEV)
+        st = status_word()
+        fused_step(n, [g.to(DEV) for g in g_cpu], pp, params, HP, 1, st)
+        torch.cuda.synchronize()
+        assert status_flags(st) == 0
+        skipped, w, mm, vv, p = oracle.step([g.numpy() for g in g_cpu], master.numpy(),
+                                            m.numpy(), v.numpy(), ORC_HP, 1)
+        check_f32("master", f32np(pp.nxt[0]), w)
+        check_f16("params", f16np(params), p)

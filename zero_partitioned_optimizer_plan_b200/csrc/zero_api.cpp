@@ -2,6 +2,7 @@
 // launches. Every function returns a zero_status and never throws.
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 
 #include <cuda_runtime.h>
@@ -60,9 +61,17 @@ AdamConsts make_adam(const zero_adam_hparams* hp, int64_t t) {
     return a;
 }
 
-zero_status from_cuda(cudaError_t e) { return e == cudaSuccess ? ZERO_OK : ZERO_ECUDA; }
-
 }  // namespace
+
+// The last CUDA failure seen by a libzero call on this host thread.
+thread_local char g_last_error[256] = "";
+
+zero_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return ZERO_OK;
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e),
+             cudaGetErrorString(e));
+    return ZERO_ECUDA;
+}
 
 MeanConsts make_mean(int nd) {
     MeanConsts mc;
@@ -98,6 +107,8 @@ const char* zero_status_string(zero_status s) {
 }
 
 uint64_t zero_kernel_launches(void) { return zk::launches(); }
+
+const char* zero_last_error(void) { return zk::g_last_error; }
 
 zero_status zero_reduce_scatter_bucket(const zero_plan* plan, int k,
                                        const uint16_t* const* rank_grads,
@@ -214,9 +225,9 @@ zero_status zero_step_status(const uint32_t* d_status, zero_stream_t stream, uin
     cudaError_t e = cudaMemcpyAsync(&flags, d_status, sizeof(flags), cudaMemcpyDeviceToHost,
                                     (cudaStream_t)stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
-    if (e != cudaSuccess) return ZERO_ECUDA;
+    if (e != cudaSuccess) return zk::from_cuda(e);
     if (flags_out) *flags_out = flags;
-    if (flags & ZERO_FLAG_TIMEOUT) return ZERO_ECUDA;
+    if (flags & (ZERO_FLAG_TIMEOUT | ZERO_FLAG_BOUNDS)) return ZERO_ECUDA;
     if (flags & ZERO_FLAG_SKIPPED) return ZERO_STEP_SKIPPED;
     return ZERO_OK;
 }

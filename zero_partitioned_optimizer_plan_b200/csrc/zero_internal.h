@@ -58,4 +58,7 @@ cudaError_t rs_bucket_launch(const zero_plan* plan, int k, const uint16_t* const
 
 MeanConsts make_mean(int nd);
 
+// Map a CUDA error to a zero_status, remembering its text for zero_last_error().
+zero_status from_cuda(cudaError_t e);
+
 }  // namespace zk

@@ -352,6 +352,10 @@ __device__ void produce(uint64_t num_tiles, int stages, uint64_t* full, uint64_t
 // fused step: reduce-scatter + unscale + Adam + fp16 cast + write-back, TMA-pipelined
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ void fused_element(const FusedArgs& p, uint64_t i, bool& bad) {
+    if (i >= p.n) {   // self-check: never taken when the launch arithmetic is right
+        atomicOr(p.status, ZERO_FLAG_BOUNDS);
+        return;
+    }
     float s = 0.0f;
     for (int r = 0; r < p.nd; ++r) s = __fadd_rn(s, h2f(p.grads[r][i]));
     const float red = mean_of(s, p.mc);
@@ -392,6 +396,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_tma_kernel(const __grid_con
                         const uint32_t cnt = left < T ? (uint32_t)left : T;
                         uint8_t* st = data + (size_t)s * p.stage_bytes;
                         const uint32_t gb = cnt * 2u, fb = cnt * 4u;
+                        if (base >= p.n_tiled || (cnt & 7u) || s >= p.stages) {
+                            atomicOr(p.status, ZERO_FLAG_BOUNDS);
+                            mbar_arrive_expect_tx(bar, 0);   // release the consumers, no copy
+                            return;
+                        }
                         mbar_arrive_expect_tx(bar, gb * (uint32_t)p.nd + 3u * fb);
                         for (int r = 0; r < p.nd; ++r)
                             bulk_g2s(st + (size_t)r * T * 2u, p.grads[r] + base, gb, bar);
@@ -448,6 +457,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_tma_kernel(const __grid_con
                 adam_elem(red, w[j], m[j], v[j], p.a);
             }
             const uint64_t g0 = base + e0;
+            if (g0 + E > p.n_tiled) {
+                atomicOr(p.status, ZERO_FLAG_BOUNDS);
+                continue;
+            }
             stg_f32<E>(p.master_out + g0, w);
             stg_f32<E>(p.m_out + g0, m);
             stg_f32<E>(p.v_out + g0, v);
@@ -482,10 +495,18 @@ __device__ __forceinline__ uint32_t owner_of(uint64_t f, const RsArgs& p) {
 __device__ __forceinline__ void rs_store_one(const RsArgs& p, uint64_t local, float red) {
     const uint64_t f = p.flat_lo + local;
     const uint32_t o = owner_of(f, p);
+    if (o >= (uint32_t)p.nd) {
+        atomicOr(p.status, ZERO_FLAG_BOUNDS);
+        return;
+    }
     __stcs(p.shards[o] + (f - (uint64_t)o * p.shard), red);
 }
 
 __device__ __forceinline__ void rs_element(const RsArgs& p, uint64_t i, bool& bad) {
+    if (i >= p.n) {
+        atomicOr(p.status, ZERO_FLAG_BOUNDS);
+        return;
+    }
     float s = 0.0f;
     for (int r = 0; r < p.nd; ++r) s = __fadd_rn(s, h2f(p.grads[r][i]));
     const float red = mean_of(s, p.mc);
@@ -521,6 +542,11 @@ __global__ void __launch_bounds__(kThreads, 1) rs_tma_kernel(const __grid_consta
                         const uint32_t cnt = left < T ? (uint32_t)left : T;
                         uint8_t* st = data + (size_t)s * p.stage_bytes;
                         const uint32_t gb = cnt * 2u;
+                        if (base >= p.n_tiled || (cnt & 7u) || s >= p.stages) {
+                            atomicOr(p.status, ZERO_FLAG_BOUNDS);
+                            mbar_arrive_expect_tx(bar, 0);
+                            return;
+                        }
                         mbar_arrive_expect_tx(bar, gb * (uint32_t)p.nd);
                         for (int r = 0; r < p.nd; ++r)
                             bulk_g2s(st + (size_t)r * T * 2u, p.grads[r] + base, gb, bar);
@@ -570,6 +596,10 @@ __global__ void __launch_bounds__(kThreads, 1) rs_tma_kernel(const __grid_consta
             const uint64_t f0 = p.flat_lo + l0;
             const uint32_t o0 = owner_of(f0, p);
             const uint32_t o1 = owner_of(f0 + E - 1, p);
+            if (l0 + E > p.n_tiled || o1 >= (uint32_t)p.nd) {
+                atomicOr(p.status, ZERO_FLAG_BOUNDS);
+                continue;
+            }
             if (o0 == o1) {
                 stg_f32_any<E>(p.shards[o0] + (f0 - (uint64_t)o0 * p.shard), acc);
             } else {
@@ -676,9 +706,12 @@ cudaError_t dev_info(DevInfo* out) {
 }
 
 // Resident CTAs per SM of a pipeline kernel with `smem` dynamic bytes (cached per device).
+// The kernel's dynamic shared-memory limit is raised once per device to the device's opt-in
+// maximum, so that every launch size (they differ with Nd) stays allowed.
 template <typename K>
 cudaError_t pipe_blocks_per_sm(K kernel, size_t smem, int* out) {
     static std::map<std::tuple<int, const void*, size_t>, int> cache;
+    static std::map<std::pair<int, const void*>, int> raised;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -689,8 +722,16 @@ cudaError_t pipe_blocks_per_sm(K kernel, size_t smem, int* out) {
         *out = it->second;
         return cudaSuccess;
     }
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    auto fk = std::make_pair(dev, (const void*)kernel);
+    if (raised.find(fk) == raised.end()) {
+        int optin = 0;
+        e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+        if (e != cudaSuccess) return e;
+        raised[fk] = optin;
+    }
+    if (smem > (size_t)raised[fk]) return cudaErrorInvalidValue;
     int b = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, kThreads, smem);
     if (e != cudaSuccess) return e;

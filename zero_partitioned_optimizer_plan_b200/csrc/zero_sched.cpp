@@ -109,9 +109,10 @@ zero_status zero_sched_create(const zero_plan* plan, uint16_t* slot_mem, uint64_
              cudaEventCreateWithFlags(&s->released[(size_t)i], cudaEventDisableTiming) == cudaSuccess;
     }
     if (!ok) {
+        const zero_status st = zk::from_cuda(cudaGetLastError());
         destroy_events(s);
         delete s;
-        return ZERO_ECUDA;
+        return st == ZERO_OK ? ZERO_ECUDA : st;
     }
     *out = s;
     return ZERO_OK;
@@ -124,8 +125,8 @@ zero_status zero_sched_begin_bucket(zero_sched* s, int k, zero_stream_t producer
     const int slot = k % s->n_slots;
     if (s->filled[(size_t)slot]) {
         // the slot still holds an earlier bucket until its reduce-scatter has finished
-        if (cudaStreamWaitEvent((cudaStream_t)producer, s->released[(size_t)slot], 0) != cudaSuccess)
-            return ZERO_ECUDA;
+        if (cudaError_t e = cudaStreamWaitEvent((cudaStream_t)producer, s->released[(size_t)slot], 0); e != cudaSuccess)
+            return zk::from_cuda(e);
     }
     s->bucket_of_slot[(size_t)slot] = k;
     for (int r = 0; r < s->nd; ++r)
@@ -142,13 +143,13 @@ zero_status zero_sched_end_bucket(zero_sched* s, int k, zero_stream_t producer) 
     for (int r = 0; r < s->nd; ++r)
         ptrs[r] = s->slot_mem + ((uint64_t)slot * (uint64_t)s->nd + (uint64_t)r) * s->stride;
     cudaEvent_t prod = s->produced[(size_t)slot];
-    if (cudaEventRecord(prod, (cudaStream_t)producer) != cudaSuccess) return ZERO_ECUDA;
-    if (cudaStreamWaitEvent(s->rs, prod, 0) != cudaSuccess) return ZERO_ECUDA;
-    if (zk::rs_bucket_launch(s->plan, k, ptrs, s->shards, s->status, s->rs) != cudaSuccess)
-        return ZERO_ECUDA;
+    if (cudaError_t e = cudaEventRecord(prod, (cudaStream_t)producer); e != cudaSuccess) return zk::from_cuda(e);
+    if (cudaError_t e = cudaStreamWaitEvent(s->rs, prod, 0); e != cudaSuccess) return zk::from_cuda(e);
+    if (cudaError_t e = zk::rs_bucket_launch(s->plan, k, ptrs, s->shards, s->status, s->rs); e != cudaSuccess)
+        return zk::from_cuda(e);
     ++s->launches;
     // release: the slot may be refilled once this reduce-scatter is done with it
-    if (cudaEventRecord(s->released[(size_t)slot], s->rs) != cudaSuccess) return ZERO_ECUDA;
+    if (cudaError_t e = cudaEventRecord(s->released[(size_t)slot], s->rs); e != cudaSuccess) return zk::from_cuda(e);
     s->filled[(size_t)slot] = 1;
     s->bucket_of_slot[(size_t)slot] = -1;
     return ZERO_OK;
@@ -156,8 +157,8 @@ zero_status zero_sched_end_bucket(zero_sched* s, int k, zero_stream_t producer) 
 
 zero_status zero_sched_wait(zero_sched* s, zero_stream_t stream) {
     if (!s) return ZERO_EINVAL;
-    if (cudaEventRecord(s->tail, s->rs) != cudaSuccess) return ZERO_ECUDA;
-    if (cudaStreamWaitEvent((cudaStream_t)stream, s->tail, 0) != cudaSuccess) return ZERO_ECUDA;
+    if (cudaError_t e = cudaEventRecord(s->tail, s->rs); e != cudaSuccess) return zk::from_cuda(e);
+    if (cudaError_t e = cudaStreamWaitEvent((cudaStream_t)stream, s->tail, 0); e != cudaSuccess) return zk::from_cuda(e);
     return ZERO_OK;
 }
 

@@ -28,12 +28,13 @@ ZERO_STEP_SKIPPED = 5
 ZERO_FLAG_OVERFLOW = 0x1
 ZERO_FLAG_SKIPPED = 0x2
 ZERO_FLAG_TIMEOUT = 0x4
+ZERO_FLAG_BOUNDS = 0x8
 
 ZERO_MAX_RANKS = 64
 
 # every symbol include/libzero.h declares
 SYMBOLS = (
-    "zero_status_string", "zero_kernel_launches",
+    "zero_status_string", "zero_kernel_launches", "zero_last_error",
     "zero_plan_create", "zero_plan_destroy", "zero_plan_info", "zero_plan_tensor_offsets",
     "zero_plan_bucket", "zero_state_bytes",
     "zero_reduce_scatter_bucket", "zero_adam_shard", "zero_step_fused", "zero_step_commit",
@@ -46,7 +47,10 @@ SYMBOLS = (
 class ZeroError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {zero_status_string(code)}")
+        msg = f"{where}: {zero_status_string(code)}"
+        if code == ZERO_ECUDA:
+            msg += f" ({zero_last_error()})"
+        super().__init__(msg)
 
 
 class _Bytes(C.Structure):
@@ -86,6 +90,7 @@ def _load():
     P = C.POINTER
     L.zero_status_string.argtypes, L.zero_status_string.restype = [i32], C.c_char_p
     L.zero_kernel_launches.argtypes, L.zero_kernel_launches.restype = [], u64
+    L.zero_last_error.argtypes, L.zero_last_error.restype = [], C.c_char_p
     L.zero_plan_create.argtypes = [P(u64), i32, i32, i32, u64, P(vp)]
     L.zero_plan_destroy.argtypes, L.zero_plan_destroy.restype = [vp], None
     L.zero_plan_info.argtypes = [vp, P(u64), P(u64), P(u64), P(i32)]
@@ -151,6 +156,10 @@ def zero_status_string(code: int) -> str:
 
 def zero_kernel_launches() -> int:
     return int(_lib.zero_kernel_launches())
+
+
+def zero_last_error() -> str:
+    return _lib.zero_last_error().decode()
 
 
 # ---------------------------------------------------------------------------------------------
