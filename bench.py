@@ -56,6 +56,7 @@ def parse():
                     default="gpt2_small")
     ap.add_argument("--nd", type=int, default=None)
     ap.add_argument("--bucket", type=int, default=None)
+    ap.add_argument("--psi", type=int, default=None, help="flat workload size (default 2^29)")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -114,8 +115,8 @@ class Workload:
                            "nd": nd, "owner": r, "calls_per_step": 1}
         else:
             nd = args.nd or 16
-            psi = 1 << 29
-            B = args.bucket or (1 << 26)
+            psi = args.psi or (1 << 29)
+            B = args.bucket or min(psi, 1 << 26)
             self.nd, self.n, self.psi = nd, psi, psi
             self.ranges = []
             hi = psi
@@ -128,7 +129,8 @@ class Workload:
             master, m, v = synth.state_warm(psi, seed=0, device=dev)
             self.params = torch.empty(psi, dtype=torch.float16, device=dev)
             self.param_base = 0
-            self.config = {"workload": "flat_2p29", "psi": psi, "nd": nd, "bucket": B,
+            self.config = {"workload": "flat_2p29" if psi == 1 << 29 else f"flat_{psi}",
+                           "psi": psi, "nd": nd, "bucket": B,
                            "calls_per_step": len(self.ranges)}
         self.cur = [master, m, v]
         self.nxt = [torch.empty_like(x) for x in self.cur]
