@@ -40,14 +40,42 @@ namespace zk {
 
 namespace {
 
+// Pipeline geometry. Per Nd the launcher picks the number of consumer warps W and how the
+// shared-memory budget is split into stages from a table measured on B200 (pick_variant);
+// the macros allow other geometries to be compiled and compared.
+#ifndef ZK_SMEM_BUDGET
+#define ZK_SMEM_BUDGET (220 * 1024)
+#endif
+#ifndef ZK_L2_EVICT_FIRST // streamed loads marked evict-first in L2
+#define ZK_L2_EVICT_FIRST 0
+#endif
+#ifndef ZK_COMMIT_BLOCKS_PER_SM
+#define ZK_COMMIT_BLOCKS_PER_SM 1
+#endif
+
 constexpr int kMaxRanks = ZERO_MAX_RANKS;
-constexpr int kConsumerWarps = 8;
-constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kThreads = kConsumerThreads + 32;  // + one producer warp
+constexpr int kElems = 4;                        // elements per consumer thread and tile
 constexpr int kMaxStages = 8;
 constexpr int kDataOffset = 128;                 // full[8] and empty[8] mbarriers first
-constexpr size_t kSmemBudget = 220 * 1024;       // pipeline stages per CTA
+constexpr size_t kSmemBudget = ZK_SMEM_BUDGET;   // pipeline stages per CTA
 constexpr uint64_t kWaitLimitNs = 1000000000ull; // bounded waits: 1 s
+
+template <int W>
+struct Warps {
+    static constexpr int kConsumerWarps = W;
+    static constexpr int kConsumerThreads = W * 32;
+    static constexpr int kThreads = W * 32 + 32;   // + one producer warp
+};
+
+// Shape of the shared-memory pipeline of one launch (see "the pipeline" below).
+struct Geom {
+    uint32_t tile;         // T: elements per tile
+    uint32_t rc;           // rank rows per stage
+    uint32_t nchunks;      // stages per tile: ceil(nd / rc)
+    uint32_t stage_bytes;
+    uint32_t state_off;    // byte offset of the three fp32 state rows in a stage
+    int stages;
+};
 
 struct FusedArgs {
     const uint16_t* grads[kMaxRanks];
@@ -62,10 +90,8 @@ struct FusedArgs {
     uint64_t n;          // elements of the range
     uint64_t n_tiled;    // elements covered by tiles (multiple of 8); [n_tiled, n) is the tail
     uint64_t num_tiles;
-    uint32_t tile;       // elements per tile
-    uint32_t stage_bytes;
+    Geom g;
     int nd;
-    int stages;
     int param_vec;       // widest param store the pointer's alignment allows: 16, 8, 4, 2
     AdamConsts a;
     MeanConsts mc;
@@ -81,10 +107,8 @@ struct RsArgs {
     uint64_t flat_lo;    // flat index of element 0 of the bucket
     uint64_t shard;      // S
     double inv_shard;    // 1/S, for the owner estimate
-    uint32_t tile;
-    uint32_t stage_bytes;
+    Geom g;
     int nd;
-    int stages;
     MeanConsts mc;
 };
 
@@ -205,10 +229,20 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 // Both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
                                          uint64_t* bar) {
+#if ZK_L2_EVICT_FIRST
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;"
+        ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(pol)
+        : "memory");
+#else
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
         ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
         : "memory");
+#endif
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -320,32 +354,136 @@ __device__ __forceinline__ void flag_overflow(bool bad, uint32_t* status) {
 }
 
 // ---------------------------------------------------------------------------------------------
-// the producer: one thread per CTA fills the stages of the CTA's tiles
+// the pipeline
+//
+// A tile is T consecutive elements. Its Nd gradient rows are split into chunks of at most
+// `rc` ranks; chunk c of a tile fills one shared-memory stage with rows c*rc .. c*rc+nr-1 (and,
+// for the last chunk of a fused tile, the three fp32 state rows). The CTA walks its tiles
+// round-robin and, within a tile, its chunks in rank order, so the same consumer thread adds
+// rank 0, 1, ..., Nd-1 of each of its elements into one accumulator: the order of the sum does
+// not depend on the chunking. Stage s of iteration `it` is it % stages, its use it / stages.
 // ---------------------------------------------------------------------------------------------
-template <typename IssueTile>
-__device__ void produce(uint64_t num_tiles, int stages, uint64_t* full, uint64_t* empty,
-                        uint32_t* status, IssueTile issue) {
+struct TileSpan {
+    uint64_t base;   // first element of the tile
+    uint32_t cnt;    // elements in the tile (a multiple of 8)
+};
+
+__device__ __forceinline__ TileSpan tile_span(uint64_t tile, uint32_t T, uint64_t n_tiled) {
+    TileSpan t;
+    t.base = tile * T;
+    const uint64_t left = n_tiled - t.base;
+    t.cnt = left < T ? (uint32_t)left : T;
+    return t;
+}
+
+__device__ __forceinline__ const float* state_row(const FusedArgs& p, uint32_t k) {
+    return k == 0 ? p.master_in : (k == 1 ? p.m_in : p.v_in);
+}
+
+__device__ __forceinline__ const float* state_row(const RsArgs&, uint32_t) { return nullptr; }
+
+// Producer: the whole warp; lane 0 posts each stage's byte count and all lanes issue copies.
+template <bool kState, typename Args>
+__device__ void produce(const Args& p, uint64_t* full, uint64_t* empty, uint8_t* data) {
+    const Geom& g = p.g;
+    const uint32_t T = g.tile;
+    const int lane = threadIdx.x & 31;
     uint32_t it = 0;
     bool ok = true;
-    for (uint64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-        const int s = (int)(it % (uint32_t)stages);
-        const uint32_t use = it / (uint32_t)stages;
-        // the stage's previous tile must have been read by all consumer warps
-        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1u)) {
-            ok = false;
-            break;
+    for (uint64_t tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        const TileSpan ts = tile_span(tile, T, p.n_tiled);
+        for (uint32_t c = 0; c < g.nchunks; ++c, ++it) {
+            const uint32_t s = it % g.stages;
+            const uint32_t use = it / g.stages;
+            if (use > 0) {
+                // the stage's previous fill must have been read by every consumer warp
+                bool w = true;
+                if (lane == 0) w = mbar_wait(&empty[s], (use - 1) & 1u);
+                if (!__shfl_sync(0xffffffffu, w, 0)) {
+                    ok = false;
+                    break;
+                }
+            }
+            const uint32_t r0 = c * g.rc;
+            const uint32_t nr = min(g.rc, (uint32_t)p.nd - r0);
+            const bool with_state = kState && c + 1 == g.nchunks;
+            const uint32_t gb = ts.cnt * 2u, fb = ts.cnt * 4u;
+            uint8_t* st = data + (size_t)s * g.stage_bytes;
+            const bool sane = ts.base < p.n_tiled && (ts.cnt & 7u) == 0 && ts.cnt > 0 &&
+                              r0 < (uint32_t)p.nd && nr <= g.rc && s < (uint32_t)g.stages;
+            if (lane == 0) {
+                if (!sane) atomicOr(p.status, ZERO_FLAG_BOUNDS);
+                mbar_arrive_expect_tx(&full[s], sane ? nr * gb + (with_state ? 3u * fb : 0u) : 0u);
+            }
+            __syncwarp();
+            if (!sane) continue;   // consumers are released without data; stores are checked
+            const uint32_t ncopy = nr + (with_state ? 3u : 0u);
+            for (uint32_t j = (uint32_t)lane; j < ncopy; j += 32u) {
+                if (j < nr) {
+                    bulk_g2s(st + (size_t)j * T * 2u, p.grads[r0 + j] + ts.base, gb, &full[s]);
+                } else {
+                    const uint32_t k = j - nr;
+                    bulk_g2s(st + g.state_off + (size_t)k * T * 4u, state_row(p, k) + ts.base, fb,
+                             &full[s]);
+                }
+            }
         }
-        issue(tile, s, &full[s]);
     }
-    if (!ok) {
-        atomicOr(status, ZERO_FLAG_TIMEOUT);
-        // let every copy this thread started land before the CTA can exit
-        const uint32_t issued = it;
-        for (int s = 0; s < stages && (uint32_t)s < issued; ++s) {
-            const uint32_t last = (uint32_t)s + ((issued - 1u - (uint32_t)s) / (uint32_t)stages) * (uint32_t)stages;
-            (void)mbar_wait(&full[s], (last / (uint32_t)stages) & 1u);
+    if (!ok && lane == 0) {
+        atomicOr(p.status, ZERO_FLAG_TIMEOUT);
+        // let every copy this warp started land before the CTA can exit
+        for (uint32_t s = 0; s < (uint32_t)g.stages && s < it; ++s) {
+            const uint32_t last = s + ((it - 1u - s) / (uint32_t)g.stages) * (uint32_t)g.stages;
+            (void)mbar_wait(&full[s], (last / (uint32_t)g.stages) & 1u);
         }
     }
+}
+
+__device__ __forceinline__ void init_barriers(uint64_t* full, uint64_t* empty, int stages,
+                                              int consumer_warps) {
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], (uint32_t)consumer_warps);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+}
+
+// Consumer side of one stage: wait for it, add its rank rows into acc (rank order), optionally
+// read the state rows, then release the stage. Returns false if the wait timed out.
+template <int E, bool kState>
+__device__ __forceinline__ bool consume_stage(const Geom& g, int nd, uint64_t* full,
+                                              uint64_t* empty, const uint8_t* data, uint32_t it,
+                                              uint32_t c, uint32_t e0, bool active,
+                                              float (&acc)[E], float (&w)[E], float (&m)[E],
+                                              float (&v)[E]) {
+    const uint32_t s = it % g.stages;
+    const uint32_t use = it / g.stages;
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[s], use & 1u))) return false;
+    const uint8_t* st = data + (size_t)s * g.stage_bytes;
+    const uint32_t T = g.tile;
+    if (active) {
+        const uint32_t nr = min(g.rc, (uint32_t)nd - c * g.rc);
+        const uint8_t* row = st + (size_t)e0 * 2u;
+#pragma unroll 4
+        for (uint32_t r = 0; r < nr; ++r) {
+            float x[E];
+            lds_f16<E>(row + (size_t)r * T * 2u, x);
+#pragma unroll
+            for (int j = 0; j < E; ++j) acc[j] = __fadd_rn(acc[j], x[j]);
+        }
+        if (kState && c + 1 == g.nchunks) {
+            const uint8_t* sf = st + g.state_off + (size_t)e0 * 4u;
+            lds_f32<E>(sf, w);
+            lds_f32<E>(sf + (size_t)T * 4u, m);
+            lds_f32<E>(sf + (size_t)T * 8u, v);
+        }
+    }
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[s]);   // stage s may be refilled
+    return true;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -368,104 +506,56 @@ __device__ __forceinline__ void fused_element(const FusedArgs& p, uint64_t i, bo
     p.param_out[i] = f2h(w);
 }
 
-template <int E>
-__global__ void __launch_bounds__(kThreads, 1) fused_tma_kernel(const __grid_constant__ FusedArgs p) {
+template <int E, int W>
+__global__ void __launch_bounds__(Warps<W>::kThreads, 1)
+    fused_tma_kernel(const __grid_constant__ FusedArgs p) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
     uint8_t* data = smem + kDataOffset;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const uint32_t T = p.tile;
+    init_barriers(full, empty, p.g.stages, W);
 
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < p.stages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
-        }
-        fence_mbar_init();
-    }
-    __syncthreads();
-
-    if (warp == kConsumerWarps) {
-        if (lane == 0) {
-            produce(p.num_tiles, p.stages, full, empty, p.status,
-                    [&](uint64_t tile, int s, uint64_t* bar) {
-                        const uint64_t base = tile * T;
-                        const uint64_t left = p.n_tiled - base;
-                        const uint32_t cnt = left < T ? (uint32_t)left : T;
-                        uint8_t* st = data + (size_t)s * p.stage_bytes;
-                        const uint32_t gb = cnt * 2u, fb = cnt * 4u;
-                        if (base >= p.n_tiled || (cnt & 7u) || s >= p.stages) {
-                            atomicOr(p.status, ZERO_FLAG_BOUNDS);
-                            mbar_arrive_expect_tx(bar, 0);   // release the consumers, no copy
-                            return;
-                        }
-                        mbar_arrive_expect_tx(bar, gb * (uint32_t)p.nd + 3u * fb);
-                        for (int r = 0; r < p.nd; ++r)
-                            bulk_g2s(st + (size_t)r * T * 2u, p.grads[r] + base, gb, bar);
-                        uint8_t* sf = st + (size_t)p.nd * T * 2u;
-                        bulk_g2s(sf, p.master_in + base, fb, bar);
-                        bulk_g2s(sf + (size_t)T * 4u, p.m_in + base, fb, bar);
-                        bulk_g2s(sf + (size_t)T * 8u, p.v_in + base, fb, bar);
-                    });
-        }
+    if ((threadIdx.x >> 5) == W) {
+        produce<true>(p, full, empty, data);
         return;
     }
 
     // consumers: thread t owns elements [t*E, t*E + E) of every tile
     bool bad = false;
+    const uint32_t T = p.g.tile;
     const uint32_t e0 = (uint32_t)threadIdx.x * E;
     uint32_t it = 0;
-    for (uint64_t tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
-        const int s = (int)(it % (uint32_t)p.stages);
-        const uint32_t use = it / (uint32_t)p.stages;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], use & 1u));
-        if (!ok) {
-            if (lane == 0) atomicOr(p.status, ZERO_FLAG_TIMEOUT);
-            break;
-        }
-        const uint64_t base = tile * T;
-        const uint64_t left = p.n_tiled - base;
-        const uint32_t cnt = left < T ? (uint32_t)left : T;
-        const bool active = e0 < cnt;   // cnt is a multiple of 8, E divides 8
-        const uint8_t* st = data + (size_t)s * p.stage_bytes;
+    bool ok = true;
+    for (uint64_t tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        const TileSpan ts = tile_span(tile, T, p.n_tiled);
+        const bool active = e0 < ts.cnt;   // cnt is a multiple of 8, E divides 8
         float acc[E], w[E], m[E], v[E];
-        if (active) {
 #pragma unroll
-            for (int j = 0; j < E; ++j) acc[j] = 0.0f;
-            const uint8_t* row = st + (size_t)e0 * 2u;
-#pragma unroll 4
-            for (int r = 0; r < p.nd; ++r) {
-                float x[E];
-                lds_f16<E>(row + (size_t)r * T * 2u, x);
-#pragma unroll
-                for (int j = 0; j < E; ++j) acc[j] = __fadd_rn(acc[j], x[j]);
+        for (int j = 0; j < E; ++j) acc[j] = 0.0f;
+        for (uint32_t c = 0; c < p.g.nchunks; ++c, ++it) {
+            if (!consume_stage<E, true>(p.g, p.nd, full, empty, data, it, c, e0, active, acc, w,
+                                        m, v)) {
+                if ((threadIdx.x & 31) == 0) atomicOr(p.status, ZERO_FLAG_TIMEOUT);
+                ok = false;
+                break;
             }
-            const uint8_t* sf = st + (size_t)p.nd * T * 2u + (size_t)e0 * 4u;
-            lds_f32<E>(sf, w);
-            lds_f32<E>(sf + (size_t)T * 4u, m);
-            lds_f32<E>(sf + (size_t)T * 8u, v);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);   // stage s may be refilled
-        if (active) {
-#pragma unroll
-            for (int j = 0; j < E; ++j) {
-                const float red = mean_of(acc[j], p.mc);
-                bad |= non_finite(red);
-                adam_elem(red, w[j], m[j], v[j], p.a);
-            }
-            const uint64_t g0 = base + e0;
-            if (g0 + E > p.n_tiled) {
-                atomicOr(p.status, ZERO_FLAG_BOUNDS);
-                continue;
-            }
-            stg_f32<E>(p.master_out + g0, w);
-            stg_f32<E>(p.m_out + g0, m);
-            stg_f32<E>(p.v_out + g0, v);
-            stg_f16<E>(p.param_out + g0, w, p.param_vec);
+        if (!ok || !active) continue;
+        const uint64_t g0 = ts.base + e0;
+        if (g0 + E > p.n_tiled) {
+            atomicOr(p.status, ZERO_FLAG_BOUNDS);
+            continue;
         }
+#pragma unroll
+        for (int j = 0; j < E; ++j) {
+            const float red = mean_of(acc[j], p.mc);
+            bad |= non_finite(red);
+            adam_elem(red, w[j], m[j], v[j], p.a);
+        }
+        stg_f32<E>(p.master_out + g0, w);
+        stg_f32<E>(p.m_out + g0, m);
+        stg_f32<E>(p.v_out + g0, v);
+        stg_f16<E>(p.param_out + g0, w, p.param_vec);
     }
     // the < 8 elements past the last tile
     if (blockIdx.x == 0 && (uint64_t)threadIdx.x < p.n - p.n_tiled)
@@ -514,98 +604,58 @@ __device__ __forceinline__ void rs_element(const RsArgs& p, uint64_t i, bool& ba
     rs_store_one(p, i, red);
 }
 
-template <int E>
-__global__ void __launch_bounds__(kThreads, 1) rs_tma_kernel(const __grid_constant__ RsArgs p) {
+template <int E, int W>
+__global__ void __launch_bounds__(Warps<W>::kThreads, 1)
+    rs_tma_kernel(const __grid_constant__ RsArgs p) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
     uint8_t* data = smem + kDataOffset;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const uint32_t T = p.tile;
+    init_barriers(full, empty, p.g.stages, W);
 
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < p.stages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
-        }
-        fence_mbar_init();
-    }
-    __syncthreads();
-
-    if (warp == kConsumerWarps) {
-        if (lane == 0) {
-            produce(p.num_tiles, p.stages, full, empty, p.status,
-                    [&](uint64_t tile, int s, uint64_t* bar) {
-                        const uint64_t base = tile * T;
-                        const uint64_t left = p.n_tiled - base;
-                        const uint32_t cnt = left < T ? (uint32_t)left : T;
-                        uint8_t* st = data + (size_t)s * p.stage_bytes;
-                        const uint32_t gb = cnt * 2u;
-                        if (base >= p.n_tiled || (cnt & 7u) || s >= p.stages) {
-                            atomicOr(p.status, ZERO_FLAG_BOUNDS);
-                            mbar_arrive_expect_tx(bar, 0);
-                            return;
-                        }
-                        mbar_arrive_expect_tx(bar, gb * (uint32_t)p.nd);
-                        for (int r = 0; r < p.nd; ++r)
-                            bulk_g2s(st + (size_t)r * T * 2u, p.grads[r] + base, gb, bar);
-                    });
-        }
+    if ((threadIdx.x >> 5) == W) {
+        produce<false>(p, full, empty, data);
         return;
     }
 
     bool bad = false;
+    const uint32_t T = p.g.tile;
     const uint32_t e0 = (uint32_t)threadIdx.x * E;
     uint32_t it = 0;
-    for (uint64_t tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
-        const int s = (int)(it % (uint32_t)p.stages);
-        const uint32_t use = it / (uint32_t)p.stages;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], use & 1u));
-        if (!ok) {
-            if (lane == 0) atomicOr(p.status, ZERO_FLAG_TIMEOUT);
-            break;
-        }
-        const uint64_t base = tile * T;
-        const uint64_t left = p.n_tiled - base;
-        const uint32_t cnt = left < T ? (uint32_t)left : T;
-        const bool active = e0 < cnt;
-        const uint8_t* st = data + (size_t)s * p.stage_bytes;
-        float acc[E];
-        if (active) {
+    bool ok = true;
+    for (uint64_t tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        const TileSpan ts = tile_span(tile, T, p.n_tiled);
+        const bool active = e0 < ts.cnt;
+        float acc[E], unused[E];
 #pragma unroll
-            for (int j = 0; j < E; ++j) acc[j] = 0.0f;
-            const uint8_t* row = st + (size_t)e0 * 2u;
-#pragma unroll 4
-            for (int r = 0; r < p.nd; ++r) {
-                float x[E];
-                lds_f16<E>(row + (size_t)r * T * 2u, x);
-#pragma unroll
-                for (int j = 0; j < E; ++j) acc[j] = __fadd_rn(acc[j], x[j]);
+        for (int j = 0; j < E; ++j) acc[j] = 0.0f;
+        for (uint32_t c = 0; c < p.g.nchunks; ++c, ++it) {
+            if (!consume_stage<E, false>(p.g, p.nd, full, empty, data, it, c, e0, active, acc,
+                                         unused, unused, unused)) {
+                if ((threadIdx.x & 31) == 0) atomicOr(p.status, ZERO_FLAG_TIMEOUT);
+                ok = false;
+                break;
             }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-        if (active) {
+        if (!ok || !active) continue;
 #pragma unroll
-            for (int j = 0; j < E; ++j) {
-                acc[j] = mean_of(acc[j], p.mc);
-                bad |= non_finite(acc[j]);
-            }
-            const uint64_t l0 = base + e0;
-            const uint64_t f0 = p.flat_lo + l0;
-            const uint32_t o0 = owner_of(f0, p);
-            const uint32_t o1 = owner_of(f0 + E - 1, p);
-            if (l0 + E > p.n_tiled || o1 >= (uint32_t)p.nd) {
-                atomicOr(p.status, ZERO_FLAG_BOUNDS);
-                continue;
-            }
-            if (o0 == o1) {
-                stg_f32_any<E>(p.shards[o0] + (f0 - (uint64_t)o0 * p.shard), acc);
-            } else {
+        for (int j = 0; j < E; ++j) {
+            acc[j] = mean_of(acc[j], p.mc);
+            bad |= non_finite(acc[j]);
+        }
+        const uint64_t l0 = ts.base + e0;
+        const uint64_t f0 = p.flat_lo + l0;
+        const uint32_t o0 = owner_of(f0, p);
+        const uint32_t o1 = owner_of(f0 + E - 1, p);
+        if (l0 + E > p.n_tiled || o1 >= (uint32_t)p.nd) {
+            atomicOr(p.status, ZERO_FLAG_BOUNDS);
+            continue;
+        }
+        if (o0 == o1) {
+            stg_f32_any<E>(p.shards[o0] + (f0 - (uint64_t)o0 * p.shard), acc);
+        } else {
 #pragma unroll
-                for (int j = 0; j < E; ++j) rs_store_one(p, l0 + j, acc[j]);
-            }
+            for (int j = 0; j < E; ++j) rs_store_one(p, l0 + j, acc[j]);
         }
     }
     if (blockIdx.x == 0 && (uint64_t)threadIdx.x < p.n - p.n_tiled)
@@ -709,7 +759,7 @@ cudaError_t dev_info(DevInfo* out) {
 // The kernel's dynamic shared-memory limit is raised once per device to the device's opt-in
 // maximum, so that every launch size (they differ with Nd) stays allowed.
 template <typename K>
-cudaError_t pipe_blocks_per_sm(K kernel, size_t smem, int* out) {
+cudaError_t pipe_blocks_per_sm(K kernel, int threads, size_t smem, int* out) {
     static std::map<std::tuple<int, const void*, size_t>, int> cache;
     static std::map<std::pair<int, const void*>, int> raised;
     int dev = 0;
@@ -733,7 +783,7 @@ cudaError_t pipe_blocks_per_sm(K kernel, size_t smem, int* out) {
     }
     if (smem > (size_t)raised[fk]) return cudaErrorInvalidValue;
     int b = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, kThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, threads, smem);
     if (e != cudaSuccess) return e;
     if (b < 1) return cudaErrorInvalidConfiguration;
     cache[key] = b;
@@ -742,24 +792,50 @@ cudaError_t pipe_blocks_per_sm(K kernel, size_t smem, int* out) {
 }
 
 struct PipeShape {
-    int E;
-    uint32_t tile;
-    uint32_t stage_bytes;
-    int stages;
+    Geom g;
     size_t smem;
+    int warps;       // consumer warps
 };
 
-PipeShape pipe_shape(int nd, uint32_t state_bytes_per_elem) {
-    PipeShape s;
-    s.E = nd <= 8 ? 8 : (nd <= 24 ? 4 : 2);
-    s.tile = (uint32_t)(kConsumerThreads * s.E);
-    s.stage_bytes = s.tile * (2u * (uint32_t)nd + state_bytes_per_elem);
-    size_t st = kSmemBudget / s.stage_bytes;
+// Consumer warps and stage split per Nd, measured on B200 (HBM GB/s of the fused step over
+// geometries with 4 elements per thread): few ranks need more warps to hide the latency of the
+// Adam arithmetic; many ranks need large stages so that a tile takes few chunks.
+struct Variant {
+    int warps;
+    int target_stages;
+};
+
+Variant pick_variant(int nd) {
+    if (nd <= 2) return {20, 2};
+    if (nd <= 4) return {16, 2};
+    if (nd <= 8) return {24, 3};
+    if (nd <= 16) return {16, 2};
+    return {20, 2};
+}
+
+// Tile = 32 * warps * kElems elements; as many rank rows per stage as leave target_stages
+// stages inside the shared-memory budget, the ranks split evenly into chunks.
+PipeShape pipe_shape(int nd, bool with_state) {
+    const Variant var = pick_variant(nd);
+    PipeShape sh;
+    sh.warps = var.warps;
+    Geom& g = sh.g;
+    g.tile = (uint32_t)(32 * var.warps * kElems);
+    const size_t row = (size_t)g.tile * 2u;
+    const size_t state = with_state ? (size_t)g.tile * 12u : 0u;
+    const size_t per_stage = kSmemBudget / (size_t)var.target_stages;
+    size_t rc_max = per_stage > state + row ? (per_stage - state) / row : 1;
+    if (rc_max > (size_t)nd) rc_max = (size_t)nd;
+    g.nchunks = (uint32_t)(((size_t)nd + rc_max - 1) / rc_max);
+    g.rc = (uint32_t)(((size_t)nd + g.nchunks - 1) / g.nchunks);
+    g.state_off = (uint32_t)(g.rc * row);
+    g.stage_bytes = (uint32_t)(g.state_off + state);
+    size_t st = kSmemBudget / g.stage_bytes;
     if (st < 2) st = 2;
     if (st > kMaxStages) st = kMaxStages;
-    s.stages = (int)st;
-    s.smem = (size_t)kDataOffset + st * s.stage_bytes;
-    return s;
+    g.stages = (int)st;
+    sh.smem = (size_t)kDataOffset + st * g.stage_bytes;
+    return sh;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -776,20 +852,21 @@ cudaError_t launch_pipe(K kernel, const A& args, const PipeShape& sh, cudaStream
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
+    const int threads = 32 * sh.warps + 32;
     int bps = 1;
-    e = pipe_blocks_per_sm(kernel, sh.smem, &bps);
+    e = pipe_blocks_per_sm(kernel, threads, sh.smem, &bps);
     if (e != cudaSuccess) return e;
     uint64_t grid = (uint64_t)di.sms * (uint64_t)bps;
     if (args.num_tiles < grid) grid = args.num_tiles;
     if (grid < 1) grid = 1;
-    kernel<<<(unsigned)grid, kThreads, sh.smem, stream>>>(args);
+    kernel<<<(unsigned)grid, threads, sh.smem, stream>>>(args);
     count_launch();
     return cudaGetLastError();
 }
 
-unsigned plain_grid(uint64_t n, int sms) {
+unsigned plain_grid(uint64_t n, int sms, int per_sm = 8) {
     uint64_t blocks = (n + 255) / 256;
-    const uint64_t cap = (uint64_t)sms * 8;
+    const uint64_t cap = (uint64_t)sms * (uint64_t)per_sm;
     if (blocks > cap) blocks = cap;
     return (unsigned)(blocks ? blocks : 1);
 }
@@ -833,17 +910,16 @@ cudaError_t launch_fused(uint64_t n, int nd, const uint16_t* const* grads, const
         count_launch();
         return cudaGetLastError();
     }
-    const PipeShape sh = pipe_shape(nd, 12);
-    p.tile = sh.tile;
-    p.stage_bytes = sh.stage_bytes;
-    p.stages = sh.stages;
+    const PipeShape sh = pipe_shape(nd, true);
+    p.g = sh.g;
     p.n_tiled = n & ~(uint64_t)7;
-    p.num_tiles = (p.n_tiled + sh.tile - 1) / sh.tile;
-    switch (sh.E) {
-        case 8: return launch_pipe(fused_tma_kernel<8>, p, sh, stream);
-        case 4: return launch_pipe(fused_tma_kernel<4>, p, sh, stream);
-        default: return launch_pipe(fused_tma_kernel<2>, p, sh, stream);
+    p.num_tiles = (p.n_tiled + sh.g.tile - 1) / sh.g.tile;
+    switch (sh.warps) {
+        case 16: return launch_pipe(fused_tma_kernel<kElems, 16>, p, sh, stream);
+        case 20: return launch_pipe(fused_tma_kernel<kElems, 20>, p, sh, stream);
+        case 24: return launch_pipe(fused_tma_kernel<kElems, 24>, p, sh, stream);
     }
+    return cudaErrorInvalidConfiguration;
 }
 
 cudaError_t launch_reduce_scatter(uint64_t n, int nd, const uint16_t* const* grads,
@@ -872,17 +948,16 @@ cudaError_t launch_reduce_scatter(uint64_t n, int nd, const uint16_t* const* gra
         count_launch();
         return cudaGetLastError();
     }
-    const PipeShape sh = pipe_shape(nd, 0);
-    p.tile = sh.tile;
-    p.stage_bytes = sh.stage_bytes;
-    p.stages = sh.stages;
+    const PipeShape sh = pipe_shape(nd, false);
+    p.g = sh.g;
     p.n_tiled = n & ~(uint64_t)7;
-    p.num_tiles = (p.n_tiled + sh.tile - 1) / sh.tile;
-    switch (sh.E) {
-        case 8: return launch_pipe(rs_tma_kernel<8>, p, sh, stream);
-        case 4: return launch_pipe(rs_tma_kernel<4>, p, sh, stream);
-        default: return launch_pipe(rs_tma_kernel<2>, p, sh, stream);
+    p.num_tiles = (p.n_tiled + sh.g.tile - 1) / sh.g.tile;
+    switch (sh.warps) {
+        case 16: return launch_pipe(rs_tma_kernel<kElems, 16>, p, sh, stream);
+        case 20: return launch_pipe(rs_tma_kernel<kElems, 20>, p, sh, stream);
+        case 24: return launch_pipe(rs_tma_kernel<kElems, 24>, p, sh, stream);
     }
+    return cudaErrorInvalidConfiguration;
 }
 
 cudaError_t launch_adam(uint64_t n, const float* grad, float* master, float* m, float* v,
@@ -926,7 +1001,7 @@ cudaError_t launch_commit(uint64_t n, const float* master_in, const float* m_in,
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
-    commit_kernel<<<plain_grid(n, di.sms), 256, 0, stream>>>(p);
+    commit_kernel<<<plain_grid(n, di.sms, ZK_COMMIT_BLOCKS_PER_SM), 256, 0, stream>>>(p);
     count_launch();
     return cudaGetLastError();
 }
