@@ -378,7 +378,8 @@ def run_ours(args):
     achieved = bytes_per_launch / launch_s / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": peak_kind,
-                "traffic": traffic_per_launch("fused_tma_kernel", wl.config["workload"]),
+                "traffic": traffic_per_launch("fused_tma_kernel",
+                                              f"{wl.config['workload']}_nd{wl.nd}"),
                 "kernel": "fused_tma_kernel", "bytes_per_launch": bytes_per_launch,
                 "kernel_ms_mean": launch_s * 1e3}
 
