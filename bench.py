@@ -263,11 +263,27 @@ def cpu_oracle_rate(nd: int, n_sample: int, target_s: float, seed=0):
     return n_sample * reps / total, reps, total
 
 
-def dist_setup(args):
+def dist_setup(args=None):
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return ws, rank, local
+
+
+def max_over_ranks(ms: float, ws: int, device) -> float:
+    """The slowest rank's time: every rank must call this, in the same order."""
+    if ws == 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(ws: int, units_per_rank_step: int, steps: int, ms: float) -> float:
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return ws * units_per_rank_step * steps / (ms / 1e3)
 
 
 # ---------------------------------------------------------------------------------------------
@@ -363,12 +379,9 @@ def run_ours(args):
     flags = status.cpu()
     if int((flags != 0).sum()):
         raise RuntimeError(f"unexpected status flags in the timed steps: {set(flags.tolist())}")
-    if ws > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, ws, dev)
     ms_per_step = ms / K
-    value = ws * wl.n * K / (ms / 1e3)
+    value = aggregate_rate(ws, wl.n, K, ms)
 
     # roofline of the dominant kernel: algorithmic bytes per launch / mean launch time
     calls = len(wl.ranges)
@@ -411,12 +424,8 @@ def run_ours(args):
                 raise RuntimeError("unexpected status in the end-to-end steps")
         e1.record()
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if ws > 1:
-            t = torch.tensor([ems], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": ws * wl.n * E / (ems / 1e3), "unit": "params/s",
+        ems = max_over_ranks(e0.elapsed_time(e1), ws, dev)
+        e2e = {"value": aggregate_rate(ws, wl.n, E, ems), "unit": "params/s",
                "h2d_bytes_per_step": 2 * wl.nd * wl.n, "d2h_bytes_per_step": 2 * wl.n + 4,
                "steps": E}
 
