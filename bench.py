@@ -52,7 +52,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["gpt2_small", "shard_7p5b", "flat"],
+    ap.add_argument("--workload", choices=["gpt2_small", "shard_7p5b", "flat", "zero2_1p3b"],
                     default="gpt2_small")
     ap.add_argument("--nd", type=int, default=None)
     ap.add_argument("--bucket", type=int, default=None)
@@ -113,6 +113,9 @@ class Workload:
             self.param_base = r * S
             self.config = {"workload": "shard_7p5b_rank31", "psi_total": total, "shard": S,
                            "nd": nd, "owner": r, "calls_per_step": 1}
+        elif kind == "zero2_1p3b":
+            self._init_zero2(args, dev)
+            return
         else:
             nd = args.nd or 16
             psi = args.psi or (1 << 29)
@@ -135,11 +138,15 @@ class Workload:
         self.cur = [master, m, v]
         self.nxt = [torch.empty_like(x) for x in self.cur]
         self.bytes_per_step = (2 * self.nd + 26) * self.n     # algorithmic HBM bytes
-        self.launches_per_step = len(self.ranges) + 1
+        # the dominant kernel: its bytes and launches per step
+        self.dominant = "fused_tma_kernel"
+        self.dominant_bytes = self.bytes_per_step
+        self.dominant_calls = len(self.ranges)
+        self.side = None
 
     def step(self, t, status, ev=None, grads=None):
-        """Enqueue one step on the current stream; ev = (start, end) events around the fused
-        launches."""
+        """Enqueue one step on the current stream; ev = (start, end) events around the
+        dominant kernel's launches."""
         lz = self.lz
         grads = grads or self.grads
         if ev is not None:
@@ -152,6 +159,79 @@ class Workload:
             ev[1].record()
         lz.zero_step_commit(self.n, *self.cur, *self.nxt, self.params, status)
         self.cur, self.nxt = self.nxt, self.cur
+
+
+def _init_zero2(self, args, dev):
+    """Stage 2 on the 1.3B list: Nd = 16, buckets of 50,000,000 elements. The backward pass's
+    output (every bucket's local gradients of every rank) is already in the scheduler's staging
+    slots, one slot per bucket; a step is the reduce-scatter of the 27 buckets in backward
+    order through the scheduler, then the 16 owners' updates (zero_adam_shard)."""
+    torch, lz = self.torch, self.lz
+    from zero_partitioned_optimizer_plan_b200 import synth
+    nd = args.nd or 16
+    B = args.bucket or 50_000_000
+    numels = synth.gpt_1p3b_list()
+    self.plan = pl = lz.zero_plan_create(numels, nd, 2, B)
+    psi, psi_p, S, nb = lz.zero_plan_info(pl)
+    self.nd, self.n, self.psi, self.S, self.nb = nd, psi_p, psi, S, nb
+    self.slot_elems = lz.zero_sched_slot_elems(pl, nb)
+    self.slots = torch.empty(self.slot_elems, dtype=torch.float16, device=dev)
+    stride = self.slot_elems // (nb * nd)
+    for k in range(nb):
+        lo, ln, _, _ = lz.zero_plan_bucket(pl, k)
+        for r in range(nd):
+            base = (k * nd + r) * stride
+            synth.grad_f16(ln, 1e-3, seed=0, rank=r, step=1000 + k,
+                           out=self.slots[base:base + ln])
+    self.master, self.m, self.v = synth.state_small(psi_p, seed=0, device=dev)
+    self.params = torch.empty(psi_p, dtype=torch.float16, device=dev)
+    self.shards = torch.empty(psi_p, dtype=torch.float32, device=dev)
+    self.grads = None
+    self.ranges = [(0, psi_p)]
+    self.param_base = 0
+    self.config = {"workload": "zero2_1p3b", "psi": psi, "nd": nd, "stage": 2, "bucket": B,
+                   "buckets": nb, "calls_per_step": nb + nd}
+    rs_bytes = (2 * nd + 4) * psi_p
+    adam_bytes = 30 * psi_p
+    self.bytes_per_step = rs_bytes + adam_bytes
+    self.dominant = "rs_tma_kernel"
+    self.dominant_bytes = rs_bytes
+    self.dominant_calls = nb
+    self.side = {"kernel": "adam_kernel", "bytes": adam_bytes, "calls": nd, "ms": []}
+    self.step = self._step_zero2
+
+
+def _step_zero2(self, t, status, ev=None, grads=None):
+    lz, torch = self.lz, self.torch
+    if grads is not None:
+        raise ValueError("the stage-2 workload has no host-buffer variant")
+    S, nd = self.S, self.nd
+    stream = torch.cuda.current_stream()
+    sch = lz.zero_sched_create(self.plan, self.slots, self.slot_elems, self.nb,
+                               [self.shards[r * S:(r + 1) * S] for r in range(nd)], status,
+                               stream)
+    if ev is not None:
+        ev[0].record()
+    for k in range(self.nb):
+        lz.zero_sched_begin_bucket(sch, k, stream)
+        lz.zero_sched_end_bucket(sch, k, stream)
+    lz.zero_sched_wait(sch, stream)
+    if ev is not None:
+        ev[1].record()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+    for r in range(nd):
+        sl = slice(r * S, (r + 1) * S)
+        lz.zero_adam_shard(S, self.shards[sl], self.master[sl], self.m[sl], self.v[sl],
+                           self.params[sl], self.hp, t, status)
+    if ev is not None:
+        a1.record()
+        self.side["ms"].append((a0, a1))
+    lz.zero_sched_destroy(sch)
+
+
+Workload._init_zero2 = _init_zero2
+Workload._step_zero2 = _step_zero2
 
 
 # ---------------------------------------------------------------------------------------------
@@ -384,22 +464,28 @@ def run_ours(args):
     value = aggregate_rate(ws, wl.n, K, ms)
 
     # roofline of the dominant kernel: algorithmic bytes per launch / mean launch time
-    calls = len(wl.ranges)
+    calls = wl.dominant_calls
     launch_s = statistics.mean(kernel_ms) / 1e3 / calls
-    bytes_per_launch = wl.bytes_per_step / calls
+    bytes_per_launch = wl.dominant_bytes / calls
     peak, peak_kind = measured_peak()
     achieved = bytes_per_launch / launch_s / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": peak_kind,
-                "traffic": traffic_per_launch("fused_tma_kernel",
+                "traffic": traffic_per_launch(wl.dominant,
                                               f"{wl.config['workload']}_nd{wl.nd}"),
-                "kernel": "fused_tma_kernel", "bytes_per_launch": bytes_per_launch,
+                "kernel": wl.dominant, "bytes_per_launch": bytes_per_launch,
                 "kernel_ms_mean": launch_s * 1e3}
+    if wl.side is not None:   # the other kernel of a two-kernel step
+        side_s = statistics.mean(a.elapsed_time(b) for a, b in wl.side["ms"][-K:]) / 1e3
+        roofline["other"] = {"kernel": wl.side["kernel"],
+                             "achieved": wl.side["bytes"] / side_s / 1e9,
+                             "frac": wl.side["bytes"] / side_s / 1e9 / peak,
+                             "ms_per_step": side_s * 1e3}
 
     # end to end through the public API with host buffers: H2D of the step's gradients from
     # pinned memory, the step, D2H of the updated fp16 parameters and the status word
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and wl.grads is not None:
         E = args.e2e_steps or max(3, min(K, 10))
         h_grads = [torch.empty(g.numel(), dtype=torch.float16, pin_memory=True)
                    for g in wl.grads]
@@ -439,7 +525,7 @@ def run_ours(args):
 
     if rank == 0:
         cfg = dict(wl.config)
-        cfg.update({"l2": "no flush: every step streams (2*Nd+26)*psi bytes, far above L2",
+        cfg.update({"l2": "no flush: every step streams several GB, far above L2",
                     "bytes_per_step": wl.bytes_per_step, "parallelism": f"replicas{ws}",
                     "hbm_gbs": wl.bytes_per_step / (ms_per_step / 1e3) / 1e9})
         line = {
