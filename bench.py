@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--nd", type=int, default=None)
     ap.add_argument("--bucket", type=int, default=None)
     ap.add_argument("--psi", type=int, default=None, help="flat workload size (default 2^29)")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture a step's calls in CUDA graphs (constants in device memory)")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -143,6 +145,67 @@ class Workload:
         self.dominant_bytes = self.bytes_per_step
         self.dominant_calls = len(self.ranges)
         self.side = None
+
+    # --- CUDA-graph mode: the step's calls read the Adam constants from device memory -------
+    def enable_graph(self):
+        torch, lz = self.torch, self.lz
+        dev = self.cur[0].device
+        self.d_consts = torch.empty(40, dtype=torch.uint8, device=dev)
+        self.h_consts = [torch.empty(40, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
+        self.h_done = [None, None]
+        self.g_status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.g_flags = torch.zeros(1, dtype=torch.int32, device=dev)
+        a, b = self.cur, self.nxt
+
+        def body(src, dst):
+            self.g_status.zero_()
+            for lo, hi in self.ranges:
+                lz.zero_step_fused_dc(hi - lo, self.nd, [g[lo:hi] for g in self.grads],
+                                      *[x[lo:hi] for x in src], *[x[lo:hi] for x in dst],
+                                      self.params[lo:hi], self.d_consts, self.g_status)
+            lz.zero_step_commit(self.n, *src, *dst, self.params, self.g_status)
+            self.g_flags.bitwise_or_(self.g_status)
+
+        self._load_consts(1)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            body(a, b)                  # first use outside the capture
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.graphs = []
+        for src, dst in ((a, b), (b, a)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                body(src, dst)
+            self.graphs.append(g)
+        self.g_flags.zero_()
+        self.graph_dir = 0
+        self.step = self._graph_step
+
+    def _load_consts(self, t):
+        """Copy step t's constants to the device, double-buffered in pinned host memory."""
+        torch, lz = self.torch, self.lz
+        i = t % 2
+        if self.h_done[i] is not None:
+            self.h_done[i].synchronize()      # the copy that last read this buffer is done
+        c = lz.zero_adam_consts_for_step(self.hp, t)
+        self.h_consts[i].copy_(torch.frombuffer(bytearray(bytes(c)), dtype=torch.uint8))
+        self.d_consts.copy_(self.h_consts[i], non_blocking=True)
+        e = torch.cuda.Event()
+        e.record()
+        self.h_done[i] = e
+
+    def _graph_step(self, t, status, ev=None, grads=None):
+        if grads is not None:
+            raise ValueError("graph mode has no host-buffer variant")
+        self._load_consts(t)
+        if ev is not None:
+            ev[0].record()
+        self.graphs[self.graph_dir].replay()
+        if ev is not None:
+            ev[1].record()
+        self.graph_dir ^= 1
 
     def step(self, t, status, ev=None, grads=None):
         """Enqueue one step on the current stream; ev = (start, end) events around the
@@ -425,6 +488,10 @@ def run_ours(args):
     from zero_partitioned_optimizer_plan_b200 import libzero as lz
 
     wl = Workload(args, dev)
+    if args.graph:
+        if wl.grads is None:
+            raise SystemExit("--graph applies to the stage-1 and flat workloads")
+        wl.enable_graph()
     K, W = args.steps, args.warmup
     status = torch.zeros(K + W, dtype=torch.int32, device=dev)   # one status word per step
     torch.cuda.synchronize()
@@ -453,6 +520,10 @@ def run_ours(args):
         end.record()
         torch.cuda.synchronize()
     launches = lz.zero_kernel_launches() - launches0
+    if args.graph:   # replays launch the captured kernels without the host library
+        launches = K * (len(wl.ranges) + 1)
+        if int(wl.g_flags.item()) != 0:
+            raise RuntimeError(f"unexpected status flags in the timed steps: {wl.g_flags.item()}")
     barrier()
     ms = start.elapsed_time(end)
     kernel_ms = [a.elapsed_time(b) for a, b in evs]
@@ -485,7 +556,7 @@ def run_ours(args):
     # end to end through the public API with host buffers: H2D of the step's gradients from
     # pinned memory, the step, D2H of the updated fp16 parameters and the status word
     e2e = None
-    if not args.no_e2e and wl.grads is not None:
+    if not args.no_e2e and wl.grads is not None and not args.graph:
         E = args.e2e_steps or max(3, min(K, 10))
         h_grads = [torch.empty(g.numel(), dtype=torch.float16, pin_memory=True)
                    for g in wl.grads]
@@ -525,6 +596,8 @@ def run_ours(args):
 
     if rank == 0:
         cfg = dict(wl.config)
+        if args.graph:
+            cfg["cuda_graph"] = "one replay per step; kernel time includes the commit"
         cfg.update({"l2": "no flush: every step streams several GB, far above L2",
                     "bytes_per_step": wl.bytes_per_step, "parallelism": f"replicas{ws}",
                     "hbm_gbs": wl.bytes_per_step / (ms_per_step / 1e3) / 1e9})

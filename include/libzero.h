@@ -135,6 +135,22 @@ typedef struct {
     double lr, beta1, beta2, eps, loss_scale;
 } zero_adam_hparams;
 
+/* The fp32 constants of one Adam step t, in the layout the kernels read them. */
+typedef struct {
+    float beta1, one_minus_beta1, beta2, one_minus_beta2;
+    float step_size;      /* lr / (1 - beta1^t) */
+    float bias2_sqrt;     /* sqrt(1 - beta2^t) */
+    float eps;
+    float loss_scale;     /* the unscale divisor */
+    float inv_loss_scale; /* 1/loss_scale if loss_scale is a power of two, else 0 */
+    int32_t loss_scale_pow2;
+} zero_adam_consts;
+
+/* Fill *out with the constants of step t (t >= 1) exactly as zero_adam_shard and
+ * zero_step_fused compute them. Errors: ZERO_EINVAL (null pointers, t < 1, bad hparams). */
+zero_status zero_adam_consts_for_step(const zero_adam_hparams* hp, int64_t step,
+                                      zero_adam_consts* out);
+
 /* ------------------------------------------------------------------------------------------
  * Bucketed reduce-scatter (stage 2). "ZeRO-2" card, "Gradient 생명주기": as soon as a bucket's
  * local gradient exists it is reduce-scattered; each GPU keeps only its reduced shard.
@@ -203,6 +219,21 @@ zero_status zero_step_fused(uint64_t n, int nd, const uint16_t* const* rank_grad
                             float* master_out, float* m_out, float* v_out, uint16_t* param_out,
                             const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
                             zero_stream_t stream);
+
+/* zero_adam_shard and zero_step_fused with the step's constants read from device memory when
+ * the kernel runs (d_consts: a zero_adam_consts in device memory, 4-byte aligned), so that a
+ * stream capture of a step (a CUDA graph) can be replayed for every step: before each replay
+ * the caller copies that step's constants (zero_adam_consts_for_step) into *d_consts. Same
+ * arithmetic and results as the calls above. Errors: as those calls (ZERO_EINVAL for a null
+ * d_consts). */
+zero_status zero_adam_shard_dc(uint64_t n, const float* grad, float* master, float* m, float* v,
+                               uint16_t* param_out, const zero_adam_consts* d_consts,
+                               uint32_t* d_status, zero_stream_t stream);
+zero_status zero_step_fused_dc(uint64_t n, int nd, const uint16_t* const* rank_grads,
+                               const float* master_in, const float* m_in, const float* v_in,
+                               float* master_out, float* m_out, float* v_out,
+                               uint16_t* param_out, const zero_adam_consts* d_consts,
+                               uint32_t* d_status, zero_stream_t stream);
 
 /* Close a step made of zero_step_fused calls, on the same stream, over the same range(s).
  * If ZERO_FLAG_OVERFLOW is set: (master_out, m_out, v_out) = (master_in, m_in, v_in),

@@ -215,3 +215,38 @@ def test_scheduler_rejects():
 def test_status_strings():
     for code in range(6):
         assert lz.zero_status_string(code).startswith("ZERO_")
+
+
+@pytest.mark.parametrize("t", [1, 2, 3, 10, 1000, 123456])
+@pytest.mark.parametrize("hp", [lz.AdamHP(), lz.AdamHP(lr=3e-4, beta1=0.8, beta2=0.95, eps=1e-6,
+                                                     loss_scale=1000.0),
+                                lz.AdamHP(loss_scale=0.5)])
+def test_adam_consts_match_oracle_bitwise(hp, t):
+    c = lz.zero_adam_consts_for_step(hp, t)
+    o = oracle.adam_scalars(oracle.AdamHP(hp.lr, hp.beta1, hp.beta2, hp.eps, hp.loss_scale), t)
+    pairs = [("beta1", "b1"), ("one_minus_beta1", "omb1"), ("beta2", "b2"),
+             ("one_minus_beta2", "omb2"), ("step_size", "step_size"), ("bias2_sqrt", "bc2s"),
+             ("eps", "eps"), ("loss_scale", "loss_scale")]
+    for a, b in pairs:
+        assert np.float32(getattr(c, a)).view(np.uint32) == np.float32(o[b]).view(np.uint32), a
+    pow2 = hp.loss_scale in (1024.0, 0.5)
+    assert c.loss_scale_pow2 == int(pow2)
+    if pow2:
+        assert c.inv_loss_scale == 1.0 / hp.loss_scale
+
+
+def test_dc_variants_reject():
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_adam_consts_for_step(HP, 0)
+    assert e.value.code == lz.ZERO_EINVAL
+    grads = [A + i * MB for i in range(2)]
+    ins = [A + 100 * MB, A + 101 * MB, A + 102 * MB]
+    outs = [A + 110 * MB, A + 111 * MB, A + 112 * MB]
+    for dc, code in [(0, lz.ZERO_EINVAL), (A + 140 * MB + 2, lz.ZERO_EALIGN)]:
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_step_fused_dc(1000, 2, grads, *ins, *outs, A + 120 * MB, dc, A + 130 * MB, 0)
+        assert e.value.code == code
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_adam_shard_dc(10, A, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, dc,
+                                  A + 5 * MB, 0)
+        assert e.value.code == code

@@ -347,3 +347,99 @@ def test_launch_sizes_in_any_order():
                                             m.numpy(), v.numpy(), ORC_HP, 1)
         check_f32("master", f32np(pp.nxt[0]), w)
         check_f16("params", f16np(params), p)
+
+
+def _consts_on_device(t):
+    c = lz.zero_adam_consts_for_step(HP, t)
+    host = torch.frombuffer(bytearray(bytes(c)), dtype=torch.uint8)
+    return host.to(DEV)
+
+
+@pytest.mark.parametrize("nd", [2, 8, 64])
+def test_device_constants_variants_match(nd):
+    """zero_step_fused_dc / zero_adam_shard_dc (constants read from device memory) give the
+    same bits as the calls that take the hyperparameters and t."""
+    n = 2048 * 21 + 3
+    g_dev = [g.to(DEV) for g in _rank_grads_cpu(n, nd, 61, 1)]
+    master, m, v = (x.to(DEV) for x in synth.state_warm(n, seed=62))
+    for t in (1, 7):
+        dc = _consts_on_device(t)
+        outs_a = [torch.empty_like(x) for x in (master, m, v)]
+        outs_b = [torch.empty_like(x) for x in (master, m, v)]
+        pa = torch.empty(n, dtype=torch.float16, device=DEV)
+        pb = torch.empty(n, dtype=torch.float16, device=DEV)
+        st = status_word()
+        lz.zero_step_fused(n, nd, g_dev, master, m, v, *outs_a, pa, HP, t, st)
+        lz.zero_step_fused_dc(n, nd, g_dev, master, m, v, *outs_b, pb, dc, st)
+        red = torch.full((n,), 3e-6, device=DEV)
+        ua = [x.clone() for x in (master, m, v)]
+        ub = [x.clone() for x in (master, m, v)]
+        qa = torch.empty(n, dtype=torch.float16, device=DEV)
+        qb = torch.empty(n, dtype=torch.float16, device=DEV)
+        lz.zero_adam_shard(n, red, *ua, qa, HP, t, st)
+        lz.zero_adam_shard_dc(n, red, *ub, qb, dc, st)
+        torch.cuda.synchronize()
+        assert status_flags(st) == 0
+        for a, b in list(zip(outs_a, outs_b)) + list(zip(ua, ub)) + [(pa, pb), (qa, qb)]:
+            assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_graph_replay_of_bucketed_step():
+    """A step of per-bucket zero_step_fused_dc calls and a commit, captured once per direction
+    of the ping-pong as CUDA graphs and replayed for t = 1, 2, 3 with that step's constants
+    copied in before each replay, equals the oracle's three steps."""
+    nd, n, B = 4, 2048 * 30 + 7, 9000
+    master, m, v = synth.state_warm(n, seed=71)
+    bufs = [[x.to(DEV) for x in (master, m, v)], [torch.empty(n, device=DEV) for _ in range(3)]]
+    grads = [torch.empty(n, dtype=torch.float16, device=DEV) for _ in range(nd)]
+    params = torch.empty(n, dtype=torch.float16, device=DEV)
+    dc = torch.empty(40, dtype=torch.uint8, device=DEV)
+    st = status_word()
+    flags = status_word()
+    bounds, hi = [], n
+    while hi > 0:
+        bounds.append((max(0, hi - B), hi))
+        hi = max(0, hi - B)
+
+    def step(src, dst):
+        st.zero_()
+        for lo, hi in bounds:
+            lz.zero_step_fused_dc(hi - lo, nd, [g[lo:hi] for g in grads],
+                                  *[x[lo:hi] for x in src], *[x[lo:hi] for x in dst],
+                                  params[lo:hi], dc, st)
+        lz.zero_step_commit(n, *src, *dst, params, st)
+        flags.bitwise_or_(st)
+
+    dc.copy_(_consts_on_device(1))
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step(bufs[0], bufs[1])        # warm-up outside capture (sets launch attributes)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graphs = []
+    for src, dst in ((bufs[0], bufs[1]), (bufs[1], bufs[0])):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(src, dst)
+        graphs.append(g)
+    # restore the state the warm-up overwrote, then run three steps by replay
+    for x, y in zip(bufs[0], (master, m, v)):
+        x.copy_(y.to(DEV))
+    flags.zero_()
+    w_r, m_r, v_r = master.numpy(), m.numpy(), v.numpy()
+    for t in (1, 2, 3):
+        g_cpu = _rank_grads_cpu(n, nd, 72, t)
+        for d, s in zip(grads, g_cpu):
+            d.copy_(s.to(DEV))
+        dc.copy_(_consts_on_device(t))
+        graphs[(t - 1) % 2].replay()
+        torch.cuda.synchronize()
+        assert status_flags(flags) == 0
+        skipped, w_r, m_r, v_r, p_r = oracle.step([g.numpy() for g in g_cpu], w_r, m_r, v_r,
+                                                  ORC_HP, t)
+        out = bufs[t % 2]
+        check_f32(f"step {t} master", f32np(out[0]), w_r)
+        check_f32(f"step {t} m", f32np(out[1]), m_r)
+        check_f32(f"step {t} v", f32np(out[2]), v_r)
+        check_f16(f"step {t} params", f16np(params), p_r)

@@ -48,16 +48,17 @@ AdamConsts make_adam(const zero_adam_hparams* hp, int64_t t) {
     AdamConsts a;
     const double c1 = 1.0 - std::pow(hp->beta1, (double)t);
     const double c2 = 1.0 - std::pow(hp->beta2, (double)t);
-    a.b1 = (float)hp->beta1;
-    a.omb1 = (float)(1.0 - hp->beta1);
-    a.b2 = (float)hp->beta2;
-    a.omb2 = (float)(1.0 - hp->beta2);
+    a.beta1 = (float)hp->beta1;
+    a.one_minus_beta1 = (float)(1.0 - hp->beta1);
+    a.beta2 = (float)hp->beta2;
+    a.one_minus_beta2 = (float)(1.0 - hp->beta2);
     a.step_size = (float)(hp->lr / c1);
-    a.bc2s = (float)std::sqrt(c2);
+    a.bias2_sqrt = (float)std::sqrt(c2);
     a.eps = (float)hp->eps;
     a.loss_scale = (float)hp->loss_scale;
-    a.inv_ls = 0.0f;
-    a.ls_pow2 = pow2_with_normal_reciprocal((double)a.loss_scale, &a.inv_ls) ? 1 : 0;
+    a.inv_loss_scale = 0.0f;
+    a.loss_scale_pow2 =
+        pow2_with_normal_reciprocal((double)a.loss_scale, &a.inv_loss_scale) ? 1 : 0;
     return a;
 }
 
@@ -138,10 +139,9 @@ zero_status zero_reduce_scatter_bucket(const zero_plan* plan, int k,
                                               (cudaStream_t)stream));
 }
 
-zero_status zero_adam_shard(uint64_t n, const float* grad, float* master, float* m, float* v,
-                            uint16_t* param_out, const zero_adam_hparams* hp, int64_t step,
-                            uint32_t* d_status, zero_stream_t stream) {
-    if (!zk::hparams_ok(hp) || step < 1 || !d_status) return ZERO_EINVAL;
+static zero_status check_adam(uint64_t n, const float* grad, float* master, float* m, float* v,
+                              uint16_t* param_out, uint32_t* d_status) {
+    if (!d_status) return ZERO_EINVAL;
     if (n == 0) return ZERO_OK;
     if (!grad || !master || !m || !v || !param_out) return ZERO_EINVAL;
     if (n > (UINT64_MAX / 8)) return ZERO_EINVAL;
@@ -153,9 +153,38 @@ zero_status zero_adam_shard(uint64_t n, const float* grad, float* master, float*
     for (int i = 0; i < 6; ++i)
         for (int j = i + 1; j < 6; ++j)
             if (zk::overlap(arr[i], len[i], arr[j], len[j])) return ZERO_EINVAL;
+    return ZERO_OK;
+}
+
+zero_status zero_adam_consts_for_step(const zero_adam_hparams* hp, int64_t step,
+                                      zero_adam_consts* out) {
+    if (!zk::hparams_ok(hp) || step < 1 || !out) return ZERO_EINVAL;
+    *out = zk::make_adam(hp, step);
+    return ZERO_OK;
+}
+
+zero_status zero_adam_shard(uint64_t n, const float* grad, float* master, float* m, float* v,
+                            uint16_t* param_out, const zero_adam_hparams* hp, int64_t step,
+                            uint32_t* d_status, zero_stream_t stream) {
+    if (!zk::hparams_ok(hp) || step < 1) return ZERO_EINVAL;
+    const zero_status st = check_adam(n, grad, master, m, v, param_out, d_status);
+    if (st != ZERO_OK || n == 0) return st;
     return zk::from_cuda(zk::launch_adam(n, grad, master, m, v, param_out,
-                                         zk::make_adam(hp, step), d_status,
+                                         zk::make_adam(hp, step), nullptr, d_status,
                                          (cudaStream_t)stream));
+}
+
+zero_status zero_adam_shard_dc(uint64_t n, const float* grad, float* master, float* m, float* v,
+                               uint16_t* param_out, const zero_adam_consts* d_consts,
+                               uint32_t* d_status, zero_stream_t stream) {
+    if (!d_consts) return ZERO_EINVAL;
+    if (!zk::aligned(d_consts, 4)) return ZERO_EALIGN;
+    const zero_status st = check_adam(n, grad, master, m, v, param_out, d_status);
+    if (st != ZERO_OK || n == 0) return st;
+    zero_adam_consts unused;
+    memset(&unused, 0, sizeof(unused));
+    return zk::from_cuda(zk::launch_adam(n, grad, master, m, v, param_out, unused, d_consts,
+                                         d_status, (cudaStream_t)stream));
 }
 
 static zero_status check_fused_state(uint64_t n, const float* master_in, const float* m_in,
@@ -181,13 +210,11 @@ static zero_status check_fused_state(uint64_t n, const float* master_in, const f
     return ZERO_OK;
 }
 
-zero_status zero_step_fused(uint64_t n, int nd, const uint16_t* const* rank_grads,
-                            const float* master_in, const float* m_in, const float* v_in,
-                            float* master_out, float* m_out, float* v_out, uint16_t* param_out,
-                            const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
-                            zero_stream_t stream) {
-    if (nd < 1 || nd > ZERO_MAX_RANKS || !zk::hparams_ok(hp) || step < 1 || !d_status)
-        return ZERO_EINVAL;
+static zero_status check_fused(uint64_t n, int nd, const uint16_t* const* rank_grads,
+                               const float* master_in, const float* m_in, const float* v_in,
+                               float* master_out, float* m_out, float* v_out,
+                               uint16_t* param_out, uint32_t* d_status) {
+    if (nd < 1 || nd > ZERO_MAX_RANKS || !d_status) return ZERO_EINVAL;
     if (n == 0) return ZERO_OK;
     if (!rank_grads) return ZERO_EINVAL;
     zero_status st = check_fused_state(n, master_in, m_in, v_in, master_out, m_out, v_out,
@@ -201,8 +228,38 @@ zero_status zero_step_fused(uint64_t n, int nd, const uint16_t* const* rank_grad
         for (int i = 0; i < 5; ++i)
             if (zk::overlap(outs[i], olen[i], rank_grads[r], n * 2)) return ZERO_EINVAL;
     }
+    return ZERO_OK;
+}
+
+zero_status zero_step_fused(uint64_t n, int nd, const uint16_t* const* rank_grads,
+                            const float* master_in, const float* m_in, const float* v_in,
+                            float* master_out, float* m_out, float* v_out, uint16_t* param_out,
+                            const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
+                            zero_stream_t stream) {
+    if (!zk::hparams_ok(hp) || step < 1) return ZERO_EINVAL;
+    const zero_status st = check_fused(n, nd, rank_grads, master_in, m_in, v_in, master_out,
+                                       m_out, v_out, param_out, d_status);
+    if (st != ZERO_OK || n == 0) return st;
     return zk::from_cuda(zk::launch_fused(n, nd, rank_grads, master_in, m_in, v_in, master_out,
                                           m_out, v_out, param_out, zk::make_adam(hp, step),
+                                          nullptr, zk::make_mean(nd), d_status,
+                                          (cudaStream_t)stream));
+}
+
+zero_status zero_step_fused_dc(uint64_t n, int nd, const uint16_t* const* rank_grads,
+                               const float* master_in, const float* m_in, const float* v_in,
+                               float* master_out, float* m_out, float* v_out,
+                               uint16_t* param_out, const zero_adam_consts* d_consts,
+                               uint32_t* d_status, zero_stream_t stream) {
+    if (!d_consts) return ZERO_EINVAL;
+    if (!zk::aligned(d_consts, 4)) return ZERO_EALIGN;
+    const zero_status st = check_fused(n, nd, rank_grads, master_in, m_in, v_in, master_out,
+                                       m_out, v_out, param_out, d_status);
+    if (st != ZERO_OK || n == 0) return st;
+    zero_adam_consts unused;
+    memset(&unused, 0, sizeof(unused));
+    return zk::from_cuda(zk::launch_fused(n, nd, rank_grads, master_in, m_in, v_in, master_out,
+                                          m_out, v_out, param_out, unused, d_consts,
                                           zk::make_mean(nd), d_status, (cudaStream_t)stream));
 }
 

@@ -9,16 +9,8 @@
 
 namespace zk {
 
-// fp32 constants of one Adam step, computed on the host (see zero_api.cpp).
-struct AdamConsts {
-    float b1, omb1, b2, omb2;
-    float step_size;   // lr / (1 - beta1^t)
-    float bc2s;        // sqrt(1 - beta2^t)
-    float eps;
-    float loss_scale;  // the divisor of the unscale
-    float inv_ls;      // 1/loss_scale when loss_scale is a power of two (then x*inv_ls == x/ls)
-    int ls_pow2;
-};
+// fp32 constants of one Adam step, computed on the host (zero_api.cpp), in the public layout.
+using AdamConsts = zero_adam_consts;
 
 // The division of the rank sum by nd.
 struct MeanConsts {
@@ -34,10 +26,12 @@ uint64_t plan_max_bucket(const zero_plan* p);
 uint64_t plan_n_buckets(const zero_plan* p);
 
 // Launchers (zero_kernels.cu). They validate nothing: the C ABI layer has done that.
+// `ad` (device memory) overrides `a` when it is not null.
 cudaError_t launch_fused(uint64_t n, int nd, const uint16_t* const* grads, const float* master_in,
                          const float* m_in, const float* v_in, float* master_out, float* m_out,
                          float* v_out, uint16_t* param_out, const AdamConsts& a,
-                         const MeanConsts& mc, uint32_t* status, cudaStream_t stream);
+                         const AdamConsts* ad, const MeanConsts& mc, uint32_t* status,
+                         cudaStream_t stream);
 cudaError_t launch_commit(uint64_t n, const float* master_in, const float* m_in,
                           const float* v_in, float* master_out, float* m_out, float* v_out,
                           uint16_t* param_out, uint32_t* status, cudaStream_t stream);
@@ -45,8 +39,8 @@ cudaError_t launch_reduce_scatter(uint64_t n, int nd, const uint16_t* const* gra
                                   float* const* shards, uint64_t flat_lo, uint64_t shard,
                                   const MeanConsts& mc, uint32_t* status, cudaStream_t stream);
 cudaError_t launch_adam(uint64_t n, const float* grad, float* master, float* m, float* v,
-                        uint16_t* param_out, const AdamConsts& a, uint32_t* status,
-                        cudaStream_t stream);
+                        uint16_t* param_out, const AdamConsts& a, const AdamConsts* ad,
+                        uint32_t* status, cudaStream_t stream);
 
 // Count of kernels this library has launched in this process.
 void count_launch();

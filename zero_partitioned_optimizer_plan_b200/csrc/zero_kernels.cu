@@ -94,6 +94,7 @@ struct FusedArgs {
     int nd;
     int param_vec;       // widest param store the pointer's alignment allows: 16, 8, 4, 2
     AdamConsts a;
+    const AdamConsts* ad;  // when not null: the constants, read from device memory at run time
     MeanConsts mc;
 };
 
@@ -135,6 +136,7 @@ struct AdamArgs {
     int vec;             // 1: every fp32 pointer 16-byte aligned (float4 path)
     int param_vec;       // 8, 4 or 2
     AdamConsts a;
+    const AdamConsts* ad;  // when not null: the constants, read from device memory at run time
 };
 
 // ---------------------------------------------------------------------------------------------
@@ -161,14 +163,21 @@ __device__ __forceinline__ bool non_finite(float x) {
 // Adam on one element from its reduced (still loss-scaled) gradient; w, m, v updated in place.
 __device__ __forceinline__ void adam_elem(float red, float& w, float& m, float& v,
                                           const AdamConsts& a) {
-    const float g = a.ls_pow2 ? __fmul_rn(red, a.inv_ls) : __fdiv_rn(red, a.loss_scale);
-    const float mt = __fadd_rn(__fmul_rn(a.b1, m), __fmul_rn(a.omb1, g));
-    const float vt = __fadd_rn(__fmul_rn(a.b2, v), __fmul_rn(a.omb2, __fmul_rn(g, g)));
-    const float denom = __fadd_rn(__fdiv_rn(__fsqrt_rn(vt), a.bc2s), a.eps);
+    const float g = a.loss_scale_pow2 ? __fmul_rn(red, a.inv_loss_scale)
+                                      : __fdiv_rn(red, a.loss_scale);
+    const float mt = __fadd_rn(__fmul_rn(a.beta1, m), __fmul_rn(a.one_minus_beta1, g));
+    const float vt =
+        __fadd_rn(__fmul_rn(a.beta2, v), __fmul_rn(a.one_minus_beta2, __fmul_rn(g, g)));
+    const float denom = __fadd_rn(__fdiv_rn(__fsqrt_rn(vt), a.bias2_sqrt), a.eps);
     const float delta = __fmul_rn(a.step_size, __fdiv_rn(mt, denom));
     w = __fsub_rn(w, delta);
     m = mt;
     v = vt;
+}
+
+// The step's constants: from the launch, or from device memory for graph replays.
+__device__ __forceinline__ AdamConsts load_consts(const AdamConsts& a, const AdamConsts* ad) {
+    return ad ? *ad : a;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -489,7 +498,8 @@ __device__ __forceinline__ bool consume_stage(const Geom& g, int nd, uint64_t* f
 // ---------------------------------------------------------------------------------------------
 // fused step: reduce-scatter + unscale + Adam + fp16 cast + write-back, TMA-pipelined
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ void fused_element(const FusedArgs& p, uint64_t i, bool& bad) {
+__device__ __forceinline__ void fused_element(const FusedArgs& p, const AdamConsts& a, uint64_t i,
+                                              bool& bad) {
     if (i >= p.n) {   // self-check: never taken when the launch arithmetic is right
         atomicOr(p.status, ZERO_FLAG_BOUNDS);
         return;
@@ -499,7 +509,7 @@ __device__ __forceinline__ void fused_element(const FusedArgs& p, uint64_t i, bo
     const float red = mean_of(s, p.mc);
     bad |= non_finite(red);
     float w = p.master_in[i], m = p.m_in[i], v = p.v_in[i];
-    adam_elem(red, w, m, v, p.a);
+    adam_elem(red, w, m, v, a);
     p.master_out[i] = w;
     p.m_out[i] = m;
     p.v_out[i] = v;
@@ -521,6 +531,7 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
     }
 
     // consumers: thread t owns elements [t*E, t*E + E) of every tile
+    const AdamConsts a = load_consts(p.a, p.ad);
     bool bad = false;
     const uint32_t T = p.g.tile;
     const uint32_t e0 = (uint32_t)threadIdx.x * E;
@@ -550,7 +561,7 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
         for (int j = 0; j < E; ++j) {
             const float red = mean_of(acc[j], p.mc);
             bad |= non_finite(red);
-            adam_elem(red, w[j], m[j], v[j], p.a);
+            adam_elem(red, w[j], m[j], v[j], a);
         }
         stg_f32<E>(p.master_out + g0, w);
         stg_f32<E>(p.m_out + g0, m);
@@ -559,16 +570,17 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
     }
     // the < 8 elements past the last tile
     if (blockIdx.x == 0 && (uint64_t)threadIdx.x < p.n - p.n_tiled)
-        fused_element(p, p.n_tiled + threadIdx.x, bad);
+        fused_element(p, a, p.n_tiled + threadIdx.x, bad);
     flag_overflow(bad, p.status);
 }
 
 // plain-load variant for ranges whose pointers are not 16-byte aligned (or tiny ranges)
 __global__ void __launch_bounds__(256) fused_plain_kernel(const __grid_constant__ FusedArgs p) {
+    const AdamConsts a = load_consts(p.a, p.ad);
     bool bad = false;
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
     for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n; i += stride)
-        fused_element(p, i, bad);
+        fused_element(p, a, i, bad);
     flag_overflow(bad, p.status);
 }
 
@@ -680,6 +692,7 @@ __global__ void __launch_bounds__(256) adam_kernel(const __grid_constant__ AdamA
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.status, ZERO_FLAG_SKIPPED);
         return;
     }
+    const AdamConsts a = load_consts(p.a, p.ad);
     const uint64_t tid = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
     uint64_t done = 0;
@@ -690,10 +703,10 @@ __global__ void __launch_bounds__(256) adam_kernel(const __grid_constant__ AdamA
             float4 w = __ldcs(reinterpret_cast<const float4*>(p.master) + q);
             float4 m = __ldcs(reinterpret_cast<const float4*>(p.m) + q);
             float4 v = __ldcs(reinterpret_cast<const float4*>(p.v) + q);
-            adam_elem(g.x, w.x, m.x, v.x, p.a);
-            adam_elem(g.y, w.y, m.y, v.y, p.a);
-            adam_elem(g.z, w.z, m.z, v.z, p.a);
-            adam_elem(g.w, w.w, m.w, v.w, p.a);
+            adam_elem(g.x, w.x, m.x, v.x, a);
+            adam_elem(g.y, w.y, m.y, v.y, a);
+            adam_elem(g.z, w.z, m.z, v.z, a);
+            adam_elem(g.w, w.w, m.w, v.w, a);
             __stcs(reinterpret_cast<float4*>(p.master) + q, w);
             __stcs(reinterpret_cast<float4*>(p.m) + q, m);
             __stcs(reinterpret_cast<float4*>(p.v) + q, v);
@@ -704,7 +717,7 @@ __global__ void __launch_bounds__(256) adam_kernel(const __grid_constant__ AdamA
     }
     for (uint64_t i = done + tid; i < p.n; i += stride) {
         float w = p.master[i], m = p.m[i], v = p.v[i];
-        adam_elem(p.grad[i], w, m, v, p.a);
+        adam_elem(p.grad[i], w, m, v, a);
         p.master[i] = w;
         p.m[i] = m;
         p.v[i] = v;
@@ -880,7 +893,8 @@ uint64_t launches() { return g_launches.load(std::memory_order_relaxed); }
 cudaError_t launch_fused(uint64_t n, int nd, const uint16_t* const* grads, const float* master_in,
                          const float* m_in, const float* v_in, float* master_out, float* m_out,
                          float* v_out, uint16_t* param_out, const AdamConsts& a,
-                         const MeanConsts& mc, uint32_t* status, cudaStream_t stream) {
+                         const AdamConsts* ad, const MeanConsts& mc, uint32_t* status,
+                         cudaStream_t stream) {
     FusedArgs p;
     memset(&p, 0, sizeof(p));
     bool all16 = aligned16(master_in) && aligned16(m_in) && aligned16(v_in) &&
@@ -901,6 +915,7 @@ cudaError_t launch_fused(uint64_t n, int nd, const uint16_t* const* grads, const
     p.nd = nd;
     p.param_vec = store_vec(param_out);
     p.a = a;
+    p.ad = ad;
     p.mc = mc;
     DevInfo di;
     cudaError_t e = dev_info(&di);
@@ -961,8 +976,8 @@ cudaError_t launch_reduce_scatter(uint64_t n, int nd, const uint16_t* const* gra
 }
 
 cudaError_t launch_adam(uint64_t n, const float* grad, float* master, float* m, float* v,
-                        uint16_t* param_out, const AdamConsts& a, uint32_t* status,
-                        cudaStream_t stream) {
+                        uint16_t* param_out, const AdamConsts& a, const AdamConsts* ad,
+                        uint32_t* status, cudaStream_t stream) {
     AdamArgs p;
     memset(&p, 0, sizeof(p));
     p.grad = grad;
@@ -976,6 +991,7 @@ cudaError_t launch_adam(uint64_t n, const float* grad, float* master, float* m, 
     const int pv = store_vec(param_out);
     p.param_vec = pv > 8 ? 8 : pv;
     p.a = a;
+    p.ad = ad;
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;

@@ -38,7 +38,7 @@ SYMBOLS = (
     "zero_plan_create", "zero_plan_destroy", "zero_plan_info", "zero_plan_tensor_offsets",
     "zero_plan_bucket", "zero_state_bytes",
     "zero_reduce_scatter_bucket", "zero_adam_shard", "zero_step_fused", "zero_step_commit",
-    "zero_step_status",
+    "zero_step_status", "zero_adam_consts_for_step", "zero_adam_shard_dc", "zero_step_fused_dc",
     "zero_sched_slot_elems", "zero_sched_create", "zero_sched_begin_bucket",
     "zero_sched_end_bucket", "zero_sched_wait", "zero_sched_launches", "zero_sched_destroy",
 )
@@ -66,6 +66,15 @@ class _Report(C.Structure):
 class _HP(C.Structure):
     _fields_ = [("lr", C.c_double), ("beta1", C.c_double), ("beta2", C.c_double),
                 ("eps", C.c_double), ("loss_scale", C.c_double)]
+
+
+class AdamConsts(C.Structure):
+    """zero_adam_consts: one step's fp32 constants (copy into device memory for the _dc calls;
+    bytes(obj) gives its 40-byte image)."""
+    _fields_ = [("beta1", C.c_float), ("one_minus_beta1", C.c_float), ("beta2", C.c_float),
+                ("one_minus_beta2", C.c_float), ("step_size", C.c_float),
+                ("bias2_sqrt", C.c_float), ("eps", C.c_float), ("loss_scale", C.c_float),
+                ("inv_loss_scale", C.c_float), ("loss_scale_pow2", C.c_int32)]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -103,6 +112,9 @@ def _load():
                                   vp, vp]
     L.zero_step_commit.argtypes = [u64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.zero_step_status.argtypes = [vp, vp, P(C.c_uint32)]
+    L.zero_adam_consts_for_step.argtypes = [P(_HP), i64, P(AdamConsts)]
+    L.zero_adam_shard_dc.argtypes = [u64, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.zero_step_fused_dc.argtypes = [u64, i32, P(vp), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.zero_sched_slot_elems.argtypes = [vp, i32, P(u64)]
     L.zero_sched_create.argtypes = [vp, vp, u64, i32, P(vp), vp, vp, P(vp)]
     L.zero_sched_begin_bucket.argtypes = [vp, i32, vp, P(vp)]
@@ -253,6 +265,29 @@ def zero_step_fused(n: int, nd: int, rank_grads, master_in, m_in, v_in, master_o
                                 _ptr(m_in, 4), _ptr(v_in, 4), _ptr(master_out, 4),
                                 _ptr(m_out, 4), _ptr(v_out, 4), _ptr(param_out, 2), C.byref(h),
                                 step, _ptr(d_status, 4), _stream(stream)), "zero_step_fused")
+
+
+def zero_adam_consts_for_step(hp: AdamHP, step: int) -> AdamConsts:
+    out = AdamConsts()
+    h = hp._c()
+    _check(_lib.zero_adam_consts_for_step(C.byref(h), step, C.byref(out)),
+           "zero_adam_consts_for_step")
+    return out
+
+
+def zero_adam_shard_dc(n: int, grad, master, m, v, param_out, d_consts, d_status, stream=None):
+    _check(_lib.zero_adam_shard_dc(n, _ptr(grad, 4), _ptr(master, 4), _ptr(m, 4), _ptr(v, 4),
+                                   _ptr(param_out, 2), _ptr(d_consts), _ptr(d_status, 4),
+                                   _stream(stream)), "zero_adam_shard_dc")
+
+
+def zero_step_fused_dc(n: int, nd: int, rank_grads, master_in, m_in, v_in, master_out, m_out,
+                       v_out, param_out, d_consts, d_status, stream=None):
+    _check(_lib.zero_step_fused_dc(n, nd, _ptr_array(rank_grads, 2), _ptr(master_in, 4),
+                                   _ptr(m_in, 4), _ptr(v_in, 4), _ptr(master_out, 4),
+                                   _ptr(m_out, 4), _ptr(v_out, 4), _ptr(param_out, 2),
+                                   _ptr(d_consts), _ptr(d_status, 4), _stream(stream)),
+           "zero_step_fused_dc")
 
 
 def zero_step_commit(n: int, master_in, m_in, v_in, master_out, m_out, v_out, param_out,
