@@ -175,10 +175,13 @@ __device__ __forceinline__ void adam_elem(float red, float& w, float& m, float& 
     v = vt;
 }
 
-// The step's constants: from the launch, or from device memory for graph replays.
-__device__ __forceinline__ AdamConsts load_consts(const AdamConsts& a, const AdamConsts* ad) {
-    return ad ? *ad : a;
-}
+// The step's constants. kDC = false: straight from the kernel parameters (operands from the
+// constant bank, no registers held); kDC = true: loaded once from device memory, for launches
+// captured in a CUDA graph and replayed with other constants.
+#define ZK_STEP_CONSTS(p, a)             \
+    AdamConsts a##_dev;                  \
+    if constexpr (kDC) a##_dev = *(p).ad; \
+    const AdamConsts& a = kDC ? a##_dev : (p).a
 
 // ---------------------------------------------------------------------------------------------
 // mbarrier and bulk-copy primitives (PTX)
@@ -516,7 +519,7 @@ __device__ __forceinline__ void fused_element(const FusedArgs& p, const AdamCons
     p.param_out[i] = f2h(w);
 }
 
-template <int E, int W>
+template <int E, int W, bool kDC>
 __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
     fused_tma_kernel(const __grid_constant__ FusedArgs p) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -531,7 +534,7 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
     }
 
     // consumers: thread t owns elements [t*E, t*E + E) of every tile
-    const AdamConsts a = load_consts(p.a, p.ad);
+    ZK_STEP_CONSTS(p, a);
     bool bad = false;
     const uint32_t T = p.g.tile;
     const uint32_t e0 = (uint32_t)threadIdx.x * E;
@@ -575,8 +578,9 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
 }
 
 // plain-load variant for ranges whose pointers are not 16-byte aligned (or tiny ranges)
+template <bool kDC>
 __global__ void __launch_bounds__(256) fused_plain_kernel(const __grid_constant__ FusedArgs p) {
-    const AdamConsts a = load_consts(p.a, p.ad);
+    ZK_STEP_CONSTS(p, a);
     bool bad = false;
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
     for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n; i += stride)
@@ -686,13 +690,14 @@ __global__ void __launch_bounds__(256) rs_plain_kernel(const __grid_constant__ R
 // ---------------------------------------------------------------------------------------------
 // owner update of a shard from its reduced gradient (unfused path), in place
 // ---------------------------------------------------------------------------------------------
+template <bool kDC>
 __global__ void __launch_bounds__(256) adam_kernel(const __grid_constant__ AdamArgs p) {
     // skip the whole step if any reduce-scatter of it saw inf/NaN
     if (*reinterpret_cast<volatile uint32_t*>(p.status) & ZERO_FLAG_OVERFLOW) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.status, ZERO_FLAG_SKIPPED);
         return;
     }
-    const AdamConsts a = load_consts(p.a, p.ad);
+    ZK_STEP_CONSTS(p, a);
     const uint64_t tid = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
     uint64_t done = 0;
@@ -921,7 +926,10 @@ cudaError_t launch_fused(uint64_t n, int nd, const uint16_t* const* grads, const
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
     if (!all16 || n < kMinTiledElems) {
-        fused_plain_kernel<<<plain_grid(n, di.sms), 256, 0, stream>>>(p);
+        if (ad)
+            fused_plain_kernel<true><<<plain_grid(n, di.sms), 256, 0, stream>>>(p);
+        else
+            fused_plain_kernel<false><<<plain_grid(n, di.sms), 256, 0, stream>>>(p);
         count_launch();
         return cudaGetLastError();
     }
@@ -929,10 +937,18 @@ cudaError_t launch_fused(uint64_t n, int nd, const uint16_t* const* grads, const
     p.g = sh.g;
     p.n_tiled = n & ~(uint64_t)7;
     p.num_tiles = (p.n_tiled + sh.g.tile - 1) / sh.g.tile;
-    switch (sh.warps) {
-        case 16: return launch_pipe(fused_tma_kernel<kElems, 16>, p, sh, stream);
-        case 20: return launch_pipe(fused_tma_kernel<kElems, 20>, p, sh, stream);
-        case 24: return launch_pipe(fused_tma_kernel<kElems, 24>, p, sh, stream);
+    if (ad) {
+        switch (sh.warps) {
+            case 16: return launch_pipe(fused_tma_kernel<kElems, 16, true>, p, sh, stream);
+            case 20: return launch_pipe(fused_tma_kernel<kElems, 20, true>, p, sh, stream);
+            case 24: return launch_pipe(fused_tma_kernel<kElems, 24, true>, p, sh, stream);
+        }
+    } else {
+        switch (sh.warps) {
+            case 16: return launch_pipe(fused_tma_kernel<kElems, 16, false>, p, sh, stream);
+            case 20: return launch_pipe(fused_tma_kernel<kElems, 20, false>, p, sh, stream);
+            case 24: return launch_pipe(fused_tma_kernel<kElems, 24, false>, p, sh, stream);
+        }
     }
     return cudaErrorInvalidConfiguration;
 }
@@ -996,7 +1012,10 @@ cudaError_t launch_adam(uint64_t n, const float* grad, float* master, float* m, 
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
     uint64_t work = p.vec ? (n + 3) / 4 : n;
-    adam_kernel<<<plain_grid(work, di.sms), 256, 0, stream>>>(p);
+    if (ad)
+        adam_kernel<true><<<plain_grid(work, di.sms), 256, 0, stream>>>(p);
+    else
+        adam_kernel<false><<<plain_grid(work, di.sms), 256, 0, stream>>>(p);
     count_launch();
     return cudaGetLastError();
 }
