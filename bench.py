@@ -52,7 +52,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["gpt2_small", "shard_7p5b", "flat", "zero2_1p3b"],
+    ap.add_argument("--workload", choices=["gpt2_small", "shard_7p5b", "flat", "zero2_1p3b",
+                                           "zero2_gpt2_small"],
                     default="gpt2_small")
     ap.add_argument("--nd", type=int, default=None)
     ap.add_argument("--bucket", type=int, default=None)
@@ -115,7 +116,7 @@ class Workload:
             self.param_base = r * S
             self.config = {"workload": "shard_7p5b_rank31", "psi_total": total, "shard": S,
                            "nd": nd, "owner": r, "calls_per_step": 1}
-        elif kind == "zero2_1p3b":
+        elif kind in ("zero2_1p3b", "zero2_gpt2_small"):
             self._init_zero2(args, dev)
             return
         else:
@@ -225,15 +226,17 @@ class Workload:
 
 
 def _init_zero2(self, args, dev):
-    """Stage 2 on the 1.3B list: Nd = 16, buckets of 50,000,000 elements. The backward pass's
+    """Stage 2 on the 1.3B list (Nd = 16, buckets of 50,000,000 elements), or on the GPT-2-small
+    list (Nd = 8, buckets of 10,000,000; a smaller case for profiling). The backward pass's
     output (every bucket's local gradients of every rank) is already in the scheduler's staging
-    slots, one slot per bucket; a step is the reduce-scatter of the 27 buckets in backward
-    order through the scheduler, then the 16 owners' updates (zero_adam_shard)."""
+    slots, one slot per bucket; a step is the reduce-scatter of the buckets in backward order
+    through the scheduler, then the owners' updates (zero_adam_shard)."""
     torch, lz = self.torch, self.lz
     from zero_partitioned_optimizer_plan_b200 import synth
-    nd = args.nd or 16
-    B = args.bucket or 50_000_000
-    numels = synth.gpt_1p3b_list()
+    small = args.workload == "zero2_gpt2_small"
+    nd = args.nd or (8 if small else 16)
+    B = args.bucket or (10_000_000 if small else 50_000_000)
+    numels = synth.gpt2_small_list() if small else synth.gpt_1p3b_list()
     self.plan = pl = lz.zero_plan_create(numels, nd, 2, B)
     psi, psi_p, S, nb = lz.zero_plan_info(pl)
     self.nd, self.n, self.psi, self.S, self.nb = nd, psi_p, psi, S, nb
@@ -252,7 +255,7 @@ def _init_zero2(self, args, dev):
     self.grads = None
     self.ranges = [(0, psi_p)]
     self.param_base = 0
-    self.config = {"workload": "zero2_1p3b", "psi": psi, "nd": nd, "stage": 2, "bucket": B,
+    self.config = {"workload": args.workload, "psi": psi, "nd": nd, "stage": 2, "bucket": B,
                    "buckets": nb, "calls_per_step": nb + nd}
     rs_bytes = (2 * nd + 4) * psi_p
     adam_bytes = 30 * psi_p
