@@ -52,6 +52,9 @@ namespace {
 #ifndef ZK_COMMIT_BLOCKS_PER_SM
 #define ZK_COMMIT_BLOCKS_PER_SM 1
 #endif
+#ifndef ZK_ADAM_UNROLL     // float4 groups per thread and iteration of the plain owner update
+#define ZK_ADAM_UNROLL 2
+#endif
 
 constexpr int kMaxRanks = ZERO_MAX_RANKS;
 constexpr int kElems = 4;                        // elements per consumer thread and tile
@@ -688,7 +691,10 @@ __global__ void __launch_bounds__(256) rs_plain_kernel(const __grid_constant__ R
 }
 
 // ---------------------------------------------------------------------------------------------
-// owner update of a shard from its reduced gradient (unfused path), in place
+// owner update of a shard from its reduced gradient (unfused path), in place.
+// 30 bytes per parameter, half of them written back to the addresses just read; plain
+// 128-bit loads with two groups in flight per thread measured faster on B200 (6.18 TB/s) than
+// a bulk-copy pipeline like the fused kernel's (5.2-6.0 TB/s for 8-24 consumer warps).
 // ---------------------------------------------------------------------------------------------
 template <bool kDC>
 __global__ void __launch_bounds__(256) adam_kernel(const __grid_constant__ AdamArgs p) {
@@ -702,21 +708,36 @@ __global__ void __launch_bounds__(256) adam_kernel(const __grid_constant__ AdamA
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
     uint64_t done = 0;
     if (p.vec) {
+        // U float4 groups per thread and iteration: all their loads are issued before any
+        // arithmetic, so U*64 bytes per thread are in flight
+        constexpr int U = ZK_ADAM_UNROLL;
         const uint64_t n4 = p.n / 4;
-        for (uint64_t q = tid; q < n4; q += stride) {
-            const float4 g = __ldcs(reinterpret_cast<const float4*>(p.grad) + q);
-            float4 w = __ldcs(reinterpret_cast<const float4*>(p.master) + q);
-            float4 m = __ldcs(reinterpret_cast<const float4*>(p.m) + q);
-            float4 v = __ldcs(reinterpret_cast<const float4*>(p.v) + q);
-            adam_elem(g.x, w.x, m.x, v.x, a);
-            adam_elem(g.y, w.y, m.y, v.y, a);
-            adam_elem(g.z, w.z, m.z, v.z, a);
-            adam_elem(g.w, w.w, m.w, v.w, a);
-            __stcs(reinterpret_cast<float4*>(p.master) + q, w);
-            __stcs(reinterpret_cast<float4*>(p.m) + q, m);
-            __stcs(reinterpret_cast<float4*>(p.v) + q, v);
-            const float x[4] = {w.x, w.y, w.z, w.w};
-            stg_f16<4>(p.param_out + 4 * q, x, p.param_vec);
+        for (uint64_t q0 = tid; q0 < n4; q0 += stride * U) {
+            float4 g[U], w[U], m[U], v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const uint64_t q = q0 + (uint64_t)u * stride;
+                if (q < n4) {
+                    g[u] = __ldcs(reinterpret_cast<const float4*>(p.grad) + q);
+                    w[u] = __ldcs(reinterpret_cast<const float4*>(p.master) + q);
+                    m[u] = __ldcs(reinterpret_cast<const float4*>(p.m) + q);
+                    v[u] = __ldcs(reinterpret_cast<const float4*>(p.v) + q);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const uint64_t q = q0 + (uint64_t)u * stride;
+                if (q >= n4) break;
+                adam_elem(g[u].x, w[u].x, m[u].x, v[u].x, a);
+                adam_elem(g[u].y, w[u].y, m[u].y, v[u].y, a);
+                adam_elem(g[u].z, w[u].z, m[u].z, v[u].z, a);
+                adam_elem(g[u].w, w[u].w, m[u].w, v[u].w, a);
+                __stcs(reinterpret_cast<float4*>(p.master) + q, w[u]);
+                __stcs(reinterpret_cast<float4*>(p.m) + q, m[u]);
+                __stcs(reinterpret_cast<float4*>(p.v) + q, v[u]);
+                const float x[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+                stg_f16<4>(p.param_out + 4 * q, x, p.param_vec);
+            }
         }
         done = n4 * 4;
     }
