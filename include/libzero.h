@@ -249,6 +249,14 @@ zero_status zero_step_commit(uint64_t n, const float* master_in, const float* m_
  * set or the copy fails, else ZERO_OK. This is the only call that blocks the host. */
 zero_status zero_step_status(const uint32_t* d_status, zero_stream_t stream, uint32_t* flags_out);
 
+/* Self-test of the kernels' bounded waits (failure detection without a fault): launches the
+ * fused pipeline on one tile with its copy-issuing warp switched off, so every consumer's wait
+ * on shared-memory data expires after about one second; the kernel then sets
+ * ZERO_FLAG_TIMEOUT in *d_status and returns, and the CUDA context stays usable. No other
+ * memory is read or written. The pages have no counterpart; it checks this library's own
+ * error path. Errors: ZERO_EINVAL (null), ZERO_EALIGN, ZERO_ECUDA. */
+zero_status zero_selftest_timeout(uint32_t* d_status, zero_stream_t stream);
+
 /* ------------------------------------------------------------------------------------------
  * Stream-ordered bucket scheduler for stage 2. "ZeRO-2" card, "Gradient 생명주기": after a
  * bucket's reduce-scatter the GPU keeps its own reduced shard and releases the rest of the

@@ -443,3 +443,29 @@ def test_graph_replay_of_bucketed_step():
         check_f32(f"step {t} m", f32np(out[1]), m_r)
         check_f32(f"step {t} v", f32np(out[2]), v_r)
         check_f16(f"step {t} params", f16np(params), p_r)
+
+
+def test_bounded_wait_expires_and_context_survives():
+    """Failure detection without a fault: the pipeline's wait for data that never comes gives up
+    after about a second with ZERO_FLAG_TIMEOUT, and the next step on the same context works."""
+    import time
+    st = status_word()
+    t0 = time.perf_counter()
+    lz.zero_selftest_timeout(st)
+    code, flags = lz.zero_step_status(st)
+    dt = time.perf_counter() - t0
+    assert code == lz.ZERO_ECUDA and flags == lz.ZERO_FLAG_TIMEOUT
+    assert 0.5 < dt < 30.0
+    # the context is still usable
+    n, nd = 5000, 3
+    master, m, v = synth.state_warm(n, seed=81)
+    pp = PingPong(master, m, v)
+    g_cpu = _rank_grads_cpu(n, nd, 82, 1)
+    params = torch.empty(n, dtype=torch.float16, device=DEV)
+    st = status_word()
+    fused_step(n, [g.to(DEV) for g in g_cpu], pp, params, HP, 1, st)
+    assert lz.zero_step_status(st) == (lz.ZERO_OK, 0)
+    skipped, w, mm, vv, p = oracle.step([g.numpy() for g in g_cpu], master.numpy(), m.numpy(),
+                                        v.numpy(), ORC_HP, 1)
+    check_f32("master", f32np(pp.nxt[0]), w)
+    check_f16("params", f16np(params), p)

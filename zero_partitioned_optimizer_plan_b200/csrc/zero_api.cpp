@@ -111,6 +111,12 @@ uint64_t zero_kernel_launches(void) { return zk::launches(); }
 
 const char* zero_last_error(void) { return zk::g_last_error; }
 
+zero_status zero_selftest_timeout(uint32_t* d_status, zero_stream_t stream) {
+    if (!d_status) return ZERO_EINVAL;
+    if (!zk::aligned(d_status, 4)) return ZERO_EALIGN;
+    return zk::from_cuda(zk::launch_selftest_timeout(d_status, (cudaStream_t)stream));
+}
+
 zero_status zero_reduce_scatter_bucket(const zero_plan* plan, int k,
                                        const uint16_t* const* rank_grads,
                                        float* const* owner_grad_shards, uint32_t* d_status,

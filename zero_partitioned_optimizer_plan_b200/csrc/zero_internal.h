@@ -42,6 +42,8 @@ cudaError_t launch_adam(uint64_t n, const float* grad, float* master, float* m, 
                         uint16_t* param_out, const AdamConsts& a, const AdamConsts* ad,
                         uint32_t* status, cudaStream_t stream);
 
+cudaError_t launch_selftest_timeout(uint32_t* status, cudaStream_t stream);
+
 // Count of kernels this library has launched in this process.
 void count_launch();
 uint64_t launches();

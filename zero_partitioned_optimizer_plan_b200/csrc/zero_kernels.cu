@@ -99,6 +99,7 @@ struct FusedArgs {
     AdamConsts a;
     const AdamConsts* ad;  // when not null: the constants, read from device memory at run time
     MeanConsts mc;
+    int selftest_no_copies;  // self-test only: the producer issues nothing (waits must expire)
 };
 
 struct RsArgs {
@@ -532,7 +533,7 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
     init_barriers(full, empty, p.g.stages, W);
 
     if ((threadIdx.x >> 5) == W) {
-        produce<true>(p, full, empty, data);
+        if (!p.selftest_no_copies) produce<true>(p, full, empty, data);
         return;
     }
 
@@ -913,6 +914,29 @@ unsigned plain_grid(uint64_t n, int sms, int per_sm = 8) {
 }  // namespace
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+// Launch the fused pipeline on one tile whose producer issues nothing: every consumer's bounded
+// wait on the first stage expires, the kernel sets ZERO_FLAG_TIMEOUT and returns. No global
+// memory is read or written except the status word.
+cudaError_t launch_selftest_timeout(uint32_t* status, cudaStream_t stream) {
+    FusedArgs p;
+    memset(&p, 0, sizeof(p));
+    p.status = status;
+    p.nd = 1;
+    p.n = 4096;
+    p.n_tiled = 4096;
+    p.selftest_no_copies = 1;
+    p.mc = make_mean(1);
+    const PipeShape sh = pipe_shape(1, true);
+    p.g = sh.g;
+    p.num_tiles = 1;
+    switch (sh.warps) {
+        case 16: return launch_pipe(fused_tma_kernel<kElems, 16, false>, p, sh, stream);
+        case 20: return launch_pipe(fused_tma_kernel<kElems, 20, false>, p, sh, stream);
+        case 24: return launch_pipe(fused_tma_kernel<kElems, 24, false>, p, sh, stream);
+    }
+    return cudaErrorInvalidConfiguration;
+}
 
 uint64_t launches() { return g_launches.load(std::memory_order_relaxed); }
 

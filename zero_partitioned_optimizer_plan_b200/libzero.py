@@ -39,6 +39,7 @@ SYMBOLS = (
     "zero_plan_bucket", "zero_state_bytes",
     "zero_reduce_scatter_bucket", "zero_adam_shard", "zero_step_fused", "zero_step_commit",
     "zero_step_status", "zero_adam_consts_for_step", "zero_adam_shard_dc", "zero_step_fused_dc",
+    "zero_selftest_timeout",
     "zero_sched_slot_elems", "zero_sched_create", "zero_sched_begin_bucket",
     "zero_sched_end_bucket", "zero_sched_wait", "zero_sched_launches", "zero_sched_destroy",
 )
@@ -115,6 +116,7 @@ def _load():
     L.zero_adam_consts_for_step.argtypes = [P(_HP), i64, P(AdamConsts)]
     L.zero_adam_shard_dc.argtypes = [u64, vp, vp, vp, vp, vp, vp, vp, vp]
     L.zero_step_fused_dc.argtypes = [u64, i32, P(vp), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.zero_selftest_timeout.argtypes = [vp, vp]
     L.zero_sched_slot_elems.argtypes = [vp, i32, P(u64)]
     L.zero_sched_create.argtypes = [vp, vp, u64, i32, P(vp), vp, vp, P(vp)]
     L.zero_sched_begin_bucket.argtypes = [vp, i32, vp, P(vp)]
@@ -303,6 +305,10 @@ def zero_step_status(d_status, stream=None):
     flags = C.c_uint32()
     code = _lib.zero_step_status(_ptr(d_status, 4), _stream(stream), C.byref(flags))
     return int(code), int(flags.value)
+
+
+def zero_selftest_timeout(d_status, stream=None):
+    _check(_lib.zero_selftest_timeout(_ptr(d_status, 4), _stream(stream)), "zero_selftest_timeout")
 
 
 # ---------------------------------------------------------------------------------------------
