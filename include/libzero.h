@@ -235,6 +235,55 @@ zero_status zero_step_fused_dc(uint64_t n, int nd, const uint16_t* const* rank_g
                                uint16_t* param_out, const zero_adam_consts* d_consts,
                                uint32_t* d_status, zero_stream_t stream);
 
+/* ------------------------------------------------------------------------------------------
+ * Dynamic loss scaling on the device. The pages fix only a static picture (fp16 gradients,
+ * mixed-precision Adam); this is the rule of Micikevicius et al., "Mixed Precision Training"
+ * (ICLR 2018, section 3.2), as torch.cuda.amp.GradScaler states it: a step whose reduced
+ * gradients overflow is skipped and the scale is multiplied by backoff_factor; after
+ * growth_interval consecutive applied steps it is multiplied by growth_factor. Adam's t counts
+ * applied steps only. Everything lives in device memory, so a step needs no host read:
+ *   zero_scaler_prepare -> zero_step_fused_dc (per bucket) -> zero_step_commit
+ *                       -> zero_scaler_update          (or ... zero_adam_shard_dc ... update)
+ * and the whole sequence can be captured once as a CUDA graph.
+ * ---------------------------------------------------------------------------------------- */
+typedef struct {
+    float scale;             /* the scale the next step's gradients carry */
+    int32_t good_steps;      /* consecutive applied steps since the scale last changed */
+    int64_t next_step;       /* Adam t of the next applied step (starts at 1) */
+    int64_t skipped_steps;   /* steps skipped so far */
+} zero_scaler_state;
+
+typedef struct {
+    float growth_factor;     /* e.g. 2 */
+    float backoff_factor;    /* e.g. 0.5 */
+    int32_t growth_interval; /* e.g. 2000, >= 1 */
+} zero_scaler_params;
+
+/* Host: out[i] = the constants of step first_step + i, i < count (as zero_adam_consts_for_step).
+ * Copy the table to device memory for zero_scaler_prepare. Errors: ZERO_EINVAL. */
+zero_status zero_adam_consts_table(const zero_adam_hparams* hp, int64_t first_step, int64_t count,
+                                   zero_adam_consts* out);
+
+/* Device, first call of a step: *d_status = 0 and *d_consts = d_table[t - 1] with t =
+ * d_state->next_step and the loss scale replaced by d_state->scale. If t is outside
+ * [1, table_len] the step is refused: *d_status = ZERO_FLAG_OVERFLOW | ZERO_FLAG_BOUNDS, so the
+ * step's kernels skip it, zero_scaler_update leaves the scaler alone and zero_step_status
+ * reports ZERO_ECUDA. All pointers device memory; d_state 8-byte aligned, the others 4.
+ * Errors: ZERO_EINVAL (null, table_len < 1), ZERO_EALIGN, ZERO_ECUDA. */
+zero_status zero_scaler_prepare(const zero_scaler_state* d_state, const zero_adam_consts* d_table,
+                                int64_t table_len, zero_adam_consts* d_consts, uint32_t* d_status,
+                                zero_stream_t stream);
+
+/* Device, after the step's last kernel (zero_step_commit or the last zero_adam_shard_dc):
+ * if *d_status has ZERO_FLAG_OVERFLOW the scale is multiplied by backoff_factor, good_steps
+ * reset and skipped_steps counted; otherwise next_step and good_steps advance and the scale is
+ * multiplied by growth_factor when good_steps reaches growth_interval. A status with
+ * ZERO_FLAG_TIMEOUT or ZERO_FLAG_BOUNDS leaves the scaler unchanged.
+ * Errors: ZERO_EINVAL (null pointers, growth_interval < 1, non-finite or non-positive
+ * factors), ZERO_EALIGN, ZERO_ECUDA. */
+zero_status zero_scaler_update(zero_scaler_state* d_state, const zero_scaler_params* params,
+                               const uint32_t* d_status, zero_stream_t stream);
+
 /* Close a step made of zero_step_fused calls, on the same stream, over the same range(s).
  * If ZERO_FLAG_OVERFLOW is set: (master_out, m_out, v_out) = (master_in, m_in, v_in),
  * param_out = fp16(master_in), and ZERO_FLAG_SKIPPED is set -- the step did not happen.

@@ -354,3 +354,42 @@ def ulp_diff_f16(a, b) -> np.ndarray:
     na = ((a & 0x7c00) == 0x7c00) & ((a & 0x3ff) != 0)
     nb = ((b & 0x7c00) == 0x7c00) & ((b & 0x3ff) != 0)
     return np.where(na & nb, 0, np.where(na ^ nb, 1 << 32, d))
+
+
+# ---------------------------------------------------------------------------------------------
+# dynamic loss scaling (the pages say nothing about it; the rule is the one of Micikevicius et
+# al., "Mixed Precision Training", ICLR 2018, section 3.2, in the form of torch.cuda.amp's
+# GradScaler): an overflowing step is skipped and the scale is multiplied by backoff_factor;
+# after growth_interval consecutive applied steps it is multiplied by growth_factor. The Adam
+# step t counts applied steps only. The scale is a binary32 number.
+# ---------------------------------------------------------------------------------------------
+@dataclasses.dataclass
+class Scaler:
+    scale: float = 1024.0
+    good_steps: int = 0
+    next_step: int = 1
+    skipped_steps: int = 0
+    growth_factor: float = 2.0
+    backoff_factor: float = 0.5
+    growth_interval: int = 2000
+
+    def update(self, overflowed: bool):
+        if overflowed:
+            self.scale = float(np.float32(self.scale) * np.float32(self.backoff_factor))
+            self.good_steps = 0
+            self.skipped_steps += 1
+        else:
+            self.next_step += 1
+            self.good_steps += 1
+            if self.good_steps >= self.growth_interval:
+                self.scale = float(np.float32(self.scale) * np.float32(self.growth_factor))
+                self.good_steps = 0
+
+
+def scaled_step(grads, master, m, v, hp: AdamHP, sc: Scaler):
+    """One step under dynamic loss scaling: the gradients carry sc.scale, Adam uses step
+    sc.next_step; then the scaler is updated. Returns (skipped, master, m, v, p16)."""
+    hp_t = dataclasses.replace(hp, loss_scale=sc.scale)
+    skipped, w, mm, vv, p16 = step(grads, master, m, v, hp_t, sc.next_step)
+    sc.update(skipped)
+    return skipped, w, mm, vv, p16

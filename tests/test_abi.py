@@ -250,3 +250,32 @@ def test_dc_variants_reject():
             lz.zero_adam_shard_dc(10, A, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, dc,
                                   A + 5 * MB, 0)
         assert e.value.code == code
+
+
+def test_consts_table_matches_per_step():
+    tab = lz.zero_adam_consts_table(HP, 5, 20)
+    for i in range(20):
+        c = lz.zero_adam_consts_for_step(HP, 5 + i)
+        assert bytes(tab[i]) == bytes(c)
+    with pytest.raises(lz.ZeroError):
+        lz.zero_adam_consts_table(HP, 0, 3)
+
+
+def test_scaler_rejects():
+    ok = lz.ScalerParams(2.0, 0.5, 2000)
+    for args, code in [((0, A, 10, A + MB, A + 2 * MB), lz.ZERO_EINVAL),
+                       ((A, A, 0, A + MB, A + 2 * MB), lz.ZERO_EINVAL),
+                       ((A + 4, A, 10, A + MB, A + 2 * MB), lz.ZERO_EALIGN),
+                       ((A, A + MB, 10, A + MB + 40, A + 2 * MB), lz.ZERO_EINVAL)]:  # in table
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_scaler_prepare(*args, 0)
+        assert e.value.code == code
+    for prm, code in [(lz.ScalerParams(2.0, 0.5, 0), lz.ZERO_EINVAL),
+                      (lz.ScalerParams(float("inf"), 0.5, 10), lz.ZERO_EINVAL),
+                      (lz.ScalerParams(2.0, -0.5, 10), lz.ZERO_EINVAL)]:
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_scaler_update(A, prm, A + MB, 0)
+        assert e.value.code == code
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_scaler_update(A + 4, ok, A + MB, 0)
+    assert e.value.code == lz.ZERO_EALIGN

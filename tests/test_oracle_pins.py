@@ -467,3 +467,36 @@ def test_ulp_metric():
     h = np.array([0x3c00, 0x8000, 0x0001], np.uint16)
     k = np.array([0x3c01, 0x0000, 0x8001], np.uint16)
     assert list(oracle.ulp_diff_f16(h, k)) == [1, 0, 2]
+
+
+def test_dynamic_scale_golden_sequence():
+    g = _golden("dynamic_scale_sequence.json")
+    sc = oracle.Scaler(scale=g["init_scale"], growth_factor=g["growth_factor"],
+                       backoff_factor=g["backoff_factor"], growth_interval=g["growth_interval"])
+    for ovf, s_before, t in zip(g["overflow"], g["scale_before_step"], g["adam_t_of_step"]):
+        assert sc.scale == s_before
+        if t is not None:
+            assert sc.next_step == t
+        sc.update(ovf)
+    assert (sc.scale, sc.good_steps, sc.next_step, sc.skipped_steps) == tuple(g["final"].values())
+
+
+def test_scaled_step_unscales_by_the_current_scale():
+    # the same gradients at scale 2S against halved inputs at scale S give the same update:
+    # the update only sees g = red / scale
+    rng = np.random.default_rng(5)
+    n = 512
+    g16 = (rng.standard_normal(n) * 1e-2).astype(np.float16)
+    half = (g16.astype(np.float32) / 2).astype(np.float16)
+    ok = g16.astype(np.float32) / 2 == half.astype(np.float32)   # exactly halved elements
+    master = rng.standard_normal(n).astype(np.float32)
+    z = np.zeros(n, np.float32)
+    a = oracle.scaled_step([g16], master, z, z, HP, oracle.Scaler(scale=2048.0))
+    b = oracle.scaled_step([half], master, z, z, HP, oracle.Scaler(scale=1024.0))
+    assert np.array_equal(a[1][ok].view(np.uint32), b[1][ok].view(np.uint32))
+    # a skipped step leaves t where it was and halves the scale
+    bad = g16.copy()
+    bad[7] = np.float16(np.inf)
+    sc = oracle.Scaler(scale=1024.0)
+    skipped, *_ = oracle.scaled_step([bad], master, z, z, HP, sc)
+    assert skipped and sc.next_step == 1 and sc.scale == 512.0 and sc.skipped_steps == 1

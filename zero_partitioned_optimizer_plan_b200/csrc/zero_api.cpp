@@ -169,6 +169,42 @@ zero_status zero_adam_consts_for_step(const zero_adam_hparams* hp, int64_t step,
     return ZERO_OK;
 }
 
+zero_status zero_adam_consts_table(const zero_adam_hparams* hp, int64_t first_step, int64_t count,
+                                   zero_adam_consts* out) {
+    if (!zk::hparams_ok(hp) || first_step < 1 || count < 0 || (count > 0 && !out))
+        return ZERO_EINVAL;
+    if (count > 0 && first_step > INT64_MAX - count) return ZERO_EINVAL;
+    for (int64_t i = 0; i < count; ++i) out[i] = zk::make_adam(hp, first_step + i);
+    return ZERO_OK;
+}
+
+zero_status zero_scaler_prepare(const zero_scaler_state* d_state, const zero_adam_consts* d_table,
+                                int64_t table_len, zero_adam_consts* d_consts, uint32_t* d_status,
+                                zero_stream_t stream) {
+    if (!d_state || !d_table || !d_consts || !d_status || table_len < 1) return ZERO_EINVAL;
+    if (!zk::aligned(d_state, 8) || !zk::aligned(d_table, 4) || !zk::aligned(d_consts, 4) ||
+        !zk::aligned(d_status, 4))
+        return ZERO_EALIGN;
+    if (zk::overlap(d_consts, sizeof(zero_adam_consts), d_table,
+                    (uint64_t)table_len * sizeof(zero_adam_consts)) ||
+        zk::overlap(d_consts, sizeof(zero_adam_consts), d_status, 4) ||
+        zk::overlap(d_consts, sizeof(zero_adam_consts), d_state, sizeof(zero_scaler_state)))
+        return ZERO_EINVAL;
+    return zk::from_cuda(zk::launch_scaler_prepare(d_state, d_table, table_len, d_consts,
+                                                   d_status, (cudaStream_t)stream));
+}
+
+zero_status zero_scaler_update(zero_scaler_state* d_state, const zero_scaler_params* params,
+                               const uint32_t* d_status, zero_stream_t stream) {
+    if (!d_state || !params || !d_status || params->growth_interval < 1) return ZERO_EINVAL;
+    if (!zk::finite(params->growth_factor) || !(params->growth_factor > 0.0f) ||
+        !zk::finite(params->backoff_factor) || !(params->backoff_factor > 0.0f))
+        return ZERO_EINVAL;
+    if (!zk::aligned(d_state, 8) || !zk::aligned(d_status, 4)) return ZERO_EALIGN;
+    return zk::from_cuda(zk::launch_scaler_update(d_state, *params, d_status,
+                                                  (cudaStream_t)stream));
+}
+
 zero_status zero_adam_shard(uint64_t n, const float* grad, float* master, float* m, float* v,
                             uint16_t* param_out, const zero_adam_hparams* hp, int64_t step,
                             uint32_t* d_status, zero_stream_t stream) {

@@ -43,6 +43,11 @@ cudaError_t launch_adam(uint64_t n, const float* grad, float* master, float* m, 
                         uint32_t* status, cudaStream_t stream);
 
 cudaError_t launch_selftest_timeout(uint32_t* status, cudaStream_t stream);
+cudaError_t launch_scaler_prepare(const zero_scaler_state* st, const AdamConsts* table,
+                                  int64_t table_len, AdamConsts* out, uint32_t* status,
+                                  cudaStream_t stream);
+cudaError_t launch_scaler_update(zero_scaler_state* st, const zero_scaler_params& prm,
+                                 const uint32_t* status, cudaStream_t stream);
 
 // Count of kernels this library has launched in this process.
 void count_launch();

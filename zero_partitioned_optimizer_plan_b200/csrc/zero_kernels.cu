@@ -769,6 +769,50 @@ __global__ void __launch_bounds__(256) commit_kernel(const __grid_constant__ Com
 }
 
 // ---------------------------------------------------------------------------------------------
+// dynamic loss scaling: one thread each, before and after a step
+// ---------------------------------------------------------------------------------------------
+__global__ void scaler_prepare_kernel(const zero_scaler_state* st, const AdamConsts* table,
+                                      int64_t table_len, AdamConsts* out, uint32_t* status) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    const int64_t t = st->next_step;
+    if (t < 1 || t > table_len) {   // refuse the step: skipped by its kernels, scaler kept
+        *status = ZERO_FLAG_OVERFLOW | ZERO_FLAG_BOUNDS;
+        return;
+    }
+    *status = 0u;
+    AdamConsts c = table[t - 1];
+    const float s = st->scale;
+    const uint32_t bits = __float_as_uint(s);
+    const uint32_t e = (bits >> 23) & 0xffu;
+    // a positive power of two 2^k whose reciprocal 2^-k is a normal number (1 <= e <= 253):
+    // the unscale may multiply by the exact reciprocal instead of dividing
+    const bool pow2 = (bits & 0x807fffffu) == 0u && e >= 1u && e <= 253u;
+    c.loss_scale = s;
+    c.inv_loss_scale = pow2 ? __uint_as_float((254u - e) << 23) : 0.0f;
+    c.loss_scale_pow2 = pow2 ? 1 : 0;
+    *out = c;
+}
+
+__global__ void scaler_update_kernel(zero_scaler_state* st, zero_scaler_params prm,
+                                     const uint32_t* status) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    const uint32_t f = *status;
+    if (f & (ZERO_FLAG_TIMEOUT | ZERO_FLAG_BOUNDS)) return;   // an error, not an overflow
+    if (f & ZERO_FLAG_OVERFLOW) {
+        st->scale = __fmul_rn(st->scale, prm.backoff_factor);
+        st->good_steps = 0;
+        st->skipped_steps += 1;
+    } else {
+        st->next_step += 1;
+        st->good_steps += 1;
+        if (st->good_steps >= prm.growth_interval) {
+            st->scale = __fmul_rn(st->scale, prm.growth_factor);
+            st->good_steps = 0;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------------
 std::atomic<uint64_t> g_launches{0};
@@ -1061,6 +1105,21 @@ cudaError_t launch_adam(uint64_t n, const float* grad, float* master, float* m, 
         adam_kernel<true><<<plain_grid(work, di.sms), 256, 0, stream>>>(p);
     else
         adam_kernel<false><<<plain_grid(work, di.sms), 256, 0, stream>>>(p);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scaler_prepare(const zero_scaler_state* st, const AdamConsts* table,
+                                  int64_t table_len, AdamConsts* out, uint32_t* status,
+                                  cudaStream_t stream) {
+    scaler_prepare_kernel<<<1, 32, 0, stream>>>(st, table, table_len, out, status);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scaler_update(zero_scaler_state* st, const zero_scaler_params& prm,
+                                 const uint32_t* status, cudaStream_t stream) {
+    scaler_update_kernel<<<1, 32, 0, stream>>>(st, prm, status);
     count_launch();
     return cudaGetLastError();
 }

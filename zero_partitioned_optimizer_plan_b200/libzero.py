@@ -39,7 +39,8 @@ SYMBOLS = (
     "zero_plan_bucket", "zero_state_bytes",
     "zero_reduce_scatter_bucket", "zero_adam_shard", "zero_step_fused", "zero_step_commit",
     "zero_step_status", "zero_adam_consts_for_step", "zero_adam_shard_dc", "zero_step_fused_dc",
-    "zero_selftest_timeout",
+    "zero_selftest_timeout", "zero_adam_consts_table", "zero_scaler_prepare",
+    "zero_scaler_update",
     "zero_sched_slot_elems", "zero_sched_create", "zero_sched_begin_bucket",
     "zero_sched_end_bucket", "zero_sched_wait", "zero_sched_launches", "zero_sched_destroy",
 )
@@ -76,6 +77,17 @@ class AdamConsts(C.Structure):
                 ("one_minus_beta2", C.c_float), ("step_size", C.c_float),
                 ("bias2_sqrt", C.c_float), ("eps", C.c_float), ("loss_scale", C.c_float),
                 ("inv_loss_scale", C.c_float), ("loss_scale_pow2", C.c_int32)]
+
+
+class ScalerState(C.Structure):
+    """zero_scaler_state (24 bytes; copy into 8-byte-aligned device memory)."""
+    _fields_ = [("scale", C.c_float), ("good_steps", C.c_int32), ("next_step", C.c_int64),
+                ("skipped_steps", C.c_int64)]
+
+
+class ScalerParams(C.Structure):
+    _fields_ = [("growth_factor", C.c_float), ("backoff_factor", C.c_float),
+                ("growth_interval", C.c_int32)]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -117,6 +129,9 @@ def _load():
     L.zero_adam_shard_dc.argtypes = [u64, vp, vp, vp, vp, vp, vp, vp, vp]
     L.zero_step_fused_dc.argtypes = [u64, i32, P(vp), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.zero_selftest_timeout.argtypes = [vp, vp]
+    L.zero_adam_consts_table.argtypes = [P(_HP), i64, i64, P(AdamConsts)]
+    L.zero_scaler_prepare.argtypes = [vp, vp, i64, vp, vp, vp]
+    L.zero_scaler_update.argtypes = [vp, P(ScalerParams), vp, vp]
     L.zero_sched_slot_elems.argtypes = [vp, i32, P(u64)]
     L.zero_sched_create.argtypes = [vp, vp, u64, i32, P(vp), vp, vp, P(vp)]
     L.zero_sched_begin_bucket.argtypes = [vp, i32, vp, P(vp)]
@@ -305,6 +320,24 @@ def zero_step_status(d_status, stream=None):
     flags = C.c_uint32()
     code = _lib.zero_step_status(_ptr(d_status, 4), _stream(stream), C.byref(flags))
     return int(code), int(flags.value)
+
+
+def zero_adam_consts_table(hp: AdamHP, first_step: int, count: int):
+    out = (AdamConsts * max(count, 1))()
+    h = hp._c()
+    _check(_lib.zero_adam_consts_table(C.byref(h), first_step, count, out),
+           "zero_adam_consts_table")
+    return out
+
+
+def zero_scaler_prepare(d_state, d_table, table_len: int, d_consts, d_status, stream=None):
+    _check(_lib.zero_scaler_prepare(_ptr(d_state), _ptr(d_table), table_len, _ptr(d_consts),
+                                    _ptr(d_status, 4), _stream(stream)), "zero_scaler_prepare")
+
+
+def zero_scaler_update(d_state, params: ScalerParams, d_status, stream=None):
+    _check(_lib.zero_scaler_update(_ptr(d_state), C.byref(params), _ptr(d_status, 4),
+                                   _stream(stream)), "zero_scaler_update")
 
 
 def zero_selftest_timeout(d_status, stream=None):
