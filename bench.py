@@ -60,6 +60,9 @@ def parse():
     ap.add_argument("--psi", type=int, default=None, help="flat workload size (default 2^29)")
     ap.add_argument("--graph", action="store_true",
                     help="capture a step's calls in CUDA graphs (constants in device memory)")
+    ap.add_argument("--dynamic-scale", action="store_true",
+                    help="with --graph: dynamic loss scaling on the device (scaler prepare and "
+                         "update kernels in the graph, no host work per step)")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -148,23 +151,39 @@ class Workload:
         self.side = None
 
     # --- CUDA-graph mode: the step's calls read the Adam constants from device memory -------
-    def enable_graph(self):
+    def enable_graph(self, dynamic=False, max_steps=0):
         torch, lz = self.torch, self.lz
         dev = self.cur[0].device
+        self.dynamic = dynamic
         self.d_consts = torch.empty(40, dtype=torch.uint8, device=dev)
         self.h_consts = [torch.empty(40, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
         self.h_done = [None, None]
         self.g_status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.g_flags = torch.zeros(1, dtype=torch.int32, device=dev)
         a, b = self.cur, self.nxt
+        if dynamic:
+            n_tab = max_steps + 2
+            tab = lz.zero_adam_consts_table(self.hp, 1, n_tab)
+            self.d_table = torch.frombuffer(bytearray(bytes(tab)), dtype=torch.uint8).to(dev)
+            self.n_tab = n_tab
+            init = lz.ScalerState(self.hp.loss_scale, 0, 1, 0)
+            self.d_scaler0 = torch.frombuffer(bytearray(bytes(init)), dtype=torch.uint8).to(dev)
+            self.d_scaler = self.d_scaler0.clone()
+            self.scaler_prm = lz.ScalerParams(2.0, 0.5, 2000)
 
         def body(src, dst):
-            self.g_status.zero_()
+            if dynamic:
+                lz.zero_scaler_prepare(self.d_scaler, self.d_table, self.n_tab, self.d_consts,
+                                       self.g_status)
+            else:
+                self.g_status.zero_()
             for lo, hi in self.ranges:
                 lz.zero_step_fused_dc(hi - lo, self.nd, [g[lo:hi] for g in self.grads],
                                       *[x[lo:hi] for x in src], *[x[lo:hi] for x in dst],
                                       self.params[lo:hi], self.d_consts, self.g_status)
             lz.zero_step_commit(self.n, *src, *dst, self.params, self.g_status)
+            if dynamic:
+                lz.zero_scaler_update(self.d_scaler, self.scaler_prm, self.g_status)
             self.g_flags.bitwise_or_(self.g_status)
 
         self._load_consts(1)
@@ -181,6 +200,8 @@ class Workload:
                 body(src, dst)
             self.graphs.append(g)
         self.g_flags.zero_()
+        if dynamic:
+            self.d_scaler.copy_(self.d_scaler0)
         self.graph_dir = 0
         self.step = self._graph_step
 
@@ -200,7 +221,8 @@ class Workload:
     def _graph_step(self, t, status, ev=None, grads=None):
         if grads is not None:
             raise ValueError("graph mode has no host-buffer variant")
-        self._load_consts(t)
+        if not self.dynamic:   # with the device scaler, the graph picks t's constants itself
+            self._load_consts(t)
         if ev is not None:
             ev[0].record()
         self.graphs[self.graph_dir].replay()
@@ -491,10 +513,12 @@ def run_ours(args):
     from zero_partitioned_optimizer_plan_b200 import libzero as lz
 
     wl = Workload(args, dev)
+    if args.dynamic_scale and not args.graph:
+        raise SystemExit("--dynamic-scale needs --graph")
     if args.graph:
         if wl.grads is None:
             raise SystemExit("--graph applies to the stage-1 and flat workloads")
-        wl.enable_graph()
+        wl.enable_graph(dynamic=args.dynamic_scale, max_steps=args.steps + args.warmup + 4)
     K, W = args.steps, args.warmup
     status = torch.zeros(K + W, dtype=torch.int32, device=dev)   # one status word per step
     torch.cuda.synchronize()
@@ -524,7 +548,7 @@ def run_ours(args):
         torch.cuda.synchronize()
     launches = lz.zero_kernel_launches() - launches0
     if args.graph:   # replays launch the captured kernels without the host library
-        launches = K * (len(wl.ranges) + 1)
+        launches = K * (len(wl.ranges) + 1 + (2 if args.dynamic_scale else 0))
         if int(wl.g_flags.item()) != 0:
             raise RuntimeError(f"unexpected status flags in the timed steps: {wl.g_flags.item()}")
     barrier()
@@ -601,6 +625,8 @@ def run_ours(args):
         cfg = dict(wl.config)
         if args.graph:
             cfg["cuda_graph"] = "one replay per step; kernel time includes the commit"
+            if args.dynamic_scale:
+                cfg["loss_scale"] = "dynamic, on the device (scaler kernels inside the graph)"
         cfg.update({"l2": "no flush: every step streams several GB, far above L2",
                     "bytes_per_step": wl.bytes_per_step, "parallelism": f"replicas{ws}",
                     "hbm_gbs": wl.bytes_per_step / (ms_per_step / 1e3) / 1e9})
