@@ -580,8 +580,10 @@ def run_ours(args):
                              "frac": wl.side["bytes"] / side_s / 1e9 / peak,
                              "ms_per_step": side_s * 1e3}
 
-    # end to end through the public API with host buffers: H2D of the step's gradients from
-    # pinned memory, the step, D2H of the updated fp16 parameters and the status word
+    # end to end through the public API with host buffers: every step uploads its gradients
+    # from pinned host memory, runs, and downloads the updated fp16 parameters and its status
+    # word, which the host reads. The upload of step i+1 overlaps step i's compute and download
+    # (double-buffered device gradients; copies on their own streams, ordered by events).
     e2e = None
     if not args.no_e2e and wl.grads is not None and not args.graph:
         E = args.e2e_steps or max(3, min(K, 10))
@@ -589,29 +591,57 @@ def run_ours(args):
                    for g in wl.grads]
         for h, g in zip(h_grads, wl.grads):
             h.copy_(g)
-        h_params = torch.empty(wl.params.numel(), dtype=torch.float16, pin_memory=True)
-        h_status = torch.empty(1, dtype=torch.int32, pin_memory=True)
-        d_grads = [torch.empty_like(g) for g in wl.grads]
+        h_params = [torch.empty(wl.params.numel(), dtype=torch.float16, pin_memory=True)
+                    for _ in range(2)]
+        h_status = [torch.empty(1, dtype=torch.int32, pin_memory=True) for _ in range(2)]
+        d_grads = [[torch.empty_like(g) for g in wl.grads] for _ in range(2)]
         st = torch.zeros(E, dtype=torch.int32, device=dev)
+        main = torch.cuda.current_stream()
+        up, down = torch.cuda.Stream(), torch.cuda.Stream()
+        ev = lambda: torch.cuda.Event()   # noqa: E731
+        up_done, comp_done, down_done = [None, None], [None, None], [None, None]
         torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for i in range(E):
-            for d, h in zip(d_grads, h_grads):
-                d.copy_(h, non_blocking=True)
-            wl.step(W + K + i + 1, st[i:i + 1], grads=d_grads)
-            h_params.copy_(wl.params, non_blocking=True)
-            h_status.copy_(st[i:i + 1], non_blocking=True)
-            torch.cuda.current_stream().synchronize()      # the caller reads the result
-            if int(h_status.item()) != 0:
+        e0.record(main)
+        up.wait_event(e0)
+
+        def read_result(j):
+            down_done[j % 2].synchronize()            # the caller reads step j's result
+            if int(h_status[j % 2].item()) != 0:
                 raise RuntimeError("unexpected status in the end-to-end steps")
-        e1.record()
+
+        for i in range(E):
+            b = i % 2
+            with torch.cuda.stream(up):
+                if comp_done[b] is not None:
+                    up.wait_event(comp_done[b])     # step i-2 is done with these buffers
+                for d, h in zip(d_grads[b], h_grads):
+                    d.copy_(h, non_blocking=True)
+                up_done[b] = ev()
+                up_done[b].record(up)
+            main.wait_event(up_done[b])
+            if down_done[1 - b] is not None:
+                main.wait_event(down_done[1 - b])   # step i-1's parameters are downloaded
+            wl.step(W + K + i + 1, st[i:i + 1], grads=d_grads[b])
+            comp_done[b] = ev()
+            comp_done[b].record(main)
+            with torch.cuda.stream(down):
+                down.wait_event(comp_done[b])
+                h_params[b].copy_(wl.params, non_blocking=True)
+                h_status[b].copy_(st[i:i + 1], non_blocking=True)
+                down_done[b] = ev()
+                down_done[b].record(down)
+            if i > 0:
+                read_result(i - 1)
+        main.wait_event(down_done[(E - 1) % 2])
+        e1.record(main)
+        read_result(E - 1)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), ws, dev)
         e2e = {"value": aggregate_rate(ws, wl.n, E, ems), "unit": "params/s",
                "h2d_bytes_per_step": 2 * wl.nd * wl.n, "d2h_bytes_per_step": 2 * wl.n + 4,
-               "steps": E}
+               "steps": E, "overlap": "upload of step i+1 overlaps compute and download of step i"}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
