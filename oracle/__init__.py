@@ -65,6 +65,9 @@ def bind(path: str):
     L.orc_adam.argtypes = [u64, f32p, f32p, f32p, f32p, u16p, C.c_void_p]
     L.orc_step.argtypes = [u64, C.c_int, C.POINTER(u16p), f32p, f32p, f32p, u16p,
                            C.c_void_p, i64, f32p]
+    i8p = C.POINTER(C.c_int8)
+    L.orc_quant_q8.argtypes = [u64, u16p, i8p, f32p]
+    L.orc_reduce_mean_q8.argtypes = [u64, C.c_int, C.POINTER(i8p), C.POINTER(f32p), f32p]
     return L
 
 
@@ -393,3 +396,41 @@ def scaled_step(grads, master, m, v, hp: AdamHP, sc: Scaler):
     skipped, w, mm, vv, p16 = step(grads, master, m, v, hp_t, sc.next_step)
     sc.update(skipped)
     return skipped, w, mm, vv, p16
+
+
+# ---------------------------------------------------------------------------------------------
+# compressed reduce-scatter payload: int8 with one fp32 scale per block of 128 elements
+# ("ZeRO" (lastdictionary): extensions compress communication, ZeRO++; the format is this
+# library's reading, see oracle.c)
+# ---------------------------------------------------------------------------------------------
+QB = 128
+
+
+def quant_q8(g):
+    """A rank's fp16 slice -> (int8 values, fp32 scale per block of 128)."""
+    g = _as_u16(g)
+    q = np.empty(g.size, np.int8)
+    sc = np.empty((g.size + QB - 1) // QB, np.float32)
+    lib().orc_quant_q8(g.size, _u16p(g), q.ctypes.data_as(C.POINTER(C.c_int8)), _f32p(sc))
+    return q, sc
+
+
+def reduce_mean_q8(qs, scales):
+    n = qs[0].size
+    qs = [np.ascontiguousarray(q, np.int8) for q in qs]
+    scales = [np.ascontiguousarray(s, np.float32) for s in scales]
+    qp = (C.POINTER(C.c_int8) * len(qs))(*[q.ctypes.data_as(C.POINTER(C.c_int8)) for q in qs])
+    sp = (C.POINTER(C.c_float) * len(qs))(*[_f32p(s) for s in scales])
+    red = np.empty(n, np.float32)
+    lib().orc_reduce_mean_q8(n, len(qs), qp, sp, _f32p(red))
+    return red
+
+
+def step_q8(qs, scales, master, m, v, hp: AdamHP, t: int):
+    """The owner's step from int8 payloads: (skipped, master, m, v, p16 or None)."""
+    red = reduce_mean_q8(qs, scales)
+    if not all_finite(red):
+        return True, np.array(master, np.float32), np.array(m, np.float32), \
+            np.array(v, np.float32), None
+    w, mm, vv, p16 = adam(red, master, m, v, hp, t)
+    return False, w, mm, vv, p16

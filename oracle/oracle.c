@@ -307,3 +307,70 @@ int orc_step(uint64_t n, int nd, const uint16_t* const* g, float* master, float*
     orc_adam(n, red_scratch, master, m, v, p16, &s);
     return 0;
 }
+
+/* ------------------------------------------------------------------------------------------
+ * Compressed reduce-scatter payload (int8 + one fp32 scale per block of 128 elements).
+ * "ZeRO" (lastdictionary), main definition: extensions compress the communication (ZeRO++).
+ * The pages give no format; the one used: for each block of ORC_QB consecutive elements of a
+ * rank's slice (the last block may be short),
+ *   amax  = max |x|                          (exact; any inf/NaN in the block poisons it)
+ *   scale = amax / 127                        (binary32 division), NaN for a poisoned block
+ *   q     = round_half_even(x / scale), clamped to [-127, 127]; 0 if scale is 0 or NaN
+ * and the owner dequantizes x' = float(q) * scale (one rounded product), sums the ranks in
+ * order 0..nd-1 and divides by nd, exactly as for fp16 slices.
+ * ---------------------------------------------------------------------------------------- */
+#define ORC_QB 128
+
+static int finite_f32(float x) { return ((bits_of(x) >> 23) & 0xffu) != 0xffu; }
+
+/* nearest integer to x, ties to even, for |x| < 2^23 */
+static float rint_even(float x)
+{
+    float a = x < 0 ? -x : x;
+    float f = (float)(int32_t)a;          /* truncation toward zero, exact */
+    float r = a - f;                      /* exact: the fraction */
+    if (r > 0.5f || (r == 0.5f && ((int32_t)f & 1))) f = f + 1.0f;
+    return x < 0 ? -f : f;
+}
+
+void orc_quant_q8(uint64_t n, const uint16_t* g, int8_t* q, float* scales)
+{
+    for (uint64_t b0 = 0; b0 < n; b0 += ORC_QB) {
+        uint64_t b1 = b0 + ORC_QB < n ? b0 + ORC_QB : n;
+        float amax = 0.0f;
+        int poisoned = 0;
+        for (uint64_t i = b0; i < b1; i++) {
+            float x = orc_h2f(g[i]);
+            if (!finite_f32(x)) poisoned = 1;
+            else {
+                float a = x < 0 ? -x : x;
+                if (a > amax) amax = a;
+            }
+        }
+        float scale = poisoned ? float_of(0x7fc00000u) : amax / 127.0f;
+        scales[b0 / ORC_QB] = scale;
+        for (uint64_t i = b0; i < b1; i++) {
+            if (poisoned || scale == 0.0f) { q[i] = 0; continue; }
+            float k = rint_even(orc_h2f(g[i]) / scale);
+            if (k > 127.0f) k = 127.0f;
+            if (k < -127.0f) k = -127.0f;
+            q[i] = (int8_t)k;
+        }
+    }
+}
+
+/* The owner's reduced gradient from nd int8 payloads (q[r], scales[r] cover the same n
+ * elements, blocks counted from element 0). */
+void orc_reduce_mean_q8(uint64_t n, int nd, const int8_t* const* q, const float* const* scales,
+                        float* red)
+{
+    float fnd = (float)nd;
+    for (uint64_t i = 0; i < n; i++) {
+        float s = 0.0f;
+        for (int r = 0; r < nd; r++) {
+            float x = (float)q[r][i] * scales[r][i / ORC_QB];
+            s = s + x;
+        }
+        red[i] = s / fnd;
+    }
+}

@@ -36,7 +36,8 @@ C_MUTANTS = [
      "float v_new = s->omb2 * g;", ["adam_textbook"]),
     ("ranks summed in reverse order", "for (int r = 0; r < nd; r++) s = s + orc_h2f(g[r][i]);",
      "for (int r = nd - 1; r >= 0; r--) s = s + orc_h2f(g[r][i]);", ["sum_order"]),
-    ("sum, not mean", "red[i] = s / fnd;", "red[i] = s;", ["exact_sums"]),
+    ("sum, not mean", "s = s + orc_h2f(g[r][i]);\n        red[i] = s / fnd;",
+     "s = s + orc_h2f(g[r][i]);\n        red[i] = s;", ["exact_sums"]),
     ("ties rounded away from zero in the fp16 cast",
      "if (rem > half || (rem == half && (n & 1u))) n += 1u;", "if (rem >= half) n += 1u;",
      ["f2h_mid"]),
@@ -46,6 +47,13 @@ C_MUTANTS = [
      ["memory"]),
     ("overflow check ignores NaN", "if (((u >> 23) & 0xffu) == 0xffu) return 0;",
      "if (u == 0x7f800000u || u == 0xff800000u) return 0;", ["overflow_nan"]),
+    ("payload scale divides by 128", "float scale = poisoned ? float_of(0x7fc00000u) : amax / 127.0f;",
+     "float scale = poisoned ? float_of(0x7fc00000u) : amax / 128.0f;", ["q8_bf"]),
+    ("payload ties rounded away from zero",
+     "if (r > 0.5f || (r == 0.5f && ((int32_t)f & 1))) f = f + 1.0f;",
+     "if (r >= 0.5f) f = f + 1.0f;", ["q8_ties"]),
+    ("payload scale of the wrong block", "float x = (float)q[r][i] * scales[r][i / ORC_QB];",
+     "float x = (float)q[r][i] * scales[r][(i + 1) / ORC_QB];", ["q8_red"]),
 ]
 
 PINS = {
@@ -58,6 +66,9 @@ PINS = {
     "plan_bf": lambda: [pins.test_plan_brute_force(s) for s in range(20)],
     "memory": pins.test_memory_figures_of_the_7p5b_example,
     "overflow_nan": lambda: pins.test_overflow_skips_whole_step(0x7e00),
+    "q8_bf": lambda: pins.test_quant_q8_brute_force(0),
+    "q8_ties": pins.test_quant_q8_ties_go_to_even,
+    "q8_red": lambda: pins.test_reduce_mean_q8_brute_force(3),
 }
 
 

@@ -500,3 +500,90 @@ def test_scaled_step_unscales_by_the_current_scale():
     sc = oracle.Scaler(scale=1024.0)
     skipped, *_ = oracle.scaled_step([bad], master, z, z, HP, sc)
     assert skipped and sc.next_step == 1 and sc.scale == 512.0 and sc.skipped_steps == 1
+
+
+# ---------------------------------------------------------------------------------------------
+# compressed payload: int8 + one fp32 scale per block of 128
+# ---------------------------------------------------------------------------------------------
+def _rint_half_even(fr: Fraction) -> int:
+    n = fr.numerator // fr.denominator
+    rem = fr - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return n
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_quant_q8_brute_force(seed):
+    # every q from the definition with exact rationals: scale = fl(amax / 127),
+    # q = half-even integer of fl(x / scale), clamped; blocks of 128 from element 0
+    rng = np.random.default_rng(200 + seed)
+    n = 128 * 3 + 37
+    g = (rng.standard_normal(n) * 10.0 ** rng.uniform(-4, 1)).astype(np.float16)
+    g[128:256] = 0                                    # a zero block
+    q, sc = oracle.quant_q8(g)
+    assert sc.size == 4
+    for b in range(4):
+        blk = g[128 * b:128 * (b + 1)].astype(np.float64)
+        amax = Fraction(float(np.max(np.abs(blk))))
+        scale = round_f32(amax / 127)
+        assert sc[b] == scale
+        for j, x in enumerate(blk):
+            i = 128 * b + j
+            if scale == 0:
+                assert q[i] == 0
+                continue
+            k = _rint_half_even(frac(round_f32(Fraction(float(x)) / frac(scale))))
+            assert q[i] == max(-127, min(127, k)), (i, x, q[i], k)
+
+
+def test_quant_q8_grid_values_round_trip_exactly():
+    # values k * 2^-7 with max |k| = 127: scale is exactly 2^-7 and every q is exactly k
+    rng = np.random.default_rng(7)
+    k = rng.integers(-127, 128, size=256)
+    k[0], k[128] = 127, -127
+    x = (k * 2.0 ** -7).astype(np.float16)
+    q, sc = oracle.quant_q8(x)
+    assert np.all(sc == np.float32(2.0 ** -7)) and np.array_equal(q.astype(np.int64), k)
+
+
+def test_quant_q8_ties_go_to_even():
+    x = np.zeros(128, np.float16)
+    x[0] = 127 * 2.0 ** -7                        # scale 2^-7
+    x[1], x[2], x[3], x[4] = 2.5 * 2.0 ** -7, 3.5 * 2.0 ** -7, -2.5 * 2.0 ** -7, 0.5 * 2.0 ** -7
+    q, _ = oracle.quant_q8(x)
+    assert list(q[:5]) == [127, 2, 4, -2, 0]
+
+
+def test_quant_q8_poisoned_block_skips_the_step():
+    rng = np.random.default_rng(8)
+    g = [(rng.standard_normal(300) * 1e-2).astype(np.float16) for _ in range(3)]
+    g[1][200] = np.float16(np.inf)
+    qs, scs = zip(*[oracle.quant_q8(x) for x in g])
+    assert np.isnan(scs[1][1]) and not np.isnan(scs[1][0]) and not scs[1][1:2].size == 0
+    assert not qs[1][128:256].any()
+    master = rng.standard_normal(300).astype(np.float32)
+    z = np.zeros(300, np.float32)
+    skipped, w, *_ = oracle.step_q8(qs, scs, master, z, z, HP, 1)
+    assert skipped and np.array_equal(w, master)
+
+
+@pytest.mark.parametrize("nd", [1, 3, 8])
+def test_reduce_mean_q8_brute_force(nd):
+    # dequantize (one rounded product), add in rank order (rounded), divide once
+    rng = np.random.default_rng(300 + nd)
+    n = 128 * 2 + 5
+    g = [(rng.standard_normal(n) * 1e-2).astype(np.float16) for _ in range(nd)]
+    qs, scs = zip(*[oracle.quant_q8(x) for x in g])
+    red = oracle.reduce_mean_q8(qs, scs)
+    for i in range(n):
+        s = Fraction(0)
+        for r in range(nd):
+            prod = frac(round_f32(Fraction(int(qs[r][i])) * frac(scs[r][i // 128])))
+            s = frac(round_f32(s + prod))
+        assert red[i] == round_f32(s / nd)
+    # and the payload is close to the fp16 gradients it stands for (half a step per element)
+    for r in range(nd):
+        deq = qs[r].astype(np.float64) * np.repeat(scs[r].astype(np.float64), 128)[:n]
+        err = np.abs(deq - g[r].astype(np.float64))
+        assert np.all(err <= 0.5 * np.repeat(scs[r], 128)[:n] * (1 + 2.0 ** -20) + 1e-30)

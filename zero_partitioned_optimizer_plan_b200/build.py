@@ -40,7 +40,8 @@ def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = _sources() + glob.glob(os.path.join(CSRC, "*.h")) + [HEADER, __file__]
+    deps = _sources() + glob.glob(os.path.join(CSRC, "*.h")) + \
+        glob.glob(os.path.join(CSRC, "*.cuh")) + [HEADER, __file__]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
