@@ -63,6 +63,9 @@ def parse():
     ap.add_argument("--dynamic-scale", action="store_true",
                     help="with --graph: dynamic loss scaling on the device (scaler prepare and "
                          "update kernels in the graph, no host work per step)")
+    ap.add_argument("--payload", choices=["fp16", "q8"], default="fp16",
+                    help="q8: the owner reduces int8 payloads with one fp32 scale per 128 "
+                         "elements (quantized once per rank before timing)")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -149,6 +152,42 @@ class Workload:
         self.dominant_bytes = self.bytes_per_step
         self.dominant_calls = len(self.ranges)
         self.side = None
+        self.payload = args.payload
+        if self.payload == "q8":
+            self._quantize_payload()
+
+    def _quantize_payload(self):
+        """Each rank's gradients as int8 + one fp32 scale per 128 (the senders' work, done once
+        before timing and timed on its own)."""
+        torch, lz = self.torch, self.lz
+        if len(self.ranges) != 1:
+            raise SystemExit("--payload q8 takes one call per step (no --bucket)")
+        n, nd = self.n, self.nd
+        nb = (n + 127) // 128
+        self.q = [torch.empty(n, dtype=torch.int8, device=self.dev) for _ in range(nd)]
+        self.scales = [torch.empty(nb, dtype=torch.float32, device=self.dev) for _ in range(nd)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for g, q, sc in zip(self.grads, self.q, self.scales):
+            lz.zero_quantize_q8(n, g, q, sc)
+        e1.record()
+        torch.cuda.synchronize()
+        qbytes = nd * (2 * n + n + 4 * nb)
+        self.side = {"kernel": "quant_q8_kernel (senders, once)", "bytes": qbytes,
+                     "calls": nd, "ms": [(e0, e1)]}
+        self.grads = None
+        torch.cuda.empty_cache()
+        self.bytes_per_step = nd * (n + 4 * nb) + 26 * n
+        self.dominant = "fused_q8_tma_kernel"
+        self.dominant_bytes = self.bytes_per_step
+        self.config["payload"] = "int8, one fp32 scale per 128 elements"
+        self.config["workload"] += "_q8"
+
+    def inputs(self):
+        """The tensors a step consumes that a host would have to upload."""
+        if self.payload == "q8":
+            return self.q + self.scales
+        return self.grads
 
     # --- CUDA-graph mode: the step's calls read the Adam constants from device memory -------
     def enable_graph(self, dynamic=False, max_steps=0):
@@ -232,8 +271,21 @@ class Workload:
 
     def step(self, t, status, ev=None, grads=None):
         """Enqueue one step on the current stream; ev = (start, end) events around the
-        dominant kernel's launches."""
+        dominant kernel's launches. grads: the step's inputs (as inputs() lists them) when
+        they are not the workload's own buffers."""
         lz = self.lz
+        if self.payload == "q8":
+            ins = grads or self.inputs()
+            qs, scs = ins[:self.nd], ins[self.nd:]
+            if ev is not None:
+                ev[0].record()
+            lz.zero_step_fused_q8(self.n, self.nd, qs, scs, *self.cur, *self.nxt, self.params,
+                                  self.hp, t, status)
+            if ev is not None:
+                ev[1].record()
+            lz.zero_step_commit(self.n, *self.cur, *self.nxt, self.params, status)
+            self.cur, self.nxt = self.nxt, self.cur
+            return
         grads = grads or self.grads
         if ev is not None:
             ev[0].record()
@@ -255,6 +307,9 @@ def _init_zero2(self, args, dev):
     through the scheduler, then the owners' updates (zero_adam_shard)."""
     torch, lz = self.torch, self.lz
     from zero_partitioned_optimizer_plan_b200 import synth
+    if args.payload != "fp16":
+        raise SystemExit("the stage-2 workloads take fp16 payloads")
+    self.payload = "fp16"
     small = args.workload == "zero2_gpt2_small"
     nd = args.nd or (8 if small else 16)
     B = args.bucket or (10_000_000 if small else 50_000_000)
@@ -517,7 +572,7 @@ def run_ours(args):
         raise SystemExit("--dynamic-scale needs --graph")
     if args.graph:
         if wl.grads is None:
-            raise SystemExit("--graph applies to the stage-1 and flat workloads")
+            raise SystemExit("--graph applies to the fp16 stage-1 and flat workloads")
         wl.enable_graph(dynamic=args.dynamic_scale, max_steps=args.steps + args.warmup + 4)
     K, W = args.steps, args.warmup
     status = torch.zeros(K + W, dtype=torch.int32, device=dev)   # one status word per step
@@ -573,7 +628,7 @@ def run_ours(args):
                                               f"{wl.config['workload']}_nd{wl.nd}"),
                 "kernel": wl.dominant, "bytes_per_launch": bytes_per_launch,
                 "kernel_ms_mean": launch_s * 1e3}
-    if wl.side is not None:   # the other kernel of a two-kernel step
+    if wl.side is not None:   # the other kernel of the step (or the senders' quantization)
         side_s = statistics.mean(a.elapsed_time(b) for a, b in wl.side["ms"][-K:]) / 1e3
         roofline["other"] = {"kernel": wl.side["kernel"],
                              "achieved": wl.side["bytes"] / side_s / 1e9,
@@ -585,16 +640,15 @@ def run_ours(args):
     # word, which the host reads. The upload of step i+1 overlaps step i's compute and download
     # (double-buffered device gradients; copies on their own streams, ordered by events).
     e2e = None
-    if not args.no_e2e and wl.grads is not None and not args.graph:
+    if not args.no_e2e and wl.inputs() is not None and not args.graph:
         E = args.e2e_steps or max(3, min(K, 10))
-        h_grads = [torch.empty(g.numel(), dtype=torch.float16, pin_memory=True)
-                   for g in wl.grads]
-        for h, g in zip(h_grads, wl.grads):
+        h_grads = [torch.empty(g.numel(), dtype=g.dtype, pin_memory=True) for g in wl.inputs()]
+        for h, g in zip(h_grads, wl.inputs()):
             h.copy_(g)
         h_params = [torch.empty(wl.params.numel(), dtype=torch.float16, pin_memory=True)
                     for _ in range(2)]
         h_status = [torch.empty(1, dtype=torch.int32, pin_memory=True) for _ in range(2)]
-        d_grads = [[torch.empty_like(g) for g in wl.grads] for _ in range(2)]
+        d_grads = [[torch.empty_like(g) for g in wl.inputs()] for _ in range(2)]
         st = torch.zeros(E, dtype=torch.int32, device=dev)
         main = torch.cuda.current_stream()
         up, down = torch.cuda.Stream(), torch.cuda.Stream()
@@ -640,7 +694,8 @@ def run_ours(args):
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), ws, dev)
         e2e = {"value": aggregate_rate(ws, wl.n, E, ems), "unit": "params/s",
-               "h2d_bytes_per_step": 2 * wl.nd * wl.n, "d2h_bytes_per_step": 2 * wl.n + 4,
+               "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h in h_grads),
+               "d2h_bytes_per_step": 2 * wl.n + 4,
                "steps": E, "overlap": "upload of step i+1 overlaps compute and download of step i"}
 
     cpu = None

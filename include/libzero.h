@@ -298,6 +298,34 @@ zero_status zero_step_commit(uint64_t n, const float* master_in, const float* m_
  * set or the copy fails, else ZERO_OK. This is the only call that blocks the host. */
 zero_status zero_step_status(const uint32_t* d_status, zero_stream_t stream, uint32_t* flags_out);
 
+/* ------------------------------------------------------------------------------------------
+ * Compressed reduce-scatter payload. "ZeRO" (lastdictionary.com), main definition: extensions
+ * compress the communication (ZeRO++). The pages give no format; this library's: each rank's
+ * slice travels as int8 values with one fp32 scale per block of ZERO_Q8_BLOCK elements
+ * (blocks counted from the slice's first element):
+ *   scale = amax/127 (binary32), q = round_half_even(x/scale) clamped to [-127, 127],
+ *   a block with an inf or NaN gets scale NaN and q = 0 (so the owner sees the overflow).
+ * ---------------------------------------------------------------------------------------- */
+#define ZERO_Q8_BLOCK 128
+
+/* Quantize one rank's n fp16 gradients: q[n] (any alignment), scales[ceil(n/128)] (4-byte
+ * aligned), all device memory. Errors: ZERO_EINVAL (null, overlap), ZERO_EALIGN, ZERO_ECUDA. */
+zero_status zero_quantize_q8(uint64_t n, const uint16_t* grad, int8_t* q, float* scales,
+                             zero_stream_t stream);
+
+/* zero_step_fused with int8 payloads: red = (sum_{r=0..nd-1} float(q_r[i]) * scale_r[i/128])/nd,
+ * each product and sum an IEEE binary32 operation, then the same update, overflow flag and
+ * commit protocol as zero_step_fused. rank_q / rank_scales: nd device pointers each (host
+ * arrays) to this range's n values and ceil(n/128) scales, as zero_quantize_q8 wrote them.
+ * 16-byte aligned payload and state pointers (and n >= 4096) take the bulk-copy kernel.
+ * Errors: as zero_step_fused. */
+zero_status zero_step_fused_q8(uint64_t n, int nd, const int8_t* const* rank_q,
+                               const float* const* rank_scales, const float* master_in,
+                               const float* m_in, const float* v_in, float* master_out,
+                               float* m_out, float* v_out, uint16_t* param_out,
+                               const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
+                               zero_stream_t stream);
+
 /* Self-test of the kernels' bounded waits (failure detection without a fault): launches the
  * fused pipeline on one tile with its copy-issuing warp switched off, so every consumer's wait
  * on shared-memory data expires after about one second; the kernel then sets

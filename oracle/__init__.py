@@ -68,6 +68,7 @@ def bind(path: str):
     i8p = C.POINTER(C.c_int8)
     L.orc_quant_q8.argtypes = [u64, u16p, i8p, f32p]
     L.orc_reduce_mean_q8.argtypes = [u64, C.c_int, C.POINTER(i8p), C.POINTER(f32p), f32p]
+    L.orc_reduce_mean_q8_gathered.argtypes = [u64, C.c_int, C.POINTER(i8p), C.POINTER(f32p), f32p]
     return L
 
 
@@ -429,6 +430,22 @@ def reduce_mean_q8(qs, scales):
 def step_q8(qs, scales, master, m, v, hp: AdamHP, t: int):
     """The owner's step from int8 payloads: (skipped, master, m, v, p16 or None)."""
     red = reduce_mean_q8(qs, scales)
+    if not all_finite(red):
+        return True, np.array(master, np.float32), np.array(m, np.float32), \
+            np.array(v, np.float32), None
+    w, mm, vv, p16 = adam(red, master, m, v, hp, t)
+    return False, w, mm, vv, p16
+
+
+def step_q8_gathered(qs, scale_of_elem, master, m, v, hp: AdamHP, t: int):
+    """step_q8 on gathered samples: scale_of_elem[r][i] is the scale of sample i's block."""
+    n = qs[0].size
+    qs = [np.ascontiguousarray(q, np.int8) for q in qs]
+    sc = [np.ascontiguousarray(s, np.float32) for s in scale_of_elem]
+    qp = (C.POINTER(C.c_int8) * len(qs))(*[q.ctypes.data_as(C.POINTER(C.c_int8)) for q in qs])
+    sp = (C.POINTER(C.c_float) * len(qs))(*[_f32p(s) for s in sc])
+    red = np.empty(n, np.float32)
+    lib().orc_reduce_mean_q8_gathered(n, len(qs), qp, sp, _f32p(red))
     if not all_finite(red):
         return True, np.array(master, np.float32), np.array(m, np.float32), \
             np.array(v, np.float32), None

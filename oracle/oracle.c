@@ -374,3 +374,18 @@ void orc_reduce_mean_q8(uint64_t n, int nd, const int8_t* const* q, const float*
         red[i] = s / fnd;
     }
 }
+
+/* The same reduction on gathered samples: scale[r][i] is the scale of sample i's block. */
+void orc_reduce_mean_q8_gathered(uint64_t n, int nd, const int8_t* const* q,
+                                 const float* const* scale, float* red)
+{
+    float fnd = (float)nd;
+    for (uint64_t i = 0; i < n; i++) {
+        float s = 0.0f;
+        for (int r = 0; r < nd; r++) {
+            float x = (float)q[r][i] * scale[r][i];
+            s = s + x;
+        }
+        red[i] = s / fnd;
+    }
+}

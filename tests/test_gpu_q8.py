@@ -1,0 +1,168 @@
+"""The compressed (int8 + per-128 fp32 scale) reduce-scatter payload on the GPU against the
+oracle: the quantizer bit for bit, the owner's fused step from the payload within the usual
+tolerances (fp32 state 2 ulp, fp16 params 1 ulp), overflow carried through a poisoned block,
+unaligned fallbacks, and the 7.5B shard view at Nd = 64 on sampled elements."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests._gpu import (DEV, HP, ORC_HP, PingPong, check_f16, check_f32, f16np, f32np, lz,
+                        require_gpu, status_flags, status_word)
+from zero_partitioned_optimizer_plan_b200 import synth
+
+pytestmark = pytest.mark.gpu
+QB = 128
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    require_gpu()
+    torch.cuda.set_device(0)
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def _quant_dev(g_dev, q_off=0):
+    n = g_dev.numel()
+    qbig = torch.zeros(n + 16, dtype=torch.int8, device=DEV)
+    q = qbig[q_off:q_off + n]
+    sc = torch.empty((n + QB - 1) // QB, dtype=torch.float32, device=DEV)
+    lz.zero_quantize_q8(n, g_dev, q, sc)
+    return q, sc
+
+
+def _same_scales(a, b):
+    return np.array_equal(np.isnan(a), np.isnan(b)) and \
+        np.array_equal(a[~np.isnan(a)].view(np.uint32), b[~np.isnan(b)].view(np.uint32))
+
+
+@pytest.mark.parametrize("n", [1, 127, 128, 129, 4096 + 77, 300_005])
+@pytest.mark.parametrize("kind", ["normal", "zeros", "poisoned", "unaligned"])
+def test_quantize_bit_exact(n, kind):
+    rng_seed = n + len(kind)
+    g = synth.grad_f16(n, 1e-2, seed=rng_seed)
+    if kind == "zeros":
+        g[: min(n, 300)] = 0
+    if kind == "poisoned":
+        g[n // 2] = float("nan")
+        g[0] = float("-inf")
+    goff = 1 if kind == "unaligned" else 0
+    gbig = torch.zeros(n + 8, dtype=torch.float16, device=DEV)
+    gbig[goff:goff + n] = g.to(DEV)
+    q, sc = _quant_dev(gbig[goff:goff + n], q_off=1 if kind == "unaligned" else 0)
+    torch.cuda.synchronize()
+    q_ref, sc_ref = oracle.quant_q8(g.numpy())
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert _same_scales(sc.cpu().numpy(), sc_ref)
+
+
+@pytest.mark.parametrize("nd", [1, 2, 3, 8, 16, 25, 64])
+@pytest.mark.parametrize("n", [9, 4096, 4096 + 300, 2048 * 40 + 777])
+def test_fused_q8_vs_oracle(n, nd):
+    seed = 7 * n + nd
+    master, m, v = synth.state_warm(n, seed=seed)
+    pp = PingPong(master, m, v)
+    w_r, m_r, v_r = master.numpy(), m.numpy(), v.numpy()
+    params = torch.empty(n, dtype=torch.float16, device=DEV)
+    for t in (1, 2):
+        g_cpu = [synth.grad_f16(n, 1e-2, seed=seed, rank=r, step=t) for r in range(nd)]
+        pay = [_quant_dev(g.to(DEV)) for g in g_cpu]
+        st = status_word()
+        ins, outs = pp.cur, pp.nxt
+        lz.zero_step_fused_q8(n, nd, [q for q, _ in pay], [s for _, s in pay], *ins, *outs,
+                              params, HP, t, st)
+        lz.zero_step_commit(n, *ins, *outs, params, st)
+        torch.cuda.synchronize()
+        assert status_flags(st) == 0
+        pp.swap()
+        ref_pay = [oracle.quant_q8(g.numpy()) for g in g_cpu]      # the oracle's own payload
+        skipped, w_r, m_r, v_r, p_r = oracle.step_q8([q for q, _ in ref_pay],
+                                                     [s for _, s in ref_pay], w_r, m_r, v_r,
+                                                     ORC_HP, t)
+        assert not skipped
+        w, mm, vv = pp.numpy()
+        check_f32("master", w, w_r)
+        check_f32("m", mm, m_r)
+        check_f32("v", vv, v_r)
+        check_f16("params", f16np(params), p_r)
+
+
+def test_fused_q8_overflow_through_poisoned_block():
+    n, nd = 2048 * 9 + 3, 4
+    master, m, v = synth.state_warm(n, seed=5)
+    pp = PingPong(master, m, v)
+    g_dev = [synth.grad_f16(n, 1e-2, seed=6, rank=r).to(DEV) for r in range(nd)]
+    g_dev[2][5000] = float("inf")
+    pay = [_quant_dev(g) for g in g_dev]
+    params = torch.zeros(n, dtype=torch.float16, device=DEV)
+    st = status_word()
+    lz.zero_step_fused_q8(n, nd, [q for q, _ in pay], [s for _, s in pay], *pp.cur, *pp.nxt,
+                          params, HP, 1, st)
+    lz.zero_step_commit(n, *pp.cur, *pp.nxt, params, st)
+    assert lz.zero_step_status(st)[0] == lz.ZERO_STEP_SKIPPED
+    for a, b in zip(pp.cur, pp.nxt):
+        assert torch.equal(a, b)
+    assert np.array_equal(f16np(params), oracle.f2h(master.numpy()))
+
+
+def test_fused_q8_unaligned_payload_takes_plain_kernel():
+    n, nd = 50_000, 3
+    master, m, v = synth.state_warm(n, seed=8)
+    pp = PingPong(master, m, v)
+    g_cpu = [synth.grad_f16(n, 1e-2, seed=9, rank=r) for r in range(nd)]
+    pay = [_quant_dev(g.to(DEV), q_off=3) for g in g_cpu]
+    params = torch.empty(n, dtype=torch.float16, device=DEV)
+    st = status_word()
+    lz.zero_step_fused_q8(n, nd, [q for q, _ in pay], [s for _, s in pay], *pp.cur, *pp.nxt,
+                          params, HP, 1, st)
+    torch.cuda.synchronize()
+    assert status_flags(st) == 0
+    ref = [oracle.quant_q8(g.numpy()) for g in g_cpu]
+    skipped, w, mm, vv, p = oracle.step_q8([q for q, _ in ref], [s for _, s in ref],
+                                           master.numpy(), m.numpy(), v.numpy(), ORC_HP, 1)
+    check_f32("master", f32np(pp.nxt[0]), w)
+    check_f16("params", f16np(params), p)
+
+
+def test_7p5b_shard_view_q8_sampled():
+    """Owner 63 of 7.5e9 parameters at Nd = 64 from int8 payloads, in the bench's launch
+    configuration; sampled elements against the oracle on the gathered payload."""
+    total, nd = 7_500_000_000, 64
+    S = total // nd
+    owner = 63
+    full = torch.zeros(total, dtype=torch.float16, device=DEV)
+    qs, scs = [], []
+    g = torch.empty(S, dtype=torch.float16, device=DEV)
+    for r in range(nd):
+        synth.grad_f16(S, 1e-3, seed=11, rank=r, out=g)
+        q = torch.empty(S, dtype=torch.int8, device=DEV)
+        sc = torch.empty((S + QB - 1) // QB, dtype=torch.float32, device=DEV)
+        lz.zero_quantize_q8(S, g, q, sc)
+        qs.append(q)
+        scs.append(sc)
+    del g
+    cur = list(synth.state_warm(S, seed=12, device=DEV))
+    nxt = [torch.empty_like(x) for x in cur]
+    rng = np.random.default_rng(13)
+    idx = np.unique(np.concatenate([rng.integers(0, S, 100_000), np.arange(S - 600, S),
+                                    np.arange(0, 256)]))
+    idx_dev = torch.from_numpy(idx).to(DEV)
+    bidx_dev = torch.from_numpy(idx // QB).to(DEV)
+    w0, m0, v0 = (x[idx_dev].cpu().numpy() for x in cur)
+    out = full[owner * S:(owner + 1) * S]
+    st = status_word()
+    lz.zero_step_fused_q8(S, nd, qs, scs, *cur, *nxt, out, HP, 1, st)
+    lz.zero_step_commit(S, *cur, *nxt, out, st)
+    torch.cuda.synchronize()
+    assert status_flags(st) == 0
+    gq = [q[idx_dev].cpu().numpy() for q in qs]
+    gs = [s[bidx_dev].cpu().numpy() for s in scs]
+    skipped, w, mm, vv, p = oracle.step_q8_gathered(gq, gs, w0, m0, v0, ORC_HP, 1)
+    assert not skipped
+    check_f32("master", nxt[0][idx_dev].cpu().numpy(), w)
+    check_f32("m", nxt[1][idx_dev].cpu().numpy(), mm)
+    check_f32("v", nxt[2][idx_dev].cpu().numpy(), vv)
+    check_f16("params", out[idx_dev].cpu().numpy().view(np.uint16), p)
+    assert int(torch.count_nonzero(full[:owner * S].view(torch.int16))) == 0

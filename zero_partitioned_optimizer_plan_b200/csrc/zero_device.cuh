@@ -448,5 +448,21 @@ unsigned plain_grid(uint64_t n, int sms, int per_sm = 8) {
     return (unsigned)(blocks ? blocks : 1);
 }
 
+// Consumer warps and stage split per Nd, measured on B200 (HBM GB/s of the fused step over
+// geometries with 4 elements per thread): few ranks need more warps to hide the latency of the
+// Adam arithmetic; many ranks need large stages so that a tile takes few chunks.
+struct Variant {
+    int warps;
+    int target_stages;
+};
+
+Variant pick_variant(int nd) {
+    if (nd <= 2) return {20, 2};
+    if (nd <= 4) return {16, 2};
+    if (nd <= 8) return {24, 3};
+    if (nd <= 16) return {16, 2};
+    return {20, 2};
+}
+
 }  // namespace
 }  // namespace zk

@@ -493,22 +493,6 @@ __global__ void scaler_update_kernel(zero_scaler_state* st, zero_scaler_params p
 std::atomic<uint64_t> g_launches{0};
 
 
-// Consumer warps and stage split per Nd, measured on B200 (HBM GB/s of the fused step over
-// geometries with 4 elements per thread): few ranks need more warps to hide the latency of the
-// Adam arithmetic; many ranks need large stages so that a tile takes few chunks.
-struct Variant {
-    int warps;
-    int target_stages;
-};
-
-Variant pick_variant(int nd) {
-    if (nd <= 2) return {20, 2};
-    if (nd <= 4) return {16, 2};
-    if (nd <= 8) return {24, 3};
-    if (nd <= 16) return {16, 2};
-    return {20, 2};
-}
-
 // Tile = 32 * warps * kElems elements; as many rank rows per stage as leave target_stages
 // stages inside the shared-memory budget, the ranks split evenly into chunks.
 PipeShape pipe_shape(int nd, bool with_state) {

@@ -1,0 +1,383 @@
+// Compressed reduce-scatter payload for sm_100a: int8 values with one fp32 scale per block of
+// 128 elements ("ZeRO" (lastdictionary.com), main definition: extensions compress the
+// communication, ZeRO++; the pages give no format, this is the library's).
+//
+//   quantize (each sending rank, on its own slice):
+//     amax  = max |x| over the block (any inf/NaN poisons the block: scale NaN, q 0)
+//     scale = amax / 127                      (IEEE binary32 division)
+//     q     = round_half_even(x / scale), clamped to [-127, 127]; 0 when scale is 0
+//   owner's fused step:
+//     red = (sum_{r=0..nd-1} float(q_r) * scale_r) / nd      (each product and sum rounded)
+//     then the same unscale, Adam, fp16 cast and write-back as the fp16 fused step.
+//
+// Per parameter the owner reads nd * (1 + 4/128) payload bytes instead of 2 * nd: at Nd = 64 the
+// fused step moves 92 bytes per parameter instead of 154.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "zero_device.cuh"
+#include "zero_internal.h"
+
+namespace zk {
+
+namespace {
+
+constexpr int kQB = 128;                 // elements per scale block
+constexpr uint64_t kQTileAlign = 512;    // tiles cover a multiple of 512 elements (16-byte rows)
+
+struct QuantArgs {
+    const uint16_t* g;
+    int8_t* q;
+    float* scales;
+    uint64_t n;
+    int vec;   // g 8-byte and q 4-byte aligned: 4 elements per lane in one load and one store
+};
+
+// One warp per block of 128: lane l holds elements 4l .. 4l+3.
+__global__ void __launch_bounds__(256) quant_q8_kernel(const __grid_constant__ QuantArgs p) {
+    const int lane = threadIdx.x & 31;
+    const uint64_t nblocks = (p.n + kQB - 1) / kQB;
+    const uint64_t nwarps = ((uint64_t)gridDim.x * blockDim.x) >> 5;
+    for (uint64_t b = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; b < nblocks;
+         b += nwarps) {
+        const uint64_t i0 = b * kQB + (uint64_t)lane * 4u;
+        const bool whole = (b + 1) * kQB <= p.n && p.vec;
+        float x[4];
+        bool valid[4];
+        if (whole) {
+            const uint2 u = *reinterpret_cast<const uint2*>(p.g + i0);
+            const float2 a = h2x2_to_f2(u.x), c = h2x2_to_f2(u.y);
+            x[0] = a.x; x[1] = a.y; x[2] = c.x; x[3] = c.y;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) valid[j] = true;
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                valid[j] = i0 + j < p.n;
+                x[j] = valid[j] ? h2f(p.g[i0 + j]) : 0.0f;
+            }
+        }
+        float amax = 0.0f;
+        bool bad = false;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (!valid[j]) continue;
+            if (non_finite(x[j])) bad = true;
+            else amax = fmaxf(amax, fabsf(x[j]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        bad = __any_sync(0xffffffffu, bad);
+        const float scale = bad ? __uint_as_float(0x7fc00000u) : __fdiv_rn(amax, 127.0f);
+        uint32_t packed = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            int k = 0;
+            if (!bad && scale != 0.0f) {
+                k = __float2int_rn(__fdiv_rn(x[j], scale));   // nearest, ties to even
+                k = k > 127 ? 127 : (k < -127 ? -127 : k);
+            }
+            packed |= (uint32_t)(uint8_t)(int8_t)k << (8 * j);
+        }
+        if (whole) {
+            *reinterpret_cast<uint32_t*>(p.q + i0) = packed;
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (valid[j]) p.q[i0 + j] = (int8_t)(uint8_t)(packed >> (8 * j));
+        }
+        if (lane == 0) p.scales[b] = scale;
+    }
+}
+
+struct FusedQ8Args {
+    const int8_t* q[kMaxRanks];
+    const float* scales[kMaxRanks];
+    const float* master_in;
+    const float* m_in;
+    const float* v_in;
+    float* master_out;
+    float* m_out;
+    float* v_out;
+    uint16_t* param_out;
+    uint32_t* status;
+    uint64_t n;
+    uint64_t n_tiled;    // multiple of 512
+    uint64_t num_tiles;
+    Geom g;              // rank rows: rc int8 rows of T bytes, then rc scale rows of T/32 bytes
+    uint32_t srow_off;   // byte offset of the scale rows in a stage
+    int nd;
+    int param_vec;
+    AdamConsts a;
+    MeanConsts mc;
+};
+
+__device__ __forceinline__ float dequant(int8_t q, float scale) {
+    return __fmul_rn(__int2float_rn((int)q), scale);
+}
+
+__device__ __forceinline__ void fused_q8_element(const FusedQ8Args& p, uint64_t i, bool& bad) {
+    if (i >= p.n) {
+        atomicOr(p.status, ZERO_FLAG_BOUNDS);
+        return;
+    }
+    float s = 0.0f;
+    for (int r = 0; r < p.nd; ++r) s = __fadd_rn(s, dequant(p.q[r][i], p.scales[r][i / kQB]));
+    const float red = mean_of(s, p.mc);
+    bad |= non_finite(red);
+    float w = p.master_in[i], m = p.m_in[i], v = p.v_in[i];
+    adam_elem(red, w, m, v, p.a);
+    p.master_out[i] = w;
+    p.m_out[i] = m;
+    p.v_out[i] = v;
+    p.param_out[i] = f2h(w);
+}
+
+__device__ __forceinline__ const float* q8_state_row(const FusedQ8Args& p, uint32_t k) {
+    return k == 0 ? p.master_in : (k == 1 ? p.m_in : p.v_in);
+}
+
+// Producer warp: lane 0 posts the byte count, all lanes issue the row copies.
+__device__ void produce_q8(const FusedQ8Args& p, uint64_t* full, uint64_t* empty, uint8_t* data) {
+    const Geom& g = p.g;
+    const uint32_t T = g.tile;
+    const int lane = threadIdx.x & 31;
+    uint32_t it = 0;
+    bool ok = true;
+    for (uint64_t tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        const TileSpan ts = tile_span(tile, T, p.n_tiled);
+        for (uint32_t c = 0; c < g.nchunks; ++c, ++it) {
+            const uint32_t s = it % g.stages;
+            const uint32_t use = it / g.stages;
+            if (use > 0) {
+                bool w = true;
+                if (lane == 0) w = mbar_wait(&empty[s], (use - 1) & 1u);
+                if (!__shfl_sync(0xffffffffu, w, 0)) {
+                    ok = false;
+                    break;
+                }
+            }
+            const uint32_t r0 = c * g.rc;
+            const uint32_t nr = min(g.rc, (uint32_t)p.nd - r0);
+            const bool with_state = c + 1 == g.nchunks;
+            const uint32_t qb = ts.cnt, sb = ts.cnt / 32u, fb = ts.cnt * 4u;
+            uint8_t* st = data + (size_t)s * g.stage_bytes;
+            const bool sane = ts.base < p.n_tiled && (ts.cnt % kQTileAlign) == 0 && ts.cnt > 0 &&
+                              r0 < (uint32_t)p.nd && nr <= g.rc && s < (uint32_t)g.stages;
+            if (lane == 0) {
+                if (!sane) atomicOr(p.status, ZERO_FLAG_BOUNDS);
+                mbar_arrive_expect_tx(&full[s],
+                                      sane ? nr * (qb + sb) + (with_state ? 3u * fb : 0u) : 0u);
+            }
+            __syncwarp();
+            if (!sane) continue;
+            const uint32_t ncopy = 2u * nr + (with_state ? 3u : 0u);
+            for (uint32_t j = (uint32_t)lane; j < ncopy; j += 32u) {
+                if (j < nr) {
+                    bulk_g2s(st + (size_t)j * T, p.q[r0 + j] + ts.base, qb, &full[s]);
+                } else if (j < 2u * nr) {
+                    const uint32_t r = j - nr;
+                    bulk_g2s(st + p.srow_off + (size_t)r * (T / 32u),
+                             p.scales[r0 + r] + ts.base / kQB, sb, &full[s]);
+                } else {
+                    const uint32_t k = j - 2u * nr;
+                    bulk_g2s(st + g.state_off + (size_t)k * T * 4u, q8_state_row(p, k) + ts.base,
+                             fb, &full[s]);
+                }
+            }
+        }
+    }
+    if (!ok && lane == 0) {
+        atomicOr(p.status, ZERO_FLAG_TIMEOUT);
+        for (uint32_t s = 0; s < (uint32_t)g.stages && s < it; ++s) {
+            const uint32_t last = s + ((it - 1u - s) / (uint32_t)g.stages) * (uint32_t)g.stages;
+            (void)mbar_wait(&full[s], (last / (uint32_t)g.stages) & 1u);
+        }
+    }
+}
+
+template <int W>
+__global__ void __launch_bounds__(Warps<W>::kThreads, 1)
+    fused_q8_tma_kernel(const __grid_constant__ FusedQ8Args p) {
+    constexpr int E = kElems;
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + kMaxStages;
+    uint8_t* data = smem + kDataOffset;
+    init_barriers(full, empty, p.g.stages, W);
+    if ((threadIdx.x >> 5) == W) {
+        produce_q8(p, full, empty, data);
+        return;
+    }
+    const int lane = threadIdx.x & 31;
+    const uint32_t T = p.g.tile;
+    const uint32_t e0 = (uint32_t)threadIdx.x * E;
+    bool bad = false;
+    uint32_t it = 0;
+    bool ok = true;
+    for (uint64_t tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        const TileSpan ts = tile_span(tile, T, p.n_tiled);
+        const bool active = e0 < ts.cnt;
+        float acc[E], w[E], m[E], v[E];
+#pragma unroll
+        for (int j = 0; j < E; ++j) acc[j] = 0.0f;
+        for (uint32_t c = 0; c < p.g.nchunks; ++c, ++it) {
+            const uint32_t s = it % p.g.stages;
+            const uint32_t use = it / p.g.stages;
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[s], use & 1u))) {
+                if (lane == 0) atomicOr(p.status, ZERO_FLAG_TIMEOUT);
+                ok = false;
+                break;
+            }
+            const uint8_t* st = data + (size_t)s * p.g.stage_bytes;
+            if (active) {
+                const uint32_t nr = min(p.g.rc, (uint32_t)p.nd - c * p.g.rc);
+#pragma unroll 4
+                for (uint32_t r = 0; r < nr; ++r) {
+                    const uint32_t qq = *reinterpret_cast<const uint32_t*>(st + (size_t)r * T + e0);
+                    const float sc = *reinterpret_cast<const float*>(
+                        st + p.srow_off + (size_t)r * (T / 32u) + (size_t)(e0 / kQB) * 4u);
+#pragma unroll
+                    for (int j = 0; j < E; ++j)
+                        acc[j] = __fadd_rn(acc[j], dequant((int8_t)(uint8_t)(qq >> (8 * j)), sc));
+                }
+                if (c + 1 == p.g.nchunks) {
+                    const uint8_t* sf = st + p.g.state_off + (size_t)e0 * 4u;
+                    lds_f32<E>(sf, w);
+                    lds_f32<E>(sf + (size_t)T * 4u, m);
+                    lds_f32<E>(sf + (size_t)T * 8u, v);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+        if (!ok || !active) continue;
+        const uint64_t g0 = ts.base + e0;
+        if (g0 + E > p.n_tiled) {
+            atomicOr(p.status, ZERO_FLAG_BOUNDS);
+            continue;
+        }
+#pragma unroll
+        for (int j = 0; j < E; ++j) {
+            const float red = mean_of(acc[j], p.mc);
+            bad |= non_finite(red);
+            adam_elem(red, w[j], m[j], v[j], p.a);
+        }
+        stg_f32<E>(p.master_out + g0, w);
+        stg_f32<E>(p.m_out + g0, m);
+        stg_f32<E>(p.v_out + g0, v);
+        stg_f16<E>(p.param_out + g0, w, p.param_vec);
+    }
+    // the < 512 elements past the last tile (W >= 16 warps: 512 or more consumer threads)
+    if (blockIdx.x == 0 && (uint64_t)threadIdx.x < p.n - p.n_tiled)
+        fused_q8_element(p, p.n_tiled + threadIdx.x, bad);
+    flag_overflow(bad, p.status);
+}
+
+__global__ void __launch_bounds__(256) fused_q8_plain_kernel(const __grid_constant__ FusedQ8Args p) {
+    bool bad = false;
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n; i += stride)
+        fused_q8_element(p, i, bad);
+    flag_overflow(bad, p.status);
+}
+
+// Rank rows of T int8 values plus T/32 bytes of scales; same per-Nd warps and stage split as
+// the fp16 fused step.
+PipeShape q8_shape(int nd, int warps, int target_stages) {
+    PipeShape sh;
+    sh.warps = warps;
+    Geom& g = sh.g;
+    g.tile = (uint32_t)(32 * warps * kElems);
+    const size_t row = (size_t)g.tile + g.tile / 32u;
+    const size_t state = (size_t)g.tile * 12u;
+    const size_t per_stage = kSmemBudget / (size_t)target_stages;
+    size_t rc_max = per_stage > state + row ? (per_stage - state) / row : 1;
+    if (rc_max > (size_t)nd) rc_max = (size_t)nd;
+    g.nchunks = (uint32_t)(((size_t)nd + rc_max - 1) / rc_max);
+    g.rc = (uint32_t)(((size_t)nd + g.nchunks - 1) / g.nchunks);
+    g.state_off = (uint32_t)(g.rc * row);
+    g.stage_bytes = (uint32_t)(g.state_off + state);
+    size_t st = kSmemBudget / g.stage_bytes;
+    if (st < 2) st = 2;
+    if (st > kMaxStages) st = kMaxStages;
+    g.stages = (int)st;
+    sh.smem = (size_t)kDataOffset + st * g.stage_bytes;
+    return sh;
+}
+
+}  // namespace
+
+cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, int8_t* q, float* scales,
+                            cudaStream_t stream) {
+    QuantArgs p;
+    p.g = grad;
+    p.q = q;
+    p.scales = scales;
+    p.n = n;
+    p.vec = (reinterpret_cast<uintptr_t>(grad) & 7u) == 0 && (reinterpret_cast<uintptr_t>(q) & 3u) == 0;
+    DevInfo di;
+    cudaError_t e = dev_info(&di);
+    if (e != cudaSuccess) return e;
+    const uint64_t nblocks = (n + kQB - 1) / kQB;          // one warp each, 8 per CTA
+    uint64_t grid = (nblocks + 7) / 8;
+    const uint64_t cap = (uint64_t)di.sms * 8;
+    if (grid > cap) grid = cap;
+    quant_q8_kernel<<<(unsigned)(grid ? grid : 1), 256, 0, stream>>>(p);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fused_q8(uint64_t n, int nd, const int8_t* const* q, const float* const* scales,
+                            const float* master_in, const float* m_in, const float* v_in,
+                            float* master_out, float* m_out, float* v_out, uint16_t* param_out,
+                            const AdamConsts& a, const MeanConsts& mc, uint32_t* status,
+                            cudaStream_t stream) {
+    FusedQ8Args p;
+    memset(&p, 0, sizeof(p));
+    bool all16 = aligned16(master_in) && aligned16(m_in) && aligned16(v_in) &&
+                 aligned16(master_out) && aligned16(m_out) && aligned16(v_out);
+    for (int r = 0; r < nd; ++r) {
+        p.q[r] = q[r];
+        p.scales[r] = scales[r];
+        all16 = all16 && aligned16(q[r]) && aligned16(scales[r]);
+    }
+    p.master_in = master_in;
+    p.m_in = m_in;
+    p.v_in = v_in;
+    p.master_out = master_out;
+    p.m_out = m_out;
+    p.v_out = v_out;
+    p.param_out = param_out;
+    p.status = status;
+    p.n = n;
+    p.nd = nd;
+    p.param_vec = store_vec(param_out);
+    p.a = a;
+    p.mc = mc;
+    DevInfo di;
+    cudaError_t e = dev_info(&di);
+    if (e != cudaSuccess) return e;
+    if (!all16 || n < kMinTiledElems) {
+        fused_q8_plain_kernel<<<plain_grid(n, di.sms), 256, 0, stream>>>(p);
+        count_launch();
+        return cudaGetLastError();
+    }
+    const Variant var = pick_variant(nd);
+    const PipeShape sh = q8_shape(nd, var.warps, var.target_stages);
+    p.g = sh.g;
+    p.srow_off = sh.g.rc * sh.g.tile;
+    p.n_tiled = n & ~(kQTileAlign - 1);
+    p.num_tiles = (p.n_tiled + sh.g.tile - 1) / sh.g.tile;
+    switch (sh.warps) {
+        case 16: return launch_pipe(fused_q8_tma_kernel<16>, p, sh, stream);
+        case 20: return launch_pipe(fused_q8_tma_kernel<20>, p, sh, stream);
+        case 24: return launch_pipe(fused_q8_tma_kernel<24>, p, sh, stream);
+    }
+    return cudaErrorInvalidConfiguration;
+}
+
+}  // namespace zk
