@@ -33,63 +33,74 @@ struct QuantArgs {
     int8_t* q;
     float* scales;
     uint64_t n;
-    int vec;   // g 8-byte and q 4-byte aligned: 4 elements per lane in one load and one store
+    int vec;   // g 16-byte and q 8-byte aligned: 8 elements per thread in one load and one store
 };
 
-// One warp per block of 128: lane l holds elements 4l .. 4l+3.
+// A half-warp per block of 128: thread h of the half holds elements 8h .. 8h+7; a warp takes two
+// consecutive blocks per iteration.
 __global__ void __launch_bounds__(256) quant_q8_kernel(const __grid_constant__ QuantArgs p) {
     const int lane = threadIdx.x & 31;
+    const int half = lane >> 4;
+    const int hl = lane & 15;
     const uint64_t nblocks = (p.n + kQB - 1) / kQB;
+    const uint64_t npairs = (nblocks + 1) / 2;
     const uint64_t nwarps = ((uint64_t)gridDim.x * blockDim.x) >> 5;
-    for (uint64_t b = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; b < nblocks;
-         b += nwarps) {
-        const uint64_t i0 = b * kQB + (uint64_t)lane * 4u;
-        const bool whole = (b + 1) * kQB <= p.n && p.vec;
-        float x[4];
-        bool valid[4];
+    for (uint64_t pr = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; pr < npairs;
+         pr += nwarps) {
+        const uint64_t b = 2 * pr + (uint64_t)half;
+        const bool exists = b < nblocks;
+        const uint64_t i0 = b * kQB + (uint64_t)hl * 8u;
+        const bool whole = exists && (b + 1) * kQB <= p.n && p.vec;
+        float x[8];
+        bool valid[8];
         if (whole) {
-            const uint2 u = *reinterpret_cast<const uint2*>(p.g + i0);
-            const float2 a = h2x2_to_f2(u.x), c = h2x2_to_f2(u.y);
-            x[0] = a.x; x[1] = a.y; x[2] = c.x; x[3] = c.y;
+            const uint4 u = *reinterpret_cast<const uint4*>(p.g + i0);
+            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) valid[j] = true;
+            for (int k = 0; k < 4; ++k) {
+                const float2 f = h2x2_to_f2(w4[k]);
+                x[2 * k] = f.x;
+                x[2 * k + 1] = f.y;
+                valid[2 * k] = valid[2 * k + 1] = true;
+            }
         } else {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                valid[j] = i0 + j < p.n;
+            for (int j = 0; j < 8; ++j) {
+                valid[j] = exists && i0 + j < p.n;
                 x[j] = valid[j] ? h2f(p.g[i0 + j]) : 0.0f;
             }
         }
         float amax = 0.0f;
         bool bad = false;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 8; ++j) {
             if (!valid[j]) continue;
             if (non_finite(x[j])) bad = true;
             else amax = fmaxf(amax, fabsf(x[j]));
         }
+        // reductions inside each half-warp (xor offsets below 16 stay in the half)
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        bad = __any_sync(0xffffffffu, bad);
+        for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        bad = ((__ballot_sync(0xffffffffu, bad) >> (16 * half)) & 0xffffu) != 0;
         const float scale = bad ? __uint_as_float(0x7fc00000u) : __fdiv_rn(amax, 127.0f);
-        uint32_t packed = 0;
+        uint32_t packed[2] = {0u, 0u};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 8; ++j) {
             int k = 0;
             if (!bad && scale != 0.0f) {
                 k = __float2int_rn(__fdiv_rn(x[j], scale));   // nearest, ties to even
                 k = k > 127 ? 127 : (k < -127 ? -127 : k);
             }
-            packed |= (uint32_t)(uint8_t)(int8_t)k << (8 * j);
+            packed[j / 4] |= (uint32_t)(uint8_t)(int8_t)k << (8 * (j % 4));
         }
         if (whole) {
-            *reinterpret_cast<uint32_t*>(p.q + i0) = packed;
+            *reinterpret_cast<uint2*>(p.q + i0) = make_uint2(packed[0], packed[1]);
         } else {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (valid[j]) p.q[i0 + j] = (int8_t)(uint8_t)(packed >> (8 * j));
+            for (int j = 0; j < 8; ++j)
+                if (valid[j]) p.q[i0 + j] = (int8_t)(uint8_t)(packed[j / 4] >> (8 * (j % 4)));
         }
-        if (lane == 0) p.scales[b] = scale;
+        if (exists && hl == 0) p.scales[b] = scale;
     }
 }
 
@@ -117,6 +128,15 @@ struct FusedQ8Args {
 
 __device__ __forceinline__ float dequant(int8_t q, float scale) {
     return __fmul_rn(__int2float_rn((int)q), scale);
+}
+
+// Byte j of `biased` (q + 128, in 0..255) placed in the low mantissa bits of 2^23 gives the
+// float 2^23 + q + 128; subtracting 2^23 + 128 leaves q exactly. Two full-rate instructions
+// instead of an integer-to-float conversion (a quarter-rate pipe), which otherwise bounds the
+// owner's step at large Nd.
+__device__ __forceinline__ float q_to_float(uint32_t biased, int j) {
+    return __fsub_rn(__uint_as_float(__byte_perm(biased, 0x4B000000u, 0x7440u | (uint32_t)j)),
+                     8388736.0f);
 }
 
 __device__ __forceinline__ void fused_q8_element(const FusedQ8Args& p, uint64_t i, bool& bad) {
@@ -240,9 +260,10 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
                     const uint32_t qq = *reinterpret_cast<const uint32_t*>(st + (size_t)r * T + e0);
                     const float sc = *reinterpret_cast<const float*>(
                         st + p.srow_off + (size_t)r * (T / 32u) + (size_t)(e0 / kQB) * 4u);
+                    const uint32_t biased = qq ^ 0x80808080u;   // each byte q + 128
 #pragma unroll
                     for (int j = 0; j < E; ++j)
-                        acc[j] = __fadd_rn(acc[j], dequant((int8_t)(uint8_t)(qq >> (8 * j)), sc));
+                        acc[j] = __fadd_rn(acc[j], __fmul_rn(q_to_float(biased, j), sc));
                 }
                 if (c + 1 == p.g.nchunks) {
                     const uint8_t* sf = st + p.g.state_off + (size_t)e0 * 4u;
@@ -318,12 +339,13 @@ cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, int8_t* q, float* 
     p.q = q;
     p.scales = scales;
     p.n = n;
-    p.vec = (reinterpret_cast<uintptr_t>(grad) & 7u) == 0 && (reinterpret_cast<uintptr_t>(q) & 3u) == 0;
+    p.vec = (reinterpret_cast<uintptr_t>(grad) & 15u) == 0 &&
+            (reinterpret_cast<uintptr_t>(q) & 7u) == 0;
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
-    const uint64_t nblocks = (n + kQB - 1) / kQB;          // one warp each, 8 per CTA
-    uint64_t grid = (nblocks + 7) / 8;
+    const uint64_t npairs = ((n + kQB - 1) / kQB + 1) / 2;   // two blocks per warp, 8 warps/CTA
+    uint64_t grid = (npairs + 7) / 8;
     const uint64_t cap = (uint64_t)di.sms * 8;
     if (grid > cap) grid = cap;
     quant_q8_kernel<<<(unsigned)(grid ? grid : 1), 256, 0, stream>>>(p);
