@@ -302,7 +302,8 @@ zero_status zero_step_status(const uint32_t* d_status, zero_stream_t stream, uin
  * Compressed reduce-scatter payload. "ZeRO" (lastdictionary.com), main definition: extensions
  * compress the communication (ZeRO++). The pages give no format; this library's: each rank's
  * slice travels as int8 values with one fp32 scale per block of ZERO_Q8_BLOCK elements
- * (blocks counted from the slice's first element):
+ * (blocks counted from the slice's first element), and the owner accumulates q*scale with
+ * fused multiply-adds:
  *   scale = amax/127 (binary32), q = round_half_even(x/scale) clamped to [-127, 127],
  *   a block with an inf or NaN gets scale NaN and q = 0 (so the owner sees the overflow).
  * ---------------------------------------------------------------------------------------- */
@@ -313,8 +314,9 @@ zero_status zero_step_status(const uint32_t* d_status, zero_stream_t stream, uin
 zero_status zero_quantize_q8(uint64_t n, const uint16_t* grad, int8_t* q, float* scales,
                              zero_stream_t stream);
 
-/* zero_step_fused with int8 payloads: red = (sum_{r=0..nd-1} float(q_r[i]) * scale_r[i/128])/nd,
- * each product and sum an IEEE binary32 operation, then the same update, overflow flag and
+/* zero_step_fused with int8 payloads: s = fma(float(q_r[i]), scale_r[i/128], s) for r = 0..nd-1
+ * (each a binary32 fused multiply-add, one rounding), red = s/nd, then the same update, overflow
+ * flag and
  * commit protocol as zero_step_fused. rank_q / rank_scales: nd device pointers each (host
  * arrays) to this range's n values and ceil(n/128) scales, as zero_quantize_q8 wrote them.
  * 16-byte aligned payload and state pointers (and n >= 4096) take the bulk-copy kernel.

@@ -316,8 +316,9 @@ int orc_step(uint64_t n, int nd, const uint16_t* const* g, float* master, float*
  *   amax  = max |x|                          (exact; any inf/NaN in the block poisons it)
  *   scale = amax / 127                        (binary32 division), NaN for a poisoned block
  *   q     = round_half_even(x / scale), clamped to [-127, 127]; 0 if scale is 0 or NaN
- * and the owner dequantizes x' = float(q) * scale (one rounded product), sums the ranks in
- * order 0..nd-1 and divides by nd, exactly as for fp16 slices.
+ * and the owner accumulates the ranks in order 0..nd-1 with one fused multiply-add each,
+ * s = fma(float(q), scale, s) (the product and the sum rounded once, C99 fmaf), then divides by
+ * nd, exactly as for fp16 slices.
  * ---------------------------------------------------------------------------------------- */
 #define ORC_QB 128
 
@@ -367,10 +368,7 @@ void orc_reduce_mean_q8(uint64_t n, int nd, const int8_t* const* q, const float*
     float fnd = (float)nd;
     for (uint64_t i = 0; i < n; i++) {
         float s = 0.0f;
-        for (int r = 0; r < nd; r++) {
-            float x = (float)q[r][i] * scales[r][i / ORC_QB];
-            s = s + x;
-        }
+        for (int r = 0; r < nd; r++) s = fmaf((float)q[r][i], scales[r][i / ORC_QB], s);
         red[i] = s / fnd;
     }
 }
@@ -382,10 +380,7 @@ void orc_reduce_mean_q8_gathered(uint64_t n, int nd, const int8_t* const* q,
     float fnd = (float)nd;
     for (uint64_t i = 0; i < n; i++) {
         float s = 0.0f;
-        for (int r = 0; r < nd; r++) {
-            float x = (float)q[r][i] * scale[r][i];
-            s = s + x;
-        }
+        for (int r = 0; r < nd; r++) s = fmaf((float)q[r][i], scale[r][i], s);
         red[i] = s / fnd;
     }
 }

@@ -52,8 +52,11 @@ C_MUTANTS = [
     ("payload ties rounded away from zero",
      "if (r > 0.5f || (r == 0.5f && ((int32_t)f & 1))) f = f + 1.0f;",
      "if (r >= 0.5f) f = f + 1.0f;", ["q8_ties"]),
-    ("payload scale of the wrong block", "float x = (float)q[r][i] * scales[r][i / ORC_QB];",
-     "float x = (float)q[r][i] * scales[r][(i + 1) / ORC_QB];", ["q8_red"]),
+    ("payload scale of the wrong block", "s = fmaf((float)q[r][i], scales[r][i / ORC_QB], s);",
+     "s = fmaf((float)q[r][i], scales[r][(i + 1) / ORC_QB], s);", ["q8_red"]),
+    ("payload product rounded before the sum",
+     "s = fmaf((float)q[r][i], scales[r][i / ORC_QB], s);",
+     "{ float x = (float)q[r][i] * scales[r][i / ORC_QB]; s = s + x; }", ["q8_red"]),
 ]
 
 PINS = {

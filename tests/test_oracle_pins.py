@@ -570,7 +570,8 @@ def test_quant_q8_poisoned_block_skips_the_step():
 
 @pytest.mark.parametrize("nd", [1, 3, 8])
 def test_reduce_mean_q8_brute_force(nd):
-    # dequantize (one rounded product), add in rank order (rounded), divide once
+    # per rank in order: the exact product q*scale added to the running sum, rounded once
+    # (a fused multiply-add); then one division
     rng = np.random.default_rng(300 + nd)
     n = 128 * 2 + 5
     g = [(rng.standard_normal(n) * 1e-2).astype(np.float16) for _ in range(nd)]
@@ -579,8 +580,7 @@ def test_reduce_mean_q8_brute_force(nd):
     for i in range(n):
         s = Fraction(0)
         for r in range(nd):
-            prod = frac(round_f32(Fraction(int(qs[r][i])) * frac(scs[r][i // 128])))
-            s = frac(round_f32(s + prod))
+            s = frac(round_f32(s + Fraction(int(qs[r][i])) * frac(scs[r][i // 128])))
         assert red[i] == round_f32(s / nd)
     # and the payload is close to the fp16 gradients it stands for (half a step per element)
     for r in range(nd):

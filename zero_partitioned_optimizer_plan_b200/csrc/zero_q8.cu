@@ -7,11 +7,14 @@
 //     scale = amax / 127                      (IEEE binary32 division)
 //     q     = round_half_even(x / scale), clamped to [-127, 127]; 0 when scale is 0
 //   owner's fused step:
-//     red = (sum_{r=0..nd-1} float(q_r) * scale_r) / nd      (each product and sum rounded)
+//     s = fma(float(q_r), scale_r, s) for r = 0..nd-1 (one rounding each), red = s / nd,
 //     then the same unscale, Adam, fp16 cast and write-back as the fp16 fused step.
 //
 // Per parameter the owner reads nd * (1 + 4/128) payload bytes instead of 2 * nd: at Nd = 64 the
-// fused step moves 92 bytes per parameter instead of 154.
+// fused step moves 92 bytes per parameter instead of 154. Per element and rank it issues a byte
+// conversion and a fused multiply-add; half of the bytes go through the integer-to-float
+// conversion pipe, half through the mantissa-placement trick on the integer and FMA pipes, so
+// neither pipe bounds the step.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -126,8 +129,9 @@ struct FusedQ8Args {
     MeanConsts mc;
 };
 
-__device__ __forceinline__ float dequant(int8_t q, float scale) {
-    return __fmul_rn(__int2float_rn((int)q), scale);
+// acc + float(q) * scale with one rounding
+__device__ __forceinline__ float dequant_add(int8_t q, float scale, float acc) {
+    return __fmaf_rn(__int2float_rn((int)q), scale, acc);
 }
 
 // Byte j of `biased` (q + 128, in 0..255) placed in the low mantissa bits of 2^23 gives the
@@ -145,7 +149,7 @@ __device__ __forceinline__ void fused_q8_element(const FusedQ8Args& p, uint64_t 
         return;
     }
     float s = 0.0f;
-    for (int r = 0; r < p.nd; ++r) s = __fadd_rn(s, dequant(p.q[r][i], p.scales[r][i / kQB]));
+    for (int r = 0; r < p.nd; ++r) s = dequant_add(p.q[r][i], p.scales[r][i / kQB], s);
     const float red = mean_of(s, p.mc);
     bad |= non_finite(red);
     float w = p.master_in[i], m = p.m_in[i], v = p.v_in[i];
@@ -262,8 +266,12 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
                         st + p.srow_off + (size_t)r * (T / 32u) + (size_t)(e0 / kQB) * 4u);
                     const uint32_t biased = qq ^ 0x80808080u;   // each byte q + 128
 #pragma unroll
-                    for (int j = 0; j < E; ++j)
-                        acc[j] = __fadd_rn(acc[j], __fmul_rn(q_to_float(biased, j), sc));
+                    for (int j = 0; j < E; ++j) {
+                        // bytes 0, 1: conversion pipe; bytes 2, 3: integer and FMA pipes
+                        const float qf = (j < 2) ? __int2float_rn((int)(int8_t)(uint8_t)(qq >> (8 * j)))
+                                                 : q_to_float(biased, j);
+                        acc[j] = __fmaf_rn(qf, sc, acc[j]);
+                    }
                 }
                 if (c + 1 == p.g.nchunks) {
                     const uint8_t* sf = st + p.g.state_off + (size_t)e0 * 4u;
