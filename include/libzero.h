@@ -308,25 +308,29 @@ zero_status zero_step_status(const uint32_t* d_status, zero_stream_t stream, uin
  *   a block with an inf or NaN gets scale NaN and q = 0 (so the owner sees the overflow).
  * ---------------------------------------------------------------------------------------- */
 #define ZERO_Q8_BLOCK 128
+#define ZERO_Q8_RECORD 132   /* bytes per block: 128 int8 values, then the fp32 scale */
 
-/* Quantize one rank's n fp16 gradients: q[n] (any alignment), scales[ceil(n/128)] (4-byte
- * aligned), all device memory. Errors: ZERO_EINVAL (null, overlap), ZERO_EALIGN, ZERO_ECUDA. */
-zero_status zero_quantize_q8(uint64_t n, const uint16_t* grad, int8_t* q, float* scales,
+/* Bytes of the payload of n elements: ceil(n/128) records of 132 bytes. */
+#define ZERO_Q8_PAYLOAD_BYTES(n) ((((uint64_t)(n) + 127u) / 128u) * 132u)
+
+/* Quantize one rank's n fp16 gradients into its payload: record b holds q of elements
+ * [128b, 128b+128) in bytes 0..127 (unused bytes of a short last block are 0) and the block's
+ * scale in bytes 128..131. Device memory; payload 4-byte aligned (16 for the bulk-copy path of
+ * zero_step_fused_q8). Errors: ZERO_EINVAL (null, overlap), ZERO_EALIGN, ZERO_ECUDA. */
+zero_status zero_quantize_q8(uint64_t n, const uint16_t* grad, uint8_t* payload,
                              zero_stream_t stream);
 
 /* zero_step_fused with int8 payloads: s = fma(float(q_r[i]), scale_r[i/128], s) for r = 0..nd-1
  * (each a binary32 fused multiply-add, one rounding), red = s/nd, then the same update, overflow
- * flag and
- * commit protocol as zero_step_fused. rank_q / rank_scales: nd device pointers each (host
- * arrays) to this range's n values and ceil(n/128) scales, as zero_quantize_q8 wrote them.
- * 16-byte aligned payload and state pointers (and n >= 4096) take the bulk-copy kernel.
- * Errors: as zero_step_fused. */
-zero_status zero_step_fused_q8(uint64_t n, int nd, const int8_t* const* rank_q,
-                               const float* const* rank_scales, const float* master_in,
-                               const float* m_in, const float* v_in, float* master_out,
-                               float* m_out, float* v_out, uint16_t* param_out,
-                               const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
-                               zero_stream_t stream);
+ * flag and commit protocol as zero_step_fused. rank_payload: nd device pointers (host array),
+ * each to this range's ZERO_Q8_PAYLOAD_BYTES(n) bytes as zero_quantize_q8 wrote them (records
+ * counted from the range's first element). 16-byte aligned payload and state pointers (and
+ * n >= 4096) take the bulk-copy kernel. Errors: as zero_step_fused. */
+zero_status zero_step_fused_q8(uint64_t n, int nd, const uint8_t* const* rank_payload,
+                               const float* master_in, const float* m_in, const float* v_in,
+                               float* master_out, float* m_out, float* v_out,
+                               uint16_t* param_out, const zero_adam_hparams* hp, int64_t step,
+                               uint32_t* d_status, zero_stream_t stream);
 
 /* Self-test of the kernels' bounded waits (failure detection without a fault): launches the
  * fused pipeline on one tile with its copy-issuing warp switched off, so every consumer's wait

@@ -283,18 +283,17 @@ def test_scaler_rejects():
 
 def test_q8_rejects():
     with pytest.raises(lz.ZeroError) as e:
-        lz.zero_quantize_q8(100, A, A + 10, A + MB + 2, 0)
+        lz.zero_quantize_q8(100, A, A + MB + 2, 0)
     assert e.value.code == lz.ZERO_EALIGN
     with pytest.raises(lz.ZeroError) as e:
-        lz.zero_quantize_q8(100, A, A + 100, A + MB, 0)                 # q over grad
+        lz.zero_quantize_q8(100, A, A + 100, 0)                     # payload over grad
     assert e.value.code == lz.ZERO_EINVAL
-    qs = [A + i * MB for i in range(2)]
-    scs = [A + (10 + i) * MB for i in range(2)]
+    assert lz.q8_payload_bytes(1) == 132 and lz.q8_payload_bytes(256) == 264
+    ps = [A + i * MB for i in range(2)]
     ins = [A + 100 * MB, A + 101 * MB, A + 102 * MB]
     outs = [A + 110 * MB, A + 111 * MB, A + 112 * MB]
-    for q, s, code in [(qs[:1] + [0], scs, lz.ZERO_EINVAL), (qs, scs[:1] + [A + 11 * MB + 2],
-                                                              lz.ZERO_EALIGN),
-                       (qs, [A + 110 * MB, scs[1]], lz.ZERO_EINVAL)]:
+    for pay, code in [(ps[:1] + [0], lz.ZERO_EINVAL), (ps[:1] + [A + MB + 2], lz.ZERO_EALIGN),
+                      ([A + 110 * MB, ps[1]], lz.ZERO_EINVAL)]:
         with pytest.raises(lz.ZeroError) as e:
-            lz.zero_step_fused_q8(1000, 2, q, s, *ins, *outs, A + 120 * MB, HP, 1, A + 130 * MB, 0)
+            lz.zero_step_fused_q8(1000, 2, pay, *ins, *outs, A + 120 * MB, HP, 1, A + 130 * MB, 0)
         assert e.value.code == code

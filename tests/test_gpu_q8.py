@@ -24,12 +24,21 @@ def _gpu():
     torch.cuda.empty_cache()
 
 
-def _quant_dev(g_dev, q_off=0):
+def _quant_dev(g_dev, off=0):
+    """A rank's payload on the device (optionally at a byte offset inside a larger buffer)."""
     n = g_dev.numel()
-    qbig = torch.zeros(n + 16, dtype=torch.int8, device=DEV)
-    q = qbig[q_off:q_off + n]
-    sc = torch.empty((n + QB - 1) // QB, dtype=torch.float32, device=DEV)
-    lz.zero_quantize_q8(n, g_dev, q, sc)
+    nbytes = lz.q8_payload_bytes(n)
+    big = torch.zeros(nbytes + 32, dtype=torch.uint8, device=DEV)
+    pay = big[off:off + nbytes]
+    lz.zero_quantize_q8(n, g_dev, pay)
+    return pay
+
+
+def _split(pay, n):
+    """Payload records -> (int8 values of the n elements, fp32 scale per block)."""
+    rec = pay.cpu().numpy().reshape(-1, 132)
+    q = rec[:, :128].reshape(-1).view(np.int8)[:n]
+    sc = np.ascontiguousarray(rec[:, 128:]).view(np.float32).reshape(-1)
     return q, sc
 
 
@@ -51,11 +60,16 @@ def test_quantize_bit_exact(n, kind):
     goff = 1 if kind == "unaligned" else 0
     gbig = torch.zeros(n + 8, dtype=torch.float16, device=DEV)
     gbig[goff:goff + n] = g.to(DEV)
-    q, sc = _quant_dev(gbig[goff:goff + n], q_off=1 if kind == "unaligned" else 0)
+    pay = _quant_dev(gbig[goff:goff + n], off=4 if kind == "unaligned" else 0)
     torch.cuda.synchronize()
+    q, sc = _split(pay, n)
     q_ref, sc_ref = oracle.quant_q8(g.numpy())
-    assert np.array_equal(q.cpu().numpy(), q_ref)
-    assert _same_scales(sc.cpu().numpy(), sc_ref)
+    assert np.array_equal(q, q_ref)
+    assert _same_scales(sc, sc_ref)
+    # a short last block's unused bytes are zero
+    tail = n % 128
+    if tail:
+        assert not pay.cpu().numpy().reshape(-1, 132)[-1, tail:128].any()
 
 
 @pytest.mark.parametrize("nd", [1, 2, 3, 8, 16, 25, 64])
@@ -71,8 +85,7 @@ def test_fused_q8_vs_oracle(n, nd):
         pay = [_quant_dev(g.to(DEV)) for g in g_cpu]
         st = status_word()
         ins, outs = pp.cur, pp.nxt
-        lz.zero_step_fused_q8(n, nd, [q for q, _ in pay], [s for _, s in pay], *ins, *outs,
-                              params, HP, t, st)
+        lz.zero_step_fused_q8(n, nd, pay, *ins, *outs, params, HP, t, st)
         lz.zero_step_commit(n, *ins, *outs, params, st)
         torch.cuda.synchronize()
         assert status_flags(st) == 0
@@ -98,8 +111,7 @@ def test_fused_q8_overflow_through_poisoned_block():
     pay = [_quant_dev(g) for g in g_dev]
     params = torch.zeros(n, dtype=torch.float16, device=DEV)
     st = status_word()
-    lz.zero_step_fused_q8(n, nd, [q for q, _ in pay], [s for _, s in pay], *pp.cur, *pp.nxt,
-                          params, HP, 1, st)
+    lz.zero_step_fused_q8(n, nd, pay, *pp.cur, *pp.nxt, params, HP, 1, st)
     lz.zero_step_commit(n, *pp.cur, *pp.nxt, params, st)
     assert lz.zero_step_status(st)[0] == lz.ZERO_STEP_SKIPPED
     for a, b in zip(pp.cur, pp.nxt):
@@ -112,11 +124,10 @@ def test_fused_q8_unaligned_payload_takes_plain_kernel():
     master, m, v = synth.state_warm(n, seed=8)
     pp = PingPong(master, m, v)
     g_cpu = [synth.grad_f16(n, 1e-2, seed=9, rank=r) for r in range(nd)]
-    pay = [_quant_dev(g.to(DEV), q_off=3) for g in g_cpu]
+    pay = [_quant_dev(g.to(DEV), off=4) for g in g_cpu]     # 4- but not 16-byte aligned
     params = torch.empty(n, dtype=torch.float16, device=DEV)
     st = status_word()
-    lz.zero_step_fused_q8(n, nd, [q for q, _ in pay], [s for _, s in pay], *pp.cur, *pp.nxt,
-                          params, HP, 1, st)
+    lz.zero_step_fused_q8(n, nd, pay, *pp.cur, *pp.nxt, params, HP, 1, st)
     torch.cuda.synchronize()
     assert status_flags(st) == 0
     ref = [oracle.quant_q8(g.numpy()) for g in g_cpu]
@@ -133,15 +144,13 @@ def test_7p5b_shard_view_q8_sampled():
     S = total // nd
     owner = 63
     full = torch.zeros(total, dtype=torch.float16, device=DEV)
-    qs, scs = [], []
+    pays = []
     g = torch.empty(S, dtype=torch.float16, device=DEV)
     for r in range(nd):
         synth.grad_f16(S, 1e-3, seed=11, rank=r, out=g)
-        q = torch.empty(S, dtype=torch.int8, device=DEV)
-        sc = torch.empty((S + QB - 1) // QB, dtype=torch.float32, device=DEV)
-        lz.zero_quantize_q8(S, g, q, sc)
-        qs.append(q)
-        scs.append(sc)
+        pay = torch.empty(lz.q8_payload_bytes(S), dtype=torch.uint8, device=DEV)
+        lz.zero_quantize_q8(S, g, pay)
+        pays.append(pay)
     del g
     cur = list(synth.state_warm(S, seed=12, device=DEV))
     nxt = [torch.empty_like(x) for x in cur]
@@ -149,16 +158,17 @@ def test_7p5b_shard_view_q8_sampled():
     idx = np.unique(np.concatenate([rng.integers(0, S, 100_000), np.arange(S - 600, S),
                                     np.arange(0, 256)]))
     idx_dev = torch.from_numpy(idx).to(DEV)
-    bidx_dev = torch.from_numpy(idx // QB).to(DEV)
+    qpos = torch.from_numpy((idx // QB) * 132 + idx % QB).to(DEV)
+    spos = torch.from_numpy(((idx // QB) * 132 + 128)[:, None] + np.arange(4)).to(DEV)
     w0, m0, v0 = (x[idx_dev].cpu().numpy() for x in cur)
     out = full[owner * S:(owner + 1) * S]
     st = status_word()
-    lz.zero_step_fused_q8(S, nd, qs, scs, *cur, *nxt, out, HP, 1, st)
+    lz.zero_step_fused_q8(S, nd, pays, *cur, *nxt, out, HP, 1, st)
     lz.zero_step_commit(S, *cur, *nxt, out, st)
     torch.cuda.synchronize()
     assert status_flags(st) == 0
-    gq = [q[idx_dev].cpu().numpy() for q in qs]
-    gs = [s[bidx_dev].cpu().numpy() for s in scs]
+    gq = [p[qpos].cpu().numpy().view(np.int8) for p in pays]
+    gs = [np.ascontiguousarray(p[spos].cpu().numpy()).view(np.float32).reshape(-1) for p in pays]
     skipped, w, mm, vv, p = oracle.step_q8_gathered(gq, gs, w0, m0, v0, ORC_HP, 1)
     assert not skipped
     check_f32("master", nxt[0][idx_dev].cpu().numpy(), w)

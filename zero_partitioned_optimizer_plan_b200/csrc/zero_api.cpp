@@ -305,43 +305,37 @@ zero_status zero_step_fused_dc(uint64_t n, int nd, const uint16_t* const* rank_g
                                           zk::make_mean(nd), d_status, (cudaStream_t)stream));
 }
 
-zero_status zero_quantize_q8(uint64_t n, const uint16_t* grad, int8_t* q, float* scales,
+zero_status zero_quantize_q8(uint64_t n, const uint16_t* grad, uint8_t* payload,
                              zero_stream_t stream) {
     if (n == 0) return ZERO_OK;
-    if (!grad || !q || !scales || n > (UINT64_MAX / 8)) return ZERO_EINVAL;
-    if (!zk::aligned(grad, 2) || !zk::aligned(scales, 4)) return ZERO_EALIGN;
-    const uint64_t nb = (n + ZERO_Q8_BLOCK - 1) / ZERO_Q8_BLOCK;
-    if (zk::overlap(q, n, grad, n * 2) || zk::overlap(scales, nb * 4, grad, n * 2) ||
-        zk::overlap(q, n, scales, nb * 4))
-        return ZERO_EINVAL;
-    return zk::from_cuda(zk::launch_quant_q8(n, grad, q, scales, (cudaStream_t)stream));
+    if (!grad || !payload || n > (UINT64_MAX / 8)) return ZERO_EINVAL;
+    if (!zk::aligned(grad, 2) || !zk::aligned(payload, 4)) return ZERO_EALIGN;
+    if (zk::overlap(payload, ZERO_Q8_PAYLOAD_BYTES(n), grad, n * 2)) return ZERO_EINVAL;
+    return zk::from_cuda(zk::launch_quant_q8(n, grad, payload, (cudaStream_t)stream));
 }
 
-zero_status zero_step_fused_q8(uint64_t n, int nd, const int8_t* const* rank_q,
-                               const float* const* rank_scales, const float* master_in,
-                               const float* m_in, const float* v_in, float* master_out,
-                               float* m_out, float* v_out, uint16_t* param_out,
-                               const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
-                               zero_stream_t stream) {
+zero_status zero_step_fused_q8(uint64_t n, int nd, const uint8_t* const* rank_payload,
+                               const float* master_in, const float* m_in, const float* v_in,
+                               float* master_out, float* m_out, float* v_out,
+                               uint16_t* param_out, const zero_adam_hparams* hp, int64_t step,
+                               uint32_t* d_status, zero_stream_t stream) {
     if (nd < 1 || nd > ZERO_MAX_RANKS || !zk::hparams_ok(hp) || step < 1 || !d_status)
         return ZERO_EINVAL;
     if (n == 0) return ZERO_OK;
-    if (!rank_q || !rank_scales) return ZERO_EINVAL;
+    if (!rank_payload) return ZERO_EINVAL;
     zero_status st = check_fused_state(n, master_in, m_in, v_in, master_out, m_out, v_out,
                                        param_out, d_status);
     if (st != ZERO_OK) return st;
-    const uint64_t nb = (n + ZERO_Q8_BLOCK - 1) / ZERO_Q8_BLOCK;
+    const uint64_t pb = ZERO_Q8_PAYLOAD_BYTES(n);
     const void* outs[5] = {master_out, m_out, v_out, param_out, d_status};
     const uint64_t olen[5] = {n * 4, n * 4, n * 4, n * 2, 4};
     for (int r = 0; r < nd; ++r) {
-        if (!rank_q[r] || !rank_scales[r]) return ZERO_EINVAL;
-        if (!zk::aligned(rank_scales[r], 4)) return ZERO_EALIGN;
+        if (!rank_payload[r]) return ZERO_EINVAL;
+        if (!zk::aligned(rank_payload[r], 4)) return ZERO_EALIGN;
         for (int i = 0; i < 5; ++i)
-            if (zk::overlap(outs[i], olen[i], rank_q[r], n) ||
-                zk::overlap(outs[i], olen[i], rank_scales[r], nb * 4))
-                return ZERO_EINVAL;
+            if (zk::overlap(outs[i], olen[i], rank_payload[r], pb)) return ZERO_EINVAL;
     }
-    return zk::from_cuda(zk::launch_fused_q8(n, nd, rank_q, rank_scales, master_in, m_in, v_in,
+    return zk::from_cuda(zk::launch_fused_q8(n, nd, rank_payload, master_in, m_in, v_in,
                                              master_out, m_out, v_out, param_out,
                                              zk::make_adam(hp, step), zk::make_mean(nd),
                                              d_status, (cudaStream_t)stream));

@@ -43,9 +43,9 @@ cudaError_t launch_adam(uint64_t n, const float* grad, float* master, float* m, 
                         uint32_t* status, cudaStream_t stream);
 
 cudaError_t launch_selftest_timeout(uint32_t* status, cudaStream_t stream);
-cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, int8_t* q, float* scales,
+cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, uint8_t* payload,
                             cudaStream_t stream);
-cudaError_t launch_fused_q8(uint64_t n, int nd, const int8_t* const* q, const float* const* scales,
+cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,
                             const float* master_in, const float* m_in, const float* v_in,
                             float* master_out, float* m_out, float* v_out, uint16_t* param_out,
                             const AdamConsts& a, const MeanConsts& mc, uint32_t* status,

@@ -10,7 +10,12 @@
 //     s = fma(float(q_r), scale_r, s) for r = 0..nd-1 (one rounding each), red = s / nd,
 //     then the same unscale, Adam, fp16 cast and write-back as the fp16 fused step.
 //
-// Per parameter the owner reads nd * (1 + 4/128) payload bytes instead of 2 * nd: at Nd = 64 the
+// Layout: a rank's payload is an array of 132-byte records, one per block: the block's 128 int8
+// values, then its fp32 scale (a short last block is padded to a full record). A tile of a
+// multiple of 512 elements is then one contiguous, 16-byte-aligned run of records per rank:
+// one bulk copy per rank and tile.
+//
+// Per parameter the owner reads nd * 132/128 payload bytes instead of 2 * nd: at Nd = 64 the
 // fused step moves 92 bytes per parameter instead of 154. Per element and rank it issues a byte
 // conversion and a fused multiply-add; half of the bytes go through the integer-to-float
 // conversion pipe, half through the mantissa-placement trick on the integer and FMA pipes, so
@@ -29,14 +34,14 @@ namespace zk {
 namespace {
 
 constexpr int kQB = 128;                 // elements per scale block
-constexpr uint64_t kQTileAlign = 512;    // tiles cover a multiple of 512 elements (16-byte rows)
+constexpr int kRec = 132;                // bytes per record: 128 int8 values, one fp32 scale
+constexpr uint64_t kQTileAlign = 512;    // tiles cover a multiple of 512 elements (528-byte runs)
 
 struct QuantArgs {
     const uint16_t* g;
-    int8_t* q;
-    float* scales;
+    uint8_t* rec;        // ceil(n/128) records
     uint64_t n;
-    int vec;   // g 16-byte and q 8-byte aligned: 8 elements per thread in one load and one store
+    int vec;   // g 16-byte and rec 4-byte aligned: 8 elements per thread in one load, two stores
 };
 
 // A half-warp per block of 128: thread h of the half holds elements 8h .. 8h+7; a warp takes two
@@ -53,7 +58,7 @@ __global__ void __launch_bounds__(256) quant_q8_kernel(const __grid_constant__ Q
         const uint64_t b = 2 * pr + (uint64_t)half;
         const bool exists = b < nblocks;
         const uint64_t i0 = b * kQB + (uint64_t)hl * 8u;
-        const bool whole = exists && (b + 1) * kQB <= p.n && p.vec;
+        const bool whole = exists && (b + 1) * kQB <= p.n && p.vec;   // uniform per half
         float x[8];
         bool valid[8];
         if (whole) {
@@ -96,20 +101,21 @@ __global__ void __launch_bounds__(256) quant_q8_kernel(const __grid_constant__ Q
             }
             packed[j / 4] |= (uint32_t)(uint8_t)(int8_t)k << (8 * (j % 4));
         }
-        if (whole) {
-            *reinterpret_cast<uint2*>(p.q + i0) = make_uint2(packed[0], packed[1]);
-        } else {
+        uint8_t* r = p.rec + b * kRec;
+        if (whole) {   // the record base is 4-byte aligned (132 = 4 * 33), 8 * hl too
+            reinterpret_cast<uint32_t*>(r + hl * 8)[0] = packed[0];
+            reinterpret_cast<uint32_t*>(r + hl * 8)[1] = packed[1];
+        } else if (exists) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                if (valid[j]) p.q[i0 + j] = (int8_t)(uint8_t)(packed[j / 4] >> (8 * (j % 4)));
+            for (int j = 0; j < 8; ++j)   // a short block's unused bytes are written as 0
+                r[hl * 8 + j] = valid[j] ? (uint8_t)(packed[j / 4] >> (8 * (j % 4))) : 0u;
         }
-        if (exists && hl == 0) p.scales[b] = scale;
+        if (exists && hl == 0) *reinterpret_cast<float*>(r + kQB) = scale;
     }
 }
 
 struct FusedQ8Args {
-    const int8_t* q[kMaxRanks];
-    const float* scales[kMaxRanks];
+    const uint8_t* rec[kMaxRanks];   // each rank's records for this range
     const float* master_in;
     const float* m_in;
     const float* v_in;
@@ -121,8 +127,8 @@ struct FusedQ8Args {
     uint64_t n;
     uint64_t n_tiled;    // multiple of 512
     uint64_t num_tiles;
-    Geom g;              // rank rows: rc int8 rows of T bytes, then rc scale rows of T/32 bytes
-    uint32_t srow_off;   // byte offset of the scale rows in a stage
+    Geom g;              // rank rows: rc runs of T/128 records (T*132/128 bytes each)
+    uint32_t row;        // bytes of one rank's run in a stage
     int nd;
     int param_vec;
     AdamConsts a;
@@ -149,7 +155,11 @@ __device__ __forceinline__ void fused_q8_element(const FusedQ8Args& p, uint64_t 
         return;
     }
     float s = 0.0f;
-    for (int r = 0; r < p.nd; ++r) s = dequant_add(p.q[r][i], p.scales[r][i / kQB], s);
+    const uint64_t off = (i / kQB) * kRec;
+    for (int r = 0; r < p.nd; ++r) {
+        const uint8_t* rec = p.rec[r] + off;
+        s = dequant_add((int8_t)rec[i % kQB], *reinterpret_cast<const float*>(rec + kQB), s);
+    }
     const float red = mean_of(s, p.mc);
     bad |= non_finite(red);
     float w = p.master_in[i], m = p.m_in[i], v = p.v_in[i];
@@ -187,27 +197,23 @@ __device__ void produce_q8(const FusedQ8Args& p, uint64_t* full, uint64_t* empty
             const uint32_t r0 = c * g.rc;
             const uint32_t nr = min(g.rc, (uint32_t)p.nd - r0);
             const bool with_state = c + 1 == g.nchunks;
-            const uint32_t qb = ts.cnt, sb = ts.cnt / 32u, fb = ts.cnt * 4u;
+            const uint32_t rb = ts.cnt / kQB * kRec, fb = ts.cnt * 4u;
             uint8_t* st = data + (size_t)s * g.stage_bytes;
             const bool sane = ts.base < p.n_tiled && (ts.cnt % kQTileAlign) == 0 && ts.cnt > 0 &&
                               r0 < (uint32_t)p.nd && nr <= g.rc && s < (uint32_t)g.stages;
             if (lane == 0) {
                 if (!sane) atomicOr(p.status, ZERO_FLAG_BOUNDS);
-                mbar_arrive_expect_tx(&full[s],
-                                      sane ? nr * (qb + sb) + (with_state ? 3u * fb : 0u) : 0u);
+                mbar_arrive_expect_tx(&full[s], sane ? nr * rb + (with_state ? 3u * fb : 0u) : 0u);
             }
             __syncwarp();
             if (!sane) continue;
-            const uint32_t ncopy = 2u * nr + (with_state ? 3u : 0u);
+            const uint32_t ncopy = nr + (with_state ? 3u : 0u);
             for (uint32_t j = (uint32_t)lane; j < ncopy; j += 32u) {
                 if (j < nr) {
-                    bulk_g2s(st + (size_t)j * T, p.q[r0 + j] + ts.base, qb, &full[s]);
-                } else if (j < 2u * nr) {
-                    const uint32_t r = j - nr;
-                    bulk_g2s(st + p.srow_off + (size_t)r * (T / 32u),
-                             p.scales[r0 + r] + ts.base / kQB, sb, &full[s]);
+                    bulk_g2s(st + (size_t)j * p.row, p.rec[r0 + j] + ts.base / kQB * kRec, rb,
+                             &full[s]);
                 } else {
-                    const uint32_t k = j - 2u * nr;
+                    const uint32_t k = j - nr;
                     bulk_g2s(st + g.state_off + (size_t)k * T * 4u, q8_state_row(p, k) + ts.base,
                              fb, &full[s]);
                 }
@@ -259,11 +265,13 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
             const uint8_t* st = data + (size_t)s * p.g.stage_bytes;
             if (active) {
                 const uint32_t nr = min(p.g.rc, (uint32_t)p.nd - c * p.g.rc);
+                // this thread's record in each rank's run; its 4 values share the scale
+                const uint8_t* rec0 = st + (size_t)(e0 / kQB) * kRec;
 #pragma unroll 4
                 for (uint32_t r = 0; r < nr; ++r) {
-                    const uint32_t qq = *reinterpret_cast<const uint32_t*>(st + (size_t)r * T + e0);
-                    const float sc = *reinterpret_cast<const float*>(
-                        st + p.srow_off + (size_t)r * (T / 32u) + (size_t)(e0 / kQB) * 4u);
+                    const uint8_t* rec = rec0 + (size_t)r * p.row;
+                    const uint32_t qq = *reinterpret_cast<const uint32_t*>(rec + e0 % kQB);
+                    const float sc = *reinterpret_cast<const float*>(rec + kQB);
                     const uint32_t biased = qq ^ 0x80808080u;   // each byte q + 128
 #pragma unroll
                     for (int j = 0; j < E; ++j) {
@@ -314,14 +322,13 @@ __global__ void __launch_bounds__(256) fused_q8_plain_kernel(const __grid_consta
     flag_overflow(bad, p.status);
 }
 
-// Rank rows of T int8 values plus T/32 bytes of scales; same per-Nd warps and stage split as
-// the fp16 fused step.
+// A rank's run of T/128 records per stage; same per-Nd warps and stage split as the fp16 step.
 PipeShape q8_shape(int nd, int warps, int target_stages) {
     PipeShape sh;
     sh.warps = warps;
     Geom& g = sh.g;
     g.tile = (uint32_t)(32 * warps * kElems);
-    const size_t row = (size_t)g.tile + g.tile / 32u;
+    const size_t row = (size_t)g.tile / kQB * kRec;
     const size_t state = (size_t)g.tile * 12u;
     const size_t per_stage = kSmemBudget / (size_t)target_stages;
     size_t rc_max = per_stage > state + row ? (per_stage - state) / row : 1;
@@ -340,15 +347,14 @@ PipeShape q8_shape(int nd, int warps, int target_stages) {
 
 }  // namespace
 
-cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, int8_t* q, float* scales,
+cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, uint8_t* payload,
                             cudaStream_t stream) {
     QuantArgs p;
     p.g = grad;
-    p.q = q;
-    p.scales = scales;
+    p.rec = payload;
     p.n = n;
     p.vec = (reinterpret_cast<uintptr_t>(grad) & 15u) == 0 &&
-            (reinterpret_cast<uintptr_t>(q) & 7u) == 0;
+            (reinterpret_cast<uintptr_t>(payload) & 3u) == 0;
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
@@ -361,7 +367,7 @@ cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, int8_t* q, float* 
     return cudaGetLastError();
 }
 
-cudaError_t launch_fused_q8(uint64_t n, int nd, const int8_t* const* q, const float* const* scales,
+cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,
                             const float* master_in, const float* m_in, const float* v_in,
                             float* master_out, float* m_out, float* v_out, uint16_t* param_out,
                             const AdamConsts& a, const MeanConsts& mc, uint32_t* status,
@@ -371,9 +377,8 @@ cudaError_t launch_fused_q8(uint64_t n, int nd, const int8_t* const* q, const fl
     bool all16 = aligned16(master_in) && aligned16(m_in) && aligned16(v_in) &&
                  aligned16(master_out) && aligned16(m_out) && aligned16(v_out);
     for (int r = 0; r < nd; ++r) {
-        p.q[r] = q[r];
-        p.scales[r] = scales[r];
-        all16 = all16 && aligned16(q[r]) && aligned16(scales[r]);
+        p.rec[r] = payload[r];
+        all16 = all16 && aligned16(payload[r]);
     }
     p.master_in = master_in;
     p.m_in = m_in;
@@ -399,7 +404,7 @@ cudaError_t launch_fused_q8(uint64_t n, int nd, const int8_t* const* q, const fl
     const Variant var = pick_variant(nd);
     const PipeShape sh = q8_shape(nd, var.warps, var.target_stages);
     p.g = sh.g;
-    p.srow_off = sh.g.rc * sh.g.tile;
+    p.row = sh.g.tile / kQB * kRec;
     p.n_tiled = n & ~(kQTileAlign - 1);
     p.num_tiles = (p.n_tiled + sh.g.tile - 1) / sh.g.tile;
     switch (sh.warps) {

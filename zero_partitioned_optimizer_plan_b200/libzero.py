@@ -32,6 +32,12 @@ ZERO_FLAG_BOUNDS = 0x8
 
 ZERO_MAX_RANKS = 64
 ZERO_Q8_BLOCK = 128
+ZERO_Q8_RECORD = 132
+
+
+def q8_payload_bytes(n: int) -> int:
+    """ZERO_Q8_PAYLOAD_BYTES(n)."""
+    return (n + 127) // 128 * 132
 
 # every symbol include/libzero.h declares
 SYMBOLS = (
@@ -130,8 +136,8 @@ def _load():
     L.zero_adam_shard_dc.argtypes = [u64, vp, vp, vp, vp, vp, vp, vp, vp]
     L.zero_step_fused_dc.argtypes = [u64, i32, P(vp), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.zero_selftest_timeout.argtypes = [vp, vp]
-    L.zero_quantize_q8.argtypes = [u64, vp, vp, vp, vp]
-    L.zero_step_fused_q8.argtypes = [u64, i32, P(vp), P(vp), vp, vp, vp, vp, vp, vp, vp,
+    L.zero_quantize_q8.argtypes = [u64, vp, vp, vp]
+    L.zero_step_fused_q8.argtypes = [u64, i32, P(vp), vp, vp, vp, vp, vp, vp, vp,
                                      P(_HP), i64, vp, vp]
     L.zero_adam_consts_table.argtypes = [P(_HP), i64, i64, P(AdamConsts)]
     L.zero_scaler_prepare.argtypes = [vp, vp, i64, vp, vp, vp]
@@ -311,19 +317,19 @@ def zero_step_fused_dc(n: int, nd: int, rank_grads, master_in, m_in, v_in, maste
            "zero_step_fused_dc")
 
 
-def zero_quantize_q8(n: int, grad, q, scales, stream=None):
-    _check(_lib.zero_quantize_q8(n, _ptr(grad, 2), _ptr(q, 1), _ptr(scales, 4), _stream(stream)),
+def zero_quantize_q8(n: int, grad, payload, stream=None):
+    _check(_lib.zero_quantize_q8(n, _ptr(grad, 2), _ptr(payload, 1), _stream(stream)),
            "zero_quantize_q8")
 
 
-def zero_step_fused_q8(n: int, nd: int, rank_q, rank_scales, master_in, m_in, v_in, master_out,
-                       m_out, v_out, param_out, hp: AdamHP, step: int, d_status, stream=None):
+def zero_step_fused_q8(n: int, nd: int, rank_payload, master_in, m_in, v_in, master_out, m_out,
+                       v_out, param_out, hp: AdamHP, step: int, d_status, stream=None):
     h = hp._c()
-    _check(_lib.zero_step_fused_q8(n, nd, _ptr_array(rank_q, 1), _ptr_array(rank_scales, 4),
-                                   _ptr(master_in, 4), _ptr(m_in, 4), _ptr(v_in, 4),
-                                   _ptr(master_out, 4), _ptr(m_out, 4), _ptr(v_out, 4),
-                                   _ptr(param_out, 2), C.byref(h), step, _ptr(d_status, 4),
-                                   _stream(stream)), "zero_step_fused_q8")
+    _check(_lib.zero_step_fused_q8(n, nd, _ptr_array(rank_payload, 1), _ptr(master_in, 4),
+                                   _ptr(m_in, 4), _ptr(v_in, 4), _ptr(master_out, 4),
+                                   _ptr(m_out, 4), _ptr(v_out, 4), _ptr(param_out, 2),
+                                   C.byref(h), step, _ptr(d_status, 4), _stream(stream)),
+           "zero_step_fused_q8")
 
 
 def zero_step_commit(n: int, master_in, m_in, v_in, master_out, m_out, v_out, param_out,
