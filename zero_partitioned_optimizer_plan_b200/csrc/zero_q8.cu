@@ -322,7 +322,16 @@ __global__ void __launch_bounds__(256) fused_q8_plain_kernel(const __grid_consta
     flag_overflow(bad, p.status);
 }
 
-// A rank's run of T/128 records per stage; same per-Nd warps and stage split as the fp16 step.
+// Consumer warps and stage split per Nd for the int8 payload, measured on B200: the
+// dequantizing accumulation issues about twice the instructions per byte of the fp16 sum, so up
+// to Nd = 16 the most warps win (Nd = 2/8/16: 6.4/6.7/6.6 TB/s with 24 warps against 5.0/5.4/5.5
+// with 16); above, 16 warps with the budget split in two (Nd = 32/64: 5.7/4.8 TB/s).
+Variant pick_variant_q8(int nd) {
+    if (nd <= 16) return {24, 2};
+    return {16, 2};
+}
+
+// A rank's run of T/128 records per stage.
 PipeShape q8_shape(int nd, int warps, int target_stages) {
     PipeShape sh;
     sh.warps = warps;
@@ -401,7 +410,13 @@ cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,
         count_launch();
         return cudaGetLastError();
     }
-    const Variant var = pick_variant(nd);
+    Variant var = pick_variant_q8(nd);
+#ifdef ZK_Q8_WARPS
+    var.warps = ZK_Q8_WARPS;
+#endif
+#ifdef ZK_Q8_TARGET_STAGES
+    var.target_stages = ZK_Q8_TARGET_STAGES;
+#endif
     const PipeShape sh = q8_shape(nd, var.warps, var.target_stages);
     p.g = sh.g;
     p.row = sh.g.tile / kQB * kRec;
