@@ -41,7 +41,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SRC = os.path.join(ROOT, "zero_partitioned_optimizer_plan_b200", "csrc", "zero_kernels.cu")
+CSRC = os.path.join(ROOT, "zero_partitioned_optimizer_plan_b200", "csrc")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 METRIC = "fused ZeRO shard step params/sec"
 
@@ -452,14 +452,23 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def kernel_sources_sha256() -> str:
+    """One hash over every CUDA source of the library (the kernels the counters describe)."""
+    import glob
+    h = hashlib.sha256()
+    for path in sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))):
+        with open(path, "rb") as f:
+            h.update(os.path.basename(path).encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
 def traffic_per_launch(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
     kernel source; else None."""
     try:
         with open(TRAFFIC_FILE) as f:
             tab = json.load(f)
-        with open(KERNEL_SRC, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
+        sha = kernel_sources_sha256()
         ent = tab.get(workload, {}).get(kernel)
         if ent and ent.get("kernel_src_sha256") == sha:
             return ent["dram_bytes_per_launch"]
