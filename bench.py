@@ -66,6 +66,9 @@ def parse():
     ap.add_argument("--payload", choices=["fp16", "q8"], default="fp16",
                     help="q8: the owner reduces int8 payloads with one fp32 scale per 128 "
                          "elements (quantized once per rank before timing)")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="launch the per-bucket calls of a step strictly one after another "
+                         "(default: inside a zero_overlap_begin/end region)")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -153,6 +156,10 @@ class Workload:
         self.dominant_calls = len(self.ranges)
         self.side = None
         self.payload = args.payload
+        # the per-bucket calls of a step touch disjoint ranges: declare them independent
+        self.overlap = len(self.ranges) > 1 and not args.no_overlap
+        if len(self.ranges) > 1:
+            self.config["overlap"] = self.overlap
         if self.payload == "q8":
             self._quantize_payload()
 
@@ -217,10 +224,14 @@ class Workload:
                                        self.g_status)
             else:
                 self.g_status.zero_()
+            if self.overlap:
+                lz.zero_overlap_begin()
             for lo, hi in self.ranges:
                 lz.zero_step_fused_dc(hi - lo, self.nd, [g[lo:hi] for g in self.grads],
                                       *[x[lo:hi] for x in src], *[x[lo:hi] for x in dst],
                                       self.params[lo:hi], self.d_consts, self.g_status)
+            if self.overlap:
+                lz.zero_overlap_end()
             lz.zero_step_commit(self.n, *src, *dst, self.params, self.g_status)
             if dynamic:
                 lz.zero_scaler_update(self.d_scaler, self.scaler_prm, self.g_status)
@@ -289,10 +300,14 @@ class Workload:
         grads = grads or self.grads
         if ev is not None:
             ev[0].record()
+        if self.overlap:
+            lz.zero_overlap_begin()
         for lo, hi in self.ranges:
             lz.zero_step_fused(hi - lo, self.nd, [g[lo:hi] for g in grads],
                                *[x[lo:hi] for x in self.cur], *[x[lo:hi] for x in self.nxt],
                                self.params[lo:hi], self.hp, t, status)
+        if self.overlap:
+            lz.zero_overlap_end()
         if ev is not None:
             ev[1].record()
         lz.zero_step_commit(self.n, *self.cur, *self.nxt, self.params, status)
@@ -331,6 +346,7 @@ def _init_zero2(self, args, dev):
     self.shards = torch.empty(psi_p, dtype=torch.float32, device=dev)
     self.grads = None
     self.ranges = [(0, psi_p)]
+    self.overlap = False
     self.param_base = 0
     self.config = {"workload": args.workload, "psi": psi, "nd": nd, "stage": 2, "bucket": B,
                    "buckets": nb, "calls_per_step": nb + nd}

@@ -341,6 +341,30 @@ zero_status zero_step_fused_q8(uint64_t n, int nd, const uint8_t* const* rank_pa
 zero_status zero_selftest_timeout(uint32_t* d_status, zero_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Overlap of independent calls on one stream. The bulk-copy kernels of zero_step_fused(_dc),
+ * zero_step_fused_q8 and zero_reduce_scatter_bucket are launched with programmatic stream
+ * serialization: their CTAs may be scheduled while the kernel before them on the stream
+ * drains, but by default each waits for that kernel to complete before it touches global
+ * memory, so stream order is kept exactly.
+ * Between zero_overlap_begin(stream) and zero_overlap_end(stream) the caller declares those
+ * calls on `stream` mutually independent: none writes memory that another one of them reads
+ * or writes, except the shared status word, into which they only OR flags. The per-bucket
+ * calls of one step are such a set (disjoint ranges). Every such call after the region's first
+ * may then run alongside the calls before it, and each completes only after all earlier ones,
+ * so work enqueued after the region (zero_step_commit, a copy, an event) is ordered after the
+ * whole region as usual. Calls that take the plain-load kernels, and all other calls, stay
+ * ordered. Other work enqueued on the stream inside the region must be ordinary launches,
+ * copies or event waits (a kernel that itself uses programmatic dependent launch, as some
+ * libraries' kernels do, needs the region closed before it).
+ * Host-side state only (one flag per stream, thread-safe): both calls enqueue nothing and can
+ * be used while a CUDA graph is captured. The pages have no counterpart; this is a launch
+ * device of this library. Errors: ZERO_EINVAL (begin on a stream whose region is open, end on
+ * a stream without one).
+ * ---------------------------------------------------------------------------------------- */
+zero_status zero_overlap_begin(zero_stream_t stream);
+zero_status zero_overlap_end(zero_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * Stream-ordered bucket scheduler for stage 2. "ZeRO-2" card, "Gradient 생명주기": after a
  * bucket's reduce-scatter the GPU keeps its own reduced shard and releases the rest of the
  * local gradient. The local gradients of a bucket live in a staging slot (nd regions of

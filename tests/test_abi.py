@@ -297,3 +297,24 @@ def test_q8_rejects():
         with pytest.raises(lz.ZeroError) as e:
             lz.zero_step_fused_q8(1000, 2, pay, *ins, *outs, A + 120 * MB, HP, 1, A + 130 * MB, 0)
         assert e.value.code == code
+
+
+def test_overlap_region_bookkeeping():
+    """zero_overlap_begin/end keep one open region per stream and reject misuse; they touch
+    no device (host-side flags only)."""
+    s1, s2 = 0x1000, 0x2000
+    lz.zero_overlap_begin(s1)
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_overlap_begin(s1)                  # already open on this stream
+    assert e.value.code == lz.ZERO_EINVAL
+    lz.zero_overlap_begin(s2)                      # another stream is independent
+    lz.zero_overlap_end(s1)
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_overlap_end(s1)                    # closed already
+    assert e.value.code == lz.ZERO_EINVAL
+    with lz.overlap(s1):
+        pass
+    lz.zero_overlap_end(s2)
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_overlap_end(0)                     # never opened
+    assert e.value.code == lz.ZERO_EINVAL

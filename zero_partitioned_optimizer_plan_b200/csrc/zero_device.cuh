@@ -140,6 +140,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
+// ---------------------------------------------------------------------------------------------
+// programmatic dependent launch
+//
+// The pipeline kernels are launched with programmatic stream serialization allowed, so that a
+// kernel's CTAs can be scheduled while the kernel before it on the stream drains.
+//   ordered (default): wait for the previous kernel to complete and its writes to be visible,
+//     before the first global-memory access; then let the next kernel be scheduled. Stream
+//     order is kept exactly.
+//   chained (a later call of a zero_overlap_begin/end region, which the caller declares
+//     independent of the region's other calls): let the next kernel be scheduled at once, run,
+//     and wait for the previous kernel only before exiting. A kernel therefore completes only
+//     after every kernel before it, and the first ordinary launch after the region sees all of
+//     the region's writes.
+// Without the launch attribute both instructions are no-ops.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_enter(int chained) {
+    if (!chained) asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_leave(int chained) {
+    if (chained) asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -436,8 +460,19 @@ cudaError_t launch_pipe(K kernel, const A& args, const PipeShape& sh, cudaStream
     uint64_t grid = (uint64_t)di.sms * (uint64_t)bps;
     if (args.num_tiles < grid) grid = args.num_tiles;
     if (grid < 1) grid = 1;
-    kernel<<<(unsigned)grid, threads, sh.smem, stream>>>(args);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = sh.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kernel, args);
     count_launch();
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

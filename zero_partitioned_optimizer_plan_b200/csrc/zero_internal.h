@@ -56,6 +56,11 @@ cudaError_t launch_scaler_prepare(const zero_scaler_state* st, const AdamConsts*
 cudaError_t launch_scaler_update(zero_scaler_state* st, const zero_scaler_params& prm,
                                  const uint32_t* status, cudaStream_t stream);
 
+// Whether the pipeline launch about to be made on `stream` may be chained to the previous one
+// (a later call inside a zero_overlap_begin/end region); the first call of a region, and every
+// call outside one, is ordered (zero_api.cpp).
+bool overlap_next(cudaStream_t stream);
+
 // Count of kernels this library has launched in this process.
 void count_launch();
 uint64_t launches();

@@ -6,13 +6,15 @@
 // HBM bandwidth, and the design is about keeping enough bytes in flight:
 //
 //   * persistent grid, one CTA per SM, tiles of T elements taken round-robin;
-//   * one elected producer thread per CTA streams each tile's Nd gradient rows and three state
-//     rows into a ring of shared-memory stages with 1-D bulk async copies
-//     (cp.async.bulk ... mbarrier::complete_tx, no multicast), so 100-200 KB per SM are in
-//     flight without spending registers on it;
-//   * eight consumer warps sum the Nd rows in rank order in fp32, release the stage, then
-//     run Adam and store fp32 state and fp16 parameters straight from registers;
-//   * a warp vote collects the overflow (inf/NaN) check, one atomicOr per warp at the end.
+//   * one producer warp per CTA streams each tile's Nd gradient rows and three state rows into
+//     a ring of shared-memory stages with 1-D bulk async copies (cp.async.bulk ...
+//     mbarrier::complete_tx, no multicast), so 100-200 KB per SM are in flight without
+//     spending registers on it;
+//   * 16-24 consumer warps (by Nd) sum the Nd rows in rank order in fp32, release the stage,
+//     then run Adam and store fp32 state and fp16 parameters straight from registers;
+//   * a warp vote collects the overflow (inf/NaN) check, one atomicOr per warp at the end;
+//   * programmatic dependent launch lets the next call's CTAs start while this one drains
+//     (ordered by default; overlapped inside a zero_overlap_begin/end region).
 //
 // Every wait on an mbarrier is bounded (1 s); on expiry the kernel sets ZERO_FLAG_TIMEOUT,
 // lets its own copies in flight land, and returns.
@@ -61,6 +63,7 @@ struct FusedArgs {
     const AdamConsts* ad;  // when not null: the constants, read from device memory at run time
     MeanConsts mc;
     int selftest_no_copies;  // self-test only: the producer issues nothing (waits must expire)
+    int chained;         // programmatic launch chained to the previous call (see pdl_enter)
 };
 
 struct RsArgs {
@@ -76,6 +79,7 @@ struct RsArgs {
     Geom g;
     int nd;
     MeanConsts mc;
+    int chained;         // programmatic launch chained to the previous call (see pdl_enter)
 };
 
 struct CommitArgs {
@@ -206,9 +210,11 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
     uint64_t* empty = full + kMaxStages;
     uint8_t* data = smem + kDataOffset;
     init_barriers(full, empty, p.g.stages, W);
+    pdl_enter(p.chained);
 
     if ((threadIdx.x >> 5) == W) {
         if (!p.selftest_no_copies) produce<true>(p, full, empty, data);
+        pdl_leave(p.chained);
         return;
     }
 
@@ -254,6 +260,7 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
     if (blockIdx.x == 0 && (uint64_t)threadIdx.x < p.n - p.n_tiled)
         fused_element(p, a, p.n_tiled + threadIdx.x, bad);
     flag_overflow(bad, p.status);
+    pdl_leave(p.chained);
 }
 
 // plain-load variant for ranges whose pointers are not 16-byte aligned (or tiny ranges)
@@ -307,9 +314,11 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
     uint64_t* empty = full + kMaxStages;
     uint8_t* data = smem + kDataOffset;
     init_barriers(full, empty, p.g.stages, W);
+    pdl_enter(p.chained);
 
     if ((threadIdx.x >> 5) == W) {
         produce<false>(p, full, empty, data);
+        pdl_leave(p.chained);
         return;
     }
 
@@ -356,6 +365,7 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
     if (blockIdx.x == 0 && (uint64_t)threadIdx.x < p.n - p.n_tiled)
         rs_element(p, p.n_tiled + threadIdx.x, bad);
     flag_overflow(bad, p.status);
+    pdl_leave(p.chained);
 }
 
 __global__ void __launch_bounds__(256) rs_plain_kernel(const __grid_constant__ RsArgs p) {
@@ -589,6 +599,7 @@ cudaError_t launch_fused(uint64_t n, int nd, const uint16_t* const* grads, const
     p.g = sh.g;
     p.n_tiled = n & ~(uint64_t)7;
     p.num_tiles = (p.n_tiled + sh.g.tile - 1) / sh.g.tile;
+    p.chained = overlap_next(stream) ? 1 : 0;
     if (ad) {
         switch (sh.warps) {
             case 16: return launch_pipe(fused_tma_kernel<kElems, 16, true>, p, sh, stream);
@@ -635,6 +646,7 @@ cudaError_t launch_reduce_scatter(uint64_t n, int nd, const uint16_t* const* gra
     p.g = sh.g;
     p.n_tiled = n & ~(uint64_t)7;
     p.num_tiles = (p.n_tiled + sh.g.tile - 1) / sh.g.tile;
+    p.chained = overlap_next(stream) ? 1 : 0;
     switch (sh.warps) {
         case 16: return launch_pipe(rs_tma_kernel<kElems, 16>, p, sh, stream);
         case 20: return launch_pipe(rs_tma_kernel<kElems, 20>, p, sh, stream);

@@ -133,6 +133,7 @@ struct FusedQ8Args {
     int param_vec;
     AdamConsts a;
     MeanConsts mc;
+    int chained;         // programmatic launch chained to the previous call (see pdl_enter)
 };
 
 // acc + float(q) * scale with one rounding
@@ -238,8 +239,10 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
     uint64_t* empty = full + kMaxStages;
     uint8_t* data = smem + kDataOffset;
     init_barriers(full, empty, p.g.stages, W);
+    pdl_enter(p.chained);
     if ((threadIdx.x >> 5) == W) {
         produce_q8(p, full, empty, data);
+        pdl_leave(p.chained);
         return;
     }
     const int lane = threadIdx.x & 31;
@@ -312,6 +315,7 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
     if (blockIdx.x == 0 && (uint64_t)threadIdx.x < p.n - p.n_tiled)
         fused_q8_element(p, p.n_tiled + threadIdx.x, bad);
     flag_overflow(bad, p.status);
+    pdl_leave(p.chained);
 }
 
 __global__ void __launch_bounds__(256) fused_q8_plain_kernel(const __grid_constant__ FusedQ8Args p) {
@@ -422,6 +426,7 @@ cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,
     p.row = sh.g.tile / kQB * kRec;
     p.n_tiled = n & ~(kQTileAlign - 1);
     p.num_tiles = (p.n_tiled + sh.g.tile - 1) / sh.g.tile;
+    p.chained = overlap_next(stream) ? 1 : 0;
     switch (sh.warps) {
         case 16: return launch_pipe(fused_q8_tma_kernel<16>, p, sh, stream);
         case 20: return launch_pipe(fused_q8_tma_kernel<20>, p, sh, stream);

@@ -48,6 +48,7 @@ SYMBOLS = (
     "zero_step_status", "zero_adam_consts_for_step", "zero_adam_shard_dc", "zero_step_fused_dc",
     "zero_selftest_timeout", "zero_adam_consts_table", "zero_scaler_prepare",
     "zero_scaler_update", "zero_quantize_q8", "zero_step_fused_q8",
+    "zero_overlap_begin", "zero_overlap_end",
     "zero_sched_slot_elems", "zero_sched_create", "zero_sched_begin_bucket",
     "zero_sched_end_bucket", "zero_sched_wait", "zero_sched_launches", "zero_sched_destroy",
 )
@@ -142,6 +143,8 @@ def _load():
     L.zero_adam_consts_table.argtypes = [P(_HP), i64, i64, P(AdamConsts)]
     L.zero_scaler_prepare.argtypes = [vp, vp, i64, vp, vp, vp]
     L.zero_scaler_update.argtypes = [vp, P(ScalerParams), vp, vp]
+    L.zero_overlap_begin.argtypes = [vp]
+    L.zero_overlap_end.argtypes = [vp]
     L.zero_sched_slot_elems.argtypes = [vp, i32, P(u64)]
     L.zero_sched_create.argtypes = [vp, vp, u64, i32, P(vp), vp, vp, P(vp)]
     L.zero_sched_begin_bucket.argtypes = [vp, i32, vp, P(vp)]
@@ -367,6 +370,29 @@ def zero_scaler_update(d_state, params: ScalerParams, d_status, stream=None):
 
 def zero_selftest_timeout(d_status, stream=None):
     _check(_lib.zero_selftest_timeout(_ptr(d_status, 4), _stream(stream)), "zero_selftest_timeout")
+
+
+def zero_overlap_begin(stream=None):
+    _check(_lib.zero_overlap_begin(_stream(stream)), "zero_overlap_begin")
+
+
+def zero_overlap_end(stream=None):
+    _check(_lib.zero_overlap_end(_stream(stream)), "zero_overlap_end")
+
+
+class overlap:
+    """Context manager: zero_overlap_begin(stream) ... zero_overlap_end(stream)."""
+
+    def __init__(self, stream=None):
+        self.stream = _stream(stream)
+
+    def __enter__(self):
+        zero_overlap_begin(self.stream)
+        return self
+
+    def __exit__(self, *exc):
+        zero_overlap_end(self.stream)
+        return False
 
 
 # ---------------------------------------------------------------------------------------------
