@@ -62,6 +62,41 @@ def test_fused_step_vs_oracle(n, nd):
     print(f"PARITY fused n={n} nd={nd}: max ulp fp32 {worst[0]}, fp16 {worst[1]}")
 
 
+def _large_shape_elems(nd):
+    """Smallest call that takes the large (per-Nd table) pipeline shape rather than the
+    small-call shape, plus a ragged remainder: tiles of 32 * warps * 4 elements, at least 32
+    tiles per SM at Nd <= 2 and 4 above."""
+    warps = 20 if nd <= 2 else 16 if nd <= 4 else 24 if nd <= 8 else 16 if nd <= 16 else 20
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    return (32 if nd <= 2 else 4) * sms * 32 * warps * 4 + 1000 + 5
+
+
+@pytest.mark.parametrize("nd", [1, 2, 4, 8, 16, 64])
+def test_fused_step_large_shape_vs_oracle(nd):
+    """The large shape (full shared-memory budget, 16-24 consumer warps, every SM busy) on
+    every element of a call just above its threshold, two steps."""
+    n = _large_shape_elems(nd)
+    seed = 7000 + nd
+    master, m, v = synth.state_warm(n, seed=seed)
+    pp = PingPong(master, m, v)
+    w_ref, m_ref, v_ref = master.numpy(), m.numpy(), v.numpy()
+    params = torch.empty(n, dtype=torch.float16, device=DEV)
+    for t in (1, 2):
+        g_cpu = _rank_grads_cpu(n, nd, seed, t, spike=0.01)
+        st = status_word()
+        fused_step(n, [g.to(DEV) for g in g_cpu], pp, params, HP, t, st)
+        torch.cuda.synchronize()
+        assert status_flags(st) == 0
+        pp.swap()
+        skipped, w_ref, m_ref, v_ref, p_ref = oracle.step([g.numpy() for g in g_cpu], w_ref,
+                                                          m_ref, v_ref, ORC_HP, t)
+        w, mm, vv = pp.numpy()
+        check_f32("master", w, w_ref)
+        check_f32("m", mm, m_ref)
+        check_f32("v", vv, v_ref)
+        check_f16("param", f16np(params), p_ref)
+
+
 @pytest.mark.parametrize("nd", [1, 3, 4, 16, 64])
 @pytest.mark.parametrize("numels,bucket", [([1000, 37, 4099, 12345], 0),
                                            ([1000, 37, 4099, 12345], 4096),

@@ -33,6 +33,12 @@ namespace {
 #ifndef ZK_ADAM_UNROLL     // float4 groups per thread and iteration of the plain owner update
 #define ZK_ADAM_UNROLL 2
 #endif
+// Small calls take a shape with fewer consumer warps and ZK_SMALL_BUDGET bytes of stages,
+// launched one CTA per SM, so that two CTAs fit on an SM and the next call's CTAs load while
+// this call's finish (pick_small_variant).
+#ifndef ZK_SMALL_BUDGET
+#define ZK_SMALL_BUDGET (100 * 1024)
+#endif
 
 constexpr int kMaxRanks = ZERO_MAX_RANKS;
 constexpr int kElems = 4;                        // elements per consumer thread and tile
@@ -46,6 +52,8 @@ struct Warps {
     static constexpr int kConsumerWarps = W;
     static constexpr int kConsumerThreads = W * 32;
     static constexpr int kThreads = W * 32 + 32;   // + one producer warp
+    // up to 12 consumer warps (the small-call shapes), two CTAs must fit on an SM
+    static constexpr int kMinBlocks = W <= 12 ? 2 : 1;
 };
 
 // Shape of the shared-memory pipeline of one launch (see "the pipeline" below).
@@ -436,7 +444,8 @@ cudaError_t pipe_blocks_per_sm(K kernel, int threads, size_t smem, int* out) {
 struct PipeShape {
     Geom g;
     size_t smem;
-    int warps;       // consumer warps
+    int warps;        // consumer warps
+    int grid_per_sm;  // CTAs per SM in the grid (0: as many as fit)
 };
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -457,6 +466,7 @@ cudaError_t launch_pipe(K kernel, const A& args, const PipeShape& sh, cudaStream
     int bps = 1;
     e = pipe_blocks_per_sm(kernel, threads, sh.smem, &bps);
     if (e != cudaSuccess) return e;
+    if (sh.grid_per_sm > 0 && sh.grid_per_sm < bps) bps = sh.grid_per_sm;
     uint64_t grid = (uint64_t)di.sms * (uint64_t)bps;
     if (args.num_tiles < grid) grid = args.num_tiles;
     if (grid < 1) grid = 1;
@@ -497,6 +507,26 @@ Variant pick_variant(int nd) {
     if (nd <= 8) return {24, 3};
     if (nd <= 16) return {16, 2};
     return {20, 2};
+}
+
+// The small-call shape, also measured on B200 (graph-captured chains of 1 MiB and 16 MiB
+// bucket calls in an overlap region): 12 consumer warps up to Nd = 8, 8 above; a call takes it
+// when the large shape would give each SM fewer than `max_tiles_per_sm` tiles (at Nd <= 2 the
+// ramp and tail of a launch weigh more, so calls up to 32 tiles per SM gain from it).
+struct SmallVariant {
+    int warps;
+    int max_tiles_per_sm;
+};
+
+SmallVariant pick_small_variant(int nd) {
+    SmallVariant v{nd <= 8 ? 12 : 8, nd <= 2 ? 32 : 4};
+#ifdef ZK_SMALL_WARPS
+    v.warps = ZK_SMALL_WARPS;
+#endif
+#ifdef ZK_SMALL_TILES_PER_SM
+    v.max_tiles_per_sm = ZK_SMALL_TILES_PER_SM;
+#endif
+    return v;
 }
 
 }  // namespace

@@ -203,7 +203,7 @@ __device__ __forceinline__ void fused_element(const FusedArgs& p, const AdamCons
 }
 
 template <int E, int W, bool kDC>
-__global__ void __launch_bounds__(Warps<W>::kThreads, 1)
+__global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
     fused_tma_kernel(const __grid_constant__ FusedArgs p) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -307,7 +307,7 @@ __device__ __forceinline__ void rs_element(const RsArgs& p, uint64_t i, bool& ba
 }
 
 template <int E, int W>
-__global__ void __launch_bounds__(Warps<W>::kThreads, 1)
+__global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
     rs_tma_kernel(const __grid_constant__ RsArgs p) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -505,28 +505,55 @@ std::atomic<uint64_t> g_launches{0};
 
 // Tile = 32 * warps * kElems elements; as many rank rows per stage as leave target_stages
 // stages inside the shared-memory budget, the ranks split evenly into chunks.
-PipeShape pipe_shape(int nd, bool with_state) {
-    const Variant var = pick_variant(nd);
+PipeShape make_shape(int nd, bool with_state, int warps, int target_stages, size_t budget) {
     PipeShape sh;
-    sh.warps = var.warps;
+    sh.warps = warps;
+    sh.grid_per_sm = 0;
     Geom& g = sh.g;
-    g.tile = (uint32_t)(32 * var.warps * kElems);
+    g.tile = (uint32_t)(32 * warps * kElems);
     const size_t row = (size_t)g.tile * 2u;
     const size_t state = with_state ? (size_t)g.tile * 12u : 0u;
-    const size_t per_stage = kSmemBudget / (size_t)var.target_stages;
+    const size_t per_stage = budget / (size_t)target_stages;
     size_t rc_max = per_stage > state + row ? (per_stage - state) / row : 1;
     if (rc_max > (size_t)nd) rc_max = (size_t)nd;
     g.nchunks = (uint32_t)(((size_t)nd + rc_max - 1) / rc_max);
     g.rc = (uint32_t)(((size_t)nd + g.nchunks - 1) / g.nchunks);
     g.state_off = (uint32_t)(g.rc * row);
     g.stage_bytes = (uint32_t)(g.state_off + state);
-    size_t st = kSmemBudget / g.stage_bytes;
+    size_t st = budget / g.stage_bytes;
     if (st < 2) st = 2;
     if (st > kMaxStages) st = kMaxStages;
     g.stages = (int)st;
     sh.smem = (size_t)kDataOffset + st * g.stage_bytes;
     return sh;
 }
+
+// The shape of a call over n elements: the per-Nd table, or for a call too small to give
+// every SM several tiles, the small shape (one CTA per SM, room for a second CTA of the next
+// call on the same SM).
+PipeShape pipe_shape(int nd, bool with_state, uint64_t n, int sms) {
+    const Variant var = pick_variant(nd);
+    const SmallVariant small = pick_small_variant(nd);
+    const uint64_t big_tile = 32ull * (uint64_t)var.warps * kElems;
+    const uint64_t tiles = (n + big_tile - 1) / big_tile;
+    if (tiles < (uint64_t)small.max_tiles_per_sm * (uint64_t)sms) {
+        PipeShape sh = make_shape(nd, with_state, small.warps, 2, ZK_SMALL_BUDGET);
+        sh.grid_per_sm = 1;
+        return sh;
+    }
+    return make_shape(nd, with_state, var.warps, var.target_stages, kSmemBudget);
+}
+
+// Launch a bulk-copy kernel template instantiated for the shape's number of consumer warps.
+#define ZK_LAUNCH_BY_WARPS(KERNEL, ...)                                                    \
+    switch (sh.warps) {                                                                    \
+        case 8: return launch_pipe(KERNEL<kElems, 8 __VA_ARGS__>, p, sh, stream);          \
+        case 12: return launch_pipe(KERNEL<kElems, 12 __VA_ARGS__>, p, sh, stream);        \
+        case 16: return launch_pipe(KERNEL<kElems, 16 __VA_ARGS__>, p, sh, stream);        \
+        case 20: return launch_pipe(KERNEL<kElems, 20 __VA_ARGS__>, p, sh, stream);        \
+        case 24: return launch_pipe(KERNEL<kElems, 24 __VA_ARGS__>, p, sh, stream);        \
+    }                                                                                      \
+    return cudaErrorInvalidConfiguration
 
 }  // namespace
 
@@ -544,15 +571,13 @@ cudaError_t launch_selftest_timeout(uint32_t* status, cudaStream_t stream) {
     p.n_tiled = 4096;
     p.selftest_no_copies = 1;
     p.mc = make_mean(1);
-    const PipeShape sh = pipe_shape(1, true);
+    DevInfo di;
+    cudaError_t e = dev_info(&di);
+    if (e != cudaSuccess) return e;
+    const PipeShape sh = pipe_shape(1, true, p.n, di.sms);
     p.g = sh.g;
     p.num_tiles = 1;
-    switch (sh.warps) {
-        case 16: return launch_pipe(fused_tma_kernel<kElems, 16, false>, p, sh, stream);
-        case 20: return launch_pipe(fused_tma_kernel<kElems, 20, false>, p, sh, stream);
-        case 24: return launch_pipe(fused_tma_kernel<kElems, 24, false>, p, sh, stream);
-    }
-    return cudaErrorInvalidConfiguration;
+    ZK_LAUNCH_BY_WARPS(fused_tma_kernel, , false);
 }
 
 uint64_t launches() { return g_launches.load(std::memory_order_relaxed); }
@@ -595,25 +620,15 @@ cudaError_t launch_fused(uint64_t n, int nd, const uint16_t* const* grads, const
         count_launch();
         return cudaGetLastError();
     }
-    const PipeShape sh = pipe_shape(nd, true);
+    const PipeShape sh = pipe_shape(nd, true, n, di.sms);
     p.g = sh.g;
     p.n_tiled = n & ~(uint64_t)7;
     p.num_tiles = (p.n_tiled + sh.g.tile - 1) / sh.g.tile;
     p.chained = overlap_next(stream) ? 1 : 0;
     if (ad) {
-        switch (sh.warps) {
-            case 16: return launch_pipe(fused_tma_kernel<kElems, 16, true>, p, sh, stream);
-            case 20: return launch_pipe(fused_tma_kernel<kElems, 20, true>, p, sh, stream);
-            case 24: return launch_pipe(fused_tma_kernel<kElems, 24, true>, p, sh, stream);
-        }
-    } else {
-        switch (sh.warps) {
-            case 16: return launch_pipe(fused_tma_kernel<kElems, 16, false>, p, sh, stream);
-            case 20: return launch_pipe(fused_tma_kernel<kElems, 20, false>, p, sh, stream);
-            case 24: return launch_pipe(fused_tma_kernel<kElems, 24, false>, p, sh, stream);
-        }
+        ZK_LAUNCH_BY_WARPS(fused_tma_kernel, , true);
     }
-    return cudaErrorInvalidConfiguration;
+    ZK_LAUNCH_BY_WARPS(fused_tma_kernel, , false);
 }
 
 cudaError_t launch_reduce_scatter(uint64_t n, int nd, const uint16_t* const* grads,
@@ -642,17 +657,12 @@ cudaError_t launch_reduce_scatter(uint64_t n, int nd, const uint16_t* const* gra
         count_launch();
         return cudaGetLastError();
     }
-    const PipeShape sh = pipe_shape(nd, false);
+    const PipeShape sh = pipe_shape(nd, false, n, di.sms);
     p.g = sh.g;
     p.n_tiled = n & ~(uint64_t)7;
     p.num_tiles = (p.n_tiled + sh.g.tile - 1) / sh.g.tile;
     p.chained = overlap_next(stream) ? 1 : 0;
-    switch (sh.warps) {
-        case 16: return launch_pipe(rs_tma_kernel<kElems, 16>, p, sh, stream);
-        case 20: return launch_pipe(rs_tma_kernel<kElems, 20>, p, sh, stream);
-        case 24: return launch_pipe(rs_tma_kernel<kElems, 24>, p, sh, stream);
-    }
-    return cudaErrorInvalidConfiguration;
+    ZK_LAUNCH_BY_WARPS(rs_tma_kernel);
 }
 
 cudaError_t launch_adam(uint64_t n, const float* grad, float* master, float* m, float* v,

@@ -339,6 +339,7 @@ Variant pick_variant_q8(int nd) {
 PipeShape q8_shape(int nd, int warps, int target_stages) {
     PipeShape sh;
     sh.warps = warps;
+    sh.grid_per_sm = 0;
     Geom& g = sh.g;
     g.tile = (uint32_t)(32 * warps * kElems);
     const size_t row = (size_t)g.tile / kQB * kRec;
