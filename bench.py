@@ -478,6 +478,15 @@ def kernel_sources_sha256() -> str:
     return h.hexdigest()
 
 
+def traffic_key(wl) -> str:
+    """Key of a workload's entry in the traffic table: workload and Nd, and the bucket size
+    when a step is several calls (a launch's bytes depend on it)."""
+    key = f"{wl.config['workload']}_nd{wl.nd}"
+    if wl.config.get("calls_per_step", 1) > 1 and "bucket" in wl.config:
+        key += f"_b{wl.config['bucket']}"
+    return key
+
+
 def traffic_per_launch(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
     kernel source; else None."""
@@ -649,8 +658,7 @@ def run_ours(args):
     achieved = bytes_per_launch / launch_s / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": peak_kind,
-                "traffic": traffic_per_launch(wl.dominant,
-                                              f"{wl.config['workload']}_nd{wl.nd}"),
+                "traffic": traffic_per_launch(wl.dominant, traffic_key(wl)),
                 "kernel": wl.dominant, "bytes_per_launch": bytes_per_launch,
                 "kernel_ms_mean": launch_s * 1e3}
     if wl.side is not None:   # the other kernel of the step (or the senders' quantization)
