@@ -214,8 +214,11 @@ def test_7p5b_shard_view(big_7p5b, owner):
 @pytest.mark.parametrize("nd", [2, 4, 8, 16, 64])
 def test_flat_sweep_bucketed_calls(nd):
     """Psi = 2^29 flat buffer, one fused call per bucket of B in {2^19, 2^23, 2^26, 2^29}
-    elements (1 MB ... 1 GB of fp16 gradient per rank) in backward order, then one commit;
-    every bucketing gives the oracle's step on the sample."""
+    elements (1 MB ... 1 GB of fp16 gradient per rank) in backward order inside an overlap
+    region, then one commit -- the launch configuration bench.py times, eagerly and, for the
+    two smaller bucket sizes, as a CUDA-graph replay of zero_step_fused_dc calls (outputs
+    poisoned with NaN before the replay); every bucketing gives the oracle's step on the
+    sample."""
     psi = 1 << 29
     grads = [synth.grad_f16(psi, 1e-3, seed=5, rank=r, step=nd, device=DEV) for r in range(nd)]
     init = list(synth.state_warm(psi, seed=50 + nd, device=DEV))
@@ -227,21 +230,55 @@ def test_flat_sweep_bucketed_calls(nd):
     assert not skipped
     params = torch.empty(psi, dtype=torch.float16, device=DEV)
     nxt = [torch.empty_like(x) for x in init]
+    c = lz.zero_adam_consts_for_step(HP, 1)
+    d_consts = torch.frombuffer(bytearray(bytes(c)), dtype=torch.uint8).to(DEV)
     for B in (1 << 19, 1 << 23, 1 << 26, 1 << 29):
-        st = status_word()
+        ranges = []
         hi = psi
-        calls = 0
         while hi > 0:
-            lo = max(0, hi - B)
-            lz.zero_step_fused(hi - lo, nd, [g[lo:hi] for g in grads], *[x[lo:hi] for x in init],
-                               *[x[lo:hi] for x in nxt], params[lo:hi], HP, 1, st)
-            hi = lo
-            calls += 1
-        lz.zero_step_commit(psi, *init, *nxt, params, st)
-        torch.cuda.synchronize()
-        assert status_flags(st) == 0 and calls == psi // B
-        check_f32(f"B={B} master", gather(nxt[0], idx_dev), w)
-        check_f32(f"B={B} m", gather(nxt[1], idx_dev), mm)
-        check_f32(f"B={B} v", gather(nxt[2], idx_dev), vv)
-        check_f16(f"B={B} params", gather(params, idx_dev), p)
-    print(f"PARITY flat 2^29 Nd={nd}: 4 bucket sizes, {idx.size} sampled elements")
+            ranges.append((max(0, hi - B), hi))
+            hi = max(0, hi - B)
+        assert len(ranges) == psi // B
+        st = status_word()
+
+        def step(dc):
+            st.zero_()
+            with lz.overlap():
+                for lo, hi in ranges:
+                    if dc:
+                        lz.zero_step_fused_dc(hi - lo, nd, [g[lo:hi] for g in grads],
+                                              *[x[lo:hi] for x in init], *[x[lo:hi] for x in nxt],
+                                              params[lo:hi], d_consts, st)
+                    else:
+                        lz.zero_step_fused(hi - lo, nd, [g[lo:hi] for g in grads],
+                                           *[x[lo:hi] for x in init], *[x[lo:hi] for x in nxt],
+                                           params[lo:hi], HP, 1, st)
+            lz.zero_step_commit(psi, *init, *nxt, params, st)
+
+        modes = ["eager", "graph"] if B <= 1 << 23 else ["eager"]
+        for mode in modes:
+            if mode == "eager":
+                step(False)
+            else:
+                side = torch.cuda.Stream()
+                side.wait_stream(torch.cuda.current_stream())
+                with torch.cuda.stream(side):
+                    step(True)
+                torch.cuda.current_stream().wait_stream(side)
+                torch.cuda.synchronize()
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph):
+                    step(True)
+                for x in nxt:
+                    x.fill_(float("nan"))
+                params.fill_(float("nan"))
+                graph.replay()
+            torch.cuda.synchronize()
+            assert status_flags(st) == 0
+            check_f32(f"B={B} {mode} master", gather(nxt[0], idx_dev), w)
+            check_f32(f"B={B} {mode} m", gather(nxt[1], idx_dev), mm)
+            check_f32(f"B={B} {mode} v", gather(nxt[2], idx_dev), vv)
+            check_f16(f"B={B} {mode} params", gather(params, idx_dev), p)
+            if mode == "graph":
+                del graph
+    print(f"PARITY flat 2^29 Nd={nd}: 4 bucket sizes (2 also by graph), {idx.size} sampled elements")
