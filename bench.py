@@ -66,6 +66,9 @@ def parse():
     ap.add_argument("--payload", choices=["fp16", "q8"], default="fp16",
                     help="q8: the owner reduces int8 payloads with one fp32 scale per 128 "
                          "elements (quantized once per rank before timing)")
+    ap.add_argument("--stage2-fused", action="store_true",
+                    help="stage-2 workloads: the bucket scheduler launches the fused step per "
+                         "bucket (zero_sched_create_fused) instead of reduce-scatter + update")
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch the per-bucket calls of a step strictly one after another "
                          "(default: inside a zero_overlap_begin/end region)")
@@ -350,6 +353,22 @@ def _init_zero2(self, args, dev):
     self.param_base = 0
     self.config = {"workload": args.workload, "psi": psi, "nd": nd, "stage": 2, "bucket": B,
                    "buckets": nb, "calls_per_step": nb + nd}
+    if args.stage2_fused:
+        # the scheduler launches the fused step per bucket; ping-pong state, commit at the end
+        self.cur = [self.master, self.m, self.v]
+        self.nxt = [torch.empty_like(x) for x in self.cur]
+        self.d_consts = torch.empty(40, dtype=torch.uint8, device=dev)
+        self.h_consts = [torch.empty(40, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
+        self.h_done = [None, None]
+        self.config["workload"] = args.workload + "_fused"
+        self.config["calls_per_step"] = nb + 1
+        self.bytes_per_step = (2 * nd + 26) * psi_p
+        self.dominant = "fused_tma_kernel"
+        self.dominant_bytes = self.bytes_per_step
+        self.dominant_calls = nb
+        self.side = None
+        self.step = self._step_zero2_fused
+        return
     rs_bytes = (2 * nd + 4) * psi_p
     adam_bytes = 30 * psi_p
     self.bytes_per_step = rs_bytes + adam_bytes
@@ -389,8 +408,32 @@ def _step_zero2(self, t, status, ev=None, grads=None):
     lz.zero_sched_destroy(sch)
 
 
+def _step_zero2_fused(self, t, status, ev=None, grads=None):
+    """Stage 2 with the fused step per bucket: the scheduler launches each bucket's fused
+    kernel as the bucket arrives (its slot released after it), then one commit."""
+    lz, torch = self.lz, self.torch
+    if grads is not None:
+        raise ValueError("the stage-2 workload has no host-buffer variant")
+    stream = torch.cuda.current_stream()
+    self._load_consts(t)
+    sch = lz.zero_sched_create_fused(self.plan, self.slots, self.slot_elems, self.nb, *self.cur,
+                                     *self.nxt, self.params, self.d_consts, status, stream)
+    if ev is not None:
+        ev[0].record()
+    for k in range(self.nb):
+        lz.zero_sched_begin_bucket(sch, k, stream)
+        lz.zero_sched_end_bucket(sch, k, stream)
+    lz.zero_sched_wait(sch, stream)
+    if ev is not None:
+        ev[1].record()
+    lz.zero_step_commit(self.n, *self.cur, *self.nxt, self.params, status)
+    lz.zero_sched_destroy(sch)
+    self.cur, self.nxt = self.nxt, self.cur
+
+
 Workload._init_zero2 = _init_zero2
 Workload._step_zero2 = _step_zero2
+Workload._step_zero2_fused = _step_zero2_fused
 
 
 # ---------------------------------------------------------------------------------------------

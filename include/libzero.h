@@ -385,16 +385,35 @@ zero_status zero_sched_slot_elems(const zero_plan* plan, int n_slots, uint64_t* 
 zero_status zero_sched_create(const zero_plan* plan, uint16_t* slot_mem, uint64_t slot_mem_elems,
                               int n_slots, float* const* owner_grad_shards, uint32_t* d_status,
                               zero_stream_t rs_stream, zero_sched** out);
+/* Fused mode: the kernel launched for bucket k (on `stream`) is the fused step over the
+ * bucket's range [lo, lo+len) of the flat padded buffer -- rank-ordered reduction, unscale,
+ * Adam, fp16 cast and write-back, as zero_step_fused_dc with the step's constants read from
+ * d_consts -- so the reduced gradient never reaches memory (the survey's a7 applied to stage 2,
+ * bucket by bucket, with the same release of each slot after its kernel). master_in/m_in/v_in
+ * and master_out/m_out/v_out: psi_p fp32 values each (flat, padded), param_out: psi_p fp16
+ * values; they stay fixed for the scheduler's life (with ping-pong state, create one per
+ * step). After the last bucket the caller makes its stream wait (zero_sched_wait) and calls
+ * zero_step_commit over all psi_p elements, which skips the whole step if any bucket
+ * overflowed. Errors: as zero_sched_create, and ZERO_EINVAL for outputs that overlap the
+ * inputs, each other or the staging slots. The pages' stage 2 keeps the reduced shard in
+ * memory for a later optimizer step; this mode is this library's fusion of the two. */
+zero_status zero_sched_create_fused(const zero_plan* plan, uint16_t* slot_mem,
+                                    uint64_t slot_mem_elems, int n_slots, const float* master_in,
+                                    const float* m_in, const float* v_in, float* master_out,
+                                    float* m_out, float* v_out, uint16_t* param_out,
+                                    const zero_adam_consts* d_consts, uint32_t* d_status,
+                                    zero_stream_t stream, zero_sched** out);
 /* Choose the slot for bucket k, make `producer` wait until that slot is released, and write
  * the nd device pointers (rank r's region, bucket k's len values) the producer must fill. */
 zero_status zero_sched_begin_bucket(zero_sched* s, int k, zero_stream_t producer,
                                     uint16_t** rank_ptrs);
-/* The producer has enqueued the fill of bucket k on `producer`: the reduce-scatter of
- * bucket k is enqueued on rs_stream after it, followed by the release of its slot. */
+/* The producer has enqueued the fill of bucket k on `producer`: the bucket's kernel (the
+ * reduce-scatter, or the fused step in fused mode) is enqueued on the scheduler's stream after
+ * it, followed by the release of its slot. */
 zero_status zero_sched_end_bucket(zero_sched* s, int k, zero_stream_t producer);
 /* Make `stream` wait for every reduce-scatter enqueued so far (e.g. before zero_adam_shard). */
 zero_status zero_sched_wait(zero_sched* s, zero_stream_t stream);
-/* Number of reduce-scatter kernels the scheduler has launched since creation. */
+/* Number of bucket kernels (reduce-scatter or fused) the scheduler has launched since creation. */
 zero_status zero_sched_launches(const zero_sched* s, uint64_t* count);
 void zero_sched_destroy(zero_sched* s);
 

@@ -318,3 +318,35 @@ def test_overlap_region_bookkeeping():
     with pytest.raises(lz.ZeroError) as e:
         lz.zero_overlap_end(0)                     # never opened
     assert e.value.code == lz.ZERO_EINVAL
+
+
+def test_fused_scheduler_rejects():
+    """zero_sched_create_fused checks the plan, the state arrays (psi_p values each), the
+    constants pointer and that no output overlaps an input, another output or the slots."""
+    pl = lz.zero_plan_create([100, 28], 4, 2, 32)     # psi_p = 128
+    need = lz.zero_sched_slot_elems(pl, 2)
+    slots = A
+    ins = [A + 10 * MB, A + 11 * MB, A + 12 * MB]
+    outs = [A + 20 * MB, A + 21 * MB, A + 22 * MB]
+    par, dc, st = A + 30 * MB, A + 31 * MB, A + 32 * MB
+    ok = dict(master_in=ins[0], m_in=ins[1], v_in=ins[2], master_out=outs[0], m_out=outs[1],
+              v_out=outs[2], param_out=par, d_consts=dc, d_status=st)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lz.zero_sched_create_fused(pl, slots, need, 2, a["master_in"], a["m_in"],
+                                          a["v_in"], a["master_out"], a["m_out"], a["v_out"],
+                                          a["param_out"], a["d_consts"], a["d_status"], 0)
+
+    for kw, code in [({"d_consts": 0}, lz.ZERO_EINVAL), ({"d_consts": dc + 2}, lz.ZERO_EALIGN),
+                     ({"master_in": 0}, lz.ZERO_EINVAL), ({"m_out": outs[1] + 2}, lz.ZERO_EALIGN),
+                     ({"v_out": ins[2] + 4}, lz.ZERO_EINVAL),          # output over an input
+                     ({"param_out": outs[0] + 100}, lz.ZERO_EINVAL),   # over another output
+                     ({"master_out": slots + 64}, lz.ZERO_EINVAL),     # over the slots
+                     ({"d_status": slots + 16}, lz.ZERO_EINVAL)]:
+        with pytest.raises(lz.ZeroError) as e:
+            call(**kw)
+        assert e.value.code == code, kw
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_sched_create_fused(pl, slots, need - 1, 2, *ins, *outs, par, dc, st, 0)
+    assert e.value.code == lz.ZERO_ENOMEM

@@ -326,6 +326,73 @@ def test_stage2_scheduler_vs_oracle(n_slots):
     lz.zero_sched_destroy(sch)
 
 
+@pytest.mark.parametrize("n_slots", [1, 3])
+def test_stage2_fused_scheduler_vs_oracle(n_slots):
+    """The scheduler in fused mode: each bucket's kernel is the fused step over its range (the
+    reduced gradient never stored), slots released after it; commit after the last bucket.
+    Equals the oracle's stage-2 step; then an inf in one bucket skips the whole step."""
+    numels, nd, bucket = [40000, 1234, 30000, 777], 6, 9000
+    pl = lz.zero_plan_create(numels, nd, 2, bucket)
+    psi, psi_p, S, nb = lz.zero_plan_info(pl)
+    ref_plan = oracle.plan(numels, nd, bucket)
+    g_cpu = []
+    for r in range(nd):
+        g = torch.zeros(psi_p, dtype=torch.float16)
+        g[:psi] = synth.grad_f16(psi, 1e-3, seed=23, rank=r)
+        g_cpu.append(g)
+    master, m, v = synth.state_warm(psi_p, seed=24)
+    w_np, m_np, v_np = master.numpy(), m.numpy(), v.numpy()
+    slot_elems = lz.zero_sched_slot_elems(pl, n_slots)
+    slots = torch.empty(slot_elems, dtype=torch.float16, device=DEV)
+    dc = torch.frombuffer(bytearray(bytes(lz.zero_adam_consts_for_step(HP, 3))),
+                          dtype=torch.uint8).to(DEV)
+
+    def run(g_src):
+        ins = [x.to(DEV) for x in (master, m, v)]
+        outs = [torch.full_like(x, float("nan")) for x in ins]
+        params = torch.zeros(psi_p, dtype=torch.float16, device=DEV)
+        st = status_word()
+        producer, stream = torch.cuda.Stream(), torch.cuda.Stream()
+        torch.cuda.synchronize()
+        sch = lz.zero_sched_create_fused(pl, slots, slot_elems, n_slots, *ins, *outs, params,
+                                         dc, st, stream)
+        with torch.cuda.stream(producer):
+            for k in range(nb):
+                lo, ln, _, _ = lz.zero_plan_bucket(pl, k)
+                ptrs = lz.zero_sched_begin_bucket(sch, k, producer)
+                for r in range(nd):
+                    dst = torch.empty(0, dtype=torch.float16, device=DEV).set_(
+                        slots.untyped_storage(), (ptrs[r] - slots.data_ptr()) // 2, (ln,))
+                    dst.copy_(g_src[r][lo:lo + ln])
+                lz.zero_sched_end_bucket(sch, k, producer)
+        main = torch.cuda.current_stream()
+        lz.zero_sched_wait(sch, main)
+        lz.zero_step_commit(psi_p, *ins, *outs, params, st)
+        code, flags = lz.zero_step_status(st)
+        assert lz.zero_sched_launches(sch) == nb
+        lz.zero_sched_destroy(sch)
+        return code, flags, ins, outs, params
+
+    code, flags, ins, outs, params = run([g.to(DEV) for g in g_cpu])
+    assert code == lz.ZERO_OK and flags == 0
+    ref = oracle.zero2_step(ref_plan, lambda k, r: g_cpu[r].numpy()[
+        ref_plan.buckets[k][0]:sum(ref_plan.buckets[k])], w_np, m_np, v_np,
+        oracle.f2h(w_np), ORC_HP, 3)
+    check_f32("master", f32np(outs[0]), ref.master)
+    check_f32("m", f32np(outs[1]), ref.m)
+    check_f32("v", f32np(outs[2]), ref.v)
+    check_f16("params", f16np(params), ref.params16)
+    # an inf in the middle bucket's gradient of rank 2: the whole step is skipped
+    g_bad = [g.to(DEV) for g in g_cpu]
+    lo_mid, _, _, _ = lz.zero_plan_bucket(pl, nb // 2)
+    g_bad[2][lo_mid + 5] = float("inf")
+    code, flags, ins, outs, params = run(g_bad)
+    assert code == lz.ZERO_STEP_SKIPPED
+    for a, b in zip(ins, outs):
+        assert torch.equal(a, b)
+    assert np.array_equal(f16np(params), oracle.f2h(w_np))
+
+
 def test_step_split_into_bucket_calls():
     """One step made of several zero_step_fused calls (one per bucket, backward order) and one
     commit equals the single-call step; an overflow in a late bucket skips all of it."""

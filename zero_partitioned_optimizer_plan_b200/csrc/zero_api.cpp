@@ -91,6 +91,29 @@ cudaError_t rs_bucket_launch(const zero_plan* plan, int k, const uint16_t* const
     return launch_reduce_scatter(len, nd, rank_grads, shards, lo, S, make_mean(nd), status, stream);
 }
 
+zero_status check_fused_state(uint64_t n, const float* master_in, const float* m_in,
+                              const float* v_in, float* master_out, float* m_out,
+                              float* v_out, uint16_t* param_out, uint32_t* d_status) {
+    if (!master_in || !m_in || !v_in || !master_out || !m_out || !v_out || !param_out ||
+        !d_status)
+        return ZERO_EINVAL;
+    if (n > (UINT64_MAX / 8)) return ZERO_EINVAL;
+    if (!zk::aligned(master_in, 4) || !zk::aligned(m_in, 4) || !zk::aligned(v_in, 4) ||
+        !zk::aligned(master_out, 4) || !zk::aligned(m_out, 4) || !zk::aligned(v_out, 4) ||
+        !zk::aligned(param_out, 2) || !zk::aligned(d_status, 4))
+        return ZERO_EALIGN;
+    const void* outs[5] = {master_out, m_out, v_out, param_out, d_status};
+    const uint64_t olen[5] = {n * 4, n * 4, n * 4, n * 2, 4};
+    const void* ins[3] = {master_in, m_in, v_in};
+    for (int i = 0; i < 5; ++i) {
+        for (int j = 0; j < 3; ++j)
+            if (zk::overlap(outs[i], olen[i], ins[j], n * 4)) return ZERO_EINVAL;
+        for (int j = i + 1; j < 5; ++j)
+            if (zk::overlap(outs[i], olen[i], outs[j], olen[j])) return ZERO_EINVAL;
+    }
+    return ZERO_OK;
+}
+
 }  // namespace zk
 
 extern "C" {
@@ -229,28 +252,6 @@ zero_status zero_adam_shard_dc(uint64_t n, const float* grad, float* master, flo
                                          d_status, (cudaStream_t)stream));
 }
 
-static zero_status check_fused_state(uint64_t n, const float* master_in, const float* m_in,
-                                     const float* v_in, float* master_out, float* m_out,
-                                     float* v_out, uint16_t* param_out, uint32_t* d_status) {
-    if (!master_in || !m_in || !v_in || !master_out || !m_out || !v_out || !param_out ||
-        !d_status)
-        return ZERO_EINVAL;
-    if (n > (UINT64_MAX / 8)) return ZERO_EINVAL;
-    if (!zk::aligned(master_in, 4) || !zk::aligned(m_in, 4) || !zk::aligned(v_in, 4) ||
-        !zk::aligned(master_out, 4) || !zk::aligned(m_out, 4) || !zk::aligned(v_out, 4) ||
-        !zk::aligned(param_out, 2) || !zk::aligned(d_status, 4))
-        return ZERO_EALIGN;
-    const void* outs[5] = {master_out, m_out, v_out, param_out, d_status};
-    const uint64_t olen[5] = {n * 4, n * 4, n * 4, n * 2, 4};
-    const void* ins[3] = {master_in, m_in, v_in};
-    for (int i = 0; i < 5; ++i) {
-        for (int j = 0; j < 3; ++j)
-            if (zk::overlap(outs[i], olen[i], ins[j], n * 4)) return ZERO_EINVAL;
-        for (int j = i + 1; j < 5; ++j)
-            if (zk::overlap(outs[i], olen[i], outs[j], olen[j])) return ZERO_EINVAL;
-    }
-    return ZERO_OK;
-}
 
 static zero_status check_fused(uint64_t n, int nd, const uint16_t* const* rank_grads,
                                const float* master_in, const float* m_in, const float* v_in,
@@ -259,8 +260,8 @@ static zero_status check_fused(uint64_t n, int nd, const uint16_t* const* rank_g
     if (nd < 1 || nd > ZERO_MAX_RANKS || !d_status) return ZERO_EINVAL;
     if (n == 0) return ZERO_OK;
     if (!rank_grads) return ZERO_EINVAL;
-    zero_status st = check_fused_state(n, master_in, m_in, v_in, master_out, m_out, v_out,
-                                       param_out, d_status);
+    zero_status st = zk::check_fused_state(n, master_in, m_in, v_in, master_out, m_out, v_out,
+                                           param_out, d_status);
     if (st != ZERO_OK) return st;
     const void* outs[5] = {master_out, m_out, v_out, param_out, d_status};
     const uint64_t olen[5] = {n * 4, n * 4, n * 4, n * 2, 4};
@@ -323,8 +324,8 @@ zero_status zero_step_fused_q8(uint64_t n, int nd, const uint8_t* const* rank_pa
         return ZERO_EINVAL;
     if (n == 0) return ZERO_OK;
     if (!rank_payload) return ZERO_EINVAL;
-    zero_status st = check_fused_state(n, master_in, m_in, v_in, master_out, m_out, v_out,
-                                       param_out, d_status);
+    zero_status st = zk::check_fused_state(n, master_in, m_in, v_in, master_out, m_out, v_out,
+                                           param_out, d_status);
     if (st != ZERO_OK) return st;
     const uint64_t pb = ZERO_Q8_PAYLOAD_BYTES(n);
     const void* outs[5] = {master_out, m_out, v_out, param_out, d_status};
@@ -346,8 +347,8 @@ zero_status zero_step_commit(uint64_t n, const float* master_in, const float* m_
                              uint16_t* param_out, uint32_t* d_status, zero_stream_t stream) {
     if (!d_status) return ZERO_EINVAL;
     if (n == 0) return ZERO_OK;
-    zero_status st = check_fused_state(n, master_in, m_in, v_in, master_out, m_out, v_out,
-                                       param_out, d_status);
+    zero_status st = zk::check_fused_state(n, master_in, m_in, v_in, master_out, m_out, v_out,
+                                           param_out, d_status);
     if (st != ZERO_OK) return st;
     return zk::from_cuda(zk::launch_commit(n, master_in, m_in, v_in, master_out, m_out, v_out,
                                            param_out, d_status, (cudaStream_t)stream));

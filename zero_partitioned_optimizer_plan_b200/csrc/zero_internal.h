@@ -71,6 +71,12 @@ cudaError_t rs_bucket_launch(const zero_plan* plan, int k, const uint16_t* const
 
 MeanConsts make_mean(int nd);
 
+// Argument checks of a fused update over n elements (null, alignment, outputs overlapping
+// inputs or each other); zero_api.cpp.
+zero_status check_fused_state(uint64_t n, const float* master_in, const float* m_in,
+                              const float* v_in, float* master_out, float* m_out, float* v_out,
+                              uint16_t* param_out, uint32_t* d_status);
+
 // Map a CUDA error to a zero_status, remembering its text for zero_last_error().
 zero_status from_cuda(cudaError_t e);
 

@@ -12,7 +12,12 @@
 // stream waits on that event before it fills the slot with a later bucket. The host never
 // blocks: all ordering is carried by events, so the fill of bucket k+1 overlaps the
 // reduce-scatter of bucket k whenever more than one slot exists.
+//
+// In the fused mode (zero_sched_create_fused) the kernel launched for a bucket is the fused
+// step over the bucket's range -- reduce, unscale, Adam, fp16 cast and write-back -- so the
+// reduced gradient never reaches memory; the caller commits the step after the last bucket.
 #include <cstdint>
+#include <cstring>
 #include <new>
 #include <vector>
 
@@ -36,6 +41,16 @@ struct zero_sched {
     std::vector<int> bucket_of_slot;     // per slot: the bucket begun in it (-1: none)
     cudaEvent_t tail = nullptr;          // scratch event for zero_sched_wait
     uint64_t launches = 0;
+    // fused mode: the step's state (flat, psi_p elements each) and constants
+    bool fused = false;
+    const float* w_in = nullptr;
+    const float* m_in = nullptr;
+    const float* v_in = nullptr;
+    float* w_out = nullptr;
+    float* m_out = nullptr;
+    float* v_out = nullptr;
+    uint16_t* param_out = nullptr;
+    const zero_adam_consts* consts = nullptr;
 };
 
 namespace {
@@ -65,25 +80,24 @@ zero_status zero_sched_slot_elems(const zero_plan* plan, int n_slots, uint64_t* 
     return ZERO_OK;
 }
 
-zero_status zero_sched_create(const zero_plan* plan, uint16_t* slot_mem, uint64_t slot_mem_elems,
-                              int n_slots, float* const* owner_grad_shards, uint32_t* d_status,
-                              zero_stream_t rs_stream, zero_sched** out) {
+}  // extern "C"
+
+namespace {
+
+// Validation and set-up shared by both modes (everything but what the bucket kernel writes).
+zero_status create_common(const zero_plan* plan, uint16_t* slot_mem, uint64_t slot_mem_elems,
+                          int n_slots, uint32_t* d_status, cudaStream_t stream, zero_sched** out) {
     if (!out) return ZERO_EINVAL;
     *out = nullptr;
     int nd = 0;
     uint64_t psi_p = 0, S = 0;
-    if (!zk::plan_geometry(plan, &nd, &psi_p, &S) || n_slots < 1 || !slot_mem ||
-        !owner_grad_shards || !d_status)
+    if (!zk::plan_geometry(plan, &nd, &psi_p, &S) || n_slots < 1 || !slot_mem || !d_status)
         return ZERO_EINVAL;
     if ((reinterpret_cast<uintptr_t>(slot_mem) & 15u) || (reinterpret_cast<uintptr_t>(d_status) & 3u))
         return ZERO_EALIGN;
     uint64_t need = 0;
     zero_sched_slot_elems(plan, n_slots, &need);
     if (slot_mem_elems < need) return ZERO_ENOMEM;
-    for (int r = 0; r < nd; ++r) {
-        if (!owner_grad_shards[r]) return ZERO_EINVAL;
-        if (reinterpret_cast<uintptr_t>(owner_grad_shards[r]) & 3u) return ZERO_EALIGN;
-    }
     zero_sched* s = new (std::nothrow) zero_sched();
     if (!s) return ZERO_ENOMEM;
     s->plan = plan;
@@ -91,9 +105,8 @@ zero_status zero_sched_create(const zero_plan* plan, uint16_t* slot_mem, uint64_
     s->n_slots = n_slots;
     s->stride = round8(zk::plan_max_bucket(plan));
     s->slot_mem = slot_mem;
-    for (int r = 0; r < nd; ++r) s->shards[r] = owner_grad_shards[r];
     s->status = d_status;
-    s->rs = (cudaStream_t)rs_stream;
+    s->rs = stream;
     try {
         s->produced.assign((size_t)n_slots, nullptr);
         s->released.assign((size_t)n_slots, nullptr);
@@ -114,6 +127,75 @@ zero_status zero_sched_create(const zero_plan* plan, uint16_t* slot_mem, uint64_
         delete s;
         return st == ZERO_OK ? ZERO_ECUDA : st;
     }
+    *out = s;
+    return ZERO_OK;
+}
+
+bool overlaps(const void* a, uint64_t na, const void* b, uint64_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return na && nb && x < y + nb && y < x + na;
+}
+
+}  // namespace
+
+extern "C" {
+
+zero_status zero_sched_create(const zero_plan* plan, uint16_t* slot_mem, uint64_t slot_mem_elems,
+                              int n_slots, float* const* owner_grad_shards, uint32_t* d_status,
+                              zero_stream_t rs_stream, zero_sched** out) {
+    int nd = 0;
+    uint64_t psi_p = 0, S = 0;
+    if (!out) return ZERO_EINVAL;
+    *out = nullptr;
+    if (!zk::plan_geometry(plan, &nd, &psi_p, &S) || !owner_grad_shards) return ZERO_EINVAL;
+    for (int r = 0; r < nd; ++r) {
+        if (!owner_grad_shards[r]) return ZERO_EINVAL;
+        if (reinterpret_cast<uintptr_t>(owner_grad_shards[r]) & 3u) return ZERO_EALIGN;
+    }
+    zero_sched* s = nullptr;
+    const zero_status st = create_common(plan, slot_mem, slot_mem_elems, n_slots, d_status,
+                                         (cudaStream_t)rs_stream, &s);
+    if (st != ZERO_OK) return st;
+    for (int r = 0; r < nd; ++r) s->shards[r] = owner_grad_shards[r];
+    *out = s;
+    return ZERO_OK;
+}
+
+zero_status zero_sched_create_fused(const zero_plan* plan, uint16_t* slot_mem,
+                                    uint64_t slot_mem_elems, int n_slots, const float* master_in,
+                                    const float* m_in, const float* v_in, float* master_out,
+                                    float* m_out, float* v_out, uint16_t* param_out,
+                                    const zero_adam_consts* d_consts, uint32_t* d_status,
+                                    zero_stream_t stream, zero_sched** out) {
+    int nd = 0;
+    uint64_t psi_p = 0, S = 0;
+    if (!out) return ZERO_EINVAL;
+    *out = nullptr;
+    if (!zk::plan_geometry(plan, &nd, &psi_p, &S) || !d_consts) return ZERO_EINVAL;
+    if (reinterpret_cast<uintptr_t>(d_consts) & 3u) return ZERO_EALIGN;
+    zero_status st = zk::check_fused_state(psi_p, master_in, m_in, v_in, master_out, m_out, v_out,
+                                           param_out, d_status);
+    if (st != ZERO_OK) return st;
+    // the staging slots are read by the bucket kernels: no output may overlap them
+    uint64_t need = 0;
+    zero_sched_slot_elems(plan, n_slots < 1 ? 1 : n_slots, &need);
+    const void* outs[4] = {master_out, m_out, v_out, param_out};
+    const uint64_t olen[4] = {psi_p * 4, psi_p * 4, psi_p * 4, psi_p * 2};
+    for (int i = 0; i < 4; ++i)
+        if (overlaps(outs[i], olen[i], slot_mem, need * 2)) return ZERO_EINVAL;
+    if (overlaps(d_status, 4, slot_mem, need * 2)) return ZERO_EINVAL;
+    zero_sched* s = nullptr;
+    st = create_common(plan, slot_mem, slot_mem_elems, n_slots, d_status, (cudaStream_t)stream, &s);
+    if (st != ZERO_OK) return st;
+    s->fused = true;
+    s->w_in = master_in;
+    s->m_in = m_in;
+    s->v_in = v_in;
+    s->w_out = master_out;
+    s->m_out = m_out;
+    s->v_out = v_out;
+    s->param_out = param_out;
+    s->consts = d_consts;
     *out = s;
     return ZERO_OK;
 }
@@ -145,8 +227,17 @@ zero_status zero_sched_end_bucket(zero_sched* s, int k, zero_stream_t producer) 
     cudaEvent_t prod = s->produced[(size_t)slot];
     if (cudaError_t e = cudaEventRecord(prod, (cudaStream_t)producer); e != cudaSuccess) return zk::from_cuda(e);
     if (cudaError_t e = cudaStreamWaitEvent(s->rs, prod, 0); e != cudaSuccess) return zk::from_cuda(e);
-    if (cudaError_t e = zk::rs_bucket_launch(s->plan, k, ptrs, s->shards, s->status, s->rs); e != cudaSuccess)
-        return zk::from_cuda(e);
+    cudaError_t e = cudaSuccess;
+    if (s->fused) {
+        zero_adam_consts unused;
+        memset(&unused, 0, sizeof(unused));
+        e = zk::launch_fused(len, s->nd, ptrs, s->w_in + lo, s->m_in + lo, s->v_in + lo,
+                             s->w_out + lo, s->m_out + lo, s->v_out + lo, s->param_out + lo, unused,
+                             s->consts, zk::make_mean(s->nd), s->status, s->rs);
+    } else {
+        e = zk::rs_bucket_launch(s->plan, k, ptrs, s->shards, s->status, s->rs);
+    }
+    if (e != cudaSuccess) return zk::from_cuda(e);
     ++s->launches;
     // release: the slot may be refilled once this reduce-scatter is done with it
     if (cudaError_t e = cudaEventRecord(s->released[(size_t)slot], s->rs); e != cudaSuccess) return zk::from_cuda(e);

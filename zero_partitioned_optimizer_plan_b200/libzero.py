@@ -49,7 +49,8 @@ SYMBOLS = (
     "zero_selftest_timeout", "zero_adam_consts_table", "zero_scaler_prepare",
     "zero_scaler_update", "zero_quantize_q8", "zero_step_fused_q8",
     "zero_overlap_begin", "zero_overlap_end",
-    "zero_sched_slot_elems", "zero_sched_create", "zero_sched_begin_bucket",
+    "zero_sched_slot_elems", "zero_sched_create", "zero_sched_create_fused",
+    "zero_sched_begin_bucket",
     "zero_sched_end_bucket", "zero_sched_wait", "zero_sched_launches", "zero_sched_destroy",
 )
 
@@ -147,6 +148,8 @@ def _load():
     L.zero_overlap_end.argtypes = [vp]
     L.zero_sched_slot_elems.argtypes = [vp, i32, P(u64)]
     L.zero_sched_create.argtypes = [vp, vp, u64, i32, P(vp), vp, vp, P(vp)]
+    L.zero_sched_create_fused.argtypes = [vp, vp, u64, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                          vp, P(vp)]
     L.zero_sched_begin_bucket.argtypes = [vp, i32, vp, P(vp)]
     L.zero_sched_end_bucket.argtypes = [vp, i32, vp]
     L.zero_sched_wait.argtypes = [vp, vp]
@@ -423,6 +426,19 @@ def zero_sched_create(plan: Plan, slot_mem, slot_mem_elems: int, n_slots: int,
                                   _ptr_array(owner_grad_shards, 4), _ptr(d_status, 4),
                                   _stream(rs_stream), C.byref(h)), "zero_sched_create")
     return Sched(h.value, len(owner_grad_shards))
+
+
+def zero_sched_create_fused(plan: Plan, slot_mem, slot_mem_elems: int, n_slots: int,
+                            master_in, m_in, v_in, master_out, m_out, v_out, param_out,
+                            d_consts, d_status, stream=None) -> Sched:
+    h = C.c_void_p()
+    _check(_lib.zero_sched_create_fused(plan.handle, _ptr(slot_mem, 2), slot_mem_elems, n_slots,
+                                        _ptr(master_in, 4), _ptr(m_in, 4), _ptr(v_in, 4),
+                                        _ptr(master_out, 4), _ptr(m_out, 4), _ptr(v_out, 4),
+                                        _ptr(param_out, 2), _ptr(d_consts), _ptr(d_status, 4),
+                                        _stream(stream), C.byref(h)), "zero_sched_create_fused")
+    _, psi_p, shard, _ = zero_plan_info(plan)
+    return Sched(h.value, psi_p // shard if shard else 1)
 
 
 def zero_sched_begin_bucket(s: Sched, k: int, producer=None) -> List[int]:
