@@ -90,6 +90,75 @@ def test_gpt2_small_stage1_ten_steps():
     print(f"PARITY gpt2-small stage 1: {idx.size} sampled elements x 10 steps within tolerance")
 
 
+def test_1p3b_stage2_fused_scheduler_with_overflow_run():
+    """The same 1.3B stage-2 step with the scheduler in fused mode (the launch configuration of
+    bench.py --workload zero2_1p3b --stage2-fused): each bucket's fused step is launched as the
+    bucket arrives, two staging slots, then one commit. An overflow run (+inf in rank 3, first
+    element of bucket 7) leaves the state unchanged; then 3 steps against the oracle."""
+    numels, nd, B = synth.gpt_1p3b_list(), 16, 50_000_000
+    pl = lz.zero_plan_create(numels, nd, 2, B)
+    psi, psi_p, S, nb = lz.zero_plan_info(pl)
+    bounds = [lz.zero_plan_bucket(pl, k)[0] for k in range(nb)] + [r * S for r in range(nd + 1)]
+    idx = sample_idx(psi_p, 200_000, 5, boundaries=bounds + lz.zero_plan_tensor_offsets(pl))
+    idx_dev = torch.from_numpy(idx).to(DEV)
+    cur = list(synth.state_small(psi_p, seed=5, device=DEV))
+    nxt = [torch.empty_like(x) for x in cur]
+    params = torch.zeros(psi_p, dtype=torch.float16, device=DEV)
+    n_slots = 2
+    slot_elems = lz.zero_sched_slot_elems(pl, n_slots)
+    slots = torch.empty(slot_elems, dtype=torch.float16, device=DEV)
+    d_consts = torch.empty(40, dtype=torch.uint8, device=DEV)
+    producer, stream = torch.cuda.Stream(), torch.cuda.Stream()
+    main = torch.cuda.current_stream()
+
+    def run_step(t, inject):
+        st = status_word()
+        c = lz.zero_adam_consts_for_step(HP, t)
+        d_consts.copy_(torch.frombuffer(bytearray(bytes(c)), dtype=torch.uint8))
+        torch.cuda.synchronize()
+        sch = lz.zero_sched_create_fused(pl, slots, slot_elems, n_slots, *cur, *nxt, params,
+                                         d_consts, st, stream)
+        gathered = [np.empty(idx.size, np.uint16) for _ in range(nd)]
+        with torch.cuda.stream(producer):
+            for k in range(nb):
+                lo, ln, _, _ = lz.zero_plan_bucket(pl, k)
+                ptrs = lz.zero_sched_begin_bucket(sch, k, producer)
+                views = [view_at(slots, p, ln) for p in ptrs]
+                for r in range(nd):
+                    synth.grad_f16(ln, 1e-3, seed=5, rank=r, step=1000 * t + k, out=views[r])
+                if inject and k == 7:
+                    views[3][0] = float("inf")
+                sel = np.nonzero((idx >= lo) & (idx < lo + ln))[0]
+                local = torch.from_numpy(idx[sel] - lo).to(DEV)
+                for r in range(nd):
+                    gathered[r][sel] = views[r][local].cpu().numpy().view(np.uint16)
+                lz.zero_sched_end_bucket(sch, k, producer)
+        lz.zero_sched_wait(sch, main)
+        lz.zero_step_commit(psi_p, *cur, *nxt, params, st, main)
+        code, flags = lz.zero_step_status(st, main)
+        assert lz.zero_sched_launches(sch) == nb
+        lz.zero_sched_destroy(sch)
+        return code, flags, gathered
+
+    code, flags, _ = run_step(1, inject=True)
+    assert code == lz.ZERO_STEP_SKIPPED and flags == lz.ZERO_FLAG_OVERFLOW | lz.ZERO_FLAG_SKIPPED
+    for a, b in zip(cur, nxt):    # the commit restored every element
+        assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+    w_s, m_s, v_s = (gather(x, idx_dev) for x in cur)
+    check_f16("skipped step params", gather(params, idx_dev), oracle.f2h(w_s))
+    for t in range(1, 4):
+        code, flags, gs = run_step(t, inject=False)
+        assert (code, flags) == (lz.ZERO_OK, 0)
+        cur, nxt = nxt, cur
+        skipped, w_s, m_s, v_s, p_s = oracle.step(gs, w_s, m_s, v_s, ORC_HP, t)
+        assert not skipped
+        check_f32(f"step {t} master", gather(cur[0], idx_dev), w_s)
+        check_f32(f"step {t} m", gather(cur[1], idx_dev), m_s)
+        check_f32(f"step {t} v", gather(cur[2], idx_dev), v_s)
+        check_f16(f"step {t} params", gather(params, idx_dev), p_s)
+    print(f"PARITY 1.3B stage 2 fused scheduler: skip run + 3 steps, {idx.size} sampled elements")
+
+
 def test_1p3b_stage2_buckets_with_overflow_run():
     """1.3B list (Psi = 1,311,528,960), Nd = 16, stage 2, buckets of 50,000,000 elements in
     backward order through the scheduler (two staging slots, producer and reduce-scatter on
