@@ -388,7 +388,7 @@ zero_status zero_sched_create(const zero_plan* plan, uint16_t* slot_mem, uint64_
 /* Fused mode: the kernel launched for bucket k (on `stream`) is the fused step over the
  * bucket's range [lo, lo+len) of the flat padded buffer -- rank-ordered reduction, unscale,
  * Adam, fp16 cast and write-back, as zero_step_fused_dc with the step's constants read from
- * d_consts -- so the reduced gradient never reaches memory (the survey's a7 applied to stage 2,
+ * d_consts -- so the reduced gradient never reaches memory (the fused step applied to stage 2
  * bucket by bucket, with the same release of each slot after its kernel). master_in/m_in/v_in
  * and master_out/m_out/v_out: psi_p fp32 values each (flat, padded), param_out: psi_p fp16
  * values; they stay fixed for the scheduler's life (with ping-pong state, create one per
