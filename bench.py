@@ -170,25 +170,27 @@ class Workload:
         """Each rank's gradients as int8 + one fp32 scale per 128 (the senders' work, done once
         before timing and timed on its own)."""
         torch, lz = self.torch, self.lz
-        if len(self.ranges) != 1:
-            raise SystemExit("--payload q8 takes one call per step (no --bucket)")
         n, nd = self.n, self.nd
-        nb = (n + 127) // 128
-        self.q = [torch.empty(lz.q8_payload_bytes(n), dtype=torch.uint8, device=self.dev)
-                  for _ in range(nd)]
+        # one payload per range and rank, records counted from the range's first element;
+        # self.q[i * nd + r] is range i's payload of rank r
+        self.q = [torch.empty(lz.q8_payload_bytes(hi - lo), dtype=torch.uint8, device=self.dev)
+                  for lo, hi in self.ranges for _ in range(nd)]
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        lz.zero_quantize_q8(n, self.grads[0], self.q[0])     # first use outside the timing
+        lo0, hi0 = self.ranges[0]
+        lz.zero_quantize_q8(hi0 - lo0, self.grads[0][lo0:hi0], self.q[0])   # first use untimed
         e0.record()
-        for g, q in zip(self.grads, self.q):
-            lz.zero_quantize_q8(n, g, q)
+        for i, (lo, hi) in enumerate(self.ranges):
+            for r, g in enumerate(self.grads):
+                lz.zero_quantize_q8(hi - lo, g[lo:hi], self.q[i * nd + r])
         e1.record()
         torch.cuda.synchronize()
-        qbytes = nd * (2 * n + 132 * nb)
+        recs = sum((hi - lo + 127) // 128 for lo, hi in self.ranges)
+        qbytes = nd * (2 * n + 132 * recs)
         self.side = {"kernel": "quant_q8_kernel (senders, once)", "bytes": qbytes,
-                     "calls": nd, "ms": [(e0, e1)]}
+                     "calls": nd * len(self.ranges), "ms": [(e0, e1)]}
         self.grads = None
         torch.cuda.empty_cache()
-        self.bytes_per_step = nd * 132 * nb + 26 * n
+        self.bytes_per_step = nd * 132 * recs + 26 * n
         self.dominant = "fused_q8_tma_kernel"
         self.dominant_bytes = self.bytes_per_step
         self.config["payload"] = "int8 records: 128 values and their fp32 scale"
@@ -291,10 +293,17 @@ class Workload:
         lz = self.lz
         if self.payload == "q8":
             pays = grads or self.inputs()
+            nd = self.nd
             if ev is not None:
                 ev[0].record()
-            lz.zero_step_fused_q8(self.n, self.nd, pays, *self.cur, *self.nxt, self.params,
-                                  self.hp, t, status)
+            if self.overlap:
+                lz.zero_overlap_begin()
+            for i, (lo, hi) in enumerate(self.ranges):
+                lz.zero_step_fused_q8(hi - lo, nd, pays[i * nd:(i + 1) * nd],
+                                      *[x[lo:hi] for x in self.cur], *[x[lo:hi] for x in self.nxt],
+                                      self.params[lo:hi], self.hp, t, status)
+            if self.overlap:
+                lz.zero_overlap_end()
             if ev is not None:
                 ev[1].record()
             lz.zero_step_commit(self.n, *self.cur, *self.nxt, self.params, status)

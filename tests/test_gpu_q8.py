@@ -73,8 +73,12 @@ def test_quantize_bit_exact(n, kind):
 
 
 @pytest.mark.parametrize("nd", [1, 2, 3, 8, 16, 25, 64])
-@pytest.mark.parametrize("n", [9, 4096, 4096 + 300, 2048 * 40 + 777])
+@pytest.mark.parametrize("n", [9, 4096, 4096 + 300, 4096 + 511, 2048 * 40 + 777,
+                               1_900_000 + 77])
 def test_fused_q8_vs_oracle(n, nd):
+    """Sizes for the plain kernel (9), the small-call shape (its tail of up to 511 elements
+    past the last whole tile taken in several passes by 8 or 12 warps) and the large shape
+    (1.9 M elements, above 4 tiles per SM)."""
     seed = 7 * n + nd
     master, m, v = synth.state_warm(n, seed=seed)
     pp = PingPong(master, m, v)

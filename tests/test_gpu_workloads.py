@@ -351,3 +351,31 @@ def test_flat_sweep_bucketed_calls(nd):
             if mode == "graph":
                 del graph
     print(f"PARITY flat 2^29 Nd={nd}: 4 bucket sizes (2 also by graph), {idx.size} sampled elements")
+
+
+def test_fused_call_beyond_2p31_elements():
+    """Maximum size: one zero_step_fused call over 2^31 + 4101 elements (Nd = 2; 64 GB on the
+    device), so every element index past 2^31 goes through the tile, copy and store arithmetic;
+    sampled around 2^31, tile boundaries and the end, then the commit."""
+    nd, n = 2, (1 << 31) + 4101
+    grads = [synth.grad_f16(n, 1e-3, seed=9, rank=r, step=1, device=DEV) for r in range(nd)]
+    cur = list(synth.state_warm(n, seed=90, device=DEV))
+    nxt = [torch.empty_like(x) for x in cur]
+    params = torch.empty(n, dtype=torch.float16, device=DEV)
+    idx = sample_idx(n, 100_000, 9, boundaries=[1 << 31, (1 << 31) - 2560 * 7, n - 4101,
+                                                 n - 5, (1 << 30) * 3 // 2])
+    idx_dev = torch.from_numpy(idx).to(DEV)
+    st = status_word()
+    lz.zero_step_fused(n, nd, grads, *cur, *nxt, params, HP, 1, st)
+    lz.zero_step_commit(n, *cur, *nxt, params, st)
+    torch.cuda.synchronize()
+    assert status_flags(st) == 0
+    skipped, w, mm, vv, p = oracle.step([gather(g, idx_dev) for g in grads],
+                                        *(gather(x, idx_dev) for x in cur), ORC_HP, 1)
+    assert not skipped
+    check_f32("master", gather(nxt[0], idx_dev), w)
+    check_f32("m", gather(nxt[1], idx_dev), mm)
+    check_f32("v", gather(nxt[2], idx_dev), vv)
+    check_f16("params", gather(params, idx_dev), p)
+    print(f"PARITY fused call of {n} elements: {idx.size} sampled")
+

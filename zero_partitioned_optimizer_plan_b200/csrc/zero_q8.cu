@@ -231,7 +231,7 @@ __device__ void produce_q8(const FusedQ8Args& p, uint64_t* full, uint64_t* empty
 }
 
 template <int W>
-__global__ void __launch_bounds__(Warps<W>::kThreads, 1)
+__global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
     fused_q8_tma_kernel(const __grid_constant__ FusedQ8Args p) {
     constexpr int E = kElems;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -311,9 +311,10 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, 1)
         stg_f32<E>(p.v_out + g0, v);
         stg_f16<E>(p.param_out + g0, w, p.param_vec);
     }
-    // the < 512 elements past the last tile (W >= 16 warps: 512 or more consumer threads)
-    if (blockIdx.x == 0 && (uint64_t)threadIdx.x < p.n - p.n_tiled)
-        fused_q8_element(p, p.n_tiled + threadIdx.x, bad);
+    // the < 512 elements past the last tile
+    if (blockIdx.x == 0)
+        for (uint64_t i = threadIdx.x; i < p.n - p.n_tiled; i += 32u * W)
+            fused_q8_element(p, p.n_tiled + i, bad);
     flag_overflow(bad, p.status);
     pdl_leave(p.chained);
 }
@@ -335,8 +336,13 @@ Variant pick_variant_q8(int nd) {
     return {16, 2};
 }
 
+// Small calls (fewer than 4 tiles of the large shape per SM): as for the fp16 step, 12
+// consumer warps up to Nd = 8 and 8 above, 100 KB of stages and one CTA per SM, so that the
+// next call of an overlap region loads beside this one.
+constexpr size_t kQ8SmallBudget = 100 * 1024;
+
 // A rank's run of T/128 records per stage.
-PipeShape q8_shape(int nd, int warps, int target_stages) {
+PipeShape q8_shape(int nd, int warps, int target_stages, size_t budget) {
     PipeShape sh;
     sh.warps = warps;
     sh.grid_per_sm = 0;
@@ -344,14 +350,14 @@ PipeShape q8_shape(int nd, int warps, int target_stages) {
     g.tile = (uint32_t)(32 * warps * kElems);
     const size_t row = (size_t)g.tile / kQB * kRec;
     const size_t state = (size_t)g.tile * 12u;
-    const size_t per_stage = kSmemBudget / (size_t)target_stages;
+    const size_t per_stage = budget / (size_t)target_stages;
     size_t rc_max = per_stage > state + row ? (per_stage - state) / row : 1;
     if (rc_max > (size_t)nd) rc_max = (size_t)nd;
     g.nchunks = (uint32_t)(((size_t)nd + rc_max - 1) / rc_max);
     g.rc = (uint32_t)(((size_t)nd + g.nchunks - 1) / g.nchunks);
     g.state_off = (uint32_t)(g.rc * row);
     g.stage_bytes = (uint32_t)(g.state_off + state);
-    size_t st = kSmemBudget / g.stage_bytes;
+    size_t st = budget / g.stage_bytes;
     if (st < 2) st = 2;
     if (st > kMaxStages) st = kMaxStages;
     g.stages = (int)st;
@@ -422,13 +428,22 @@ cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,
 #ifdef ZK_Q8_TARGET_STAGES
     var.target_stages = ZK_Q8_TARGET_STAGES;
 #endif
-    const PipeShape sh = q8_shape(nd, var.warps, var.target_stages);
+    const uint64_t big_tiles = n / (32ull * (uint64_t)var.warps * kElems);
+    PipeShape sh;
+    if (big_tiles < 4ull * (uint64_t)di.sms) {
+        sh = q8_shape(nd, nd <= 8 ? 12 : 8, 2, kQ8SmallBudget);
+        sh.grid_per_sm = 1;
+    } else {
+        sh = q8_shape(nd, var.warps, var.target_stages, kSmemBudget);
+    }
     p.g = sh.g;
     p.row = sh.g.tile / kQB * kRec;
     p.n_tiled = n & ~(kQTileAlign - 1);
     p.num_tiles = (p.n_tiled + sh.g.tile - 1) / sh.g.tile;
     p.chained = overlap_next(stream) ? 1 : 0;
     switch (sh.warps) {
+        case 8: return launch_pipe(fused_q8_tma_kernel<8>, p, sh, stream);
+        case 12: return launch_pipe(fused_q8_tma_kernel<12>, p, sh, stream);
         case 16: return launch_pipe(fused_q8_tma_kernel<16>, p, sh, stream);
         case 20: return launch_pipe(fused_q8_tma_kernel<20>, p, sh, stream);
         case 24: return launch_pipe(fused_q8_tma_kernel<24>, p, sh, stream);
