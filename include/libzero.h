@@ -332,6 +332,18 @@ zero_status zero_step_fused_q8(uint64_t n, int nd, const uint8_t* const* rank_pa
                                uint16_t* param_out, const zero_adam_hparams* hp, int64_t step,
                                uint32_t* d_status, zero_stream_t stream);
 
+/* zero_step_fused_q8 with the step's constants read from device memory (d_consts: a
+ * zero_adam_consts, 4-byte aligned, e.g. written by zero_scaler_prepare), as
+ * zero_step_fused_dc: the call can be captured in a CUDA graph and replayed for every step,
+ * with dynamic loss scaling on the device. Same results, bit for bit, as the by-value call with
+ * the same constants. Errors: as zero_step_fused_q8, and ZERO_EINVAL / ZERO_EALIGN for
+ * d_consts. */
+zero_status zero_step_fused_q8_dc(uint64_t n, int nd, const uint8_t* const* rank_payload,
+                                  const float* master_in, const float* m_in, const float* v_in,
+                                  float* master_out, float* m_out, float* v_out,
+                                  uint16_t* param_out, const zero_adam_consts* d_consts,
+                                  uint32_t* d_status, zero_stream_t stream);
+
 /* Self-test of the kernels' bounded waits (failure detection without a fault): launches the
  * fused pipeline on one tile with its copy-issuing warp switched off, so every consumer's wait
  * on shared-memory data expires after about one second; the kernel then sets

@@ -350,3 +350,14 @@ def test_fused_scheduler_rejects():
     with pytest.raises(lz.ZeroError) as e:
         lz.zero_sched_create_fused(pl, slots, need - 1, 2, *ins, *outs, par, dc, st, 0)
     assert e.value.code == lz.ZERO_ENOMEM
+
+
+def test_q8_dc_rejects():
+    ins = [A + 100 * MB, A + 101 * MB, A + 102 * MB]
+    outs = [A + 110 * MB, A + 111 * MB, A + 112 * MB]
+    pays = [A + i * MB for i in range(2)]
+    for dc, code in [(0, lz.ZERO_EINVAL), (A + 140 * MB + 2, lz.ZERO_EALIGN)]:
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_step_fused_q8_dc(1000, 2, pays, *ins, *outs, A + 120 * MB, dc, A + 130 * MB, 0)
+        assert e.value.code == code
+    lz.zero_step_fused_q8_dc(0, 2, pays, *ins, *outs, A + 120 * MB, A + 140 * MB, A + 130 * MB, 0)

@@ -180,3 +180,119 @@ def test_7p5b_shard_view_q8_sampled():
     check_f32("v", nxt[2][idx_dev].cpu().numpy(), vv)
     check_f16("params", out[idx_dev].cpu().numpy().view(np.uint16), p)
     assert int(torch.count_nonzero(full[:owner * S].view(torch.int16))) == 0
+
+
+@pytest.mark.parametrize("nd", [2, 64])
+def test_q8_device_constants_match(nd):
+    """zero_step_fused_q8_dc (constants from device memory) gives the same bits as
+    zero_step_fused_q8 with the hyperparameters and t, for the small and the large shape."""
+    for n in (2048 * 21 + 3, 1_900_000 + 77):
+        g_dev = [synth.grad_f16(n, 1e-2, seed=81, rank=r, step=1).to(DEV) for r in range(nd)]
+        pay = [_quant_dev(g) for g in g_dev]
+        master, m, v = (x.to(DEV) for x in synth.state_warm(n, seed=82))
+        for t in (1, 7):
+            c = lz.zero_adam_consts_for_step(HP, t)
+            dc = torch.frombuffer(bytearray(bytes(c)), dtype=torch.uint8).to(DEV)
+            outs_a = [torch.empty_like(x) for x in (master, m, v)]
+            outs_b = [torch.empty_like(x) for x in (master, m, v)]
+            pa = torch.empty(n, dtype=torch.float16, device=DEV)
+            pb = torch.empty(n, dtype=torch.float16, device=DEV)
+            st = status_word()
+            lz.zero_step_fused_q8(n, nd, pay, master, m, v, *outs_a, pa, HP, t, st)
+            lz.zero_step_fused_q8_dc(n, nd, pay, master, m, v, *outs_b, pb, dc, st)
+            torch.cuda.synchronize()
+            assert status_flags(st) == 0
+            for a, b in list(zip(outs_a, outs_b)) + [(pa, pb)]:
+                assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_q8_graph_with_device_scaler():
+    """Per-bucket int8 steps in an overlap region between zero_scaler_prepare and
+    zero_scaler_update, captured as CUDA graphs and replayed for ten steps, three of them with
+    an inf in a rank's gradient (its block poisoned by the quantizer): state, parameters and
+    scaler equal the oracle's int8 steps under the same scaling rule."""
+    import dataclasses
+    nd, n, B = 4, 2048 * 12 + 5, 7168
+    overflow = [False, False, False, True, True, False, False, False, True, False]
+    bounds = [(lo, min(n, lo + B)) for lo in range(0, n, B)][::-1]
+    master, m, v = synth.state_warm(n, seed=83)
+    bufs = [[x.to(DEV) for x in (master, m, v)], [torch.empty(n, device=DEV) for _ in range(3)]]
+    grads = [torch.empty(n, dtype=torch.float16, device=DEV) for _ in range(nd)]
+    pays = {lo: [torch.empty(lz.q8_payload_bytes(hi - lo), dtype=torch.uint8, device=DEV)
+                 for _ in range(nd)] for lo, hi in bounds}
+    params = torch.empty(n, dtype=torch.float16, device=DEV)
+    table = lz.zero_adam_consts_table(HP, 1, 32)
+    d_table = torch.frombuffer(bytearray(bytes(table)), dtype=torch.uint8).to(DEV)
+    d_consts = torch.empty(40, dtype=torch.uint8, device=DEV)
+    init = lz.ScalerState(1024.0, 0, 1, 0)
+    d_state = torch.frombuffer(bytearray(bytes(init)), dtype=torch.uint8).to(DEV)
+    prm = lz.ScalerParams(2.0, 0.5, 2)
+    st = status_word()
+
+    def step(src, dst):
+        lz.zero_scaler_prepare(d_state, d_table, 32, d_consts, st)
+        with lz.overlap():
+            for lo, hi in bounds:
+                lz.zero_step_fused_q8_dc(hi - lo, nd, pays[lo], *[x[lo:hi] for x in src],
+                                         *[x[lo:hi] for x in dst], params[lo:hi], d_consts, st)
+        lz.zero_step_commit(n, *src, *dst, params, st)
+        lz.zero_scaler_update(d_state, prm, st)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step(bufs[0], bufs[1])
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graphs = []
+    for src, dst in ((bufs[0], bufs[1]), (bufs[1], bufs[0])):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(src, dst)
+        graphs.append(g)
+    for x, y in zip(bufs[0], (master, m, v)):
+        x.copy_(y.to(DEV))
+    d_state.copy_(torch.frombuffer(bytearray(bytes(init)), dtype=torch.uint8).to(DEV))
+    torch.cuda.synchronize()
+
+    sc = oracle.Scaler(scale=1024.0, growth_interval=2)
+    w_r, m_r, v_r = master.numpy(), m.numpy(), v.numpy()
+    p_r = None
+    for i, bad in enumerate(overflow):
+        g_cpu = [synth.grad_f16(n, 1e-2, seed=84, rank=r, step=i) for r in range(nd)]
+        if bad:
+            g_cpu[nd - 1][n // 3] = float("inf")
+        for d, s in zip(grads, g_cpu):
+            d.copy_(s.to(DEV))
+        for lo, hi in bounds:                    # the senders quantize each bucket
+            for r in range(nd):
+                lz.zero_quantize_q8(hi - lo, grads[r][lo:hi], pays[lo][r])
+        graphs[i % 2].replay()
+        # oracle: each bucket's payload from its own range; one skip decision for the step
+        hp_t = dataclasses.replace(ORC_HP, loss_scale=sc.scale)
+        parts, skipped = {}, False
+        for lo, hi in bounds:
+            ref = [oracle.quant_q8(g.numpy()[lo:hi]) for g in g_cpu]
+            sk, w, mm, vv, p = oracle.step_q8([q for q, _ in ref], [s for _, s in ref],
+                                              w_r[lo:hi], m_r[lo:hi], v_r[lo:hi], hp_t,
+                                              sc.next_step)
+            skipped |= sk
+            parts[lo] = (w, mm, vv, p)
+        assert skipped == bad
+        if not skipped:
+            w_r, m_r, v_r = (np.concatenate([parts[lo][k] for lo, _ in bounds[::-1]])
+                             for k in range(3))
+            p_r = np.concatenate([parts[lo][3] for lo, _ in bounds[::-1]])
+        sc.update(skipped)
+    torch.cuda.synchronize()
+    out = bufs[len(overflow) % 2]
+    check_f32("master", f32np(out[0]), w_r)
+    check_f32("m", f32np(out[1]), m_r)
+    check_f32("v", f32np(out[2]), v_r)
+    check_f16("params", f16np(params), p_r)
+    s = lz.ScalerState()
+    import ctypes as C
+    C.memmove(C.addressof(s), bytes(d_state.cpu().numpy().tobytes()), C.sizeof(s))
+    assert (s.scale, s.good_steps, s.next_step, s.skipped_steps) == \
+        (np.float32(sc.scale), sc.good_steps, sc.next_step, sc.skipped_steps)
+    del graphs

@@ -315,13 +315,11 @@ zero_status zero_quantize_q8(uint64_t n, const uint16_t* grad, uint8_t* payload,
     return zk::from_cuda(zk::launch_quant_q8(n, grad, payload, (cudaStream_t)stream));
 }
 
-zero_status zero_step_fused_q8(uint64_t n, int nd, const uint8_t* const* rank_payload,
-                               const float* master_in, const float* m_in, const float* v_in,
-                               float* master_out, float* m_out, float* v_out,
-                               uint16_t* param_out, const zero_adam_hparams* hp, int64_t step,
-                               uint32_t* d_status, zero_stream_t stream) {
-    if (nd < 1 || nd > ZERO_MAX_RANKS || !zk::hparams_ok(hp) || step < 1 || !d_status)
-        return ZERO_EINVAL;
+static zero_status check_fused_q8(uint64_t n, int nd, const uint8_t* const* rank_payload,
+                                  const float* master_in, const float* m_in, const float* v_in,
+                                  float* master_out, float* m_out, float* v_out,
+                                  uint16_t* param_out, uint32_t* d_status) {
+    if (nd < 1 || nd > ZERO_MAX_RANKS || !d_status) return ZERO_EINVAL;
     if (n == 0) return ZERO_OK;
     if (!rank_payload) return ZERO_EINVAL;
     zero_status st = zk::check_fused_state(n, master_in, m_in, v_in, master_out, m_out, v_out,
@@ -336,10 +334,40 @@ zero_status zero_step_fused_q8(uint64_t n, int nd, const uint8_t* const* rank_pa
         for (int i = 0; i < 5; ++i)
             if (zk::overlap(outs[i], olen[i], rank_payload[r], pb)) return ZERO_EINVAL;
     }
+    return ZERO_OK;
+}
+
+zero_status zero_step_fused_q8(uint64_t n, int nd, const uint8_t* const* rank_payload,
+                               const float* master_in, const float* m_in, const float* v_in,
+                               float* master_out, float* m_out, float* v_out,
+                               uint16_t* param_out, const zero_adam_hparams* hp, int64_t step,
+                               uint32_t* d_status, zero_stream_t stream) {
+    if (!zk::hparams_ok(hp) || step < 1) return ZERO_EINVAL;
+    const zero_status st = check_fused_q8(n, nd, rank_payload, master_in, m_in, v_in, master_out,
+                                          m_out, v_out, param_out, d_status);
+    if (st != ZERO_OK || n == 0) return st;
     return zk::from_cuda(zk::launch_fused_q8(n, nd, rank_payload, master_in, m_in, v_in,
                                              master_out, m_out, v_out, param_out,
-                                             zk::make_adam(hp, step), zk::make_mean(nd),
+                                             zk::make_adam(hp, step), nullptr, zk::make_mean(nd),
                                              d_status, (cudaStream_t)stream));
+}
+
+zero_status zero_step_fused_q8_dc(uint64_t n, int nd, const uint8_t* const* rank_payload,
+                                  const float* master_in, const float* m_in, const float* v_in,
+                                  float* master_out, float* m_out, float* v_out,
+                                  uint16_t* param_out, const zero_adam_consts* d_consts,
+                                  uint32_t* d_status, zero_stream_t stream) {
+    if (!d_consts) return ZERO_EINVAL;
+    if (!zk::aligned(d_consts, 4)) return ZERO_EALIGN;
+    const zero_status st = check_fused_q8(n, nd, rank_payload, master_in, m_in, v_in, master_out,
+                                          m_out, v_out, param_out, d_status);
+    if (st != ZERO_OK || n == 0) return st;
+    zero_adam_consts unused;
+    memset(&unused, 0, sizeof(unused));
+    return zk::from_cuda(zk::launch_fused_q8(n, nd, rank_payload, master_in, m_in, v_in,
+                                             master_out, m_out, v_out, param_out, unused,
+                                             d_consts, zk::make_mean(nd), d_status,
+                                             (cudaStream_t)stream));
 }
 
 zero_status zero_step_commit(uint64_t n, const float* master_in, const float* m_in,

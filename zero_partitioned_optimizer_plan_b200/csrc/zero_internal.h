@@ -48,8 +48,8 @@ cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, uint8_t* payload,
 cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,
                             const float* master_in, const float* m_in, const float* v_in,
                             float* master_out, float* m_out, float* v_out, uint16_t* param_out,
-                            const AdamConsts& a, const MeanConsts& mc, uint32_t* status,
-                            cudaStream_t stream);
+                            const AdamConsts& a, const AdamConsts* ad, const MeanConsts& mc,
+                            uint32_t* status, cudaStream_t stream);
 cudaError_t launch_scaler_prepare(const zero_scaler_state* st, const AdamConsts* table,
                                   int64_t table_len, AdamConsts* out, uint32_t* status,
                                   cudaStream_t stream);

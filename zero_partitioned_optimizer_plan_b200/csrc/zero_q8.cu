@@ -132,6 +132,7 @@ struct FusedQ8Args {
     int nd;
     int param_vec;
     AdamConsts a;
+    const AdamConsts* ad;  // when not null: the constants, read from device memory at run time
     MeanConsts mc;
     int chained;         // programmatic launch chained to the previous call (see pdl_enter)
 };
@@ -150,7 +151,8 @@ __device__ __forceinline__ float q_to_float(uint32_t biased, int j) {
                      8388736.0f);
 }
 
-__device__ __forceinline__ void fused_q8_element(const FusedQ8Args& p, uint64_t i, bool& bad) {
+__device__ __forceinline__ void fused_q8_element(const FusedQ8Args& p, const AdamConsts& a,
+                                                 uint64_t i, bool& bad) {
     if (i >= p.n) {
         atomicOr(p.status, ZERO_FLAG_BOUNDS);
         return;
@@ -164,7 +166,7 @@ __device__ __forceinline__ void fused_q8_element(const FusedQ8Args& p, uint64_t 
     const float red = mean_of(s, p.mc);
     bad |= non_finite(red);
     float w = p.master_in[i], m = p.m_in[i], v = p.v_in[i];
-    adam_elem(red, w, m, v, p.a);
+    adam_elem(red, w, m, v, a);
     p.master_out[i] = w;
     p.m_out[i] = m;
     p.v_out[i] = v;
@@ -230,7 +232,7 @@ __device__ void produce_q8(const FusedQ8Args& p, uint64_t* full, uint64_t* empty
     }
 }
 
-template <int W>
+template <int W, bool kDC>
 __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
     fused_q8_tma_kernel(const __grid_constant__ FusedQ8Args p) {
     constexpr int E = kElems;
@@ -245,6 +247,7 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
         pdl_leave(p.chained);
         return;
     }
+    ZK_STEP_CONSTS(p, a);
     const int lane = threadIdx.x & 31;
     const uint32_t T = p.g.tile;
     const uint32_t e0 = (uint32_t)threadIdx.x * E;
@@ -304,7 +307,7 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
         for (int j = 0; j < E; ++j) {
             const float red = mean_of(acc[j], p.mc);
             bad |= non_finite(red);
-            adam_elem(red, w[j], m[j], v[j], p.a);
+            adam_elem(red, w[j], m[j], v[j], a);
         }
         stg_f32<E>(p.master_out + g0, w);
         stg_f32<E>(p.m_out + g0, m);
@@ -314,16 +317,18 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
     // the < 512 elements past the last tile
     if (blockIdx.x == 0)
         for (uint64_t i = threadIdx.x; i < p.n - p.n_tiled; i += 32u * W)
-            fused_q8_element(p, p.n_tiled + i, bad);
+            fused_q8_element(p, a, p.n_tiled + i, bad);
     flag_overflow(bad, p.status);
     pdl_leave(p.chained);
 }
 
+template <bool kDC>
 __global__ void __launch_bounds__(256) fused_q8_plain_kernel(const __grid_constant__ FusedQ8Args p) {
+    ZK_STEP_CONSTS(p, a);
     bool bad = false;
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
     for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n; i += stride)
-        fused_q8_element(p, i, bad);
+        fused_q8_element(p, a, i, bad);
     flag_overflow(bad, p.status);
 }
 
@@ -390,8 +395,8 @@ cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, uint8_t* payload,
 cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,
                             const float* master_in, const float* m_in, const float* v_in,
                             float* master_out, float* m_out, float* v_out, uint16_t* param_out,
-                            const AdamConsts& a, const MeanConsts& mc, uint32_t* status,
-                            cudaStream_t stream) {
+                            const AdamConsts& a, const AdamConsts* ad, const MeanConsts& mc,
+                            uint32_t* status, cudaStream_t stream) {
     FusedQ8Args p;
     memset(&p, 0, sizeof(p));
     bool all16 = aligned16(master_in) && aligned16(m_in) && aligned16(v_in) &&
@@ -412,12 +417,16 @@ cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,
     p.nd = nd;
     p.param_vec = store_vec(param_out);
     p.a = a;
+    p.ad = ad;
     p.mc = mc;
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
     if (!all16 || n < kMinTiledElems) {
-        fused_q8_plain_kernel<<<plain_grid(n, di.sms), 256, 0, stream>>>(p);
+        if (ad)
+            fused_q8_plain_kernel<true><<<plain_grid(n, di.sms), 256, 0, stream>>>(p);
+        else
+            fused_q8_plain_kernel<false><<<plain_grid(n, di.sms), 256, 0, stream>>>(p);
         count_launch();
         return cudaGetLastError();
     }
@@ -441,12 +450,22 @@ cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,
     p.n_tiled = n & ~(kQTileAlign - 1);
     p.num_tiles = (p.n_tiled + sh.g.tile - 1) / sh.g.tile;
     p.chained = overlap_next(stream) ? 1 : 0;
+    if (ad) {
+        switch (sh.warps) {
+            case 8: return launch_pipe(fused_q8_tma_kernel<8, true>, p, sh, stream);
+            case 12: return launch_pipe(fused_q8_tma_kernel<12, true>, p, sh, stream);
+            case 16: return launch_pipe(fused_q8_tma_kernel<16, true>, p, sh, stream);
+            case 20: return launch_pipe(fused_q8_tma_kernel<20, true>, p, sh, stream);
+            case 24: return launch_pipe(fused_q8_tma_kernel<24, true>, p, sh, stream);
+        }
+        return cudaErrorInvalidConfiguration;
+    }
     switch (sh.warps) {
-        case 8: return launch_pipe(fused_q8_tma_kernel<8>, p, sh, stream);
-        case 12: return launch_pipe(fused_q8_tma_kernel<12>, p, sh, stream);
-        case 16: return launch_pipe(fused_q8_tma_kernel<16>, p, sh, stream);
-        case 20: return launch_pipe(fused_q8_tma_kernel<20>, p, sh, stream);
-        case 24: return launch_pipe(fused_q8_tma_kernel<24>, p, sh, stream);
+        case 8: return launch_pipe(fused_q8_tma_kernel<8, false>, p, sh, stream);
+        case 12: return launch_pipe(fused_q8_tma_kernel<12, false>, p, sh, stream);
+        case 16: return launch_pipe(fused_q8_tma_kernel<16, false>, p, sh, stream);
+        case 20: return launch_pipe(fused_q8_tma_kernel<20, false>, p, sh, stream);
+        case 24: return launch_pipe(fused_q8_tma_kernel<24, false>, p, sh, stream);
     }
     return cudaErrorInvalidConfiguration;
 }

@@ -47,7 +47,7 @@ SYMBOLS = (
     "zero_reduce_scatter_bucket", "zero_adam_shard", "zero_step_fused", "zero_step_commit",
     "zero_step_status", "zero_adam_consts_for_step", "zero_adam_shard_dc", "zero_step_fused_dc",
     "zero_selftest_timeout", "zero_adam_consts_table", "zero_scaler_prepare",
-    "zero_scaler_update", "zero_quantize_q8", "zero_step_fused_q8",
+    "zero_scaler_update", "zero_quantize_q8", "zero_step_fused_q8", "zero_step_fused_q8_dc",
     "zero_overlap_begin", "zero_overlap_end",
     "zero_sched_slot_elems", "zero_sched_create", "zero_sched_create_fused",
     "zero_sched_begin_bucket",
@@ -141,6 +141,7 @@ def _load():
     L.zero_quantize_q8.argtypes = [u64, vp, vp, vp]
     L.zero_step_fused_q8.argtypes = [u64, i32, P(vp), vp, vp, vp, vp, vp, vp, vp,
                                      P(_HP), i64, vp, vp]
+    L.zero_step_fused_q8_dc.argtypes = [u64, i32, P(vp), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.zero_adam_consts_table.argtypes = [P(_HP), i64, i64, P(AdamConsts)]
     L.zero_scaler_prepare.argtypes = [vp, vp, i64, vp, vp, vp]
     L.zero_scaler_update.argtypes = [vp, P(ScalerParams), vp, vp]
@@ -336,6 +337,15 @@ def zero_step_fused_q8(n: int, nd: int, rank_payload, master_in, m_in, v_in, mas
                                    _ptr(m_out, 4), _ptr(v_out, 4), _ptr(param_out, 2),
                                    C.byref(h), step, _ptr(d_status, 4), _stream(stream)),
            "zero_step_fused_q8")
+
+
+def zero_step_fused_q8_dc(n: int, nd: int, rank_payload, master_in, m_in, v_in, master_out,
+                          m_out, v_out, param_out, d_consts, d_status, stream=None):
+    _check(_lib.zero_step_fused_q8_dc(n, nd, _ptr_array(rank_payload, 1), _ptr(master_in, 4),
+                                      _ptr(m_in, 4), _ptr(v_in, 4), _ptr(master_out, 4),
+                                      _ptr(m_out, 4), _ptr(v_out, 4), _ptr(param_out, 2),
+                                      _ptr(d_consts), _ptr(d_status, 4), _stream(stream)),
+           "zero_step_fused_q8_dc")
 
 
 def zero_step_commit(n: int, master_in, m_in, v_in, master_out, m_out, v_out, param_out,
