@@ -231,10 +231,16 @@ class Workload:
                 self.g_status.zero_()
             if self.overlap:
                 lz.zero_overlap_begin()
-            for lo, hi in self.ranges:
-                lz.zero_step_fused_dc(hi - lo, self.nd, [g[lo:hi] for g in self.grads],
-                                      *[x[lo:hi] for x in src], *[x[lo:hi] for x in dst],
-                                      self.params[lo:hi], self.d_consts, self.g_status)
+            nd = self.nd
+            for i, (lo, hi) in enumerate(self.ranges):
+                if self.payload == "q8":
+                    lz.zero_step_fused_q8_dc(hi - lo, nd, self.q[i * nd:(i + 1) * nd],
+                                             *[x[lo:hi] for x in src], *[x[lo:hi] for x in dst],
+                                             self.params[lo:hi], self.d_consts, self.g_status)
+                else:
+                    lz.zero_step_fused_dc(hi - lo, nd, [g[lo:hi] for g in self.grads],
+                                          *[x[lo:hi] for x in src], *[x[lo:hi] for x in dst],
+                                          self.params[lo:hi], self.d_consts, self.g_status)
             if self.overlap:
                 lz.zero_overlap_end()
             lz.zero_step_commit(self.n, *src, *dst, self.params, self.g_status)
@@ -657,8 +663,8 @@ def run_ours(args):
     if args.dynamic_scale and not args.graph:
         raise SystemExit("--dynamic-scale needs --graph")
     if args.graph:
-        if wl.grads is None:
-            raise SystemExit("--graph applies to the fp16 stage-1 and flat workloads")
+        if wl.grads is None and wl.payload != "q8":
+            raise SystemExit("--graph applies to the stage-1 and flat workloads")
         wl.enable_graph(dynamic=args.dynamic_scale, max_steps=args.steps + args.warmup + 4)
     K, W = args.steps, args.warmup
     status = torch.zeros(K + W, dtype=torch.int32, device=dev)   # one status word per step
