@@ -84,6 +84,48 @@ def parse():
 # ---------------------------------------------------------------------------------------------
 # workloads
 # ---------------------------------------------------------------------------------------------
+def workload_config(args) -> dict:
+    """The workload's name and sizes as both arms report them (no device needed)."""
+    from zero_partitioned_optimizer_plan_b200 import synth
+    kind = args.workload
+    if kind == "gpt2_small":
+        nd = args.nd or 8
+        numels = synth.gpt2_small_list()
+        cfg = {"workload": "gpt2_small_stage1", "psi": sum(numels), "nd": nd, "stage": 1,
+               "calls_per_step": 1, "tensors": len(numels)}
+    elif kind == "shard_7p5b":
+        nd = args.nd or 64
+        total = 7_500_000_000
+        cfg = {"workload": "shard_7p5b_rank31", "psi_total": total, "shard": total // nd,
+               "nd": nd, "owner": 31, "calls_per_step": 1}
+    elif kind in ("zero2_1p3b", "zero2_gpt2_small"):
+        small = kind == "zero2_gpt2_small"
+        nd = args.nd or (8 if small else 16)
+        B = args.bucket or (10_000_000 if small else 50_000_000)
+        numels = synth.gpt2_small_list() if small else synth.gpt_1p3b_list()
+        psi = sum(numels)
+        psi_p = -(-psi // nd) * nd
+        nb = -(-psi_p // B)
+        cfg = {"workload": kind, "psi": psi, "nd": nd, "stage": 2, "bucket": B, "buckets": nb,
+               "calls_per_step": nb + nd}
+        if args.stage2_fused:
+            cfg["workload"] = kind + "_fused"
+            cfg["calls_per_step"] = nb + 1
+        return cfg
+    else:
+        nd = args.nd or 16
+        psi = args.psi or (1 << 29)
+        B = args.bucket or min(psi, 1 << 26)
+        cfg = {"workload": "flat_2p29" if psi == 1 << 29 else f"flat_{psi}", "psi": psi,
+               "nd": nd, "bucket": B, "calls_per_step": -(-psi // B)}
+    if cfg["calls_per_step"] > 1:
+        cfg["overlap"] = not args.no_overlap
+    if args.payload == "q8":
+        cfg["payload"] = "int8 records: 128 values and their fp32 scale"
+        cfg["workload"] += "_q8"
+    return cfg
+
+
 class Workload:
     """Device buffers and the per-step call sequence of one workload."""
 
@@ -111,8 +153,7 @@ class Workload:
             master, m, v = synth.state_small(psi_p, seed=0, device=dev)
             self.params = torch.empty(psi_p, dtype=torch.float16, device=dev)
             self.param_base = 0
-            self.config = {"workload": "gpt2_small_stage1", "psi": psi, "nd": nd, "stage": 1,
-                           "calls_per_step": 1, "tensors": len(numels)}
+            self.config = workload_config(args)
         elif kind == "shard_7p5b":
             nd = args.nd or 64
             total = 7_500_000_000
@@ -126,8 +167,7 @@ class Workload:
             self.full = torch.zeros(total, dtype=torch.float16, device=dev)
             self.params = self.full[r * S:(r + 1) * S]
             self.param_base = r * S
-            self.config = {"workload": "shard_7p5b_rank31", "psi_total": total, "shard": S,
-                           "nd": nd, "owner": r, "calls_per_step": 1}
+            self.config = workload_config(args)
         elif kind in ("zero2_1p3b", "zero2_gpt2_small"):
             self._init_zero2(args, dev)
             return
@@ -147,9 +187,8 @@ class Workload:
             master, m, v = synth.state_warm(psi, seed=0, device=dev)
             self.params = torch.empty(psi, dtype=torch.float16, device=dev)
             self.param_base = 0
-            self.config = {"workload": "flat_2p29" if psi == 1 << 29 else f"flat_{psi}",
-                           "psi": psi, "nd": nd, "bucket": B,
-                           "calls_per_step": len(self.ranges)}
+            self.config = workload_config(args)
+            assert self.config["calls_per_step"] == len(self.ranges)
         self.cur = [master, m, v]
         self.nxt = [torch.empty_like(x) for x in self.cur]
         self.bytes_per_step = (2 * self.nd + 26) * self.n     # algorithmic HBM bytes
@@ -161,8 +200,6 @@ class Workload:
         self.payload = args.payload
         # the per-bucket calls of a step touch disjoint ranges: declare them independent
         self.overlap = len(self.ranges) > 1 and not args.no_overlap
-        if len(self.ranges) > 1:
-            self.config["overlap"] = self.overlap
         if self.payload == "q8":
             self._quantize_payload()
 
@@ -193,8 +230,6 @@ class Workload:
         self.bytes_per_step = nd * 132 * recs + 26 * n
         self.dominant = "fused_q8_tma_kernel"
         self.dominant_bytes = self.bytes_per_step
-        self.config["payload"] = "int8 records: 128 values and their fp32 scale"
-        self.config["workload"] += "_q8"
 
     def inputs(self):
         """The tensors a step consumes that a host would have to upload."""
@@ -366,8 +401,8 @@ def _init_zero2(self, args, dev):
     self.ranges = [(0, psi_p)]
     self.overlap = False
     self.param_base = 0
-    self.config = {"workload": args.workload, "psi": psi, "nd": nd, "stage": 2, "bucket": B,
-                   "buckets": nb, "calls_per_step": nb + nd}
+    self.config = workload_config(args)
+    assert (self.config["psi"], self.config["buckets"]) == (psi, nb)
     if args.stage2_fused:
         # the scheduler launches the fused step per bucket; ping-pong state, commit at the end
         self.cur = [self.master, self.m, self.v]
@@ -375,8 +410,6 @@ def _init_zero2(self, args, dev):
         self.d_consts = torch.empty(40, dtype=torch.uint8, device=dev)
         self.h_consts = [torch.empty(40, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
         self.h_done = [None, None]
-        self.config["workload"] = args.workload + "_fused"
-        self.config["calls_per_step"] = nb + 1
         self.bytes_per_step = (2 * nd + 26) * psi_p
         self.dominant = "fused_tma_kernel"
         self.dominant_bytes = self.bytes_per_step
@@ -560,6 +593,20 @@ def traffic_per_launch(kernel: str, workload: str):
     return None
 
 
+def host_cpu() -> dict:
+    """The host's CPU model and hardware thread count (the oracle itself uses one core)."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu": model, "threads": os.cpu_count()}
+
+
 def cpu_oracle_rate(nd: int, n_sample: int, target_s: float, seed=0):
     """Time the oracle (single-threaded C, as it stands) on n_sample elements of the workload's
     distribution; repeat until target_s seconds have passed. Returns (params/s, reps, secs)."""
@@ -608,7 +655,8 @@ def run_reference(args):
     ws, rank, _ = dist_setup(args)
     if rank != 0:
         return 0
-    nd = args.nd or {"gpt2_small": 8, "shard_7p5b": 64, "flat": 16}[args.workload]
+    cfg = workload_config(args)
+    nd = cfg["nd"]
     # calibrate, then size each step so that the whole run takes about two minutes
     rate, _, _ = cpu_oracle_rate(nd, 200_000, 0.2)
     per_step_s = max(0.05, 120.0 / (args.steps + args.warmup))
@@ -626,16 +674,16 @@ def run_reference(args):
         _, master, m, v, _ = oracle.step(g, master, m, v, hp, t)
     dt = time.perf_counter() - t0
     value = n_sample * args.steps / dt
-    sample = (f"first {n_sample} elements of the {args.workload} workload's distribution, "
-              f"Nd={nd}, one oracle step per timed step")
+    sample = (f"first {n_sample} elements of the {cfg['workload']} workload's gradient "
+              f"distribution, Nd={nd}, one oracle step per timed step")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "params/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": args.workload, "nd": nd, "sample_elems": n_sample},
+        "config": dict(cfg, sample_elems=n_sample, parallelism="replicas1"),
         "cpu_baseline": {"value": value, "unit": "params/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "host": host_cpu()},
         "e2e": {"value": value, "unit": "params/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -795,7 +843,8 @@ def run_ours(args):
         rate, reps, secs = cpu_oracle_rate(wl.nd, n_sample, 10.0)
         cpu = {"value": rate, "unit": "params/s", "cores": 1, "kind": "oracle",
                "sample": f"{n_sample} elements with the workload's gradient distribution, "
-                         f"Nd={wl.nd}, {reps} oracle steps, {secs:.1f} s"}
+                         f"Nd={wl.nd}, {reps} oracle steps, {secs:.1f} s",
+               "host": host_cpu()}
 
     if rank == 0:
         cfg = dict(wl.config)
