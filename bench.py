@@ -111,6 +111,7 @@ def workload_config(args) -> dict:
         if args.stage2_fused:
             cfg["workload"] = kind + "_fused"
             cfg["calls_per_step"] = nb + 1
+        cfg["overlap"] = not args.no_overlap
         return cfg
     else:
         nd = args.nd or 16
@@ -399,7 +400,8 @@ def _init_zero2(self, args, dev):
     self.shards = torch.empty(psi_p, dtype=torch.float32, device=dev)
     self.grads = None
     self.ranges = [(0, psi_p)]
-    self.overlap = False
+    # the buckets' reduce-scatters (or fused steps) of a step touch disjoint ranges
+    self.overlap = not args.no_overlap
     self.param_base = 0
     self.config = workload_config(args)
     assert (self.config["psi"], self.config["buckets"]) == (psi, nb)
@@ -438,9 +440,13 @@ def _step_zero2(self, t, status, ev=None, grads=None):
                                stream)
     if ev is not None:
         ev[0].record()
+    if self.overlap:
+        lz.zero_overlap_begin(stream)
     for k in range(self.nb):
         lz.zero_sched_begin_bucket(sch, k, stream)
         lz.zero_sched_end_bucket(sch, k, stream)
+    if self.overlap:
+        lz.zero_overlap_end(stream)
     lz.zero_sched_wait(sch, stream)
     if ev is not None:
         ev[1].record()
@@ -468,9 +474,13 @@ def _step_zero2_fused(self, t, status, ev=None, grads=None):
                                      *self.nxt, self.params, self.d_consts, status, stream)
     if ev is not None:
         ev[0].record()
+    if self.overlap:
+        lz.zero_overlap_begin(stream)
     for k in range(self.nb):
         lz.zero_sched_begin_bucket(sch, k, stream)
         lz.zero_sched_end_bucket(sch, k, stream)
+    if self.overlap:
+        lz.zero_overlap_end(stream)
     lz.zero_sched_wait(sch, stream)
     if ev is not None:
         ev[1].record()

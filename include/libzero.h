@@ -366,8 +366,10 @@ zero_status zero_selftest_timeout(uint32_t* d_status, zero_stream_t stream);
  * so work enqueued after the region (zero_step_commit, a copy, an event) is ordered after the
  * whole region as usual. Calls that take the plain-load kernels, and all other calls, stay
  * ordered. Other work enqueued on the stream inside the region must be ordinary launches,
- * copies or event waits (a kernel that itself uses programmatic dependent launch, as some
- * libraries' kernels do, needs the region closed before it).
+ * copies, event records or event waits (a kernel that itself uses programmatic dependent
+ * launch, as some libraries' kernels do, needs the region closed before it); an event recorded
+ * after a call completes only when that call and every call before it have. The bucket
+ * scheduler's calls (zero_sched_end_bucket on its stream) may sit in a region.
  * Host-side state only (one flag per stream, thread-safe): both calls enqueue nothing and can
  * be used while a CUDA graph is captured. The pages have no counterpart; this is a launch
  * device of this library. Errors: ZERO_EINVAL (begin on a stream whose region is open, end on

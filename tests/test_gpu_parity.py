@@ -273,11 +273,14 @@ def test_alignment_variants(grad_off, state_off, param_off):
     assert not pbig[param_off + n:].view(torch.int16).any()
 
 
+@pytest.mark.parametrize("overlap", [False, True])
 @pytest.mark.parametrize("n_slots", [1, 2, 3])
-def test_stage2_scheduler_vs_oracle(n_slots):
+def test_stage2_scheduler_vs_oracle(n_slots, overlap):
     """Buckets in backward order through the scheduler: the producer fills a staging slot on
     its own stream, the reduce-scatter runs on the scheduler's stream after it, the slot is
-    released for a later bucket when the reduce-scatter is done; then the owner updates."""
+    released for a later bucket when the reduce-scatter is done; then the owner updates. With
+    `overlap` the scheduler's stream is an overlap region (the bucket kernels chained), so the
+    release events follow kernels that may overlap the next bucket's."""
     numels, nd, bucket = [40000, 1234, 30000, 777], 6, 9000
     pl = lz.zero_plan_create(numels, nd, 2, bucket)
     psi, psi_p, S, nb = lz.zero_plan_info(pl)
@@ -297,6 +300,8 @@ def test_stage2_scheduler_vs_oracle(n_slots):
     torch.cuda.synchronize()
     sch = lz.zero_sched_create(pl, slots, slot_elems, n_slots,
                                [shards[r * S:(r + 1) * S] for r in range(nd)], st, rs)
+    if overlap:
+        lz.zero_overlap_begin(rs)
     with torch.cuda.stream(producer):
         for k in range(nb):
             lo, ln, _, _ = lz.zero_plan_bucket(pl, k)
@@ -306,6 +311,8 @@ def test_stage2_scheduler_vs_oracle(n_slots):
                     slots.untyped_storage(), (ptrs[r] - slots.data_ptr()) // 2, (ln,))
                 dst.copy_(g_src[r][lo:lo + ln])      # the "backward pass" writes bucket k
             lz.zero_sched_end_bucket(sch, k, producer)
+    if overlap:
+        lz.zero_overlap_end(rs)
     main = torch.cuda.current_stream()
     lz.zero_sched_wait(sch, main)
     assert lz.zero_sched_launches(sch) == nb
@@ -326,8 +333,9 @@ def test_stage2_scheduler_vs_oracle(n_slots):
     lz.zero_sched_destroy(sch)
 
 
+@pytest.mark.parametrize("overlap", [False, True])
 @pytest.mark.parametrize("n_slots", [1, 3])
-def test_stage2_fused_scheduler_vs_oracle(n_slots):
+def test_stage2_fused_scheduler_vs_oracle(n_slots, overlap):
     """The scheduler in fused mode: each bucket's kernel is the fused step over its range (the
     reduced gradient never stored), slots released after it; commit after the last bucket.
     Equals the oracle's stage-2 step; then an inf in one bucket skips the whole step."""
@@ -356,6 +364,8 @@ def test_stage2_fused_scheduler_vs_oracle(n_slots):
         torch.cuda.synchronize()
         sch = lz.zero_sched_create_fused(pl, slots, slot_elems, n_slots, *ins, *outs, params,
                                          dc, st, stream)
+        if overlap:
+            lz.zero_overlap_begin(stream)
         with torch.cuda.stream(producer):
             for k in range(nb):
                 lo, ln, _, _ = lz.zero_plan_bucket(pl, k)
@@ -365,6 +375,8 @@ def test_stage2_fused_scheduler_vs_oracle(n_slots):
                         slots.untyped_storage(), (ptrs[r] - slots.data_ptr()) // 2, (ln,))
                     dst.copy_(g_src[r][lo:lo + ln])
                 lz.zero_sched_end_bucket(sch, k, producer)
+        if overlap:
+            lz.zero_overlap_end(stream)
         main = torch.cuda.current_stream()
         lz.zero_sched_wait(sch, main)
         lz.zero_step_commit(psi_p, *ins, *outs, params, st)

@@ -119,6 +119,7 @@ def test_1p3b_stage2_fused_scheduler_with_overflow_run():
         sch = lz.zero_sched_create_fused(pl, slots, slot_elems, n_slots, *cur, *nxt, params,
                                          d_consts, st, stream)
         gathered = [np.empty(idx.size, np.uint16) for _ in range(nd)]
+        lz.zero_overlap_begin(stream)      # as bench.py: the bucket kernels chained
         with torch.cuda.stream(producer):
             for k in range(nb):
                 lo, ln, _, _ = lz.zero_plan_bucket(pl, k)
@@ -133,6 +134,7 @@ def test_1p3b_stage2_fused_scheduler_with_overflow_run():
                 for r in range(nd):
                     gathered[r][sel] = views[r][local].cpu().numpy().view(np.uint16)
                 lz.zero_sched_end_bucket(sch, k, producer)
+        lz.zero_overlap_end(stream)
         lz.zero_sched_wait(sch, main)
         lz.zero_step_commit(psi_p, *cur, *nxt, params, st, main)
         code, flags = lz.zero_step_status(st, main)
@@ -188,6 +190,7 @@ def test_1p3b_stage2_buckets_with_overflow_run():
         sch = lz.zero_sched_create(pl, slots, slot_elems, n_slots,
                                    [shards[r * S:(r + 1) * S] for r in range(nd)], st, rs)
         gathered = [np.empty(idx.size, np.uint16) for _ in range(nd)]
+        lz.zero_overlap_begin(rs)          # as bench.py: the bucket kernels chained
         with torch.cuda.stream(producer):
             for k in range(nb):
                 lo, ln, _, _ = lz.zero_plan_bucket(pl, k)
@@ -202,6 +205,7 @@ def test_1p3b_stage2_buckets_with_overflow_run():
                 for r in range(nd):
                     gathered[r][sel] = views[r][local].cpu().numpy().view(np.uint16)
                 lz.zero_sched_end_bucket(sch, k, producer)
+        lz.zero_overlap_end(rs)
         lz.zero_sched_wait(sch, main)
         assert lz.zero_sched_launches(sch) == nb
         for r in range(nd):   # each owner updates its shard and writes it into the full buffer
