@@ -371,7 +371,8 @@ zero_status zero_selftest_timeout(uint32_t* d_status, zero_stream_t stream);
  * after a call completes only when that call and every call before it have. The bucket
  * scheduler's calls (zero_sched_end_bucket on its stream) may sit in a region.
  * Host-side state only (one flag per stream, thread-safe): both calls enqueue nothing and can
- * be used while a CUDA graph is captured. The pages have no counterpart; this is a launch
+ * be used while a CUDA graph is captured. Close a region before its stream is destroyed (the
+ * flag is keyed by the stream handle, which a later stream may reuse). The pages have no counterpart; this is a launch
  * device of this library. Errors: ZERO_EINVAL (begin on a stream whose region is open, end on
  * a stream without one).
  * ---------------------------------------------------------------------------------------- */
