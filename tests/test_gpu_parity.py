@@ -405,6 +405,52 @@ def test_stage2_fused_scheduler_vs_oracle(n_slots, overlap):
     assert np.array_equal(f16np(params), oracle.f2h(w_np))
 
 
+@pytest.mark.parametrize("nd", [3, 8])
+@pytest.mark.parametrize("loss_scale", [1000.0, 1024.0, 1.0])
+def test_fused_step_special_values(nd, loss_scale):
+    """Gradients made of special fp16 values -- +0, -0, subnormals (the smallest, the largest),
+    the smallest and largest normals, 65504 and its negation, and values whose sum cancels --
+    with a non-power-of-two Nd (the mean by division) and a loss scale that is not a power of
+    two (the unscale by division), over a range that takes the bulk-copy pipeline with a
+    ragged tail. Zero gradients with zero m and v leave master unchanged."""
+    n = 3072 * 9 + 5
+    special = np.array([0x0000, 0x8000, 0x0001, 0x8001, 0x03ff, 0x83ff, 0x0400, 0x8400,
+                        0x7bff, 0xfbff, 0x3c00, 0xbc00, 0x1400, 0x9400], np.uint16)
+    rng = np.random.default_rng(1000 + nd)
+    g_cpu = []
+    for r in range(nd):
+        pick = special[rng.integers(0, special.size, size=n)]
+        g = torch.from_numpy(pick.view(np.int16).copy()).view(torch.float16)
+        g_cpu.append(g)
+    # a block of exact cancellation: rank r holds (-1)^r * 65504 (Nd = 8: sum 0)
+    for r in range(nd):
+        g_cpu[r][100:200] = 65504.0 if r % 2 == 0 else -65504.0
+    # a block of all-zero gradients at all ranks
+    for r in range(nd):
+        g_cpu[r][3000:3100] = 0.0
+    master, m, v = synth.state_warm(n, seed=77)
+    m[3000:3050] = 0.0
+    v[3000:3050] = 0.0
+    hp = lz.AdamHP(loss_scale=loss_scale)
+    ohp = oracle.AdamHP(loss_scale=loss_scale)
+    pp = PingPong(master, m, v)
+    params = torch.empty(n, dtype=torch.float16, device=DEV)
+    st = status_word()
+    fused_step(n, [g.to(DEV) for g in g_cpu], pp, params, hp, 2, st)
+    torch.cuda.synchronize()
+    assert status_flags(st) == 0
+    pp.swap()
+    skipped, w, mm, vv, p = oracle.step([g.numpy() for g in g_cpu], master.numpy(), m.numpy(),
+                                        v.numpy(), ohp, 2)
+    assert not skipped
+    got = pp.numpy()
+    check_f32("master", got[0], w)
+    check_f32("m", got[1], mm)
+    check_f32("v", got[2], vv)
+    check_f16("params", f16np(params), p)
+    assert np.array_equal(got[0][3000:3050], master.numpy()[3000:3050])
+
+
 def test_step_split_into_bucket_calls():
     """One step made of several zero_step_fused calls (one per bucket, backward order) and one
     commit equals the single-call step; an overflow in a late bucket skips all of it."""
