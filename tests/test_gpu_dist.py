@@ -1,0 +1,84 @@
+"""The distributed step (dist.py) on the GPU through NCCL and the library's kernels, with the one
+rank a single-GPU run allows (the all-to-all, all-reduce and all-gather then move data only
+within the rank); the exchange between several ranks is tested on CPU processes over gloo
+(test_multirank.py). Against the oracle's data-parallel step, tolerances as in
+test_gpu_parity.py."""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+pytestmark = pytest.mark.gpu
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _case(numels):
+    import torch
+    from zero_partitioned_optimizer_plan_b200 import synth
+    psi = sum(numels)
+    grad = synth.grad_f16(psi, 1e-3, seed=11, rank=0, step=1)
+    master, m, v = synth.state_warm(psi, seed=12)
+    return psi, grad, master, m, v, torch
+
+
+def _worker(port, numels, bucket, out):
+    import datetime
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from zero_partitioned_optimizer_plan_b200 import libzero as lz
+    from zero_partitioned_optimizer_plan_b200.dist import DistZeroStep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.cuda.set_device(0)
+    dist.init_process_group("nccl", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        psi, grad, master, m, v, _ = _case(numels)
+        dev = "cuda:0"
+        st_in = [x.to(dev) for x in (master, m, v)]
+        st_out = [torch.full_like(x, float("nan")) for x in st_in]
+        params = torch.zeros(psi, dtype=torch.float16, device=dev)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        step = DistZeroStep(psi, bucket)
+        flag = step.step(grad.to(dev), st_in, st_out, params, lz.AdamHP(), 1, status)
+        torch.cuda.synchronize()
+        out.put((int(flag.item()), int(status.item()), [x.cpu().numpy() for x in st_out],
+                 params.cpu().numpy().view(np.uint16)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("bucket", [0, 3000])
+def test_distributed_step_one_rank_nccl(bucket):
+    import oracle
+    numels = [1000, 37, 4099, 12345]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_worker, args=(_free_port(), numels, bucket, q))
+    p.start()
+    try:
+        flag, status, shard, params = q.get(timeout=240)
+    finally:
+        p.join(60)
+        if p.exitcode is None:
+            p.kill()
+    assert p.exitcode == 0
+    psi, grad, master, m, v, _ = _case(numels)
+    ref = oracle.dp_step([grad.numpy()], master.numpy(), m.numpy(), v.numpy(),
+                         oracle.f2h(master.numpy()), oracle.AdamHP(), 1)
+    assert (flag, status) == (0, 0) and not ref.skipped
+    for name, got, want in zip(("master", "m", "v"), shard, (ref.master, ref.m, ref.v)):
+        d = oracle.ulp_diff_f32(got, want)
+        assert int(d.max()) <= 2, name
+    assert int(oracle.ulp_diff_f16(params, ref.params16).max()) <= 1

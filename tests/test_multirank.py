@@ -112,3 +112,115 @@ def test_failed_rank_is_detected_on_the_host(mode):
     rank, verdict, _ = q.get()
     assert (rank, verdict) == (0, "error")
     assert time.monotonic() - t0 < 170
+
+
+# ---------------------------------------------------------------------------------------------
+# the distributed step (dist.py): its exchange on CPU processes over gloo, with the owner's
+# fused step and commit done by the oracle (the library needs a GPU)
+# ---------------------------------------------------------------------------------------------
+class _OracleCompute:
+    def fused(self, n, rows, state_in, state_out, params, hp, t, status):
+        import numpy as np
+        import oracle
+        red = oracle.reduce_mean([row.numpy() for row in rows])
+        if not oracle.all_finite(red):
+            status |= 1
+            return
+        w, m, v, p16 = oracle.adam(red, *(x.numpy() for x in state_in), hp, t)
+        for dst, src in zip(state_out, (w, m, v)):
+            dst.copy_(__import__("torch").from_numpy(np.ascontiguousarray(src)))
+        params.view(__import__("torch").int16).copy_(
+            __import__("torch").from_numpy(np.ascontiguousarray(p16).view(np.int16)))
+
+    def commit(self, n, state_in, state_out, params, status):
+        import numpy as np
+        import torch
+        import oracle
+        if int(status.item()) & 1:
+            for dst, src in zip(state_out, state_in):
+                dst.copy_(src)
+            params.view(torch.int16).copy_(
+                torch.from_numpy(oracle.f2h(state_in[0].numpy()).view(np.int16)))
+            status |= 2
+
+
+def _dist_case(numels, ws, bad_rank):
+    """Every rank's inputs of the case, the same on every process (seeded)."""
+    import torch
+    from zero_partitioned_optimizer_plan_b200 import synth
+    psi = sum(numels)
+    psi_p = -(-psi // ws) * ws
+    grads = []
+    for r in range(ws):
+        g = torch.zeros(psi_p, dtype=torch.float16)
+        g[:psi] = synth.grad_f16(psi, 1e-3, seed=7, rank=r, step=1)
+        if r == bad_rank:
+            g[psi // 2] = float("inf")
+        grads.append(g)
+    master, m, v = synth.state_warm(psi_p, seed=8)
+    return psi_p, grads, master, m, v
+
+
+def _worker_dist(rank, ws, port, numels, bucket, bad_rank, out):
+    import datetime
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle
+    from zero_partitioned_optimizer_plan_b200.dist import DistZeroStep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        psi_p, grads, master, m, v = _dist_case(numels, ws, bad_rank)
+        S = psi_p // ws
+        st_in = [x[rank * S:(rank + 1) * S].clone() for x in (master, m, v)]
+        st_out = [torch.full_like(x, float("nan")) for x in st_in]
+        params = torch.zeros(psi_p, dtype=torch.float16)
+        params[rank * S:(rank + 1) * S] = torch.from_numpy(
+            oracle.f2h(st_in[0].numpy()).view("float16"))
+        status = torch.zeros(1, dtype=torch.int32)
+        step = DistZeroStep(psi_p, bucket, compute=_OracleCompute())
+        flag = step.step(grads[rank], st_in, st_out, params, oracle.AdamHP(), 1, status)
+        out.put((rank, int(flag.item()), int(status.item()), [x.numpy() for x in st_out],
+                 params.numpy().view("uint16")))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("ws,bucket,bad_rank", [(2, 0, -1), (3, 0, -1), (2, 3000, -1),
+                                                (3, 2500, -1), (3, 2500, 1)])
+def test_distributed_step_exchange_gloo(ws, bucket, bad_rank):
+    """The distributed step's all-to-all / all-reduce / all-gather on gloo ranks gives the
+    single-process data-parallel step of the oracle (all ranks' gradients summed in rank
+    order): every rank's shard of the state and every rank's full fp16 parameters; an inf in
+    one rank's gradient skips the step on every rank."""
+    import numpy as np
+    import oracle
+    numels = [1000, 37, 4099, 12345]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_dist, args=(r, ws, port, numels, bucket, bad_rank, q))
+             for r in range(ws)]
+    for p in procs:
+        p.start()
+    try:   # read before joining: a result larger than the pipe buffer blocks its sender
+        res = sorted((q.get(timeout=240) for _ in range(ws)), key=lambda x: x[0])
+    finally:
+        for p in procs:
+            p.join(60)
+            if p.exitcode is None:
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    psi_p, grads, master, m, v = _dist_case(numels, ws, bad_rank)
+    ref = oracle.dp_step([g.numpy() for g in grads], master.numpy(), m.numpy(), v.numpy(),
+                         oracle.f2h(master.numpy()), oracle.AdamHP(), 1)
+    S = psi_p // ws
+    for rank, flag, status, shard, params in res:
+        assert flag == (1 if bad_rank >= 0 else 0)
+        assert bool(status & 2) == ref.skipped == (bad_rank >= 0)
+        for got, want in zip(shard, (ref.master, ref.m, ref.v)):
+            assert np.array_equal(got.view(np.uint32),
+                                  want[rank * S:(rank + 1) * S].view(np.uint32))
+        assert np.array_equal(params, ref.params16)
