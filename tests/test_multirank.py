@@ -224,3 +224,23 @@ def test_distributed_step_exchange_gloo(ws, bucket, bad_rank):
             assert np.array_equal(got.view(np.uint32),
                                   want[rank * S:(rank + 1) * S].view(np.uint32))
         assert np.array_equal(params, ref.params16)
+
+
+def test_dist_bucket_map_matches_the_plan():
+    """dist.py's bucket ranges and per-owner split sizes agree with the oracle's plan (backward
+    order, element-granular, last bucket short) for several sizes, bucket lengths and Nd."""
+    import oracle
+    from zero_partitioned_optimizer_plan_b200.dist import bucket_ranges, owner_parts
+    for numels, nd, bucket in [([1000, 37, 4099, 12345], 3, 2500), ([70001, 3], 4, 7),
+                               ([300000, 250000, 250000, 248576], 4, 100000),
+                               ([5, 5, 5], 2, 0), ([123457], 64, 1000)]:
+        pl = oracle.plan(numels, nd, bucket)
+        psi_p, S = pl.psi_p, pl.shard
+        got = bucket_ranges(psi_p, bucket)
+        want = [(lo, lo + ln) for lo, ln in pl.buckets]
+        assert got == want
+        for lo, hi in got:
+            parts = owner_parts(lo, hi, S, nd)
+            assert sum(parts) == hi - lo
+            owned = [q for q in range(nd) if parts[q] > 0]
+            assert owned == list(range(lo // S, (hi - 1) // S + 1))
