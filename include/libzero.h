@@ -111,7 +111,8 @@ zero_status zero_plan_bucket(const zero_plan* plan, int k, uint64_t* flat_lo, ui
  * A partitioned quantity counts ceil(psi/Nd) elements. Communication per step in elements:
  * 2psi (DP, Pos, Pos+g: reduce-scatter + all-gather), 3psi (Pos+g+p: two parameter
  * all-gathers + the reduce-scatter); comm_bytes_fp16 is twice that.
- * Errors: ZERO_EINVAL for out == NULL, nd < 1 or K < 0.
+ * Errors: ZERO_EINVAL for out == NULL, nd < 1, K < 0, or psi so large that a byte count
+ * would not fit in 64 bits (psi > UINT64_MAX / (K + 6)).
  * ---------------------------------------------------------------------------------------- */
 typedef struct {
     uint64_t params, grads, optim, total;

@@ -361,3 +361,13 @@ def test_q8_dc_rejects():
             lz.zero_step_fused_q8_dc(1000, 2, pays, *ins, *outs, A + 120 * MB, dc, A + 130 * MB, 0)
         assert e.value.code == code
     lz.zero_step_fused_q8_dc(0, 2, pays, *ins, *outs, A + 120 * MB, A + 140 * MB, A + 130 * MB, 0)
+
+
+def test_state_bytes_rejects_overflowing_sizes():
+    K = 12
+    lim = (2**64 - 1) // (K + 6)
+    rep = lz.zero_state_bytes(lim, 8, K)
+    assert rep[lz.STAGES[0]]["total"] == 16 * lim
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_state_bytes(lim + 1, 8, K)
+    assert e.value.code == lz.ZERO_EINVAL

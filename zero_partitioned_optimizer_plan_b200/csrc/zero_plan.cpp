@@ -128,8 +128,9 @@ zero_status zero_plan_bucket(const zero_plan* plan, int k, uint64_t* flat_lo, ui
 
 zero_status zero_state_bytes(uint64_t psi, int nd, int K, zero_state_report* out) {
     if (!out || nd < 1 || K < 0) return ZERO_EINVAL;
-    const uint64_t part = psi / (uint64_t)nd + (psi % (uint64_t)nd ? 1 : 0);
     const uint64_t k = (uint64_t)K;
+    if (psi > UINT64_MAX / (k + 6)) return ZERO_EINVAL;   // every byte count fits in 64 bits
+    const uint64_t part = psi / (uint64_t)nd + (psi % (uint64_t)nd ? 1 : 0);
     // {params, grads, optimizer} per stage: which of the three is partitioned
     const bool split[4][3] = {
         {false, false, false},   // plain DP: full replica
