@@ -569,13 +569,22 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_sources_sha256() -> str:
-    """One hash over every CUDA source of the library (the kernels the counters describe)."""
-    import glob
+# The source files each kernel is built from: a kernel's DRAM counters stay valid while these
+# files are unchanged.
+KERNEL_SOURCES = {
+    "fused_tma_kernel": ("zero_kernels.cu", "zero_device.cuh", "zero_internal.h"),
+    "rs_tma_kernel": ("zero_kernels.cu", "zero_device.cuh", "zero_internal.h"),
+    "adam_kernel": ("zero_kernels.cu", "zero_device.cuh", "zero_internal.h"),
+    "fused_q8_tma_kernel": ("zero_q8.cu", "zero_device.cuh", "zero_internal.h"),
+}
+
+
+def kernel_sources_sha256(kernel: str) -> str:
+    """One hash over the sources of `kernel` (the code the ncu counters describe)."""
     h = hashlib.sha256()
-    for path in sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))):
-        with open(path, "rb") as f:
-            h.update(os.path.basename(path).encode() + b"\0" + f.read())
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()
 
 
@@ -594,7 +603,7 @@ def traffic_per_launch(kernel: str, workload: str):
     try:
         with open(TRAFFIC_FILE) as f:
             tab = json.load(f)
-        sha = kernel_sources_sha256()
+        sha = kernel_sources_sha256(kernel)
         ent = tab.get(workload, {}).get(kernel)
         if ent and ent.get("kernel_src_sha256") == sha:
             return ent["dram_bytes_per_launch"]

@@ -17,9 +17,8 @@
 //
 // Per parameter the owner reads nd * 132/128 payload bytes instead of 2 * nd: at Nd = 64 the
 // fused step moves 92 bytes per parameter instead of 154. Per element and rank it issues a byte
-// conversion and a fused multiply-add; half of the bytes go through the integer-to-float
-// conversion pipe, half through the mantissa-placement trick on the integer and FMA pipes, so
-// neither pipe bounds the step.
+// conversion (the mantissa-placement trick: a byte permute, then the bias removal) and a fused
+// multiply-add, the float halves of both as packed two-wide fp32 instructions.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -143,12 +142,35 @@ __device__ __forceinline__ float dequant_add(int8_t q, float scale, float acc) {
 }
 
 // Byte j of `biased` (q + 128, in 0..255) placed in the low mantissa bits of 2^23 gives the
-// float 2^23 + q + 128; subtracting 2^23 + 128 leaves q exactly. Two full-rate instructions
-// instead of an integer-to-float conversion (a quarter-rate pipe), which otherwise bounds the
-// owner's step at large Nd.
-__device__ __forceinline__ float q_to_float(uint32_t biased, int j) {
-    return __fsub_rn(__uint_as_float(__byte_perm(biased, 0x4B000000u, 0x7440u | (uint32_t)j)),
-                     8388736.0f);
+// float 2^23 + q + 128; subtracting 2^23 + 128 leaves q exactly. Full-rate instructions instead
+// of an integer-to-float conversion (a quarter-rate pipe), which otherwise bounds the owner's
+// step at large Nd.
+__device__ __forceinline__ float q_placed(uint32_t biased, int j) {
+    return __uint_as_float(__byte_perm(biased, 0x4B000000u, 0x7440u | (uint32_t)j));
+}
+
+// Packed pairs of binary32 values (sm_100 executes two-wide fp32 add and fused multiply-add as
+// one instruction; each half is an ordinary IEEE operation rounded to nearest even).
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
 }
 
 __device__ __forceinline__ void fused_q8_element(const FusedQ8Args& p, const AdamConsts& a,
@@ -273,20 +295,27 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
                 const uint32_t nr = min(p.g.rc, (uint32_t)p.nd - c * p.g.rc);
                 // this thread's record in each rank's run; its 4 values share the scale
                 const uint8_t* rec0 = st + (size_t)(e0 / kQB) * kRec;
+                // the four accumulators as two packed pairs: per rank, two packed bias
+                // removals and two packed fused multiply-adds for the four values
+                static_assert(E == 4, "the rank loop packs four values per thread");
+                uint64_t a01 = f2_pack(acc[0], acc[1]), a23 = f2_pack(acc[2], acc[3]);
+                const uint64_t nbias = f2_pack(-8388736.0f, -8388736.0f);   // -(2^23 + 128)
 #pragma unroll 4
                 for (uint32_t r = 0; r < nr; ++r) {
                     const uint8_t* rec = rec0 + (size_t)r * p.row;
                     const uint32_t qq = *reinterpret_cast<const uint32_t*>(rec + e0 % kQB);
                     const float sc = *reinterpret_cast<const float*>(rec + kQB);
                     const uint32_t biased = qq ^ 0x80808080u;   // each byte q + 128
-#pragma unroll
-                    for (int j = 0; j < E; ++j) {
-                        // bytes 0, 1: conversion pipe; bytes 2, 3: integer and FMA pipes
-                        const float qf = (j < 2) ? __int2float_rn((int)(int8_t)(uint8_t)(qq >> (8 * j)))
-                                                 : q_to_float(biased, j);
-                        acc[j] = __fmaf_rn(qf, sc, acc[j]);
-                    }
+                    const uint64_t ss = f2_pack(sc, sc);
+                    const uint64_t q01 =
+                        f2_add(f2_pack(q_placed(biased, 0), q_placed(biased, 1)), nbias);
+                    const uint64_t q23 =
+                        f2_add(f2_pack(q_placed(biased, 2), q_placed(biased, 3)), nbias);
+                    a01 = f2_fma(q01, ss, a01);   // acc + q * scale, one rounding each
+                    a23 = f2_fma(q23, ss, a23);
                 }
+                f2_unpack(a01, acc[0], acc[1]);
+                f2_unpack(a23, acc[2], acc[3]);
                 if (c + 1 == p.g.nchunks) {
                     const uint8_t* sf = st + p.g.state_off + (size_t)e0 * 4u;
                     lds_f32<E>(sf, w);
