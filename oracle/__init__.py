@@ -17,8 +17,13 @@ adds the partitioning that ZeRO-DP performs around it, written with numpy slicin
                       as it is produced, the owner keeps its slice and the rest is released;
                       then the owner update and the all-gather ("ZeRO-2" card, "Gradient
                       생명주기" and "왜 all-gather는 그대로 필요한가").
+* ``zero3_step``   -- stage 3 (Pos+g+p): the fp16 parameters are partitioned as well; each
+                      layer's parameters are gathered just in time in the forward pass and again
+                      in the backward pass, each layer's gradient is reduce-scattered, and the
+                      owners update their partitions ("Como funciona": 16 psi/Nd, 3 psi of
+                      communication; "ZeRO" (lastdictionary), main definition).
 
-All three produce the same numbers ("ZeRO" (lastdictionary), "Usage note": ZeRO changes where
+All four produce the same numbers ("ZeRO" (lastdictionary), "Usage note": ZeRO changes where
 state is stored, not how updates are computed); the pins in tests/test_oracle_pins.py check it.
 
 Parity status: every function here is pinned (see tests/test_oracle_pins.py).
@@ -332,6 +337,103 @@ def zero2_step(pl: Plan, bucket_grad: Callable[[int, int], np.ndarray], master, 
         w_out[sl], m_out[sl], v_out[sl] = w, mm, vv
         p_out[sl] = p16
     return Result(False, w_out, m_out, v_out, p_out, np.concatenate(grad_shard))
+
+
+# ---------------------------------------------------------------------------------------------
+# stage 3 (Pos+g+p): the parameters are partitioned too
+#
+# "ZeRO: particionar estados do treino entre GPUs", "Como funciona": in the third stage the
+# fp16 parameters are also split among the Nd processes, a process that needs a partition it
+# does not own receives it from the owner, and a step moves 3 psi: a parameter all-gather in
+# the forward pass, another in the backward pass, and the gradient reduce-scatter (1.5 times the
+# 2 psi of plain DP). "ZeRO" (lastdictionary), main definition: each layer's parameters are
+# gathered just in time for its computation and discarded afterwards; stage 3 adds about 50 %
+# communication.
+#
+# Readings (the pages are silent on them): a layer is a run of consecutive tensors of the
+# forward-order list; the backward pass reduce-scatters each layer's local gradient as soon as
+# the layer is done (a bucket per layer, as stage 2 does per bucket); the owner's update writes
+# its fp16 values into its own parameter shard, and nothing gathers them after the step (the
+# next forward pass does, layer by layer).
+# ---------------------------------------------------------------------------------------------
+def layer_ranges(pl: Plan, layer_tensors: Sequence[int]) -> List[tuple]:
+    """Flat ranges [lo, hi) of the layers, in forward order: layer l is the next
+    layer_tensors[l] tensors of the plan's list."""
+    if sum(layer_tensors) != len(pl.numels) or any(c < 1 for c in layer_tensors):
+        raise ValueError("layer_tensors must split the tensor list into non-empty runs")
+    out, i = [], 0
+    for c in layer_tensors:
+        lo = pl.tensor_off[i]
+        last = i + c - 1
+        out.append((lo, pl.tensor_off[last] + pl.numels[last]))
+        i += c
+    return out
+
+
+def gather_params(param_shards, S: int, lo: int, hi: int) -> np.ndarray:
+    """The just-in-time all-gather of the flat range [lo, hi): every owner q whose shard
+    [q*S, (q+1)*S) meets the range hands over that part; the pieces, in owner order, make up
+    the layer's fp16 parameters."""
+    out = np.empty(hi - lo, np.uint16)
+    for q in range(lo // S, (hi - 1) // S + 1):
+        a, b = max(lo, q * S), min(hi, (q + 1) * S)
+        out[a - lo:b - lo] = _as_u16(param_shards[q])[a - q * S:b - q * S]
+    return out
+
+
+@dataclasses.dataclass
+class Result3:
+    skipped: bool
+    master: np.ndarray
+    m: np.ndarray
+    v: np.ndarray
+    param_shards: List[np.ndarray]       # owner q's fp16 parameter partition (S values each)
+    gathered_fwd: List[np.ndarray]       # layer l's gathered parameters in the forward pass
+    gathered_bwd: List[np.ndarray]       # ... and in the backward pass (index l, not order)
+    comm_elems: int                      # elements moved by the step's collectives
+    reduced: np.ndarray = None           # the owners' reduced gradient shards, end to end
+
+
+def zero3_step(pl: Plan, layers: Sequence[tuple], layer_grad: Callable[[int, int], np.ndarray],
+               master, m, v, param_shards, hp: AdamHP, t: int) -> Result3:
+    """Stage 3: forward gathers layer by layer, backward gathers again in reverse order and
+    reduce-scatters each layer's local gradient, then every owner updates its shard.
+
+    layers: flat ranges (layer_ranges); layer_grad(l, rank): rank's local fp16 gradient of
+    layer l (hi - lo values); param_shards: Nd arrays of S fp16 values (owner q's partition).
+    """
+    S, nd = pl.shard, pl.nd
+    shards = [_as_u16(p).copy() for p in param_shards]
+    assert len(shards) == nd and all(p.size == S for p in shards)
+    comm = 0
+    fwd, bwd = [None] * len(layers), [None] * len(layers)
+    for l, (lo, hi) in enumerate(layers):                    # forward pass
+        fwd[l] = gather_params(shards, S, lo, hi)             # used, then discarded
+        comm += hi - lo
+    grad_shard = [np.zeros(S, np.float32) for _ in range(nd)]
+    for l in reversed(range(len(layers))):                    # backward pass
+        lo, hi = layers[l]
+        bwd[l] = gather_params(shards, S, lo, hi)
+        comm += hi - lo
+        local = [_as_u16(layer_grad(l, j)) for j in range(nd)]
+        assert all(g.size == hi - lo for g in local)
+        for q in range(lo // S, (hi - 1) // S + 1):           # reduce-scatter of the layer
+            a, b = max(lo, q * S), min(hi, (q + 1) * S)
+            grad_shard[q][a - q * S:b - q * S] = reduce_mean([g[a - lo:b - lo] for g in local])
+        comm += hi - lo
+        del local                                             # released
+    w_out = np.array(master, np.float32)
+    m_out = np.array(m, np.float32)
+    v_out = np.array(v, np.float32)
+    red = np.concatenate(grad_shard)
+    if not all(all_finite(sh) for sh in grad_shard):
+        return Result3(True, w_out, m_out, v_out, shards, fwd, bwd, comm, red)
+    for q in range(nd):
+        sl = slice(q * S, (q + 1) * S)
+        w, mm, vv, p16 = adam(grad_shard[q], master[sl], m[sl], v[sl], hp, t)
+        w_out[sl], m_out[sl], v_out[sl] = w, mm, vv
+        shards[q] = p16                  # the owner's partition; no all-gather after the step
+    return Result3(False, w_out, m_out, v_out, shards, fwd, bwd, comm, red)
 
 
 def ulp_diff_f32(a, b) -> np.ndarray:

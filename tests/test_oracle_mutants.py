@@ -140,3 +140,43 @@ def test_partition_mutant_is_caught(name, old, new, monkeypatch):
         except (AssertionError, ValueError):
             failed += 1
     assert failed, f"slip '{name}' went unnoticed"
+
+
+# slips in the stage-3 partitioning (parameters partitioned and gathered per layer)
+STAGE3_MUTANTS = [
+    ("gather takes the neighbour's partition",
+     "out[a - lo:b - lo] = _as_u16(param_shards[q])[a - q * S:b - q * S]",
+     "out[a - lo:b - lo] = _as_u16(param_shards[(q + 1) % len(param_shards)])[a - q * S:b - q * S]"),
+    ("backward parameter all-gather not counted",
+     "        bwd[l] = gather_params(shards, S, lo, hi)\n        comm += hi - lo",
+     "        bwd[l] = gather_params(shards, S, lo, hi)"),
+    ("updated partition stored at the wrong owner",
+     "        shards[q] = p16                  # the owner's partition",
+     "        shards[(q + 1) % nd] = p16       # the owner's partition"),
+    ("layer gradient reduced from the wrong slice",
+     "grad_shard[q][a - q * S:b - q * S] = reduce_mean([g[a - lo:b - lo] for g in local])",
+     "grad_shard[q][a - q * S:b - q * S] = reduce_mean([g[::-1][a - lo:b - lo] for g in local])"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", STAGE3_MUTANTS, ids=[m[0] for m in STAGE3_MUTANTS])
+def test_stage3_mutant_is_caught(name, old, new, monkeypatch):
+    with open(os.path.join(ORACLE_DIR, "__init__.py")) as f:
+        src = f.read()
+    assert src.count(old) == 1, old
+    spec = importlib.util.spec_from_loader("oracle._mutant3", loader=None)
+    mod = importlib.util.module_from_spec(spec)
+    mod.__package__ = "oracle"
+    monkeypatch.setitem(sys.modules, "oracle._mutant3", mod)
+    exec(compile(src.replace(old, new), "oracle_mutant3.py", "exec"), mod.__dict__)
+    monkeypatch.setattr(pins, "oracle", mod)
+    failed = 0
+    checks = [lambda: pins.test_stage3_equals_plain_dp(3, [50, 1, 64, 13], [2, 1, 1]),
+              lambda: pins.test_stage3_gathers_are_the_layer_parameters(3),
+              lambda: pins.test_stage3_moves_three_psi(4, [300, 250, 250, 249])]
+    for c in checks:
+        try:
+            c()
+        except (AssertionError, ValueError):
+            failed += 1
+    assert failed, f"slip '{name}' went unnoticed"

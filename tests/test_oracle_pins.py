@@ -460,6 +460,99 @@ def test_zero_stages_skip_together():
         assert np.array_equal(z.master, master) and np.array_equal(z.params16, p16)
 
 
+# ---------------------------------------------------------------------------------------------
+# stage 3 (Pos+g+p): parameters partitioned too, gathered just in time per layer
+# ("Como funciona": 16 psi/Nd and 3 psi of communication; "ZeRO" (lastdictionary), main
+# definition: layers gathered just in time and discarded, about 50 % more communication)
+# ---------------------------------------------------------------------------------------------
+def _split_shards(full16, nd):
+    """The owners' fp16 partitions of a flat padded buffer (numpy's split, not the oracle's
+    gather, so that the gather is checked against an independent partitioning)."""
+    return [x.copy() for x in np.split(full16, nd)]
+
+
+@pytest.mark.parametrize("nd", [1, 2, 3, 4, 7, 8])
+@pytest.mark.parametrize("numels,layer_tensors", [([300, 250, 250, 249], [1, 2, 1]),
+                                                   ([7], [1]),
+                                                   ([50, 1, 64, 13], [2, 1, 1]),
+                                                   ([1000, 3, 999, 5], [1, 3])])
+def test_stage3_equals_plain_dp(nd, numels, layer_tensors):
+    """ZeRO changes where state lives, not the update ("ZeRO" (lastdictionary), "Usage note"):
+    two stage-3 steps give plain DP's master, m, v, reduced gradients and fp16 parameters bit
+    for bit, the parameters held as Nd partitions."""
+    rng = np.random.default_rng(nd * 7919 + sum(numels))
+    pl, grads, master, m, v, p16 = _random_model(rng, numels, nd, 0)
+    layers = oracle.layer_ranges(pl, layer_tensors)
+    shards = _split_shards(p16, nd)
+    for t in (1, 2):
+        dp = oracle.dp_step(grads, master, m, v, p16, HP, t)
+        z3 = oracle.zero3_step(pl, layers, lambda l, r: grads[r][layers[l][0]:layers[l][1]],
+                               master, m, v, shards, HP, t)
+        assert z3.skipped == dp.skipped is False
+        for a, b in ((z3.master, dp.master), (z3.m, dp.m), (z3.v, dp.v),
+                     (z3.reduced, dp.reduced)):
+            assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+        assert np.array_equal(np.concatenate(z3.param_shards), dp.params16)
+        master, m, v, p16, shards = dp.master, dp.m, dp.v, dp.params16, z3.param_shards
+
+
+@pytest.mark.parametrize("nd", [1, 3, 4, 8])
+def test_stage3_gathers_are_the_layer_parameters(nd):
+    """Every gathered layer, forward and backward, is exactly the layer's slice of the full
+    fp16 buffer the partitions were cut from -- including layers that straddle owners, a layer
+    smaller than a shard and one larger than several shards; values that encode their own flat
+    index make any misplaced element visible."""
+    numels = [5, 40, 1, 17, 3, 90, 2]
+    pl = oracle.plan(numels, nd, 0)
+    full = np.arange(1, pl.psi_p + 1, dtype=np.uint16)          # element i holds i + 1
+    full[pl.psi:] = 0
+    shards = _split_shards(full, nd)
+    for split in ([1] * 7, [2, 2, 3], [7], [3, 1, 3]):
+        layers = oracle.layer_ranges(pl, split)
+        assert layers[0][0] == 0 and layers[-1][1] == pl.psi
+        z = np.zeros(pl.psi_p, np.float32)
+        res = oracle.zero3_step(pl, layers,
+                                lambda l, r: np.zeros(layers[l][1] - layers[l][0], np.float16),
+                                z, z, z, shards, HP, 1)
+        for l, (lo, hi) in enumerate(layers):
+            want = np.arange(lo + 1, hi + 1, dtype=np.uint16)
+            assert np.array_equal(res.gathered_fwd[l], want)
+            assert np.array_equal(res.gathered_bwd[l], want)
+
+
+@pytest.mark.parametrize("nd,numels", [(4, [300, 250, 250, 249]), (3, [50, 1, 64, 13]),
+                                       (8, [1000, 3, 999, 5])])
+def test_stage3_moves_three_psi(nd, numels):
+    """The step's collectives move 3 psi elements -- the forward and backward parameter
+    all-gathers and the gradient reduce-scatter -- which is zero_state_bytes' closed form and
+    1.5 times the 2 psi of stages 0-2 ("Como funciona"; "ZeRO" (lastdictionary): stage 3 adds
+    about 50 %)."""
+    rng = np.random.default_rng(nd)
+    pl, grads, master, m, v, p16 = _random_model(rng, numels, nd, 0)
+    layers = oracle.layer_ranges(pl, [1] * len(numels))
+    res = oracle.zero3_step(pl, layers, lambda l, r: grads[r][layers[l][0]:layers[l][1]],
+                            master, m, v, _split_shards(p16, nd), HP, 1)
+    acct = oracle.state_bytes(pl.psi, nd)
+    assert res.comm_elems == 3 * pl.psi == acct["pos_g_p"]["comm_elems"]
+    assert 2 * res.comm_elems == 3 * acct["pos_g"]["comm_elems"] == 3 * acct["dp"]["comm_elems"]
+
+
+def test_stage3_skips_together():
+    """An inf in one rank's gradient of one layer skips the whole stage-3 step: state and every
+    parameter partition unchanged, like plain DP."""
+    rng = np.random.default_rng(19)
+    pl, grads, master, m, v, p16 = _random_model(rng, [40, 40, 21], 4, 0)
+    grads[1][45] = np.float16(np.inf)
+    layers = oracle.layer_ranges(pl, [1, 1, 1])
+    shards = _split_shards(p16, 4)
+    z3 = oracle.zero3_step(pl, layers, lambda l, r: grads[r][layers[l][0]:layers[l][1]],
+                           master, m, v, shards, HP, 1)
+    dp = oracle.dp_step(grads, master, m, v, p16, HP, 1)
+    assert z3.skipped and dp.skipped
+    assert np.array_equal(z3.master, master) and np.array_equal(z3.v, v)
+    assert np.array_equal(np.concatenate(z3.param_shards), p16)
+
+
 def test_ulp_metric():
     a = np.array([1.0, -0.0, np.nan, 1.0], np.float32)
     b = np.array([np.nextafter(np.float32(1), np.float32(2)), 0.0, np.nan, np.nan], np.float32)
