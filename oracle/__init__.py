@@ -352,9 +352,11 @@ def zero2_step(pl: Plan, bucket_grad: Callable[[int, int], np.ndarray], master, 
 #
 # Readings (the pages are silent on them): a layer is a run of consecutive tensors of the
 # forward-order list; the backward pass reduce-scatters each layer's local gradient as soon as
-# the layer is done (a bucket per layer, as stage 2 does per bucket); the owner's update writes
-# its fp16 values into its own parameter shard, and nothing gathers them after the step (the
-# next forward pass does, layer by layer).
+# the layer is done (a bucket per layer, as stage 2 does per bucket); the zero padding at the
+# end of the flat list rides with the first gradient bucket of the backward pass, the last
+# layer's, as it does in stage 2's bucket map; the owner's update writes its fp16 values into
+# its own parameter shard, and nothing gathers them after the step (the next forward pass does,
+# layer by layer). Communication counts the model's elements (the padding is not model state).
 # ---------------------------------------------------------------------------------------------
 def layer_ranges(pl: Plan, layer_tensors: Sequence[int]) -> List[tuple]:
     """Flat ranges [lo, hi) of the layers, in forward order: layer l is the next
@@ -367,6 +369,15 @@ def layer_ranges(pl: Plan, layer_tensors: Sequence[int]) -> List[tuple]:
         last = i + c - 1
         out.append((lo, pl.tensor_off[last] + pl.numels[last]))
         i += c
+    return out
+
+
+def grad_buckets(pl: Plan, layers: Sequence[tuple]) -> List[tuple]:
+    """The gradient bucket of each layer: its range, the last layer's extended over the zero
+    padding to psi_p (the backward pass produces the end of the flat list first)."""
+    out = list(layers)
+    lo, _ = out[-1]
+    out[-1] = (lo, pl.psi_p)
     return out
 
 
@@ -400,7 +411,8 @@ def zero3_step(pl: Plan, layers: Sequence[tuple], layer_grad: Callable[[int, int
     reduce-scatters each layer's local gradient, then every owner updates its shard.
 
     layers: flat ranges (layer_ranges); layer_grad(l, rank): rank's local fp16 gradient of
-    layer l (hi - lo values); param_shards: Nd arrays of S fp16 values (owner q's partition).
+    layer l's gradient bucket (grad_buckets: the layer's range, the last one extended over the
+    padding); param_shards: Nd arrays of S fp16 values (owner q's partition).
     """
     S, nd = pl.shard, pl.nd
     shards = [_as_u16(p).copy() for p in param_shards]
@@ -411,14 +423,16 @@ def zero3_step(pl: Plan, layers: Sequence[tuple], layer_grad: Callable[[int, int
         fwd[l] = gather_params(shards, S, lo, hi)             # used, then discarded
         comm += hi - lo
     grad_shard = [np.zeros(S, np.float32) for _ in range(nd)]
+    buckets = grad_buckets(pl, layers)
     for l in reversed(range(len(layers))):                    # backward pass
         lo, hi = layers[l]
         bwd[l] = gather_params(shards, S, lo, hi)
         comm += hi - lo
+        _, ghi = buckets[l]
         local = [_as_u16(layer_grad(l, j)) for j in range(nd)]
-        assert all(g.size == hi - lo for g in local)
-        for q in range(lo // S, (hi - 1) // S + 1):           # reduce-scatter of the layer
-            a, b = max(lo, q * S), min(hi, (q + 1) * S)
+        assert all(g.size == ghi - lo for g in local)
+        for q in range(lo // S, (ghi - 1) // S + 1):          # reduce-scatter of the layer
+            a, b = max(lo, q * S), min(ghi, (q + 1) * S)
             grad_shard[q][a - q * S:b - q * S] = reduce_mean([g[a - lo:b - lo] for g in local])
         comm += hi - lo
         del local                                             # released

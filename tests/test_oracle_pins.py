@@ -483,10 +483,11 @@ def test_stage3_equals_plain_dp(nd, numels, layer_tensors):
     rng = np.random.default_rng(nd * 7919 + sum(numels))
     pl, grads, master, m, v, p16 = _random_model(rng, numels, nd, 0)
     layers = oracle.layer_ranges(pl, layer_tensors)
+    gb = oracle.grad_buckets(pl, layers)
     shards = _split_shards(p16, nd)
     for t in (1, 2):
         dp = oracle.dp_step(grads, master, m, v, p16, HP, t)
-        z3 = oracle.zero3_step(pl, layers, lambda l, r: grads[r][layers[l][0]:layers[l][1]],
+        z3 = oracle.zero3_step(pl, layers, lambda l, r: grads[r][gb[l][0]:gb[l][1]],
                                master, m, v, shards, HP, t)
         assert z3.skipped == dp.skipped is False
         for a, b in ((z3.master, dp.master), (z3.m, dp.m), (z3.v, dp.v),
@@ -511,8 +512,9 @@ def test_stage3_gathers_are_the_layer_parameters(nd):
         layers = oracle.layer_ranges(pl, split)
         assert layers[0][0] == 0 and layers[-1][1] == pl.psi
         z = np.zeros(pl.psi_p, np.float32)
+        gb = oracle.grad_buckets(pl, layers)
         res = oracle.zero3_step(pl, layers,
-                                lambda l, r: np.zeros(layers[l][1] - layers[l][0], np.float16),
+                                lambda l, r: np.zeros(gb[l][1] - gb[l][0], np.float16),
                                 z, z, z, shards, HP, 1)
         for l, (lo, hi) in enumerate(layers):
             want = np.arange(lo + 1, hi + 1, dtype=np.uint16)
@@ -530,11 +532,33 @@ def test_stage3_moves_three_psi(nd, numels):
     rng = np.random.default_rng(nd)
     pl, grads, master, m, v, p16 = _random_model(rng, numels, nd, 0)
     layers = oracle.layer_ranges(pl, [1] * len(numels))
-    res = oracle.zero3_step(pl, layers, lambda l, r: grads[r][layers[l][0]:layers[l][1]],
+    gb = oracle.grad_buckets(pl, layers)
+    res = oracle.zero3_step(pl, layers, lambda l, r: grads[r][gb[l][0]:gb[l][1]],
                             master, m, v, _split_shards(p16, nd), HP, 1)
     acct = oracle.state_bytes(pl.psi, nd)
     assert res.comm_elems == 3 * pl.psi == acct["pos_g_p"]["comm_elems"]
     assert 2 * res.comm_elems == 3 * acct["pos_g"]["comm_elems"] == 3 * acct["dp"]["comm_elems"]
+
+
+@pytest.mark.parametrize("nd", [3, 4, 7])
+def test_stage3_padding_is_updated_like_plain_dp(nd):
+    """The zero padding at the end of the flat list rides with the first backward bucket, so
+    it is updated exactly as plain DP updates it, even from non-zero state."""
+    rng = np.random.default_rng(100 + nd)
+    pl, grads, master, m, v, p16 = _random_model(rng, [50, 1, 64, 15], nd, 0)
+    assert pl.psi_p > pl.psi
+    master[pl.psi:] = 0.5
+    m[pl.psi:] = 1e-3
+    v[pl.psi:] = 1e-6
+    layers = oracle.layer_ranges(pl, [2, 2])
+    gb = oracle.grad_buckets(pl, layers)
+    assert gb[-1] == (layers[-1][0], pl.psi_p) and gb[:-1] == layers[:-1]
+    z3 = oracle.zero3_step(pl, layers, lambda l, r: grads[r][gb[l][0]:gb[l][1]], master, m, v,
+                           _split_shards(oracle.f2h(master), nd), HP, 1)
+    dp = oracle.dp_step(grads, master, m, v, oracle.f2h(master), HP, 1)
+    assert np.array_equal(z3.master.view(np.uint32), dp.master.view(np.uint32))
+    assert np.array_equal(np.concatenate(z3.param_shards), dp.params16)
+    assert not np.array_equal(dp.master[pl.psi:], master[pl.psi:])   # it did move
 
 
 def test_stage3_skips_together():
@@ -544,8 +568,9 @@ def test_stage3_skips_together():
     pl, grads, master, m, v, p16 = _random_model(rng, [40, 40, 21], 4, 0)
     grads[1][45] = np.float16(np.inf)
     layers = oracle.layer_ranges(pl, [1, 1, 1])
+    gb = oracle.grad_buckets(pl, layers)
     shards = _split_shards(p16, 4)
-    z3 = oracle.zero3_step(pl, layers, lambda l, r: grads[r][layers[l][0]:layers[l][1]],
+    z3 = oracle.zero3_step(pl, layers, lambda l, r: grads[r][gb[l][0]:gb[l][1]],
                            master, m, v, shards, HP, 1)
     dp = oracle.dp_step(grads, master, m, v, p16, HP, 1)
     assert z3.skipped and dp.skipped
