@@ -3,7 +3,8 @@
 the measured HBM roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gpt2_small|shard_7p5b|flat] [--nd ND] [--bucket B]
+                    [--workload zero2_1p3b|gpt2_small|shard_7p5b|flat|zero2_gpt2_small]
+                    [--stage2 fused|unfused] [--nd ND] [--bucket B] [--no-sweep]
 
 One step is one pass of the whole hot path over one batch of synthetic input: the
 reduce-scatter of the Nd simulated ranks' fp16 gradients, the unscale, the fp32 Adam update of
@@ -11,17 +12,31 @@ every owner's shard, the fp16 cast and the all-gather write-back into the full p
 (zero_step_fused over the step's range(s), then zero_step_commit), all resident in HBM.
 
 Workloads (synthetic, seeded):
+  zero2_1p3b  ZeRO stage 2 on a 1.3B GPT-shaped list (24 layers, hidden 2048, FFN 8192, vocab
+              50257; psi = 1,311,528,960), Nd = 16, buckets of 50,000,000 elements in backward
+              order (27 buckets). The bucket scheduler launches the fused step per bucket as the
+              bucket arrives and releases its staging slot after it, then one commit (--stage2
+              unfused: the reduce-scatter per bucket, then the 16 owner updates). Grads
+              N(0, 1e-3^2); master N(0, 0.02^2), m = v = 0 at the start.    (default)
+  zero2_gpt2_small  the same on the GPT-2-small list, Nd = 8, buckets of 10,000,000.
+  zero3_gpt2_small  ZeRO stage 3 on the GPT-2-small list, Nd = 8: the fp16 parameters live in
+              8 partitions; a step gathers each of the 14 layers (embedding, 12 blocks, final
+              LayerNorm) in forward order, then in backward order gathers each layer again and
+              runs its fused update into the owners' partitions, then commits.
+  zero3_1p3b  the same on the 1.3B list (26 layers), Nd = 16.
   gpt2_small  GPT-2-small parameter list (psi = 123,653,376), Nd = 8, stage 1 (full local
               gradients, one fused call per step); grads N(0, 1e-3^2) with 1% x100; master
-              N(0, 0.02^2), m = v = 0 at the start.               (default)
+              N(0, 0.02^2), m = v = 0 at the start.
   shard_7p5b  one owner's view of 7.5e9 parameters at Nd = 64: a 117,187,500-element shard,
               64 separate fp16 gradient slices, written into a 7.5e9-element fp16 buffer at
               r*S (r = 31); master U(-0.05, 0.05), m N(0, 1e-4^2), v |N(0, 1e-6^2)|.
   flat        psi = 2^29 flat buffer, one fused call per bucket of B elements in backward
               order, Nd in {2, 4, 8, 16, 64}; state as shard_7p5b.
 
-Every step reads and writes far more than the 126 MB L2 (5.2 GB for gpt2_small), so no L2 flush
-is needed between steps. With N > 1 (torchrun), every rank runs its own replica of the
+The default line also carries the bucket / Nd sweep ("sweep" in config: the flat workload at
+Nd in {2, 4, 8, 16, 64} with 128 MiB buckets, each point timed the same way; --no-sweep skips
+it). Every step reads and writes far more than the 126 MB L2 (76 GB for zero2_1p3b, 5.2 GB for
+gpt2_small), so no L2 flush is needed between steps. With N > 1 (torchrun), every rank runs its own replica of the
 simulated Nd-rank step on its own GPU (the Nd ranks are simulated on one device; no data
 crosses GPUs), and the time is the maximum over ranks.
 """
@@ -29,6 +44,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import gc
 import hashlib
 import json
 import os
@@ -53,8 +69,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["gpt2_small", "shard_7p5b", "flat", "zero2_1p3b",
-                                           "zero2_gpt2_small"],
-                    default="gpt2_small")
+                                           "zero2_gpt2_small", "zero3_gpt2_small",
+                                           "zero3_1p3b"],
+                    default="zero2_1p3b")
     ap.add_argument("--nd", type=int, default=None)
     ap.add_argument("--bucket", type=int, default=None)
     ap.add_argument("--psi", type=int, default=None, help="flat workload size (default 2^29)")
@@ -66,9 +83,13 @@ def parse():
     ap.add_argument("--payload", choices=["fp16", "q8"], default="fp16",
                     help="q8: the owner reduces int8 payloads with one fp32 scale per 128 "
                          "elements (quantized once per rank before timing)")
-    ap.add_argument("--stage2-fused", action="store_true",
+    ap.add_argument("--stage2", choices=["fused", "unfused"], default="fused",
                     help="stage-2 workloads: the bucket scheduler launches the fused step per "
-                         "bucket (zero_sched_create_fused) instead of reduce-scatter + update")
+                         "bucket (zero_sched_create_fused), or the reduce-scatter per bucket "
+                         "and then the owner updates")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="leave out the bucket / Nd sweep of the default line")
+    ap.add_argument("--sweep-steps", type=int, default=None)
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch the per-bucket calls of a step strictly one after another "
                          "(default: inside a zero_overlap_begin/end region)")
@@ -98,6 +119,14 @@ def workload_config(args) -> dict:
         total = 7_500_000_000
         cfg = {"workload": "shard_7p5b_rank31", "psi_total": total, "shard": total // nd,
                "nd": nd, "owner": 31, "calls_per_step": 1}
+    elif kind in ("zero3_gpt2_small", "zero3_1p3b"):
+        small = kind == "zero3_gpt2_small"
+        nd = args.nd or (8 if small else 16)
+        numels = synth.gpt2_small_list() if small else synth.gpt_1p3b_list()
+        layers = synth.gpt2_small_layers() if small else synth.gpt_1p3b_layers()
+        cfg = {"workload": kind, "psi": sum(numels), "nd": nd, "stage": 3,
+               "layers": len(layers), "calls_per_step": None, "tensors": len(numels)}
+        return cfg
     elif kind in ("zero2_1p3b", "zero2_gpt2_small"):
         small = kind == "zero2_gpt2_small"
         nd = args.nd or (8 if small else 16)
@@ -108,7 +137,7 @@ def workload_config(args) -> dict:
         nb = -(-psi_p // B)
         cfg = {"workload": kind, "psi": psi, "nd": nd, "stage": 2, "bucket": B, "buckets": nb,
                "calls_per_step": nb + nd}
-        if args.stage2_fused:
+        if args.stage2 == "fused":
             cfg["workload"] = kind + "_fused"
             cfg["calls_per_step"] = nb + 1
         cfg["overlap"] = not args.no_overlap
@@ -138,6 +167,8 @@ class Workload:
         self.hp = lz.AdamHP()
         kind = args.workload
         self.kind = kind
+        self.e2e = None          # a workload-specific end-to-end leg (stage 2 fused)
+        self.kernel_times = None  # per-step dominant-kernel time, when not the ev pair's
         if kind == "gpt2_small":
             nd = args.nd or 8
             numels = synth.gpt2_small_list()
@@ -172,6 +203,9 @@ class Workload:
         elif kind in ("zero2_1p3b", "zero2_gpt2_small"):
             self._init_zero2(args, dev)
             return
+        elif kind in ("zero3_gpt2_small", "zero3_1p3b"):
+            self._init_zero3(args, dev)
+            return
         else:
             nd = args.nd or 16
             psi = args.psi or (1 << 29)
@@ -192,6 +226,8 @@ class Workload:
             assert self.config["calls_per_step"] == len(self.ranges)
         self.cur = [master, m, v]
         self.nxt = [torch.empty_like(x) for x in self.cur]
+        self.state_a0 = self.cur[0].data_ptr()
+        self.prepared = [None, None]                          # per ping-pong direction
         self.bytes_per_step = (2 * self.nd + 26) * self.n     # algorithmic HBM bytes
         # the dominant kernel: its bytes and launches per step
         self.dominant = "fused_tma_kernel"
@@ -231,6 +267,11 @@ class Workload:
         self.bytes_per_step = nd * 132 * recs + 26 * n
         self.dominant = "fused_q8_tma_kernel"
         self.dominant_bytes = self.bytes_per_step
+
+    def outputs(self):
+        """The step's result a host reads back: the fp16 parameters (stage 3: every owner's
+        partition)."""
+        return self.shards if self.kind.startswith("zero3") else [self.params]
 
     def inputs(self):
         """The tensors a step consumes that a host would have to upload."""
@@ -351,6 +392,9 @@ class Workload:
             lz.zero_step_commit(self.n, *self.cur, *self.nxt, self.params, status)
             self.cur, self.nxt = self.nxt, self.cur
             return
+        if grads is None and len(self.ranges) > 1:   # per-bucket calls, marshalled once
+            self._step_prepared(t, status, ev)
+            return
         grads = grads or self.grads
         if ev is not None:
             ev[0].record()
@@ -368,12 +412,43 @@ class Workload:
         self.cur, self.nxt = self.nxt, self.cur
 
 
+def _step_prepared(self, t, status, ev=None):
+    """The per-bucket zero_step_fused calls of a step with their pointers marshalled once per
+    ping-pong direction (the host cost of a call is then the C entry point's and the launch's,
+    which matters for 1 MiB buckets)."""
+    lz, torch = self.lz, self.torch
+    d = 0 if self.cur[0].data_ptr() == self.state_a0 else 1
+    if self.prepared[d] is None:
+        self.prepared[d] = [
+            lz.PreparedStepFused(hi - lo, self.nd, [g[lo:hi] for g in self.grads],
+                                 *[x[lo:hi] for x in self.cur], *[x[lo:hi] for x in self.nxt],
+                                 self.params[lo:hi]) for lo, hi in self.ranges]
+    hp = lz.hparams_ref(self.hp)
+    st = lz.status_ptr(status)
+    stream = torch.cuda.current_stream()
+    sh = lz.stream_handle(stream)
+    if ev is not None:
+        ev[0].record()
+    if self.overlap:
+        lz.zero_overlap_begin(sh)
+    for call in self.prepared[d]:
+        call(hp, t, st, sh)
+    if self.overlap:
+        lz.zero_overlap_end(sh)
+    if ev is not None:
+        ev[1].record()
+    lz.zero_step_commit(self.n, *self.cur, *self.nxt, self.params, status)
+    self.cur, self.nxt = self.nxt, self.cur
+
+
 def _init_zero2(self, args, dev):
     """Stage 2 on the 1.3B list (Nd = 16, buckets of 50,000,000 elements), or on the GPT-2-small
     list (Nd = 8, buckets of 10,000,000; a smaller case for profiling). The backward pass's
     output (every bucket's local gradients of every rank) is already in the scheduler's staging
-    slots, one slot per bucket; a step is the reduce-scatter of the buckets in backward order
-    through the scheduler, then the owners' updates (zero_adam_shard)."""
+    slots, one slot per bucket; a step runs the buckets in backward order through the
+    scheduler: the fused step per bucket and one commit, or (--stage2 unfused) the
+    reduce-scatter per bucket and then the owners' updates (zero_adam_shard). One scheduler
+    serves every step; between steps it is rebound to the step's buffers and status word."""
     torch, lz = self.torch, self.lz
     from zero_partitioned_optimizer_plan_b200 import synth
     if args.payload != "fp16":
@@ -388,16 +463,15 @@ def _init_zero2(self, args, dev):
     self.nd, self.n, self.psi, self.S, self.nb = nd, psi_p, psi, S, nb
     self.slot_elems = lz.zero_sched_slot_elems(pl, nb)
     self.slots = torch.empty(self.slot_elems, dtype=torch.float16, device=dev)
-    stride = self.slot_elems // (nb * nd)
-    for k in range(nb):
-        lo, ln, _, _ = lz.zero_plan_bucket(pl, k)
+    self.stride = self.slot_elems // (nb * nd)
+    self.buckets = [lz.zero_plan_bucket(pl, k)[:2] for k in range(nb)]
+    for k, (lo, ln) in enumerate(self.buckets):
         for r in range(nd):
-            base = (k * nd + r) * stride
+            base = (k * nd + r) * self.stride
             synth.grad_f16(ln, 1e-3, seed=0, rank=r, step=1000 + k,
                            out=self.slots[base:base + ln])
     self.master, self.m, self.v = synth.state_small(psi_p, seed=0, device=dev)
     self.params = torch.empty(psi_p, dtype=torch.float16, device=dev)
-    self.shards = torch.empty(psi_p, dtype=torch.float32, device=dev)
     self.grads = None
     self.ranges = [(0, psi_p)]
     # the buckets' reduce-scatters (or fused steps) of a step touch disjoint ranges
@@ -405,20 +479,30 @@ def _init_zero2(self, args, dev):
     self.param_base = 0
     self.config = workload_config(args)
     assert (self.config["psi"], self.config["buckets"]) == (psi, nb)
-    if args.stage2_fused:
+    stream = torch.cuda.current_stream()
+    self.st_create = torch.zeros(1, dtype=torch.int32, device=dev)   # rebound before each step
+    if args.stage2 == "fused":
         # the scheduler launches the fused step per bucket; ping-pong state, commit at the end
         self.cur = [self.master, self.m, self.v]
         self.nxt = [torch.empty_like(x) for x in self.cur]
         self.d_consts = torch.empty(40, dtype=torch.uint8, device=dev)
         self.h_consts = [torch.empty(40, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
         self.h_done = [None, None]
+        self.sched = lz.zero_sched_create_fused(pl, self.slots, self.slot_elems, nb, *self.cur,
+                                                *self.nxt, self.params, self.d_consts,
+                                                self.st_create, stream)
         self.bytes_per_step = (2 * nd + 26) * psi_p
         self.dominant = "fused_tma_kernel"
         self.dominant_bytes = self.bytes_per_step
         self.dominant_calls = nb
         self.side = None
         self.step = self._step_zero2_fused
+        self.e2e = self._e2e_zero2_fused
         return
+    self.shards = torch.empty(psi_p, dtype=torch.float32, device=dev)
+    self.sched = lz.zero_sched_create(pl, self.slots, self.slot_elems, nb,
+                                      [self.shards[r * S:(r + 1) * S] for r in range(nd)],
+                                      self.st_create, stream)
     rs_bytes = (2 * nd + 4) * psi_p
     adam_bytes = 30 * psi_p
     self.bytes_per_step = rs_bytes + adam_bytes
@@ -432,12 +516,10 @@ def _init_zero2(self, args, dev):
 def _step_zero2(self, t, status, ev=None, grads=None):
     lz, torch = self.lz, self.torch
     if grads is not None:
-        raise ValueError("the stage-2 workload has no host-buffer variant")
-    S, nd = self.S, self.nd
+        raise ValueError("the unfused stage-2 workload has no host-buffer variant")
+    S, nd, sch = self.S, self.nd, self.sched
     stream = torch.cuda.current_stream()
-    sch = lz.zero_sched_create(self.plan, self.slots, self.slot_elems, self.nb,
-                               [self.shards[r * S:(r + 1) * S] for r in range(nd)], status,
-                               stream)
+    lz.zero_sched_rebind_status(sch, status)
     if ev is not None:
         ev[0].record()
     if self.overlap:
@@ -459,7 +541,6 @@ def _step_zero2(self, t, status, ev=None, grads=None):
     if ev is not None:
         a1.record()
         self.side["ms"].append((a0, a1))
-    lz.zero_sched_destroy(sch)
 
 
 def _step_zero2_fused(self, t, status, ev=None, grads=None):
@@ -467,11 +548,11 @@ def _step_zero2_fused(self, t, status, ev=None, grads=None):
     kernel as the bucket arrives (its slot released after it), then one commit."""
     lz, torch = self.lz, self.torch
     if grads is not None:
-        raise ValueError("the stage-2 workload has no host-buffer variant")
+        raise ValueError("use the workload's e2e() for host buffers")
     stream = torch.cuda.current_stream()
+    sch = self.sched
     self._load_consts(t)
-    sch = lz.zero_sched_create_fused(self.plan, self.slots, self.slot_elems, self.nb, *self.cur,
-                                     *self.nxt, self.params, self.d_consts, status, stream)
+    lz.zero_sched_rebind_fused(sch, *self.cur, *self.nxt, self.params, status)
     if ev is not None:
         ev[0].record()
     if self.overlap:
@@ -485,13 +566,210 @@ def _step_zero2_fused(self, t, status, ev=None, grads=None):
     if ev is not None:
         ev[1].record()
     lz.zero_step_commit(self.n, *self.cur, *self.nxt, self.params, status)
-    lz.zero_sched_destroy(sch)
     self.cur, self.nxt = self.nxt, self.cur
 
 
+def _e2e_zero2_fused(self, t0, E, barrier, max_ms):
+    """End to end through the C ABI with host buffers: every step uploads each bucket's Nd
+    gradient slices from pinned host memory into a staging slot (two slots on the device; the
+    upload of a bucket waits, on the upload stream, for the release of its slot by
+    zero_sched_begin_bucket), the scheduler launches the bucket's fused step after the upload,
+    then the commit; the fp16 parameters and the status word are downloaded and the host reads
+    the status. The next step's uploads overlap this step's tail and download."""
+    torch, lz = self.torch, self.lz
+    dev, nd, pl = self.params.device, self.nd, self.plan
+    n_slots = 2
+    slot_elems = lz.zero_sched_slot_elems(pl, n_slots)
+    d_slots = torch.empty(slot_elems, dtype=torch.float16, device=dev)
+    region = nd * self.stride
+    total = self.nb * region
+    h_grads = pinned_host(total, torch.float16)
+    h_grads.copy_(self.slots[:total])          # the same gradients as the device-resident run
+    h_params = [torch.empty(self.n, dtype=torch.float16, pin_memory=True) for _ in range(2)]
+    h_status = [torch.empty(1, dtype=torch.int32, pin_memory=True) for _ in range(2)]
+    st = torch.zeros(E, dtype=torch.int32, device=dev)
+    main = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    sch = lz.zero_sched_create_fused(pl, d_slots, slot_elems, n_slots, *self.cur, *self.nxt,
+                                     self.params, self.d_consts, st[0:1], main)
+    h2d = 0
+    comp_done, down_done = [None, None], [None, None]
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    up.wait_event(e0)
+
+    def read_result(j):
+        down_done[j % 2].synchronize()            # the caller reads step j's result
+        if int(h_status[j % 2].item()) != 0:
+            raise RuntimeError("unexpected status in the end-to-end steps")
+
+    for i in range(E):
+        b = i % 2
+        t = t0 + i
+        self._load_consts(t)
+        lz.zero_sched_rebind_fused(sch, *self.cur, *self.nxt, self.params, st[i:i + 1])
+        if down_done[1 - b] is not None:
+            main.wait_event(down_done[1 - b])   # step i-1's parameters are downloaded
+        if self.overlap:
+            lz.zero_overlap_begin(main)
+        for k, (lo, ln) in enumerate(self.buckets):
+            ptrs = lz.zero_sched_begin_bucket(sch, k, up)
+            with torch.cuda.stream(up):
+                for r in range(nd):
+                    off = (ptrs[r] - d_slots.data_ptr()) // 2
+                    src = h_grads[k * region + r * self.stride:k * region + r * self.stride + ln]
+                    d_slots[off:off + ln].copy_(src, non_blocking=True)
+                    h2d += 2 * ln if i == 0 else 0
+            lz.zero_sched_end_bucket(sch, k, up)
+        if self.overlap:
+            lz.zero_overlap_end(main)
+        lz.zero_sched_wait(sch, main)
+        lz.zero_step_commit(self.n, *self.cur, *self.nxt, self.params, st[i:i + 1], main)
+        self.cur, self.nxt = self.nxt, self.cur
+        comp = torch.cuda.Event()
+        comp.record(main)
+        comp_done[b] = comp
+        with torch.cuda.stream(down):
+            down.wait_event(comp)
+            h_params[b].copy_(self.params, non_blocking=True)
+            h_status[b].copy_(st[i:i + 1], non_blocking=True)
+            dd = torch.cuda.Event()
+            dd.record(down)
+            down_done[b] = dd
+        if i > 0:
+            read_result(i - 1)
+    main.wait_event(down_done[(E - 1) % 2])
+    e1.record(main)
+    read_result(E - 1)
+    torch.cuda.synchronize()
+    lz.zero_sched_destroy(sch)
+    ems = max_ms(e0.elapsed_time(e1))
+    out = {"ms": ems, "steps": E, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 2 * self.n + 4,
+           "overlap": "bucket uploads into two staging slots, each gated by the release of its "
+                      "slot; the next step's uploads overlap this step's tail and download"}
+    unpin_host(h_grads)
+    del h_grads, h_params, d_slots
+    return out
+
+
+def _init_zero3(self, args, dev):
+    """Stage 3 on a GPT-shaped list: every rank's full local gradient is resident (as the
+    backward pass would leave it layer by layer); the fp16 parameters are Nd partitions of S
+    values; the optimizer state is flat and ping-ponged. A step: forward gathers of every
+    layer, then per layer in backward order its gather and its fused update (zero_stage3_step_fused),
+    then zero_stage3_step_commit. Each fused and each gather call is timed with its own events."""
+    torch, lz = self.torch, self.lz
+    from zero_partitioned_optimizer_plan_b200 import synth
+    if args.payload != "fp16":
+        raise SystemExit("the stage-3 workloads take fp16 payloads")
+    self.payload = "fp16"
+    small = args.workload == "zero3_gpt2_small"
+    nd = args.nd or (8 if small else 16)
+    numels = synth.gpt2_small_list() if small else synth.gpt_1p3b_list()
+    split = synth.gpt2_small_layers() if small else synth.gpt_1p3b_layers()
+    self.plan = pl = lz.zero_plan_create(numels, nd, 3, 0)
+    psi, psi_p, S, _ = lz.zero_plan_info(pl)
+    offs = lz.zero_plan_tensor_offsets(pl)
+    self.layers, i = [], 0
+    for c in split:
+        self.layers.append((offs[i], offs[i + c - 1] + numels[i + c - 1]))
+        i += c
+    self.nd, self.n, self.psi, self.S = nd, psi_p, psi, S
+    self.grads = []
+    for r in range(nd):
+        g = torch.zeros(psi_p, dtype=torch.float16, device=dev)
+        synth.grad_f16(psi, 1e-3, seed=0, rank=r, step=1, out=g[:psi])
+        self.grads.append(g)
+    master, m, v = synth.state_small(psi_p, seed=0, device=dev)
+    self.cur = [master, m, v]
+    self.nxt = [torch.empty_like(x) for x in self.cur]
+    self.shards = []
+    for q in range(nd):
+        part = torch.empty(S, dtype=torch.float16, device=dev)
+        part.copy_(master[q * S:(q + 1) * S])
+        self.shards.append(part)
+    self.layer_buf = torch.empty(max(hi - lo for lo, hi in self.layers), dtype=torch.float16,
+                                 device=dev)
+    self.params = self.shards[0]          # (the e2e leg downloads every partition)
+    self.ranges = [(0, psi_p)]
+    self.overlap = False
+    self.param_base = 0
+    self.config = workload_config(args)
+    n_fused = sum(((psi_p if l == len(self.layers) - 1 else hi) - 1) // S - lo // S + 1
+                  for l, (lo, hi) in enumerate(self.layers))
+    self.config["calls_per_step"] = 2 * len(self.layers) + n_fused + nd
+    self.config["fused_calls_per_step"] = n_fused
+    gather_bytes = 2 * 4 * psi              # two gathers: 2 bytes read + 2 written each
+    fused_bytes = (2 * nd + 26) * psi_p
+    self.bytes_per_step = gather_bytes + fused_bytes
+    self.dominant = "fused_tma_kernel"
+    self.dominant_bytes = fused_bytes
+    self.dominant_calls = n_fused
+    self.side = {"kernel": "gather_kernel", "bytes": gather_bytes, "calls": 2 * len(self.layers),
+                 "ms": []}
+    self.fused_evs = []
+    self.step = self._step_zero3
+    self.kernel_times = self._kernel_times_zero3
+
+
+def _step_zero3(self, t, status, ev=None, grads=None):
+    lz, torch = self.lz, self.torch
+    grads = grads or self.grads
+    pl, buf, shards = self.plan, self.layer_buf, self.shards
+    timed = ev is not None
+    mk = lambda: torch.cuda.Event(enable_timing=True)   # noqa: E731
+    g_evs, f_evs = [], []
+
+    def gather(lo, hi):
+        if timed:
+            e = (mk(), mk())
+            e[0].record()
+        lz.zero_gather_params(pl, lo, hi - lo, shards, buf, status)
+        if timed:
+            e[1].record()
+            g_evs.append(e)
+
+    if timed:
+        ev[0].record()
+    for lo, hi in self.layers:                          # forward
+        gather(lo, hi)
+    last = len(self.layers) - 1
+    for l in range(last, -1, -1):                       # backward
+        lo, hi = self.layers[l]
+        gather(lo, hi)
+        if timed:
+            e = (mk(), mk())
+            e[0].record()
+        ghi = self.n if l == last else hi               # the padding rides with the last layer
+        lz.zero_stage3_step_fused(pl, lo, ghi - lo, [g[lo:ghi] for g in grads],
+                                  *[x[lo:ghi] for x in self.cur], *[x[lo:ghi] for x in self.nxt],
+                                  shards, self.hp, t, status)
+        if timed:
+            e[1].record()
+            f_evs.append(e)
+    lz.zero_stage3_step_commit(pl, *self.cur, *self.nxt, shards, status)
+    if timed:
+        ev[1].record()
+        self.side["ms"].append(g_evs)
+        self.fused_evs.append(f_evs)
+    self.cur, self.nxt = self.nxt, self.cur
+
+
+def _kernel_times_zero3(self, evs):
+    """Per step: the fused calls' summed durations (ms)."""
+    return [sum(a.elapsed_time(b) for a, b in step) for step in self.fused_evs[-len(evs):]]
+
+
+Workload._init_zero3 = _init_zero3
+Workload._step_zero3 = _step_zero3
+Workload._kernel_times_zero3 = _kernel_times_zero3
+Workload._step_prepared = _step_prepared
 Workload._init_zero2 = _init_zero2
 Workload._step_zero2 = _step_zero2
 Workload._step_zero2_fused = _step_zero2_fused
+Workload._e2e_zero2_fused = _e2e_zero2_fused
 
 
 # ---------------------------------------------------------------------------------------------
@@ -580,11 +858,14 @@ KERNEL_SOURCES = {
 
 
 def kernel_sources_sha256(kernel: str) -> str:
-    """One hash over the sources of `kernel` (the code the ncu counters describe)."""
+    """One hash over the sources of `kernel` and the build script that holds its compiler
+    flags and geometry macros (the code the ncu counters describe)."""
     h = hashlib.sha256()
     for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(CSRC, name), "rb") as f:
             h.update(name.encode() + b"\0" + f.read())
+    with open(os.path.join(os.path.dirname(CSRC), "build.py"), "rb") as f:
+        h.update(b"build.py\0" + f.read())
     return h.hexdigest()
 
 
@@ -665,6 +946,137 @@ def max_over_ranks(ms: float, ws: int, device) -> float:
 def aggregate_rate(ws: int, units_per_rank_step: int, steps: int, ms: float) -> float:
     """Whole-job throughput: every rank's units over the slowest rank's time."""
     return ws * units_per_rank_step * steps / (ms / 1e3)
+
+
+def pinned_host(n: int, dtype):
+    """A host tensor of exactly n elements, page-locked with cudaHostRegister (torch's pinned
+    allocator rounds a request up to a power of two: 42 GB would take 64 GB)."""
+    import torch
+    t = torch.empty(n, dtype=dtype)
+    err = torch.cuda.cudart().cudaHostRegister(t.data_ptr(), t.numel() * t.element_size(), 0)
+    if int(err) != 0:
+        raise RuntimeError(f"cudaHostRegister of {t.numel() * t.element_size()} bytes failed "
+                           f"({int(err)})")
+    return t
+
+
+def unpin_host(t):
+    import torch
+    torch.cuda.cudart().cudaHostUnregister(t.data_ptr())
+
+
+def e2e_resident_inputs(wl, t0, E, barrier, max_ms):
+    """End to end for the workloads whose inputs are whole device tensors: the upload of step
+    i+1 overlaps step i's compute and download (double-buffered device gradients; copies on
+    their own streams, ordered by events)."""
+    import torch
+    dev = wl.params.device
+    h_grads = [torch.empty(g.numel(), dtype=g.dtype, pin_memory=True) for g in wl.inputs()]
+    for h, g in zip(h_grads, wl.inputs()):
+        h.copy_(g)
+    outs = wl.outputs()
+    h_params = [[torch.empty(o.numel(), dtype=o.dtype, pin_memory=True) for o in outs]
+                for _ in range(2)]
+    h_status = [torch.empty(1, dtype=torch.int32, pin_memory=True) for _ in range(2)]
+    d_grads = [[torch.empty_like(g) for g in wl.inputs()] for _ in range(2)]
+    st = torch.zeros(E, dtype=torch.int32, device=dev)
+    main = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()   # noqa: E731
+    up_done, comp_done, down_done = [None, None], [None, None], [None, None]
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    up.wait_event(e0)
+
+    def read_result(j):
+        down_done[j % 2].synchronize()            # the caller reads step j's result
+        if int(h_status[j % 2].item()) != 0:
+            raise RuntimeError("unexpected status in the end-to-end steps")
+
+    for i in range(E):
+        b = i % 2
+        with torch.cuda.stream(up):
+            if comp_done[b] is not None:
+                up.wait_event(comp_done[b])     # step i-2 is done with these buffers
+            for d, h in zip(d_grads[b], h_grads):
+                d.copy_(h, non_blocking=True)
+            up_done[b] = ev()
+            up_done[b].record(up)
+        main.wait_event(up_done[b])
+        if down_done[1 - b] is not None:
+            main.wait_event(down_done[1 - b])   # step i-1's parameters are downloaded
+        wl.step(t0 + i, st[i:i + 1], grads=d_grads[b])
+        comp_done[b] = ev()
+        comp_done[b].record(main)
+        with torch.cuda.stream(down):
+            down.wait_event(comp_done[b])
+            for h, o in zip(h_params[b], outs):
+                h.copy_(o, non_blocking=True)
+            h_status[b].copy_(st[i:i + 1], non_blocking=True)
+            down_done[b] = ev()
+            down_done[b].record(down)
+        if i > 0:
+            read_result(i - 1)
+    main.wait_event(down_done[(E - 1) % 2])
+    e1.record(main)
+    read_result(E - 1)
+    torch.cuda.synchronize()
+    return {"ms": max_ms(e0.elapsed_time(e1)), "steps": E,
+            "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h in h_grads),
+            "d2h_bytes_per_step": sum(o.numel() * o.element_size() for o in outs) + 4,
+            "overlap": "upload of step i+1 overlaps compute and download of step i"}
+
+
+SWEEP_ND = (2, 4, 8, 16, 64)
+SWEEP_PSI = 1 << 29
+SWEEP_BUCKET = 1 << 26      # 128 MiB of fp16 per rank
+
+
+def run_sweep(args, dev, ws, barrier):
+    """The bucket / Nd sweep on the flat workload (psi = 2^29, 128 MiB buckets, one fused call
+    per bucket in backward order inside an overlap region, then the commit), each point timed
+    like the main line (CUDA events on the stream, max over ranks); the point's buffers are
+    freed before the next."""
+    import copy
+
+    import torch
+    peak, _ = measured_peak()
+    K = args.sweep_steps or max(5, min(args.steps, 20))
+    W = 3
+    out = []
+    for nd in SWEEP_ND:
+        a = copy.copy(args)
+        a.workload, a.nd, a.psi, a.bucket, a.payload = "flat", nd, SWEEP_PSI, SWEEP_BUCKET, "fp16"
+        wl = Workload(a, dev)
+        status = torch.zeros(K + W, dtype=torch.int32, device=dev)
+        for i in range(W):
+            wl.step(i + 1, status[i:i + 1])
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        barrier()
+        start.record()
+        for i in range(K):
+            wl.step(W + i + 1, status[W + i:W + i + 1], ev=evs[i])
+        end.record()
+        torch.cuda.synchronize()
+        if int((status != 0).sum().item()):
+            raise RuntimeError(f"unexpected status flags in the sweep at Nd={nd}")
+        ms = max_over_ranks(start.elapsed_time(end), ws, dev) / K
+        kms = max_over_ranks(statistics.mean(x.elapsed_time(y) for x, y in evs), ws, dev)
+        gbs = wl.bytes_per_step / (kms / 1e3) / 1e9
+        out.append({"nd": nd, "psi": SWEEP_PSI, "bucket": SWEEP_BUCKET,
+                    "calls_per_step": len(wl.ranges), "steps": K, "ms_per_step": ms,
+                    "params_per_s": aggregate_rate(ws, wl.n, 1, ms),
+                    "kernel_gbs": gbs, "frac": gbs / peak,
+                    "bytes_per_step": wl.bytes_per_step})
+        del wl, status
+        gc.collect()
+        torch.cuda.empty_cache()
+    return out
 
 
 # ---------------------------------------------------------------------------------------------
@@ -767,7 +1179,7 @@ def run_ours(args):
             raise RuntimeError(f"unexpected status flags in the timed steps: {wl.g_flags.item()}")
     barrier()
     ms = start.elapsed_time(end)
-    kernel_ms = [a.elapsed_time(b) for a, b in evs]
+    kernel_ms = wl.kernel_times(evs) if wl.kernel_times else [a.elapsed_time(b) for a, b in evs]
     flags = status.cpu()
     if int((flags != 0).sum()):
         raise RuntimeError(f"unexpected status flags in the timed steps: {set(flags.tolist())}")
@@ -787,7 +1199,10 @@ def run_ours(args):
                 "kernel": wl.dominant, "bytes_per_launch": bytes_per_launch,
                 "kernel_ms_mean": launch_s * 1e3}
     if wl.side is not None:   # the other kernel of the step (or the senders' quantization)
-        side_s = statistics.mean(a.elapsed_time(b) for a, b in wl.side["ms"][-K:]) / 1e3
+        def dur(x):    # one (start, end) pair per step, or a list of pairs (one per call)
+            return x[0].elapsed_time(x[1]) if isinstance(x, tuple) else \
+                sum(a.elapsed_time(b) for a, b in x)
+        side_s = statistics.mean(dur(x) for x in wl.side["ms"][-K:]) / 1e3
         roofline["other"] = {"kernel": wl.side["kernel"],
                              "achieved": wl.side["bytes"] / side_s / 1e9,
                              "frac": wl.side["bytes"] / side_s / 1e9 / peak,
@@ -795,66 +1210,17 @@ def run_ours(args):
 
     # end to end through the public API with host buffers: every step uploads its gradients
     # from pinned host memory, runs, and downloads the updated fp16 parameters and its status
-    # word, which the host reads. The upload of step i+1 overlaps step i's compute and download
-    # (double-buffered device gradients; copies on their own streams, ordered by events).
+    # word, which the host reads.
     e2e = None
-    if not args.no_e2e and wl.inputs() is not None and not args.graph:
+    if not args.no_e2e and not args.graph and (wl.e2e is not None or wl.inputs() is not None):
         E = args.e2e_steps or max(3, min(K, 10))
-        h_grads = [torch.empty(g.numel(), dtype=g.dtype, pin_memory=True) for g in wl.inputs()]
-        for h, g in zip(h_grads, wl.inputs()):
-            h.copy_(g)
-        h_params = [torch.empty(wl.params.numel(), dtype=torch.float16, pin_memory=True)
-                    for _ in range(2)]
-        h_status = [torch.empty(1, dtype=torch.int32, pin_memory=True) for _ in range(2)]
-        d_grads = [[torch.empty_like(g) for g in wl.inputs()] for _ in range(2)]
-        st = torch.zeros(E, dtype=torch.int32, device=dev)
-        main = torch.cuda.current_stream()
-        up, down = torch.cuda.Stream(), torch.cuda.Stream()
-        ev = lambda: torch.cuda.Event()   # noqa: E731
-        up_done, comp_done, down_done = [None, None], [None, None], [None, None]
-        torch.cuda.synchronize()
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(main)
-        up.wait_event(e0)
-
-        def read_result(j):
-            down_done[j % 2].synchronize()            # the caller reads step j's result
-            if int(h_status[j % 2].item()) != 0:
-                raise RuntimeError("unexpected status in the end-to-end steps")
-
-        for i in range(E):
-            b = i % 2
-            with torch.cuda.stream(up):
-                if comp_done[b] is not None:
-                    up.wait_event(comp_done[b])     # step i-2 is done with these buffers
-                for d, h in zip(d_grads[b], h_grads):
-                    d.copy_(h, non_blocking=True)
-                up_done[b] = ev()
-                up_done[b].record(up)
-            main.wait_event(up_done[b])
-            if down_done[1 - b] is not None:
-                main.wait_event(down_done[1 - b])   # step i-1's parameters are downloaded
-            wl.step(W + K + i + 1, st[i:i + 1], grads=d_grads[b])
-            comp_done[b] = ev()
-            comp_done[b].record(main)
-            with torch.cuda.stream(down):
-                down.wait_event(comp_done[b])
-                h_params[b].copy_(wl.params, non_blocking=True)
-                h_status[b].copy_(st[i:i + 1], non_blocking=True)
-                down_done[b] = ev()
-                down_done[b].record(down)
-            if i > 0:
-                read_result(i - 1)
-        main.wait_event(down_done[(E - 1) % 2])
-        e1.record(main)
-        read_result(E - 1)
-        torch.cuda.synchronize()
-        ems = max_over_ranks(e0.elapsed_time(e1), ws, dev)
-        e2e = {"value": aggregate_rate(ws, wl.n, E, ems), "unit": "params/s",
-               "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h in h_grads),
-               "d2h_bytes_per_step": 2 * wl.n + 4,
-               "steps": E, "overlap": "upload of step i+1 overlaps compute and download of step i"}
+        mx = lambda ms: max_over_ranks(ms, ws, dev)   # noqa: E731
+        if wl.e2e is not None:
+            r = wl.e2e(W + K + 1, E, barrier, mx)
+        else:
+            r = e2e_resident_inputs(wl, W + K + 1, E, barrier, mx)
+        e2e = {"value": aggregate_rate(ws, wl.n, r["steps"], r["ms"]), "unit": "params/s",
+               **{k: v for k, v in r.items() if k != "ms"}}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -862,18 +1228,33 @@ def run_ours(args):
         rate, reps, secs = cpu_oracle_rate(wl.nd, n_sample, 10.0)
         cpu = {"value": rate, "unit": "params/s", "cores": 1, "kind": "oracle",
                "sample": f"{n_sample} elements with the workload's gradient distribution, "
-                         f"Nd={wl.nd}, {reps} oracle steps, {secs:.1f} s",
+                         f"Nd={wl.nd}, {reps} oracle steps, {secs:.1f} s (the oracle's step "
+                         "is the same element arithmetic for every stage and bucketing)",
                "host": host_cpu()}
 
+    main_line = wl.config["workload"].startswith("zero2_1p3b") and args.stage2 == "fused" and \
+        not args.graph
+    sweep = None
+    if main_line and not args.no_sweep:
+        cfg0, nd0, bytes0 = dict(wl.config), wl.nd, wl.bytes_per_step
+        del wl
+        gc.collect()            # a workload refers to itself through its bound step method
+        torch.cuda.empty_cache()
+        sweep = run_sweep(args, dev, ws, barrier)
+    else:
+        cfg0, nd0, bytes0 = dict(wl.config), wl.nd, wl.bytes_per_step
+
     if rank == 0:
-        cfg = dict(wl.config)
+        cfg = cfg0
         if args.graph:
             cfg["cuda_graph"] = "one replay per step; kernel time includes the commit"
             if args.dynamic_scale:
                 cfg["loss_scale"] = "dynamic, on the device (scaler kernels inside the graph)"
         cfg.update({"l2": "no flush: every step streams several GB, far above L2",
-                    "bytes_per_step": wl.bytes_per_step, "parallelism": f"replicas{ws}",
-                    "hbm_gbs": wl.bytes_per_step / (ms_per_step / 1e3) / 1e9})
+                    "bytes_per_step": bytes0, "parallelism": f"replicas{ws}",
+                    "hbm_gbs": bytes0 / (ms_per_step / 1e3) / 1e9})
+        if sweep is not None:
+            cfg["sweep"] = sweep
         line = {
             "metric": METRIC, "value": value, "unit": "params/s", "n_gpus": ws, "steps": K,
             "warmup": W, "ms_per_step": ms_per_step, "higher_is_better": True,

@@ -81,9 +81,9 @@ const char* zero_last_error(void);
  * one flat list of psi elements, padded with zeros to psi_padded = ceil(psi/nd)*nd. Owner r
  * holds shard [r*S, (r+1)*S) with S = psi_padded/nd. Bucket k (k = 0 is produced first) is
  * [max(0, psi_padded - (k+1)*B), psi_padded - k*B) with B = bucket_elems (0: one bucket of
- * everything). stage is 1 or 2 (recorded; the map is the same).
+ * everything). stage is 1, 2 or 3 (recorded; the map is the same).
  * Errors: ZERO_EINVAL for out == NULL, numels == NULL with n_tensors > 0, n_tensors < 0,
- * nd outside [1, ZERO_MAX_RANKS], stage outside {1, 2}, or psi == 0; ZERO_ENOMEM if the host
+ * nd outside [1, ZERO_MAX_RANKS], stage outside {1, 2, 3}, or psi == 0; ZERO_ENOMEM if the host
  * allocation fails. On success *out owns host memory released by zero_plan_destroy.
  * ---------------------------------------------------------------------------------------- */
 typedef struct zero_plan zero_plan;
@@ -180,7 +180,8 @@ zero_status zero_reduce_scatter_bucket(const zero_plan* plan, int k,
  * parameter shard r from reduced-gradient shard r; "왜 all-gather는 그대로 필요한가": the
  * updated shards are gathered into every GPU's full parameters.
  *
- * If ZERO_FLAG_OVERFLOW is set in *d_status when the kernel runs, nothing is written except
+ * If ZERO_FLAG_OVERFLOW (or ZERO_FLAG_TIMEOUT / ZERO_FLAG_BOUNDS: a reduce-scatter of the
+ * step failed) is set in *d_status when the kernel runs, nothing is written except
  * ZERO_FLAG_SKIPPED into *d_status. Otherwise, in place, for i in [0, n):
  *   g = grad[i] / loss_scale
  *   m = beta1*m + (1-beta1)*g ;  v = beta2*v + (1-beta2)*(g*g)
@@ -286,9 +287,12 @@ zero_status zero_scaler_update(zero_scaler_state* d_state, const zero_scaler_par
                                const uint32_t* d_status, zero_stream_t stream);
 
 /* Close a step made of zero_step_fused calls, on the same stream, over the same range(s).
- * If ZERO_FLAG_OVERFLOW is set: (master_out, m_out, v_out) = (master_in, m_in, v_in),
- * param_out = fp16(master_in), and ZERO_FLAG_SKIPPED is set -- the step did not happen.
- * Otherwise nothing is written. Either way the caller may then swap the in/out buffers.
+ * If ZERO_FLAG_OVERFLOW, ZERO_FLAG_TIMEOUT or ZERO_FLAG_BOUNDS is set (a gradient overflowed,
+ * or a kernel of the step gave up and left part of its outputs unwritten):
+ * (master_out, m_out, v_out) = (master_in, m_in, v_in), param_out = fp16(master_in), and
+ * ZERO_FLAG_SKIPPED is set -- the step did not happen, and the fp16 parameters of the range
+ * are restored too. Otherwise nothing is written. Either way the caller may then swap the
+ * in/out buffers (zero_step_status still reports ZERO_ECUDA for the error bits).
  * Errors: as zero_step_fused. */
 zero_status zero_step_commit(uint64_t n, const float* master_in, const float* m_in,
                              const float* v_in, float* master_out, float* m_out, float* v_out,
@@ -298,6 +302,57 @@ zero_status zero_step_commit(uint64_t n, const float* master_in, const float* m_
  * ZERO_STEP_SKIPPED if ZERO_FLAG_SKIPPED is set, ZERO_ECUDA if ZERO_FLAG_TIMEOUT or ZERO_FLAG_BOUNDS is
  * set or the copy fails, else ZERO_OK. This is the only call that blocks the host. */
 zero_status zero_step_status(const uint32_t* d_status, zero_stream_t stream, uint32_t* flags_out);
+
+/* ------------------------------------------------------------------------------------------
+ * Stage 3 (Pos+g+p): the fp16 parameters are partitioned too. "Como funciona": a process that
+ * needs a partition it does not own receives it from the owner; a step moves 3 psi -- a
+ * parameter all-gather in the forward pass, another in the backward pass, and the gradient
+ * reduce-scatter. "ZeRO" (lastdictionary.com), main definition: each layer's parameters are
+ * gathered just in time for its computation and discarded afterwards.
+ * Owner q's parameter partition is its own buffer of S fp16 values (flat elements
+ * [q*S, (q+1)*S) of the plan's padded list); param_shards is a host array of the nd device
+ * pointers. A step: for every layer in forward order zero_gather_params; for every layer in
+ * backward order zero_gather_params, then zero_stage3_step_fused over the layer's gradient
+ * bucket (its reduce-scatter, unscale, Adam, and the fp16 cast into the owners' partitions) --
+ * the layer's range, the last layer's extended to psi_padded so that the zero padding is
+ * updated as in stages 1 and 2 (the backward pass produces the end of the flat list first);
+ * then zero_stage3_step_commit. Optimizer state as in stages 1-2: flat fp32 arrays, owner q's part at q*S.
+ * ---------------------------------------------------------------------------------------- */
+
+/* The just-in-time all-gather of one layer: out[i] = element flat_lo + i of the parameters,
+ * taken from the partition of its owner, for i in [0, len); out stands for every rank's
+ * gathered copy. A pure copy (bit-exact). out: len fp16 values, 2-byte aligned (16-byte
+ * aligned stores after the first few elements); the partitions 2-byte aligned (each owner's
+ * segment takes 16-, 4- or 2-byte loads by its alignment). d_status: the bounds self-check
+ * bit. Errors: ZERO_EINVAL (null plan/pointers of an owner the range touches, range beyond
+ * psi_padded, out overlapping a partition or the status word), ZERO_EALIGN, ZERO_ECUDA.
+ * len == 0 launches nothing. */
+zero_status zero_gather_params(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                               const uint16_t* const* param_shards, uint16_t* out,
+                               uint32_t* d_status, zero_stream_t stream);
+
+/* The owners' update of the flat range [flat_lo, flat_lo + len) (one layer's gradient bucket,
+ * in backward order): zero_step_fused over each owner's part of the range, with that part's
+ * fp16 values written into the owner's partition (param_shards[q] + (a - q*S) for the part
+ * starting at flat element a). rank_grads: nd device pointers to the range's len fp16 local
+ * gradients; master_in ... v_out: device pointers to the range's first element of the flat
+ * fp32 arrays. Same arithmetic, overflow flag and commit protocol as zero_step_fused. Every
+ * part is checked before any is launched. Errors: as zero_step_fused, and ZERO_EINVAL for a
+ * range beyond psi_padded or overlapping partitions. */
+zero_status zero_stage3_step_fused(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                             const uint16_t* const* rank_grads, const float* master_in,
+                             const float* m_in, const float* v_in, float* master_out,
+                             float* m_out, float* v_out, uint16_t* const* param_shards,
+                             const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
+                             zero_stream_t stream);
+
+/* Close a stage-3 step: zero_step_commit on every owner's part, over the whole padded list
+ * (master_in ... v_out: the flat fp32 arrays, psi_padded values each), the fp16 values of a
+ * voided step restored into each owner's partition. Errors: as zero_step_commit. */
+zero_status zero_stage3_step_commit(const zero_plan* plan, const float* master_in, const float* m_in,
+                              const float* v_in, float* master_out, float* m_out, float* v_out,
+                              uint16_t* const* param_shards, uint32_t* d_status,
+                              zero_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
  * Compressed reduce-scatter payload. "ZeRO" (lastdictionary.com), main definition: extensions
@@ -373,9 +428,10 @@ zero_status zero_selftest_timeout(uint32_t* d_status, zero_stream_t stream);
  * scheduler's calls (zero_sched_end_bucket on its stream) may sit in a region.
  * Host-side state only (one flag per stream, thread-safe): both calls enqueue nothing and can
  * be used while a CUDA graph is captured. Close a region before its stream is destroyed (the
- * flag is keyed by the stream handle, which a later stream may reuse). The pages have no counterpart; this is a launch
- * device of this library. Errors: ZERO_EINVAL (begin on a stream whose region is open, end on
- * a stream without one).
+ * flag is keyed by the stream handle, which a later stream may reuse); at most 64 regions are
+ * open at once. The launch path reads the flags without a lock. The pages have no counterpart;
+ * this is a launch device of this library. Errors: ZERO_EINVAL (begin on a stream whose region
+ * is open, end on a stream without one), ZERO_ENOMEM (64 regions already open).
  * ---------------------------------------------------------------------------------------- */
 zero_status zero_overlap_begin(zero_stream_t stream);
 zero_status zero_overlap_end(zero_stream_t stream);
@@ -407,8 +463,9 @@ zero_status zero_sched_create(const zero_plan* plan, uint16_t* slot_mem, uint64_
  * d_consts -- so the reduced gradient never reaches memory (the fused step applied to stage 2
  * bucket by bucket, with the same release of each slot after its kernel). master_in/m_in/v_in
  * and master_out/m_out/v_out: psi_p fp32 values each (flat, padded), param_out: psi_p fp16
- * values; they stay fixed for the scheduler's life (with ping-pong state, create one per
- * step). After the last bucket the caller makes its stream wait (zero_sched_wait) and calls
+ * values; zero_sched_rebind_fused points a later step at other buffers (ping-pong state), so
+ * one scheduler serves every step. After the last bucket the caller makes its stream wait
+ * (zero_sched_wait) and calls
  * zero_step_commit over all psi_p elements, which skips the whole step if any bucket
  * overflowed. Errors: as zero_sched_create, and ZERO_EINVAL for outputs that overlap the
  * inputs, each other or the staging slots. The pages' stage 2 keeps the reduced shard in
@@ -419,8 +476,22 @@ zero_status zero_sched_create_fused(const zero_plan* plan, uint16_t* slot_mem,
                                     float* m_out, float* v_out, uint16_t* param_out,
                                     const zero_adam_consts* d_consts, uint32_t* d_status,
                                     zero_stream_t stream, zero_sched** out);
+/* Between steps: point the fused scheduler at the next step's state, parameters and status
+ * word (same layout and checks as zero_sched_create_fused), e.g. the swapped ping-pong buffers.
+ * Kernels already enqueued keep the old pointers; the CUDA events and slots are reused, so a
+ * step through a rebound scheduler creates nothing. Errors: ZERO_EINVAL (not a fused
+ * scheduler, a bucket begun and not ended, null or overlapping buffers), ZERO_EALIGN. */
+zero_status zero_sched_rebind_fused(zero_sched* s, const float* master_in, const float* m_in,
+                                    const float* v_in, float* master_out, float* m_out,
+                                    float* v_out, uint16_t* param_out, uint32_t* d_status);
+/* Between steps, either mode: later bucket kernels OR their flags into d_status (e.g. one
+ * status word per step). Errors: ZERO_EINVAL (null, a bucket begun and not ended, d_status
+ * inside a buffer the kernels write or the slots), ZERO_EALIGN. */
+zero_status zero_sched_rebind_status(zero_sched* s, uint32_t* d_status);
 /* Choose the slot for bucket k, make `producer` wait until that slot is released, and write
- * the nd device pointers (rank r's region, bucket k's len values) the producer must fill. */
+ * the nd device pointers (rank r's region, bucket k's len values) the producer must fill.
+ * ZERO_EINVAL if k is out of range or the slot holds a bucket that was begun and not yet
+ * ended (with n_slots slots, bucket k and bucket k + n_slots share one). */
 zero_status zero_sched_begin_bucket(zero_sched* s, int k, zero_stream_t producer,
                                     uint16_t** rank_ptrs);
 /* The producer has enqueued the fill of bucket k on `producer`: the bucket's kernel (the

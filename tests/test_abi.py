@@ -107,7 +107,8 @@ def test_state_bytes_matches_oracle(psi, nd, K):
 
 
 def test_plan_rejects_bad_arguments():
-    for args in [([], 4, 1, 0), ([5], 0, 1, 0), ([5], 65, 1, 0), ([5], 4, 3, 0), ([0, 0], 2, 1, 0)]:
+    for args in [([], 4, 1, 0), ([5], 0, 1, 0), ([5], 65, 1, 0), ([5], 4, 4, 0), ([5], 4, 0, 0),
+                 ([0, 0], 2, 1, 0)]:
         with pytest.raises(lz.ZeroError) as e:
             lz.zero_plan_create(*args)
         assert e.value.code == lz.ZERO_EINVAL
@@ -371,3 +372,57 @@ def test_state_bytes_rejects_overflowing_sizes():
     with pytest.raises(lz.ZeroError) as e:
         lz.zero_state_bytes(lim + 1, 8, K)
     assert e.value.code == lz.ZERO_EINVAL
+
+
+# ---------------------------------------------------------------------------------------------
+# stage 3: gather and the per-owner update, argument errors on the host
+# ---------------------------------------------------------------------------------------------
+def _stage3_plan():
+    return lz.zero_plan_create([100, 28], 4, 3, 0)     # psi_p = 128, S = 32
+
+
+@pytest.mark.parametrize("lo,n,shards,out,st,code", [
+    (0, 129, None, A + 50 * MB, A + 60 * MB, lz.ZERO_EINVAL),        # beyond psi_padded
+    (127, 2, None, A + 50 * MB, A + 60 * MB, lz.ZERO_EINVAL),
+    (0, 40, [A, 0, A + 2 * MB, A + 3 * MB], A + 50 * MB, A + 60 * MB, lz.ZERO_EINVAL),
+    (0, 10, None, A + 50 * MB + 1, A + 60 * MB, lz.ZERO_EALIGN),     # out not 2-byte aligned
+    (0, 10, [A + 1, A + MB, A + 2 * MB, A + 3 * MB], A + 50 * MB, A + 60 * MB, lz.ZERO_EALIGN),
+    (0, 10, None, A + 10, A + 60 * MB, lz.ZERO_EINVAL),              # out over partition 0
+    (0, 10, None, A + 50 * MB, A + 8, lz.ZERO_EINVAL),               # status in partition 0
+    (0, 10, None, A + 50 * MB, 0, lz.ZERO_EINVAL),
+])
+def test_gather_params_rejects(lo, n, shards, out, st, code):
+    pl = _stage3_plan()
+    shards = shards or [A + q * MB for q in range(4)]
+    before = lz.zero_kernel_launches()
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_gather_params(pl, lo, n, shards, out, st, 0)
+    assert e.value.code == code
+    assert lz.zero_kernel_launches() == before
+
+
+def test_stage3_update_rejects_and_launches_nothing():
+    pl = _stage3_plan()
+    grads = [A + (10 + r) * MB for r in range(4)]
+    ins = [A + 20 * MB, A + 21 * MB, A + 22 * MB]
+    outs = [A + 23 * MB, A + 24 * MB, A + 25 * MB]
+    parts = [A + q * MB for q in range(4)]
+    st = A + 30 * MB
+    before = lz.zero_kernel_launches()
+    for kw, code in [(dict(lo=100, n=29), lz.ZERO_EINVAL),            # beyond psi_padded
+                     (dict(parts=[A, A + 16, A + 2 * MB, A + 3 * MB]), lz.ZERO_EINVAL),
+                     (dict(parts=[A, A + MB, 0, A + 3 * MB]), lz.ZERO_EINVAL),
+                     (dict(step=0), lz.ZERO_EINVAL),
+                     (dict(outs=[A + 20 * MB, A + 24 * MB, A + 25 * MB]), lz.ZERO_EINVAL)]:
+        a = dict(lo=10, n=60, parts=parts, step=1, outs=outs)
+        a.update(kw)
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_stage3_step_fused(pl, a["lo"], a["n"], grads, *ins, *a["outs"], a["parts"],
+                                      HP, a["step"], st, 0)
+        assert e.value.code == code, kw
+    with pytest.raises(lz.ZeroError) as e:       # overlapping partitions in the commit
+        lz.zero_stage3_step_commit(pl, *ins, *outs, [A, A + 32, A + 2 * MB, A + 3 * MB], st, 0)
+    assert e.value.code == lz.ZERO_EINVAL
+    lz.zero_gather_params(pl, 5, 0, parts, A + 50 * MB, st, 0)          # zero length: nothing
+    lz.zero_stage3_step_fused(pl, 5, 0, grads, *ins, *outs, parts, HP, 1, st, 0)
+    assert lz.zero_kernel_launches() == before

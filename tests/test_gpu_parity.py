@@ -103,8 +103,8 @@ def test_fused_step_large_shape_vs_oracle(nd):
                                            ([70001, 3], 7),
                                            ([300000, 250000, 250000, 248576], 100000)])
 def test_reduce_scatter_and_adam_vs_oracle(numels, bucket, nd):
-    if bucket == 7 and nd > 4:
-        pytest.skip("10^4 launches")
+    """Every owner's reduced shard bit for bit, then the owner updates; the 7-element buckets
+    give about 10^4 bucket calls, each touching one or two owners' shards."""
     pl = lz.zero_plan_create(numels, nd, 2, bucket)
     psi, psi_p, S, nb = lz.zero_plan_info(pl)
     ref_plan = oracle.plan(numels, nd, bucket)
@@ -122,9 +122,11 @@ def test_reduce_scatter_and_adam_vs_oracle(numels, bucket, nd):
     shards = torch.empty(psi_p, dtype=torch.float32, device=DEV)   # owner r: [r*S, (r+1)*S)
     shard_views = [shards[r * S:(r + 1) * S] for r in range(nd)]
     st = status_word()
+    base = [g.data_ptr() for g in g_dev]      # raw addresses: ~10^4 calls stay quick
+    shard_ptrs = [x.data_ptr() for x in shard_views]
     for k in range(nb):
         lo, ln, _, _ = lz.zero_plan_bucket(pl, k)
-        lz.zero_reduce_scatter_bucket(pl, k, [g[lo:lo + ln] for g in g_dev], shard_views, st)
+        lz.zero_reduce_scatter_bucket(pl, k, [b + 2 * lo for b in base], shard_ptrs, st)
     ref = oracle.zero2_step(ref_plan, lambda k, r: g_cpu[r].numpy()[
         ref_plan.buckets[k][0]:sum(ref_plan.buckets[k])], master.numpy(), m.numpy(), v.numpy(),
         oracle.f2h(master.numpy()), ORC_HP, 1)

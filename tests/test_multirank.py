@@ -119,9 +119,16 @@ def test_failed_rank_is_detected_on_the_host(mode):
 # fused step and commit done by the oracle (the library needs a GPU)
 # ---------------------------------------------------------------------------------------------
 class _OracleCompute:
+    def __init__(self, fail=False):
+        self.fail = fail     # report a kernel timeout (as a library kernel that gave up would)
+
     def fused(self, n, rows, state_in, state_out, params, hp, t, status):
         import numpy as np
         import oracle
+        if self.fail:
+            status |= 4
+            state_out[0].fill_(float("nan"))    # a half-written output
+            return
         red = oracle.reduce_mean([row.numpy() for row in rows])
         if not oracle.all_finite(red):
             status |= 1
@@ -136,7 +143,7 @@ class _OracleCompute:
         import numpy as np
         import torch
         import oracle
-        if int(status.item()) & 1:
+        if int(status.item()) & (1 | 4 | 8):
             for dst, src in zip(state_out, state_in):
                 dst.copy_(src)
             params.view(torch.int16).copy_(
@@ -224,6 +231,76 @@ def test_distributed_step_exchange_gloo(ws, bucket, bad_rank):
             assert np.array_equal(got.view(np.uint32),
                                   want[rank * S:(rank + 1) * S].view(np.uint32))
         assert np.array_equal(params, ref.params16)
+
+
+def _worker_dist_fail(rank, ws, port, numels, bucket, fail_rank, out):
+    import datetime
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle
+    from zero_partitioned_optimizer_plan_b200.dist import DistStepError, DistZeroStep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        psi_p, grads, master, m, v = _dist_case(numels, ws, -1)
+        S = psi_p // ws
+        st_in = [x[rank * S:(rank + 1) * S].clone() for x in (master, m, v)]
+        st_out = [torch.full_like(x, float("nan")) for x in st_in]
+        params = torch.zeros(psi_p, dtype=torch.float16)
+        status = torch.zeros(1, dtype=torch.int32)
+        step = DistZeroStep(psi_p, bucket, compute=_OracleCompute(fail=rank == fail_rank))
+        raised = None
+        try:
+            step.step(grads[rank], st_in, st_out, params, oracle.AdamHP(), 1, status)
+        except DistStepError as e:
+            raised = e.bits
+        # the ranks are still in step: one more collective completes on every rank
+        t = torch.ones(1)
+        dist.all_reduce(t)
+        out.put((rank, raised, int(status.item()), [x.numpy() for x in st_in],
+                 [x.numpy() for x in st_out], params.numpy().view("uint16"), float(t.item())))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("ws,fail_rank", [(2, 1), (3, 0)])
+def test_distributed_step_failure_on_one_rank_voids_it_everywhere(ws, fail_rank):
+    """One rank's kernels report a timeout (made on the host: the fake compute sets the bit and
+    leaves a half-written output). Every rank learns it from the combined status, restores its
+    shard through the commit, skips the parameter all-gather and raises DistStepError; the
+    ranks stay in step (a later collective completes)."""
+    import numpy as np
+    import oracle
+    numels = [1000, 37, 4099, 12345]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_dist_fail,
+                         args=(r, ws, port, numels, 3000, fail_rank, q)) for r in range(ws)]
+    for p in procs:
+        p.start()
+    try:
+        res = sorted((q.get(timeout=240) for _ in range(ws)), key=lambda x: x[0])
+    finally:
+        for p in procs:
+            p.join(60)
+            if p.exitcode is None:
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    psi_p = sum(numels) + (-sum(numels)) % ws
+    S = psi_p // ws
+    for rank, raised, status, st_in, st_out, params, t in res:
+        assert raised == 4                       # the timeout bit, seen on every rank
+        assert status == 4 | 2                   # combined bits + skipped
+        for a, b in zip(st_in, st_out):          # the commit restored the shard
+            assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+        own = params[rank * S:(rank + 1) * S]
+        assert np.array_equal(own, oracle.f2h(st_in[0]))
+        rest = np.concatenate([params[:rank * S], params[(rank + 1) * S:]])
+        assert not rest.any()                    # no all-gather ran
+        assert t == ws
 
 
 def test_dist_bucket_map_matches_the_plan():

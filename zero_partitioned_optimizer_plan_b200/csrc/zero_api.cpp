@@ -382,6 +382,123 @@ zero_status zero_step_commit(uint64_t n, const float* master_in, const float* m_
                                            param_out, d_status, (cudaStream_t)stream));
 }
 
+// ---------------------------------------------------------------------------------------------
+// stage 3: parameters partitioned, gathered per layer
+// ---------------------------------------------------------------------------------------------
+// The owners whose partitions meet [flat_lo, flat_lo + len), and that range against the plan.
+static zero_status stage3_range(const zero_plan* plan, uint64_t flat_lo, uint64_t len, int* nd,
+                                uint64_t* psi_p, uint64_t* S, uint64_t* q_lo, uint64_t* q_hi) {
+    if (!zk::plan_geometry(plan, nd, psi_p, S)) return ZERO_EINVAL;
+    if (flat_lo > *psi_p || len > *psi_p - flat_lo) return ZERO_EINVAL;
+    if (len) {
+        *q_lo = flat_lo / *S;
+        *q_hi = (flat_lo + len - 1) / *S;
+    }
+    return ZERO_OK;
+}
+
+zero_status zero_gather_params(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                               const uint16_t* const* param_shards, uint16_t* out,
+                               uint32_t* d_status, zero_stream_t stream) {
+    int nd = 0;
+    uint64_t psi_p = 0, S = 0, q_lo = 0, q_hi = 0;
+    zero_status st = stage3_range(plan, flat_lo, len, &nd, &psi_p, &S, &q_lo, &q_hi);
+    if (st != ZERO_OK) return st;
+    if (!d_status) return ZERO_EINVAL;
+    if (!zk::aligned(d_status, 4)) return ZERO_EALIGN;
+    if (len == 0) return ZERO_OK;
+    if (!param_shards || !out) return ZERO_EINVAL;
+    if (!zk::aligned(out, 2)) return ZERO_EALIGN;
+    if (zk::overlap(out, len * 2, d_status, 4)) return ZERO_EINVAL;
+    for (uint64_t q = q_lo; q <= q_hi; ++q) {
+        const uint16_t* sh = param_shards[q];
+        if (!sh) return ZERO_EINVAL;
+        if (!zk::aligned(sh, 2)) return ZERO_EALIGN;
+        if (zk::overlap(out, len * 2, sh, S * 2) || zk::overlap(d_status, 4, sh, S * 2))
+            return ZERO_EINVAL;
+    }
+    return zk::from_cuda(zk::launch_gather(flat_lo, len, S, nd, param_shards, out, d_status,
+                                           (cudaStream_t)stream));
+}
+
+zero_status zero_stage3_step_fused(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                             const uint16_t* const* rank_grads, const float* master_in,
+                             const float* m_in, const float* v_in, float* master_out,
+                             float* m_out, float* v_out, uint16_t* const* param_shards,
+                             const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
+                             zero_stream_t stream) {
+    int nd = 0;
+    uint64_t psi_p = 0, S = 0, q_lo = 0, q_hi = 0;
+    if (!zk::hparams_ok(hp) || step < 1) return ZERO_EINVAL;
+    zero_status st = stage3_range(plan, flat_lo, len, &nd, &psi_p, &S, &q_lo, &q_hi);
+    if (st != ZERO_OK) return st;
+    if (!d_status) return ZERO_EINVAL;
+    if (len == 0) return ZERO_OK;
+    if (!rank_grads || !param_shards || !master_in || !m_in || !v_in || !master_out || !m_out ||
+        !v_out)
+        return ZERO_EINVAL;
+    // every owner's part is checked before anything is launched
+    const uint16_t* part_grads[ZERO_MAX_RANKS];
+    for (int pass = 0; pass < 2; ++pass) {
+        for (uint64_t q = q_lo; q <= q_hi; ++q) {
+            const uint64_t a = flat_lo > q * S ? flat_lo : q * S;
+            const uint64_t b = (q + 1) * S < flat_lo + len ? (q + 1) * S : flat_lo + len;
+            const uint64_t off = a - flat_lo, n = b - a;
+            for (int r = 0; r < nd; ++r) part_grads[r] = rank_grads[r] ? rank_grads[r] + off : nullptr;
+            uint16_t* pout = param_shards[q] ? param_shards[q] + (a - q * S) : nullptr;
+            if (pass == 0) {
+                st = check_fused(n, nd, part_grads, master_in + off, m_in + off, v_in + off,
+                                 master_out + off, m_out + off, v_out + off, pout, d_status);
+                if (st != ZERO_OK) return st;
+                for (uint64_t o = q_lo; o < q; ++o)   // partitions are distinct buffers
+                    if (param_shards[o] &&
+                        zk::overlap(param_shards[o], S * 2, param_shards[q], S * 2))
+                        return ZERO_EINVAL;
+            } else {
+                const cudaError_t e = zk::launch_fused(
+                    n, nd, part_grads, master_in + off, m_in + off, v_in + off, master_out + off,
+                    m_out + off, v_out + off, pout, zk::make_adam(hp, step), nullptr,
+                    zk::make_mean(nd), d_status, (cudaStream_t)stream);
+                if (e != cudaSuccess) return zk::from_cuda(e);
+            }
+        }
+    }
+    return ZERO_OK;
+}
+
+zero_status zero_stage3_step_commit(const zero_plan* plan, const float* master_in, const float* m_in,
+                              const float* v_in, float* master_out, float* m_out, float* v_out,
+                              uint16_t* const* param_shards, uint32_t* d_status,
+                              zero_stream_t stream) {
+    int nd = 0;
+    uint64_t psi_p = 0, S = 0;
+    if (!zk::plan_geometry(plan, &nd, &psi_p, &S)) return ZERO_EINVAL;
+    if (!d_status || !param_shards || !master_in || !m_in || !v_in || !master_out || !m_out ||
+        !v_out)
+        return ZERO_EINVAL;
+    for (int pass = 0; pass < 2; ++pass) {
+        for (int q = 0; q < nd; ++q) {
+            const uint64_t off = (uint64_t)q * S;
+            if (pass == 0) {
+                const zero_status st = zk::check_fused_state(
+                    S, master_in + off, m_in + off, v_in + off, master_out + off, m_out + off,
+                    v_out + off, param_shards[q], d_status);
+                if (st != ZERO_OK) return st;
+                for (int o = 0; o < q; ++o)
+                    if (zk::overlap(param_shards[o], S * 2, param_shards[q], S * 2))
+                        return ZERO_EINVAL;
+            } else {
+                const cudaError_t e = zk::launch_commit(S, master_in + off, m_in + off, v_in + off,
+                                                        master_out + off, m_out + off, v_out + off,
+                                                        param_shards[q], d_status,
+                                                        (cudaStream_t)stream);
+                if (e != cudaSuccess) return zk::from_cuda(e);
+            }
+        }
+    }
+    return ZERO_OK;
+}
+
 zero_status zero_step_status(const uint32_t* d_status, zero_stream_t stream, uint32_t* flags_out) {
     if (!d_status) return ZERO_EINVAL;
     if (!zk::aligned(d_status, 4)) return ZERO_EALIGN;

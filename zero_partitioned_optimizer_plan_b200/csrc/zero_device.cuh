@@ -7,11 +7,9 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
-#include <map>
-#include <mutex>
-#include <tuple>
 
 #include "zero_internal.h"
 
@@ -382,61 +380,66 @@ __device__ __forceinline__ bool consume_stage(const Geom& g, int nd, uint64_t* f
 // ---------------------------------------------------------------------------------------------
 // host side: device attributes, launch limits, grids
 // ---------------------------------------------------------------------------------------------
-std::mutex g_mu;
+// Nothing on the launch path takes a lock: the per-device attributes live in a fixed array of
+// atomics (a racing first call on two threads computes the same value twice), and the
+// occupancy of each (device, kernel, shared memory, threads) in a small per-thread table.
+constexpr int kMaxDevices = 64;
 
 struct DevInfo {
     int sms = 0;
+    int dev = 0;
 };
 
 cudaError_t dev_info(DevInfo* out) {
-    static DevInfo cache[64];
+    static std::atomic<int> sms_of[kMaxDevices];   // 0: not known yet
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (cache[dev].sms == 0) {
-        int sms = 0;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    int sms = sms_of[dev].load(std::memory_order_relaxed);
+    if (sms == 0) {
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
-        cache[dev].sms = sms;
+        sms_of[dev].store(sms, std::memory_order_relaxed);
     }
-    *out = cache[dev];
+    out->sms = sms;
+    out->dev = dev;
     return cudaSuccess;
 }
 
-// Resident CTAs per SM of a pipeline kernel with `smem` dynamic bytes (cached per device).
-// The kernel's dynamic shared-memory limit is raised once per device to the device's opt-in
-// maximum, so that every launch size (they differ with Nd) stays allowed.
+// Resident CTAs per SM of a pipeline kernel with `smem` dynamic bytes and `threads` threads on
+// device `dev`. The first time a host thread meets a (device, kernel) pair, the kernel's
+// dynamic shared-memory limit is raised to the device's opt-in maximum (setting it again from
+// another thread is harmless), so that every launch size (they differ with Nd) stays allowed.
 template <typename K>
-cudaError_t pipe_blocks_per_sm(K kernel, int threads, size_t smem, int* out) {
-    static std::map<std::tuple<int, const void*, size_t>, int> cache;
-    static std::map<std::pair<int, const void*>, int> raised;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+cudaError_t pipe_blocks_per_sm(K kernel, int dev, int threads, size_t smem, int* out) {
+    struct Entry {
+        const void* kernel;
+        size_t smem;
+        int dev, threads, blocks;
+    };
+    constexpr int kSlots = 64;
+    thread_local Entry cache[kSlots];
+    thread_local int used = 0;
+    const void* kp = reinterpret_cast<const void*>(kernel);
+    for (int i = 0; i < used; ++i) {
+        const Entry& c = cache[i];
+        if (c.kernel == kp && c.smem == smem && c.dev == dev && c.threads == threads) {
+            *out = c.blocks;
+            return cudaSuccess;
+        }
+    }
+    int optin = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return e;
-    std::lock_guard<std::mutex> lk(g_mu);
-    auto key = std::make_tuple(dev, (const void*)kernel, smem);
-    auto it = cache.find(key);
-    if (it != cache.end()) {
-        *out = it->second;
-        return cudaSuccess;
-    }
-    auto fk = std::make_pair(dev, (const void*)kernel);
-    if (raised.find(fk) == raised.end()) {
-        int optin = 0;
-        e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-        if (e != cudaSuccess) return e;
-        raised[fk] = optin;
-    }
-    if (smem > (size_t)raised[fk]) return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    if (e != cudaSuccess) return e;
+    if (smem > (size_t)optin) return cudaErrorInvalidValue;
     int b = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, threads, smem);
     if (e != cudaSuccess) return e;
     if (b < 1) return cudaErrorInvalidConfiguration;
-    cache[key] = b;
+    if (used < kSlots) cache[used++] = Entry{kp, smem, dev, threads, b};
     *out = b;
     return cudaSuccess;
 }
@@ -464,7 +467,7 @@ cudaError_t launch_pipe(K kernel, const A& args, const PipeShape& sh, cudaStream
     if (e != cudaSuccess) return e;
     const int threads = 32 * sh.warps + 32;
     int bps = 1;
-    e = pipe_blocks_per_sm(kernel, threads, sh.smem, &bps);
+    e = pipe_blocks_per_sm(kernel, di.dev, threads, sh.smem, &bps);
     if (e != cudaSuccess) return e;
     if (sh.grid_per_sm > 0 && sh.grid_per_sm < bps) bps = sh.grid_per_sm;
     uint64_t grid = (uint64_t)di.sms * (uint64_t)bps;
@@ -502,7 +505,16 @@ struct Variant {
 };
 
 Variant pick_variant(int nd) {
-    if (nd <= 2) return {20, 2};
+    if (nd <= 2) {
+        Variant v{20, 2};
+#ifdef ZK_ND2_WARPS
+        v.warps = ZK_ND2_WARPS;
+#endif
+#ifdef ZK_ND2_STAGES
+        v.target_stages = ZK_ND2_STAGES;
+#endif
+        return v;
+    }
     if (nd <= 4) return {16, 2};
     if (nd <= 8) return {24, 3};
     if (nd <= 16) return {16, 2};

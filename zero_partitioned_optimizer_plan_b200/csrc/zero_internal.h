@@ -43,6 +43,11 @@ cudaError_t launch_adam(uint64_t n, const float* grad, float* master, float* m, 
                         uint32_t* status, cudaStream_t stream);
 
 cudaError_t launch_selftest_timeout(uint32_t* status, cudaStream_t stream);
+// Stage 3 (zero_stage3.cu): copy the flat range [flat_lo, flat_lo + len) out of the owners'
+// fp16 partitions (shards[q]: S values) into out.
+cudaError_t launch_gather(uint64_t flat_lo, uint64_t len, uint64_t shard, int nd,
+                          const uint16_t* const* shards, uint16_t* out, uint32_t* status,
+                          cudaStream_t stream);
 cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, uint8_t* payload,
                             cudaStream_t stream);
 cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,

@@ -32,9 +32,6 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
-#include <map>
-#include <mutex>
-#include <tuple>
 
 #include "zero_device.cuh"
 #include "zero_internal.h"
@@ -42,6 +39,9 @@
 namespace zk {
 
 namespace {
+
+// Status bits under which a step is not applied.
+constexpr uint32_t kStepVoid = ZERO_FLAG_OVERFLOW | ZERO_FLAG_TIMEOUT | ZERO_FLAG_BOUNDS;
 
 struct FusedArgs {
     const uint16_t* grads[kMaxRanks];
@@ -384,8 +384,9 @@ __global__ void __launch_bounds__(256) rs_plain_kernel(const __grid_constant__ R
 // ---------------------------------------------------------------------------------------------
 template <bool kDC>
 __global__ void __launch_bounds__(256) adam_kernel(const __grid_constant__ AdamArgs p) {
-    // skip the whole step if any reduce-scatter of it saw inf/NaN
-    if (*reinterpret_cast<volatile uint32_t*>(p.status) & ZERO_FLAG_OVERFLOW) {
+    // skip the whole step if any reduce-scatter of it saw inf/NaN, or if one of them failed
+    // (its reduced shard is then incomplete)
+    if (*reinterpret_cast<volatile uint32_t*>(p.status) & kStepVoid) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.status, ZERO_FLAG_SKIPPED);
         return;
     }
@@ -440,8 +441,11 @@ __global__ void __launch_bounds__(256) adam_kernel(const __grid_constant__ AdamA
 // ---------------------------------------------------------------------------------------------
 // commit / skip of a fused step
 // ---------------------------------------------------------------------------------------------
+// The step is void -- its inputs are restored over its outputs -- when a reduced gradient
+// overflowed, and also when a kernel of the step gave up on a wait or failed its bounds
+// self-check: those leave some tiles of the outputs unwritten.
 __global__ void __launch_bounds__(256) commit_kernel(const __grid_constant__ CommitArgs p) {
-    if (!(*reinterpret_cast<volatile uint32_t*>(p.status) & ZERO_FLAG_OVERFLOW)) return;
+    if (!(*reinterpret_cast<volatile uint32_t*>(p.status) & kStepVoid)) return;
     if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.status, ZERO_FLAG_SKIPPED);
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
     for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n; i += stride) {
@@ -552,6 +556,7 @@ PipeShape pipe_shape(int nd, bool with_state, uint64_t n, int sms) {
         case 16: return launch_pipe(KERNEL<kElems, 16 __VA_ARGS__>, p, sh, stream);        \
         case 20: return launch_pipe(KERNEL<kElems, 20 __VA_ARGS__>, p, sh, stream);        \
         case 24: return launch_pipe(KERNEL<kElems, 24 __VA_ARGS__>, p, sh, stream);        \
+        case 28: return launch_pipe(KERNEL<kElems, 28 __VA_ARGS__>, p, sh, stream);        \
     }                                                                                      \
     return cudaErrorInvalidConfiguration
 

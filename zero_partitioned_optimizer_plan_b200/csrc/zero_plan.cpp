@@ -59,7 +59,7 @@ zero_status zero_plan_create(const uint64_t* numels, int n_tensors, int nd, int 
     *out = nullptr;
     if (n_tensors < 0 || (n_tensors > 0 && !numels)) return ZERO_EINVAL;
     if (nd < 1 || nd > ZERO_MAX_RANKS) return ZERO_EINVAL;
-    if (stage != 1 && stage != 2) return ZERO_EINVAL;
+    if (stage < 1 || stage > 3) return ZERO_EINVAL;
     zero_plan* p = new (std::nothrow) zero_plan();
     if (!p) return ZERO_ENOMEM;
     try {

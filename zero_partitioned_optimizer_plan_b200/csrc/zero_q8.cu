@@ -254,10 +254,10 @@ __device__ void produce_q8(const FusedQ8Args& p, uint64_t* full, uint64_t* empty
     }
 }
 
-template <int W, bool kDC>
+template <int W, int E, bool kDC>
 __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
     fused_q8_tma_kernel(const __grid_constant__ FusedQ8Args p) {
-    constexpr int E = kElems;
+    static_assert(E == 4 || E == 8, "a thread's values sit in one record");
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
@@ -293,29 +293,37 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
             const uint8_t* st = data + (size_t)s * p.g.stage_bytes;
             if (active) {
                 const uint32_t nr = min(p.g.rc, (uint32_t)p.nd - c * p.g.rc);
-                // this thread's record in each rank's run; its 4 values share the scale
+                // this thread's record in each rank's run; its E values share the scale
                 const uint8_t* rec0 = st + (size_t)(e0 / kQB) * kRec;
-                // the four accumulators as two packed pairs: per rank, two packed bias
-                // removals and two packed fused multiply-adds for the four values
-                static_assert(E == 4, "the rank loop packs four values per thread");
-                uint64_t a01 = f2_pack(acc[0], acc[1]), a23 = f2_pack(acc[2], acc[3]);
+                // the E accumulators as E/2 packed pairs: per rank and four values, one
+                // 4-byte load (records are 4-byte aligned), two packed bias removals and two
+                // packed fused multiply-adds
+                constexpr int P = E / 2;
+                uint64_t ap[P];
+#pragma unroll
+                for (int k = 0; k < P; ++k) ap[k] = f2_pack(acc[2 * k], acc[2 * k + 1]);
                 const uint64_t nbias = f2_pack(-8388736.0f, -8388736.0f);   // -(2^23 + 128)
-#pragma unroll 4
+#pragma unroll(16 / E)
                 for (uint32_t r = 0; r < nr; ++r) {
                     const uint8_t* rec = rec0 + (size_t)r * p.row;
-                    const uint32_t qq = *reinterpret_cast<const uint32_t*>(rec + e0 % kQB);
                     const float sc = *reinterpret_cast<const float*>(rec + kQB);
-                    const uint32_t biased = qq ^ 0x80808080u;   // each byte q + 128
                     const uint64_t ss = f2_pack(sc, sc);
-                    const uint64_t q01 =
-                        f2_add(f2_pack(q_placed(biased, 0), q_placed(biased, 1)), nbias);
-                    const uint64_t q23 =
-                        f2_add(f2_pack(q_placed(biased, 2), q_placed(biased, 3)), nbias);
-                    a01 = f2_fma(q01, ss, a01);   // acc + q * scale, one rounding each
-                    a23 = f2_fma(q23, ss, a23);
+#pragma unroll
+                    for (int k4 = 0; k4 < E / 4; ++k4) {
+                        const uint32_t qq =
+                            *reinterpret_cast<const uint32_t*>(rec + e0 % kQB + 4 * k4);
+                        const uint32_t biased = qq ^ 0x80808080u;   // each byte q + 128
+                        const uint64_t q01 =
+                            f2_add(f2_pack(q_placed(biased, 0), q_placed(biased, 1)), nbias);
+                        const uint64_t q23 =
+                            f2_add(f2_pack(q_placed(biased, 2), q_placed(biased, 3)), nbias);
+                        // acc + q * scale, one rounding each
+                        ap[2 * k4] = f2_fma(q01, ss, ap[2 * k4]);
+                        ap[2 * k4 + 1] = f2_fma(q23, ss, ap[2 * k4 + 1]);
+                    }
                 }
-                f2_unpack(a01, acc[0], acc[1]);
-                f2_unpack(a23, acc[2], acc[3]);
+#pragma unroll
+                for (int k = 0; k < P; ++k) f2_unpack(ap[k], acc[2 * k], acc[2 * k + 1]);
                 if (c + 1 == p.g.nchunks) {
                     const uint8_t* sf = st + p.g.state_off + (size_t)e0 * 4u;
                     lds_f32<E>(sf, w);
@@ -361,13 +369,28 @@ __global__ void __launch_bounds__(256) fused_q8_plain_kernel(const __grid_consta
     flag_overflow(bad, p.status);
 }
 
-// Consumer warps and stage split per Nd for the int8 payload, measured on B200: the
-// dequantizing accumulation issues about twice the instructions per byte of the fp16 sum, so up
-// to Nd = 16 the most warps win (Nd = 2/8/16: 6.4/6.7/6.6 TB/s with 24 warps against 5.0/5.4/5.5
-// with 16); above, 16 warps with the budget split in two (Nd = 32/64: 5.7/4.8 TB/s).
-Variant pick_variant_q8(int nd) {
-    if (nd <= 16) return {24, 2};
-    return {16, 2};
+// Consumer warps, values per thread and stage split per Nd for the int8 payload, measured on
+// B200: the dequantizing accumulation issues about twice the instructions per byte of the fp16
+// sum, so up to Nd = 16 the most warps win (Nd = 2/8/16: 6.4/6.7/6.6 TB/s with 24 warps against
+// 5.0/5.4/5.5 with 16); above, 16 warps with the budget split in two (Nd = 32/64: 5.7/4.8 TB/s).
+struct VariantQ8 {
+    int warps;
+    int elems;           // values per consumer thread and tile
+    int target_stages;
+};
+
+VariantQ8 pick_variant_q8(int nd) {
+    VariantQ8 v = nd <= 16 ? VariantQ8{24, 4, 2} : VariantQ8{16, 4, 2};
+#ifdef ZK_Q8_WARPS
+    v.warps = ZK_Q8_WARPS;
+#endif
+#ifdef ZK_Q8_ELEMS
+    if (nd > ZK_Q8_ELEMS_MIN_ND) v.elems = ZK_Q8_ELEMS;
+#endif
+#ifdef ZK_Q8_TARGET_STAGES
+    v.target_stages = ZK_Q8_TARGET_STAGES;
+#endif
+    return v;
 }
 
 // Small calls (fewer than 4 tiles of the large shape per SM): as for the fp16 step, 12
@@ -376,12 +399,12 @@ Variant pick_variant_q8(int nd) {
 constexpr size_t kQ8SmallBudget = 100 * 1024;
 
 // A rank's run of T/128 records per stage.
-PipeShape q8_shape(int nd, int warps, int target_stages, size_t budget) {
+PipeShape q8_shape(int nd, int warps, int elems, int target_stages, size_t budget) {
     PipeShape sh;
     sh.warps = warps;
     sh.grid_per_sm = 0;
     Geom& g = sh.g;
-    g.tile = (uint32_t)(32 * warps * kElems);
+    g.tile = (uint32_t)(32 * warps * elems);
     const size_t row = (size_t)g.tile / kQB * kRec;
     const size_t state = (size_t)g.tile * 12u;
     const size_t per_stage = budget / (size_t)target_stages;
@@ -459,43 +482,36 @@ cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,
         count_launch();
         return cudaGetLastError();
     }
-    Variant var = pick_variant_q8(nd);
-#ifdef ZK_Q8_WARPS
-    var.warps = ZK_Q8_WARPS;
-#endif
-#ifdef ZK_Q8_TARGET_STAGES
-    var.target_stages = ZK_Q8_TARGET_STAGES;
-#endif
-    const uint64_t big_tiles = n / (32ull * (uint64_t)var.warps * kElems);
+    const VariantQ8 var = pick_variant_q8(nd);
+    const uint64_t big_tiles = n / (32ull * (uint64_t)var.warps * (uint64_t)var.elems);
     PipeShape sh;
+    int elems = var.elems;
     if (big_tiles < 4ull * (uint64_t)di.sms) {
-        sh = q8_shape(nd, nd <= 8 ? 12 : 8, 2, kQ8SmallBudget);
+        elems = kElems;
+        sh = q8_shape(nd, nd <= 8 ? 12 : 8, elems, 2, kQ8SmallBudget);
         sh.grid_per_sm = 1;
     } else {
-        sh = q8_shape(nd, var.warps, var.target_stages, kSmemBudget);
+        sh = q8_shape(nd, var.warps, elems, var.target_stages, kSmemBudget);
     }
     p.g = sh.g;
     p.row = sh.g.tile / kQB * kRec;
     p.n_tiled = n & ~(kQTileAlign - 1);
     p.num_tiles = (p.n_tiled + sh.g.tile - 1) / sh.g.tile;
     p.chained = overlap_next(stream) ? 1 : 0;
-    if (ad) {
-        switch (sh.warps) {
-            case 8: return launch_pipe(fused_q8_tma_kernel<8, true>, p, sh, stream);
-            case 12: return launch_pipe(fused_q8_tma_kernel<12, true>, p, sh, stream);
-            case 16: return launch_pipe(fused_q8_tma_kernel<16, true>, p, sh, stream);
-            case 20: return launch_pipe(fused_q8_tma_kernel<20, true>, p, sh, stream);
-            case 24: return launch_pipe(fused_q8_tma_kernel<24, true>, p, sh, stream);
-        }
-        return cudaErrorInvalidConfiguration;
-    }
-    switch (sh.warps) {
-        case 8: return launch_pipe(fused_q8_tma_kernel<8, false>, p, sh, stream);
-        case 12: return launch_pipe(fused_q8_tma_kernel<12, false>, p, sh, stream);
-        case 16: return launch_pipe(fused_q8_tma_kernel<16, false>, p, sh, stream);
-        case 20: return launch_pipe(fused_q8_tma_kernel<20, false>, p, sh, stream);
-        case 24: return launch_pipe(fused_q8_tma_kernel<24, false>, p, sh, stream);
-    }
+    // the instantiated shapes: (warps, values per thread) with 32 * warps * values a multiple
+    // of 512, so that a tile is a whole number of 4-record runs
+#define ZK_Q8_CASE(WW, EE)                                                                  \
+    if (sh.warps == WW && elems == EE)                                                     \
+        return ad ? launch_pipe(fused_q8_tma_kernel<WW, EE, true>, p, sh, stream)          \
+                  : launch_pipe(fused_q8_tma_kernel<WW, EE, false>, p, sh, stream)
+    ZK_Q8_CASE(8, 4);
+    ZK_Q8_CASE(12, 4);
+    ZK_Q8_CASE(16, 4);
+    ZK_Q8_CASE(24, 4);
+    ZK_Q8_CASE(8, 8);
+    ZK_Q8_CASE(12, 8);
+    ZK_Q8_CASE(16, 8);
+#undef ZK_Q8_CASE
     return cudaErrorInvalidConfiguration;
 }
 

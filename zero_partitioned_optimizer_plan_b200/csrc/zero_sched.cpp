@@ -200,11 +200,70 @@ zero_status zero_sched_create_fused(const zero_plan* plan, uint16_t* slot_mem,
     return ZERO_OK;
 }
 
+zero_status zero_sched_rebind_fused(zero_sched* s, const float* master_in, const float* m_in,
+                                    const float* v_in, float* master_out, float* m_out,
+                                    float* v_out, uint16_t* param_out, uint32_t* d_status) {
+    if (!s || !s->fused) return ZERO_EINVAL;
+    for (int b : s->bucket_of_slot)
+        if (b != -1) return ZERO_EINVAL;   // a bucket is between begin and end
+    int nd = 0;
+    uint64_t psi_p = 0, S = 0;
+    zk::plan_geometry(s->plan, &nd, &psi_p, &S);
+    zero_status st = zk::check_fused_state(psi_p, master_in, m_in, v_in, master_out, m_out, v_out,
+                                           param_out, d_status);
+    if (st != ZERO_OK) return st;
+    uint64_t need = 0;
+    zero_sched_slot_elems(s->plan, s->n_slots, &need);
+    const void* outs[4] = {master_out, m_out, v_out, param_out};
+    const uint64_t olen[4] = {psi_p * 4, psi_p * 4, psi_p * 4, psi_p * 2};
+    for (int i = 0; i < 4; ++i)
+        if (overlaps(outs[i], olen[i], s->slot_mem, need * 2)) return ZERO_EINVAL;
+    if (overlaps(d_status, 4, s->slot_mem, need * 2)) return ZERO_EINVAL;
+    s->w_in = master_in;
+    s->m_in = m_in;
+    s->v_in = v_in;
+    s->w_out = master_out;
+    s->m_out = m_out;
+    s->v_out = v_out;
+    s->param_out = param_out;
+    s->status = d_status;
+    return ZERO_OK;
+}
+
+zero_status zero_sched_rebind_status(zero_sched* s, uint32_t* d_status) {
+    if (!s || !d_status) return ZERO_EINVAL;
+    if (reinterpret_cast<uintptr_t>(d_status) & 3u) return ZERO_EALIGN;
+    for (int b : s->bucket_of_slot)
+        if (b != -1) return ZERO_EINVAL;
+    uint64_t need = 0;
+    zero_sched_slot_elems(s->plan, s->n_slots, &need);
+    if (overlaps(d_status, 4, s->slot_mem, need * 2)) return ZERO_EINVAL;
+    if (!s->fused) {
+        int nd = 0;
+        uint64_t psi_p = 0, S = 0;
+        zk::plan_geometry(s->plan, &nd, &psi_p, &S);
+        for (int r = 0; r < nd; ++r)
+            if (overlaps(d_status, 4, s->shards[r], S * 4)) return ZERO_EINVAL;
+    } else {
+        int nd = 0;
+        uint64_t psi_p = 0, S = 0;
+        zk::plan_geometry(s->plan, &nd, &psi_p, &S);
+        const void* arr[7] = {s->w_in, s->m_in, s->v_in, s->w_out, s->m_out, s->v_out,
+                              s->param_out};
+        for (int i = 0; i < 7; ++i)
+            if (overlaps(d_status, 4, arr[i], psi_p * (i == 6 ? 2 : 4))) return ZERO_EINVAL;
+    }
+    s->status = d_status;
+    return ZERO_OK;
+}
+
 zero_status zero_sched_begin_bucket(zero_sched* s, int k, zero_stream_t producer,
                                     uint16_t** rank_ptrs) {
     uint64_t lo = 0, len = 0;
     if (!s || !rank_ptrs || !zk::plan_bucket_range(s->plan, k, &lo, &len)) return ZERO_EINVAL;
     const int slot = k % s->n_slots;
+    // the slot still holds a bucket that was begun and not ended: its fill would be lost
+    if (s->bucket_of_slot[(size_t)slot] != -1) return ZERO_EINVAL;
     if (s->filled[(size_t)slot]) {
         // the slot still holds an earlier bucket until its reduce-scatter has finished
         if (cudaError_t e = cudaStreamWaitEvent((cudaStream_t)producer, s->released[(size_t)slot], 0); e != cudaSuccess)

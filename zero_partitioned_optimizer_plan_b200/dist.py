@@ -16,10 +16,21 @@ padded list) and its own shard [r*S, (r+1)*S) of the fp32 master, m and v. A ste
      cast into its own range of the full parameter buffer) -- the reduction runs in the
      library kernel, not in the collective, so the sum order (rank 0 first) and hence every
      bit match the single-device step;
-  3. one skip decision for the whole job: the overflow bit of every rank's status word is
-     combined with an all-reduce (max), then each owner commits its shard (restoring it and
-     its fp16 parameters if any rank overflowed);
+  3. one verdict for the whole job: the overflow, timeout and bounds bits of every rank's
+     status word are combined across ranks (an all-reduce), then each owner commits its shard,
+     which restores it and its fp16 parameters if any rank overflowed or failed; a failure
+     (timeout or bounds bit anywhere) raises DistStepError on every rank before the gather;
   4. an all-gather of the fp16 shards into every rank's full parameter buffer.
+
+Pipelining. The exchange of bucket k+1 is issued (asynchronously) before the owner step of
+bucket k, so the transfer of the next bucket runs while the current one is reduced and updated,
+as the pages' bucket-by-bucket reduce-scatter intends. The received rows live in two buffers
+allocated once per DistZeroStep (bucket k uses buffer k % 2). With NCCL, a collective issued
+from the current stream starts only after the work already enqueued there, so the exchange of
+bucket k+1 (buffer (k+1) % 2) cannot overwrite rows that the owner step of bucket k-1 still
+reads, and waiting on bucket k's exchange makes the current stream, not the host, wait. The
+all-gather runs in place on NCCL (each rank's shard already sits at its offset of the output);
+other backends gather from a shard copy held in a buffer allocated once.
 
 The collectives are torch.distributed calls (NCCL on GPUs, gloo on CPUs); the arithmetic is the
 library's. ``compute`` replaces the two library calls (the tests run the exchange on CPU
@@ -30,6 +41,21 @@ from __future__ import annotations
 from typing import List, Sequence, Tuple
 
 ZERO_FLAG_OVERFLOW = 0x1
+ZERO_FLAG_TIMEOUT = 0x4
+ZERO_FLAG_BOUNDS = 0x8
+# the status bits combined across ranks: any of them voids the step on every rank
+VOID_BITS = (ZERO_FLAG_OVERFLOW, ZERO_FLAG_TIMEOUT, ZERO_FLAG_BOUNDS)
+ERROR_BITS = ZERO_FLAG_TIMEOUT | ZERO_FLAG_BOUNDS
+
+
+class DistStepError(RuntimeError):
+    """A rank's kernels reported a failure (timeout or bounds bit); the step was voided on
+    every rank (state and parameters restored) and the parameter all-gather was not run."""
+
+    def __init__(self, bits: int):
+        self.bits = bits
+        super().__init__(f"distributed ZeRO step failed on some rank: status bits {bits:#x} "
+                         "(state restored, parameters not gathered)")
 
 
 def bucket_ranges(psi_p: int, bucket: int) -> List[Tuple[int, int]]:
@@ -78,36 +104,82 @@ class DistZeroStep:
         self.psi_p = psi_p
         self.shard = psi_p // self.nd
         self.buckets = bucket_ranges(psi_p, bucket)
+        self.parts = [owner_parts(lo, hi, self.shard, self.nd) for lo, hi in self.buckets]
         self.compute = compute or LibzeroCompute()
+        self.in_place_gather = dist.get_backend(group) == "nccl"
+        self._recv = None      # two receive buffers, nd * (largest owner part) values each
+        self._bits = None      # the three void bits, combined across ranks
+        self._masks = None
+        self._gather_src = None
+
+    def _buffers(self, local_grad, params_full, status):
+        import torch
+        if self._recv is None or self._recv[0].device != local_grad.device or \
+                self._recv[0].dtype != local_grad.dtype:
+            most = max(p[self.rank] for p in self.parts)
+            self._recv = [torch.empty(self.nd * most, dtype=local_grad.dtype,
+                                      device=local_grad.device) for _ in range(2)]
+        if self._bits is None or self._bits.device != status.device:
+            self._masks = torch.tensor(VOID_BITS, dtype=status.dtype, device=status.device)
+            self._bits = torch.empty_like(self._masks)
+        if not self.in_place_gather and (
+                self._gather_src is None or self._gather_src.device != params_full.device):
+            self._gather_src = torch.empty(self.shard, dtype=params_full.dtype,
+                                           device=params_full.device)
+        return self._recv
 
     def step(self, local_grad, state_in: Sequence, state_out: Sequence, params_full, hp,
              t: int, status):
-        """local_grad: this rank's fp16 gradient (psi_p); state_in / state_out: this rank's
-        fp32 master, m, v shards (S each, distinct buffers); params_full: the fp16 parameter
-        buffer (psi_p), whose own range is updated and the rest gathered; status: this rank's
-        zeroed int32 status word, which ends with the job-wide overflow bit and, if set, the
-        skipped bit (every rank agrees). Returns the job-wide overflow flag (a one-element
-        tensor on the status word's device; reading it waits for the step)."""
-        import torch
+        """local_grad: this rank's fp16 gradient (psi_p, contiguous); state_in / state_out:
+        this rank's fp32 master, m, v shards (S each, distinct buffers); params_full: the fp16
+        parameter buffer (psi_p), whose own range is updated and the rest gathered; status:
+        this rank's zeroed int32 status word, which ends with the job-wide void bits and, if
+        any is set, the skipped bit (every rank agrees). Returns the job-wide void bits (a
+        one-element tensor on the status word's device; 1 = overflow). Raises DistStepError on
+        every rank if any rank's kernels failed."""
         dist, nd, r, S = self.dist, self.nd, self.rank, self.shard
+        recv = self._buffers(local_grad, params_full, status)
         own = params_full[r * S:(r + 1) * S]
-        for lo, hi in self.buckets:
-            parts = owner_parts(lo, hi, S, nd)
+        nb = len(self.buckets)
+        works = [None] * nb
+
+        def exchange(k):
+            lo, hi = self.buckets[k]
+            parts = self.parts[k]
             mine = parts[r]
-            recv = torch.empty(nd * mine, dtype=local_grad.dtype, device=local_grad.device)
-            dist.all_to_all_single(recv, local_grad[lo:hi].contiguous(),
-                                   output_split_sizes=[mine] * nd, input_split_sizes=parts,
-                                   group=self.group)
+            works[k] = dist.all_to_all_single(recv[k % 2][:nd * mine], local_grad[lo:hi],
+                                              output_split_sizes=[mine] * nd,
+                                              input_split_sizes=parts, group=self.group,
+                                              async_op=True)
+
+        exchange(0)
+        for k, (lo, hi) in enumerate(self.buckets):
+            if k + 1 < nb:
+                exchange(k + 1)     # in flight while bucket k is reduced and updated
+            works[k].wait()
+            works[k] = None
+            mine = self.parts[k][r]
             if mine == 0:
                 continue
             a = max(lo, r * S) - r * S            # the bucket's part of my shard
-            rows = [recv[j * mine:(j + 1) * mine] for j in range(nd)]
+            buf = recv[k % 2]
+            rows = [buf[j * mine:(j + 1) * mine] for j in range(nd)]
             self.compute.fused(mine, rows, [x[a:a + mine] for x in state_in],
                                [x[a:a + mine] for x in state_out], own[a:a + mine], hp, t,
                                status)
-        flag = torch.bitwise_and(status, ZERO_FLAG_OVERFLOW)
-        dist.all_reduce(flag, op=dist.ReduceOp.MAX, group=self.group)
+        # one verdict for the job: OR of every rank's void bits (MAX per bit)
+        import torch
+        torch.bitwise_and(status.expand(len(VOID_BITS)), self._masks, out=self._bits)
+        dist.all_reduce(self._bits, op=dist.ReduceOp.MAX, group=self.group)
+        flag = self._bits.sum(dim=0, keepdim=True)
         status.bitwise_or_(flag)
         self.compute.commit(S, state_in, state_out, own, status)
-        dist.all_gather_into_tensor(params_full, own.clone(), group=self.group)
+        bits = int(flag.item())
+        if bits & ERROR_BITS:
+            raise DistStepError(bits)
+        if self.in_place_gather:
+            dist.all_gather_into_tensor(params_full, own, group=self.group)
+        else:
+            self._gather_src.copy_(own)
+            dist.all_gather_into_tensor(params_full, self._gather_src, group=self.group)
         return flag

@@ -49,8 +49,9 @@ SYMBOLS = (
     "zero_selftest_timeout", "zero_adam_consts_table", "zero_scaler_prepare",
     "zero_scaler_update", "zero_quantize_q8", "zero_step_fused_q8", "zero_step_fused_q8_dc",
     "zero_overlap_begin", "zero_overlap_end",
+    "zero_gather_params", "zero_stage3_step_fused", "zero_stage3_step_commit",
     "zero_sched_slot_elems", "zero_sched_create", "zero_sched_create_fused",
-    "zero_sched_begin_bucket",
+    "zero_sched_begin_bucket", "zero_sched_rebind_fused", "zero_sched_rebind_status",
     "zero_sched_end_bucket", "zero_sched_wait", "zero_sched_launches", "zero_sched_destroy",
 )
 
@@ -145,12 +146,18 @@ def _load():
     L.zero_adam_consts_table.argtypes = [P(_HP), i64, i64, P(AdamConsts)]
     L.zero_scaler_prepare.argtypes = [vp, vp, i64, vp, vp, vp]
     L.zero_scaler_update.argtypes = [vp, P(ScalerParams), vp, vp]
+    L.zero_gather_params.argtypes = [vp, u64, u64, P(vp), vp, vp, vp]
+    L.zero_stage3_step_fused.argtypes = [vp, u64, u64, P(vp), vp, vp, vp, vp, vp, vp, P(vp), P(_HP),
+                                   i64, vp, vp]
+    L.zero_stage3_step_commit.argtypes = [vp, vp, vp, vp, vp, vp, vp, P(vp), vp, vp]
     L.zero_overlap_begin.argtypes = [vp]
     L.zero_overlap_end.argtypes = [vp]
     L.zero_sched_slot_elems.argtypes = [vp, i32, P(u64)]
     L.zero_sched_create.argtypes = [vp, vp, u64, i32, P(vp), vp, vp, P(vp)]
     L.zero_sched_create_fused.argtypes = [vp, vp, u64, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                           vp, P(vp)]
+    L.zero_sched_rebind_fused.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.zero_sched_rebind_status.argtypes = [vp, vp]
     L.zero_sched_begin_bucket.argtypes = [vp, i32, vp, P(vp)]
     L.zero_sched_end_bucket.argtypes = [vp, i32, vp]
     L.zero_sched_wait.argtypes = [vp, vp]
@@ -301,6 +308,37 @@ def zero_step_fused(n: int, nd: int, rank_grads, master_in, m_in, v_in, master_o
                                 step, _ptr(d_status, 4), _stream(stream)), "zero_step_fused")
 
 
+class PreparedStepFused:
+    """zero_step_fused with its pointer arguments marshalled once, for a call repeated every
+    step (e.g. one per bucket): calling it passes the stored addresses, the step's
+    hyperparameters, t, the status word and the stream straight to the C entry point."""
+
+    def __init__(self, n: int, nd: int, rank_grads, master_in, m_in, v_in, master_out, m_out,
+                 v_out, param_out):
+        self._args = (n, nd, _ptr_array(rank_grads, 2), _ptr(master_in, 4), _ptr(m_in, 4),
+                      _ptr(v_in, 4), _ptr(master_out, 4), _ptr(m_out, 4), _ptr(v_out, 4),
+                      _ptr(param_out, 2))
+
+    def __call__(self, hp_ref, step: int, d_status: int, stream: int):
+        """hp_ref: hparams_ref(hp); d_status, stream: raw addresses (status_ptr, stream_handle)."""
+        code = _lib.zero_step_fused(*self._args, hp_ref, step, d_status, stream)
+        if code:
+            raise ZeroError(code, "zero_step_fused")
+
+
+def hparams_ref(hp: AdamHP):
+    """The C struct of hp, by reference, for prepared calls (build once per step)."""
+    return C.byref(hp._c())
+
+
+def status_ptr(d_status) -> int:
+    return _ptr(d_status, 4)
+
+
+def stream_handle(stream=None) -> int:
+    return _stream(stream)
+
+
 def zero_adam_consts_for_step(hp: AdamHP, step: int) -> AdamConsts:
     out = AdamConsts()
     h = hp._c()
@@ -385,6 +423,32 @@ def zero_selftest_timeout(d_status, stream=None):
     _check(_lib.zero_selftest_timeout(_ptr(d_status, 4), _stream(stream)), "zero_selftest_timeout")
 
 
+def zero_gather_params(plan: Plan, flat_lo: int, length: int, param_shards, out, d_status,
+                       stream=None):
+    _check(_lib.zero_gather_params(plan.handle, flat_lo, length, _ptr_array(param_shards, 2),
+                                   _ptr(out, 2), _ptr(d_status, 4), _stream(stream)),
+           "zero_gather_params")
+
+
+def zero_stage3_step_fused(plan: Plan, flat_lo: int, length: int, rank_grads, master_in, m_in, v_in,
+                     master_out, m_out, v_out, param_shards, hp: AdamHP, step: int, d_status,
+                     stream=None):
+    h = hp._c()
+    _check(_lib.zero_stage3_step_fused(plan.handle, flat_lo, length, _ptr_array(rank_grads, 2),
+                                 _ptr(master_in, 4), _ptr(m_in, 4), _ptr(v_in, 4),
+                                 _ptr(master_out, 4), _ptr(m_out, 4), _ptr(v_out, 4),
+                                 _ptr_array(param_shards, 2), C.byref(h), step,
+                                 _ptr(d_status, 4), _stream(stream)), "zero_stage3_step_fused")
+
+
+def zero_stage3_step_commit(plan: Plan, master_in, m_in, v_in, master_out, m_out, v_out, param_shards,
+                      d_status, stream=None):
+    _check(_lib.zero_stage3_step_commit(plan.handle, _ptr(master_in, 4), _ptr(m_in, 4), _ptr(v_in, 4),
+                                  _ptr(master_out, 4), _ptr(m_out, 4), _ptr(v_out, 4),
+                                  _ptr_array(param_shards, 2), _ptr(d_status, 4),
+                                  _stream(stream)), "zero_stage3_step_commit")
+
+
 def zero_overlap_begin(stream=None):
     _check(_lib.zero_overlap_begin(_stream(stream)), "zero_overlap_begin")
 
@@ -449,6 +513,18 @@ def zero_sched_create_fused(plan: Plan, slot_mem, slot_mem_elems: int, n_slots: 
                                         _stream(stream), C.byref(h)), "zero_sched_create_fused")
     _, psi_p, shard, _ = zero_plan_info(plan)
     return Sched(h.value, psi_p // shard if shard else 1)
+
+
+def zero_sched_rebind_fused(s: Sched, master_in, m_in, v_in, master_out, m_out, v_out,
+                            param_out, d_status):
+    _check(_lib.zero_sched_rebind_fused(s.handle, _ptr(master_in, 4), _ptr(m_in, 4),
+                                        _ptr(v_in, 4), _ptr(master_out, 4), _ptr(m_out, 4),
+                                        _ptr(v_out, 4), _ptr(param_out, 2), _ptr(d_status, 4)),
+           "zero_sched_rebind_fused")
+
+
+def zero_sched_rebind_status(s: Sched, d_status):
+    _check(_lib.zero_sched_rebind_status(s.handle, _ptr(d_status, 4)), "zero_sched_rebind_status")
 
 
 def zero_sched_begin_bucket(s: Sched, k: int, producer=None) -> List[int]:

@@ -140,12 +140,26 @@ def gpt_param_list(vocab: int, hidden: int, layers: int, ffn: int):
     return shapes
 
 
+def gpt_layer_tensors(layers: int):
+    """How many consecutive tensors of gpt_param_list make up each layer, in forward order:
+    the embedding, one transformer block (12 tensors) per layer, the final LayerNorm."""
+    return [1] + [12] * layers + [2]
+
+
 def gpt2_small_list():
     return gpt_param_list(50257, 768, 12, 3072)
 
 
+def gpt2_small_layers():
+    return gpt_layer_tensors(12)
+
+
 def gpt_1p3b_list():
     return gpt_param_list(50257, 2048, 24, 8192)
+
+
+def gpt_1p3b_layers():
+    return gpt_layer_tensors(24)
 
 
 TINY_LIST = [300000, 250000, 250000, 248576]
