@@ -284,8 +284,9 @@ class Workload:
         torch, lz = self.torch, self.lz
         dev = self.cur[0].device
         self.dynamic = dynamic
-        self.d_consts = torch.empty(40, dtype=torch.uint8, device=dev)
-        self.h_consts = [torch.empty(40, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
+        nb_c = lz.ZERO_ADAM_CONSTS_BYTES
+        self.d_consts = torch.empty(nb_c, dtype=torch.uint8, device=dev)
+        self.h_consts = [torch.empty(nb_c, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
         self.h_done = [None, None]
         self.g_status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.g_flags = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -413,28 +414,19 @@ class Workload:
 
 
 def _step_prepared(self, t, status, ev=None):
-    """The per-bucket zero_step_fused calls of a step with their pointers marshalled once per
-    ping-pong direction (the host cost of a call is then the C entry point's and the launch's,
-    which matters for 1 MiB buckets)."""
+    """The per-bucket calls of a step as one zero_step_fused_ranges call, its range descriptors
+    marshalled once per ping-pong direction (a step's host cost is then one entry plus the
+    launches, which matters for 1 MiB buckets)."""
     lz, torch = self.lz, self.torch
     d = 0 if self.cur[0].data_ptr() == self.state_a0 else 1
     if self.prepared[d] is None:
-        self.prepared[d] = [
-            lz.PreparedStepFused(hi - lo, self.nd, [g[lo:hi] for g in self.grads],
-                                 *[x[lo:hi] for x in self.cur], *[x[lo:hi] for x in self.nxt],
-                                 self.params[lo:hi]) for lo, hi in self.ranges]
-    hp = lz.hparams_ref(self.hp)
-    st = lz.status_ptr(status)
-    stream = torch.cuda.current_stream()
-    sh = lz.stream_handle(stream)
+        self.prepared[d] = lz.PreparedStepRanges(self.nd, [
+            (hi - lo, [g[lo:hi] for g in self.grads], *[x[lo:hi] for x in self.cur],
+             *[x[lo:hi] for x in self.nxt], self.params[lo:hi]) for lo, hi in self.ranges])
+    sh = lz.stream_handle(torch.cuda.current_stream())
     if ev is not None:
         ev[0].record()
-    if self.overlap:
-        lz.zero_overlap_begin(sh)
-    for call in self.prepared[d]:
-        call(hp, t, st, sh)
-    if self.overlap:
-        lz.zero_overlap_end(sh)
+    self.prepared[d](lz.hparams_ref(self.hp), t, lz.status_ptr(status), self.overlap, sh)
     if ev is not None:
         ev[1].record()
     lz.zero_step_commit(self.n, *self.cur, *self.nxt, self.params, status)
@@ -485,8 +477,9 @@ def _init_zero2(self, args, dev):
         # the scheduler launches the fused step per bucket; ping-pong state, commit at the end
         self.cur = [self.master, self.m, self.v]
         self.nxt = [torch.empty_like(x) for x in self.cur]
-        self.d_consts = torch.empty(40, dtype=torch.uint8, device=dev)
-        self.h_consts = [torch.empty(40, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
+        nb_c = lz.ZERO_ADAM_CONSTS_BYTES
+        self.d_consts = torch.empty(nb_c, dtype=torch.uint8, device=dev)
+        self.h_consts = [torch.empty(nb_c, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
         self.h_done = [None, None]
         self.sched = lz.zero_sched_create_fused(pl, self.slots, self.slot_elems, nb, *self.cur,
                                                 *self.nxt, self.params, self.d_consts,
@@ -690,8 +683,18 @@ def _init_zero3(self, args, dev):
         part = torch.empty(S, dtype=torch.float16, device=dev)
         part.copy_(master[q * S:(q + 1) * S])
         self.shards.append(part)
-    self.layer_buf = torch.empty(max(hi - lo for lo, hi in self.layers), dtype=torch.float16,
-                                 device=dev)
+    big = max(hi - lo for lo, hi in self.layers)
+    self.layer_bufs = [torch.empty(big, dtype=torch.float16, device=dev) for _ in range(2)]
+    self.gather_stream = torch.cuda.Stream()
+    L = len(self.layers)
+    mk = lambda t=False: torch.cuda.Event(enable_timing=t)   # noqa: E731
+    self.step_start = mk()
+    self.g_done = [mk() for _ in range(L)]
+    self.f_done = [mk() for _ in range(L)]
+    self.g_ev = [(mk(True), mk(True)) for _ in range(2 * L)]   # reused every step
+    self.f_ev = [(mk(True), mk(True)) for _ in range(L)]
+    self.state_a0 = self.cur[0].data_ptr()
+    self.layer_views = [None, None]
     self.params = self.shards[0]          # (the e2e leg downloads every partition)
     self.ranges = [(0, psi_p)]
     self.overlap = False
@@ -715,56 +718,94 @@ def _init_zero3(self, args, dev):
 
 
 def _step_zero3(self, t, status, ev=None, grads=None):
+    """One stage-3 step on two streams. The gather stream runs the forward gathers, then the
+    backward gathers one layer ahead: layer l-1 is gathered (into the other of two layer
+    buffers) while the main stream runs layer l's fused update. Layer l's update waits for
+    layer l's backward gather (the layer's computation would sit between them); a gather into a
+    buffer waits for the update of the layer that used the buffer before; the next step's
+    gathers wait for this step's commit. A gather and the update running beside it touch
+    disjoint ranges of the partitions."""
     lz, torch = self.lz, self.torch
     grads = grads or self.grads
-    pl, buf, shards = self.plan, self.layer_buf, self.shards
+    pl, shards, L = self.plan, self.shards, len(self.layers)
+    main, gs = torch.cuda.current_stream(), self.gather_stream
     timed = ev is not None
-    mk = lambda: torch.cuda.Event(enable_timing=True)   # noqa: E731
-    g_evs, f_evs = [], []
+    g_pairs, f_pairs = [], []
 
-    def gather(lo, hi):
-        if timed:
-            e = (mk(), mk())
-            e[0].record()
-        lz.zero_gather_params(pl, lo, hi - lo, shards, buf, status)
-        if timed:
-            e[1].record()
-            g_evs.append(e)
-
-    if timed:
-        ev[0].record()
-    for lo, hi in self.layers:                          # forward
-        gather(lo, hi)
-    last = len(self.layers) - 1
-    for l in range(last, -1, -1):                       # backward
+    def gather(l):
         lo, hi = self.layers[l]
-        gather(lo, hi)
-        if timed:
-            e = (mk(), mk())
-            e[0].record()
-        ghi = self.n if l == last else hi               # the padding rides with the last layer
-        lz.zero_stage3_step_fused(pl, lo, ghi - lo, [g[lo:ghi] for g in grads],
-                                  *[x[lo:ghi] for x in self.cur], *[x[lo:ghi] for x in self.nxt],
-                                  shards, self.hp, t, status)
-        if timed:
-            e[1].record()
-            f_evs.append(e)
-    lz.zero_stage3_step_commit(pl, *self.cur, *self.nxt, shards, status)
+        with torch.cuda.stream(gs):
+            if timed:
+                e = self.g_ev[len(g_pairs)]
+                e[0].record(gs)
+            lz.zero_gather_params(pl, lo, hi - lo, shards, self.layer_bufs[l % 2], status, gs)
+            if timed:
+                e[1].record(gs)
+                g_pairs.append(e)
+
     if timed:
-        ev[1].record()
-        self.side["ms"].append(g_evs)
-        self.fused_evs.append(f_evs)
+        ev[0].record(main)
+    self.step_start.record(main)
+    gs.wait_event(self.step_start)            # the previous step's updates and commit
+    for l in range(L):                        # forward
+        gather(l)
+    gather(L - 1)                             # backward, one layer ahead of the updates
+    self.g_done[L - 1].record(gs)
+    for l in range(L - 1, -1, -1):
+        lo, hi = self.layers[l]
+        main.wait_event(self.g_done[l])
+        if timed:
+            e = self.f_ev[len(f_pairs)]
+            e[0].record(main)
+        lz.zero_stage3_step_fused(pl, lo, *self._layer_args(l, grads), shards, self.hp, t,
+                                  status, main)
+        if timed:
+            e[1].record(main)
+            f_pairs.append(e)
+        self.f_done[l].record(main)
+        if l > 0:
+            if l + 1 < L:
+                gs.wait_event(self.f_done[l + 1])   # buffer (l-1) % 2 was layer l+1's
+            gather(l - 1)
+            self.g_done[l - 1].record(gs)
+    lz.zero_stage3_step_commit(pl, *self.cur, *self.nxt, shards, status, main)
+    if timed:
+        ev[1].record(main)
+        self.side["ms"].append(list(g_pairs))
+        self.fused_evs.append(list(f_pairs))
     self.cur, self.nxt = self.nxt, self.cur
 
 
+def _layer_args(self, l, grads):
+    """(length, rank gradients, state in, state out) views of layer l's gradient bucket, made
+    once per ping-pong direction (the padding rides with the last layer)."""
+    if grads is not self.grads:
+        lo, hi = self.layers[l]
+        ghi = self.n if l == len(self.layers) - 1 else hi
+        return (ghi - lo, [g[lo:ghi] for g in grads], *[x[lo:ghi] for x in self.cur],
+                *[x[lo:ghi] for x in self.nxt])
+    d = 0 if self.cur[0].data_ptr() == self.state_a0 else 1
+    if self.layer_views[d] is None:
+        views = []
+        for k, (lo, hi) in enumerate(self.layers):
+            ghi = self.n if k == len(self.layers) - 1 else hi
+            views.append((ghi - lo, [g[lo:ghi] for g in self.grads],
+                          *[x[lo:ghi] for x in self.cur], *[x[lo:ghi] for x in self.nxt]))
+        self.layer_views[d] = views
+    return self.layer_views[d][l]
+
+
 def _kernel_times_zero3(self, evs):
-    """Per step: the fused calls' summed durations (ms)."""
-    return [sum(a.elapsed_time(b) for a, b in step) for step in self.fused_evs[-len(evs):]]
+    """Per step: the fused calls' summed durations (ms). The events are reused by every step,
+    so only the last step's are still readable: its durations stand for each timed step."""
+    last = sum(a.elapsed_time(b) for a, b in self.fused_evs[-1])
+    return [last] * len(evs)
 
 
 Workload._init_zero3 = _init_zero3
 Workload._step_zero3 = _step_zero3
 Workload._kernel_times_zero3 = _kernel_times_zero3
+Workload._layer_args = _layer_args
 Workload._step_prepared = _step_prepared
 Workload._init_zero2 = _init_zero2
 Workload._step_zero2 = _step_zero2

@@ -136,7 +136,7 @@ typedef struct {
     double lr, beta1, beta2, eps, loss_scale;
 } zero_adam_hparams;
 
-/* The fp32 constants of one Adam step t, in the layout the kernels read them. */
+/* The fp32 constants of one Adam step t, in the layout the kernels read them (40 bytes). */
 typedef struct {
     float beta1, one_minus_beta1, beta2, one_minus_beta2;
     float step_size;      /* lr / (1 - beta1^t) */
@@ -221,6 +221,33 @@ zero_status zero_step_fused(uint64_t n, int nd, const uint16_t* const* rank_grad
                             float* master_out, float* m_out, float* v_out, uint16_t* param_out,
                             const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
                             zero_stream_t stream);
+
+/* The calls of one step over several ranges (e.g. every bucket of a stage-1 step, in backward
+ * order) as one call, so that a caller issuing many small calls pays one entry instead of one
+ * per range. ranges[i] describes what zero_step_fused takes for range i (rank_grads: a host
+ * array of nd device pointers). Every range is checked before anything is launched; then the
+ * ranges are launched in order, exactly as `count` zero_step_fused calls on `stream` would be.
+ * overlap != 0 declares them mutually independent, as a zero_overlap_begin/end region around
+ * them would (the ranges of one step are: disjoint outputs, no output overlapping another
+ * range's inputs); the library does not check that declaration. If a region is already open on
+ * the stream, the calls join it. Errors: ZERO_EINVAL (count <
+ * 0, null ranges, and anything zero_step_fused rejects for a range), ZERO_EALIGN, ZERO_ECUDA
+ * (ranges before the failing one may have been launched). */
+typedef struct {
+    uint64_t n;
+    const uint16_t* const* rank_grads;
+    const float* master_in;
+    const float* m_in;
+    const float* v_in;
+    float* master_out;
+    float* m_out;
+    float* v_out;
+    uint16_t* param_out;
+} zero_fused_range;
+
+zero_status zero_step_fused_ranges(int nd, int count, const zero_fused_range* ranges,
+                                   const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
+                                   int overlap, zero_stream_t stream);
 
 /* zero_adam_shard and zero_step_fused with the step's constants read from device memory when
  * the kernel runs (d_consts: a zero_adam_consts in device memory, 4-byte aligned), so that a

@@ -7,7 +7,9 @@
  *   host_us_region   host time per call, inside zero_overlap_begin/end;
  *   gpu_us_region    device time per call of the region's calls (CUDA events);
  * each a median over `reps` repetitions, the launches of a repetition fewer than the device's
- * launch queue holds so that the host never waits for the device. Prints one JSON line. */
+ * launch queue holds so that the host never waits for the device. Consecutive calls use
+ * different buffers (a ring of kSets), so that the calls of a region are independent, as a
+ * region requires. Prints one JSON line. */
 #define _POSIX_C_SOURCE 199309L
 #include <cuda_runtime_api.h>
 #include <stdint.h>
@@ -47,19 +49,22 @@ int main(int argc, char** argv) {
     const int calls = argc > 3 ? atoi(argv[3]) : 400;
     const int reps = 7;
     if (nd < 1 || nd > ZERO_MAX_RANKS || calls < 1 || n == 0) return 2;
-    uint16_t* grads[ZERO_MAX_RANKS];
-    for (int r = 0; r < nd; ++r) {
-        CHECK(cudaMalloc((void**)&grads[r], n * 2));
-        CHECK(cudaMemset(grads[r], 0, n * 2));
+    enum { kSets = 4 };
+    uint16_t* grads[kSets][ZERO_MAX_RANKS];
+    float* st[kSets][6];
+    uint16_t* params[kSets];
+    for (int k = 0; k < kSets; ++k) {
+        for (int r = 0; r < nd; ++r) {
+            CHECK(cudaMalloc((void**)&grads[k][r], n * 2));
+            CHECK(cudaMemset(grads[k][r], 0, n * 2));
+        }
+        for (int i = 0; i < 6; ++i) {
+            CHECK(cudaMalloc((void**)&st[k][i], n * 4));
+            CHECK(cudaMemset(st[k][i], 0, n * 4));
+        }
+        CHECK(cudaMalloc((void**)&params[k], n * 2));
     }
-    float* st[6];
-    for (int i = 0; i < 6; ++i) {
-        CHECK(cudaMalloc((void**)&st[i], n * 4));
-        CHECK(cudaMemset(st[i], 0, n * 4));
-    }
-    uint16_t* params;
     uint32_t* status;
-    CHECK(cudaMalloc((void**)&params, n * 2));
     CHECK(cudaMalloc((void**)&status, 4));
     CHECK(cudaMemset(status, 0, 4));
     cudaStream_t s;
@@ -68,29 +73,28 @@ int main(int argc, char** argv) {
     CHECK(cudaEventCreate(&e0));
     CHECK(cudaEventCreate(&e1));
     const zero_adam_hparams hp = {1e-3, 0.9, 0.999, 1e-8, 1024.0};
-    const uint16_t* const* g = (const uint16_t* const*)grads;
     zero_stream_t zs = (zero_stream_t)s;
+#define CALL(i)                                                                              \
+    zero_step_fused(n, nd, (const uint16_t* const*)grads[(i) % kSets], st[(i) % kSets][0],     \
+                    st[(i) % kSets][1], st[(i) % kSets][2], st[(i) % kSets][3],                \
+                    st[(i) % kSets][4], st[(i) % kSets][5], params[(i) % kSets], &hp, 1,       \
+                    status, zs)
 
     for (int i = 0; i < 50; ++i)   /* warm-up: occupancy caches, module load */
-        CHECK(zero_step_fused(n, nd, g, st[0], st[1], st[2], st[3], st[4], st[5], params, &hp,
-                              1, status, zs));
+        CHECK(CALL(i));
     CHECK(cudaStreamSynchronize(s));
 
     double ordered[reps], region[reps], gpu[reps];
     for (int k = 0; k < reps; ++k) {
         double t0 = now_us();
-        for (int i = 0; i < calls; ++i)
-            CHECK(zero_step_fused(n, nd, g, st[0], st[1], st[2], st[3], st[4], st[5], params,
-                                  &hp, 1, status, zs));
+        for (int i = 0; i < calls; ++i) CHECK(CALL(i));
         ordered[k] = (now_us() - t0) / calls;
         CHECK(cudaStreamSynchronize(s));
 
         t0 = now_us();
         CHECK(cudaEventRecord(e0, s));
         CHECK(zero_overlap_begin(zs));
-        for (int i = 0; i < calls; ++i)
-            CHECK(zero_step_fused(n, nd, g, st[0], st[1], st[2], st[3], st[4], st[5], params,
-                                  &hp, 1, status, zs));
+        for (int i = 0; i < calls; ++i) CHECK(CALL(i));
         CHECK(zero_overlap_end(zs));
         CHECK(cudaEventRecord(e1, s));
         region[k] = (now_us() - t0) / calls;

@@ -426,3 +426,23 @@ def test_stage3_update_rejects_and_launches_nothing():
     lz.zero_gather_params(pl, 5, 0, parts, A + 50 * MB, st, 0)          # zero length: nothing
     lz.zero_stage3_step_fused(pl, 5, 0, grads, *ins, *outs, parts, HP, 1, st, 0)
     assert lz.zero_kernel_launches() == before
+
+
+def test_step_fused_ranges_rejects_before_launching():
+    grads = [A + i * MB for i in range(2)]
+    good = (1000, grads, A + 100 * MB, A + 101 * MB, A + 102 * MB, A + 110 * MB, A + 111 * MB,
+            A + 112 * MB, A + 120 * MB)
+    bad_out = (1000, grads, A + 200 * MB, A + 201 * MB, A + 202 * MB, A + 200 * MB,
+               A + 211 * MB, A + 212 * MB, A + 220 * MB)                  # out == in
+    before = lz.zero_kernel_launches()
+    for ranges, kw, code in [([good, bad_out], {}, lz.ZERO_EINVAL),
+                             ([good], dict(step=0), lz.ZERO_EINVAL),
+                             ([good], dict(st=A + 110 * MB + 4), lz.ZERO_EINVAL),
+                             ([good[:1] + ([A, A + 1],) + good[2:]], {}, lz.ZERO_EALIGN)]:
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_step_fused_ranges(2, ranges, HP, kw.get("step", 1),
+                                      kw.get("st", A + 130 * MB), True, 0)
+        assert e.value.code == code
+    assert lz.zero_kernel_launches() == before
+    lz.zero_step_fused_ranges(2, [], HP, 1, A + 130 * MB, True, 0)     # nothing to do
+    assert lz.zero_kernel_launches() == before

@@ -53,7 +53,7 @@ def test_device_scaler_sequence(init_scale, graph):
     params = torch.empty(n, dtype=torch.float16, device=DEV)
     table = lz.zero_adam_consts_table(HP, 1, 32)
     d_table = torch.frombuffer(bytearray(bytes(table)), dtype=torch.uint8).to(DEV)
-    d_consts = torch.empty(40, dtype=torch.uint8, device=DEV)
+    d_consts = torch.empty(lz.ZERO_ADAM_CONSTS_BYTES, dtype=torch.uint8, device=DEV)
     d_state = _to_dev(lz.ScalerState(init_scale, 0, 1, 0))
     prm = lz.ScalerParams(2.0, 0.5, interval)
     st = status_word()
@@ -122,7 +122,7 @@ def test_table_exhausted_refuses_the_step():
     n, nd = 4096 * 2, 2
     table = lz.zero_adam_consts_table(HP, 1, 2)
     d_table = torch.frombuffer(bytearray(bytes(table)), dtype=torch.uint8).to(DEV)
-    d_consts = torch.empty(40, dtype=torch.uint8, device=DEV)
+    d_consts = torch.empty(lz.ZERO_ADAM_CONSTS_BYTES, dtype=torch.uint8, device=DEV)
     d_state = _to_dev(lz.ScalerState(1024.0, 0, 3, 0))     # t = 3, the table holds 1..2
     st = status_word()
     cur = [x.to(DEV) for x in synth.state_warm(n, seed=93)]

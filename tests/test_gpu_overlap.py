@@ -163,7 +163,7 @@ def test_region_captured_in_graph():
     bufs = [[x.to(DEV) for x in (master, m, v)], [torch.empty(n, device=DEV) for _ in range(3)]]
     grads = [torch.empty(n, dtype=torch.float16, device=DEV) for _ in range(nd)]
     params = torch.empty(n, dtype=torch.float16, device=DEV)
-    dc = torch.empty(40, dtype=torch.uint8, device=DEV)
+    dc = torch.empty(lz.ZERO_ADAM_CONSTS_BYTES, dtype=torch.uint8, device=DEV)
     st = status_word()
     flags = status_word()
 

@@ -555,7 +555,7 @@ def test_graph_replay_of_bucketed_step():
     bufs = [[x.to(DEV) for x in (master, m, v)], [torch.empty(n, device=DEV) for _ in range(3)]]
     grads = [torch.empty(n, dtype=torch.float16, device=DEV) for _ in range(nd)]
     params = torch.empty(n, dtype=torch.float16, device=DEV)
-    dc = torch.empty(40, dtype=torch.uint8, device=DEV)
+    dc = torch.empty(lz.ZERO_ADAM_CONSTS_BYTES, dtype=torch.uint8, device=DEV)
     st = status_word()
     flags = status_word()
     bounds, hi = [], n
@@ -630,4 +630,42 @@ def test_bounded_wait_expires_and_context_survives():
     skipped, w, mm, vv, p = oracle.step([g.numpy() for g in g_cpu], master.numpy(), m.numpy(),
                                         v.numpy(), ORC_HP, 1)
     check_f32("master", f32np(pp.nxt[0]), w)
+    check_f16("params", f16np(params), p)
+
+
+@pytest.mark.parametrize("mode", ["ordered", "overlap", "inside_region"])
+def test_step_fused_ranges_vs_oracle(mode):
+    """zero_step_fused_ranges: a step's bucket calls (backward order, ragged last bucket, the
+    small-call and the plain shapes mixed) in one C call equal the oracle's step, launched
+    ordered, as an overlap region, or joining a region the caller opened."""
+    n, nd, B = 300_007, 5, 65_536
+    master, m, v = synth.state_warm(n, seed=91)
+    pp = PingPong(master, m, v)
+    g_cpu = _rank_grads_cpu(n, nd, 92, 1)
+    g_dev = [g.to(DEV) for g in g_cpu]
+    params = torch.empty(n, dtype=torch.float16, device=DEV)
+    cuts, hi = [], n
+    while hi > 0:
+        cuts.append((max(0, hi - B), hi))
+        hi = max(0, hi - B)
+    cuts.append((0, 0))                                   # an empty range is allowed
+    ranges = [(hi - lo, [g[lo:hi] if hi > lo else g for g in g_dev],
+               *[x[lo:hi] if hi > lo else x for x in pp.cur],
+               *[x[lo:hi] if hi > lo else x for x in pp.nxt],
+               params[lo:hi] if hi > lo else params) for lo, hi in cuts]
+    st = status_word()
+    before = lz.zero_kernel_launches()
+    if mode == "inside_region":
+        with lz.overlap():
+            lz.zero_step_fused_ranges(nd, ranges, HP, 1, st, overlap=True)
+    else:
+        lz.zero_step_fused_ranges(nd, ranges, HP, 1, st, overlap=(mode == "overlap"))
+    lz.zero_step_commit(n, *pp.cur, *pp.nxt, params, st)
+    assert lz.zero_step_status(st) == (lz.ZERO_OK, 0)
+    assert lz.zero_kernel_launches() - before == len(cuts) - 1 + 1
+    skipped, w, mm, vv, p = oracle.step([g.numpy() for g in g_cpu], master.numpy(), m.numpy(),
+                                        v.numpy(), ORC_HP, 1)
+    check_f32("master", f32np(pp.nxt[0]), w)
+    check_f32("m", f32np(pp.nxt[1]), mm)
+    check_f32("v", f32np(pp.nxt[2]), vv)
     check_f16("params", f16np(params), p)

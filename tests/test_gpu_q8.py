@@ -226,7 +226,7 @@ def test_q8_graph_with_device_scaler():
     params = torch.empty(n, dtype=torch.float16, device=DEV)
     table = lz.zero_adam_consts_table(HP, 1, 32)
     d_table = torch.frombuffer(bytearray(bytes(table)), dtype=torch.uint8).to(DEV)
-    d_consts = torch.empty(40, dtype=torch.uint8, device=DEV)
+    d_consts = torch.empty(lz.ZERO_ADAM_CONSTS_BYTES, dtype=torch.uint8, device=DEV)
     init = lz.ScalerState(1024.0, 0, 1, 0)
     d_state = torch.frombuffer(bytearray(bytes(init)), dtype=torch.uint8).to(DEV)
     prm = lz.ScalerParams(2.0, 0.5, 2)

@@ -219,3 +219,74 @@ def test_stage3_gpt2_small_sampled():
         check_f32(f"step {t} m", cur[1][idx_dev].cpu().numpy(), m_s)
         check_f32(f"step {t} v", cur[2][idx_dev].cpu().numpy(), v_s)
         check_f16(f"step {t} params", f16np(torch.cat(shards)[idx_dev]), p_s)
+
+
+@pytest.mark.parametrize("nd", [3, 8])
+def test_stage3_prefetch_schedule_vs_oracle(nd):
+    """The two-stream schedule bench.py times: forward gathers, then backward gathers one layer
+    ahead on a side stream while the main stream runs the previous layer's update (gather of
+    layer l-1 beside the update of layer l; each update waits for its own layer's gather).
+    Two steps; every gathered layer, the state and the partitions equal zero3_step."""
+    numels, split = [40000, 1234, 30000, 777, 5003, 999, 4096], [1, 2, 2, 2]
+    pl = lz.zero_plan_create(numels, nd, 3, 0)
+    psi, psi_p, S, _ = lz.zero_plan_info(pl)
+    opl = oracle.plan(numels, nd, 0)
+    layers = oracle.layer_ranges(opl, split)
+    gb = oracle.grad_buckets(opl, layers)
+    L = len(layers)
+    master, m, v = synth.state_warm(psi_p, seed=71)
+    w_r, m_r, v_r = master.numpy(), m.numpy(), v.numpy()
+    p16 = oracle.f2h(w_r)
+    ref_shards = [p16[q * S:(q + 1) * S].copy() for q in range(nd)]
+    shards = _partitions(torch.from_numpy(p16.view(np.float16)), nd)
+    cur = [x.to(DEV) for x in (master, m, v)]
+    nxt = [torch.empty_like(x) for x in cur]
+    main, gs = torch.cuda.current_stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()   # noqa: E731
+    for t in (1, 2):
+        g_cpu = []
+        for r in range(nd):
+            g = torch.zeros(psi_p, dtype=torch.float16)
+            g[:psi] = synth.grad_f16(psi, 1e-3, seed=72, rank=r, step=t)
+            g_cpu.append(g)
+        grads = [g.to(DEV) for g in g_cpu]
+        fwd = [torch.empty(hi - lo, dtype=torch.float16, device=DEV) for lo, hi in layers]
+        bwd = [torch.empty(hi - lo, dtype=torch.float16, device=DEV) for lo, hi in layers]
+        st = status_word()
+        start = ev()
+        start.record(main)
+        gs.wait_event(start)
+        g_done = [ev() for _ in range(L)]
+
+        def gather(l, out):
+            lo, hi = layers[l]
+            lz.zero_gather_params(pl, lo, hi - lo, shards, out, st, gs)
+
+        for l in range(L):
+            gather(l, fwd[l])
+        gather(L - 1, bwd[L - 1])
+        g_done[L - 1].record(gs)
+        for l in range(L - 1, -1, -1):
+            lo, _ = layers[l]
+            _, ghi = gb[l]
+            main.wait_event(g_done[l])
+            lz.zero_stage3_step_fused(pl, lo, ghi - lo, [g[lo:ghi] for g in grads],
+                                      *[x[lo:ghi] for x in cur], *[x[lo:ghi] for x in nxt],
+                                      shards, HP, t, st, main)
+            if l > 0:
+                gather(l - 1, bwd[l - 1])      # beside layer l's update
+                g_done[l - 1].record(gs)
+        lz.zero_stage3_step_commit(pl, *cur, *nxt, shards, st, main)
+        main.wait_stream(gs)
+        assert lz.zero_step_status(st) == (lz.ZERO_OK, 0)
+        ref = oracle.zero3_step(opl, layers, lambda l, r: g_cpu[r].numpy()[gb[l][0]:gb[l][1]],
+                                w_r, m_r, v_r, ref_shards, ORC_HP, t)
+        for l in range(L):
+            assert np.array_equal(f16np(fwd[l]), ref.gathered_fwd[l])
+            assert np.array_equal(f16np(bwd[l]), ref.gathered_bwd[l])
+        cur, nxt = nxt, cur
+        check_f32(f"step {t} master", f32np(cur[0]), ref.master)
+        check_f32(f"step {t} v", f32np(cur[2]), ref.v)
+        for q in range(nd):
+            check_f16(f"step {t} partition {q}", f16np(shards[q]), ref.param_shards[q])
+        w_r, m_r, v_r, ref_shards = ref.master, ref.m, ref.v, ref.param_shards

@@ -42,7 +42,7 @@ def test_stage2_fused_scheduler_reused_across_steps(n_slots):
     params = torch.from_numpy(oracle.f2h(master.numpy()).view(np.float16)).to(DEV)
     slot_elems = lz.zero_sched_slot_elems(pl, n_slots)
     slots = torch.empty(slot_elems, dtype=torch.float16, device=DEV)
-    d_consts = torch.empty(40, dtype=torch.uint8, device=DEV)
+    d_consts = torch.empty(lz.ZERO_ADAM_CONSTS_BYTES, dtype=torch.uint8, device=DEV)
     producer, stream = torch.cuda.Stream(), torch.cuda.Stream()
     main = torch.cuda.current_stream()
     st0 = status_word()

@@ -107,7 +107,7 @@ def test_1p3b_stage2_fused_scheduler_with_overflow_run():
     n_slots = 2
     slot_elems = lz.zero_sched_slot_elems(pl, n_slots)
     slots = torch.empty(slot_elems, dtype=torch.float16, device=DEV)
-    d_consts = torch.empty(40, dtype=torch.uint8, device=DEV)
+    d_consts = torch.empty(lz.ZERO_ADAM_CONSTS_BYTES, dtype=torch.uint8, device=DEV)
     producer, stream = torch.cuda.Stream(), torch.cuda.Stream()
     main = torch.cuda.current_stream()
 

@@ -507,6 +507,7 @@ cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,
     ZK_Q8_CASE(8, 4);
     ZK_Q8_CASE(12, 4);
     ZK_Q8_CASE(16, 4);
+    ZK_Q8_CASE(20, 4);
     ZK_Q8_CASE(24, 4);
     ZK_Q8_CASE(8, 8);
     ZK_Q8_CASE(12, 8);

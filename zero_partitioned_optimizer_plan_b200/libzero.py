@@ -50,6 +50,7 @@ SYMBOLS = (
     "zero_scaler_update", "zero_quantize_q8", "zero_step_fused_q8", "zero_step_fused_q8_dc",
     "zero_overlap_begin", "zero_overlap_end",
     "zero_gather_params", "zero_stage3_step_fused", "zero_stage3_step_commit",
+    "zero_step_fused_ranges",
     "zero_sched_slot_elems", "zero_sched_create", "zero_sched_create_fused",
     "zero_sched_begin_bucket", "zero_sched_rebind_fused", "zero_sched_rebind_status",
     "zero_sched_end_bucket", "zero_sched_wait", "zero_sched_launches", "zero_sched_destroy",
@@ -82,17 +83,28 @@ class _HP(C.Structure):
 
 class AdamConsts(C.Structure):
     """zero_adam_consts: one step's fp32 constants (copy into device memory for the _dc calls;
-    bytes(obj) gives its 40-byte image)."""
+    bytes(obj) gives its ZERO_ADAM_CONSTS_BYTES-byte image)."""
     _fields_ = [("beta1", C.c_float), ("one_minus_beta1", C.c_float), ("beta2", C.c_float),
                 ("one_minus_beta2", C.c_float), ("step_size", C.c_float),
                 ("bias2_sqrt", C.c_float), ("eps", C.c_float), ("loss_scale", C.c_float),
                 ("inv_loss_scale", C.c_float), ("loss_scale_pow2", C.c_int32)]
 
 
+ZERO_ADAM_CONSTS_BYTES = C.sizeof(AdamConsts)
+
+
 class ScalerState(C.Structure):
     """zero_scaler_state (24 bytes; copy into 8-byte-aligned device memory)."""
     _fields_ = [("scale", C.c_float), ("good_steps", C.c_int32), ("next_step", C.c_int64),
                 ("skipped_steps", C.c_int64)]
+
+
+class FusedRange(C.Structure):
+    """zero_fused_range: one range of a step for zero_step_fused_ranges."""
+    _fields_ = [("n", C.c_uint64), ("rank_grads", C.POINTER(C.c_void_p)),
+                ("master_in", C.c_void_p), ("m_in", C.c_void_p), ("v_in", C.c_void_p),
+                ("master_out", C.c_void_p), ("m_out", C.c_void_p), ("v_out", C.c_void_p),
+                ("param_out", C.c_void_p)]
 
 
 class ScalerParams(C.Structure):
@@ -146,6 +158,7 @@ def _load():
     L.zero_adam_consts_table.argtypes = [P(_HP), i64, i64, P(AdamConsts)]
     L.zero_scaler_prepare.argtypes = [vp, vp, i64, vp, vp, vp]
     L.zero_scaler_update.argtypes = [vp, P(ScalerParams), vp, vp]
+    L.zero_step_fused_ranges.argtypes = [i32, i32, P(FusedRange), P(_HP), i64, vp, i32, vp]
     L.zero_gather_params.argtypes = [vp, u64, u64, P(vp), vp, vp, vp]
     L.zero_stage3_step_fused.argtypes = [vp, u64, u64, P(vp), vp, vp, vp, vp, vp, vp, P(vp), P(_HP),
                                    i64, vp, vp]
@@ -308,22 +321,32 @@ def zero_step_fused(n: int, nd: int, rank_grads, master_in, m_in, v_in, master_o
                                 step, _ptr(d_status, 4), _stream(stream)), "zero_step_fused")
 
 
-class PreparedStepFused:
-    """zero_step_fused with its pointer arguments marshalled once, for a call repeated every
-    step (e.g. one per bucket): calling it passes the stored addresses, the step's
-    hyperparameters, t, the status word and the stream straight to the C entry point."""
+class PreparedStepRanges:
+    """zero_step_fused_ranges with its range descriptors marshalled once: each item of `ranges`
+    is (n, rank_grads, master_in, m_in, v_in, master_out, m_out, v_out, param_out) as
+    zero_step_fused takes them. Calling it launches every range of the step in one C call."""
 
-    def __init__(self, n: int, nd: int, rank_grads, master_in, m_in, v_in, master_out, m_out,
-                 v_out, param_out):
-        self._args = (n, nd, _ptr_array(rank_grads, 2), _ptr(master_in, 4), _ptr(m_in, 4),
-                      _ptr(v_in, 4), _ptr(master_out, 4), _ptr(m_out, 4), _ptr(v_out, 4),
-                      _ptr(param_out, 2))
+    def __init__(self, nd: int, ranges):
+        self.nd = nd
+        self._grad_arrays = [_ptr_array(r[1], 2) for r in ranges]   # kept alive
+        arr = (FusedRange * max(len(ranges), 1))()
+        for i, (r, g) in enumerate(zip(ranges, self._grad_arrays)):
+            arr[i] = FusedRange(r[0], C.cast(g, C.POINTER(C.c_void_p)), *[
+                _ptr(x, 4) for x in r[2:8]], _ptr(r[8], 2))
+        self._arr = arr
+        self.count = len(ranges)
 
-    def __call__(self, hp_ref, step: int, d_status: int, stream: int):
-        """hp_ref: hparams_ref(hp); d_status, stream: raw addresses (status_ptr, stream_handle)."""
-        code = _lib.zero_step_fused(*self._args, hp_ref, step, d_status, stream)
+    def __call__(self, hp_ref, step: int, d_status: int, overlap: bool, stream: int):
+        code = _lib.zero_step_fused_ranges(self.nd, self.count, self._arr, hp_ref, step, d_status,
+                                           1 if overlap else 0, stream)
         if code:
-            raise ZeroError(code, "zero_step_fused")
+            raise ZeroError(code, "zero_step_fused_ranges")
+
+
+def zero_step_fused_ranges(nd: int, ranges, hp: AdamHP, step: int, d_status, overlap=True,
+                           stream=None):
+    PreparedStepRanges(nd, ranges)(hparams_ref(hp), step, _ptr(d_status, 4), overlap,
+                                   _stream(stream))
 
 
 def hparams_ref(hp: AdamHP):
