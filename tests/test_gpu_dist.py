@@ -31,7 +31,7 @@ def _case(numels):
     return psi, grad, master, m, v, torch
 
 
-def _worker(port, numels, bucket, out):
+def _worker(port, numels, bucket, out, peer=False):
     import datetime
     import torch
     import torch.distributed as dist
@@ -50,8 +50,15 @@ def _worker(port, numels, bucket, out):
         st_out = [torch.full_like(x, float("nan")) for x in st_in]
         params = torch.zeros(psi, dtype=torch.float16, device=dev)
         status = torch.zeros(1, dtype=torch.int32, device=dev)
-        step = DistZeroStep(psi, bucket)
-        flag = step.step(grad.to(dev), st_in, st_out, params, lz.AdamHP(), 1, status)
+        if peer:    # gradients produced into symmetric memory; the owner reads them in place
+            from zero_partitioned_optimizer_plan_b200.dist import SymmetricPeerBuffers
+            peers = SymmetricPeerBuffers(psi, torch.float16, dev)
+            peers.local.copy_(grad.to(dev))
+            step = DistZeroStep(psi, bucket, peers=peers)
+            flag = step.step(peers.local, st_in, st_out, params, lz.AdamHP(), 1, status)
+        else:
+            step = DistZeroStep(psi, bucket)
+            flag = step.step(grad.to(dev), st_in, st_out, params, lz.AdamHP(), 1, status)
         torch.cuda.synchronize()
         out.put((int(flag.item()), int(status.item()), [x.cpu().numpy() for x in st_out],
                  params.cpu().numpy().view(np.uint16)))
@@ -59,13 +66,16 @@ def _worker(port, numels, bucket, out):
         dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("peer", [False, True])
 @pytest.mark.parametrize("bucket", [0, 3000])
-def test_distributed_step_one_rank_nccl(bucket):
+def test_distributed_step_one_rank_nccl(bucket, peer):
+    """The all-to-all form and the peer-read form (the rank's gradient in torch symmetric
+    memory, read by the owner's kernel through its symmetric address)."""
     import oracle
     numels = [1000, 37, 4099, 12345]
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    p = ctx.Process(target=_worker, args=(_free_port(), numels, bucket, q))
+    p = ctx.Process(target=_worker, args=(_free_port(), numels, bucket, q, peer))
     p.start()
     try:
         flag, status, shard, params = q.get(timeout=240)

@@ -303,6 +303,76 @@ def test_distributed_step_failure_on_one_rank_voids_it_everywhere(ws, fail_rank)
         assert t == ws
 
 
+def _worker_dist_peer(rank, ws, port, numels, bucket, bad_rank, bufs, out):
+    import datetime
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle
+    from zero_partitioned_optimizer_plan_b200.dist import DistZeroStep, SharedPeerBuffers
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        psi_p, grads, master, m, v = _dist_case(numels, ws, bad_rank)
+        S = psi_p // ws
+        peers = SharedPeerBuffers(bufs, rank)
+        peers.local.copy_(grads[rank])        # this rank's backward pass, into its own buffer
+        st_in = [x[rank * S:(rank + 1) * S].clone() for x in (master, m, v)]
+        st_out = [torch.full_like(x, float("nan")) for x in st_in]
+        params = torch.zeros(psi_p, dtype=torch.float16)
+        status = torch.zeros(1, dtype=torch.int32)
+        step = DistZeroStep(psi_p, bucket, compute=_OracleCompute(), peers=peers)
+        flag = step.step(peers.local, st_in, st_out, params, oracle.AdamHP(), 1, status)
+        out.put((rank, int(flag.item()), int(status.item()), [x.numpy() for x in st_out],
+                 params.numpy().view("uint16"), step._recv is None))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("ws,bucket,bad_rank", [(2, 0, -1), (3, 2500, -1), (3, 2500, 2)])
+def test_distributed_step_peer_reads_gloo(ws, bucket, bad_rank):
+    """The peer-read form of the distributed step: each rank writes its gradient into its own
+    buffer, readable by every rank (here CPU tensors in memory the processes share, standing
+    for NVLink peer mappings); per bucket a barrier, then each owner reduces its part straight
+    from the peers' buffers -- no all-to-all, no receive buffers. Every rank's shard and full
+    fp16 parameters equal the oracle's data-parallel step bit for bit; an inf on one rank
+    skips the step everywhere."""
+    import numpy as np
+    import torch
+    import oracle
+    numels = [1000, 37, 4099, 12345]
+    psi_p = -(-sum(numels) // ws) * ws
+    bufs = [torch.zeros(psi_p, dtype=torch.float16).share_memory_() for _ in range(ws)]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_dist_peer,
+                         args=(r, ws, port, numels, bucket, bad_rank, bufs, q)) for r in range(ws)]
+    for p in procs:
+        p.start()
+    try:
+        res = sorted((q.get(timeout=240) for _ in range(ws)), key=lambda x: x[0])
+    finally:
+        for p in procs:
+            p.join(60)
+            if p.exitcode is None:
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    psi_p, grads, master, m, v = _dist_case(numels, ws, bad_rank)
+    ref = oracle.dp_step([g.numpy() for g in grads], master.numpy(), m.numpy(), v.numpy(),
+                         oracle.f2h(master.numpy()), oracle.AdamHP(), 1)
+    S = psi_p // ws
+    for rank, flag, status, shard, params, no_recv in res:
+        assert no_recv
+        assert flag == (1 if bad_rank >= 0 else 0)
+        assert bool(status & 2) == ref.skipped == (bad_rank >= 0)
+        for got, want in zip(shard, (ref.master, ref.m, ref.v)):
+            assert np.array_equal(got.view(np.uint32),
+                                  want[rank * S:(rank + 1) * S].view(np.uint32))
+        assert np.array_equal(params, ref.params16)
+
+
 def test_dist_bucket_map_matches_the_plan():
     """dist.py's bucket ranges and per-owner split sizes agree with the oracle's plan (backward
     order, element-granular, last bucket short) for several sizes, bucket lengths and Nd."""

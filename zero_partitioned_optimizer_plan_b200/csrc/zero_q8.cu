@@ -372,7 +372,10 @@ __global__ void __launch_bounds__(256) fused_q8_plain_kernel(const __grid_consta
 // Consumer warps, values per thread and stage split per Nd for the int8 payload, measured on
 // B200: the dequantizing accumulation issues about twice the instructions per byte of the fp16
 // sum, so up to Nd = 16 the most warps win (Nd = 2/8/16: 6.4/6.7/6.6 TB/s with 24 warps against
-// 5.0/5.4/5.5 with 16); above, 16 warps with the budget split in two (Nd = 32/64: 5.7/4.8 TB/s).
+// 5.0/5.4/5.5 with 16); above, 16 warps with the budget split in two (Nd = 32/64: 5.9/5.1 TB/s).
+// Not better at Nd = 64 (flat 2^28, same box): 8 values per thread with 8, 12 or 16 warps
+// (4.6-4.7 TB/s), three or four stages (4.7, 3.9), 12/20/24 warps with three stages (4.4-4.8),
+// two CTAs per SM of 8 or 12 warps with half the shared memory each (5.0, 4.8).
 struct VariantQ8 {
     int warps;
     int elems;           // values per consumer thread and tile
@@ -507,11 +510,14 @@ cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,
     ZK_Q8_CASE(8, 4);
     ZK_Q8_CASE(12, 4);
     ZK_Q8_CASE(16, 4);
-    ZK_Q8_CASE(20, 4);
     ZK_Q8_CASE(24, 4);
+#if defined(ZK_Q8_WARPS) || defined(ZK_Q8_ELEMS)
+    // shapes measured and not kept (see pick_variant_q8), compiled for comparisons only
+    ZK_Q8_CASE(20, 4);
     ZK_Q8_CASE(8, 8);
     ZK_Q8_CASE(12, 8);
     ZK_Q8_CASE(16, 8);
+#endif
 #undef ZK_Q8_CASE
     return cudaErrorInvalidConfiguration;
 }

@@ -32,6 +32,16 @@ reads, and waiting on bucket k's exchange makes the current stream, not the host
 all-gather runs in place on NCCL (each rank's shard already sits at its offset of the output);
 other backends gather from a shard copy held in a buffer allocated once.
 
+Peer reads (``peers``: SymmetricPeerBuffers or SharedPeerBuffers). In place of the all-to-all,
+every rank's local gradient lives in a buffer that every rank can address (on GPUs: torch symmetric memory, the peers'
+buffers mapped into this rank's address space over NVLink). The owner's fused step then takes
+its Nd rows straight from the peers' buffers: the bulk copies of the library's kernel read
+each slice across NVLink once, into shared memory, with no staging copy in between (plain
+loads, no multicast). Per bucket a barrier (a one-element all-reduce, ordered on the streams
+like any collective) guarantees that every rank has produced the bucket before an owner reads
+it; the all-reduce of the void bits at the end of the step is the barrier after which no
+owner reads this step's gradients any more, so the next backward pass may overwrite them.
+
 The collectives are torch.distributed calls (NCCL on GPUs, gloo on CPUs); the arithmetic is the
 library's. ``compute`` replaces the two library calls (the tests run the exchange on CPU
 processes with another implementation of them).
@@ -74,6 +84,39 @@ def owner_parts(lo: int, hi: int, shard: int, nd: int) -> List[int]:
     return [max(0, min(hi, (q + 1) * shard) - max(lo, q * shard)) for q in range(nd)]
 
 
+# Peer buffers: every rank's local-gradient buffer (psi_p values), addressable from every rank.
+# An object with ``local`` (this rank's buffer, where the backward pass writes its gradients)
+# and rows(a, b) (the Nd ranks' elements [a, b), in rank order, in the form the compute takes:
+# device addresses or tensors).
+class SymmetricPeerBuffers:
+    """The buffers in torch symmetric memory: rows are the peers' device addresses (NVLink
+    peer mappings; this rank's own buffer among them)."""
+
+    def __init__(self, psi_p: int, dtype, device, group=None):
+        import torch.distributed as dist
+        import torch.distributed._symmetric_memory as symm
+        self.local = symm.empty(psi_p, dtype=dtype, device=device)
+        name = (group or dist.group.WORLD).group_name
+        self.handle = symm.rendezvous(self.local, name)
+        self.ptrs = [int(p) for p in self.handle.buffer_ptrs]
+        self.esize = self.local.element_size()
+
+    def rows(self, a: int, b: int):
+        return [p + a * self.esize for p in self.ptrs]
+
+
+class SharedPeerBuffers:
+    """Buffers given as tensors every rank can read (e.g. CPU tensors in shared memory shared
+    by the processes of a test)."""
+
+    def __init__(self, tensors, rank: int):
+        self.tensors = list(tensors)
+        self.local = self.tensors[rank]
+
+    def rows(self, a: int, b: int):
+        return [t[a:b] for t in self.tensors]
+
+
 class LibzeroCompute:
     """The owner's fused step and commit through the library (CUDA tensors)."""
 
@@ -93,7 +136,7 @@ class DistZeroStep:
     """One rank's side of the distributed step. psi_p: the flat padded length (a multiple of
     the world size); bucket: elements per bucket (0: one bucket, stage 1)."""
 
-    def __init__(self, psi_p: int, bucket: int = 0, group=None, compute=None):
+    def __init__(self, psi_p: int, bucket: int = 0, group=None, compute=None, peers=None):
         import torch.distributed as dist
         self.dist = dist
         self.group = group
@@ -106,6 +149,7 @@ class DistZeroStep:
         self.buckets = bucket_ranges(psi_p, bucket)
         self.parts = [owner_parts(lo, hi, self.shard, self.nd) for lo, hi in self.buckets]
         self.compute = compute or LibzeroCompute()
+        self.peers = peers
         self.in_place_gather = dist.get_backend(group) == "nccl"
         self._recv = None      # two receive buffers, nd * (largest owner part) values each
         self._bits = None      # the three void bits, combined across ranks
@@ -114,14 +158,15 @@ class DistZeroStep:
 
     def _buffers(self, local_grad, params_full, status):
         import torch
-        if self._recv is None or self._recv[0].device != local_grad.device or \
-                self._recv[0].dtype != local_grad.dtype:
+        if self.peers is None and (self._recv is None or self._recv[0].device != local_grad.device
+                                   or self._recv[0].dtype != local_grad.dtype):
             most = max(p[self.rank] for p in self.parts)
             self._recv = [torch.empty(self.nd * most, dtype=local_grad.dtype,
                                       device=local_grad.device) for _ in range(2)]
         if self._bits is None or self._bits.device != status.device:
             self._masks = torch.tensor(VOID_BITS, dtype=status.dtype, device=status.device)
             self._bits = torch.empty_like(self._masks)
+            self._tick = torch.zeros(1, dtype=status.dtype, device=status.device)
         if not self.in_place_gather and (
                 self._gather_src is None or self._gather_src.device != params_full.device):
             self._gather_src = torch.empty(self.shard, dtype=params_full.dtype,
@@ -142,6 +187,11 @@ class DistZeroStep:
         own = params_full[r * S:(r + 1) * S]
         nb = len(self.buckets)
         works = [None] * nb
+        if self.peers is not None:
+            if local_grad is not self.peers.local:
+                self.peers.local.copy_(local_grad)   # produce into peers.local to avoid this
+            self._reduce_from_peers(state_in, state_out, own, hp, t, status)
+            return self._finish(state_in, state_out, own, params_full, status)
 
         def exchange(k):
             lo, hi = self.buckets[k]
@@ -167,6 +217,35 @@ class DistZeroStep:
             self.compute.fused(mine, rows, [x[a:a + mine] for x in state_in],
                                [x[a:a + mine] for x in state_out], own[a:a + mine], hp, t,
                                status)
+        return self._finish(state_in, state_out, own, params_full, status)
+
+    def _reduce_from_peers(self, state_in, state_out, own, hp, t, status):
+        """Per bucket: a barrier (every rank has produced it), then the owner's fused step on
+        its part, reading the Nd rows in the peers' buffers. The barrier of bucket k+1 is in
+        flight while bucket k is reduced."""
+        dist, nd, r, S = self.dist, self.nd, self.rank, self.shard
+        nb = len(self.buckets)
+        works = [None] * nb
+
+        def barrier(k):
+            works[k] = dist.all_reduce(self._tick, group=self.group, async_op=True)
+
+        barrier(0)
+        for k, (lo, hi) in enumerate(self.buckets):
+            if k + 1 < nb:
+                barrier(k + 1)
+            works[k].wait()
+            works[k] = None
+            a, b = max(lo, r * S), min(hi, (r + 1) * S)     # my part of the bucket
+            if a >= b:
+                continue
+            self.compute.fused(b - a, self.peers.rows(a, b),
+                               [x[a - r * S:b - r * S] for x in state_in],
+                               [x[a - r * S:b - r * S] for x in state_out],
+                               own[a - r * S:b - r * S], hp, t, status)
+
+    def _finish(self, state_in, state_out, own, params_full, status):
+        dist, S = self.dist, self.shard
         # one verdict for the job: OR of every rank's void bits (MAX per bit)
         import torch
         torch.bitwise_and(status.expand(len(VOID_BITS)), self._masks, out=self._bits)
