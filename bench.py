@@ -1114,6 +1114,10 @@ def run_sweep(args, dev, ws, barrier):
                     "params_per_s": aggregate_rate(ws, wl.n, 1, ms),
                     "kernel_gbs": gbs, "frac": gbs / peak,
                     "bytes_per_step": wl.bytes_per_step})
+        if ws == 1 and not args.no_cpu_baseline:   # the oracle at this Nd, a short sample
+            rate, reps, secs = cpu_oracle_rate(nd, 1_000_000, 2.0)
+            out[-1]["cpu_oracle_params_per_s"] = rate
+            out[-1]["cpu_oracle_sample"] = f"1,000,000 elements, {reps} steps, {secs:.1f} s, 1 core"
         del wl, status
         gc.collect()
         torch.cuda.empty_cache()

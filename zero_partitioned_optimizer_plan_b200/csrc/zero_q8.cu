@@ -28,6 +28,10 @@
 #include "zero_device.cuh"
 #include "zero_internal.h"
 
+#ifndef ZK_Q8_SHARED_LOADS   // rank loop: explicit 32-bit shared-window loads
+#define ZK_Q8_SHARED_LOADS 0
+#endif
+
 namespace zk {
 
 namespace {
@@ -258,6 +262,8 @@ template <int W, int E, bool kDC>
 __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
     fused_q8_tma_kernel(const __grid_constant__ FusedQ8Args p) {
     static_assert(E == 4 || E == 8, "a thread's values sit in one record");
+    // bytes of one rank's run of records in a stage (the launcher's p.row, checked below)
+    constexpr uint32_t kRow = (32u * W * E / kQB) * kRec;
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
@@ -275,7 +281,8 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
     const uint32_t e0 = (uint32_t)threadIdx.x * E;
     bool bad = false;
     uint32_t it = 0;
-    bool ok = true;
+    bool ok = p.row == kRow && T == 32u * W * E;   // self-check of the launch's shape
+    if (!ok && threadIdx.x == 0) atomicOr(p.status, ZERO_FLAG_BOUNDS);
     for (uint64_t tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
         const TileSpan ts = tile_span(tile, T, p.n_tiled);
         const bool active = e0 < ts.cnt;
@@ -303,15 +310,32 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
 #pragma unroll
                 for (int k = 0; k < P; ++k) ap[k] = f2_pack(acc[2 * k], acc[2 * k + 1]);
                 const uint64_t nbias = f2_pack(-8388736.0f, -8388736.0f);   // -(2^23 + 128)
+#if ZK_Q8_SHARED_LOADS
+                // 32-bit shared-window addresses: rank r's record sits kRow bytes after rank
+                // r-1's, so the unrolled loads take immediate offsets from one base
+                const uint32_t sbase = smem_addr(rec0);
+                const uint32_t qoff = e0 % kQB;
+#endif
 #pragma unroll(16 / E)
                 for (uint32_t r = 0; r < nr; ++r) {
-                    const uint8_t* rec = rec0 + (size_t)r * p.row;
+#if ZK_Q8_SHARED_LOADS
+                    const uint32_t ra = sbase + r * kRow;
+                    float sc;
+                    asm volatile("ld.shared.f32 %0, [%1+128];" : "=f"(sc) : "r"(ra));
+#else
+                    const uint8_t* rec = rec0 + (size_t)r * kRow;
                     const float sc = *reinterpret_cast<const float*>(rec + kQB);
+#endif
                     const uint64_t ss = f2_pack(sc, sc);
 #pragma unroll
                     for (int k4 = 0; k4 < E / 4; ++k4) {
+#if ZK_Q8_SHARED_LOADS
+                        uint32_t qq;
+                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(qq) : "r"(ra + qoff + 4 * k4));
+#else
                         const uint32_t qq =
                             *reinterpret_cast<const uint32_t*>(rec + e0 % kQB + 4 * k4);
+#endif
                         const uint32_t biased = qq ^ 0x80808080u;   // each byte q + 128
                         const uint64_t q01 =
                             f2_add(f2_pack(q_placed(biased, 0), q_placed(biased, 1)), nbias);
