@@ -751,6 +751,10 @@ def _step_zero3(self, t, status, ev=None, grads=None):
         gather(l)
     gather(L - 1)                             # backward, one layer ahead of the updates
     self.g_done[L - 1].record(gs)
+    # the layers' updates touch disjoint ranges: one overlap region on the main stream (its
+    # event waits and records are allowed inside; an event recorded after an update completes
+    # only when every update before it has)
+    lz.zero_overlap_begin(main)
     for l in range(L - 1, -1, -1):
         lo, hi = self.layers[l]
         main.wait_event(self.g_done[l])
@@ -768,6 +772,7 @@ def _step_zero3(self, t, status, ev=None, grads=None):
                 gs.wait_event(self.f_done[l + 1])   # buffer (l-1) % 2 was layer l+1's
             gather(l - 1)
             self.g_done[l - 1].record(gs)
+    lz.zero_overlap_end(main)
     lz.zero_stage3_step_commit(pl, *self.cur, *self.nxt, shards, status, main)
     if timed:
         ev[1].record(main)

@@ -266,6 +266,7 @@ def test_stage3_prefetch_schedule_vs_oracle(nd):
             gather(l, fwd[l])
         gather(L - 1, bwd[L - 1])
         g_done[L - 1].record(gs)
+        lz.zero_overlap_begin(main)            # the updates chained, as in bench.py
         for l in range(L - 1, -1, -1):
             lo, _ = layers[l]
             _, ghi = gb[l]
@@ -276,6 +277,7 @@ def test_stage3_prefetch_schedule_vs_oracle(nd):
             if l > 0:
                 gather(l - 1, bwd[l - 1])      # beside layer l's update
                 g_done[l - 1].record(gs)
+        lz.zero_overlap_end(main)
         lz.zero_stage3_step_commit(pl, *cur, *nxt, shards, st, main)
         main.wait_stream(gs)
         assert lz.zero_step_status(st) == (lz.ZERO_OK, 0)

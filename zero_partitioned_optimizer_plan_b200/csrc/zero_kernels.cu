@@ -224,7 +224,8 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
     const uint32_t T = p.g.tile;
     const uint32_t e0 = (uint32_t)threadIdx.x * E;
     uint32_t it = 0;
-    bool ok = true;
+    bool ok = p.g.tile == 32u * W * E;   // self-check of the launch's shape
+    if (!ok && threadIdx.x == 0) atomicOr(p.status, ZERO_FLAG_BOUNDS);
     for (uint64_t tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
         const TileSpan ts = tile_span(tile, T, p.n_tiled);
         const bool active = e0 < ts.cnt;   // cnt is a multiple of 8, E divides 8
@@ -232,7 +233,8 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
 #pragma unroll
         for (int j = 0; j < E; ++j) acc[j] = 0.0f;
         for (uint32_t c = 0; c < p.g.nchunks; ++c, ++it) {
-            if (!consume_stage<E, true>(p.g, p.nd, full, empty, data, it, c, e0, active, acc, w,
+            if (!consume_stage<E, true, 32u * W * E>(
+                    p.g, p.nd, full, empty, data, it, c, e0, active, acc, w,
                                         m, v)) {
                 if ((threadIdx.x & 31) == 0) atomicOr(p.status, ZERO_FLAG_TIMEOUT);
                 ok = false;
@@ -326,7 +328,8 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
     const uint32_t T = p.g.tile;
     const uint32_t e0 = (uint32_t)threadIdx.x * E;
     uint32_t it = 0;
-    bool ok = true;
+    bool ok = p.g.tile == 32u * W * E;   // self-check of the launch's shape
+    if (!ok && threadIdx.x == 0) atomicOr(p.status, ZERO_FLAG_BOUNDS);
     for (uint64_t tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
         const TileSpan ts = tile_span(tile, T, p.n_tiled);
         const bool active = e0 < ts.cnt;
@@ -334,7 +337,8 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
 #pragma unroll
         for (int j = 0; j < E; ++j) acc[j] = 0.0f;
         for (uint32_t c = 0; c < p.g.nchunks; ++c, ++it) {
-            if (!consume_stage<E, false>(p.g, p.nd, full, empty, data, it, c, e0, active, acc,
+            if (!consume_stage<E, false, 32u * W * E>(
+                    p.g, p.nd, full, empty, data, it, c, e0, active, acc,
                                          unused, unused, unused)) {
                 if ((threadIdx.x & 31) == 0) atomicOr(p.status, ZERO_FLAG_TIMEOUT);
                 ok = false;
