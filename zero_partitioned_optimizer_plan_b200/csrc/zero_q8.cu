@@ -28,10 +28,6 @@
 #include "zero_device.cuh"
 #include "zero_internal.h"
 
-#ifndef ZK_Q8_SHARED_LOADS   // rank loop: explicit 32-bit shared-window loads
-#define ZK_Q8_SHARED_LOADS 0
-#endif
-
 namespace zk {
 
 namespace {
@@ -310,32 +306,17 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
 #pragma unroll
                 for (int k = 0; k < P; ++k) ap[k] = f2_pack(acc[2 * k], acc[2 * k + 1]);
                 const uint64_t nbias = f2_pack(-8388736.0f, -8388736.0f);   // -(2^23 + 128)
-#if ZK_Q8_SHARED_LOADS
-                // 32-bit shared-window addresses: rank r's record sits kRow bytes after rank
-                // r-1's, so the unrolled loads take immediate offsets from one base
-                const uint32_t sbase = smem_addr(rec0);
-                const uint32_t qoff = e0 % kQB;
-#endif
+                // rank r's record sits kRow bytes after rank r-1's: the unrolled loads take
+                // immediate offsets
 #pragma unroll(16 / E)
                 for (uint32_t r = 0; r < nr; ++r) {
-#if ZK_Q8_SHARED_LOADS
-                    const uint32_t ra = sbase + r * kRow;
-                    float sc;
-                    asm volatile("ld.shared.f32 %0, [%1+128];" : "=f"(sc) : "r"(ra));
-#else
                     const uint8_t* rec = rec0 + (size_t)r * kRow;
                     const float sc = *reinterpret_cast<const float*>(rec + kQB);
-#endif
                     const uint64_t ss = f2_pack(sc, sc);
 #pragma unroll
                     for (int k4 = 0; k4 < E / 4; ++k4) {
-#if ZK_Q8_SHARED_LOADS
-                        uint32_t qq;
-                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(qq) : "r"(ra + qoff + 4 * k4));
-#else
                         const uint32_t qq =
                             *reinterpret_cast<const uint32_t*>(rec + e0 % kQB + 4 * k4);
-#endif
                         const uint32_t biased = qq ^ 0x80808080u;   // each byte q + 128
                         const uint64_t q01 =
                             f2_add(f2_pack(q_placed(biased, 0), q_placed(biased, 1)), nbias);
@@ -399,7 +380,10 @@ __global__ void __launch_bounds__(256) fused_q8_plain_kernel(const __grid_consta
 // 5.0/5.4/5.5 with 16); above, 16 warps with the budget split in two (Nd = 32/64: 5.9/5.1 TB/s).
 // Not better at Nd = 64 (flat 2^28, same box): 8 values per thread with 8, 12 or 16 warps
 // (4.6-4.7 TB/s), three or four stages (4.7, 3.9), 12/20/24 warps with three stages (4.4-4.8),
-// two CTAs per SM of 8 or 12 warps with half the shared memory each (5.0, 4.8).
+// two CTAs per SM of 8 or 12 warps with half the shared memory each (5.0, 4.8). With the
+// compile-time record stride (the current loop, 5.4 TB/s at Nd = 64): eight values per thread
+// (4.8-5.0), scalar bias removal and fused multiply-adds instead of the packed pairs (4.9),
+// packed bias removal with scalar fused multiply-adds (5.0), explicit 32-bit shared loads (5.3).
 struct VariantQ8 {
     int warps;
     int elems;           // values per consumer thread and tile
