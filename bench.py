@@ -575,7 +575,19 @@ def _e2e_zero2_fused(self, t0, E, barrier, max_ms):
     slot_elems = lz.zero_sched_slot_elems(pl, n_slots)
     d_slots = torch.empty(slot_elems, dtype=torch.float16, device=dev)
     region = nd * self.stride
-    total = self.nb * region
+    # pinned host source: every bucket's gradients when the host has room (42 GB for the 1.3B
+    # list at Nd = 16), else as many buckets as half the host's available memory allows per
+    # rank, cycled (each step still uploads every bucket's bytes; only the source is reused)
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        avail = 0
+    host_buckets = self.nb
+    if avail and self.nb * region * 2 > avail // (2 * ws):
+        host_buckets = max(2, min(self.nb, (avail // (2 * ws)) // (region * 2)))
+    total = host_buckets * region
     h_grads = pinned_host(total, torch.float16)
     h_grads.copy_(self.slots[:total])          # the same gradients as the device-resident run
     h_params = [torch.empty(self.n, dtype=torch.float16, pin_memory=True) for _ in range(2)]
@@ -610,9 +622,10 @@ def _e2e_zero2_fused(self, t0, E, barrier, max_ms):
         for k, (lo, ln) in enumerate(self.buckets):
             ptrs = lz.zero_sched_begin_bucket(sch, k, up)
             with torch.cuda.stream(up):
+                hk = k % host_buckets
                 for r in range(nd):
                     off = (ptrs[r] - d_slots.data_ptr()) // 2
-                    src = h_grads[k * region + r * self.stride:k * region + r * self.stride + ln]
+                    src = h_grads[hk * region + r * self.stride:hk * region + r * self.stride + ln]
                     d_slots[off:off + ln].copy_(src, non_blocking=True)
                     h2d += 2 * ln if i == 0 else 0
             lz.zero_sched_end_bucket(sch, k, up)
@@ -641,7 +654,9 @@ def _e2e_zero2_fused(self, t0, E, barrier, max_ms):
     ems = max_ms(e0.elapsed_time(e1))
     out = {"ms": ems, "steps": E, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 2 * self.n + 4,
            "overlap": "bucket uploads into two staging slots, each gated by the release of its "
-                      "slot; the next step's uploads overlap this step's tail and download"}
+                      "slot; the next step's uploads overlap this step's tail and download",
+           "host_source": (f"all {self.nb} buckets in pinned host memory" if host_buckets ==
+                           self.nb else f"{host_buckets} buckets in pinned host memory, cycled")}
     unpin_host(h_grads)
     del h_grads, h_params, d_slots
     return out

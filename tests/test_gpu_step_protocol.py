@@ -97,6 +97,60 @@ def test_stage2_fused_scheduler_reused_across_steps(n_slots):
     lz.zero_sched_destroy(sch)
 
 
+def test_stage2_upload_from_pinned_host_through_two_slots():
+    """The end-to-end leg's data path: each bucket's Nd gradient slices copied from pinned host
+    memory into one of two staging slots on an upload stream (each copy waits, on that stream,
+    for the release of its slot), the fused bucket kernels on the scheduler's stream, the
+    commit, and the fp16 parameters downloaded. Two steps equal the oracle's stage-2 step."""
+    numels, nd, bucket = [40000, 1234, 30000, 777, 9999], 5, 7000
+    pl = lz.zero_plan_create(numels, nd, 2, bucket)
+    psi, psi_p, S, nb = lz.zero_plan_info(pl)
+    ref_plan = oracle.plan(numels, nd, bucket)
+    master, m, v = synth.state_warm(psi_p, seed=35)
+    pp = PingPong(master, m, v)
+    params = torch.from_numpy(oracle.f2h(master.numpy()).view(np.float16)).to(DEV)
+    slot_elems = lz.zero_sched_slot_elems(pl, 2)
+    slots = torch.empty(slot_elems, dtype=torch.float16, device=DEV)
+    d_consts = torch.empty(lz.ZERO_ADAM_CONSTS_BYTES, dtype=torch.uint8, device=DEV)
+    up, main = torch.cuda.Stream(), torch.cuda.current_stream()
+    st = status_word()
+    sch = lz.zero_sched_create_fused(pl, slots, slot_elems, 2, *pp.cur, *pp.nxt, params,
+                                     d_consts, st, main)
+    ref = (master.numpy(), m.numpy(), v.numpy(), oracle.f2h(master.numpy()))
+    for t in (1, 2):
+        g = []
+        for r in range(nd):
+            x = torch.zeros(psi_p, dtype=torch.float16)
+            x[:psi] = synth.grad_f16(psi, 1e-3, seed=36, rank=r, step=t)
+            g.append(x.pin_memory())
+        st = status_word()
+        c = lz.zero_adam_consts_for_step(HP, t)
+        d_consts.copy_(torch.frombuffer(bytearray(bytes(c)), dtype=torch.uint8))
+        lz.zero_sched_rebind_fused(sch, *pp.cur, *pp.nxt, params, st)
+        lz.zero_overlap_begin(main)
+        for k in range(nb):
+            lo, ln, _, _ = lz.zero_plan_bucket(pl, k)
+            ptrs = lz.zero_sched_begin_bucket(sch, k, up)
+            with torch.cuda.stream(up):
+                for r in range(nd):
+                    _slot_view(slots, ptrs[r], ln).copy_(g[r][lo:lo + ln], non_blocking=True)
+            lz.zero_sched_end_bucket(sch, k, up)
+        lz.zero_overlap_end(main)
+        lz.zero_sched_wait(sch, main)
+        lz.zero_step_commit(psi_p, *pp.cur, *pp.nxt, params, st, main)
+        h_params = torch.empty(psi_p, dtype=torch.float16, pin_memory=True)
+        h_params.copy_(params, non_blocking=True)
+        assert lz.zero_step_status(st, main) == (lz.ZERO_OK, 0)
+        res = oracle.zero2_step(ref_plan, lambda kk, rr: g[rr].numpy()[
+            ref_plan.buckets[kk][0]:sum(ref_plan.buckets[kk])], *ref[:3], ref[3], ORC_HP, t)
+        ref = (res.master, res.m, res.v, res.params16)
+        pp.swap()
+        check_f32(f"step {t} master", f32np(pp.cur[0]), ref[0])
+        check_f32(f"step {t} v", f32np(pp.cur[2]), ref[2])
+        check_f16(f"step {t} downloaded params", h_params.numpy().view(np.uint16), ref[3])
+    lz.zero_sched_destroy(sch)
+
+
 def test_scheduler_refuses_a_slot_still_in_use():
     """With one slot, beginning bucket 1 while bucket 0 has been begun but not ended would drop
     bucket 0's fill: EINVAL. Rebinding in the middle of a bucket is refused too."""
