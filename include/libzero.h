@@ -384,20 +384,21 @@ zero_status zero_stage3_step_commit(const zero_plan* plan, const float* master_i
 /* ------------------------------------------------------------------------------------------
  * Compressed reduce-scatter payload. "ZeRO" (lastdictionary.com), main definition: extensions
  * compress the communication (ZeRO++). The pages give no format; this library's: each rank's
- * slice travels as int8 values with one fp32 scale per block of ZERO_Q8_BLOCK elements
+ * slice travels as 8-bit values with one fp32 scale per block of ZERO_Q8_BLOCK elements
  * (blocks counted from the slice's first element), and the owner accumulates q*scale with
  * fused multiply-adds:
  *   scale = amax/127 (binary32), q = round_half_even(x/scale) clamped to [-127, 127],
- *   a block with an inf or NaN gets scale NaN and q = 0 (so the owner sees the overflow).
+ *   a block with an inf or NaN gets scale NaN and q = 0 (so the owner sees the overflow);
+ *   q is stored as the unsigned byte q + 128 (offset binary, 1..255; 128 is q = 0).
  * ---------------------------------------------------------------------------------------- */
 #define ZERO_Q8_BLOCK 128
-#define ZERO_Q8_RECORD 132   /* bytes per block: 128 int8 values, then the fp32 scale */
+#define ZERO_Q8_RECORD 132   /* bytes per block: 128 bytes q + 128, then the fp32 scale */
 
 /* Bytes of the payload of n elements: ceil(n/128) records of 132 bytes. */
 #define ZERO_Q8_PAYLOAD_BYTES(n) ((((uint64_t)(n) + 127u) / 128u) * 132u)
 
-/* Quantize one rank's n fp16 gradients into its payload: record b holds q of elements
- * [128b, 128b+128) in bytes 0..127 (unused bytes of a short last block are 0) and the block's
+/* Quantize one rank's n fp16 gradients into its payload: record b holds q + 128 of elements
+ * [128b, 128b+128) in bytes 0..127 (unused bytes of a short last block are 128) and the block's
  * scale in bytes 128..131. Device memory; payload 4-byte aligned (16 for the bulk-copy path of
  * zero_step_fused_q8). Errors: ZERO_EINVAL (null, overlap), ZERO_EALIGN, ZERO_ECUDA. */
 zero_status zero_quantize_q8(uint64_t n, const uint16_t* grad, uint8_t* payload,

@@ -34,10 +34,15 @@ def _quant_dev(g_dev, off=0):
     return pay
 
 
+def _q_of(codes):
+    """Stored bytes (q + 128) -> q as int8."""
+    return (codes.astype(np.int16) - 128).astype(np.int8)
+
+
 def _split(pay, n):
     """Payload records -> (int8 values of the n elements, fp32 scale per block)."""
     rec = pay.cpu().numpy().reshape(-1, 132)
-    q = rec[:, :128].reshape(-1).view(np.int8)[:n]
+    q = _q_of(rec[:, :128].reshape(-1)[:n])
     sc = np.ascontiguousarray(rec[:, 128:]).view(np.float32).reshape(-1)
     return q, sc
 
@@ -66,10 +71,48 @@ def test_quantize_bit_exact(n, kind):
     q_ref, sc_ref = oracle.quant_q8(g.numpy())
     assert np.array_equal(q, q_ref)
     assert _same_scales(sc, sc_ref)
-    # a short last block's unused bytes are zero
+    # the stored bytes are q + 128; a short last block's unused bytes hold q = 0
     tail = n % 128
     if tail:
-        assert not pay.cpu().numpy().reshape(-1, 132)[-1, tail:128].any()
+        assert (pay.cpu().numpy().reshape(-1, 132)[-1, tail:128] == 128).all()
+
+
+def _near_tie_blocks(nblocks, seed):
+    """Blocks of fp16 values that divide by their block's scale to within 2^-12 of a
+    half-integer, some exactly onto one: the rounding decisions the quantizer must take as the
+    IEEE quotient does. Each block's first value is its max |x|. Selection only: the expected
+    bytes come from the oracle."""
+    rng = np.random.default_rng(seed)
+    pos = np.arange(1, 0x7c00, dtype=np.uint16).view(np.float16)   # positive finite fp16
+    out = []
+    while len(out) < nblocks:
+        amax = pos[rng.integers(0x0400, 0x7c00 - 1)]
+        s = np.float32(amax) / np.float32(127)
+        cand = pos[pos <= amax]
+        y = cand.astype(np.float32) / s
+        near = cand[np.abs(y - np.floor(y) - np.float32(0.5)) < 2.0 ** -12]
+        if near.size < 4:
+            continue
+        blk = near[rng.integers(0, near.size, 127)]
+        blk = np.where(rng.random(127) < 0.5, -blk, blk).astype(np.float16)
+        out.append(np.concatenate([[amax], blk]).astype(np.float16))
+    return np.concatenate(out)
+
+
+@pytest.mark.parametrize("off", [0, 1])
+def test_quantize_near_ties_bit_exact(off):
+    """Quotients at and next to half-integers (where a quotient formed by a reciprocal could
+    round the other way) give the oracle's bytes, 16-byte aligned and not."""
+    g = torch.from_numpy(_near_tie_blocks(600, seed=31 + off))
+    n = g.numel() - 5                                   # and a short last block
+    gbig = torch.zeros(g.numel() + 8, dtype=torch.float16, device=DEV)
+    gbig[off:off + n] = g[:n].to(DEV)
+    pay = _quant_dev(gbig[off:off + n])
+    torch.cuda.synchronize()
+    q, sc = _split(pay, n)
+    q_ref, sc_ref = oracle.quant_q8(g[:n].numpy())
+    assert np.array_equal(q, q_ref)
+    assert _same_scales(sc, sc_ref)
 
 
 @pytest.mark.parametrize("nd", [1, 2, 3, 8, 16, 25, 64])
@@ -174,7 +217,7 @@ def test_7p5b_shard_view_q8_sampled():
     lz.zero_step_commit(S, *cur, *nxt, out, st)
     torch.cuda.synchronize()
     assert status_flags(st) == 0
-    gq = [p[qpos].cpu().numpy().view(np.int8) for p in pays]
+    gq = [_q_of(p[qpos].cpu().numpy()) for p in pays]
     gs = [np.ascontiguousarray(p[spos].cpu().numpy()).view(np.float32).reshape(-1) for p in pays]
     skipped, w, mm, vv, p = oracle.step_q8_gathered(gq, gs, w0, m0, v0, ORC_HP, 1)
     assert not skipped
