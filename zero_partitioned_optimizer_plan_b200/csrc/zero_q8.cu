@@ -305,12 +305,16 @@ __device__ void produce_q8(const FusedQ8Args& p, uint64_t* full, uint64_t* empty
     }
 }
 
-template <int W, int E, bool kDC>
+// kFixedRow: the rank loop steps from one rank's records to the next by the compile-time kRow
+// (immediate load offsets) or by the launch's p.row (the same value, at run time); which is
+// faster depends on Nd (see pick_variant_q8).
+template <int W, int E, bool kDC, bool kFixedRow>
 __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
     fused_q8_tma_kernel(const __grid_constant__ FusedQ8Args p) {
     static_assert(E == 4 || E == 8, "a thread's values sit in one record");
     // bytes of one rank's run of records in a stage (the launcher's p.row, checked below)
     constexpr uint32_t kRow = (32u * W * E / kQB) * kRec;
+    const uint32_t row = kFixedRow ? kRow : p.row;
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
@@ -357,11 +361,10 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
 #pragma unroll
                 for (int k = 0; k < P; ++k) ap[k] = f2_pack(acc[2 * k], acc[2 * k + 1]);
                 const uint64_t nbias = f2_pack(-8388736.0f, -8388736.0f);   // -(2^23 + 128)
-                // rank r's record sits kRow bytes after rank r-1's: the unrolled loads take
-                // immediate offsets
+                // rank r's record sits `row` bytes after rank r-1's
 #pragma unroll(16 / E)
                 for (uint32_t r = 0; r < nr; ++r) {
-                    const uint8_t* rec = rec0 + (size_t)r * kRow;
+                    const uint8_t* rec = rec0 + (size_t)r * row;
                     const float sc = *reinterpret_cast<const float*>(rec + kQB);
                     const uint64_t ss = f2_pack(sc, sc);
 #pragma unroll
@@ -436,14 +439,22 @@ __global__ void __launch_bounds__(256) fused_q8_plain_kernel(const __grid_consta
 // packed bias removal with scalar fused multiply-adds (5.0), explicit 32-bit shared loads (5.3),
 // inline byte permutes into register pairs (5.46, the same as the compiler's 5.46); dropping the
 // sign-bit flip of signed bytes (offset-binary bytes, now the format) took it to 5.57.
+// The record stride as a compile-time constant against the launch's value, flat 2^28, same box,
+// two passes each (TB/s): Nd = 2 6.43 / 6.34, 4 6.22 / 6.55, 8 6.16 / 6.72, 16 6.68 / 6.84,
+// 32 6.45 / 5.85, 64 5.54 / 4.98; so the run-time stride from Nd = 4 to 16.
 struct VariantQ8 {
     int warps;
     int elems;           // values per consumer thread and tile
     int target_stages;
+    bool fixed_row;      // compile-time record stride in the rank loop
 };
 
 VariantQ8 pick_variant_q8(int nd) {
-    VariantQ8 v = nd <= 16 ? VariantQ8{24, 4, 2} : VariantQ8{16, 4, 2};
+    VariantQ8 v = nd <= 16 ? VariantQ8{24, 4, 2, true} : VariantQ8{16, 4, 2, true};
+    v.fixed_row = nd < 4 || nd > 16;
+#ifdef ZK_Q8_FIXED_ROW
+    v.fixed_row = ZK_Q8_FIXED_ROW;
+#endif
 #ifdef ZK_Q8_WARPS
     v.warps = ZK_Q8_WARPS;
 #endif
@@ -563,9 +574,13 @@ cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,
     // the instantiated shapes: (warps, values per thread) with 32 * warps * values a multiple
     // of 512, so that a tile is a whole number of 4-record runs
 #define ZK_Q8_CASE(WW, EE)                                                                  \
-    if (sh.warps == WW && elems == EE)                                                     \
-        return ad ? launch_pipe(fused_q8_tma_kernel<WW, EE, true>, p, sh, stream)          \
-                  : launch_pipe(fused_q8_tma_kernel<WW, EE, false>, p, sh, stream)
+    if (sh.warps == WW && elems == EE) {                                                   \
+        if (var.fixed_row)                                                                 \
+            return ad ? launch_pipe(fused_q8_tma_kernel<WW, EE, true, true>, p, sh, stream) \
+                      : launch_pipe(fused_q8_tma_kernel<WW, EE, false, true>, p, sh, stream); \
+        return ad ? launch_pipe(fused_q8_tma_kernel<WW, EE, true, false>, p, sh, stream)   \
+                  : launch_pipe(fused_q8_tma_kernel<WW, EE, false, false>, p, sh, stream); \
+    }
     ZK_Q8_CASE(8, 4);
     ZK_Q8_CASE(12, 4);
     ZK_Q8_CASE(16, 4);
