@@ -375,6 +375,9 @@ class Workload:
         dominant kernel's launches. grads: the step's inputs (as inputs() lists them) when
         they are not the workload's own buffers."""
         lz = self.lz
+        if grads is None and len(self.ranges) > 1:   # per-bucket calls, marshalled once
+            self._step_prepared(t, status, ev)
+            return
         if self.payload == "q8":
             pays = grads or self.inputs()
             nd = self.nd
@@ -392,9 +395,6 @@ class Workload:
                 ev[1].record()
             lz.zero_step_commit(self.n, *self.cur, *self.nxt, self.params, status)
             self.cur, self.nxt = self.nxt, self.cur
-            return
-        if grads is None and len(self.ranges) > 1:   # per-bucket calls, marshalled once
-            self._step_prepared(t, status, ev)
             return
         grads = grads or self.grads
         if ev is not None:
@@ -414,15 +414,21 @@ class Workload:
 
 
 def _step_prepared(self, t, status, ev=None):
-    """The per-bucket calls of a step as one zero_step_fused_ranges call, its range descriptors
-    marshalled once per ping-pong direction (a step's host cost is then one entry plus the
-    launches, which matters for 1 MiB buckets)."""
+    """The per-bucket calls of a step as one zero_step_fused_ranges (int8 payloads:
+    zero_step_fused_q8_ranges) call, its range descriptors marshalled once per ping-pong
+    direction (a step's host cost is then one entry plus the launches, which matters for 1 MiB
+    buckets)."""
     lz, torch = self.lz, self.torch
     d = 0 if self.cur[0].data_ptr() == self.state_a0 else 1
     if self.prepared[d] is None:
-        self.prepared[d] = lz.PreparedStepRanges(self.nd, [
-            (hi - lo, [g[lo:hi] for g in self.grads], *[x[lo:hi] for x in self.cur],
-             *[x[lo:hi] for x in self.nxt], self.params[lo:hi]) for lo, hi in self.ranges])
+        nd = self.nd
+        if self.payload == "q8":    # range i's payloads: self.q[i * nd:(i + 1) * nd]
+            ins = [self.q[i * nd:(i + 1) * nd] for i in range(len(self.ranges))]
+        else:
+            ins = [[g[lo:hi] for g in self.grads] for lo, hi in self.ranges]
+        self.prepared[d] = lz.PreparedStepRanges(nd, [
+            (hi - lo, x, *[y[lo:hi] for y in self.cur], *[y[lo:hi] for y in self.nxt],
+             self.params[lo:hi]) for (lo, hi), x in zip(self.ranges, ins)], self.payload)
     sh = lz.stream_handle(torch.cuda.current_stream())
     if ev is not None:
         ev[0].record()

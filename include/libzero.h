@@ -416,6 +416,30 @@ zero_status zero_step_fused_q8(uint64_t n, int nd, const uint8_t* const* rank_pa
                                uint16_t* param_out, const zero_adam_hparams* hp, int64_t step,
                                uint32_t* d_status, zero_stream_t stream);
 
+/* The int8 calls of one step over several ranges as one call, as zero_step_fused_ranges is for
+ * zero_step_fused: ranges[i] describes what zero_step_fused_q8 takes for range i (rank_payload:
+ * a host array of nd device pointers, each to that range's records). Every range is checked
+ * before anything is launched; then the ranges are launched in order, exactly as `count`
+ * zero_step_fused_q8 calls on `stream` would be. overlap != 0 declares them mutually
+ * independent (not checked); a region already open on the stream is joined. Errors: ZERO_EINVAL
+ * (count < 0, null ranges, and anything zero_step_fused_q8 rejects for a range), ZERO_EALIGN,
+ * ZERO_ECUDA (ranges before the failing one may have been launched). */
+typedef struct {
+    uint64_t n;
+    const uint8_t* const* rank_payload;
+    const float* master_in;
+    const float* m_in;
+    const float* v_in;
+    float* master_out;
+    float* m_out;
+    float* v_out;
+    uint16_t* param_out;
+} zero_fused_q8_range;
+
+zero_status zero_step_fused_q8_ranges(int nd, int count, const zero_fused_q8_range* ranges,
+                                      const zero_adam_hparams* hp, int64_t step,
+                                      uint32_t* d_status, int overlap, zero_stream_t stream);
+
 /* zero_step_fused_q8 with the step's constants read from device memory (d_consts: a
  * zero_adam_consts, 4-byte aligned, e.g. written by zero_scaler_prepare), as
  * zero_step_fused_dc: the call can be captured in a CUDA graph and replayed for every step,

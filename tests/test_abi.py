@@ -446,3 +446,24 @@ def test_step_fused_ranges_rejects_before_launching():
     assert lz.zero_kernel_launches() == before
     lz.zero_step_fused_ranges(2, [], HP, 1, A + 130 * MB, True, 0)     # nothing to do
     assert lz.zero_kernel_launches() == before
+
+
+def test_step_fused_q8_ranges_rejects_before_launching():
+    pays = [A + i * MB for i in range(2)]
+    good = (1000, pays, A + 100 * MB, A + 101 * MB, A + 102 * MB, A + 110 * MB, A + 111 * MB,
+            A + 112 * MB, A + 120 * MB)
+    pay_on_out = (1000, [A + 210 * MB, pays[1]], A + 200 * MB, A + 201 * MB, A + 202 * MB,
+                  A + 210 * MB, A + 211 * MB, A + 212 * MB, A + 220 * MB)   # payload == master_out
+    before = lz.zero_kernel_launches()
+    for ranges, kw, code in [([good, pay_on_out], {}, lz.ZERO_EINVAL),
+                             ([good], dict(step=0), lz.ZERO_EINVAL),
+                             ([good[:1] + ([A, A + MB + 2],) + good[2:]], {}, lz.ZERO_EALIGN),
+                             ([good[:1] + ([A, 0],) + good[2:]], {}, lz.ZERO_EINVAL)]:
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_step_fused_q8_ranges(2, ranges, HP, kw.get("step", 1), A + 130 * MB, True, 0)
+        assert e.value.code == code
+    assert lz.zero_kernel_launches() == before
+    lz.zero_step_fused_q8_ranges(2, [], HP, 1, A + 130 * MB, True, 0)   # nothing to do
+    assert lz.zero_kernel_launches() == before
+    with pytest.raises(ValueError):
+        lz.PreparedStepRanges(2, [good], "bf16")

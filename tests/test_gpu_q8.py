@@ -342,3 +342,57 @@ def test_q8_graph_with_device_scaler():
     assert (s.scale, s.good_steps, s.next_step, s.skipped_steps) == \
         (np.float32(sc.scale), sc.good_steps, sc.next_step, sc.skipped_steps)
     del graphs
+
+
+@pytest.mark.parametrize("nd", [8, 64])
+def test_step_fused_q8_ranges_vs_oracle(nd):
+    """zero_step_fused_q8_ranges over buckets of every kernel shape (one above 4 tiles per SM,
+    small-call ones, one under 4096 elements for the plain kernel), each bucket's payload
+    quantized from its own range: the same bits as per-bucket zero_step_fused_q8 calls in a
+    region, and the oracle's per-bucket owner steps (0 ulp)."""
+    sizes = [1_900_032, 3072 * 4, 3072 * 2 + 512, 1000]
+    n = sum(sizes) + 333
+    bounds, lo = [], 0
+    for sz in sizes + [333]:
+        bounds.append((lo, lo + sz))
+        lo += sz
+    bounds = bounds[::-1]                                   # backward order
+    g_cpu = [synth.grad_f16(n, 1e-2, seed=91, rank=r, step=1) for r in range(nd)]
+    g_dev = [g.to(DEV) for g in g_cpu]
+    pays = {}
+    for lo, hi in bounds:
+        pays[lo] = []
+        for g in g_dev:
+            pay = torch.empty(lz.q8_payload_bytes(hi - lo), dtype=torch.uint8, device=DEV)
+            lz.zero_quantize_q8(hi - lo, g[lo:hi], pay)
+            pays[lo].append(pay)
+    del g_dev
+    master, m, v = synth.state_warm(n, seed=92)
+    ins = [x.to(DEV) for x in (master, m, v)]
+    outs_a = [torch.empty_like(x) for x in ins]
+    outs_b = [torch.empty_like(x) for x in ins]
+    pa = torch.empty(n, dtype=torch.float16, device=DEV)
+    pb = torch.empty(n, dtype=torch.float16, device=DEV)
+    st = status_word()
+    lz.zero_step_fused_q8_ranges(nd, [
+        (hi - lo, pays[lo], *[x[lo:hi] for x in ins], *[x[lo:hi] for x in outs_a], pa[lo:hi])
+        for lo, hi in bounds], HP, 1, st)
+    with lz.overlap():
+        for lo, hi in bounds:
+            lz.zero_step_fused_q8(hi - lo, nd, pays[lo], *[x[lo:hi] for x in ins],
+                                  *[x[lo:hi] for x in outs_b], pb[lo:hi], HP, 1, st)
+    torch.cuda.synchronize()
+    assert status_flags(st) == 0
+    for a, b in list(zip(outs_a, outs_b)) + [(pa, pb)]:
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    w, mm, vv = master.numpy().copy(), m.numpy().copy(), v.numpy().copy()
+    p = np.empty(n, np.uint16)
+    for lo, hi in bounds:
+        ref = [oracle.quant_q8(g.numpy()[lo:hi]) for g in g_cpu]
+        skipped, w[lo:hi], mm[lo:hi], vv[lo:hi], p[lo:hi] = oracle.step_q8(
+            [q for q, _ in ref], [s for _, s in ref], w[lo:hi], mm[lo:hi], vv[lo:hi], ORC_HP, 1)
+        assert not skipped
+    check_f32("master", f32np(outs_a[0]), w, tol=0)
+    check_f32("m", f32np(outs_a[1]), mm, tol=0)
+    check_f32("v", f32np(outs_a[2]), vv, tol=0)
+    check_f16("params", f16np(pa), p, tol=0)

@@ -379,6 +379,35 @@ zero_status zero_step_fused_q8(uint64_t n, int nd, const uint8_t* const* rank_pa
                                              d_status, (cudaStream_t)stream));
 }
 
+zero_status zero_step_fused_q8_ranges(int nd, int count, const zero_fused_q8_range* ranges,
+                                      const zero_adam_hparams* hp, int64_t step,
+                                      uint32_t* d_status, int overlap, zero_stream_t stream) {
+    if (!zk::hparams_ok(hp) || step < 1 || count < 0 || (count > 0 && !ranges)) return ZERO_EINVAL;
+    for (int i = 0; i < count; ++i) {
+        const zero_fused_q8_range& r = ranges[i];
+        const zero_status st = check_fused_q8(r.n, nd, r.rank_payload, r.master_in, r.m_in,
+                                              r.v_in, r.master_out, r.m_out, r.v_out,
+                                              r.param_out, d_status);
+        if (st != ZERO_OK) return st;
+    }
+    if (!d_status) return ZERO_EINVAL;
+    const zk::AdamConsts a = zk::make_adam(hp, step);
+    const zk::MeanConsts mc = zk::make_mean(nd);
+    const cudaStream_t s = (cudaStream_t)stream;
+    // a region already open on the stream (the caller's) chains these calls as well
+    const bool opened = overlap && zero_overlap_begin(stream) == ZERO_OK;
+    cudaError_t e = cudaSuccess;
+    for (int i = 0; i < count && e == cudaSuccess; ++i) {
+        const zero_fused_q8_range& r = ranges[i];
+        if (r.n == 0) continue;
+        e = zk::launch_fused_q8(r.n, nd, r.rank_payload, r.master_in, r.m_in, r.v_in,
+                                r.master_out, r.m_out, r.v_out, r.param_out, a, nullptr, mc,
+                                d_status, s);
+    }
+    if (opened) zero_overlap_end(stream);
+    return zk::from_cuda(e);
+}
+
 zero_status zero_step_fused_q8_dc(uint64_t n, int nd, const uint8_t* const* rank_payload,
                                   const float* master_in, const float* m_in, const float* v_in,
                                   float* master_out, float* m_out, float* v_out,

@@ -441,7 +441,12 @@ __global__ void __launch_bounds__(256) fused_q8_plain_kernel(const __grid_consta
 // sign-bit flip of signed bytes (offset-binary bytes, now the format) took it to 5.57.
 // The record stride as a compile-time constant against the launch's value, flat 2^28, same box,
 // two passes each (TB/s): Nd = 2 6.43 / 6.34, 4 6.22 / 6.55, 8 6.16 / 6.72, 16 6.68 / 6.84,
-// 32 6.45 / 5.85, 64 5.54 / 4.98; so the run-time stride from Nd = 4 to 16.
+// 32 6.45 / 5.85, 64 5.54 / 4.98; so the run-time stride from Nd = 4 to 16. Above Nd = 48, 24
+// consumer warps again (four chunks of 16 ranks per tile): Nd = 64 5.60 against 5.52 TB/s with 16
+// warps, the 7.5B view 5.55 against 5.50 (two passes each); at Nd = 48 they lose (5.11 against
+// 5.24). A rank loop that issues the next four or eight ranks' shared loads before the current
+// ranks' arithmetic (explicit software pipelining) measured slower at every Nd (Nd = 64: 5.17 /
+// 5.41 against 5.48 TB/s).
 struct VariantQ8 {
     int warps;
     int elems;           // values per consumer thread and tile
@@ -450,7 +455,7 @@ struct VariantQ8 {
 };
 
 VariantQ8 pick_variant_q8(int nd) {
-    VariantQ8 v = nd <= 16 ? VariantQ8{24, 4, 2, true} : VariantQ8{16, 4, 2, true};
+    VariantQ8 v = nd <= 16 || nd > 48 ? VariantQ8{24, 4, 2, true} : VariantQ8{16, 4, 2, true};
     v.fixed_row = nd < 4 || nd > 16;
 #ifdef ZK_Q8_FIXED_ROW
     v.fixed_row = ZK_Q8_FIXED_ROW;
@@ -496,6 +501,21 @@ PipeShape q8_shape(int nd, int warps, int elems, int target_stages, size_t budge
     return sh;
 }
 
+// Grid of the quantizer (a grid-stride kernel of `threads` threads per block): the blocks its
+// work needs, at most `waves` full waves of resident blocks (a further, partial wave would run
+// the kernel's tail on part of the device).
+template <typename K>
+cudaError_t resident_grid(K kernel, const DevInfo& di, int threads, uint64_t blocks, int waves,
+                          unsigned* grid) {
+    int bps = 0;
+    cudaError_t e = pipe_blocks_per_sm(kernel, di.dev, threads, 0, &bps);
+    if (e != cudaSuccess) return e;
+    const uint64_t cap = (uint64_t)di.sms * (uint64_t)bps * (uint64_t)waves;
+    if (blocks > cap) blocks = cap;
+    *grid = (unsigned)(blocks ? blocks : 1);
+    return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, uint8_t* payload,
@@ -509,10 +529,12 @@ cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, uint8_t* payload,
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
     const uint64_t npairs = ((n + kQB - 1) / kQB + 1) / 2;   // two blocks per warp, 8 warps/CTA
-    uint64_t grid = (npairs + 7) / 8;
-    const uint64_t cap = (uint64_t)di.sms * 8;
-    if (grid > cap) grid = cap;
-    quant_q8_kernel<<<(unsigned)(grid ? grid : 1), 256, 0, stream>>>(p);
+    // two full waves of resident blocks: 0.64 of the peak against 0.63 with one and 0.60 with
+    // 8 blocks per SM (1.6 waves)
+    unsigned grid = 1;
+    e = resident_grid(quant_q8_kernel, di, 256, (npairs + 7) / 8, 2, &grid);
+    if (e != cudaSuccess) return e;
+    quant_q8_kernel<<<grid, 256, 0, stream>>>(p);
     count_launch();
     return cudaGetLastError();
 }

@@ -50,7 +50,7 @@ SYMBOLS = (
     "zero_scaler_update", "zero_quantize_q8", "zero_step_fused_q8", "zero_step_fused_q8_dc",
     "zero_overlap_begin", "zero_overlap_end",
     "zero_gather_params", "zero_stage3_step_fused", "zero_stage3_step_commit",
-    "zero_step_fused_ranges",
+    "zero_step_fused_ranges", "zero_step_fused_q8_ranges",
     "zero_sched_slot_elems", "zero_sched_create", "zero_sched_create_fused",
     "zero_sched_begin_bucket", "zero_sched_rebind_fused", "zero_sched_rebind_status",
     "zero_sched_end_bucket", "zero_sched_wait", "zero_sched_launches", "zero_sched_destroy",
@@ -102,6 +102,14 @@ class ScalerState(C.Structure):
 class FusedRange(C.Structure):
     """zero_fused_range: one range of a step for zero_step_fused_ranges."""
     _fields_ = [("n", C.c_uint64), ("rank_grads", C.POINTER(C.c_void_p)),
+                ("master_in", C.c_void_p), ("m_in", C.c_void_p), ("v_in", C.c_void_p),
+                ("master_out", C.c_void_p), ("m_out", C.c_void_p), ("v_out", C.c_void_p),
+                ("param_out", C.c_void_p)]
+
+
+class FusedQ8Range(C.Structure):
+    """zero_fused_q8_range: one range of a step for zero_step_fused_q8_ranges."""
+    _fields_ = [("n", C.c_uint64), ("rank_payload", C.POINTER(C.c_void_p)),
                 ("master_in", C.c_void_p), ("m_in", C.c_void_p), ("v_in", C.c_void_p),
                 ("master_out", C.c_void_p), ("m_out", C.c_void_p), ("v_out", C.c_void_p),
                 ("param_out", C.c_void_p)]
@@ -159,6 +167,7 @@ def _load():
     L.zero_scaler_prepare.argtypes = [vp, vp, i64, vp, vp, vp]
     L.zero_scaler_update.argtypes = [vp, P(ScalerParams), vp, vp]
     L.zero_step_fused_ranges.argtypes = [i32, i32, P(FusedRange), P(_HP), i64, vp, i32, vp]
+    L.zero_step_fused_q8_ranges.argtypes = [i32, i32, P(FusedQ8Range), P(_HP), i64, vp, i32, vp]
     L.zero_gather_params.argtypes = [vp, u64, u64, P(vp), vp, vp, vp]
     L.zero_stage3_step_fused.argtypes = [vp, u64, u64, P(vp), vp, vp, vp, vp, vp, vp, P(vp), P(_HP),
                                    i64, vp, vp]
@@ -322,31 +331,45 @@ def zero_step_fused(n: int, nd: int, rank_grads, master_in, m_in, v_in, master_o
 
 
 class PreparedStepRanges:
-    """zero_step_fused_ranges with its range descriptors marshalled once: each item of `ranges`
-    is (n, rank_grads, master_in, m_in, v_in, master_out, m_out, v_out, param_out) as
-    zero_step_fused takes them. Calling it launches every range of the step in one C call."""
+    """zero_step_fused_ranges (payload "fp16") or zero_step_fused_q8_ranges (payload "q8") with
+    its range descriptors marshalled once: each item of `ranges` is (n, rank inputs, master_in,
+    m_in, v_in, master_out, m_out, v_out, param_out) as zero_step_fused / zero_step_fused_q8
+    take them (rank inputs: the ranks' fp16 gradients, or their int8 payloads). Calling it
+    launches every range of the step in one C call."""
 
-    def __init__(self, nd: int, ranges):
+    def __init__(self, nd: int, ranges, payload: str = "fp16"):
+        if payload not in ("fp16", "q8"):
+            raise ValueError(f"payload {payload!r}")
         self.nd = nd
-        self._grad_arrays = [_ptr_array(r[1], 2) for r in ranges]   # kept alive
-        arr = (FusedRange * max(len(ranges), 1))()
-        for i, (r, g) in enumerate(zip(ranges, self._grad_arrays)):
-            arr[i] = FusedRange(r[0], C.cast(g, C.POINTER(C.c_void_p)), *[
+        q8 = payload == "q8"
+        self._name = "zero_step_fused_q8_ranges" if q8 else "zero_step_fused_ranges"
+        self._fn = getattr(_lib, self._name)
+        Range = FusedQ8Range if q8 else FusedRange
+        self._in_arrays = [_ptr_array(r[1], 1 if q8 else 2) for r in ranges]   # kept alive
+        arr = (Range * max(len(ranges), 1))()
+        for i, (r, g) in enumerate(zip(ranges, self._in_arrays)):
+            arr[i] = Range(r[0], C.cast(g, C.POINTER(C.c_void_p)), *[
                 _ptr(x, 4) for x in r[2:8]], _ptr(r[8], 2))
         self._arr = arr
         self.count = len(ranges)
 
     def __call__(self, hp_ref, step: int, d_status: int, overlap: bool, stream: int):
-        code = _lib.zero_step_fused_ranges(self.nd, self.count, self._arr, hp_ref, step, d_status,
-                                           1 if overlap else 0, stream)
+        code = self._fn(self.nd, self.count, self._arr, hp_ref, step, d_status,
+                        1 if overlap else 0, stream)
         if code:
-            raise ZeroError(code, "zero_step_fused_ranges")
+            raise ZeroError(code, self._name)
 
 
 def zero_step_fused_ranges(nd: int, ranges, hp: AdamHP, step: int, d_status, overlap=True,
                            stream=None):
     PreparedStepRanges(nd, ranges)(hparams_ref(hp), step, _ptr(d_status, 4), overlap,
                                    _stream(stream))
+
+
+def zero_step_fused_q8_ranges(nd: int, ranges, hp: AdamHP, step: int, d_status, overlap=True,
+                              stream=None):
+    PreparedStepRanges(nd, ranges, "q8")(hparams_ref(hp), step, _ptr(d_status, 4), overlap,
+                                         _stream(stream))
 
 
 def hparams_ref(hp: AdamHP):
