@@ -60,6 +60,7 @@ FALLBACK_HBM_GBS = 6650.0
 CSRC = os.path.join(ROOT, "zero_partitioned_optimizer_plan_b200", "csrc")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 METRIC = "fused ZeRO shard step params/sec"
+L2_BYTES = 126 * 1024 * 1024    # B200 L2
 
 
 def parse():
@@ -68,8 +69,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["gpt2_small", "shard_7p5b", "flat", "zero2_1p3b",
-                                           "zero2_gpt2_small", "zero3_gpt2_small",
+    ap.add_argument("--workload", choices=["tiny", "gpt2_small", "shard_7p5b", "flat",
+                                           "zero2_1p3b", "zero2_gpt2_small", "zero3_gpt2_small",
                                            "zero3_1p3b"],
                     default="zero2_1p3b")
     ap.add_argument("--nd", type=int, default=None)
@@ -87,6 +88,9 @@ def parse():
                     help="stage-2 workloads: the bucket scheduler launches the fused step per "
                          "bucket (zero_sched_create_fused), or the reduce-scatter per bucket "
                          "and then the owner updates")
+    ap.add_argument("--l2", choices=["warm", "flushed"], default="warm",
+                    help="flushed: write a buffer larger than L2 between timed steps and time each "
+                         "step on its own (for the L2-resident tiny workload)")
     ap.add_argument("--no-sweep", action="store_true",
                     help="leave out the bucket / Nd sweep of the default line")
     ap.add_argument("--sweep-steps", type=int, default=None)
@@ -109,11 +113,12 @@ def workload_config(args) -> dict:
     """The workload's name and sizes as both arms report them (no device needed)."""
     from zero_partitioned_optimizer_plan_b200 import synth
     kind = args.workload
-    if kind == "gpt2_small":
-        nd = args.nd or 8
-        numels = synth.gpt2_small_list()
-        cfg = {"workload": "gpt2_small_stage1", "psi": sum(numels), "nd": nd, "stage": 1,
-               "calls_per_step": 1, "tensors": len(numels)}
+    if kind in ("gpt2_small", "tiny"):
+        nd = args.nd or (8 if kind == "gpt2_small" else 4)
+        numels = synth.gpt2_small_list() if kind == "gpt2_small" else synth.TINY_LIST
+        cfg = {"workload": kind + "_stage1" if kind == "tiny" else "gpt2_small_stage1",
+               "psi": sum(numels), "nd": nd, "stage": 1, "calls_per_step": 1,
+               "tensors": len(numels)}
     elif kind == "shard_7p5b":
         nd = args.nd or 64
         total = 7_500_000_000
@@ -169,9 +174,10 @@ class Workload:
         self.kind = kind
         self.e2e = None          # a workload-specific end-to-end leg (stage 2 fused)
         self.kernel_times = None  # per-step dominant-kernel time, when not the ev pair's
-        if kind == "gpt2_small":
-            nd = args.nd or 8
-            numels = synth.gpt2_small_list()
+        if kind in ("gpt2_small", "tiny"):
+            tiny = kind == "tiny"
+            nd = args.nd or (4 if tiny else 8)
+            numels = synth.TINY_LIST if tiny else synth.gpt2_small_list()
             pl = lz.zero_plan_create(numels, nd, 1, 0)
             psi, psi_p, S, nb = lz.zero_plan_info(pl)
             self.nd, self.n, self.psi = nd, psi_p, psi
@@ -179,8 +185,11 @@ class Workload:
             self.grads = []
             for r in range(nd):
                 g = torch.zeros(psi_p, dtype=torch.float16, device=dev)
-                synth.grad_f16(psi, 1e-3, seed=0, rank=r, step=1, spike_frac=0.01,
-                               spike_scale=100.0, out=g[:psi])
+                if tiny:     # the tiny stage-1 case: N(0, 0.01^2) gradients, no spikes
+                    synth.grad_f16(psi, 0.01, seed=0, rank=r, step=1, out=g[:psi])
+                else:
+                    synth.grad_f16(psi, 1e-3, seed=0, rank=r, step=1, spike_frac=0.01,
+                                   spike_scale=100.0, out=g[:psi])
                 self.grads.append(g)
             master, m, v = synth.state_small(psi_p, seed=0, device=dev)
             self.params = torch.empty(psi_p, dtype=torch.float16, device=dev)
@@ -1233,6 +1242,11 @@ def run_ours(args):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flushed = args.l2 == "flushed"
+    if flushed:   # a buffer twice the L2 written between steps; each step timed on its own
+        flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+        sevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(K)]
     sampler = ClockSampler(local)
     barrier()
     torch.cuda.synchronize()
@@ -1240,7 +1254,12 @@ def run_ours(args):
     with sampler:
         start.record()
         for i in range(K):
+            if flushed:
+                flush_buf.fill_(i)
+                sevs[i][0].record()
             wl.step(W + i + 1, status[W + i:W + i + 1], ev=evs[i])
+            if flushed:
+                sevs[i][1].record()
         end.record()
         torch.cuda.synchronize()
     launches = lz.zero_kernel_launches() - launches0
@@ -1249,7 +1268,7 @@ def run_ours(args):
         if int(wl.g_flags.item()) != 0:
             raise RuntimeError(f"unexpected status flags in the timed steps: {wl.g_flags.item()}")
     barrier()
-    ms = start.elapsed_time(end)
+    ms = sum(a.elapsed_time(b) for a, b in sevs) if flushed else start.elapsed_time(end)
     kernel_ms = wl.kernel_times(evs) if wl.kernel_times else [a.elapsed_time(b) for a, b in evs]
     flags = status.cpu()
     if int((flags != 0).sum()):
@@ -1321,7 +1340,14 @@ def run_ours(args):
             cfg["cuda_graph"] = "one replay per step; kernel time includes the commit"
             if args.dynamic_scale:
                 cfg["loss_scale"] = "dynamic, on the device (scaler kernels inside the graph)"
-        cfg.update({"l2": "no flush: every step streams several GB, far above L2",
+        if flushed:
+            l2 = (f"flushed: {2 * L2_BYTES >> 20} MiB written between steps, each step timed "
+                  "on its own (the flush outside the timed steps)")
+        elif bytes0 > 4 * L2_BYTES:
+            l2 = "no flush: every step streams several GB, far above L2"
+        else:
+            l2 = "warm: the step's buffers stay in L2 across steps (no flush)"
+        cfg.update({"l2": l2,
                     "bytes_per_step": bytes0, "parallelism": f"replicas{ws}",
                     "hbm_gbs": bytes0 / (ms_per_step / 1e3) / 1e9})
         if sweep is not None:
