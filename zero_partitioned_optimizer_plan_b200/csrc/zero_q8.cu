@@ -530,7 +530,8 @@ cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, uint8_t* payload,
     if (e != cudaSuccess) return e;
     const uint64_t npairs = ((n + kQB - 1) / kQB + 1) / 2;   // two blocks per warp, 8 warps/CTA
     // two full waves of resident blocks: 0.64 of the peak against 0.63 with one and 0.60 with
-    // 8 blocks per SM (1.6 waves)
+    // 8 blocks per SM (1.6 waves). Not better: 6 or 8 resident blocks per SM by launch bounds
+    // (0.58 / 0.57, registers spilled), a second block pair's load in flight (0.57).
     unsigned grid = 1;
     e = resident_grid(quant_q8_kernel, di, 256, (npairs + 7) / 8, 2, &grid);
     if (e != cudaSuccess) return e;
