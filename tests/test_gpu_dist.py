@@ -31,7 +31,7 @@ def _case(numels):
     return psi, grad, master, m, v, torch
 
 
-def _worker(port, numels, bucket, out, peer=False):
+def _worker(port, numels, bucket, out, peer=False, payload="fp16"):
     import datetime
     import torch
     import torch.distributed as dist
@@ -57,7 +57,7 @@ def _worker(port, numels, bucket, out, peer=False):
             step = DistZeroStep(psi, bucket, peers=peers)
             flag = step.step(peers.local, st_in, st_out, params, lz.AdamHP(), 1, status)
         else:
-            step = DistZeroStep(psi, bucket)
+            step = DistZeroStep(psi, bucket, payload=payload)
             flag = step.step(grad.to(dev), st_in, st_out, params, lz.AdamHP(), 1, status)
         torch.cuda.synchronize()
         out.put((int(flag.item()), int(status.item()), [x.cpu().numpy() for x in st_out],
@@ -92,3 +92,36 @@ def test_distributed_step_one_rank_nccl(bucket, peer):
         d = oracle.ulp_diff_f32(got, want)
         assert int(d.max()) <= 2, name
     assert int(oracle.ulp_diff_f16(params, ref.params16).max()) <= 1
+
+
+@pytest.mark.parametrize("bucket", [0, 3000])
+def test_distributed_step_int8_payload_one_rank_nccl(bucket):
+    """payload="q8" on one NCCL rank: the library's quantizer fills the send buffer, the
+    all-to-all moves the records, the library's int8 step runs on the received payloads;
+    against the oracle's quantizer and int8 step per bucket (0 ulp)."""
+    import oracle
+    from zero_partitioned_optimizer_plan_b200.dist import bucket_ranges
+    numels = [1000, 37, 4099, 12345]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_worker, args=(_free_port(), numels, bucket, q, False, "q8"))
+    p.start()
+    try:
+        flag, status, shard, params = q.get(timeout=240)
+    finally:
+        p.join(60)
+        if p.exitcode is None:
+            p.kill()
+    assert p.exitcode == 0
+    psi, grad, master, m, v, _ = _case(numels)
+    w, mm, vv = master.numpy().copy(), m.numpy().copy(), v.numpy().copy()
+    p16 = oracle.f2h(master.numpy())
+    for lo, hi in bucket_ranges(psi, bucket):
+        qq, sc = oracle.quant_q8(grad.numpy()[lo:hi])
+        skipped, w[lo:hi], mm[lo:hi], vv[lo:hi], p16[lo:hi] = oracle.step_q8(
+            [qq], [sc], w[lo:hi], mm[lo:hi], vv[lo:hi], oracle.AdamHP(), 1)
+        assert not skipped
+    assert (flag, status) == (0, 0)
+    for name, got, want in zip(("master", "m", "v"), shard, (w, mm, vv)):
+        assert int(oracle.ulp_diff_f32(got, want).max()) == 0, name
+    assert int(oracle.ulp_diff_f16(params, p16).max()) == 0

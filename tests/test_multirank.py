@@ -118,6 +118,28 @@ def test_failed_rank_is_detected_on_the_host(mode):
 # the distributed step (dist.py): its exchange on CPU processes over gloo, with the owner's
 # fused step and commit done by the oracle (the library needs a GPU)
 # ---------------------------------------------------------------------------------------------
+def _pack_q8(q, scales):
+    """The library's payload records (128 bytes q + 128, then the fp32 scale; a short last
+    block padded with q = 0) from the oracle's logical q and scales."""
+    import numpy as np
+    nb = scales.size
+    rec = np.zeros((nb, 132), np.uint8)
+    rec[:, :128] = 128
+    codes = (q.astype(np.int16) + 128).astype(np.uint8)
+    for b in range(nb):
+        blk = codes[128 * b:128 * (b + 1)]
+        rec[b, :blk.size] = blk
+    rec[:, 128:] = np.ascontiguousarray(scales, np.float32).view(np.uint8).reshape(nb, 4)
+    return rec.reshape(-1)
+
+
+def _unpack_q8(payload, n):
+    import numpy as np
+    rec = np.asarray(payload).reshape(-1, 132)
+    q = (rec[:, :128].astype(np.int16) - 128).astype(np.int8).reshape(-1)[:n]
+    return q, np.ascontiguousarray(rec[:, 128:]).view(np.float32).reshape(-1)
+
+
 class _OracleCompute:
     def __init__(self, fail=False):
         self.fail = fail     # report a kernel timeout (as a library kernel that gave up would)
@@ -138,6 +160,26 @@ class _OracleCompute:
             dst.copy_(__import__("torch").from_numpy(np.ascontiguousarray(src)))
         params.view(__import__("torch").int16).copy_(
             __import__("torch").from_numpy(np.ascontiguousarray(p16).view(np.int16)))
+
+    def quantize(self, n, grad, payload):
+        import torch
+        import oracle
+        q, sc = oracle.quant_q8(grad.numpy())
+        payload.copy_(torch.from_numpy(_pack_q8(q, sc)))
+
+    def fused_q8(self, n, payloads, state_in, state_out, params, hp, t, status):
+        import numpy as np
+        import torch
+        import oracle
+        qs, scs = zip(*[_unpack_q8(p.numpy(), n) for p in payloads])
+        skipped, w, m, v, p16 = oracle.step_q8(list(qs), list(scs),
+                                               *(x.numpy() for x in state_in), hp, t)
+        if skipped:
+            status |= 1
+            return
+        for dst, src in zip(state_out, (w, m, v)):
+            dst.copy_(torch.from_numpy(np.ascontiguousarray(src)))
+        params.view(torch.int16).copy_(torch.from_numpy(np.ascontiguousarray(p16).view(np.int16)))
 
     def commit(self, n, state_in, state_out, params, status):
         import numpy as np
@@ -168,7 +210,7 @@ def _dist_case(numels, ws, bad_rank):
     return psi_p, grads, master, m, v
 
 
-def _worker_dist(rank, ws, port, numels, bucket, bad_rank, out):
+def _worker_dist(rank, ws, port, numels, bucket, bad_rank, out, payload="fp16"):
     import datetime
     import torch
     import torch.distributed as dist
@@ -187,7 +229,7 @@ def _worker_dist(rank, ws, port, numels, bucket, bad_rank, out):
         params[rank * S:(rank + 1) * S] = torch.from_numpy(
             oracle.f2h(st_in[0].numpy()).view("float16"))
         status = torch.zeros(1, dtype=torch.int32)
-        step = DistZeroStep(psi_p, bucket, compute=_OracleCompute())
+        step = DistZeroStep(psi_p, bucket, compute=_OracleCompute(), payload=payload)
         flag = step.step(grads[rank], st_in, st_out, params, oracle.AdamHP(), 1, status)
         out.put((rank, int(flag.item()), int(status.item()), [x.numpy() for x in st_out],
                  params.numpy().view("uint16")))
@@ -391,3 +433,58 @@ def test_dist_bucket_map_matches_the_plan():
             assert sum(parts) == hi - lo
             owned = [q for q in range(nd) if parts[q] > 0]
             assert owned == list(range(lo // S, (hi - 1) // S + 1))
+
+
+@pytest.mark.parametrize("ws,bucket,bad_rank", [(2, 0, -1), (3, 2500, -1), (3, 2500, 2)])
+def test_distributed_step_int8_payload_gloo(ws, bucket, bad_rank):
+    """payload="q8": every rank quantizes its slice of each bucket for each owner (records
+    counted from the owner's part), the all-to-all moves the records, the owner steps from the
+    Nd payloads. Against the oracle's quantizer and int8 owner step over the same
+    (bucket, owner) parts, bit for bit; an inf in one rank's gradient skips the step on every
+    rank."""
+    import numpy as np
+    import oracle
+    from zero_partitioned_optimizer_plan_b200.dist import bucket_ranges
+    numels = [1000, 37, 4099, 12345]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_dist,
+                         args=(r, ws, port, numels, bucket, bad_rank, q, "q8"))
+             for r in range(ws)]
+    for p in procs:
+        p.start()
+    try:
+        res = sorted((q.get(timeout=240) for _ in range(ws)), key=lambda x: x[0])
+    finally:
+        for p in procs:
+            p.join(60)
+            if p.exitcode is None:
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    psi_p, grads, master, m, v = _dist_case(numels, ws, bad_rank)
+    S = psi_p // ws
+    w, mm, vv = master.numpy().copy(), m.numpy().copy(), v.numpy().copy()
+    p16 = oracle.f2h(master.numpy())
+    skipped = False
+    for lo, hi in bucket_ranges(psi_p, bucket):
+        for o in range(ws):
+            a, b = max(lo, o * S), min(hi, (o + 1) * S)
+            if a >= b:
+                continue
+            pay = [oracle.quant_q8(g.numpy()[a:b]) for g in grads]
+            sk, wn, mn, vn, pn = oracle.step_q8([x for x, _ in pay], [s for _, s in pay],
+                                                w[a:b], mm[a:b], vv[a:b], oracle.AdamHP(), 1)
+            skipped |= sk
+            if not sk:
+                w[a:b], mm[a:b], vv[a:b], p16[a:b] = wn, mn, vn, pn
+    if skipped:
+        w, mm, vv = master.numpy(), m.numpy(), v.numpy()
+        p16 = oracle.f2h(master.numpy())
+    assert skipped == (bad_rank >= 0)
+    for rank, flag, status, shard, params in res:
+        assert flag == (1 if skipped else 0)
+        assert bool(status & 2) == skipped
+        for got, want in zip(shard, (w, mm, vv)):
+            assert np.array_equal(got.view(np.uint32), want[rank * S:(rank + 1) * S].view(np.uint32))
+        assert np.array_equal(params, p16)

@@ -42,8 +42,18 @@ like any collective) guarantees that every rank has produced the bucket before a
 it; the all-reduce of the void bits at the end of the step is the barrier after which no
 owner reads this step's gradients any more, so the next backward pass may overwrite them.
 
+Compressed payload (``payload="q8"``, all-to-all form). "ZeRO" (lastdictionary.com), main
+definition: extensions compress the communication (ZeRO++). Each rank quantizes its slice of
+a bucket for each owner with the library's zero_quantize_q8 (records of 128 bytes q + 128 and an
+fp32 scale, blocks counted from the start of the owner's part), the all-to-all moves those
+records (132/128 bytes per value instead of 2), and the owner runs zero_step_fused_q8 over the
+Nd received payloads in rank order. Each owner's segment is padded to a multiple of 16 bytes
+so that every received payload starts 16-byte aligned (the library's bulk-copy path). Send
+buffers are double-buffered like the receive buffers: bucket k+2 is quantized into bucket k's
+send buffer only after the current stream has waited for bucket k's exchange.
+
 The collectives are torch.distributed calls (NCCL on GPUs, gloo on CPUs); the arithmetic is the
-library's. ``compute`` replaces the two library calls (the tests run the exchange on CPU
+library's. ``compute`` replaces the library calls (the tests run the exchange on CPU
 processes with another implementation of them).
 """
 from __future__ import annotations
@@ -77,6 +87,16 @@ def bucket_ranges(psi_p: int, bucket: int) -> List[Tuple[int, int]]:
         out.append((lo, hi))
         hi = lo
     return out
+
+
+def q8_bytes(n: int) -> int:
+    """Bytes of the int8 payload of n values: ceil(n/128) records of 132 bytes."""
+    return (n + 127) // 128 * 132
+
+
+def q8_segment(n: int) -> int:
+    """An owner's segment of the int8 exchange: its payload padded to a multiple of 16 bytes."""
+    return (q8_bytes(n) + 15) // 16 * 16 if n else 0
 
 
 def owner_parts(lo: int, hi: int, shard: int, nd: int) -> List[int]:
@@ -131,12 +151,21 @@ class LibzeroCompute:
     def commit(self, n, state_in, state_out, params, status):
         self.lz.zero_step_commit(n, *state_in, *state_out, params, status)
 
+    def quantize(self, n, grad, payload):
+        self.lz.zero_quantize_q8(n, grad, payload)
+
+    def fused_q8(self, n, payloads, state_in, state_out, params, hp, t, status):
+        self.lz.zero_step_fused_q8(n, len(payloads), payloads, *state_in, *state_out, params, hp,
+                                   t, status)
+
 
 class DistZeroStep:
     """One rank's side of the distributed step. psi_p: the flat padded length (a multiple of
-    the world size); bucket: elements per bucket (0: one bucket, stage 1)."""
+    the world size); bucket: elements per bucket (0: one bucket, stage 1); payload: "fp16"
+    (the gradients themselves are exchanged) or "q8" (int8 records, all-to-all form only)."""
 
-    def __init__(self, psi_p: int, bucket: int = 0, group=None, compute=None, peers=None):
+    def __init__(self, psi_p: int, bucket: int = 0, group=None, compute=None, peers=None,
+                 payload: str = "fp16"):
         import torch.distributed as dist
         self.dist = dist
         self.group = group
@@ -149,17 +178,32 @@ class DistZeroStep:
         self.buckets = bucket_ranges(psi_p, bucket)
         self.parts = [owner_parts(lo, hi, self.shard, self.nd) for lo, hi in self.buckets]
         self.compute = compute or LibzeroCompute()
+        if payload not in ("fp16", "q8"):
+            raise ValueError(f"payload {payload!r}")
+        if payload == "q8" and peers is not None:
+            raise ValueError("the int8 payload is exchanged by all-to-all, not read from peers")
+        self.payload = payload
         self.peers = peers
         self.in_place_gather = dist.get_backend(group) == "nccl"
         self._recv = None      # two receive buffers, nd * (largest owner part) values each
+        self._send = None      # q8: two send buffers, the largest bucket's padded segments
         self._bits = None      # the three void bits, combined across ranks
         self._masks = None
         self._gather_src = None
 
     def _buffers(self, local_grad, params_full, status):
         import torch
-        if self.peers is None and (self._recv is None or self._recv[0].device != local_grad.device
-                                   or self._recv[0].dtype != local_grad.dtype):
+        if self.payload == "q8":
+            if self._recv is None or self._recv[0].device != local_grad.device:
+                most = max(q8_segment(p[self.rank]) for p in self.parts)
+                send = max(sum(q8_segment(x) for x in p) for p in self.parts)
+                self._recv = [torch.empty(self.nd * most, dtype=torch.uint8,
+                                          device=local_grad.device) for _ in range(2)]
+                self._send = [torch.empty(send, dtype=torch.uint8, device=local_grad.device)
+                              for _ in range(2)]
+        elif self.peers is None and (self._recv is None
+                                     or self._recv[0].device != local_grad.device
+                                     or self._recv[0].dtype != local_grad.dtype):
             most = max(p[self.rank] for p in self.parts)
             self._recv = [torch.empty(self.nd * most, dtype=local_grad.dtype,
                                       device=local_grad.device) for _ in range(2)]
@@ -193,13 +237,29 @@ class DistZeroStep:
             self._reduce_from_peers(state_in, state_out, own, hp, t, status)
             return self._finish(state_in, state_out, own, params_full, status)
 
+        q8 = self.payload == "q8"
+
         def exchange(k):
             lo, hi = self.buckets[k]
             parts = self.parts[k]
             mine = parts[r]
-            works[k] = dist.all_to_all_single(recv[k % 2][:nd * mine], local_grad[lo:hi],
-                                              output_split_sizes=[mine] * nd,
-                                              input_split_sizes=parts, group=self.group,
+            if not q8:
+                works[k] = dist.all_to_all_single(recv[k % 2][:nd * mine], local_grad[lo:hi],
+                                                  output_split_sizes=[mine] * nd,
+                                                  input_split_sizes=parts, group=self.group,
+                                                  async_op=True)
+                return
+            # quantize each owner's part (blocks from the part's first value) into its segment
+            segs = [q8_segment(x) for x in parts]
+            send, off = self._send[k % 2], 0
+            for q, x in enumerate(parts):
+                if x:
+                    a = max(lo, q * S)
+                    self.compute.quantize(x, local_grad[a:a + x], send[off:off + q8_bytes(x)])
+                off += segs[q]
+            works[k] = dist.all_to_all_single(recv[k % 2][:nd * segs[r]], send[:off],
+                                              output_split_sizes=[segs[r]] * nd,
+                                              input_split_sizes=segs, group=self.group,
                                               async_op=True)
 
         exchange(0)
@@ -213,10 +273,15 @@ class DistZeroStep:
                 continue
             a = max(lo, r * S) - r * S            # the bucket's part of my shard
             buf = recv[k % 2]
-            rows = [buf[j * mine:(j + 1) * mine] for j in range(nd)]
-            self.compute.fused(mine, rows, [x[a:a + mine] for x in state_in],
-                               [x[a:a + mine] for x in state_out], own[a:a + mine], hp, t,
-                               status)
+            ins = [x[a:a + mine] for x in state_in]
+            outs = [x[a:a + mine] for x in state_out]
+            if q8:
+                seg = q8_segment(mine)
+                pays = [buf[j * seg:j * seg + q8_bytes(mine)] for j in range(nd)]
+                self.compute.fused_q8(mine, pays, ins, outs, own[a:a + mine], hp, t, status)
+            else:
+                rows = [buf[j * mine:(j + 1) * mine] for j in range(nd)]
+                self.compute.fused(mine, rows, ins, outs, own[a:a + mine], hp, t, status)
         return self._finish(state_in, state_out, own, params_full, status)
 
     def _reduce_from_peers(self, state_in, state_out, own, hp, t, status):
