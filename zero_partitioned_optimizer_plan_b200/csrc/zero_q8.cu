@@ -84,16 +84,28 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
     return d;
 }
 
-// A half-warp's 8 fp16 values of block b (thread h of the half: elements 8h .. 8h+7), missing
-// elements as +0.
-__device__ __forceinline__ uint4 quant_load(const QuantArgs& p, uint64_t b, int hl) {
-    const uint64_t i0 = b * kQB + (uint64_t)hl * 8u;
-    if (p.gvec && i0 + 8 <= p.n) return *reinterpret_cast<const uint4*>(p.g + i0);
-    uint16_t h[8];
+// Thread h of a block's 128/V threads: the block's fp16 values V*h .. V*h+V-1 (V/8 16-byte
+// loads), missing elements as +0.
+template <int V>
+__device__ __forceinline__ void quant_load(const QuantArgs& p, uint64_t b, int hl,
+                                           uint4 (&u)[V / 8]) {
+    const uint64_t i0 = b * kQB + (uint64_t)hl * V;
+    if (p.gvec && i0 + V <= p.n) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.g + i0);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) h[j] = i0 + j < p.n ? p.g[i0 + j] : (uint16_t)0;
-    return make_uint4(h[0] | (uint32_t)h[1] << 16, h[2] | (uint32_t)h[3] << 16,
-                      h[4] | (uint32_t)h[5] << 16, h[6] | (uint32_t)h[7] << 16);
+        for (int k = 0; k < V / 8; ++k) u[k] = src[k];
+        return;
+    }
+    uint32_t h[V / 2];
+#pragma unroll
+    for (int j = 0; j < V / 2; ++j) {
+        const uint32_t lo = i0 + 2 * j < p.n ? p.g[i0 + 2 * j] : 0u;
+        const uint32_t hi = i0 + 2 * j + 1 < p.n ? p.g[i0 + 2 * j + 1] : 0u;
+        h[j] = lo | hi << 16;
+    }
+#pragma unroll
+    for (int k = 0; k < V / 8; ++k)
+        u[k] = make_uint4(h[4 * k], h[4 * k + 1], h[4 * k + 2], h[4 * k + 3]);
 }
 
 // 1.5 * 2^23 + 128: y + kRintBias, for |y| < 2^21, rounds y to the nearest integer (ties to even,
@@ -139,54 +151,81 @@ __device__ __forceinline__ uint32_t quant_word_div(uint32_t h01, uint32_t h23, f
     return w;
 }
 
-// A half-warp per block of 128: thread h of the half holds elements 8h .. 8h+7; a warp takes two
-// consecutive blocks per iteration and has the next iteration's load in flight. The block's
-// max |x| is an integer max over the fp16 magnitude bits (ordered like the magnitudes, inf and
-// NaN above every finite value), so a poisoned block is one compare.
+// V values per thread, 128/V threads per block of 128: a warp takes V/4 consecutive blocks per
+// iteration and has the next iteration's loads in flight; the block's scale, its reciprocal and
+// the reductions are paid once per V values. The block's max |x| is an integer max over the
+// fp16 magnitude bits (ordered like the magnitudes, inf and NaN above every finite value), so a
+// poisoned block is one compare.
+template <int V>
 __global__ void __launch_bounds__(256) quant_q8_kernel(const __grid_constant__ QuantArgs p) {
+    static_assert(V == 8 || V == 16 || V == 32, "values per thread");
+    constexpr int kTpb = kQB / V;      // threads per block of 128
+    constexpr int kBpw = 32 / kTpb;    // blocks per warp and iteration
     const int lane = threadIdx.x & 31;
-    const int half = lane >> 4;
-    const int hl = lane & 15;
+    const int part = lane / kTpb;
+    const int hl = lane % kTpb;
     const uint64_t nblocks = (p.n + kQB - 1) / kQB;
-    const uint64_t npairs = (nblocks + 1) / 2;
+    const uint64_t ngroups = (nblocks + kBpw - 1) / kBpw;
     const uint64_t nwarps = ((uint64_t)gridDim.x * blockDim.x) >> 5;
-    uint64_t pr = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    uint4 next = make_uint4(0u, 0u, 0u, 0u);
-    if (pr < npairs) next = quant_load(p, 2 * pr + (uint64_t)half, hl);
-    for (; pr < npairs; pr += nwarps) {
-        const uint64_t b = 2 * pr + (uint64_t)half;
-        const uint4 u = next;
-        if (pr + nwarps < npairs) next = quant_load(p, b + 2 * nwarps, hl);
-        const bool exists = b < nblocks;
-        uint32_t mag = __vmaxu2(u.x & 0x7fff7fffu, u.y & 0x7fff7fffu);
-        mag = __vmaxu2(mag, __vmaxu2(u.z & 0x7fff7fffu, u.w & 0x7fff7fffu));
-        mag = max(mag & 0xffffu, mag >> 16);
-        // reductions inside each half-warp (xor offsets below 16 stay in the half)
+    uint64_t pg = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    uint4 nx[V / 8];
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) mag = max(mag, __shfl_xor_sync(0xffffffffu, mag, o));
+    for (int k = 0; k < V / 8; ++k) nx[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (pg < ngroups) quant_load<V>(p, kBpw * pg + (uint64_t)part, hl, nx);
+    for (; pg < ngroups; pg += nwarps) {
+        const uint64_t b = kBpw * pg + (uint64_t)part;
+        uint4 u[V / 8];
+#pragma unroll
+        for (int k = 0; k < V / 8; ++k) u[k] = nx[k];
+        if (pg + nwarps < ngroups) quant_load<V>(p, b + kBpw * nwarps, hl, nx);
+        const bool exists = b < nblocks;
+        uint32_t mag = 0u;
+#pragma unroll
+        for (int k = 0; k < V / 8; ++k)
+            mag = __vmaxu2(mag, __vmaxu2(__vmaxu2(u[k].x & 0x7fff7fffu, u[k].y & 0x7fff7fffu),
+                                         __vmaxu2(u[k].z & 0x7fff7fffu, u[k].w & 0x7fff7fffu)));
+        mag = max(mag & 0xffffu, mag >> 16);
+        // reductions inside each block's group of lanes (xor offsets below kTpb stay in it)
+#pragma unroll
+        for (int o = kTpb / 2; o > 0; o >>= 1)
+            mag = max(mag, __shfl_xor_sync(0xffffffffu, mag, o));
         const bool bad = mag >= 0x7c00u;
         const float scale = bad ? __uint_as_float(0x7fc00000u)
                                 : __fdiv_rn(h2f((uint16_t)mag), 127.0f);
-        uint32_t w0 = 0x80808080u, w1 = 0x80808080u;   // q = 0
+        uint32_t w[V / 4];
+#pragma unroll
+        for (int k = 0; k < V / 4; ++k) w[k] = 0x80808080u;   // q = 0
         if (!bad && scale != 0.0f) {
             const float r = __frcp_rn(scale);
             const uint64_t rr = f2_pack(r, r);
             bool near = false;
-            w0 = quant_word(u.x, u.y, rr, near);
-            w1 = quant_word(u.z, u.w, rr, near);
+#pragma unroll
+            for (int k = 0; k < V / 8; ++k) {
+                w[2 * k] = quant_word(u[k].x, u[k].y, rr, near);
+                w[2 * k + 1] = quant_word(u[k].z, u[k].w, rr, near);
+            }
             if (near) {
-                w0 = quant_word_div(u.x, u.y, scale);
-                w1 = quant_word_div(u.z, u.w, scale);
+#pragma unroll
+                for (int k = 0; k < V / 8; ++k) {
+                    w[2 * k] = quant_word_div(u[k].x, u[k].y, scale);
+                    w[2 * k + 1] = quant_word_div(u[k].z, u[k].w, scale);
+                }
             }
         }
-        if (exists) {   // records are 4-byte aligned (132 = 4 * 33), 8 * hl too
+        if (exists) {   // records are 4-byte aligned (132 = 4 * 33), V * hl too
             uint8_t* rec = p.rec + b * kRec;
-            reinterpret_cast<uint32_t*>(rec + hl * 8)[0] = w0;
-            reinterpret_cast<uint32_t*>(rec + hl * 8)[1] = w1;
+            uint32_t* dst = reinterpret_cast<uint32_t*>(rec + hl * V);
+#pragma unroll
+            for (int k = 0; k < V / 4; ++k) dst[k] = w[k];
             if (hl == 0) *reinterpret_cast<float*>(rec + kQB) = scale;
         }
     }
 }
+
+// Values per thread of the quantizer, measured on B200 (the senders' side of the int8 lines,
+// flat 2^28 / the 7.5B view, two passes): 8 values 0.62 / 0.66 of the peak, 16 values 0.77 /
+// 0.82, 32 values 0.60 / 0.64 (96 registers: half the resident warps).
+constexpr int kQuantVals = 16;
 
 struct FusedQ8Args {
     const uint8_t* rec[kMaxRanks];   // each rank's records for this range
@@ -528,14 +567,16 @@ cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, uint8_t* payload,
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
-    const uint64_t npairs = ((n + kQB - 1) / kQB + 1) / 2;   // two blocks per warp, 8 warps/CTA
-    // two full waves of resident blocks: 0.64 of the peak against 0.63 with one and 0.60 with
-    // 8 blocks per SM (1.6 waves). Not better: 6 or 8 resident blocks per SM by launch bounds
-    // (0.58 / 0.57, registers spilled), a second block pair's load in flight (0.57).
+    constexpr uint64_t kBpw = 32 / (kQB / kQuantVals);          // blocks per warp, 8 warps/CTA
+    const uint64_t ngroups = ((n + kQB - 1) / kQB + kBpw - 1) / kBpw;
+    // one full wave of resident blocks: with 16 values per thread 0.77 / 0.82 against 0.76 /
+    // 0.80 with two waves and 0.74 / 0.79 with four. (With 8 values per thread two waves had
+    // won, 0.64 against 0.63 with one and 0.60 with 8 blocks per SM; 6 or 8 resident blocks per
+    // SM forced by launch bounds, registers spilled, and a second load in flight were slower.)
     unsigned grid = 1;
-    e = resident_grid(quant_q8_kernel, di, 256, (npairs + 7) / 8, 2, &grid);
+    e = resident_grid(quant_q8_kernel<kQuantVals>, di, 256, (ngroups + 7) / 8, 1, &grid);
     if (e != cudaSuccess) return e;
-    quant_q8_kernel<<<grid, 256, 0, stream>>>(p);
+    quant_q8_kernel<kQuantVals><<<grid, 256, 0, stream>>>(p);
     count_launch();
     return cudaGetLastError();
 }
