@@ -50,7 +50,13 @@ def _worker(port, numels, bucket, out, peer=False, payload="fp16"):
         st_out = [torch.full_like(x, float("nan")) for x in st_in]
         params = torch.zeros(psi, dtype=torch.float16, device=dev)
         status = torch.zeros(1, dtype=torch.int32, device=dev)
-        if peer:    # gradients produced into symmetric memory; the owner reads them in place
+        if peer and payload == "q8":   # int8 records quantized into symmetric memory
+            from zero_partitioned_optimizer_plan_b200.dist import (SymmetricPeerBuffers,
+                                                                   q8_peer_bytes)
+            peers = SymmetricPeerBuffers(q8_peer_bytes(psi, bucket, 1), torch.uint8, dev)
+            step = DistZeroStep(psi, bucket, peers=peers, payload="q8")
+            flag = step.step(grad.to(dev), st_in, st_out, params, lz.AdamHP(), 1, status)
+        elif peer:    # gradients produced into symmetric memory; the owner reads them in place
             from zero_partitioned_optimizer_plan_b200.dist import SymmetricPeerBuffers
             peers = SymmetricPeerBuffers(psi, torch.float16, dev)
             peers.local.copy_(grad.to(dev))
@@ -94,17 +100,19 @@ def test_distributed_step_one_rank_nccl(bucket, peer):
     assert int(oracle.ulp_diff_f16(params, ref.params16).max()) <= 1
 
 
+@pytest.mark.parametrize("peer", [False, True])
 @pytest.mark.parametrize("bucket", [0, 3000])
-def test_distributed_step_int8_payload_one_rank_nccl(bucket):
+def test_distributed_step_int8_payload_one_rank_nccl(bucket, peer):
     """payload="q8" on one NCCL rank: the library's quantizer fills the send buffer, the
-    all-to-all moves the records, the library's int8 step runs on the received payloads;
-    against the oracle's quantizer and int8 step per bucket (0 ulp)."""
+    all-to-all moves the records, the library's int8 step runs on the received payloads (or,
+    peer-read form, the quantizer writes into torch symmetric memory and the int8 step reads
+    the payloads there); against the oracle's quantizer and int8 step per bucket (0 ulp)."""
     import oracle
     from zero_partitioned_optimizer_plan_b200.dist import bucket_ranges
     numels = [1000, 37, 4099, 12345]
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    p = ctx.Process(target=_worker, args=(_free_port(), numels, bucket, q, False, "q8"))
+    p = ctx.Process(target=_worker, args=(_free_port(), numels, bucket, q, peer, "q8"))
     p.start()
     try:
         flag, status, shard, params = q.get(timeout=240)

@@ -442,9 +442,6 @@ def test_distributed_step_int8_payload_gloo(ws, bucket, bad_rank):
     Nd payloads. Against the oracle's quantizer and int8 owner step over the same
     (bucket, owner) parts, bit for bit; an inf in one rank's gradient skips the step on every
     rank."""
-    import numpy as np
-    import oracle
-    from zero_partitioned_optimizer_plan_b200.dist import bucket_ranges
     numels = [1000, 37, 4099, 12345]
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
@@ -462,6 +459,15 @@ def test_distributed_step_int8_payload_gloo(ws, bucket, bad_rank):
             if p.exitcode is None:
                 p.kill()
     assert all(p.exitcode == 0 for p in procs)
+    _check_q8_result(res, numels, ws, bucket, bad_rank)
+
+
+def _check_q8_result(res, numels, ws, bucket, bad_rank):
+    """Every rank's shard and full fp16 parameters against the oracle's quantizer and int8
+    owner step over the (bucket, owner) parts; one overflow skips the step everywhere."""
+    import numpy as np
+    import oracle
+    from zero_partitioned_optimizer_plan_b200.dist import bucket_ranges
     psi_p, grads, master, m, v = _dist_case(numels, ws, bad_rank)
     S = psi_p // ws
     w, mm, vv = master.numpy().copy(), m.numpy().copy(), v.numpy().copy()
@@ -482,9 +488,89 @@ def test_distributed_step_int8_payload_gloo(ws, bucket, bad_rank):
         w, mm, vv = master.numpy(), m.numpy(), v.numpy()
         p16 = oracle.f2h(master.numpy())
     assert skipped == (bad_rank >= 0)
-    for rank, flag, status, shard, params in res:
+    for rank, flag, status, shard, params in (x[:5] for x in res):
         assert flag == (1 if skipped else 0)
         assert bool(status & 2) == skipped
         for got, want in zip(shard, (w, mm, vv)):
             assert np.array_equal(got.view(np.uint32), want[rank * S:(rank + 1) * S].view(np.uint32))
         assert np.array_equal(params, p16)
+
+
+def _worker_dist_q8_peer(rank, ws, port, numels, bucket, bad_rank, bufs, out):
+    import datetime
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle
+    from zero_partitioned_optimizer_plan_b200.dist import DistZeroStep, SharedPeerBuffers
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        psi_p, grads, master, m, v = _dist_case(numels, ws, bad_rank)
+        S = psi_p // ws
+        peers = SharedPeerBuffers(bufs, rank)
+        st_in = [x[rank * S:(rank + 1) * S].clone() for x in (master, m, v)]
+        st_out = [torch.full_like(x, float("nan")) for x in st_in]
+        params = torch.zeros(psi_p, dtype=torch.float16)
+        params[rank * S:(rank + 1) * S] = torch.from_numpy(
+            oracle.f2h(st_in[0].numpy()).view("float16"))
+        status = torch.zeros(1, dtype=torch.int32)
+        step = DistZeroStep(psi_p, bucket, compute=_OracleCompute(), peers=peers, payload="q8")
+        flag = step.step(grads[rank], st_in, st_out, params, oracle.AdamHP(), 1, status)
+        out.put((rank, int(flag.item()), int(status.item()), [x.numpy() for x in st_out],
+                 params.numpy().view("uint16"), step._recv is None and step._send is None))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("ws,bucket,bad_rank", [(2, 0, -1), (3, 2500, -1), (3, 2500, 0)])
+def test_distributed_step_int8_peer_reads_gloo(ws, bucket, bad_rank):
+    """The int8 peer-read form: each rank quantizes every (bucket, owner) part into its own
+    buffer (CPU tensors shared by the processes, standing for NVLink peer mappings) at offsets
+    every rank computes alike; per bucket a barrier, then the owner's int8 step reads the Nd
+    payloads of its part in the peers' buffers -- no all-to-all, no send or receive buffers.
+    The same results as the oracle's quantizer and int8 step over the parts, bit for bit."""
+    import torch
+    from zero_partitioned_optimizer_plan_b200.dist import q8_peer_bytes
+    numels = [1000, 37, 4099, 12345]
+    psi_p = -(-sum(numels) // ws) * ws
+    nbytes = q8_peer_bytes(psi_p, bucket, ws)
+    bufs = [torch.zeros(nbytes, dtype=torch.uint8).share_memory_() for _ in range(ws)]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_dist_q8_peer,
+                         args=(r, ws, port, numels, bucket, bad_rank, bufs, q))
+             for r in range(ws)]
+    for p in procs:
+        p.start()
+    try:
+        res = sorted((q.get(timeout=240) for _ in range(ws)), key=lambda x: x[0])
+    finally:
+        for p in procs:
+            p.join(60)
+            if p.exitcode is None:
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    assert all(x[5] for x in res)          # nothing exchanged but the barriers
+    _check_q8_result(res, numels, ws, bucket, bad_rank)
+
+
+def test_q8_peer_layout_tiles_every_part():
+    """The peer buffer's layout: one 16-byte-aligned segment per (bucket, owner) part, in
+    order, each holding that part's records, none overlapping."""
+    from zero_partitioned_optimizer_plan_b200.dist import (bucket_ranges, owner_parts,
+                                                           q8_bytes, q8_peer_layout)
+    for psi_p, bucket, nd in [(17481, 0, 1), (17484, 2500, 3), (10_000_000, 1_000_003, 8),
+                              (4096, 128, 64 // 16)]:
+        offs, total = q8_peer_layout(psi_p, bucket, nd)
+        spans = []
+        for k, (lo, hi) in enumerate(bucket_ranges(psi_p, bucket)):
+            for q, x in enumerate(owner_parts(lo, hi, psi_p // nd, nd)):
+                assert offs[k][q] % 16 == 0
+                if x:
+                    spans.append((offs[k][q], offs[k][q] + q8_bytes(x)))
+        spans.sort()
+        assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+        assert spans[-1][1] <= total

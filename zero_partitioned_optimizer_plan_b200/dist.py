@@ -42,7 +42,7 @@ like any collective) guarantees that every rank has produced the bucket before a
 it; the all-reduce of the void bits at the end of the step is the barrier after which no
 owner reads this step's gradients any more, so the next backward pass may overwrite them.
 
-Compressed payload (``payload="q8"``, all-to-all form). "ZeRO" (lastdictionary.com), main
+Compressed payload (``payload="q8"``). "ZeRO" (lastdictionary.com), main
 definition: extensions compress the communication (ZeRO++). Each rank quantizes its slice of
 a bucket for each owner with the library's zero_quantize_q8 (records of 128 bytes q + 128 and an
 fp32 scale, blocks counted from the start of the owner's part), the all-to-all moves those
@@ -50,7 +50,11 @@ records (132/128 bytes per value instead of 2), and the owner runs zero_step_fus
 Nd received payloads in rank order. Each owner's segment is padded to a multiple of 16 bytes
 so that every received payload starts 16-byte aligned (the library's bulk-copy path). Send
 buffers are double-buffered like the receive buffers: bucket k+2 is quantized into bucket k's
-send buffer only after the current stream has waited for bucket k's exchange.
+send buffer only after the current stream has waited for bucket k's exchange. With ``peers``
+(their buffers of q8_peer_bytes(...) bytes), each rank quantizes every (bucket, owner) part into
+its own peer buffer at an offset every rank computes alike, and the owner's kernel reads the
+Nd payloads of its part in the peers' buffers (per bucket the same barrier as the fp16 peer
+reads); nothing is exchanged but the barriers.
 
 The collectives are torch.distributed calls (NCCL on GPUs, gloo on CPUs); the arithmetic is the
 library's. ``compute`` replaces the library calls (the tests run the exchange on CPU
@@ -97,6 +101,26 @@ def q8_bytes(n: int) -> int:
 def q8_segment(n: int) -> int:
     """An owner's segment of the int8 exchange: its payload padded to a multiple of 16 bytes."""
     return (q8_bytes(n) + 15) // 16 * 16 if n else 0
+
+
+def q8_peer_layout(psi_p: int, bucket: int, nd: int):
+    """Byte offset of every (bucket, owner) part's payload in a rank's peer buffer (buckets in
+    backward order, owners in rank order, each part's segment padded to 16 bytes), and the
+    buffer's size."""
+    shard = psi_p // nd
+    offs, total = [], 0
+    for lo, hi in bucket_ranges(psi_p, bucket):
+        row = []
+        for x in owner_parts(lo, hi, shard, nd):
+            row.append(total)
+            total += q8_segment(x)
+        offs.append(row)
+    return offs, max(total, 16)
+
+
+def q8_peer_bytes(psi_p: int, bucket: int, nd: int) -> int:
+    """Size of each rank's peer buffer for the int8 peer-read form."""
+    return q8_peer_layout(psi_p, bucket, nd)[1]
 
 
 def owner_parts(lo: int, hi: int, shard: int, nd: int) -> List[int]:
@@ -180,9 +204,11 @@ class DistZeroStep:
         self.compute = compute or LibzeroCompute()
         if payload not in ("fp16", "q8"):
             raise ValueError(f"payload {payload!r}")
-        if payload == "q8" and peers is not None:
-            raise ValueError("the int8 payload is exchanged by all-to-all, not read from peers")
         self.payload = payload
+        if payload == "q8" and peers is not None:
+            self._q8_offs, need = q8_peer_layout(psi_p, bucket, self.nd)
+            if peers.local.numel() * peers.local.element_size() < need:
+                raise ValueError(f"peer buffers of {need} bytes are needed (q8_peer_bytes)")
         self.peers = peers
         self.in_place_gather = dist.get_backend(group) == "nccl"
         self._recv = None      # two receive buffers, nd * (largest owner part) values each
@@ -193,7 +219,7 @@ class DistZeroStep:
 
     def _buffers(self, local_grad, params_full, status):
         import torch
-        if self.payload == "q8":
+        if self.payload == "q8" and self.peers is None:
             if self._recv is None or self._recv[0].device != local_grad.device:
                 most = max(q8_segment(p[self.rank]) for p in self.parts)
                 send = max(sum(q8_segment(x) for x in p) for p in self.parts)
@@ -232,6 +258,9 @@ class DistZeroStep:
         nb = len(self.buckets)
         works = [None] * nb
         if self.peers is not None:
+            if self.payload == "q8":
+                self._reduce_q8_from_peers(local_grad, state_in, state_out, own, hp, t, status)
+                return self._finish(state_in, state_out, own, params_full, status)
             if local_grad is not self.peers.local:
                 self.peers.local.copy_(local_grad)   # produce into peers.local to avoid this
             self._reduce_from_peers(state_in, state_out, own, hp, t, status)
@@ -308,6 +337,40 @@ class DistZeroStep:
                                [x[a - r * S:b - r * S] for x in state_in],
                                [x[a - r * S:b - r * S] for x in state_out],
                                own[a - r * S:b - r * S], hp, t, status)
+
+    def _reduce_q8_from_peers(self, local_grad, state_in, state_out, own, hp, t, status):
+        """Per bucket: quantize this rank's part for every owner into its own peer buffer, a
+        barrier (every rank has quantized the bucket), then the owner's int8 step over the Nd
+        payloads of its part, read in the peers' buffers. Bucket k+1 is quantized and its
+        barrier issued before bucket k's step."""
+        dist, nd, r, S = self.dist, self.nd, self.rank, self.shard
+        nb = len(self.buckets)
+        works = [None] * nb
+        mine_buf = self.peers.local
+
+        def produce(k):
+            lo, hi = self.buckets[k]
+            for q, x in enumerate(self.parts[k]):
+                if x:
+                    a, o = max(lo, q * S), self._q8_offs[k][q]
+                    self.compute.quantize(x, local_grad[a:a + x], mine_buf[o:o + q8_bytes(x)])
+            works[k] = dist.all_reduce(self._tick, group=self.group, async_op=True)
+
+        produce(0)
+        for k, (lo, hi) in enumerate(self.buckets):
+            if k + 1 < nb:
+                produce(k + 1)
+            works[k].wait()
+            works[k] = None
+            mine = self.parts[k][r]
+            if mine == 0:
+                continue
+            a = max(lo, r * S) - r * S
+            o = self._q8_offs[k][r]
+            self.compute.fused_q8(mine, self.peers.rows(o, o + q8_bytes(mine)),
+                                  [x[a:a + mine] for x in state_in],
+                                  [x[a:a + mine] for x in state_out], own[a:a + mine], hp, t,
+                                  status)
 
     def _finish(self, state_in, state_out, own, params_full, status):
         dist, S = self.dist, self.shard
