@@ -732,7 +732,7 @@ def _init_zero3(self, args, dev):
     self.config = workload_config(args)
     n_fused = sum(((psi_p if l == len(self.layers) - 1 else hi) - 1) // S - lo // S + 1
                   for l, (lo, hi) in enumerate(self.layers))
-    self.config["calls_per_step"] = 2 * len(self.layers) + n_fused + nd
+    self.config["calls_per_step"] = 2 * len(self.layers) + n_fused + 1   # + one commit
     self.config["fused_calls_per_step"] = n_fused
     gather_bytes = 2 * 4 * psi              # two gathers: 2 bytes read + 2 written each
     fused_bytes = (2 * nd + 26) * psi_p

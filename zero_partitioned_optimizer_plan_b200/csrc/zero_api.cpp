@@ -532,27 +532,19 @@ zero_status zero_stage3_step_commit(const zero_plan* plan, const float* master_i
     if (!d_status || !param_shards || !master_in || !m_in || !v_in || !master_out || !m_out ||
         !v_out)
         return ZERO_EINVAL;
-    for (int pass = 0; pass < 2; ++pass) {
-        for (int q = 0; q < nd; ++q) {
-            const uint64_t off = (uint64_t)q * S;
-            if (pass == 0) {
-                const zero_status st = zk::check_fused_state(
-                    S, master_in + off, m_in + off, v_in + off, master_out + off, m_out + off,
-                    v_out + off, param_shards[q], d_status);
-                if (st != ZERO_OK) return st;
-                for (int o = 0; o < q; ++o)
-                    if (zk::overlap(param_shards[o], S * 2, param_shards[q], S * 2))
-                        return ZERO_EINVAL;
-            } else {
-                const cudaError_t e = zk::launch_commit(S, master_in + off, m_in + off, v_in + off,
-                                                        master_out + off, m_out + off, v_out + off,
-                                                        param_shards[q], d_status,
-                                                        (cudaStream_t)stream);
-                if (e != cudaSuccess) return zk::from_cuda(e);
-            }
-        }
+    for (int q = 0; q < nd; ++q) {
+        const uint64_t off = (uint64_t)q * S;
+        const zero_status st = zk::check_fused_state(
+            S, master_in + off, m_in + off, v_in + off, master_out + off, m_out + off,
+            v_out + off, param_shards[q], d_status);
+        if (st != ZERO_OK) return st;
+        for (int o = 0; o < q; ++o)
+            if (zk::overlap(param_shards[o], S * 2, param_shards[q], S * 2)) return ZERO_EINVAL;
     }
-    return ZERO_OK;
+    if (S == 0) return ZERO_OK;
+    return zk::from_cuda(zk::launch_stage3_commit(S, nd, master_in, m_in, v_in, master_out,
+                                                  m_out, v_out, param_shards, d_status,
+                                                  (cudaStream_t)stream));
 }
 
 zero_status zero_step_status(const uint32_t* d_status, zero_stream_t stream, uint32_t* flags_out) {

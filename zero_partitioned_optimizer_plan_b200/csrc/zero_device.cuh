@@ -40,6 +40,8 @@ namespace {
 
 
 constexpr int kMaxRanks = ZERO_MAX_RANKS;
+// Status bits under which a step is not applied (its commit restores the inputs).
+constexpr uint32_t kStepVoid = ZERO_FLAG_OVERFLOW | ZERO_FLAG_TIMEOUT | ZERO_FLAG_BOUNDS;
 constexpr int kElems = 4;                        // elements per consumer thread and tile
 constexpr int kMaxStages = 8;
 constexpr int kDataOffset = 128;                 // full[8] and empty[8] mbarriers first

@@ -48,6 +48,11 @@ cudaError_t launch_selftest_timeout(uint32_t* status, cudaStream_t stream);
 cudaError_t launch_gather(uint64_t flat_lo, uint64_t len, uint64_t shard, int nd,
                           const uint16_t* const* shards, uint16_t* out, uint32_t* status,
                           cudaStream_t stream);
+// The commit of a stage-3 step over every owner in one launch (state flat, nd partitions).
+cudaError_t launch_stage3_commit(uint64_t shard, int nd, const float* master_in,
+                                 const float* m_in, const float* v_in, float* master_out,
+                                 float* m_out, float* v_out, uint16_t* const* shards,
+                                 uint32_t* status, cudaStream_t stream);
 cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, uint8_t* payload,
                             cudaStream_t stream);
 cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,

@@ -40,9 +40,6 @@ namespace zk {
 
 namespace {
 
-// Status bits under which a step is not applied.
-constexpr uint32_t kStepVoid = ZERO_FLAG_OVERFLOW | ZERO_FLAG_TIMEOUT | ZERO_FLAG_BOUNDS;
-
 struct FusedArgs {
     const uint16_t* grads[kMaxRanks];
     const float* master_in;

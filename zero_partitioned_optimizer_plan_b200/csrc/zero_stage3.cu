@@ -25,7 +25,8 @@
 // Every thread keeps U chunks' loads in flight before it stores.
 //
 // The update of stage 3 is the fused step of zero_kernels.cu applied to each owner's part of
-// a layer's range, its fp16 output written into that owner's partition; the commit likewise.
+// a layer's range, its fp16 output written into that owner's partition; the commit of a step is
+// one launch over every owner (commit3_kernel below).
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -94,6 +95,9 @@ __device__ __forceinline__ uint4 load_chunk(const uint16_t* src, int vec) {
 }
 
 __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const __grid_constant__ GatherArgs p) {
+    // launched with programmatic stream serialization: the grid may be resident before the
+    // previous kernel on the stream ends; it waits for that kernel here, before any access
+    pdl_enter(0);
     const uint64_t tid = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
     int seg = 0;
@@ -141,6 +145,58 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const __grid_con
     }
 }
 
+// The commit of a stage-3 step in one launch: when the step is void, every owner's state is
+// restored over the flat range and its fp16 partition rewritten from the restored master.
+struct Commit3Args {
+    const float* master_in;
+    const float* m_in;
+    const float* v_in;
+    float* master_out;
+    float* m_out;
+    float* v_out;
+    uint16_t* shards[kMaxRanks];
+    uint32_t* status;
+    uint64_t shard;
+    int nd;
+};
+
+__global__ void __launch_bounds__(256) commit3_kernel(const __grid_constant__ Commit3Args p) {
+    pdl_enter(0);
+    if (!(*reinterpret_cast<volatile uint32_t*>(p.status) & kStepVoid)) return;
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.status, ZERO_FLAG_SKIPPED);
+    const uint64_t n = p.shard * (uint64_t)p.nd;
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const uint64_t q = i / p.shard;
+        const float w = p.master_in[i];
+        p.master_out[i] = w;
+        p.m_out[i] = p.m_in[i];
+        p.v_out[i] = p.v_in[i];
+        p.shards[q][i - q * p.shard] = f2h(w);
+    }
+}
+
+// An ordered launch that may become resident before the previous kernel on the stream ends
+// (the kernel waits for it with griddepcontrol.wait before touching memory).
+template <typename K, typename A>
+cudaError_t launch_ordered(K kernel, const A& args, unsigned grid, unsigned threads,
+                           cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args);
+    count_launch();
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 int load_width(const void* p) {
     const uintptr_t a = reinterpret_cast<uintptr_t>(p);
     return (a & 15u) == 0 ? 16 : (a & 3u) == 0 ? 4 : 2;
@@ -185,9 +241,30 @@ cudaError_t launch_gather(uint64_t flat_lo, uint64_t len, uint64_t shard, int nd
     const uint64_t cap = (uint64_t)di.sms * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    gather_kernel<<<(unsigned)blocks, kGatherThreads, 0, stream>>>(p);
-    count_launch();
-    return cudaGetLastError();
+    return launch_ordered(gather_kernel, p, (unsigned)blocks, kGatherThreads, stream);
+}
+
+cudaError_t launch_stage3_commit(uint64_t shard, int nd, const float* master_in,
+                                 const float* m_in, const float* v_in, float* master_out,
+                                 float* m_out, float* v_out, uint16_t* const* shards,
+                                 uint32_t* status, cudaStream_t stream) {
+    Commit3Args p;
+    memset(&p, 0, sizeof(p));
+    p.master_in = master_in;
+    p.m_in = m_in;
+    p.v_in = v_in;
+    p.master_out = master_out;
+    p.m_out = m_out;
+    p.v_out = v_out;
+    for (int q = 0; q < nd; ++q) p.shards[q] = shards[q];
+    p.status = status;
+    p.shard = shard;
+    p.nd = nd;
+    DevInfo di;
+    const cudaError_t e = dev_info(&di);
+    if (e != cudaSuccess) return e;
+    return launch_ordered(commit3_kernel, p, plain_grid(shard * (uint64_t)nd, di.sms), 256,
+                          stream);
 }
 
 }  // namespace zk
