@@ -496,6 +496,27 @@ cudaError_t launch_pipe(K kernel, const A& args, const PipeShape& sh, cudaStream
     return cudaGetLastError();
 }
 
+// An ordered launch that may become resident before the previous kernel on the stream ends
+// (the kernel waits for it with griddepcontrol.wait before touching memory).
+template <typename K, typename A>
+cudaError_t launch_ordered(K kernel, const A& args, unsigned grid, unsigned threads,
+                           cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args);
+    count_launch();
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 unsigned plain_grid(uint64_t n, int sms, int per_sm = 8) {
     uint64_t blocks = (n + 255) / 256;
     const uint64_t cap = (uint64_t)sms * (uint64_t)per_sm;

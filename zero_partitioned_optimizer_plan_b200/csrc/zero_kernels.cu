@@ -385,6 +385,7 @@ __global__ void __launch_bounds__(256) rs_plain_kernel(const __grid_constant__ R
 // ---------------------------------------------------------------------------------------------
 template <bool kDC>
 __global__ void __launch_bounds__(256) adam_kernel(const __grid_constant__ AdamArgs p) {
+    pdl_enter(0);   // ordered after the reduce-scatters (see launch_ordered)
     // skip the whole step if any reduce-scatter of it saw inf/NaN, or if one of them failed
     // (its reduced shard is then incomplete)
     if (*reinterpret_cast<volatile uint32_t*>(p.status) & kStepVoid) {
@@ -446,6 +447,7 @@ __global__ void __launch_bounds__(256) adam_kernel(const __grid_constant__ AdamA
 // overflowed, and also when a kernel of the step gave up on a wait or failed its bounds
 // self-check: those leave some tiles of the outputs unwritten.
 __global__ void __launch_bounds__(256) commit_kernel(const __grid_constant__ CommitArgs p) {
+    pdl_enter(0);   // ordered after the step's kernels (see launch_ordered)
     if (!(*reinterpret_cast<volatile uint32_t*>(p.status) & kStepVoid)) return;
     if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.status, ZERO_FLAG_SKIPPED);
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
@@ -691,13 +693,9 @@ cudaError_t launch_adam(uint64_t n, const float* grad, float* master, float* m, 
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
-    uint64_t work = p.vec ? (n + 3) / 4 : n;
-    if (ad)
-        adam_kernel<true><<<plain_grid(work, di.sms), 256, 0, stream>>>(p);
-    else
-        adam_kernel<false><<<plain_grid(work, di.sms), 256, 0, stream>>>(p);
-    count_launch();
-    return cudaGetLastError();
+    const uint64_t work = p.vec ? (n + 3) / 4 : n;
+    return ad ? launch_ordered(adam_kernel<true>, p, plain_grid(work, di.sms), 256, stream)
+              : launch_ordered(adam_kernel<false>, p, plain_grid(work, di.sms), 256, stream);
 }
 
 cudaError_t launch_scaler_prepare(const zero_scaler_state* st, const AdamConsts* table,
@@ -731,9 +729,8 @@ cudaError_t launch_commit(uint64_t n, const float* master_in, const float* m_in,
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
-    commit_kernel<<<plain_grid(n, di.sms, ZK_COMMIT_BLOCKS_PER_SM), 256, 0, stream>>>(p);
-    count_launch();
-    return cudaGetLastError();
+    return launch_ordered(commit_kernel, p, plain_grid(n, di.sms, ZK_COMMIT_BLOCKS_PER_SM), 256,
+                          stream);
 }
 
 }  // namespace zk

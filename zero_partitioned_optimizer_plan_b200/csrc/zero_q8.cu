@@ -159,6 +159,7 @@ __device__ __forceinline__ uint32_t quant_word_div(uint32_t h01, uint32_t h23, f
 template <int V>
 __global__ void __launch_bounds__(256) quant_q8_kernel(const __grid_constant__ QuantArgs p) {
     static_assert(V == 8 || V == 16 || V == 32, "values per thread");
+    pdl_enter(0);   // ordered after the kernels before it (see launch_ordered)
     constexpr int kTpb = kQB / V;      // threads per block of 128
     constexpr int kBpw = 32 / kTpb;    // blocks per warp and iteration
     const int lane = threadIdx.x & 31;
@@ -576,9 +577,7 @@ cudaError_t launch_quant_q8(uint64_t n, const uint16_t* grad, uint8_t* payload,
     unsigned grid = 1;
     e = resident_grid(quant_q8_kernel<kQuantVals>, di, 256, (ngroups + 7) / 8, 1, &grid);
     if (e != cudaSuccess) return e;
-    quant_q8_kernel<kQuantVals><<<grid, 256, 0, stream>>>(p);
-    count_launch();
-    return cudaGetLastError();
+    return launch_ordered(quant_q8_kernel<kQuantVals>, p, grid, 256, stream);
 }
 
 cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,

@@ -176,27 +176,6 @@ __global__ void __launch_bounds__(256) commit3_kernel(const __grid_constant__ Co
     }
 }
 
-// An ordered launch that may become resident before the previous kernel on the stream ends
-// (the kernel waits for it with griddepcontrol.wait before touching memory).
-template <typename K, typename A>
-cudaError_t launch_ordered(K kernel, const A& args, unsigned grid, unsigned threads,
-                           cudaStream_t stream) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(threads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args);
-    count_launch();
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
-}
-
 int load_width(const void* p) {
     const uintptr_t a = reinterpret_cast<uintptr_t>(p);
     return (a & 15u) == 0 ? 16 : (a & 3u) == 0 ? 4 : 2;
