@@ -222,6 +222,34 @@ zero_status zero_step_fused(uint64_t n, int nd, const uint16_t* const* rank_grad
                             const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
                             zero_stream_t stream);
 
+/* zero_step_fused with the parameter all-gather in its epilogue. "ZeRO: particionar estados do
+ * treino entre GPUs" (upskillscore.com), "Como funciona": the updated fp16 parameters of each
+ * partition are all-gathered into every replica; "ZeRO-2" (llm-engineer.pages.dev), "왜
+ * all-gather는 그대로 필요한가". Instead of one param_out, the kernel stores each fp16 value
+ * into every replica: param_replicas is a host array of n_replicas (1..ZERO_MAX_RANKS) device
+ * pointers, each to this range's n values in one replica's full parameter buffer (a peer
+ * GPU's address where the replicas live on other GPUs, e.g. in NVLink-mapped symmetric memory;
+ * plain stores, no multicast), pairwise disjoint and checked against the step's other buffers
+ * like param_out. Same arithmetic, overflow flag and commit protocol as zero_step_fused; the
+ * commit of such a step is zero_step_commit_replicas (a void step's repair reaches every
+ * replica). Errors: as zero_step_fused, and ZERO_EINVAL for n_replicas outside 1..64, a null
+ * array or entry, or overlapping replicas. */
+zero_status zero_step_fused_replicas(uint64_t n, int nd, const uint16_t* const* rank_grads,
+                                     const float* master_in, const float* m_in, const float* v_in,
+                                     float* master_out, float* m_out, float* v_out,
+                                     int n_replicas, uint16_t* const* param_replicas,
+                                     const zero_adam_hparams* hp, int64_t step,
+                                     uint32_t* d_status, zero_stream_t stream);
+
+/* zero_step_commit for a step written with zero_step_fused_replicas: if the step is void, the
+ * inputs are copied over the outputs and fp16(master_in) is written into every replica. Errors:
+ * as zero_step_commit and zero_step_fused_replicas' replica checks. */
+zero_status zero_step_commit_replicas(uint64_t n, const float* master_in, const float* m_in,
+                                      const float* v_in, float* master_out, float* m_out,
+                                      float* v_out, int n_replicas,
+                                      uint16_t* const* param_replicas, uint32_t* d_status,
+                                      zero_stream_t stream);
+
 /* The calls of one step over several ranges (e.g. every bucket of a stage-1 step, in backward
  * order) as one call, so that a caller issuing many small calls pays one entry instead of one
  * per range. ranges[i] describes what zero_step_fused takes for range i (rank_grads: a host

@@ -467,3 +467,35 @@ def test_step_fused_q8_ranges_rejects_before_launching():
     assert lz.zero_kernel_launches() == before
     with pytest.raises(ValueError):
         lz.PreparedStepRanges(2, [good], "bf16")
+
+
+def test_step_fused_replicas_rejects_before_launching():
+    """The epilogue all-gather's replica list: 1..64 distinct, aligned ranges, each checked
+    like a param_out; anything else is refused with nothing launched."""
+    grads = [A + i * MB for i in range(2)]
+    ins = [A + 100 * MB, A + 101 * MB, A + 102 * MB]
+    outs = [A + 110 * MB, A + 111 * MB, A + 112 * MB]
+    st = A + 130 * MB
+    reps = [A + 120 * MB, A + 121 * MB, A + 122 * MB]
+    before = lz.zero_kernel_launches()
+    for replicas, code in [([], lz.ZERO_EINVAL),
+                           ([A + 120 * MB + 2 * k * 1000 for k in range(65)], lz.ZERO_EINVAL),
+                           (reps[:1] + [0], lz.ZERO_EINVAL),
+                           (reps[:1] + [A + 120 * MB + 500], lz.ZERO_EINVAL),   # overlapping
+                           (reps[:1] + [A + 110 * MB], lz.ZERO_EINVAL),         # on master_out
+                           (reps[:1] + [A + 123 * MB + 1], lz.ZERO_EALIGN)]:
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_step_fused_replicas(1000, 2, grads, *ins, *outs, replicas, HP, 1, st, 0)
+        assert e.value.code == code, replicas[:3]
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_step_commit_replicas(1000, *ins, *outs, replicas, st, 0)
+        assert e.value.code == code, replicas[:3]
+    with pytest.raises(lz.ZeroError) as e:     # a replica on a rank's gradient (the step only)
+        lz.zero_step_fused_replicas(1000, 2, grads, *ins, *outs, reps[:1] + [A + 1 * MB + 100],
+                                    HP, 1, st, 0)
+    assert e.value.code == lz.ZERO_EINVAL
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_step_fused_replicas(1000, 2, grads, *ins, *outs, reps, HP, 0, st, 0)   # t = 0
+    assert e.value.code == lz.ZERO_EINVAL
+    lz.zero_step_fused_replicas(0, 2, grads, *ins, *outs, reps, HP, 1, st, 0)   # nothing to do
+    assert lz.zero_kernel_launches() == before

@@ -31,7 +31,7 @@ def _case(numels):
     return psi, grad, master, m, v, torch
 
 
-def _worker(port, numels, bucket, out, peer=False, payload="fp16"):
+def _worker(port, numels, bucket, out, peer=False, payload="fp16", replicas=False):
     import datetime
     import torch
     import torch.distributed as dist
@@ -50,7 +50,19 @@ def _worker(port, numels, bucket, out, peer=False, payload="fp16"):
         st_out = [torch.full_like(x, float("nan")) for x in st_in]
         params = torch.zeros(psi, dtype=torch.float16, device=dev)
         status = torch.zeros(1, dtype=torch.int32, device=dev)
-        if peer and payload == "q8":   # int8 records quantized into symmetric memory
+        if replicas:   # the fp16 write-back stored by the kernel into symmetric memory
+            from zero_partitioned_optimizer_plan_b200.dist import SymmetricPeerBuffers
+            pp = SymmetricPeerBuffers(psi, torch.float16, dev)
+            pp.local.zero_()
+            gpeers = None
+            if peer:
+                gpeers = SymmetricPeerBuffers(psi, torch.float16, dev)
+                gpeers.local.copy_(grad.to(dev))
+            step = DistZeroStep(psi, bucket, peers=gpeers, param_peers=pp)
+            flag = step.step(gpeers.local if peer else grad.to(dev), st_in, st_out, pp.local,
+                             lz.AdamHP(), 1, status)
+            params = pp.local
+        elif peer and payload == "q8":   # int8 records quantized into symmetric memory
             from zero_partitioned_optimizer_plan_b200.dist import (SymmetricPeerBuffers,
                                                                    q8_peer_bytes)
             peers = SymmetricPeerBuffers(q8_peer_bytes(psi, bucket, 1), torch.uint8, dev)
@@ -133,3 +145,32 @@ def test_distributed_step_int8_payload_one_rank_nccl(bucket, peer):
     for name, got, want in zip(("master", "m", "v"), shard, (w, mm, vv)):
         assert int(oracle.ulp_diff_f32(got, want).max()) == 0, name
     assert int(oracle.ulp_diff_f16(params, p16).max()) == 0
+
+
+@pytest.mark.parametrize("peer", [False, True])
+@pytest.mark.parametrize("bucket", [0, 3000])
+def test_distributed_step_all_gather_in_epilogue_one_rank_nccl(bucket, peer):
+    """param_peers on one NCCL rank: the owner's kernel stores the fp16 values into the full
+    parameter buffer in torch symmetric memory (no all-gather collective), the gradients
+    exchanged by all-to-all or read in place from symmetric memory; against the oracle's
+    data-parallel step."""
+    import oracle
+    numels = [1000, 37, 4099, 12345]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_worker, args=(_free_port(), numels, bucket, q, peer, "fp16", True))
+    p.start()
+    try:
+        flag, status, shard, params = q.get(timeout=240)
+    finally:
+        p.join(60)
+        if p.exitcode is None:
+            p.kill()
+    assert p.exitcode == 0
+    psi, grad, master, m, v, _ = _case(numels)
+    ref = oracle.dp_step([grad.numpy()], master.numpy(), m.numpy(), v.numpy(),
+                         oracle.f2h(master.numpy()), oracle.AdamHP(), 1)
+    assert (flag, status) == (0, 0) and not ref.skipped
+    for name, got, want in zip(("master", "m", "v"), shard, (ref.master, ref.m, ref.v)):
+        assert int(oracle.ulp_diff_f32(got, want).max()) == 0, name
+    assert int(oracle.ulp_diff_f16(params, ref.params16).max()) == 0

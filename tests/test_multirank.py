@@ -161,6 +161,27 @@ class _OracleCompute:
         params.view(__import__("torch").int16).copy_(
             __import__("torch").from_numpy(np.ascontiguousarray(p16).view(np.int16)))
 
+    def fused_replicas(self, n, rows, state_in, state_out, replicas, hp, t, status):
+        import torch
+        own = torch.empty(n, dtype=torch.float16)
+        before = int(status.item())
+        self.fused(n, rows, state_in, state_out, own, hp, t, status)
+        if int(status.item()) == before:         # written: the all-gather in the epilogue
+            for rep in replicas:
+                rep.copy_(own)
+
+    def commit_replicas(self, n, state_in, state_out, replicas, status):
+        import numpy as np
+        import torch
+        import oracle
+        if int(status.item()) & (1 | 4 | 8):
+            for dst, src in zip(state_out, state_in):
+                dst.copy_(src)
+            p16 = torch.from_numpy(oracle.f2h(state_in[0].numpy()).view(np.int16))
+            for rep in replicas:
+                rep.view(torch.int16).copy_(p16)
+            status |= 2
+
     def quantize(self, n, grad, payload):
         import torch
         import oracle
@@ -574,3 +595,84 @@ def test_q8_peer_layout_tiles_every_part():
         spans.sort()
         assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
         assert spans[-1][1] <= total
+
+
+def _worker_dist_replicas(rank, ws, port, numels, bucket, bad_rank, gbufs, pbufs, fail_rank, out):
+    import datetime
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle
+    from zero_partitioned_optimizer_plan_b200.dist import (DistStepError, DistZeroStep,
+                                                           SharedPeerBuffers)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        psi_p, grads, master, m, v = _dist_case(numels, ws, bad_rank)
+        S = psi_p // ws
+        peers = SharedPeerBuffers(gbufs, rank)
+        peers.local.copy_(grads[rank])
+        params = SharedPeerBuffers(pbufs, rank)
+        st_in = [x[rank * S:(rank + 1) * S].clone() for x in (master, m, v)]
+        st_out = [torch.full_like(x, float("nan")) for x in st_in]
+        status = torch.zeros(1, dtype=torch.int32)
+        step = DistZeroStep(psi_p, bucket, compute=_OracleCompute(fail=rank == fail_rank),
+                            peers=peers, param_peers=params)
+        raised = 0
+        try:
+            flag = int(step.step(peers.local, st_in, st_out, params.local, oracle.AdamHP(), 1,
+                                 status).item())
+        except DistStepError as e:
+            flag, raised = e.bits, 1
+        out.put((rank, flag, int(status.item()), [x.numpy() for x in st_out],
+                 params.local.numpy().view("uint16").copy(), raised))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("ws,bucket,bad_rank,fail_rank", [(2, 0, -1, -1), (3, 2500, -1, -1),
+                                                          (3, 2500, 1, -1), (3, 2500, -1, 2)])
+def test_distributed_step_all_gather_in_epilogue_gloo(ws, bucket, bad_rank, fail_rank):
+    """param_peers: each owner's step writes its fp16 values into every rank's full parameter
+    buffer (CPU tensors shared by the processes, standing for NVLink peer mappings), with no
+    all-gather collective. Every rank's full buffer equals the oracle's data-parallel step; an
+    inf on one rank leaves fp16(master) in every replica (the commit repairs them all); a
+    failure reported by one rank's kernels raises on every rank after the same repair."""
+    import numpy as np
+    import torch
+    import oracle
+    numels = [1000, 37, 4099, 12345]
+    psi_p = -(-sum(numels) // ws) * ws
+    _, _, master0, _, _ = _dist_case(numels, ws, bad_rank)
+    p0 = torch.from_numpy(oracle.f2h(master0.numpy()).view(np.int16)).view(torch.float16)
+    gbufs = [torch.zeros(psi_p, dtype=torch.float16).share_memory_() for _ in range(ws)]
+    pbufs = [p0.clone().share_memory_() for _ in range(ws)]   # every replica starts at fp16(master)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_dist_replicas,
+                         args=(r, ws, port, numels, bucket, bad_rank, gbufs, pbufs, fail_rank, q))
+             for r in range(ws)]
+    for p in procs:
+        p.start()
+    try:
+        res = sorted((q.get(timeout=240) for _ in range(ws)), key=lambda x: x[0])
+    finally:
+        for p in procs:
+            p.join(60)
+            if p.exitcode is None:
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    psi_p, grads, master, m, v = _dist_case(numels, ws, bad_rank)
+    ref = oracle.dp_step([g.numpy() for g in grads], master.numpy(), m.numpy(), v.numpy(),
+                         oracle.f2h(master.numpy()), oracle.AdamHP(), 1)
+    S = psi_p // ws
+    void = ref.skipped or fail_rank >= 0
+    for rank, flag, status, shard, params, raised in res:
+        assert raised == (1 if fail_rank >= 0 else 0)
+        assert bool(status & 2) == void
+        want = (master.numpy(), m.numpy(), v.numpy()) if void else (ref.master, ref.m, ref.v)
+        for got, w in zip(shard, want):
+            assert np.array_equal(got.view(np.uint32), w[rank * S:(rank + 1) * S].view(np.uint32))
+        assert np.array_equal(params, oracle.f2h(master.numpy()) if void else ref.params16)

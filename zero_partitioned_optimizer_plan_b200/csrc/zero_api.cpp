@@ -274,6 +274,60 @@ static zero_status check_fused(uint64_t n, int nd, const uint16_t* const* rank_g
     return ZERO_OK;
 }
 
+// The replica list of the epilogue all-gather: 1..ZERO_MAX_RANKS distinct ranges, each
+// checked like a param_out against the step's other buffers (rank_grads may be null: commit).
+static zero_status check_replicas(uint64_t n, int nd, const uint16_t* const* rank_grads,
+                                  const float* master_in, const float* m_in, const float* v_in,
+                                  float* master_out, float* m_out, float* v_out, int n_replicas,
+                                  uint16_t* const* replicas, uint32_t* d_status) {
+    if (n_replicas < 1 || n_replicas > ZERO_MAX_RANKS || !replicas || !d_status)
+        return ZERO_EINVAL;
+    if (n == 0) return ZERO_OK;
+    for (int d = 0; d < n_replicas; ++d) {
+        const zero_status st =
+            rank_grads ? check_fused(n, nd, rank_grads, master_in, m_in, v_in, master_out, m_out,
+                                     v_out, replicas[d], d_status)
+                       : zk::check_fused_state(n, master_in, m_in, v_in, master_out, m_out,
+                                               v_out, replicas[d], d_status);
+        if (st != ZERO_OK) return st;
+        for (int e = 0; e < d; ++e)
+            if (zk::overlap(replicas[e], n * 2, replicas[d], n * 2)) return ZERO_EINVAL;
+    }
+    return ZERO_OK;
+}
+
+zero_status zero_step_fused_replicas(uint64_t n, int nd, const uint16_t* const* rank_grads,
+                                     const float* master_in, const float* m_in, const float* v_in,
+                                     float* master_out, float* m_out, float* v_out,
+                                     int n_replicas, uint16_t* const* param_replicas,
+                                     const zero_adam_hparams* hp, int64_t step,
+                                     uint32_t* d_status, zero_stream_t stream) {
+    if (!zk::hparams_ok(hp) || step < 1 || nd < 1 || nd > ZERO_MAX_RANKS) return ZERO_EINVAL;
+    if (n > 0 && !rank_grads) return ZERO_EINVAL;
+    const zero_status st = check_replicas(n, nd, rank_grads, master_in, m_in, v_in,
+                                          master_out, m_out, v_out, n_replicas, param_replicas,
+                                          d_status);
+    if (st != ZERO_OK || n == 0) return st;
+    return zk::from_cuda(zk::launch_fused(n, nd, rank_grads, master_in, m_in, v_in, master_out,
+                                          m_out, v_out, param_replicas[0],
+                                          zk::make_adam(hp, step), nullptr, zk::make_mean(nd),
+                                          d_status, (cudaStream_t)stream, n_replicas,
+                                          param_replicas));
+}
+
+zero_status zero_step_commit_replicas(uint64_t n, const float* master_in, const float* m_in,
+                                      const float* v_in, float* master_out, float* m_out,
+                                      float* v_out, int n_replicas,
+                                      uint16_t* const* param_replicas, uint32_t* d_status,
+                                      zero_stream_t stream) {
+    const zero_status st = check_replicas(n, 1, nullptr, master_in, m_in, v_in, master_out, m_out,
+                                          v_out, n_replicas, param_replicas, d_status);
+    if (st != ZERO_OK || n == 0) return st;
+    return zk::from_cuda(zk::launch_commit(n, master_in, m_in, v_in, master_out, m_out, v_out,
+                                           param_replicas[0], d_status, (cudaStream_t)stream,
+                                           n_replicas, param_replicas));
+}
+
 zero_status zero_step_fused(uint64_t n, int nd, const uint16_t* const* rank_grads,
                             const float* master_in, const float* m_in, const float* v_in,
                             float* master_out, float* m_out, float* v_out, uint16_t* param_out,

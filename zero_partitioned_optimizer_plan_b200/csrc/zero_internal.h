@@ -31,10 +31,14 @@ cudaError_t launch_fused(uint64_t n, int nd, const uint16_t* const* grads, const
                          const float* m_in, const float* v_in, float* master_out, float* m_out,
                          float* v_out, uint16_t* param_out, const AdamConsts& a,
                          const AdamConsts* ad, const MeanConsts& mc, uint32_t* status,
-                         cudaStream_t stream);
+                         cudaStream_t stream, int n_replicas = 0,
+                         uint16_t* const* replicas = nullptr);
+// n_replicas > 0: the fp16 write-back (and the commit's repair) goes to every replicas[d]
+// instead of param_out (the all-gather in the epilogue).
 cudaError_t launch_commit(uint64_t n, const float* master_in, const float* m_in,
                           const float* v_in, float* master_out, float* m_out, float* v_out,
-                          uint16_t* param_out, uint32_t* status, cudaStream_t stream);
+                          uint16_t* param_out, uint32_t* status, cudaStream_t stream,
+                          int n_replicas = 0, uint16_t* const* replicas = nullptr);
 cudaError_t launch_reduce_scatter(uint64_t n, int nd, const uint16_t* const* grads,
                                   float* const* shards, uint64_t flat_lo, uint64_t shard,
                                   const MeanConsts& mc, uint32_t* status, cudaStream_t stream);

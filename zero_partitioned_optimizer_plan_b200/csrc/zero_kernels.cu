@@ -61,7 +61,21 @@ struct FusedArgs {
     MeanConsts mc;
     int selftest_no_copies;  // self-test only: the producer issues nothing (waits must expire)
     int chained;         // programmatic launch chained to the previous call (see pdl_enter)
+    // the all-gather in the epilogue: when n_replicas > 0 the fp16 values go to every replica's
+    // buffer (replicas[d], possibly a peer's address) instead of param_out
+    int n_replicas;
+    uint16_t* replicas[kMaxRanks];
 };
+
+// The fp16 write-back of one value: into param_out, or into every replica.
+__device__ __forceinline__ void store_param(const FusedArgs& p, uint64_t i, float w) {
+    const uint16_t h = f2h(w);
+    if (p.n_replicas == 0) {
+        p.param_out[i] = h;
+        return;
+    }
+    for (int d = 0; d < p.n_replicas; ++d) p.replicas[d][i] = h;
+}
 
 struct RsArgs {
     const uint16_t* grads[kMaxRanks];
@@ -89,6 +103,8 @@ struct CommitArgs {
     uint16_t* param_out;
     uint32_t* status;
     uint64_t n;
+    int n_replicas;                  // > 0: restore every replica's range instead of param_out
+    uint16_t* replicas[kMaxRanks];
 };
 
 struct AdamArgs {
@@ -196,7 +212,7 @@ __device__ __forceinline__ void fused_element(const FusedArgs& p, const AdamCons
     p.master_out[i] = w;
     p.m_out[i] = m;
     p.v_out[i] = v;
-    p.param_out[i] = f2h(w);
+    store_param(p, i, w);
 }
 
 template <int E, int W, bool kDC>
@@ -253,7 +269,11 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
         stg_f32<E>(p.master_out + g0, w);
         stg_f32<E>(p.m_out + g0, m);
         stg_f32<E>(p.v_out + g0, v);
-        stg_f16<E>(p.param_out + g0, w, p.param_vec);
+        if (p.n_replicas == 0) {
+            stg_f16<E>(p.param_out + g0, w, p.param_vec);
+        } else {
+            for (int d = 0; d < p.n_replicas; ++d) stg_f16<E>(p.replicas[d] + g0, w, p.param_vec);
+        }
     }
     // the < 8 elements past the last tile
     if (blockIdx.x == 0 && (uint64_t)threadIdx.x < p.n - p.n_tiled)
@@ -456,7 +476,12 @@ __global__ void __launch_bounds__(256) commit_kernel(const __grid_constant__ Com
         p.master_out[i] = w;
         p.m_out[i] = p.m_in[i];
         p.v_out[i] = p.v_in[i];
-        p.param_out[i] = f2h(w);
+        const uint16_t h = f2h(w);
+        if (p.n_replicas == 0) {
+            p.param_out[i] = h;
+        } else {
+            for (int d = 0; d < p.n_replicas; ++d) p.replicas[d][i] = h;
+        }
     }
 }
 
@@ -594,7 +619,7 @@ cudaError_t launch_fused(uint64_t n, int nd, const uint16_t* const* grads, const
                          const float* m_in, const float* v_in, float* master_out, float* m_out,
                          float* v_out, uint16_t* param_out, const AdamConsts& a,
                          const AdamConsts* ad, const MeanConsts& mc, uint32_t* status,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, int n_replicas, uint16_t* const* replicas) {
     FusedArgs p;
     memset(&p, 0, sizeof(p));
     bool all16 = aligned16(master_in) && aligned16(m_in) && aligned16(v_in) &&
@@ -614,6 +639,12 @@ cudaError_t launch_fused(uint64_t n, int nd, const uint16_t* const* grads, const
     p.n = n;
     p.nd = nd;
     p.param_vec = store_vec(param_out);
+    p.n_replicas = n_replicas;
+    for (int d = 0; d < n_replicas; ++d) {   // one store width that every replica allows
+        p.replicas[d] = replicas[d];
+        const int v = store_vec(replicas[d]);
+        if (d == 0 || v < p.param_vec) p.param_vec = v;
+    }
     p.a = a;
     p.ad = ad;
     p.mc = mc;
@@ -715,8 +746,12 @@ cudaError_t launch_scaler_update(zero_scaler_state* st, const zero_scaler_params
 
 cudaError_t launch_commit(uint64_t n, const float* master_in, const float* m_in,
                           const float* v_in, float* master_out, float* m_out, float* v_out,
-                          uint16_t* param_out, uint32_t* status, cudaStream_t stream) {
+                          uint16_t* param_out, uint32_t* status, cudaStream_t stream,
+                          int n_replicas, uint16_t* const* replicas) {
     CommitArgs p;
+    memset(&p, 0, sizeof(p));
+    p.n_replicas = n_replicas;
+    for (int d = 0; d < n_replicas; ++d) p.replicas[d] = replicas[d];
     p.master_in = master_in;
     p.m_in = m_in;
     p.v_in = v_in;

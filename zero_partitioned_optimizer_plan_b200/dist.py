@@ -56,6 +56,15 @@ its own peer buffer at an offset every rank computes alike, and the owner's kern
 Nd payloads of its part in the peers' buffers (per bucket the same barrier as the fp16 peer
 reads); nothing is exchanged but the barriers.
 
+All-gather in the epilogue (``param_peers``: every rank's full fp16 parameter buffer,
+addressable from every rank, e.g. in torch symmetric memory). The owner's fused step stores each
+updated fp16 value straight into every replica's buffer (the library's
+zero_step_fused_replicas: plain stores to the peers' addresses over NVLink, no multicast), so the
+step's write-back needs no all-gather collective. The job-wide verdict then decides the commit,
+which on a void step writes the restored values into every replica as well
+(zero_step_commit_replicas); a barrier after the commits ends the step, so no rank reads its
+parameters while an owner still writes them.
+
 The collectives are torch.distributed calls (NCCL on GPUs, gloo on CPUs); the arithmetic is the
 library's. ``compute`` replaces the library calls (the tests run the exchange on CPU
 processes with another implementation of them).
@@ -178,6 +187,13 @@ class LibzeroCompute:
     def quantize(self, n, grad, payload):
         self.lz.zero_quantize_q8(n, grad, payload)
 
+    def fused_replicas(self, n, rows, state_in, state_out, replicas, hp, t, status):
+        self.lz.zero_step_fused_replicas(n, len(rows), rows, *state_in, *state_out, replicas, hp,
+                                         t, status)
+
+    def commit_replicas(self, n, state_in, state_out, replicas, status):
+        self.lz.zero_step_commit_replicas(n, *state_in, *state_out, replicas, status)
+
     def fused_q8(self, n, payloads, state_in, state_out, params, hp, t, status):
         self.lz.zero_step_fused_q8(n, len(payloads), payloads, *state_in, *state_out, params, hp,
                                    t, status)
@@ -189,7 +205,7 @@ class DistZeroStep:
     (the gradients themselves are exchanged) or "q8" (int8 records, all-to-all form only)."""
 
     def __init__(self, psi_p: int, bucket: int = 0, group=None, compute=None, peers=None,
-                 payload: str = "fp16"):
+                 payload: str = "fp16", param_peers=None):
         import torch.distributed as dist
         self.dist = dist
         self.group = group
@@ -205,6 +221,9 @@ class DistZeroStep:
         if payload not in ("fp16", "q8"):
             raise ValueError(f"payload {payload!r}")
         self.payload = payload
+        if param_peers is not None and payload != "fp16":
+            raise ValueError("the epilogue all-gather runs with the fp16 payload")
+        self.param_peers = param_peers
         if payload == "q8" and peers is not None:
             self._q8_offs, need = q8_peer_layout(psi_p, bucket, self.nd)
             if peers.local.numel() * peers.local.element_size() < need:
@@ -237,7 +256,7 @@ class DistZeroStep:
             self._masks = torch.tensor(VOID_BITS, dtype=status.dtype, device=status.device)
             self._bits = torch.empty_like(self._masks)
             self._tick = torch.zeros(1, dtype=status.dtype, device=status.device)
-        if not self.in_place_gather and (
+        if self.param_peers is None and not self.in_place_gather and (
                 self._gather_src is None or self._gather_src.device != params_full.device):
             self._gather_src = torch.empty(self.shard, dtype=params_full.dtype,
                                            device=params_full.device)
@@ -251,8 +270,11 @@ class DistZeroStep:
         this rank's zeroed int32 status word, which ends with the job-wide void bits and, if
         any is set, the skipped bit (every rank agrees). Returns the job-wide void bits (a
         one-element tensor on the status word's device; 1 = overflow). Raises DistStepError on
-        every rank if any rank's kernels failed."""
+        every rank if any rank's kernels failed. With param_peers, params_full is this rank's
+        buffer among them (param_peers.local), written by every owner's kernel."""
         dist, nd, r, S = self.dist, self.nd, self.rank, self.shard
+        if self.param_peers is not None and params_full is not self.param_peers.local:
+            raise ValueError("with param_peers, params_full is param_peers.local")
         recv = self._buffers(local_grad, params_full, status)
         own = params_full[r * S:(r + 1) * S]
         nb = len(self.buckets)
@@ -310,8 +332,18 @@ class DistZeroStep:
                 self.compute.fused_q8(mine, pays, ins, outs, own[a:a + mine], hp, t, status)
             else:
                 rows = [buf[j * mine:(j + 1) * mine] for j in range(nd)]
-                self.compute.fused(mine, rows, ins, outs, own[a:a + mine], hp, t, status)
+                self._update(mine, rows, ins, outs, own, a, hp, t, status)
         return self._finish(state_in, state_out, own, params_full, status)
+
+    def _update(self, n, rows, ins, outs, own, a, hp, t, status):
+        """The owner's fused step over its part [a, a + n) of its shard: the fp16 values into
+        its own range, or (param_peers) into every replica's buffer."""
+        if self.param_peers is None:
+            self.compute.fused(n, rows, ins, outs, own[a:a + n], hp, t, status)
+            return
+        lo = self.rank * self.shard + a
+        self.compute.fused_replicas(n, rows, ins, outs, self.param_peers.rows(lo, lo + n), hp,
+                                    t, status)
 
     def _reduce_from_peers(self, state_in, state_out, own, hp, t, status):
         """Per bucket: a barrier (every rank has produced it), then the owner's fused step on
@@ -333,10 +365,10 @@ class DistZeroStep:
             a, b = max(lo, r * S), min(hi, (r + 1) * S)     # my part of the bucket
             if a >= b:
                 continue
-            self.compute.fused(b - a, self.peers.rows(a, b),
-                               [x[a - r * S:b - r * S] for x in state_in],
-                               [x[a - r * S:b - r * S] for x in state_out],
-                               own[a - r * S:b - r * S], hp, t, status)
+            self._update(b - a, self.peers.rows(a, b),
+                         [x[a - r * S:b - r * S] for x in state_in],
+                         [x[a - r * S:b - r * S] for x in state_out], own, a - r * S, hp, t,
+                         status)
 
     def _reduce_q8_from_peers(self, local_grad, state_in, state_out, own, hp, t, status):
         """Per bucket: quantize this rank's part for every owner into its own peer buffer, a
@@ -380,6 +412,16 @@ class DistZeroStep:
         dist.all_reduce(self._bits, op=dist.ReduceOp.MAX, group=self.group)
         flag = self._bits.sum(dim=0, keepdim=True)
         status.bitwise_or_(flag)
+        if self.param_peers is not None:
+            r = self.rank
+            self.compute.commit_replicas(S, state_in, state_out,
+                                         self.param_peers.rows(r * S, (r + 1) * S), status)
+            # every owner's stores into this rank's buffer (step and repair) are done past here
+            dist.all_reduce(self._tick, group=self.group)
+            bits = int(flag.item())
+            if bits & ERROR_BITS:
+                raise DistStepError(bits)
+            return flag
         self.compute.commit(S, state_in, state_out, own, status)
         bits = int(flag.item())
         if bits & ERROR_BITS:

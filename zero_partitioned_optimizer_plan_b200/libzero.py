@@ -51,6 +51,7 @@ SYMBOLS = (
     "zero_overlap_begin", "zero_overlap_end",
     "zero_gather_params", "zero_stage3_step_fused", "zero_stage3_step_commit",
     "zero_step_fused_ranges", "zero_step_fused_q8_ranges",
+    "zero_step_fused_replicas", "zero_step_commit_replicas",
     "zero_sched_slot_elems", "zero_sched_create", "zero_sched_create_fused",
     "zero_sched_begin_bucket", "zero_sched_rebind_fused", "zero_sched_rebind_status",
     "zero_sched_end_bucket", "zero_sched_wait", "zero_sched_launches", "zero_sched_destroy",
@@ -168,6 +169,9 @@ def _load():
     L.zero_scaler_update.argtypes = [vp, P(ScalerParams), vp, vp]
     L.zero_step_fused_ranges.argtypes = [i32, i32, P(FusedRange), P(_HP), i64, vp, i32, vp]
     L.zero_step_fused_q8_ranges.argtypes = [i32, i32, P(FusedQ8Range), P(_HP), i64, vp, i32, vp]
+    L.zero_step_fused_replicas.argtypes = [u64, i32, P(vp), vp, vp, vp, vp, vp, vp, i32, P(vp),
+                                           P(_HP), i64, vp, vp]
+    L.zero_step_commit_replicas.argtypes = [u64, vp, vp, vp, vp, vp, vp, i32, P(vp), vp, vp]
     L.zero_gather_params.argtypes = [vp, u64, u64, P(vp), vp, vp, vp]
     L.zero_stage3_step_fused.argtypes = [vp, u64, u64, P(vp), vp, vp, vp, vp, vp, vp, P(vp), P(_HP),
                                    i64, vp, vp]
@@ -364,6 +368,28 @@ def zero_step_fused_ranges(nd: int, ranges, hp: AdamHP, step: int, d_status, ove
                            stream=None):
     PreparedStepRanges(nd, ranges)(hparams_ref(hp), step, _ptr(d_status, 4), overlap,
                                    _stream(stream))
+
+
+def zero_step_fused_replicas(n: int, nd: int, rank_grads, master_in, m_in, v_in, master_out, m_out,
+                             v_out, replicas, hp: AdamHP, step: int, d_status, stream=None):
+    """zero_step_fused with the fp16 write-back stored into every replica (the all-gather in the
+    epilogue); replicas: tensors or device addresses of this range in each replica."""
+    h = hp._c()
+    _check(_lib.zero_step_fused_replicas(n, nd, _ptr_array(rank_grads, 2), _ptr(master_in, 4),
+                                         _ptr(m_in, 4), _ptr(v_in, 4), _ptr(master_out, 4),
+                                         _ptr(m_out, 4), _ptr(v_out, 4), len(replicas),
+                                         _ptr_array(replicas, 2), C.byref(h), step,
+                                         _ptr(d_status, 4), _stream(stream)),
+           "zero_step_fused_replicas")
+
+
+def zero_step_commit_replicas(n: int, master_in, m_in, v_in, master_out, m_out, v_out, replicas,
+                              d_status, stream=None):
+    _check(_lib.zero_step_commit_replicas(n, _ptr(master_in, 4), _ptr(m_in, 4), _ptr(v_in, 4),
+                                          _ptr(master_out, 4), _ptr(m_out, 4), _ptr(v_out, 4),
+                                          len(replicas), _ptr_array(replicas, 2),
+                                          _ptr(d_status, 4), _stream(stream)),
+           "zero_step_commit_replicas")
 
 
 def zero_step_fused_q8_ranges(nd: int, ranges, hp: AdamHP, step: int, d_status, overlap=True,
