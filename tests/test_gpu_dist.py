@@ -174,3 +174,72 @@ def test_distributed_step_all_gather_in_epilogue_one_rank_nccl(bucket, peer):
     for name, got, want in zip(("master", "m", "v"), shard, (ref.master, ref.m, ref.v)):
         assert int(oracle.ulp_diff_f32(got, want).max()) == 0, name
     assert int(oracle.ulp_diff_f16(params, ref.params16).max()) == 0
+
+
+def _worker_stage3(port, numels, layer_tensors, out):
+    import datetime
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle
+    from zero_partitioned_optimizer_plan_b200 import libzero as lz
+    from zero_partitioned_optimizer_plan_b200.dist import DistStage3Step, SymmetricPeerBuffers
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.cuda.set_device(0)
+    dist.init_process_group("nccl", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        psi, grad, master, m, v, _ = _case(numels)
+        dev = "cuda:0"
+        parts = SymmetricPeerBuffers(psi, torch.float16, dev)
+        parts.local.copy_(torch.from_numpy(oracle.f2h(master.numpy()).view("float16")).to(dev))
+        st_in = [x.to(dev) for x in (master, m, v)]
+        st_out = [torch.full_like(x, float("nan")) for x in st_in]
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        step = DistStage3Step(numels, layer_tensors, parts)
+        layer_buf = torch.zeros(max(hi - lo for lo, hi in step.layers), dtype=torch.float16,
+                                device=dev)
+        rec = []
+        flag = step.step(grad.to(dev), st_in, st_out, lz.AdamHP(), 1, status, layer_buf, rec)
+        torch.cuda.synchronize()
+        out.put((int(flag.item()), int(status.item()), [x.cpu().numpy() for x in st_out],
+                 parts.local.cpu().numpy().view(np.uint16),
+                 [r.cpu().numpy().view(np.uint16) for r in rec]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_distributed_stage3_one_rank_nccl():
+    """DistStage3Step on one NCCL rank: the partition in torch symmetric memory, each layer
+    gathered by the library's gather kernel from the owner's partition address, the layers'
+    gradient buckets exchanged and the owner's update written into its partition; gathered
+    layers, partition and state against the oracle's zero3_step (0 ulp)."""
+    import oracle
+    numels, layer_tensors = [1000, 37, 4099, 12345], [1, 2, 1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_worker_stage3, args=(_free_port(), numels, layer_tensors, q))
+    p.start()
+    try:
+        flag, status, shard, part, rec = q.get(timeout=240)
+    finally:
+        p.join(60)
+        if p.exitcode is None:
+            p.kill()
+    assert p.exitcode == 0
+    psi, grad, master, m, v, _ = _case(numels)
+    pl = oracle.plan(numels, 1)
+    layers = oracle.layer_ranges(pl, layer_tensors)
+    buckets = oracle.grad_buckets(pl, layers)
+    ref = oracle.zero3_step(pl, layers, lambda l, j: grad.numpy()[buckets[l][0]:buckets[l][1]],
+                            master.numpy(), m.numpy(), v.numpy(),
+                            [oracle.f2h(master.numpy())], oracle.AdamHP(), 1)
+    assert (flag, status) == (0, 0) and not ref.skipped
+    for name, got, want in zip(("master", "m", "v"), shard, (ref.master, ref.m, ref.v)):
+        assert int(oracle.ulp_diff_f32(got, want).max()) == 0, name
+    assert int(oracle.ulp_diff_f16(part, ref.param_shards[0]).max()) == 0
+    L = len(layers)
+    for l in range(L):
+        assert np.array_equal(rec[l], ref.gathered_fwd[l])
+        assert np.array_equal(rec[L + (L - 1 - l)], ref.gathered_bwd[l])

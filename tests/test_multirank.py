@@ -161,6 +161,13 @@ class _OracleCompute:
         params.view(__import__("torch").int16).copy_(
             __import__("torch").from_numpy(np.ascontiguousarray(p16).view(np.int16)))
 
+    def gather(self, numels, nd, lo, n, partitions, out, status):
+        import torch
+        import oracle
+        S = partitions[0].numel()
+        g = oracle.gather_params([p.numpy() for p in partitions], S, lo, lo + n)
+        out.view(torch.int16).copy_(torch.from_numpy(g.view("int16")))
+
     def fused_replicas(self, n, rows, state_in, state_out, replicas, hp, t, status):
         import torch
         own = torch.empty(n, dtype=torch.float16)
@@ -676,3 +683,90 @@ def test_distributed_step_all_gather_in_epilogue_gloo(ws, bucket, bad_rank, fail
         for got, w in zip(shard, want):
             assert np.array_equal(got.view(np.uint32), w[rank * S:(rank + 1) * S].view(np.uint32))
         assert np.array_equal(params, oracle.f2h(master.numpy()) if void else ref.params16)
+
+
+S3_NUMELS = [1000, 37, 4099, 12345, 6000, 7]
+S3_LAYERS = [1, 2, 1, 2]
+
+
+def _worker_stage3(rank, ws, port, bad_rank, pbufs, out):
+    import datetime
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle
+    from zero_partitioned_optimizer_plan_b200.dist import DistStage3Step, SharedPeerBuffers
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        psi_p, grads, master, m, v = _dist_case(S3_NUMELS, ws, bad_rank)
+        S = psi_p // ws
+        parts = SharedPeerBuffers(pbufs, rank)
+        st_in = [x[rank * S:(rank + 1) * S].clone() for x in (master, m, v)]
+        st_out = [torch.full_like(x, float("nan")) for x in st_in]
+        status = torch.zeros(1, dtype=torch.int32)
+        step = DistStage3Step(S3_NUMELS, S3_LAYERS, parts, compute=_OracleCompute())
+        big = max(hi - lo for lo, hi in step.layers)
+        layer_buf = torch.zeros(big, dtype=torch.float16)
+        rec = []
+        flag = step.step(grads[rank], st_in, st_out, oracle.AdamHP(), 1, status, layer_buf, rec)
+        dist.barrier()    # every owner's partition is final before it is read back
+        out.put((rank, int(flag.item()), int(status.item()), [x.numpy() for x in st_out],
+                 [p.numpy().view(np.uint16).copy() for p in parts.tensors],
+                 [r.numpy().view(np.uint16) for r in rec]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("ws,bad_rank", [(2, -1), (3, -1), (3, 1)])
+def test_distributed_stage3_gloo(ws, bad_rank):
+    """DistStage3Step on gloo ranks, the partitions in CPU tensors shared by the processes
+    (standing for NVLink peer mappings): every gathered layer (forward and backward), every
+    owner's final partition and state shard equal the oracle's stage-3 step (zero3_step) bit
+    for bit; an inf on one rank skips the step everywhere and leaves the partitions as they
+    were."""
+    import numpy as np
+    import torch
+    import oracle
+    psi_p, grads, master, m, v = _dist_case(S3_NUMELS, ws, bad_rank)
+    S = psi_p // ws
+    p16 = oracle.f2h(master.numpy())
+    pbufs = [torch.from_numpy(p16[q * S:(q + 1) * S].copy().view(np.int16)).view(torch.float16)
+             .share_memory_() for q in range(ws)]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_stage3, args=(r, ws, port, bad_rank, pbufs, q))
+             for r in range(ws)]
+    for p in procs:
+        p.start()
+    try:
+        res = sorted((q.get(timeout=240) for _ in range(ws)), key=lambda x: x[0])
+    finally:
+        for p in procs:
+            p.join(60)
+            if p.exitcode is None:
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    pl = oracle.plan(S3_NUMELS, ws)
+    layers = oracle.layer_ranges(pl, S3_LAYERS)
+    buckets = oracle.grad_buckets(pl, layers)
+    ref = oracle.zero3_step(pl, layers,
+                            lambda l, j: grads[j].numpy()[buckets[l][0]:buckets[l][1]],
+                            master.numpy(), m.numpy(), v.numpy(),
+                            [p16[q * S:(q + 1) * S] for q in range(ws)], oracle.AdamHP(), 1)
+    assert ref.skipped == (bad_rank >= 0)
+    L = len(layers)
+    for rank, flag, status, shard, parts, rec in res:
+        assert flag == (1 if ref.skipped else 0)
+        assert bool(status & 2) == ref.skipped
+        for got, want in zip(shard, (ref.master, ref.m, ref.v)):
+            assert np.array_equal(got.view(np.uint32), want[rank * S:(rank + 1) * S].view(np.uint32))
+        for qq in range(ws):
+            assert np.array_equal(parts[qq], ref.param_shards[qq].view(np.uint16))
+        assert len(rec) == 2 * L
+        for l in range(L):
+            assert np.array_equal(rec[l], ref.gathered_fwd[l])
+            assert np.array_equal(rec[L + (L - 1 - l)], ref.gathered_bwd[l])

@@ -187,6 +187,15 @@ class LibzeroCompute:
     def quantize(self, n, grad, payload):
         self.lz.zero_quantize_q8(n, grad, payload)
 
+    def gather(self, numels, nd, lo, n, partitions, out, status):
+        """Layer [lo, lo + n) out of the owners' partitions (one address or tensor per owner)
+        into out, with the library's gather kernel (a plan of the list, made once)."""
+        key = (tuple(numels), nd)
+        if getattr(self, "_plan_key", None) != key:
+            self._plan = self.lz.zero_plan_create(list(numels), nd, 3, 0)
+            self._plan_key = key
+        self.lz.zero_gather_params(self._plan, lo, n, partitions, out, status)
+
     def fused_replicas(self, n, rows, state_in, state_out, replicas, hp, t, status):
         self.lz.zero_step_fused_replicas(n, len(rows), rows, *state_in, *state_out, replicas, hp,
                                          t, status)
@@ -205,7 +214,7 @@ class DistZeroStep:
     (the gradients themselves are exchanged) or "q8" (int8 records, all-to-all form only)."""
 
     def __init__(self, psi_p: int, bucket: int = 0, group=None, compute=None, peers=None,
-                 payload: str = "fp16", param_peers=None):
+                 payload: str = "fp16", param_peers=None, buckets=None, partitioned=False):
         import torch.distributed as dist
         self.dist = dist
         self.group = group
@@ -215,7 +224,14 @@ class DistZeroStep:
             raise ValueError("psi_p must be a multiple of the world size")
         self.psi_p = psi_p
         self.shard = psi_p // self.nd
-        self.buckets = bucket_ranges(psi_p, bucket)
+        # buckets: the gradient buckets in the order the backward pass produces them (default:
+        # element-granular buckets of `bucket` values from the end); partitioned: the fp16
+        # parameters are partitioned too (stage 3): params_full is this rank's partition of S
+        # values and nothing is gathered after the step
+        self.buckets = list(buckets) if buckets is not None else bucket_ranges(psi_p, bucket)
+        self.partitioned = partitioned
+        if partitioned and param_peers is not None:
+            raise ValueError("a partitioned step keeps its parameters on their owners")
         self.parts = [owner_parts(lo, hi, self.shard, self.nd) for lo, hi in self.buckets]
         self.compute = compute or LibzeroCompute()
         if payload not in ("fp16", "q8"):
@@ -256,7 +272,7 @@ class DistZeroStep:
             self._masks = torch.tensor(VOID_BITS, dtype=status.dtype, device=status.device)
             self._bits = torch.empty_like(self._masks)
             self._tick = torch.zeros(1, dtype=status.dtype, device=status.device)
-        if self.param_peers is None and not self.in_place_gather and (
+        if self.param_peers is None and not self.partitioned and not self.in_place_gather and (
                 self._gather_src is None or self._gather_src.device != params_full.device):
             self._gather_src = torch.empty(self.shard, dtype=params_full.dtype,
                                            device=params_full.device)
@@ -276,7 +292,7 @@ class DistZeroStep:
         if self.param_peers is not None and params_full is not self.param_peers.local:
             raise ValueError("with param_peers, params_full is param_peers.local")
         recv = self._buffers(local_grad, params_full, status)
-        own = params_full[r * S:(r + 1) * S]
+        own = params_full if self.partitioned else params_full[r * S:(r + 1) * S]
         nb = len(self.buckets)
         works = [None] * nb
         if self.peers is not None:
@@ -426,9 +442,81 @@ class DistZeroStep:
         bits = int(flag.item())
         if bits & ERROR_BITS:
             raise DistStepError(bits)
+        if self.partitioned:    # stage 3: the owners keep their partitions
+            return flag
         if self.in_place_gather:
             dist.all_gather_into_tensor(params_full, own, group=self.group)
         else:
             self._gather_src.copy_(own)
             dist.all_gather_into_tensor(params_full, self._gather_src, group=self.group)
         return flag
+
+
+def layer_ranges(numels: Sequence[int], layer_tensors: Sequence[int]) -> List[Tuple[int, int]]:
+    """Flat ranges of the layers in forward order: layer l is the next layer_tensors[l]
+    tensors of the flattened list."""
+    if sum(layer_tensors) != len(numels) or any(c < 1 for c in layer_tensors):
+        raise ValueError("layer_tensors must split the tensor list into non-empty runs")
+    out, i, off = [], 0, 0
+    for c in layer_tensors:
+        n = sum(numels[i:i + c])
+        out.append((off, off + n))
+        off += n
+        i += c
+    return out
+
+
+class DistStage3Step:
+    """Stage 3 across processes. "ZeRO: particionar estados do treino entre GPUs"
+    (upskillscore.com), "Como funciona": the fp16 parameters are partitioned among the ranks
+    too, a rank receives the partitions it needs from their owners, and a step moves 3 psi: a
+    parameter all-gather in the forward pass, another in the backward pass, the gradient
+    reduce-scatter. "ZeRO" (lastdictionary.com), main definition: each layer's parameters are
+    gathered just in time and discarded.
+
+    Rank r owns partition r of the fp16 parameters (S values, in ``part_peers``: addressable by
+    every rank, e.g. torch symmetric memory) and shard r of the fp32 state. A step: the forward
+    gathers, layer by layer (each rank's gather kernel reads the owners' partitions in place;
+    with NVLink peer addresses the kernel's loads cross NVLink, plain loads, no multicast);
+    backward, per layer in reverse order: the gather again, then the layer's gradient bucket
+    (its range; the last layer's extended over the padding, the end of the flat list being
+    produced first) reduce-scattered to its owners and each owner's fused update written into
+    its own partition (DistZeroStep with the layers' gradient buckets); the job-wide verdict;
+    nothing is gathered after the step. The gathered layer goes to ``layer_buf`` (the buffer
+    the layer's computation would read); ``record`` (a list) receives a copy of each gathered
+    layer, forward then backward, for checking."""
+
+    def __init__(self, numels: Sequence[int], layer_tensors: Sequence[int], part_peers,
+                 group=None, compute=None, peers=None):
+        import torch.distributed as dist
+        self.dist = dist
+        self.numels = list(numels)
+        self.nd = dist.get_world_size(group)
+        psi = sum(self.numels)
+        self.psi_p = -(-psi // self.nd) * self.nd
+        self.shard = self.psi_p // self.nd
+        self.layers = layer_ranges(self.numels, layer_tensors)
+        grad_buckets = list(self.layers)
+        grad_buckets[-1] = (grad_buckets[-1][0], self.psi_p)
+        self.part_peers = part_peers
+        self.compute = compute or LibzeroCompute()
+        self.inner = DistZeroStep(self.psi_p, 0, group, self.compute, peers,
+                                  buckets=grad_buckets[::-1], partitioned=True)
+
+    def gather(self, l: int, layer_buf, status):
+        lo, hi = self.layers[l]
+        parts = self.part_peers.rows(0, self.shard)
+        self.compute.gather(self.numels, self.nd, lo, hi - lo, parts, layer_buf[:hi - lo], status)
+
+    def step(self, local_grad, state_in, state_out, hp, t: int, status, layer_buf, record=None):
+        """local_grad: this rank's fp16 gradient (psi_p values; in peers.local for the
+        peer-read form); state_in / state_out: this rank's fp32 shards; layer_buf: a buffer of
+        the largest layer's length. Returns the job-wide void bits; raises DistStepError on
+        every rank if any rank's kernels failed."""
+        order = list(range(len(self.layers)))
+        for l in order + order[::-1]:        # forward, then backward
+            self.gather(l, layer_buf, status)
+            if record is not None:
+                record.append(layer_buf[:self.layers[l][1] - self.layers[l][0]].clone())
+        return self.inner.step(local_grad, state_in, state_out, self.part_peers.local, hp, t,
+                               status)
