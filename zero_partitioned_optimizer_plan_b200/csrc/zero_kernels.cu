@@ -61,20 +61,36 @@ struct FusedArgs {
     MeanConsts mc;
     int selftest_no_copies;  // self-test only: the producer issues nothing (waits must expire)
     int chained;         // programmatic launch chained to the previous call (see pdl_enter)
-    // the all-gather in the epilogue: when n_replicas > 0 the fp16 values go to every replica's
-    // buffer (replicas[d], possibly a peer's address) instead of param_out
+};
+
+// The fused step with the all-gather in its epilogue: the fp16 values go to every replica's
+// buffer (replicas[d], possibly a peer's address) instead of param_out. A separate argument
+// type, so that the one-buffer kernels keep their parameter block and code unchanged.
+struct FusedRepArgs : FusedArgs {
     int n_replicas;
     uint16_t* replicas[kMaxRanks];
 };
 
-// The fp16 write-back of one value: into param_out, or into every replica.
+// The fp16 write-back of one value, or of a thread's E values.
 __device__ __forceinline__ void store_param(const FusedArgs& p, uint64_t i, float w) {
+    p.param_out[i] = f2h(w);
+}
+
+__device__ __forceinline__ void store_param(const FusedRepArgs& p, uint64_t i, float w) {
     const uint16_t h = f2h(w);
-    if (p.n_replicas == 0) {
-        p.param_out[i] = h;
-        return;
-    }
     for (int d = 0; d < p.n_replicas; ++d) p.replicas[d][i] = h;
+}
+
+template <int E>
+__device__ __forceinline__ void store_params(const FusedArgs& p, uint64_t g0,
+                                             const float (&w)[E]) {
+    stg_f16<E>(p.param_out + g0, w, p.param_vec);
+}
+
+template <int E>
+__device__ __forceinline__ void store_params(const FusedRepArgs& p, uint64_t g0,
+                                             const float (&w)[E]) {
+    for (int d = 0; d < p.n_replicas; ++d) stg_f16<E>(p.replicas[d] + g0, w, p.param_vec);
 }
 
 struct RsArgs {
@@ -197,7 +213,8 @@ __device__ void produce(const Args& p, uint64_t* full, uint64_t* empty, uint8_t*
 // ---------------------------------------------------------------------------------------------
 // fused step: reduce-scatter + unscale + Adam + fp16 cast + write-back, TMA-pipelined
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ void fused_element(const FusedArgs& p, const AdamConsts& a, uint64_t i,
+template <typename Args>
+__device__ __forceinline__ void fused_element(const Args& p, const AdamConsts& a, uint64_t i,
                                               bool& bad) {
     if (i >= p.n) {   // self-check: never taken when the launch arithmetic is right
         atomicOr(p.status, ZERO_FLAG_BOUNDS);
@@ -215,9 +232,9 @@ __device__ __forceinline__ void fused_element(const FusedArgs& p, const AdamCons
     store_param(p, i, w);
 }
 
-template <int E, int W, bool kDC>
+template <int E, int W, bool kDC, typename Args = FusedArgs>
 __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
-    fused_tma_kernel(const __grid_constant__ FusedArgs p) {
+    fused_tma_kernel(const __grid_constant__ Args p) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
@@ -269,11 +286,7 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
         stg_f32<E>(p.master_out + g0, w);
         stg_f32<E>(p.m_out + g0, m);
         stg_f32<E>(p.v_out + g0, v);
-        if (p.n_replicas == 0) {
-            stg_f16<E>(p.param_out + g0, w, p.param_vec);
-        } else {
-            for (int d = 0; d < p.n_replicas; ++d) stg_f16<E>(p.replicas[d] + g0, w, p.param_vec);
-        }
+        store_params<E>(p, g0, w);
     }
     // the < 8 elements past the last tile
     if (blockIdx.x == 0 && (uint64_t)threadIdx.x < p.n - p.n_tiled)
@@ -283,8 +296,8 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
 }
 
 // plain-load variant for ranges whose pointers are not 16-byte aligned (or tiny ranges)
-template <bool kDC>
-__global__ void __launch_bounds__(256) fused_plain_kernel(const __grid_constant__ FusedArgs p) {
+template <bool kDC, typename Args = FusedArgs>
+__global__ void __launch_bounds__(256) fused_plain_kernel(const __grid_constant__ Args p) {
     ZK_STEP_CONSTS(p, a);
     bool bad = false;
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
@@ -615,6 +628,31 @@ cudaError_t launch_selftest_timeout(uint32_t* status, cudaStream_t stream) {
 
 uint64_t launches() { return g_launches.load(std::memory_order_relaxed); }
 
+// The launch of either argument type: the one-buffer step, or the epilogue all-gather.
+template <typename Args>
+cudaError_t launch_fused_args(Args& p, bool all16, cudaStream_t stream) {
+    DevInfo di;
+    cudaError_t e = dev_info(&di);
+    if (e != cudaSuccess) return e;
+    if (!all16 || p.n < kMinTiledElems) {
+        if (p.ad)
+            fused_plain_kernel<true, Args><<<plain_grid(p.n, di.sms), 256, 0, stream>>>(p);
+        else
+            fused_plain_kernel<false, Args><<<plain_grid(p.n, di.sms), 256, 0, stream>>>(p);
+        count_launch();
+        return cudaGetLastError();
+    }
+    const PipeShape sh = pipe_shape(p.nd, true, p.n, di.sms);
+    p.g = sh.g;
+    p.n_tiled = p.n & ~(uint64_t)7;
+    p.num_tiles = (p.n_tiled + sh.g.tile - 1) / sh.g.tile;
+    p.chained = overlap_next(stream) ? 1 : 0;
+    if (p.ad) {
+        ZK_LAUNCH_BY_WARPS(fused_tma_kernel, , true, Args);
+    }
+    ZK_LAUNCH_BY_WARPS(fused_tma_kernel, , false, Args);
+}
+
 cudaError_t launch_fused(uint64_t n, int nd, const uint16_t* const* grads, const float* master_in,
                          const float* m_in, const float* v_in, float* master_out, float* m_out,
                          float* v_out, uint16_t* param_out, const AdamConsts& a,
@@ -639,35 +677,20 @@ cudaError_t launch_fused(uint64_t n, int nd, const uint16_t* const* grads, const
     p.n = n;
     p.nd = nd;
     p.param_vec = store_vec(param_out);
-    p.n_replicas = n_replicas;
-    for (int d = 0; d < n_replicas; ++d) {   // one store width that every replica allows
-        p.replicas[d] = replicas[d];
-        const int v = store_vec(replicas[d]);
-        if (d == 0 || v < p.param_vec) p.param_vec = v;
-    }
     p.a = a;
     p.ad = ad;
     p.mc = mc;
-    DevInfo di;
-    cudaError_t e = dev_info(&di);
-    if (e != cudaSuccess) return e;
-    if (!all16 || n < kMinTiledElems) {
-        if (ad)
-            fused_plain_kernel<true><<<plain_grid(n, di.sms), 256, 0, stream>>>(p);
-        else
-            fused_plain_kernel<false><<<plain_grid(n, di.sms), 256, 0, stream>>>(p);
-        count_launch();
-        return cudaGetLastError();
+    if (n_replicas == 0) return launch_fused_args(p, all16, stream);
+    FusedRepArgs q;
+    memset(&q, 0, sizeof(q));
+    static_cast<FusedArgs&>(q) = p;
+    q.n_replicas = n_replicas;
+    for (int d = 0; d < n_replicas; ++d) {   // one store width that every replica allows
+        q.replicas[d] = replicas[d];
+        const int v = store_vec(replicas[d]);
+        if (d == 0 || v < q.param_vec) q.param_vec = v;
     }
-    const PipeShape sh = pipe_shape(nd, true, n, di.sms);
-    p.g = sh.g;
-    p.n_tiled = n & ~(uint64_t)7;
-    p.num_tiles = (p.n_tiled + sh.g.tile - 1) / sh.g.tile;
-    p.chained = overlap_next(stream) ? 1 : 0;
-    if (ad) {
-        ZK_LAUNCH_BY_WARPS(fused_tma_kernel, , true);
-    }
-    ZK_LAUNCH_BY_WARPS(fused_tma_kernel, , false);
+    return launch_fused_args(q, all16, stream);
 }
 
 cudaError_t launch_reduce_scatter(uint64_t n, int nd, const uint16_t* const* grads,
