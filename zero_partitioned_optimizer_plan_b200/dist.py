@@ -112,13 +112,13 @@ def q8_segment(n: int) -> int:
     return (q8_bytes(n) + 15) // 16 * 16 if n else 0
 
 
-def q8_peer_layout(psi_p: int, bucket: int, nd: int):
+def q8_peer_layout(psi_p: int, bucket: int, nd: int, buckets=None):
     """Byte offset of every (bucket, owner) part's payload in a rank's peer buffer (buckets in
-    backward order, owners in rank order, each part's segment padded to 16 bytes), and the
-    buffer's size."""
+    backward order -- bucket_ranges(psi_p, bucket), or the given list -- owners in rank order,
+    each part's segment padded to 16 bytes), and the buffer's size."""
     shard = psi_p // nd
     offs, total = [], 0
-    for lo, hi in bucket_ranges(psi_p, bucket):
+    for lo, hi in (buckets if buckets is not None else bucket_ranges(psi_p, bucket)):
         row = []
         for x in owner_parts(lo, hi, shard, nd):
             row.append(total)
@@ -127,9 +127,9 @@ def q8_peer_layout(psi_p: int, bucket: int, nd: int):
     return offs, max(total, 16)
 
 
-def q8_peer_bytes(psi_p: int, bucket: int, nd: int) -> int:
+def q8_peer_bytes(psi_p: int, bucket: int, nd: int, buckets=None) -> int:
     """Size of each rank's peer buffer for the int8 peer-read form."""
-    return q8_peer_layout(psi_p, bucket, nd)[1]
+    return q8_peer_layout(psi_p, bucket, nd, buckets)[1]
 
 
 def owner_parts(lo: int, hi: int, shard: int, nd: int) -> List[int]:
@@ -211,7 +211,9 @@ class LibzeroCompute:
 class DistZeroStep:
     """One rank's side of the distributed step. psi_p: the flat padded length (a multiple of
     the world size); bucket: elements per bucket (0: one bucket, stage 1); payload: "fp16"
-    (the gradients themselves are exchanged) or "q8" (int8 records, all-to-all form only)."""
+    (the gradients themselves are exchanged or read) or "q8" (int8 records); peers: the
+    gradients (fp16) or payload records (q8) read in place from the peers' buffers instead of
+    an all-to-all; param_peers: the all-gather in the owners' kernels (fp16 only)."""
 
     def __init__(self, psi_p: int, bucket: int = 0, group=None, compute=None, peers=None,
                  payload: str = "fp16", param_peers=None, buckets=None, partitioned=False):
@@ -241,7 +243,7 @@ class DistZeroStep:
             raise ValueError("the epilogue all-gather runs with the fp16 payload")
         self.param_peers = param_peers
         if payload == "q8" and peers is not None:
-            self._q8_offs, need = q8_peer_layout(psi_p, bucket, self.nd)
+            self._q8_offs, need = q8_peer_layout(psi_p, bucket, self.nd, self.buckets)
             if peers.local.numel() * peers.local.element_size() < need:
                 raise ValueError(f"peer buffers of {need} bytes are needed (q8_peer_bytes)")
         self.peers = peers
