@@ -689,7 +689,7 @@ S3_NUMELS = [1000, 37, 4099, 12345, 6000, 7]
 S3_LAYERS = [1, 2, 1, 2]
 
 
-def _worker_stage3(rank, ws, port, bad_rank, pbufs, out):
+def _worker_stage3(rank, ws, port, bad_rank, pbufs, gbufs, out):
     import datetime
     import numpy as np
     import torch
@@ -707,11 +707,16 @@ def _worker_stage3(rank, ws, port, bad_rank, pbufs, out):
         st_in = [x[rank * S:(rank + 1) * S].clone() for x in (master, m, v)]
         st_out = [torch.full_like(x, float("nan")) for x in st_in]
         status = torch.zeros(1, dtype=torch.int32)
-        step = DistStage3Step(S3_NUMELS, S3_LAYERS, parts, compute=_OracleCompute())
+        peers = None
+        if gbufs is not None:      # gradients read in place from the peers' buffers
+            peers = SharedPeerBuffers(gbufs, rank)
+            peers.local.copy_(grads[rank])
+        step = DistStage3Step(S3_NUMELS, S3_LAYERS, parts, compute=_OracleCompute(), peers=peers)
         big = max(hi - lo for lo, hi in step.layers)
         layer_buf = torch.zeros(big, dtype=torch.float16)
         rec = []
-        flag = step.step(grads[rank], st_in, st_out, oracle.AdamHP(), 1, status, layer_buf, rec)
+        flag = step.step(peers.local if peers is not None else grads[rank], st_in, st_out,
+                         oracle.AdamHP(), 1, status, layer_buf, rec)
         dist.barrier()    # every owner's partition is final before it is read back
         out.put((rank, int(flag.item()), int(status.item()), [x.numpy() for x in st_out],
                  [p.numpy().view(np.uint16).copy() for p in parts.tensors],
@@ -720,8 +725,9 @@ def _worker_stage3(rank, ws, port, bad_rank, pbufs, out):
         dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("peer", [False, True])
 @pytest.mark.parametrize("ws,bad_rank", [(2, -1), (3, -1), (3, 1)])
-def test_distributed_stage3_gloo(ws, bad_rank):
+def test_distributed_stage3_gloo(ws, bad_rank, peer):
     """DistStage3Step on gloo ranks, the partitions in CPU tensors shared by the processes
     (standing for NVLink peer mappings): every gathered layer (forward and backward), every
     owner's final partition and state shard equal the oracle's stage-3 step (zero3_step) bit
@@ -735,10 +741,12 @@ def test_distributed_stage3_gloo(ws, bad_rank):
     p16 = oracle.f2h(master.numpy())
     pbufs = [torch.from_numpy(p16[q * S:(q + 1) * S].copy().view(np.int16)).view(torch.float16)
              .share_memory_() for q in range(ws)]
+    gbufs = [torch.zeros(psi_p, dtype=torch.float16).share_memory_() for _ in range(ws)] \
+        if peer else None
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker_stage3, args=(r, ws, port, bad_rank, pbufs, q))
+    procs = [ctx.Process(target=_worker_stage3, args=(r, ws, port, bad_rank, pbufs, gbufs, q))
              for r in range(ws)]
     for p in procs:
         p.start()
