@@ -88,6 +88,9 @@ def parse():
                     help="stage-2 workloads: the bucket scheduler launches the fused step per "
                          "bucket (zero_sched_create_fused), or the reduce-scatter per bucket "
                          "and then the owner updates")
+    ap.add_argument("--replicas", type=int, default=0,
+                    help="flat workload: the fused calls store the fp16 parameters into R replica "
+                         "buffers (the all-gather in the epilogue, zero_step_fused_replicas)")
     ap.add_argument("--l2", choices=["warm", "flushed"], default="warm",
                     help="flushed: write a buffer larger than L2 between timed steps and time each "
                          "step on its own (for the L2-resident tiny workload)")
@@ -103,6 +106,10 @@ def parse():
     a = ap.parse_args()
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if a.replicas and (a.workload != "flat" or a.payload != "fp16" or a.graph):
+        ap.error("--replicas takes the flat workload, fp16 payloads, eager calls")
+    if not 0 <= a.replicas <= 64:
+        ap.error("--replicas: 1 to 64")
     return a
 
 
@@ -158,6 +165,9 @@ def workload_config(args) -> dict:
     if args.payload == "q8":
         cfg["payload"] = "int8 records: 128 values and their fp32 scale"
         cfg["workload"] += "_q8"
+    if getattr(args, "replicas", 0):
+        cfg["replicas"] = args.replicas
+        cfg["workload"] += f"_rep{args.replicas}"
     return cfg
 
 
@@ -174,6 +184,7 @@ class Workload:
         self.kind = kind
         self.e2e = None          # a workload-specific end-to-end leg (stage 2 fused)
         self.kernel_times = None  # per-step dominant-kernel time, when not the ev pair's
+        self.replicas = []        # --replicas: the full parameter buffers the fused calls write
         if kind in ("gpt2_small", "tiny"):
             tiny = kind == "tiny"
             nd = args.nd or (4 if tiny else 8)
@@ -233,11 +244,16 @@ class Workload:
             self.param_base = 0
             self.config = workload_config(args)
             assert self.config["calls_per_step"] == len(self.ranges)
+            # --replicas R: the all-gather in the epilogue, into R full parameter buffers
+            self.replicas = [self.params] + [torch.empty(psi, dtype=torch.float16, device=dev)
+                                             for _ in range(args.replicas - 1)] \
+                if args.replicas else []
         self.cur = [master, m, v]
         self.nxt = [torch.empty_like(x) for x in self.cur]
         self.state_a0 = self.cur[0].data_ptr()
         self.prepared = [None, None]                          # per ping-pong direction
-        self.bytes_per_step = (2 * self.nd + 26) * self.n     # algorithmic HBM bytes
+        # algorithmic HBM bytes: with R replicas the fp16 write is 2 R bytes per value
+        self.bytes_per_step = (2 * self.nd + 24 + 2 * max(1, len(self.replicas))) * self.n
         # the dominant kernel: its bytes and launches per step
         self.dominant = "fused_tma_kernel"
         self.dominant_bytes = self.bytes_per_step
@@ -384,6 +400,24 @@ class Workload:
         dominant kernel's launches. grads: the step's inputs (as inputs() lists them) when
         they are not the workload's own buffers."""
         lz = self.lz
+        if self.replicas:
+            grads = grads or self.grads
+            if ev is not None:
+                ev[0].record()
+            if self.overlap:
+                lz.zero_overlap_begin()
+            for lo, hi in self.ranges:
+                lz.zero_step_fused_replicas(hi - lo, self.nd, [g[lo:hi] for g in grads],
+                                            *[x[lo:hi] for x in self.cur],
+                                            *[x[lo:hi] for x in self.nxt],
+                                            [r[lo:hi] for r in self.replicas], self.hp, t, status)
+            if self.overlap:
+                lz.zero_overlap_end()
+            if ev is not None:
+                ev[1].record()
+            lz.zero_step_commit_replicas(self.n, *self.cur, *self.nxt, self.replicas, status)
+            self.cur, self.nxt = self.nxt, self.cur
+            return
         if grads is None and len(self.ranges) > 1:   # per-bucket calls, marshalled once
             self._step_prepared(t, status, ev)
             return
