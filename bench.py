@@ -185,6 +185,7 @@ class Workload:
         self.e2e = None          # a workload-specific end-to-end leg (stage 2 fused)
         self.kernel_times = None  # per-step dominant-kernel time, when not the ev pair's
         self.replicas = []        # --replicas: the full parameter buffers the fused calls write
+        self.time_calls = False   # record per-call events in this step (stage 3)
         if kind in ("gpt2_small", "tiny"):
             tiny = kind == "tiny"
             nd = args.nd or (4 if tiny else 8)
@@ -793,7 +794,10 @@ def _step_zero3(self, t, status, ev=None, grads=None):
     grads = grads or self.grads
     pl, shards, L = self.plan, self.shards, len(self.layers)
     main, gs = torch.cuda.current_stream(), self.gather_stream
-    timed = ev is not None
+    # per-call events only in the step that run_ours marks (the last timed one): recording
+    # about a hundred events and waits every step doubled the host's work per step, which at
+    # GPT-2-small sizes then set the step's pace
+    timed = ev is not None and self.time_calls
     g_pairs, f_pairs = [], []
 
     def gather(l):
@@ -807,7 +811,7 @@ def _step_zero3(self, t, status, ev=None, grads=None):
                 e[1].record(gs)
                 g_pairs.append(e)
 
-    if timed:
+    if ev is not None:
         ev[0].record(main)
     self.step_start.record(main)
     gs.wait_event(self.step_start)            # the previous step's updates and commit
@@ -838,8 +842,9 @@ def _step_zero3(self, t, status, ev=None, grads=None):
             self.g_done[l - 1].record(gs)
     lz.zero_overlap_end(main)
     lz.zero_stage3_step_commit(pl, *self.cur, *self.nxt, shards, status, main)
-    if timed:
+    if ev is not None:
         ev[1].record(main)
+    if timed:
         self.side["ms"].append(list(g_pairs))
         self.fused_evs.append(list(f_pairs))
     self.cur, self.nxt = self.nxt, self.cur
@@ -865,8 +870,8 @@ def _layer_args(self, l, grads):
 
 
 def _kernel_times_zero3(self, evs):
-    """Per step: the fused calls' summed durations (ms). The events are reused by every step,
-    so only the last step's are still readable: its durations stand for each timed step."""
+    """Per step: the fused calls' summed durations (ms). Only the last timed step records
+    per-call events (time_calls): its durations stand for each timed step."""
     last = sum(a.elapsed_time(b) for a, b in self.fused_evs[-1])
     return [last] * len(evs)
 
@@ -1291,6 +1296,7 @@ def run_ours(args):
             if flushed:
                 flush_buf.fill_(i)
                 sevs[i][0].record()
+            wl.time_calls = i == K - 1
             wl.step(W + i + 1, status[W + i:W + i + 1], ev=evs[i])
             if flushed:
                 sevs[i][1].record()

@@ -345,10 +345,32 @@ __device__ void produce_q8(const FusedQ8Args& p, uint64_t* full, uint64_t* empty
     }
 }
 
+// Rank r's contribution to a thread's E accumulators (packed pairs ap): its record's scale and
+// E bytes q + 128, converted by mantissa placement, added by fused multiply-adds.
+template <int E>
+__device__ __forceinline__ void q8_rank_fma(const uint8_t* rec, uint32_t e_in_rec,
+                                            uint64_t (&ap)[E / 2]) {
+    const uint64_t nbias = f2_pack(-8388736.0f, -8388736.0f);   // -(2^23 + 128)
+    const float sc = *reinterpret_cast<const float*>(rec + kQB);
+    const uint64_t ss = f2_pack(sc, sc);
+#pragma unroll
+    for (int k4 = 0; k4 < E / 4; ++k4) {
+        const uint32_t biased =   // four bytes, each q + 128
+            *reinterpret_cast<const uint32_t*>(rec + e_in_rec + 4 * k4);
+        const uint64_t q01 = f2_add(f2_pack(q_placed(biased, 0), q_placed(biased, 1)), nbias);
+        const uint64_t q23 = f2_add(f2_pack(q_placed(biased, 2), q_placed(biased, 3)), nbias);
+        // acc + q * scale, one rounding each
+        ap[2 * k4] = f2_fma(q01, ss, ap[2 * k4]);
+        ap[2 * k4 + 1] = f2_fma(q23, ss, ap[2 * k4 + 1]);
+    }
+}
+
 // kFixedRow: the rank loop steps from one rank's records to the next by the compile-time kRow
 // (immediate load offsets) or by the launch's p.row (the same value, at run time); which is
-// faster depends on Nd (see pick_variant_q8).
-template <int W, int E, bool kDC, bool kFixedRow>
+// faster depends on Nd (see pick_variant_q8). kRC > 0: a chunk of exactly kRC ranks runs fully
+// unrolled (no loop counter, every record at an immediate offset); a chunk of another length
+// takes the general loop.
+template <int W, int E, bool kDC, bool kFixedRow, int kRC = 0>
 __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
     fused_q8_tma_kernel(const __grid_constant__ FusedQ8Args p) {
     static_assert(E == 4 || E == 8, "a thread's values sit in one record");
@@ -400,25 +422,15 @@ __global__ void __launch_bounds__(Warps<W>::kThreads, Warps<W>::kMinBlocks)
                 uint64_t ap[P];
 #pragma unroll
                 for (int k = 0; k < P; ++k) ap[k] = f2_pack(acc[2 * k], acc[2 * k + 1]);
-                const uint64_t nbias = f2_pack(-8388736.0f, -8388736.0f);   // -(2^23 + 128)
                 // rank r's record sits `row` bytes after rank r-1's
-#pragma unroll(16 / E)
-                for (uint32_t r = 0; r < nr; ++r) {
-                    const uint8_t* rec = rec0 + (size_t)r * row;
-                    const float sc = *reinterpret_cast<const float*>(rec + kQB);
-                    const uint64_t ss = f2_pack(sc, sc);
+                if (kRC > 0 && nr == (uint32_t)kRC) {
 #pragma unroll
-                    for (int k4 = 0; k4 < E / 4; ++k4) {
-                        const uint32_t biased =   // four bytes, each q + 128
-                            *reinterpret_cast<const uint32_t*>(rec + e0 % kQB + 4 * k4);
-                        const uint64_t q01 =
-                            f2_add(f2_pack(q_placed(biased, 0), q_placed(biased, 1)), nbias);
-                        const uint64_t q23 =
-                            f2_add(f2_pack(q_placed(biased, 2), q_placed(biased, 3)), nbias);
-                        // acc + q * scale, one rounding each
-                        ap[2 * k4] = f2_fma(q01, ss, ap[2 * k4]);
-                        ap[2 * k4 + 1] = f2_fma(q23, ss, ap[2 * k4 + 1]);
-                    }
+                    for (int r = 0; r < kRC; ++r)
+                        q8_rank_fma<E>(rec0 + (size_t)r * kRow, e0 % kQB, ap);
+                } else {
+#pragma unroll(16 / E)
+                    for (uint32_t r = 0; r < nr; ++r)
+                        q8_rank_fma<E>(rec0 + (size_t)r * row, e0 % kQB, ap);
                 }
 #pragma unroll
                 for (int k = 0; k < P; ++k) f2_unpack(ap[k], acc[2 * k], acc[2 * k + 1]);
@@ -511,6 +523,11 @@ VariantQ8 pick_variant_q8(int nd) {
 #endif
     return v;
 }
+
+// Ranks per chunk of the 24-warp shape at Nd = 64 (q8_shape with the default stage budget:
+// chunks of 22, 22 and 20 ranks), for which the rank loop is instantiated fully unrolled. Same
+// box, two alternating passes each: flat 2^28 5.59 -> 5.68 TB/s, the 7.5B view 5.56 -> 5.64.
+constexpr int kRC24 = 22;
 
 // Small calls (fewer than 4 tiles of the large shape per SM): as for the fp16 step, 12
 // consumer warps up to Nd = 8 and 8 above, 100 KB of stages and one CTA per SM, so that the
@@ -644,6 +661,13 @@ cudaError_t launch_fused_q8(uint64_t n, int nd, const uint8_t* const* payload,
         return ad ? launch_pipe(fused_q8_tma_kernel<WW, EE, true, false>, p, sh, stream)   \
                   : launch_pipe(fused_q8_tma_kernel<WW, EE, false, false>, p, sh, stream); \
     }
+#ifndef ZK_Q8_NO_RC
+    // Nd = 64 in the 24-warp shape: chunks of 22 ranks (22, 22, 20), the full ones unrolled
+    if (sh.warps == 24 && elems == 4 && var.fixed_row && sh.g.rc == kRC24) {
+        return ad ? launch_pipe(fused_q8_tma_kernel<24, 4, true, true, kRC24>, p, sh, stream)
+                  : launch_pipe(fused_q8_tma_kernel<24, 4, false, true, kRC24>, p, sh, stream);
+    }
+#endif
     ZK_Q8_CASE(8, 4);
     ZK_Q8_CASE(12, 4);
     ZK_Q8_CASE(16, 4);
