@@ -22,7 +22,9 @@ Workloads (synthetic, seeded):
   zero3_gpt2_small  ZeRO stage 3 on the GPT-2-small list, Nd = 8: the fp16 parameters live in
               8 partitions; a step gathers each of the 14 layers (embedding, 12 blocks, final
               LayerNorm) in forward order, then in backward order gathers each layer again and
-              runs its fused update into the owners' partitions, then commits.
+              runs its fused update into the owners' partitions, then commits. The library's
+              layer scheduler runs the gathers one layer ahead on a second stream into two
+              layer buffers.
   zero3_1p3b  the same on the 1.3B list (26 layers), Nd = 16.
   gpt2_small  GPT-2-small parameter list (psi = 123,653,376), Nd = 8, stage 1 (full local
               gradients, one fused call per step); grads N(0, 1e-3^2) with 1% x100; master
@@ -94,6 +96,8 @@ def parse():
     ap.add_argument("--l2", choices=["warm", "flushed"], default="warm",
                     help="flushed: write a buffer larger than L2 between timed steps and time each "
                          "step on its own (for the L2-resident tiny workload)")
+    ap.add_argument("--layer-buffers", type=int, default=2,
+                    help="stage-3 workloads: layer buffers of the layer scheduler (>= 1)")
     ap.add_argument("--no-sweep", action="store_true",
                     help="leave out the bucket / Nd sweep of the default line")
     ap.add_argument("--sweep-steps", type=int, default=None)
@@ -715,9 +719,11 @@ def _e2e_zero2_fused(self, t0, E, barrier, max_ms):
 def _init_zero3(self, args, dev):
     """Stage 3 on a GPT-shaped list: every rank's full local gradient is resident (as the
     backward pass would leave it layer by layer); the fp16 parameters are Nd partitions of S
-    values; the optimizer state is flat and ping-ponged. A step: forward gathers of every
-    layer, then per layer in backward order its gather and its fused update (zero_stage3_step_fused),
-    then zero_stage3_step_commit. Each fused and each gather call is timed with its own events."""
+    values; the optimizer state is flat and ping-ponged. The library's layer scheduler gathers
+    the layers on a second stream into two layer buffers. A step: every layer acquired in
+    forward order (the next one prefetched), then per layer in backward order acquired again
+    (the previous one prefetched), released, and updated (zero_stage3_step_fused), then
+    zero_stage3_step_commit. Each fused call is timed with its own events in the last step."""
     torch, lz = self.torch, self.lz
     from zero_partitioned_optimizer_plan_b200 import synth
     if args.payload != "fp16":
@@ -748,18 +754,19 @@ def _init_zero3(self, args, dev):
         part = torch.empty(S, dtype=torch.float16, device=dev)
         part.copy_(master[q * S:(q + 1) * S])
         self.shards.append(part)
-    big = max(hi - lo for lo, hi in self.layers)
-    self.layer_bufs = [torch.empty(big, dtype=torch.float16, device=dev) for _ in range(2)]
+    bounds = [lo for lo, _ in self.layers] + [self.layers[-1][1]]
+    nb = args.layer_buffers
+    elems = lz.zero_layer_sched_buf_elems(pl, bounds, nb)
+    self.layer_mem = torch.empty(elems, dtype=torch.float16, device=dev)
     self.gather_stream = torch.cuda.Stream()
+    self.layer_sched = lz.zero_layer_sched_create(pl, bounds, self.shards, self.layer_mem, elems,
+                                                  nb, self.gather_stream)
     L = len(self.layers)
-    mk = lambda t=False: torch.cuda.Event(enable_timing=t)   # noqa: E731
-    self.step_start = mk()
-    self.g_done = [mk() for _ in range(L)]
-    self.f_done = [mk() for _ in range(L)]
-    self.g_ev = [(mk(True), mk(True)) for _ in range(2 * L)]   # reused every step
-    self.f_ev = [(mk(True), mk(True)) for _ in range(L)]
+    mk = lambda: torch.cuda.Event(enable_timing=True)   # noqa: E731
+    self.f_ev = [(mk(), mk()) for _ in range(L)]        # reused by the step that records them
     self.state_a0 = self.cur[0].data_ptr()
     self.layer_views = [None, None]
+    self.prepared3 = [None, None]         # per ping-pong direction: the layers' update calls
     self.params = self.shards[0]          # (the e2e leg downloads every partition)
     self.ranges = [(0, psi_p)]
     self.overlap = False
@@ -769,83 +776,66 @@ def _init_zero3(self, args, dev):
                   for l, (lo, hi) in enumerate(self.layers))
     self.config["calls_per_step"] = 2 * len(self.layers) + n_fused + 1   # + one commit
     self.config["fused_calls_per_step"] = n_fused
+    self.config["layer_buffers"] = nb
     gather_bytes = 2 * 4 * psi              # two gathers: 2 bytes read + 2 written each
     fused_bytes = (2 * nd + 26) * psi_p
     self.bytes_per_step = gather_bytes + fused_bytes
     self.dominant = "fused_tma_kernel"
     self.dominant_bytes = fused_bytes
     self.dominant_calls = n_fused
-    self.side = {"kernel": "gather_kernel", "bytes": gather_bytes, "calls": 2 * len(self.layers),
-                 "ms": []}
     self.fused_evs = []
+    self.side = None                      # the gathers run inside the layer scheduler
     self.step = self._step_zero3
     self.kernel_times = self._kernel_times_zero3
 
 
 def _step_zero3(self, t, status, ev=None, grads=None):
-    """One stage-3 step on two streams. The gather stream runs the forward gathers, then the
-    backward gathers one layer ahead: layer l-1 is gathered (into the other of two layer
-    buffers) while the main stream runs layer l's fused update. Layer l's update waits for
-    layer l's backward gather (the layer's computation would sit between them); a gather into a
-    buffer waits for the update of the layer that used the buffer before; the next step's
-    gathers wait for this step's commit. A gather and the update running beside it touch
-    disjoint ranges of the partitions."""
+    """One stage-3 step through the library's layer scheduler: the gathers run on its gather
+    stream one layer ahead of the main stream (forward, then backward); each layer's update on
+    the main stream follows its release. The backward gather of layer l-1 runs beside layer l's
+    update (disjoint ranges of the partitions); the next step's gathers wait for this step's
+    commit (zero_layer_sched_begin_step)."""
     lz, torch = self.lz, self.torch
     grads = grads or self.grads
-    pl, shards, L = self.plan, self.shards, len(self.layers)
-    main, gs = torch.cuda.current_stream(), self.gather_stream
+    pl, shards, L, sch = self.plan, self.shards, len(self.layers), self.layer_sched
+    main = torch.cuda.current_stream()
     # per-call events only in the step that run_ours marks (the last timed one): recording
-    # about a hundred events and waits every step doubled the host's work per step, which at
+    # events around every call of every step doubled the host's work per step, which at
     # GPT-2-small sizes then set the step's pace
     timed = ev is not None and self.time_calls
-    g_pairs, f_pairs = [], []
-
-    def gather(l):
-        lo, hi = self.layers[l]
-        with torch.cuda.stream(gs):
-            if timed:
-                e = self.g_ev[len(g_pairs)]
-                e[0].record(gs)
-            lz.zero_gather_params(pl, lo, hi - lo, shards, self.layer_bufs[l % 2], status, gs)
-            if timed:
-                e[1].record(gs)
-                g_pairs.append(e)
-
+    f_pairs = []
     if ev is not None:
         ev[0].record(main)
-    self.step_start.record(main)
-    gs.wait_event(self.step_start)            # the previous step's updates and commit
-    for l in range(L):                        # forward
-        gather(l)
-    gather(L - 1)                             # backward, one layer ahead of the updates
-    self.g_done[L - 1].record(gs)
-    # the layers' updates touch disjoint ranges: one overlap region on the main stream (its
-    # event waits and records are allowed inside; an event recorded after an update completes
-    # only when every update before it has)
+    lz.zero_layer_sched_begin_step(sch, status, main)
+    for l in range(L):                        # forward: the layer's computation would go here
+        lz.zero_layer_sched_acquire(sch, l, l + 1 if l + 1 < L else -1, main)
+        lz.zero_layer_sched_release(sch, l, main)
+    # the layers' updates touch disjoint ranges: one overlap region on the main stream (event
+    # waits and records are allowed inside; an event recorded after an update completes only
+    # when every update before it has)
+    prepared = self._layer_updates() if grads is self.grads else None
+    hp_ref, st_ptr, sh = lz.hparams_ref(self.hp), lz.status_ptr(status), lz.stream_handle(main)
     lz.zero_overlap_begin(main)
     for l in range(L - 1, -1, -1):
-        lo, hi = self.layers[l]
-        main.wait_event(self.g_done[l])
+        lo, _ = self.layers[l]
+        lz.zero_layer_sched_acquire(sch, l, l - 1, main)
+        lz.zero_layer_sched_release(sch, l, main)
         if timed:
             e = self.f_ev[len(f_pairs)]
             e[0].record(main)
-        lz.zero_stage3_step_fused(pl, lo, *self._layer_args(l, grads), shards, self.hp, t,
-                                  status, main)
+        if prepared is not None:
+            prepared[l](hp_ref, t, st_ptr, sh)
+        else:
+            lz.zero_stage3_step_fused(pl, lo, *self._layer_args(l, grads), shards, self.hp, t,
+                                      status, main)
         if timed:
             e[1].record(main)
             f_pairs.append(e)
-        self.f_done[l].record(main)
-        if l > 0:
-            if l + 1 < L:
-                gs.wait_event(self.f_done[l + 1])   # buffer (l-1) % 2 was layer l+1's
-            gather(l - 1)
-            self.g_done[l - 1].record(gs)
     lz.zero_overlap_end(main)
     lz.zero_stage3_step_commit(pl, *self.cur, *self.nxt, shards, status, main)
     if ev is not None:
         ev[1].record(main)
     if timed:
-        self.side["ms"].append(list(g_pairs))
         self.fused_evs.append(list(f_pairs))
     self.cur, self.nxt = self.nxt, self.cur
 
@@ -869,6 +859,18 @@ def _layer_args(self, l, grads):
     return self.layer_views[d][l]
 
 
+def _layer_updates(self):
+    """Each layer's zero_stage3_step_fused call for the current ping-pong direction, its
+    arguments marshalled once (PreparedStage3Update)."""
+    d = 0 if self.cur[0].data_ptr() == self.state_a0 else 1
+    if self.prepared3[d] is None:
+        self.prepared3[d] = [
+            self.lz.PreparedStage3Update(self.plan, lo, *self._layer_args(l, self.grads),
+                                         self.shards)
+            for l, (lo, _) in enumerate(self.layers)]
+    return self.prepared3[d]
+
+
 def _kernel_times_zero3(self, evs):
     """Per step: the fused calls' summed durations (ms). Only the last timed step records
     per-call events (time_calls): its durations stand for each timed step."""
@@ -880,6 +882,7 @@ Workload._init_zero3 = _init_zero3
 Workload._step_zero3 = _step_zero3
 Workload._kernel_times_zero3 = _kernel_times_zero3
 Workload._layer_args = _layer_args
+Workload._layer_updates = _layer_updates
 Workload._step_prepared = _step_prepared
 Workload._init_zero2 = _init_zero2
 Workload._step_zero2 = _step_zero2

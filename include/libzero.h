@@ -410,6 +410,64 @@ zero_status zero_stage3_step_commit(const zero_plan* plan, const float* master_i
                               zero_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Just-in-time layer scheduler for stage 3. "ZeRO" (lastdictionary.com), main definition: each
+ * layer's parameters are gathered just in time for its computation and discarded afterwards;
+ * "Como funciona": a partition a process does not own is received from its owner, once in the
+ * forward pass and again in the backward pass. The scheduler runs the gathers
+ * (zero_gather_params' kernel) on its own gather stream into a pool of n_bufs layer buffers and
+ * orders everything with CUDA events, so the host never blocks:
+ *   zero_layer_sched_begin_step(s, d_status, stream)   once per step, on the stream that ran the
+ *                                                        previous step's updates and commit
+ *   for each layer l of the pass:
+ *     zero_layer_sched_acquire(s, l, next, compute, &p) layer l's fp16 values at p (compute waits
+ *                                                        for the gather); `next`'s gather starts
+ *     ... the layer's computation on `compute` reads p ...
+ *     zero_layer_sched_release(s, l, compute)           p may be overwritten after this point
+ * and in the backward pass, after release(l), the layer's update (zero_stage3_step_fused over
+ * its gradient bucket) on the compute stream; then zero_stage3_step_commit. A gather and the
+ * updates beside it touch disjoint ranges of the partitions as long as each layer's update
+ * covers only its own range (the last layer's extended over the padding).
+ *   layer_bounds : n_layers + 1 flat offsets, 0 = b[0] < b[1] < ... < b[n_layers], with
+ *                  psi <= b[n_layers] <= psi_padded; layer l is [b[l], b[l+1]) (copied)
+ *   param_shards : the nd owners' partitions, S fp16 values each, 2-byte aligned (copied)
+ *   buf_mem      : zero_layer_sched_buf_elems(...) fp16 values of caller device memory, 16-byte
+ *                  aligned, not overlapping a partition: n_bufs buffers of the longest layer
+ *                  rounded up to 8 values. n_bufs >= 2 lets one gather run ahead.
+ * A released layer is discarded (acquiring it again gathers it again); a prefetched layer that
+ * is not acquired before its buffer is needed is dropped; begin_step drops every layer still
+ * in a buffer (the partitions have changed since). The pages have no scheduler interface; this
+ * is the library's runtime for the stage-3 data path.
+ * Errors: ZERO_EINVAL (bad plan or bounds, null pointers, a layer out of range or already
+ * acquired, release of a layer not acquired, begin_step while a layer is acquired, a status
+ * word inside a partition or the buffers), ZERO_EALIGN, ZERO_ENOMEM (buf_mem too small, every
+ * buffer holding an acquired layer, host allocation), ZERO_ECUDA (event or launch failure).
+ * ---------------------------------------------------------------------------------------- */
+typedef struct zero_layer_sched zero_layer_sched;
+
+zero_status zero_layer_sched_buf_elems(const zero_plan* plan, int n_layers,
+                                       const uint64_t* layer_bounds, int n_bufs,
+                                       uint64_t* elems);
+zero_status zero_layer_sched_create(const zero_plan* plan, int n_layers,
+                                    const uint64_t* layer_bounds,
+                                    const uint16_t* const* param_shards, uint16_t* buf_mem,
+                                    uint64_t buf_mem_elems, int n_bufs,
+                                    zero_stream_t gather_stream, zero_layer_sched** out);
+/* Start a step: its gathers OR their bounds flag into d_status (4-byte aligned) and wait for
+ * the work enqueued on `stream` so far. */
+zero_status zero_layer_sched_begin_step(zero_layer_sched* s, uint32_t* d_status,
+                                        zero_stream_t stream);
+/* Make `compute` wait until layer `layer` is gathered (gathering it now unless a prefetch
+ * already did) and write its buffer's address to *layer_params; then, if 0 <= prefetch <
+ * n_layers and a buffer is free, start the gather of layer `prefetch`. */
+zero_status zero_layer_sched_acquire(zero_layer_sched* s, int layer, int prefetch,
+                                     zero_stream_t compute, uint16_t** layer_params);
+/* Layer `layer`'s readers are enqueued on `compute`: its buffer is free after them. */
+zero_status zero_layer_sched_release(zero_layer_sched* s, int layer, zero_stream_t compute);
+/* Number of gathers the scheduler has launched since creation. */
+zero_status zero_layer_sched_gathers(const zero_layer_sched* s, uint64_t* count);
+void zero_layer_sched_destroy(zero_layer_sched* s);
+
+/* ------------------------------------------------------------------------------------------
  * Compressed reduce-scatter payload. "ZeRO" (lastdictionary.com), main definition: extensions
  * compress the communication (ZeRO++). The pages give no format; this library's: each rank's
  * slice travels as 8-bit values with one fp32 scale per block of ZERO_Q8_BLOCK elements

@@ -428,6 +428,39 @@ def test_stage3_update_rejects_and_launches_nothing():
     assert lz.zero_kernel_launches() == before
 
 
+def test_layer_scheduler_sizes_and_rejects():
+    """The stage-3 layer scheduler's buffer size (n_bufs buffers of the longest layer rounded
+    up to 8 values) and its argument errors, all found before any CUDA call."""
+    pl = _stage3_plan()                                  # psi = 128 = psi_p, S = 32
+    parts = [A + q * MB for q in range(4)]
+    good = [0, 17, 100, 128]                             # longest layer 83 -> 88 per buffer
+    assert lz.zero_layer_sched_buf_elems(pl, good, 2) == 176
+    assert lz.zero_layer_sched_buf_elems(pl, [0, 128], 3) == 3 * 128
+    for bounds in ([1, 17, 128], [0, 17, 17, 128], [0, 17, 127], [0, 17, 129], [0, 40, 20, 128],
+                   [0]):
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_layer_sched_buf_elems(pl, bounds, 2)
+        assert e.value.code == lz.ZERO_EINVAL, bounds
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_layer_sched_buf_elems(pl, good, 0)
+    assert e.value.code == lz.ZERO_EINVAL
+    buf = A + 50 * MB
+    for kw, code in [(dict(elems=175), lz.ZERO_ENOMEM),
+                     (dict(buf=buf + 8), lz.ZERO_EALIGN),
+                     (dict(buf=0), lz.ZERO_EINVAL),
+                     (dict(n_bufs=0), lz.ZERO_EINVAL),
+                     (dict(parts=[A, 0, A + 2 * MB, A + 3 * MB]), lz.ZERO_EINVAL),
+                     (dict(parts=[A + 1, A + MB, A + 2 * MB, A + 3 * MB]), lz.ZERO_EALIGN),
+                     (dict(buf=A + 2 * MB - 64), lz.ZERO_EINVAL),     # buffers over partition 2
+                     (dict(bounds=[0, 200]), lz.ZERO_EINVAL)]:
+        a = dict(elems=176, buf=buf, n_bufs=2, parts=parts, bounds=good)
+        a.update(kw)
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_layer_sched_create(pl, a["bounds"], a["parts"], a["buf"], a["elems"],
+                                       a["n_bufs"], 0)
+        assert e.value.code == code, kw
+
+
 def test_step_fused_ranges_rejects_before_launching():
     grads = [A + i * MB for i in range(2)]
     good = (1000, grads, A + 100 * MB, A + 101 * MB, A + 102 * MB, A + 110 * MB, A + 111 * MB,

@@ -55,6 +55,9 @@ SYMBOLS = (
     "zero_sched_slot_elems", "zero_sched_create", "zero_sched_create_fused",
     "zero_sched_begin_bucket", "zero_sched_rebind_fused", "zero_sched_rebind_status",
     "zero_sched_end_bucket", "zero_sched_wait", "zero_sched_launches", "zero_sched_destroy",
+    "zero_layer_sched_buf_elems", "zero_layer_sched_create", "zero_layer_sched_begin_step",
+    "zero_layer_sched_acquire", "zero_layer_sched_release", "zero_layer_sched_gathers",
+    "zero_layer_sched_destroy",
 )
 
 
@@ -189,6 +192,13 @@ def _load():
     L.zero_sched_wait.argtypes = [vp, vp]
     L.zero_sched_launches.argtypes = [vp, P(u64)]
     L.zero_sched_destroy.argtypes, L.zero_sched_destroy.restype = [vp], None
+    L.zero_layer_sched_buf_elems.argtypes = [vp, i32, P(u64), i32, P(u64)]
+    L.zero_layer_sched_create.argtypes = [vp, i32, P(u64), P(vp), vp, u64, i32, vp, P(vp)]
+    L.zero_layer_sched_begin_step.argtypes = [vp, vp, vp]
+    L.zero_layer_sched_acquire.argtypes = [vp, i32, i32, vp, P(vp)]
+    L.zero_layer_sched_release.argtypes = [vp, i32, vp]
+    L.zero_layer_sched_gathers.argtypes = [vp, P(u64)]
+    L.zero_layer_sched_destroy.argtypes, L.zero_layer_sched_destroy.restype = [vp], None
     # every other entry point returns a zero_status: ctypes' default int restype
     return L
 
@@ -513,6 +523,26 @@ def zero_stage3_step_fused(plan: Plan, flat_lo: int, length: int, rank_grads, ma
                                  _ptr(d_status, 4), _stream(stream)), "zero_stage3_step_fused")
 
 
+class PreparedStage3Update:
+    """zero_stage3_step_fused with its pointer arguments marshalled once (e.g. one layer's
+    update in one ping-pong direction); calling it with the step's hyperparameters (hparams_ref),
+    step, status address and stream handle makes the same C call."""
+
+    def __init__(self, plan: Plan, flat_lo: int, length: int, rank_grads, master_in, m_in, v_in,
+                 master_out, m_out, v_out, param_shards):
+        self._plan = plan                                     # kept alive with the handle
+        self._grads = _ptr_array(rank_grads, 2)
+        self._shards = _ptr_array(param_shards, 2)
+        self._args = (plan.handle, flat_lo, length, self._grads, _ptr(master_in, 4),
+                      _ptr(m_in, 4), _ptr(v_in, 4), _ptr(master_out, 4), _ptr(m_out, 4),
+                      _ptr(v_out, 4), self._shards)
+
+    def __call__(self, hp_ref, step: int, d_status: int, stream: int):
+        code = _lib.zero_stage3_step_fused(*self._args, hp_ref, step, d_status, stream)
+        if code:
+            raise ZeroError(code, "zero_stage3_step_fused")
+
+
 def zero_stage3_step_commit(plan: Plan, master_in, m_in, v_in, master_out, m_out, v_out, param_shards,
                       d_status, stream=None):
     _check(_lib.zero_stage3_step_commit(plan.handle, _ptr(master_in, 4), _ptr(m_in, 4), _ptr(v_in, 4),
@@ -617,6 +647,63 @@ def zero_sched_wait(s: Sched, stream=None):
 def zero_sched_launches(s: Sched) -> int:
     out = C.c_uint64()
     _check(_lib.zero_sched_launches(s.handle, C.byref(out)), "zero_sched_launches")
+    return out.value
+
+
+class LayerSched:
+    """Handle of a stage-3 layer scheduler (destroyed with this object)."""
+
+    def __init__(self, handle: int, n_layers: int):
+        self.handle = handle
+        self.n_layers = n_layers
+        self._out = C.c_void_p()
+
+    def __del__(self):
+        if getattr(self, "handle", None):
+            _lib.zero_layer_sched_destroy(self.handle)
+            self.handle = None
+
+
+def zero_layer_sched_buf_elems(plan: Plan, layer_bounds, n_bufs: int) -> int:
+    b = (C.c_uint64 * len(layer_bounds))(*layer_bounds)
+    out = C.c_uint64()
+    _check(_lib.zero_layer_sched_buf_elems(plan.handle, len(layer_bounds) - 1, b, n_bufs,
+                                           C.byref(out)), "zero_layer_sched_buf_elems")
+    return out.value
+
+
+def zero_layer_sched_create(plan: Plan, layer_bounds, param_shards, buf_mem, buf_mem_elems: int,
+                            n_bufs: int, gather_stream=None) -> LayerSched:
+    b = (C.c_uint64 * len(layer_bounds))(*layer_bounds)
+    h = C.c_void_p()
+    _check(_lib.zero_layer_sched_create(plan.handle, len(layer_bounds) - 1, b,
+                                        _ptr_array(param_shards, 2), _ptr(buf_mem, 2),
+                                        buf_mem_elems, n_bufs, _stream(gather_stream),
+                                        C.byref(h)), "zero_layer_sched_create")
+    return LayerSched(h.value, len(layer_bounds) - 1)
+
+
+def zero_layer_sched_begin_step(s: LayerSched, d_status, stream=None):
+    _check(_lib.zero_layer_sched_begin_step(s.handle, _ptr(d_status, 4), _stream(stream)),
+           "zero_layer_sched_begin_step")
+
+
+def zero_layer_sched_acquire(s: LayerSched, layer: int, prefetch: int = -1,
+                             compute=None) -> int:
+    """Returns the device address of the layer's gathered fp16 values."""
+    _check(_lib.zero_layer_sched_acquire(s.handle, layer, prefetch, _stream(compute),
+                                         C.byref(s._out)), "zero_layer_sched_acquire")
+    return int(s._out.value)
+
+
+def zero_layer_sched_release(s: LayerSched, layer: int, compute=None):
+    _check(_lib.zero_layer_sched_release(s.handle, layer, _stream(compute)),
+           "zero_layer_sched_release")
+
+
+def zero_layer_sched_gathers(s: LayerSched) -> int:
+    out = C.c_uint64()
+    _check(_lib.zero_layer_sched_gathers(s.handle, C.byref(out)), "zero_layer_sched_gathers")
     return out.value
 
 
