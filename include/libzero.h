@@ -437,9 +437,10 @@ zero_status zero_stage3_step_commit(const zero_plan* plan, const float* master_i
  * is not acquired before its buffer is needed is dropped; begin_step drops every layer still
  * in a buffer (the partitions have changed since). The pages have no scheduler interface; this
  * is the library's runtime for the stage-3 data path.
- * Errors: ZERO_EINVAL (bad plan or bounds, null pointers, a layer out of range or already
- * acquired, release of a layer not acquired, begin_step while a layer is acquired, a status
- * word inside a partition or the buffers), ZERO_EALIGN, ZERO_ENOMEM (buf_mem too small, every
+ * Errors: ZERO_EINVAL (bad plan or bounds, null pointers, an acquire before the first
+ * begin_step, a layer out of range or already acquired, release of a layer not acquired,
+ * begin_step while a layer is acquired, a status word inside a partition or the buffers),
+ * ZERO_EALIGN, ZERO_ENOMEM (buf_mem too small, every
  * buffer holding an acquired layer, host allocation), ZERO_ECUDA (event or launch failure).
  * ---------------------------------------------------------------------------------------- */
 typedef struct zero_layer_sched zero_layer_sched;
