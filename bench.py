@@ -23,8 +23,8 @@ Workloads (synthetic, seeded):
               8 partitions; a step gathers each of the 14 layers (embedding, 12 blocks, final
               LayerNorm) in forward order, then in backward order gathers each layer again and
               runs its fused update into the owners' partitions, then commits. The library's
-              layer scheduler runs the gathers one layer ahead on a second stream into two
-              layer buffers.
+              layer scheduler runs the gathers one layer ahead on a second stream into four
+              layer buffers (--layer-buffers).
   zero3_1p3b  the same on the 1.3B list (26 layers), Nd = 16.
   gpt2_small  GPT-2-small parameter list (psi = 123,653,376), Nd = 8, stage 1 (full local
               gradients, one fused call per step); grads N(0, 1e-3^2) with 1% x100; master
@@ -96,7 +96,7 @@ def parse():
     ap.add_argument("--l2", choices=["warm", "flushed"], default="warm",
                     help="flushed: write a buffer larger than L2 between timed steps and time each "
                          "step on its own (for the L2-resident tiny workload)")
-    ap.add_argument("--layer-buffers", type=int, default=2,
+    ap.add_argument("--layer-buffers", type=int, default=4,
                     help="stage-3 workloads: layer buffers of the layer scheduler (>= 1)")
     ap.add_argument("--no-sweep", action="store_true",
                     help="leave out the bucket / Nd sweep of the default line")
@@ -720,7 +720,7 @@ def _init_zero3(self, args, dev):
     """Stage 3 on a GPT-shaped list: every rank's full local gradient is resident (as the
     backward pass would leave it layer by layer); the fp16 parameters are Nd partitions of S
     values; the optimizer state is flat and ping-ponged. The library's layer scheduler gathers
-    the layers on a second stream into two layer buffers. A step: every layer acquired in
+    the layers on a second stream into --layer-buffers layer buffers. A step: every layer acquired in
     forward order (the next one prefetched), then per layer in backward order acquired again
     (the previous one prefetched), released, and updated (zero_stage3_step_fused), then
     zero_stage3_step_commit. Each fused call is timed with its own events in the last step."""

@@ -432,7 +432,9 @@ zero_status zero_stage3_step_commit(const zero_plan* plan, const float* master_i
  *   param_shards : the nd owners' partitions, S fp16 values each, 2-byte aligned (copied)
  *   buf_mem      : zero_layer_sched_buf_elems(...) fp16 values of caller device memory, 16-byte
  *                  aligned, not overlapping a partition: n_bufs buffers of the longest layer
- *                  rounded up to 8 values. n_bufs >= 2 lets one gather run ahead.
+ *                  rounded up to 8 values. n_bufs >= 2 lets one gather run ahead; with more
+ *                  buffers the gather stream waits for the compute stream less often (one wait
+ *                  covers every buffer released on that stream so far).
  * A released layer is discarded (acquiring it again gathers it again); a prefetched layer that
  * is not acquired before its buffer is needed is dropped; begin_step drops every layer still
  * in a buffer (the partitions have changed since). The pages have no scheduler interface; this

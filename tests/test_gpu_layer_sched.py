@@ -1,7 +1,7 @@
 """The stage-3 layer scheduler (zero_layer_sched_*) on the GPU against the oracle: whole
 stage-3 steps in which every layer is acquired through the scheduler in the forward pass (the
 next layer prefetched) and again in the backward pass (the previous layer prefetched, each
-layer's fused update after its release), with 1 to 3 layer buffers. Every acquired layer is
+layer's fused update after its release), with 1 to 4 layer buffers. Every acquired layer is
 copied out on the compute stream at the point where a layer's computation would read it, and
 equals the oracle's gathered layer bit for bit ("ZeRO" (lastdictionary): layers gathered just
 in time and discarded; "Como funciona": gathered in the forward and again in the backward
@@ -82,7 +82,7 @@ def _partitions(p16, nd, S):
     return out
 
 
-@pytest.mark.parametrize("nd,n_bufs", [(3, 2), (8, 2), (8, 3), (5, 1)])
+@pytest.mark.parametrize("nd,n_bufs", [(3, 2), (8, 2), (8, 3), (8, 4), (5, 1)])
 def test_layer_scheduler_steps_vs_oracle(nd, n_bufs):
     """Three attempts -- t = 1, an overflowing t = 2 (skipped), t = 2 -- through one scheduler
     on a side gather stream, layers straddling owners; with one buffer every prefetch is

@@ -37,7 +37,13 @@ struct zero_layer_sched {
     uint32_t* status = nullptr;
     std::vector<cudaEvent_t> gathered;    // per buffer: the last gather into it
     std::vector<cudaEvent_t> released;    // per buffer: its last user's release point
-    std::vector<int> rel_recorded;        // per buffer: released[] has been recorded once
+    std::vector<uint64_t> rel_seq;        // per buffer: number of its last release (0: none)
+    std::vector<cudaStream_t> rel_stream; // per buffer: the stream of its last release
+    uint64_t n_releases = 0;              // releases so far (numbers them)
+    // The gather stream has waited for every release on covered_stream numbered up to
+    // covered_seq (releases on one stream are ordered, so one wait covers the earlier ones).
+    cudaStream_t covered_stream = nullptr;
+    uint64_t covered_seq = 0;
     std::vector<int> layer_of_buf;        // per buffer: the layer it holds (-1: none)
     std::vector<int> buf_of_layer;        // per layer: the buffer holding it (-1: none)
     std::vector<int> held;                // per layer: acquired and not yet released
@@ -109,14 +115,33 @@ int free_buffer(const zero_layer_sched* s) {
     return best;
 }
 
+// Make the gather stream wait for buffer b's last release, unless an earlier wait already
+// covers it. The wait is on the latest release recorded on that stream (covering every buffer
+// released there so far), so that consecutive gathers are not each separated by a wait: a wait
+// between two kernels on the gather stream ends the programmatic overlap of the second one's
+// launch with the first one's tail.
+cudaError_t wait_release(zero_layer_sched* s, int b) {
+    const uint64_t need = s->rel_seq[(size_t)b];
+    const cudaStream_t st = s->rel_stream[(size_t)b];
+    if (need == 0 || (st == s->covered_stream && need <= s->covered_seq)) return cudaSuccess;
+    int latest = b;
+    for (int i = 0; i < s->n_bufs; ++i)
+        if (s->rel_stream[(size_t)i] == st && s->rel_seq[(size_t)i] > s->rel_seq[(size_t)latest])
+            latest = i;
+    const cudaError_t e = cudaStreamWaitEvent(s->gs, s->released[(size_t)latest], 0);
+    if (e == cudaSuccess) {
+        s->covered_stream = st;
+        s->covered_seq = s->rel_seq[(size_t)latest];
+    }
+    return e;
+}
+
 // Gather layer l into buffer b on the gather stream, after the buffer's last release.
 zero_status gather_into(zero_layer_sched* s, int l, int b) {
     const int old = s->layer_of_buf[(size_t)b];
     if (old >= 0) s->buf_of_layer[(size_t)old] = -1;   // an unused prefetch, dropped
     s->layer_of_buf[(size_t)b] = -1;
-    if (s->rel_recorded[(size_t)b] &&
-        cudaStreamWaitEvent(s->gs, s->released[(size_t)b], 0) != cudaSuccess)
-        return zk::from_cuda(cudaGetLastError());
+    if (wait_release(s, b) != cudaSuccess) return zk::from_cuda(cudaGetLastError());
     const uint64_t lo = s->bounds[(size_t)l], len = s->bounds[(size_t)l + 1] - lo;
     cudaError_t e = zk::launch_gather(lo, len, s->shard, s->nd, s->shards, buffer(s, b),
                                       s->status, s->gs);
@@ -178,7 +203,8 @@ zero_status zero_layer_sched_create(const zero_plan* plan, int n_layers,
         s->bounds.assign(layer_bounds, layer_bounds + n_layers + 1);
         s->gathered.assign((size_t)n_bufs, nullptr);
         s->released.assign((size_t)n_bufs, nullptr);
-        s->rel_recorded.assign((size_t)n_bufs, 0);
+        s->rel_seq.assign((size_t)n_bufs, 0);
+        s->rel_stream.assign((size_t)n_bufs, nullptr);
         s->layer_of_buf.assign((size_t)n_bufs, -1);
         s->stamp.assign((size_t)n_bufs, 0);
         s->buf_of_layer.assign((size_t)n_layers, -1);
@@ -219,7 +245,10 @@ zero_status zero_layer_sched_begin_step(zero_layer_sched* s, uint32_t* d_status,
     s->status = d_status;
     cudaError_t e = cudaEventRecord(s->step_ev, (cudaStream_t)stream);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(s->gs, s->step_ev, 0);
-    return e == cudaSuccess ? ZERO_OK : zk::from_cuda(e);
+    if (e != cudaSuccess) return zk::from_cuda(e);
+    s->covered_stream = (cudaStream_t)stream;   // every release on `stream` so far is covered
+    s->covered_seq = s->n_releases;
+    return ZERO_OK;
 }
 
 zero_status zero_layer_sched_acquire(zero_layer_sched* s, int layer, int prefetch,
@@ -253,7 +282,8 @@ zero_status zero_layer_sched_release(zero_layer_sched* s, int layer, zero_stream
     if (b < 0) return ZERO_EINVAL;
     const cudaError_t e = cudaEventRecord(s->released[(size_t)b], (cudaStream_t)compute);
     if (e != cudaSuccess) return zk::from_cuda(e);
-    s->rel_recorded[(size_t)b] = 1;
+    s->rel_seq[(size_t)b] = ++s->n_releases;
+    s->rel_stream[(size_t)b] = (cudaStream_t)compute;
     s->held[(size_t)layer] = 0;
     s->buf_of_layer[(size_t)layer] = -1;   // discarded
     s->layer_of_buf[(size_t)b] = -1;
