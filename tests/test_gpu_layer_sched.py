@@ -136,6 +136,54 @@ def test_layer_scheduler_steps_vs_oracle(nd, n_bufs):
         w_r, m_r, v_r, ref_shards = ref.master, ref.m, ref.v, ref.param_shards
 
 
+@pytest.mark.parametrize("n_bufs", [2, 3])
+def test_layer_scheduler_two_compute_streams(n_bufs):
+    """Layers acquired and released on two compute streams in turn (a release on one stream
+    does not order the other's): every layer as acquired, forward and backward, equals the
+    partitions' values, three steps in a row through one scheduler."""
+    numels, nd = [3000, 7001, 512, 9000, 2048, 4000], 4
+    pl = lz.zero_plan_create(numels, nd, 3, 0)
+    psi, psi_p, S, _ = lz.zero_plan_info(pl)
+    offs = lz.zero_plan_tensor_offsets(pl)
+    bounds = list(offs) + [psi_p]
+    L = len(bounds) - 1
+    pool = _Pool(pl, bounds, n_bufs)
+    gs = torch.cuda.Stream()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    main = torch.cuda.current_stream()
+    st = status_word()
+    for step in range(3):
+        full = torch.randint(-(1 << 15), 1 << 15, (psi_p,), dtype=torch.int16,
+                             device=DEV).view(torch.float16)
+        shards = [full[q * S:(q + 1) * S].clone() for q in range(nd)]
+        if step == 0:
+            sched = lz.zero_layer_sched_create(pl, bounds, shards, pool.mem, pool.elems, n_bufs,
+                                               gs)
+            keep = shards
+        else:                       # new values in the same partitions, as an update would write
+            for k, x in zip(keep, shards):
+                k.copy_(x)
+        for c in streams:
+            c.wait_stream(main)
+        lz.zero_layer_sched_begin_step(sched, st, main)
+        seen = []
+        order = list(range(L)) + list(reversed(range(L)))
+        for i, l in enumerate(order):
+            c = streams[i % 2]
+            nxt = order[i + 1] if i + 1 < len(order) else -1
+            p = lz.zero_layer_sched_acquire(sched, l, nxt, c)
+            with torch.cuda.stream(c):
+                seen.append((l, pool.view(p, bounds[l + 1] - bounds[l]).clone()))
+            lz.zero_layer_sched_release(sched, l, c)
+        for c in streams:
+            main.wait_stream(c)
+        torch.cuda.synchronize()
+        for l, got in seen:
+            lo, hi = bounds[l], bounds[l + 1]
+            assert torch.equal(got.view(torch.int16), full[lo:hi].view(torch.int16)), (step, l)
+    assert lz.zero_step_status(st) == (lz.ZERO_OK, 0)
+
+
 def test_layer_scheduler_bookkeeping():
     """Host-side rules on a live scheduler: a layer cannot be acquired twice or released
     unacquired; a step cannot begin while a layer is held; with every buffer held the next
