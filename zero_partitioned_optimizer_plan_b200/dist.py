@@ -281,8 +281,11 @@ class DistZeroStep:
         return self._recv
 
     def step(self, local_grad, state_in: Sequence, state_out: Sequence, params_full, hp,
-             t: int, status):
-        """local_grad: this rank's fp16 gradient (psi_p, contiguous); state_in / state_out:
+             t: int, status, before_bucket=None):
+        """before_bucket(k), if given, runs before bucket k's exchange is issued (stage 3: the
+        backward gather of the bucket's layer, which the layer's backward computation, and so
+        its gradient bucket, comes after).
+        local_grad: this rank's fp16 gradient (psi_p, contiguous); state_in / state_out:
         this rank's fp32 master, m, v shards (S each, distinct buffers); params_full: the fp16
         parameter buffer (psi_p), whose own range is updated and the rest gathered; status:
         this rank's zeroed int32 status word, which ends with the job-wide void bits and, if
@@ -299,16 +302,19 @@ class DistZeroStep:
         works = [None] * nb
         if self.peers is not None:
             if self.payload == "q8":
-                self._reduce_q8_from_peers(local_grad, state_in, state_out, own, hp, t, status)
+                self._reduce_q8_from_peers(local_grad, state_in, state_out, own, hp, t, status,
+                                           before_bucket)
                 return self._finish(state_in, state_out, own, params_full, status)
             if local_grad is not self.peers.local:
                 self.peers.local.copy_(local_grad)   # produce into peers.local to avoid this
-            self._reduce_from_peers(state_in, state_out, own, hp, t, status)
+            self._reduce_from_peers(state_in, state_out, own, hp, t, status, before_bucket)
             return self._finish(state_in, state_out, own, params_full, status)
 
         q8 = self.payload == "q8"
 
         def exchange(k):
+            if before_bucket is not None:
+                before_bucket(k)
             lo, hi = self.buckets[k]
             parts = self.parts[k]
             mine = parts[r]
@@ -363,7 +369,7 @@ class DistZeroStep:
         self.compute.fused_replicas(n, rows, ins, outs, self.param_peers.rows(lo, lo + n), hp,
                                     t, status)
 
-    def _reduce_from_peers(self, state_in, state_out, own, hp, t, status):
+    def _reduce_from_peers(self, state_in, state_out, own, hp, t, status, before_bucket=None):
         """Per bucket: a barrier (every rank has produced it), then the owner's fused step on
         its part, reading the Nd rows in the peers' buffers. The barrier of bucket k+1 is in
         flight while bucket k is reduced."""
@@ -372,6 +378,8 @@ class DistZeroStep:
         works = [None] * nb
 
         def barrier(k):
+            if before_bucket is not None:
+                before_bucket(k)
             works[k] = dist.all_reduce(self._tick, group=self.group, async_op=True)
 
         barrier(0)
@@ -388,7 +396,8 @@ class DistZeroStep:
                          [x[a - r * S:b - r * S] for x in state_out], own, a - r * S, hp, t,
                          status)
 
-    def _reduce_q8_from_peers(self, local_grad, state_in, state_out, own, hp, t, status):
+    def _reduce_q8_from_peers(self, local_grad, state_in, state_out, own, hp, t, status,
+                              before_bucket=None):
         """Per bucket: quantize this rank's part for every owner into its own peer buffer, a
         barrier (every rank has quantized the bucket), then the owner's int8 step over the Nd
         payloads of its part, read in the peers' buffers. Bucket k+1 is quantized and its
@@ -399,6 +408,8 @@ class DistZeroStep:
         mine_buf = self.peers.local
 
         def produce(k):
+            if before_bucket is not None:
+                before_bucket(k)
             lo, hi = self.buckets[k]
             for q, x in enumerate(self.parts[k]):
                 if x:
@@ -483,7 +494,9 @@ class DistStage3Step:
     backward, per layer in reverse order: the gather again, then the layer's gradient bucket
     (its range; the last layer's extended over the padding, the end of the flat list being
     produced first) reduce-scattered to its owners and each owner's fused update written into
-    its own partition (DistZeroStep with the layers' gradient buckets); the job-wide verdict;
+    its own partition (DistZeroStep with the layers' gradient buckets; the gather of a layer
+    runs before its bucket's exchange is issued, so it interleaves with the earlier buckets'
+    exchanges and updates, which touch other layers' ranges); the job-wide verdict;
     nothing is gathered after the step. The gathered layer goes to ``layer_buf`` (the buffer
     the layer's computation would read); ``record`` (a list) receives a copy of each gathered
     layer, forward then backward, for checking."""
@@ -515,10 +528,16 @@ class DistStage3Step:
         peer-read form); state_in / state_out: this rank's fp32 shards; layer_buf: a buffer of
         the largest layer's length. Returns the job-wide void bits; raises DistStepError on
         every rank if any rank's kernels failed."""
-        order = list(range(len(self.layers)))
-        for l in order + order[::-1]:        # forward, then backward
+        L = len(self.layers)
+
+        def use(l):                          # gather layer l just in time (and record it)
             self.gather(l, layer_buf, status)
             if record is not None:
                 record.append(layer_buf[:self.layers[l][1] - self.layers[l][0]].clone())
+
+        for l in range(L):                   # forward
+            use(l)
+        # backward: layer l's gather before its gradient bucket (bucket L-1-l) is exchanged, so
+        # the backward gathers interleave with the earlier buckets' exchanges and updates
         return self.inner.step(local_grad, state_in, state_out, self.part_peers.local, hp, t,
-                               status)
+                               status, before_bucket=lambda k: use(L - 1 - k))
