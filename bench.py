@@ -157,6 +157,9 @@ def workload_config(args) -> dict:
             cfg["workload"] = kind + "_fused"
             cfg["calls_per_step"] = nb + 1
         cfg["overlap"] = not args.no_overlap
+        if args.payload == "q8":
+            cfg["payload"] = "int8 records: 128 values and their fp32 scale"
+            cfg["workload"] += "_q8"
         return cfg
     else:
         nd = args.nd or 16
@@ -497,9 +500,10 @@ def _init_zero2(self, args, dev):
     serves every step; between steps it is rebound to the step's buffers and status word."""
     torch, lz = self.torch, self.lz
     from zero_partitioned_optimizer_plan_b200 import synth
-    if args.payload != "fp16":
-        raise SystemExit("the stage-2 workloads take fp16 payloads")
-    self.payload = "fp16"
+    q8 = args.payload == "q8"
+    if q8 and args.stage2 != "fused":
+        raise SystemExit("the int8 payload takes the fused stage-2 scheduler")
+    self.payload = args.payload
     small = args.workload == "zero2_gpt2_small"
     nd = args.nd or (8 if small else 16)
     B = args.bucket or (10_000_000 if small else 50_000_000)
@@ -507,15 +511,29 @@ def _init_zero2(self, args, dev):
     self.plan = pl = lz.zero_plan_create(numels, nd, 2, B)
     psi, psi_p, S, nb = lz.zero_plan_info(pl)
     self.nd, self.n, self.psi, self.S, self.nb = nd, psi_p, psi, S, nb
-    self.slot_elems = lz.zero_sched_slot_elems(pl, nb)
-    self.slots = torch.empty(self.slot_elems, dtype=torch.float16, device=dev)
-    self.stride = self.slot_elems // (nb * nd)
     self.buckets = [lz.zero_plan_bucket(pl, k)[:2] for k in range(nb)]
-    for k, (lo, ln) in enumerate(self.buckets):
-        for r in range(nd):
-            base = (k * nd + r) * self.stride
-            synth.grad_f16(ln, 1e-3, seed=0, rank=r, step=1000 + k,
-                           out=self.slots[base:base + ln])
+    if q8:
+        # every bucket's int8 records of every rank, quantized once from the same gradients
+        self.slot_elems = lz.zero_sched_slot_bytes_q8(pl, nb)
+        self.slots = torch.empty(self.slot_elems, dtype=torch.uint8, device=dev)
+        self.stride = self.slot_elems // (nb * nd)         # bytes per rank region
+        tmp = torch.empty(max(ln for _, ln in self.buckets), dtype=torch.float16, device=dev)
+        for k, (lo, ln) in enumerate(self.buckets):
+            for r in range(nd):
+                base = (k * nd + r) * self.stride
+                synth.grad_f16(ln, 1e-3, seed=0, rank=r, step=1000 + k, out=tmp[:ln])
+                lz.zero_quantize_q8(ln, tmp[:ln],
+                                    self.slots[base:base + lz.q8_payload_bytes(ln)])
+        del tmp
+    else:
+        self.slot_elems = lz.zero_sched_slot_elems(pl, nb)
+        self.slots = torch.empty(self.slot_elems, dtype=torch.float16, device=dev)
+        self.stride = self.slot_elems // (nb * nd)
+        for k, (lo, ln) in enumerate(self.buckets):
+            for r in range(nd):
+                base = (k * nd + r) * self.stride
+                synth.grad_f16(ln, 1e-3, seed=0, rank=r, step=1000 + k,
+                               out=self.slots[base:base + ln])
     self.master, self.m, self.v = synth.state_small(psi_p, seed=0, device=dev)
     self.params = torch.empty(psi_p, dtype=torch.float16, device=dev)
     self.grads = None
@@ -535,11 +553,19 @@ def _init_zero2(self, args, dev):
         self.d_consts = torch.empty(nb_c, dtype=torch.uint8, device=dev)
         self.h_consts = [torch.empty(nb_c, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
         self.h_done = [None, None]
-        self.sched = lz.zero_sched_create_fused(pl, self.slots, self.slot_elems, nb, *self.cur,
-                                                *self.nxt, self.params, self.d_consts,
-                                                self.st_create, stream)
-        self.bytes_per_step = (2 * nd + 26) * psi_p
-        self.dominant = "fused_tma_kernel"
+        if q8:
+            self.sched = lz.zero_sched_create_fused_q8(pl, self.slots, self.slot_elems, nb,
+                                                       *self.cur, *self.nxt, self.params,
+                                                       self.d_consts, self.st_create, stream)
+            self.bytes_per_step = (nd * sum(lz.q8_payload_bytes(ln) for _, ln in self.buckets)
+                                   + 26 * psi_p)
+            self.dominant = "fused_q8_tma_kernel"
+        else:
+            self.sched = lz.zero_sched_create_fused(pl, self.slots, self.slot_elems, nb,
+                                                    *self.cur, *self.nxt, self.params,
+                                                    self.d_consts, self.st_create, stream)
+            self.bytes_per_step = (2 * nd + 26) * psi_p
+            self.dominant = "fused_tma_kernel"
         self.dominant_bytes = self.bytes_per_step
         self.dominant_calls = nb
         self.side = None
@@ -602,10 +628,11 @@ def _step_zero2_fused(self, t, status, ev=None, grads=None):
     lz.zero_sched_rebind_fused(sch, *self.cur, *self.nxt, self.params, status)
     if ev is not None:
         ev[0].record()
+    begin = lz.zero_sched_begin_bucket_q8 if self.payload == "q8" else lz.zero_sched_begin_bucket
     if self.overlap:
         lz.zero_overlap_begin(stream)
     for k in range(self.nb):
-        lz.zero_sched_begin_bucket(sch, k, stream)
+        begin(sch, k, stream)
         lz.zero_sched_end_bucket(sch, k, stream)
     if self.overlap:
         lz.zero_overlap_end(stream)
@@ -625,9 +652,15 @@ def _e2e_zero2_fused(self, t0, E, barrier, max_ms):
     the status. The next step's uploads overlap this step's tail and download."""
     torch, lz = self.torch, self.lz
     dev, nd, pl = self.params.device, self.nd, self.plan
+    q8 = self.payload == "q8"        # int8 records uploaded instead of fp16 gradients
     n_slots = 2
-    slot_elems = lz.zero_sched_slot_elems(pl, n_slots)
-    d_slots = torch.empty(slot_elems, dtype=torch.float16, device=dev)
+    if q8:
+        slot_elems = lz.zero_sched_slot_bytes_q8(pl, n_slots)
+        d_slots = torch.empty(slot_elems, dtype=torch.uint8, device=dev)
+    else:
+        slot_elems = lz.zero_sched_slot_elems(pl, n_slots)
+        d_slots = torch.empty(slot_elems, dtype=torch.float16, device=dev)
+    esize = d_slots.element_size()
     region = nd * self.stride
     # pinned host source: every bucket's gradients when the host has room (42 GB for the 1.3B
     # list at Nd = 16), else as many buckets as half the host's available memory allows per
@@ -639,18 +672,20 @@ def _e2e_zero2_fused(self, t0, E, barrier, max_ms):
     except Exception:
         avail = 0
     host_buckets = self.nb
-    if avail and self.nb * region * 2 > avail // (2 * ws):
-        host_buckets = max(2, min(self.nb, (avail // (2 * ws)) // (region * 2)))
+    if avail and self.nb * region * esize > avail // (2 * ws):
+        host_buckets = max(2, min(self.nb, (avail // (2 * ws)) // (region * esize)))
     total = host_buckets * region
-    h_grads = pinned_host(total, torch.float16)
+    h_grads = pinned_host(total, d_slots.dtype)
     h_grads.copy_(self.slots[:total])          # the same gradients as the device-resident run
     h_params = [torch.empty(self.n, dtype=torch.float16, pin_memory=True) for _ in range(2)]
     h_status = [torch.empty(1, dtype=torch.int32, pin_memory=True) for _ in range(2)]
     st = torch.zeros(E, dtype=torch.int32, device=dev)
     main = torch.cuda.current_stream()
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
-    sch = lz.zero_sched_create_fused(pl, d_slots, slot_elems, n_slots, *self.cur, *self.nxt,
-                                     self.params, self.d_consts, st[0:1], main)
+    create = lz.zero_sched_create_fused_q8 if q8 else lz.zero_sched_create_fused
+    begin = lz.zero_sched_begin_bucket_q8 if q8 else lz.zero_sched_begin_bucket
+    sch = create(pl, d_slots, slot_elems, n_slots, *self.cur, *self.nxt, self.params,
+                 self.d_consts, st[0:1], main)
     h2d = 0
     comp_done, down_done = [None, None], [None, None]
     torch.cuda.synchronize()
@@ -674,14 +709,15 @@ def _e2e_zero2_fused(self, t0, E, barrier, max_ms):
         if self.overlap:
             lz.zero_overlap_begin(main)
         for k, (lo, ln) in enumerate(self.buckets):
-            ptrs = lz.zero_sched_begin_bucket(sch, k, up)
+            ptrs = begin(sch, k, up)
+            cnt = lz.q8_payload_bytes(ln) if q8 else ln       # elements of a rank's part
             with torch.cuda.stream(up):
                 hk = k % host_buckets
                 for r in range(nd):
-                    off = (ptrs[r] - d_slots.data_ptr()) // 2
-                    src = h_grads[hk * region + r * self.stride:hk * region + r * self.stride + ln]
-                    d_slots[off:off + ln].copy_(src, non_blocking=True)
-                    h2d += 2 * ln if i == 0 else 0
+                    off = (ptrs[r] - d_slots.data_ptr()) // esize
+                    a = hk * region + r * self.stride
+                    d_slots[off:off + cnt].copy_(h_grads[a:a + cnt], non_blocking=True)
+                    h2d += esize * cnt if i == 0 else 0
             lz.zero_sched_end_bucket(sch, k, up)
         if self.overlap:
             lz.zero_overlap_end(main)
@@ -707,8 +743,11 @@ def _e2e_zero2_fused(self, t0, E, barrier, max_ms):
     lz.zero_sched_destroy(sch)
     ems = max_ms(e0.elapsed_time(e1))
     out = {"ms": ems, "steps": E, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 2 * self.n + 4,
-           "overlap": "bucket uploads into two staging slots, each gated by the release of its "
-                      "slot; the next step's uploads overlap this step's tail and download",
+           "overlap": ("bucket uploads (int8 records) into two staging slots, each gated by the "
+                       "release of its slot; the next step's uploads overlap this step's tail "
+                       "and download") if q8 else
+                      ("bucket uploads into two staging slots, each gated by the release of its "
+                       "slot; the next step's uploads overlap this step's tail and download"),
            "host_source": (f"all {self.nb} buckets in pinned host memory" if host_buckets ==
                            self.nb else f"{host_buckets} buckets in pinned host memory, cycled")}
     unpin_host(h_grads)
@@ -1366,7 +1405,7 @@ def run_ours(args):
                "host": host_cpu()}
 
     main_line = wl.config["workload"].startswith("zero2_1p3b") and args.stage2 == "fused" and \
-        not args.graph
+        not args.graph and args.payload == "fp16"
     sweep = None
     if main_line and not args.no_sweep:
         cfg0, nd0, bytes0 = dict(wl.config), wl.nd, wl.bytes_per_step

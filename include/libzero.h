@@ -617,6 +617,27 @@ zero_status zero_sched_create_fused(const zero_plan* plan, uint16_t* slot_mem,
                                     float* m_out, float* v_out, uint16_t* param_out,
                                     const zero_adam_consts* d_consts, uint32_t* d_status,
                                     zero_stream_t stream, zero_sched** out);
+/* The int8 payload in the bucket pipeline. "ZeRO" (lastdictionary.com), main definition:
+ * ZeRO++ compresses the communication; the format is ZERO_Q8_BLOCK-value records (below).
+ * Fused mode with each rank's part of a bucket arriving as int8 records: the staging slots
+ * hold, per rank, ZERO_Q8_PAYLOAD_BYTES(len) bytes of records counted from the bucket's first
+ * element (as zero_quantize_q8 writes them for the rank's len values of the bucket), in
+ * regions of the longest bucket's record bytes rounded up to 16; the kernel launched for
+ * bucket k is zero_step_fused_q8_dc over the bucket's range. slot_mem: 16-byte aligned,
+ * zero_sched_slot_bytes_q8(...) bytes. The producer fills the regions that
+ * zero_sched_begin_bucket_q8 returns (zero_sched_begin_bucket is rejected for such a
+ * scheduler, and zero_sched_begin_bucket_q8 for the others). Rebind, wait and commit as in the
+ * fp16 fused mode. Errors: as zero_sched_create_fused. */
+zero_status zero_sched_slot_bytes_q8(const zero_plan* plan, int n_slots, uint64_t* bytes);
+zero_status zero_sched_create_fused_q8(const zero_plan* plan, uint8_t* slot_mem,
+                                       uint64_t slot_mem_bytes, int n_slots,
+                                       const float* master_in, const float* m_in,
+                                       const float* v_in, float* master_out, float* m_out,
+                                       float* v_out, uint16_t* param_out,
+                                       const zero_adam_consts* d_consts, uint32_t* d_status,
+                                       zero_stream_t stream, zero_sched** out);
+zero_status zero_sched_begin_bucket_q8(zero_sched* s, int k, zero_stream_t producer,
+                                       uint8_t** rank_ptrs);
 /* Between steps: point the fused scheduler at the next step's state, parameters and status
  * word (same layout and checks as zero_sched_create_fused), e.g. the swapped ping-pong buffers.
  * Kernels already enqueued keep the old pointers; the CUDA events and slots are reused, so a

@@ -321,6 +321,38 @@ def test_overlap_region_bookkeeping():
     assert e.value.code == lz.ZERO_EINVAL
 
 
+def test_q8_scheduler_sizes_and_rejects():
+    """zero_sched_create_fused_q8: slots of n_slots x nd regions of the longest bucket's int8
+    records rounded up to 16 bytes, and the fp16 fused mode's argument checks."""
+    pl = lz.zero_plan_create([100, 28], 4, 2, 32)     # psi_p = 128, buckets of 32
+    assert lz.zero_sched_slot_bytes_q8(pl, 2) == 2 * 4 * 144    # one 132-byte record -> 144
+    pl2 = lz.zero_plan_create([1000, 300], 2, 2, 600)          # longest bucket 600: 5 records
+    assert lz.zero_sched_slot_bytes_q8(pl2, 3) == 3 * 2 * 672   # 660 -> 672
+    need = lz.zero_sched_slot_bytes_q8(pl, 2)
+    slots = A
+    ins = [A + 10 * MB, A + 11 * MB, A + 12 * MB]
+    outs = [A + 20 * MB, A + 21 * MB, A + 22 * MB]
+    par, dc, st = A + 30 * MB, A + 31 * MB, A + 32 * MB
+    ok = dict(slots=slots, size=need, master_in=ins[0], master_out=outs[0], param_out=par,
+              d_consts=dc, d_status=st)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lz.zero_sched_create_fused_q8(pl, a["slots"], a["size"], 2, a["master_in"], ins[1],
+                                             ins[2], a["master_out"], outs[1], outs[2],
+                                             a["param_out"], a["d_consts"], a["d_status"], 0)
+
+    for kw, code in [({"size": need - 1}, lz.ZERO_ENOMEM), ({"slots": slots + 8}, lz.ZERO_EALIGN),
+                     ({"slots": 0}, lz.ZERO_EINVAL), ({"d_consts": 0}, lz.ZERO_EINVAL),
+                     ({"master_in": 0}, lz.ZERO_EINVAL),
+                     ({"master_out": ins[0]}, lz.ZERO_EINVAL),        # output over an input
+                     ({"param_out": slots + 100}, lz.ZERO_EINVAL),    # output over the slots
+                     ({"d_status": slots + need - 4}, lz.ZERO_EINVAL)]:
+        with pytest.raises(lz.ZeroError) as e:
+            call(**kw)
+        assert e.value.code == code, kw
+
+
 def test_fused_scheduler_rejects():
     """zero_sched_create_fused checks the plan, the state arrays (psi_p values each), the
     constants pointer and that no output overlaps an input, another output or the slots."""

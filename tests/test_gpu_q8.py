@@ -396,3 +396,90 @@ def test_step_fused_q8_ranges_vs_oracle(nd):
     check_f32("m", f32np(outs_a[1]), mm, tol=0)
     check_f32("v", f32np(outs_a[2]), vv, tol=0)
     check_f16("params", f16np(pa), p, tol=0)
+
+
+def _byte_view(slots, ptr, n):
+    off = ptr - slots.data_ptr()
+    assert 0 <= off and off + n <= slots.numel()
+    return slots[off:off + n]
+
+
+@pytest.mark.parametrize("n_slots", [1, 2])
+def test_q8_bucket_scheduler_vs_oracle(n_slots):
+    """Stage 2 with the int8 payload through one scheduler (zero_sched_create_fused_q8): each
+    bucket's part of every rank's gradient quantized into the slot region that
+    zero_sched_begin_bucket_q8 hands out (records counted from the bucket's first element), the
+    int8 fused step launched per bucket, one commit. Four attempts -- t = 1, an attempt with a
+    poisoned block (skipped, t not advanced), t = 2, t = 3 -- against the oracle's quantizer and
+    int8 step over the same buckets; the state bit for bit (one fma per rank, as the oracle)."""
+    numels, nd, bucket = [40000, 1234, 30000, 777], 6, 9000
+    pl = lz.zero_plan_create(numels, nd, 2, bucket)
+    psi, psi_p, S, nb = lz.zero_plan_info(pl)
+    master, m, v = synth.state_warm(psi_p, seed=141)
+    pp = PingPong(master, m, v)
+    params = torch.from_numpy(oracle.f2h(master.numpy()).view(np.float16)).to(DEV)
+    nbytes = lz.zero_sched_slot_bytes_q8(pl, n_slots)
+    slots = torch.empty(nbytes, dtype=torch.uint8, device=DEV)
+    d_consts = torch.empty(lz.ZERO_ADAM_CONSTS_BYTES, dtype=torch.uint8, device=DEV)
+    producer, stream = torch.cuda.Stream(), torch.cuda.Stream()
+    main = torch.cuda.current_stream()
+    sch = lz.zero_sched_create_fused_q8(pl, slots, nbytes, n_slots, *pp.cur, *pp.nxt, params,
+                                        d_consts, status_word(), stream)
+    with pytest.raises(lz.ZeroError):             # the fp16 hand-out is refused here
+        lz.zero_sched_begin_bucket(sch, 0, producer)
+    w, mm, vv = master.numpy(), m.numpy(), v.numpy()
+    p16 = oracle.f2h(w)
+    buckets = [lz.zero_plan_bucket(pl, k)[:2] for k in range(nb)]
+    for i, (t, bad) in enumerate([(1, None), (2, (nb // 2, 4)), (2, None), (3, None)]):
+        g = []
+        for r in range(nd):
+            x = torch.zeros(psi_p, dtype=torch.float16)
+            x[:psi] = synth.grad_f16(psi, 1e-3, seed=142, rank=r, step=10 * i + t)
+            g.append(x)
+        if bad is not None:
+            k, r = bad
+            g[r][buckets[k][0] + 5] = float("nan")
+        st = status_word()
+        c = lz.zero_adam_consts_for_step(HP, t)
+        d_consts.copy_(torch.frombuffer(bytearray(bytes(c)), dtype=torch.uint8))
+        torch.cuda.synchronize()
+        lz.zero_sched_rebind_fused(sch, *pp.cur, *pp.nxt, params, st)
+        g_dev = [x.to(DEV) for x in g]
+        torch.cuda.synchronize()
+        lz.zero_overlap_begin(stream)
+        with torch.cuda.stream(producer):
+            for k, (lo, ln) in enumerate(buckets):
+                ptrs = lz.zero_sched_begin_bucket_q8(sch, k, producer)
+                for r in range(nd):
+                    lz.zero_quantize_q8(ln, g_dev[r][lo:lo + ln],
+                                        _byte_view(slots, ptrs[r], lz.q8_payload_bytes(ln)),
+                                        producer)
+                lz.zero_sched_end_bucket(sch, k, producer)
+        lz.zero_overlap_end(stream)
+        lz.zero_sched_wait(sch, main)
+        lz.zero_step_commit(psi_p, *pp.cur, *pp.nxt, params, st, main)
+        code, flags = lz.zero_step_status(st, main)
+        # the oracle: each bucket's parts quantized from the bucket's first element, the int8
+        # step per bucket; any overflow skips the whole step
+        w2, m2, v2, p2 = w.copy(), mm.copy(), vv.copy(), p16.copy()
+        skipped = False
+        for lo, ln in buckets:
+            qs = [oracle.quant_q8(x.numpy()[lo:lo + ln]) for x in g]
+            sk, wb, mb, vb, pb = oracle.step_q8([q for q, _ in qs], [sc for _, sc in qs],
+                                                w[lo:lo + ln], mm[lo:lo + ln], vv[lo:lo + ln],
+                                                ORC_HP, t)
+            skipped |= sk
+            if not sk:
+                w2[lo:lo + ln], m2[lo:lo + ln], v2[lo:lo + ln], p2[lo:lo + ln] = wb, mb, vb, pb
+        assert skipped == (bad is not None)
+        if skipped:
+            assert code == lz.ZERO_STEP_SKIPPED
+        else:
+            assert (code, flags) == (lz.ZERO_OK, 0)
+            w, mm, vv, p16 = w2, m2, v2, p2
+        pp.swap()
+        check_f32(f"attempt {i} master", f32np(pp.cur[0]), w, tol=0)
+        check_f32(f"attempt {i} m", f32np(pp.cur[1]), mm, tol=0)
+        check_f32(f"attempt {i} v", f32np(pp.cur[2]), vv, tol=0)
+        check_f16(f"attempt {i} params", f16np(params), p16, tol=0)
+    lz.zero_sched_destroy(sch)

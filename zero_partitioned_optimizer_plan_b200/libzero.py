@@ -55,6 +55,7 @@ SYMBOLS = (
     "zero_sched_slot_elems", "zero_sched_create", "zero_sched_create_fused",
     "zero_sched_begin_bucket", "zero_sched_rebind_fused", "zero_sched_rebind_status",
     "zero_sched_end_bucket", "zero_sched_wait", "zero_sched_launches", "zero_sched_destroy",
+    "zero_sched_slot_bytes_q8", "zero_sched_create_fused_q8", "zero_sched_begin_bucket_q8",
     "zero_layer_sched_buf_elems", "zero_layer_sched_create", "zero_layer_sched_begin_step",
     "zero_layer_sched_acquire", "zero_layer_sched_release", "zero_layer_sched_gathers",
     "zero_layer_sched_destroy",
@@ -192,6 +193,10 @@ def _load():
     L.zero_sched_wait.argtypes = [vp, vp]
     L.zero_sched_launches.argtypes = [vp, P(u64)]
     L.zero_sched_destroy.argtypes, L.zero_sched_destroy.restype = [vp], None
+    L.zero_sched_slot_bytes_q8.argtypes = [vp, i32, P(u64)]
+    L.zero_sched_create_fused_q8.argtypes = [vp, vp, u64, i32, vp, vp, vp, vp, vp, vp, vp, vp,
+                                             vp, vp, P(vp)]
+    L.zero_sched_begin_bucket_q8.argtypes = [vp, i32, vp, P(vp)]
     L.zero_layer_sched_buf_elems.argtypes = [vp, i32, P(u64), i32, P(u64)]
     L.zero_layer_sched_create.argtypes = [vp, i32, P(u64), P(vp), vp, u64, i32, vp, P(vp)]
     L.zero_layer_sched_begin_step.argtypes = [vp, vp, vp]
@@ -615,6 +620,34 @@ def zero_sched_create_fused(plan: Plan, slot_mem, slot_mem_elems: int, n_slots: 
                                         _stream(stream), C.byref(h)), "zero_sched_create_fused")
     _, psi_p, shard, _ = zero_plan_info(plan)
     return Sched(h.value, psi_p // shard if shard else 1)
+
+
+def zero_sched_slot_bytes_q8(plan: Plan, n_slots: int) -> int:
+    out = C.c_uint64()
+    _check(_lib.zero_sched_slot_bytes_q8(plan.handle, n_slots, C.byref(out)),
+           "zero_sched_slot_bytes_q8")
+    return out.value
+
+
+def zero_sched_create_fused_q8(plan: Plan, slot_mem, slot_mem_bytes: int, n_slots: int,
+                               master_in, m_in, v_in, master_out, m_out, v_out, param_out,
+                               d_consts, d_status, stream=None) -> Sched:
+    h = C.c_void_p()
+    _check(_lib.zero_sched_create_fused_q8(plan.handle, _ptr(slot_mem, 1), slot_mem_bytes,
+                                           n_slots, _ptr(master_in, 4), _ptr(m_in, 4),
+                                           _ptr(v_in, 4), _ptr(master_out, 4), _ptr(m_out, 4),
+                                           _ptr(v_out, 4), _ptr(param_out, 2), _ptr(d_consts),
+                                           _ptr(d_status, 4), _stream(stream), C.byref(h)),
+           "zero_sched_create_fused_q8")
+    _, psi_p, shard, _ = zero_plan_info(plan)
+    return Sched(h.value, psi_p // shard if shard else 1)
+
+
+def zero_sched_begin_bucket_q8(s: Sched, k: int, producer=None) -> List[int]:
+    out = (C.c_void_p * s.nd)()
+    _check(_lib.zero_sched_begin_bucket_q8(s.handle, k, _stream(producer), out),
+           "zero_sched_begin_bucket_q8")
+    return [int(p) for p in out]
 
 
 def zero_sched_rebind_fused(s: Sched, master_in, m_in, v_in, master_out, m_out, v_out,
