@@ -401,6 +401,20 @@ zero_status zero_stage3_step_fused(const zero_plan* plan, uint64_t flat_lo, uint
                              const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
                              zero_stream_t stream);
 
+/* zero_stage3_step_fused with the step's constants read from device memory when the kernels
+ * run (d_consts: a zero_adam_consts, 4-byte aligned, e.g. copied in before each replay or
+ * written by zero_scaler_prepare), as zero_step_fused_dc is for zero_step_fused: a stage-3
+ * step -- the layer scheduler's gathers, these updates and the commit -- can then be captured
+ * once as a CUDA graph and replayed for every step. Same results as the by-value call with the
+ * same constants. Errors: as zero_stage3_step_fused, and ZERO_EINVAL / ZERO_EALIGN for
+ * d_consts. */
+zero_status zero_stage3_step_fused_dc(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                                      const uint16_t* const* rank_grads, const float* master_in,
+                                      const float* m_in, const float* v_in, float* master_out,
+                                      float* m_out, float* v_out, uint16_t* const* param_shards,
+                                      const zero_adam_consts* d_consts, uint32_t* d_status,
+                                      zero_stream_t stream);
+
 /* Close a stage-3 step: zero_step_commit on every owner's part, over the whole padded list
  * (master_in ... v_out: the flat fp32 arrays, psi_padded values each), the fp16 values of a
  * voided step restored into each owner's partition. Errors: as zero_step_commit. */

@@ -279,3 +279,97 @@ def test_layer_scheduler_gpt2_small_layers():
     check_f32("m", nxt[1][idx_dev].cpu().numpy(), m_s)
     check_f32("v", nxt[2][idx_dev].cpu().numpy(), v_s)
     check_f16("params", f16np(torch.cat(shards)[idx_dev]), p_s)
+
+
+def test_stage3_step_captured_in_a_graph():
+    """A whole stage-3 step -- the layer scheduler's forward and backward gathers on its gather
+    stream, each layer's update with the step's constants in device memory
+    (zero_stage3_step_fused_dc), the commit -- captured once per ping-pong direction as a CUDA
+    graph on one capture stream and replayed: an eager first step, then replays at t = 2, an
+    attempt whose gradients hold an inf (skipped, t not advanced), t = 3 and t = 4, each against
+    zero3_step (state and partitions)."""
+    numels, split, nd = [40000, 1234, 30000, 777, 5003, 999, 4096], [1, 2, 2, 2], 4
+    pl = lz.zero_plan_create(numels, nd, 3, 0)
+    psi, psi_p, S, _ = lz.zero_plan_info(pl)
+    opl = oracle.plan(numels, nd, 0)
+    layers = oracle.layer_ranges(opl, split)
+    gb = oracle.grad_buckets(opl, layers)
+    L = len(layers)
+    bounds = [lo for lo, _ in layers] + [layers[-1][1]]
+    master, m, v = synth.state_warm(psi_p, seed=101)
+    w_r, m_r, v_r = master.numpy(), m.numpy(), v.numpy()
+    p16 = oracle.f2h(w_r)
+    ref_shards = [p16[q * S:(q + 1) * S].copy() for q in range(nd)]
+    shards = _partitions(p16, nd, S)
+    bufs = [[x.to(DEV) for x in (master, m, v)], [torch.empty(psi_p, dtype=torch.float32,
+                                                              device=DEV) for _ in range(3)]]
+    grads = [torch.zeros(psi_p, dtype=torch.float16, device=DEV) for _ in range(nd)]
+    d_consts = torch.empty(lz.ZERO_ADAM_CONSTS_BYTES, dtype=torch.uint8, device=DEV)
+    st = status_word()
+    pool = _Pool(pl, bounds, 2)
+    gs, cap = torch.cuda.Stream(), torch.cuda.Stream()
+    sched = lz.zero_layer_sched_create(pl, bounds, shards, pool.mem, pool.elems, 2, gs)
+
+    def body(d):
+        cur, nxt = bufs[d], bufs[1 - d]
+        st.zero_()
+        lz.zero_layer_sched_begin_step(sched, st, cap)
+        for l in range(L):
+            lz.zero_layer_sched_acquire(sched, l, l + 1 if l + 1 < L else -1, cap)
+            lz.zero_layer_sched_release(sched, l, cap)
+        for l in reversed(range(L)):
+            lo, _ = layers[l]
+            _, ghi = gb[l]
+            lz.zero_layer_sched_acquire(sched, l, l - 1, cap)
+            lz.zero_layer_sched_release(sched, l, cap)
+            lz.zero_stage3_step_fused_dc(pl, lo, ghi - lo, [g[lo:ghi] for g in grads],
+                                         *[x[lo:ghi] for x in cur], *[x[lo:ghi] for x in nxt],
+                                         shards, d_consts, st, cap)
+        lz.zero_stage3_step_commit(pl, *cur, *nxt, shards, st, cap)
+
+    def load(t, i, bad):
+        g_cpu = []
+        for r in range(nd):
+            x = torch.zeros(psi_p, dtype=torch.float16)
+            x[:psi] = synth.grad_f16(psi, 1e-3, seed=102, rank=r, step=10 * i + t)
+            g_cpu.append(x)
+        if bad:
+            g_cpu[2][layers[1][0] + 9] = float("inf")
+        c = lz.zero_adam_consts_for_step(HP, t)
+        with torch.cuda.stream(cap):
+            for g, x in zip(grads, g_cpu):
+                g.copy_(x)
+            d_consts.copy_(torch.frombuffer(bytearray(bytes(c)), dtype=torch.uint8))
+        return g_cpu
+
+    graphs = [None, None]
+    attempts = [(1, False), (2, False), (3, True), (3, False), (4, False)]
+    for i, (t, bad) in enumerate(attempts):
+        d = i % 2
+        g_cpu = load(t, i, bad)
+        if i == 0:                                   # first use outside any capture
+            with torch.cuda.stream(cap):
+                body(d)
+            cap.synchronize()
+            for dd in (1, 0):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=cap):
+                    body(dd)
+                graphs[dd] = g
+            # the capture enqueued nothing: state and partitions hold step 1's results
+        else:
+            with torch.cuda.stream(cap):
+                graphs[d].replay()
+        cap.synchronize()
+        code, flags = lz.zero_step_status(st, cap)
+        ref = oracle.zero3_step(opl, layers, lambda l, r: g_cpu[r].numpy()[gb[l][0]:gb[l][1]],
+                                w_r, m_r, v_r, ref_shards, ORC_HP, t)
+        assert ref.skipped == bad
+        assert code == (lz.ZERO_STEP_SKIPPED if bad else lz.ZERO_OK), (i, code, flags)
+        out = bufs[1 - d]
+        check_f32(f"attempt {i} master", f32np(out[0]), ref.master)
+        check_f32(f"attempt {i} m", f32np(out[1]), ref.m)
+        check_f32(f"attempt {i} v", f32np(out[2]), ref.v)
+        for q in range(nd):
+            check_f16(f"attempt {i} partition {q}", f16np(shards[q]), ref.param_shards[q])
+        w_r, m_r, v_r, ref_shards = ref.master, ref.m, ref.v, ref.param_shards

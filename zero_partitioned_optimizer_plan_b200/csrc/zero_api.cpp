@@ -531,15 +531,19 @@ zero_status zero_gather_params(const zero_plan* plan, uint64_t flat_lo, uint64_t
                                            (cudaStream_t)stream));
 }
 
-zero_status zero_stage3_step_fused(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
-                             const uint16_t* const* rank_grads, const float* master_in,
-                             const float* m_in, const float* v_in, float* master_out,
-                             float* m_out, float* v_out, uint16_t* const* param_shards,
-                             const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
-                             zero_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The owners' update of a stage-3 range with the step's constants `a` (by value) or, when `ad`
+// is not null, read from device memory; every part is checked before any is launched.
+zero_status stage3_fused(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                         const uint16_t* const* rank_grads, const float* master_in,
+                         const float* m_in, const float* v_in, float* master_out, float* m_out,
+                         float* v_out, uint16_t* const* param_shards, const zk::AdamConsts& a,
+                         const zk::AdamConsts* ad, uint32_t* d_status, cudaStream_t stream) {
     int nd = 0;
     uint64_t psi_p = 0, S = 0, q_lo = 0, q_hi = 0;
-    if (!zk::hparams_ok(hp) || step < 1) return ZERO_EINVAL;
     zero_status st = stage3_range(plan, flat_lo, len, &nd, &psi_p, &S, &q_lo, &q_hi);
     if (st != ZERO_OK) return st;
     if (!d_status) return ZERO_EINVAL;
@@ -547,15 +551,14 @@ zero_status zero_stage3_step_fused(const zero_plan* plan, uint64_t flat_lo, uint
     if (!rank_grads || !param_shards || !master_in || !m_in || !v_in || !master_out || !m_out ||
         !v_out)
         return ZERO_EINVAL;
-    // every owner's part is checked before anything is launched
     const uint16_t* part_grads[ZERO_MAX_RANKS];
     for (int pass = 0; pass < 2; ++pass) {
         for (uint64_t q = q_lo; q <= q_hi; ++q) {
-            const uint64_t a = flat_lo > q * S ? flat_lo : q * S;
-            const uint64_t b = (q + 1) * S < flat_lo + len ? (q + 1) * S : flat_lo + len;
-            const uint64_t off = a - flat_lo, n = b - a;
+            const uint64_t lo = flat_lo > q * S ? flat_lo : q * S;
+            const uint64_t hi = (q + 1) * S < flat_lo + len ? (q + 1) * S : flat_lo + len;
+            const uint64_t off = lo - flat_lo, n = hi - lo;
             for (int r = 0; r < nd; ++r) part_grads[r] = rank_grads[r] ? rank_grads[r] + off : nullptr;
-            uint16_t* pout = param_shards[q] ? param_shards[q] + (a - q * S) : nullptr;
+            uint16_t* pout = param_shards[q] ? param_shards[q] + (lo - q * S) : nullptr;
             if (pass == 0) {
                 st = check_fused(n, nd, part_grads, master_in + off, m_in + off, v_in + off,
                                  master_out + off, m_out + off, v_out + off, pout, d_status);
@@ -567,13 +570,42 @@ zero_status zero_stage3_step_fused(const zero_plan* plan, uint64_t flat_lo, uint
             } else {
                 const cudaError_t e = zk::launch_fused(
                     n, nd, part_grads, master_in + off, m_in + off, v_in + off, master_out + off,
-                    m_out + off, v_out + off, pout, zk::make_adam(hp, step), nullptr,
-                    zk::make_mean(nd), d_status, (cudaStream_t)stream);
+                    m_out + off, v_out + off, pout, a, ad, zk::make_mean(nd), d_status, stream);
                 if (e != cudaSuccess) return zk::from_cuda(e);
             }
         }
     }
     return ZERO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+zero_status zero_stage3_step_fused(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                             const uint16_t* const* rank_grads, const float* master_in,
+                             const float* m_in, const float* v_in, float* master_out,
+                             float* m_out, float* v_out, uint16_t* const* param_shards,
+                             const zero_adam_hparams* hp, int64_t step, uint32_t* d_status,
+                             zero_stream_t stream) {
+    if (!zk::hparams_ok(hp) || step < 1) return ZERO_EINVAL;
+    return stage3_fused(plan, flat_lo, len, rank_grads, master_in, m_in, v_in, master_out, m_out,
+                        v_out, param_shards, zk::make_adam(hp, step), nullptr, d_status,
+                        (cudaStream_t)stream);
+}
+
+zero_status zero_stage3_step_fused_dc(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                                      const uint16_t* const* rank_grads, const float* master_in,
+                                      const float* m_in, const float* v_in, float* master_out,
+                                      float* m_out, float* v_out, uint16_t* const* param_shards,
+                                      const zero_adam_consts* d_consts, uint32_t* d_status,
+                                      zero_stream_t stream) {
+    if (!d_consts) return ZERO_EINVAL;
+    if (!zk::aligned(d_consts, 4)) return ZERO_EALIGN;
+    zero_adam_consts unused;
+    memset(&unused, 0, sizeof(unused));
+    return stage3_fused(plan, flat_lo, len, rank_grads, master_in, m_in, v_in, master_out, m_out,
+                        v_out, param_shards, unused, d_consts, d_status, (cudaStream_t)stream);
 }
 
 zero_status zero_stage3_step_commit(const zero_plan* plan, const float* master_in, const float* m_in,
