@@ -898,6 +898,65 @@ def _layer_args(self, l, grads):
     return self.layer_views[d][l]
 
 
+def _enable_graph_zero3(self):
+    """Capture the stage-3 step once per ping-pong direction as a CUDA graph on one capture
+    stream: the layer scheduler's gathers (on its gather stream), the layers' updates with the
+    step's constants in device memory (zero_stage3_step_fused_dc), the commit. A replay needs no
+    host work but the constants' copy."""
+    torch, lz = self.torch, self.lz
+    dev = self.cur[0].device
+    self.dynamic = False
+    nb_c = lz.ZERO_ADAM_CONSTS_BYTES
+    self.d_consts = torch.empty(nb_c, dtype=torch.uint8, device=dev)
+    self.h_consts = [torch.empty(nb_c, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
+    self.h_done = [None, None]
+    self.g_status = torch.zeros(1, dtype=torch.int32, device=dev)
+    self.g_flags = torch.zeros(1, dtype=torch.int32, device=dev)
+    cap = torch.cuda.Stream()
+    pl, sch, L, shards = self.plan, self.layer_sched, len(self.layers), self.shards
+
+    def body(src, dst):
+        self.g_status.zero_()
+        lz.zero_layer_sched_begin_step(sch, self.g_status, cap)
+        for l in range(L):
+            lz.zero_layer_sched_acquire(sch, l, l + 1 if l + 1 < L else -1, cap)
+            lz.zero_layer_sched_release(sch, l, cap)
+        lz.zero_overlap_begin(cap)
+        for l in range(L - 1, -1, -1):
+            lo, hi = self.layers[l]
+            ghi = self.n if l == L - 1 else hi
+            lz.zero_layer_sched_acquire(sch, l, l - 1, cap)
+            lz.zero_layer_sched_release(sch, l, cap)
+            lz.zero_stage3_step_fused_dc(pl, lo, ghi - lo, [g[lo:ghi] for g in self.grads],
+                                         *[x[lo:ghi] for x in src], *[x[lo:ghi] for x in dst],
+                                         shards, self.d_consts, self.g_status, cap)
+        lz.zero_overlap_end(cap)
+        lz.zero_stage3_step_commit(pl, *src, *dst, shards, self.g_status, cap)
+        self.g_flags.bitwise_or_(self.g_status)
+
+    a, b = self.cur, self.nxt
+    self._load_consts(1)
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        body(a, b)                  # first use outside the capture
+    torch.cuda.current_stream().wait_stream(cap)
+    torch.cuda.synchronize()
+    self.graphs = []
+    for src, dst in ((a, b), (b, a)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            body(src, dst)
+        self.graphs.append(g)
+    self.g_flags.zero_()
+    self.graph_dir = 0
+    self.step = self._graph_step
+    self.kernel_times = None          # the replay's events: the whole step
+    self.dominant = "stage-3 step graph (gathers, fused layer updates, commit)"
+    self.dominant_bytes = self.bytes_per_step
+    self.dominant_calls = 1
+    self.graph_launches = 2 * L + self.config["fused_calls_per_step"] + 1
+
+
 def _layer_updates(self):
     """Each layer's zero_stage3_step_fused call for the current ping-pong direction, its
     arguments marshalled once (PreparedStage3Update)."""
@@ -922,6 +981,7 @@ Workload._step_zero3 = _step_zero3
 Workload._kernel_times_zero3 = _kernel_times_zero3
 Workload._layer_args = _layer_args
 Workload._layer_updates = _layer_updates
+Workload._enable_graph_zero3 = _enable_graph_zero3
 Workload._step_prepared = _step_prepared
 Workload._init_zero2 = _init_zero2
 Workload._step_zero2 = _step_zero2
@@ -1302,9 +1362,13 @@ def run_ours(args):
     wl = Workload(args, dev)
     if args.dynamic_scale and not args.graph:
         raise SystemExit("--dynamic-scale needs --graph")
-    if args.graph:
+    if args.graph and wl.kind.startswith("zero3"):
+        if args.dynamic_scale:
+            raise SystemExit("--dynamic-scale applies to the stage-1 and flat workloads")
+        wl._enable_graph_zero3()
+    elif args.graph:
         if wl.grads is None and wl.payload != "q8":
-            raise SystemExit("--graph applies to the stage-1 and flat workloads")
+            raise SystemExit("--graph applies to the stage-1, stage-3 and flat workloads")
         wl.enable_graph(dynamic=args.dynamic_scale, max_steps=args.steps + args.warmup + 4)
     K, W = args.steps, args.warmup
     status = torch.zeros(K + W, dtype=torch.int32, device=dev)   # one status word per step
@@ -1346,7 +1410,8 @@ def run_ours(args):
         torch.cuda.synchronize()
     launches = lz.zero_kernel_launches() - launches0
     if args.graph:   # replays launch the captured kernels without the host library
-        launches = K * (len(wl.ranges) + 1 + (2 if args.dynamic_scale else 0))
+        launches = K * getattr(wl, "graph_launches",
+                               len(wl.ranges) + 1 + (2 if args.dynamic_scale else 0))
         if int(wl.g_flags.item()) != 0:
             raise RuntimeError(f"unexpected status flags in the timed steps: {wl.g_flags.item()}")
     barrier()
