@@ -33,6 +33,10 @@ def test_workload_configs():
     assert fq["workload"] == "flat_268435456_q8" and fq["calls_per_step"] == 4
     s3 = bench.workload_config(_args(workload="zero3_gpt2_small"))
     assert (s3["stage"], s3["layers"]) == (3, 14)
+    dq = bench.workload_config(_args(payload="q8"))
+    assert (dq["workload"], dq["buckets"], dq["calls_per_step"]) == ("zero2_1p3b_fused_q8", 27, 28)
+    assert bench.traffic_key(types.SimpleNamespace(config=dq, nd=16)) == \
+        "zero2_1p3b_fused_q8_nd16_b50000000"     # the key profiles/traffic.json holds
 
 
 def test_traffic_keys_name_the_bucket_only_for_multi_call_steps():
