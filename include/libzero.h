@@ -451,16 +451,17 @@ zero_status zero_stage3_step_commit(const zero_plan* plan, const float* master_i
  *                  covers every buffer released on that stream so far).
  * A released layer is discarded (acquiring it again gathers it again); a prefetched layer that
  * is not acquired before its buffer is needed is dropped; begin_step drops every layer still
- * in a buffer (the partitions have changed since). A step can be captured into a CUDA graph
- * (with zero_stage3_step_fused_dc for the updates): capture it on one stream, pass that stream
- * to begin_step, acquire and release, so that the gather stream joins the capture through
- * begin_step's event and every wait stays inside the capture. The pages have no scheduler
- * interface; this is the library's runtime for the stage-3 data path.
+ * in a buffer (the partitions have changed since). The plan, the partitions and buf_mem must
+ * outlive the scheduler; one host thread at a time may use it. A step can be captured into a
+ * CUDA graph (with zero_stage3_step_fused_dc for the updates): capture it on one stream, pass
+ * that stream to begin_step, acquire and release, so that the gather stream joins the capture
+ * through begin_step's event and every wait stays inside the capture. The pages have no
+ * scheduler interface; this is the library's runtime for the stage-3 data path.
  * Errors: ZERO_EINVAL (bad plan or bounds, null pointers, an acquire before the first
  * begin_step, a layer out of range or already acquired, release of a layer not acquired,
  * begin_step while a layer is acquired, a status word inside a partition or the buffers),
- * ZERO_EALIGN, ZERO_ENOMEM (buf_mem too small, every
- * buffer holding an acquired layer, host allocation), ZERO_ECUDA (event or launch failure).
+ * ZERO_EALIGN, ZERO_ENOMEM (buf_mem too small, every buffer holding an acquired layer, host
+ * allocation), ZERO_ECUDA (event or launch failure).
  * ---------------------------------------------------------------------------------------- */
 typedef struct zero_layer_sched zero_layer_sched;
 
@@ -606,6 +607,8 @@ zero_status zero_overlap_end(zero_stream_t stream);
  *                       aligned (zero_sched_slot_elems gives the count)
  *   owner_grad_shards : nd device pointers (copied), as for zero_reduce_scatter_bucket
  *   d_status          : the step's status word
+ * The scheduler keeps the plan's address and the slot memory: both must outlive it; one host
+ * thread at a time may use a scheduler.
  * Errors: ZERO_EINVAL, ZERO_EALIGN, ZERO_ENOMEM (slot_mem too small or host allocation),
  * ZERO_ECUDA (event creation).
  * ---------------------------------------------------------------------------------------- */
