@@ -523,6 +523,27 @@ zero_status zero_step_fused_q8(uint64_t n, int nd, const uint8_t* const* rank_pa
                                uint16_t* param_out, const zero_adam_hparams* hp, int64_t step,
                                uint32_t* d_status, zero_stream_t stream);
 
+/* The int8 payload for stage 3's per-layer gradient reduce-scatter. A layer's range is split
+ * at owner boundaries (as zero_stage3_step_fused splits it); a rank's payload for the range is
+ * one segment per owner part, in owner order, each holding the part's records counted from the
+ * part's first element (ZERO_Q8_PAYLOAD_BYTES(part length)) and rounded up to 16 bytes.
+ * zero_stage3_payload_bytes_q8 gives the total; zero_stage3_quantize_q8 writes one rank's len
+ * fp16 gradients of the range into that layout (grad 2-byte aligned, payload 16-byte aligned,
+ * not overlapping); zero_stage3_step_fused_q8 is zero_stage3_step_fused with the nd ranks'
+ * payloads (host array of nd device pointers) in place of their fp16 gradients, each part
+ * reduced as zero_step_fused_q8 reduces it. Errors: as zero_stage3_step_fused and
+ * zero_quantize_q8. */
+zero_status zero_stage3_payload_bytes_q8(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                                         uint64_t* bytes);
+zero_status zero_stage3_quantize_q8(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                                    const uint16_t* grad, uint8_t* payload, zero_stream_t stream);
+zero_status zero_stage3_step_fused_q8(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                                      const uint8_t* const* rank_payload, const float* master_in,
+                                      const float* m_in, const float* v_in, float* master_out,
+                                      float* m_out, float* v_out, uint16_t* const* param_shards,
+                                      const zero_adam_hparams* hp, int64_t step,
+                                      uint32_t* d_status, zero_stream_t stream);
+
 /* The int8 calls of one step over several ranges as one call, as zero_step_fused_ranges is for
  * zero_step_fused: ranges[i] describes what zero_step_fused_q8 takes for range i (rank_payload:
  * a host array of nd device pointers, each to that range's records). Every range is checked

@@ -493,6 +493,44 @@ def test_layer_scheduler_sizes_and_rejects():
         assert e.value.code == code, kw
 
 
+def test_stage3_q8_payload_sizes_and_rejects():
+    """The stage-3 int8 payload of a range: one segment per owner part, the part's records
+    rounded up to 16 bytes; the quantizer's and the step's argument errors."""
+    pl = _stage3_plan()                                  # psi_p = 128, S = 32, Nd = 4
+    assert lz.zero_stage3_payload_bytes_q8(pl, 10, 60) == 3 * 144   # parts of 22, 32 and 6
+    assert lz.zero_stage3_payload_bytes_q8(pl, 0, 128) == 4 * 144
+    assert lz.zero_stage3_payload_bytes_q8(pl, 5, 0) == 0
+    with pytest.raises(lz.ZeroError) as e:
+        lz.zero_stage3_payload_bytes_q8(pl, 100, 29)
+    assert e.value.code == lz.ZERO_EINVAL
+    before = lz.zero_kernel_launches()
+    for args, code in [((10, 60, A, A + 50 * MB + 4), lz.ZERO_EALIGN),      # payload not 16-aligned
+                       ((10, 60, A + 1, A + 50 * MB), lz.ZERO_EALIGN),
+                       ((10, 60, 0, A + 50 * MB), lz.ZERO_EINVAL),
+                       ((10, 60, A, A + 16), lz.ZERO_EINVAL),              # payload over the grads
+                       ((120, 9, A, A + 50 * MB), lz.ZERO_EINVAL)]:        # beyond psi_padded
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_stage3_quantize_q8(pl, *args, 0)
+        assert e.value.code == code, args
+    pays = [A + (10 + r) * MB for r in range(4)]
+    ins = [A + 20 * MB, A + 21 * MB, A + 22 * MB]
+    outs = [A + 23 * MB, A + 24 * MB, A + 25 * MB]
+    parts = [A + q * MB for q in range(4)]
+    st = A + 30 * MB
+    for kw, code in [(dict(pays=pays[:3] + [0]), lz.ZERO_EINVAL),
+                     (dict(pays=pays[:3] + [pays[3] + 2]), lz.ZERO_EALIGN),
+                     (dict(step=0), lz.ZERO_EINVAL),
+                     (dict(outs=[ins[0]] + outs[1:]), lz.ZERO_EINVAL),
+                     (dict(parts=[A, A + 16, A + 2 * MB, A + 3 * MB]), lz.ZERO_EINVAL)]:
+        a = dict(pays=pays, step=1, outs=outs, parts=parts)
+        a.update(kw)
+        with pytest.raises(lz.ZeroError) as e:
+            lz.zero_stage3_step_fused_q8(pl, 10, 60, a["pays"], *ins, *a["outs"], a["parts"], HP,
+                                         a["step"], st, 0)
+        assert e.value.code == code, kw
+    assert lz.zero_kernel_launches() == before
+
+
 def test_step_fused_ranges_rejects_before_launching():
     grads = [A + i * MB for i in range(2)]
     good = (1000, grads, A + 100 * MB, A + 101 * MB, A + 102 * MB, A + 110 * MB, A + 111 * MB,

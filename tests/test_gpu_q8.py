@@ -483,3 +483,84 @@ def test_q8_bucket_scheduler_vs_oracle(n_slots):
         check_f32(f"attempt {i} v", f32np(pp.cur[2]), vv, tol=0)
         check_f16(f"attempt {i} params", f16np(params), p16, tol=0)
     lz.zero_sched_destroy(sch)
+
+
+@pytest.mark.parametrize("nd", [3, 8])
+def test_stage3_q8_steps_vs_oracle(nd):
+    """Stage 3 with the int8 gradient payload: per layer in backward order each rank's gradient
+    bucket quantized into one segment per owner part (zero_stage3_quantize_q8; the segments
+    bit for bit against the oracle's quantizer of each part), then the owners' int8 fused
+    update into their partitions (zero_stage3_step_fused_q8), then the commit. Three attempts
+    (t = 1, a poisoned block at t = 2 that skips the step, t = 2): state and partitions
+    against the oracle's int8 step over the same parts, bit for bit."""
+    numels, split = [40000, 1234, 30000, 777, 5003], [1, 2, 2]
+    pl = lz.zero_plan_create(numels, nd, 3, 0)
+    psi, psi_p, S, _ = lz.zero_plan_info(pl)
+    opl = oracle.plan(numels, nd, 0)
+    layers = oracle.layer_ranges(opl, split)
+    gb = oracle.grad_buckets(opl, layers)
+    master, m, v = synth.state_warm(psi_p, seed=151)
+    w, mm, vv = master.numpy(), m.numpy(), v.numpy()
+    p16 = oracle.f2h(w)
+    shards = [torch.from_numpy(p16[q * S:(q + 1) * S].view(np.float16)).to(DEV)
+              for q in range(nd)]
+    pp = PingPong(master, m, v)
+
+    def parts(lo, hi):                  # the owner parts of [lo, hi), in owner order
+        out, a = [], lo
+        while a < hi:
+            b = min(hi, (a // S + 1) * S)
+            out.append((a, b))
+            a = b
+        return out
+
+    for i, (t, bad) in enumerate([(1, False), (2, True), (2, False)]):
+        g = []
+        for r in range(nd):
+            x = torch.zeros(psi_p, dtype=torch.float16)
+            x[:psi] = synth.grad_f16(psi, 1e-3, seed=152, rank=r, step=10 * i + t)
+            g.append(x)
+        if bad:
+            g[nd - 1][layers[1][0] + 11] = float("nan")
+        g_dev = [x.to(DEV) for x in g]
+        st = status_word()
+        for l in reversed(range(len(layers))):
+            lo, ghi = gb[l]
+            nb = lz.zero_stage3_payload_bytes_q8(pl, lo, ghi - lo)
+            assert nb == sum((lz.q8_payload_bytes(b - a) + 15) // 16 * 16 for a, b in parts(lo, ghi))
+            pays = [torch.empty(nb, dtype=torch.uint8, device=DEV) for _ in range(nd)]
+            for r in range(nd):
+                lz.zero_stage3_quantize_q8(pl, lo, ghi - lo, g_dev[r][lo:ghi], pays[r])
+            if l == 0:                  # the segments of rank 0 against the oracle's quantizer
+                got, off = pays[0].cpu().numpy(), 0
+                for a, b in parts(lo, ghi):
+                    q, sc = oracle.quant_q8(g[0].numpy()[a:b])
+                    rec = got[off:off + lz.q8_payload_bytes(b - a)].reshape(-1, 132)
+                    assert np.array_equal(_q_of(rec[:, :128]).reshape(-1)[:b - a], q)
+                    assert np.array_equal(rec[:, 128:].copy().view(np.float32).reshape(-1), sc)
+                    off += (lz.q8_payload_bytes(b - a) + 15) // 16 * 16
+            lz.zero_stage3_step_fused_q8(pl, lo, ghi - lo, pays, *[x[lo:ghi] for x in pp.cur],
+                                         *[x[lo:ghi] for x in pp.nxt], shards, HP, t, st)
+        lz.zero_stage3_step_commit(pl, *pp.cur, *pp.nxt, shards, st)
+        code, flags = lz.zero_step_status(st)
+        w2, m2, v2, p2 = w.copy(), mm.copy(), vv.copy(), p16.copy()
+        skipped = False
+        for lo, ghi in gb:
+            for a, b in parts(lo, ghi):
+                qs = [oracle.quant_q8(x.numpy()[a:b]) for x in g]
+                sk, wb, mb, vb, pb = oracle.step_q8([q for q, _ in qs], [c for _, c in qs],
+                                                    w[a:b], mm[a:b], vv[a:b], ORC_HP, t)
+                skipped |= sk
+                if not sk:
+                    w2[a:b], m2[a:b], v2[a:b], p2[a:b] = wb, mb, vb, pb
+        assert skipped == bad
+        assert code == (lz.ZERO_STEP_SKIPPED if bad else lz.ZERO_OK), (code, flags)
+        if not bad:
+            w, mm, vv, p16 = w2, m2, v2, p2
+        pp.swap()
+        check_f32(f"attempt {i} master", f32np(pp.cur[0]), w, tol=0)
+        check_f32(f"attempt {i} m", f32np(pp.cur[1]), mm, tol=0)
+        check_f32(f"attempt {i} v", f32np(pp.cur[2]), vv, tol=0)
+        for q in range(nd):
+            check_f16(f"attempt {i} partition {q}", f16np(shards[q]), p16[q * S:(q + 1) * S],
+                      tol=0)

@@ -608,6 +608,104 @@ zero_status zero_stage3_step_fused_dc(const zero_plan* plan, uint64_t flat_lo, u
                         v_out, param_shards, unused, d_consts, d_status, (cudaStream_t)stream);
 }
 
+// The int8 payload of a stage-3 range: one segment per owner part of the range, the part's
+// records counted from its first element, each segment rounded up to 16 bytes.
+static uint64_t q8_segment_bytes(uint64_t n) {
+    return (ZERO_Q8_PAYLOAD_BYTES(n) + 15) & ~(uint64_t)15;
+}
+
+zero_status zero_stage3_payload_bytes_q8(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                                         uint64_t* bytes) {
+    int nd = 0;
+    uint64_t psi_p = 0, S = 0, q_lo = 0, q_hi = 0;
+    if (!bytes) return ZERO_EINVAL;
+    const zero_status st = stage3_range(plan, flat_lo, len, &nd, &psi_p, &S, &q_lo, &q_hi);
+    if (st != ZERO_OK) return st;
+    uint64_t total = 0;
+    for (uint64_t q = q_lo; len > 0 && q <= q_hi; ++q) {
+        const uint64_t lo = flat_lo > q * S ? flat_lo : q * S;
+        const uint64_t hi = (q + 1) * S < flat_lo + len ? (q + 1) * S : flat_lo + len;
+        total += q8_segment_bytes(hi - lo);
+    }
+    *bytes = total;
+    return ZERO_OK;
+}
+
+zero_status zero_stage3_quantize_q8(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                                    const uint16_t* grad, uint8_t* payload,
+                                    zero_stream_t stream) {
+    int nd = 0;
+    uint64_t psi_p = 0, S = 0, q_lo = 0, q_hi = 0;
+    zero_status st = stage3_range(plan, flat_lo, len, &nd, &psi_p, &S, &q_lo, &q_hi);
+    if (st != ZERO_OK) return st;
+    if (len == 0) return ZERO_OK;
+    if (!grad || !payload) return ZERO_EINVAL;
+    if (!zk::aligned(grad, 2) || !zk::aligned(payload, 16)) return ZERO_EALIGN;
+    uint64_t bytes = 0;
+    zero_stage3_payload_bytes_q8(plan, flat_lo, len, &bytes);
+    if (zk::overlap(payload, bytes, grad, len * 2)) return ZERO_EINVAL;
+    uint64_t seg = 0;
+    for (uint64_t q = q_lo; q <= q_hi; ++q) {
+        const uint64_t lo = flat_lo > q * S ? flat_lo : q * S;
+        const uint64_t hi = (q + 1) * S < flat_lo + len ? (q + 1) * S : flat_lo + len;
+        const cudaError_t e = zk::launch_quant_q8(hi - lo, grad + (lo - flat_lo), payload + seg,
+                                                  (cudaStream_t)stream);
+        if (e != cudaSuccess) return zk::from_cuda(e);
+        seg += q8_segment_bytes(hi - lo);
+    }
+    return ZERO_OK;
+}
+
+zero_status zero_stage3_step_fused_q8(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                                      const uint8_t* const* rank_payload, const float* master_in,
+                                      const float* m_in, const float* v_in, float* master_out,
+                                      float* m_out, float* v_out, uint16_t* const* param_shards,
+                                      const zero_adam_hparams* hp, int64_t step,
+                                      uint32_t* d_status, zero_stream_t stream) {
+    int nd = 0;
+    uint64_t psi_p = 0, S = 0, q_lo = 0, q_hi = 0;
+    if (!zk::hparams_ok(hp) || step < 1) return ZERO_EINVAL;
+    zero_status st = stage3_range(plan, flat_lo, len, &nd, &psi_p, &S, &q_lo, &q_hi);
+    if (st != ZERO_OK) return st;
+    if (!d_status) return ZERO_EINVAL;
+    if (len == 0) return ZERO_OK;
+    if (!rank_payload || !param_shards || !master_in || !m_in || !v_in || !master_out ||
+        !m_out || !v_out)
+        return ZERO_EINVAL;
+    for (int r = 0; r < nd; ++r)
+        if (!rank_payload[r]) return ZERO_EINVAL;
+    // every owner's part is checked before anything is launched
+    const uint8_t* part_pay[ZERO_MAX_RANKS];
+    const zk::AdamConsts a = zk::make_adam(hp, step);
+    for (int pass = 0; pass < 2; ++pass) {
+        uint64_t seg = 0;
+        for (uint64_t q = q_lo; q <= q_hi; ++q) {
+            const uint64_t lo = flat_lo > q * S ? flat_lo : q * S;
+            const uint64_t hi = (q + 1) * S < flat_lo + len ? (q + 1) * S : flat_lo + len;
+            const uint64_t off = lo - flat_lo, n = hi - lo;
+            for (int r = 0; r < nd; ++r) part_pay[r] = rank_payload[r] + seg;
+            uint16_t* pout = param_shards[q] ? param_shards[q] + (lo - q * S) : nullptr;
+            if (pass == 0) {
+                st = check_fused_q8(n, nd, part_pay, master_in + off, m_in + off, v_in + off,
+                                    master_out + off, m_out + off, v_out + off, pout, d_status);
+                if (st != ZERO_OK) return st;
+                for (uint64_t o = q_lo; o < q; ++o)   // partitions are distinct buffers
+                    if (param_shards[o] &&
+                        zk::overlap(param_shards[o], S * 2, param_shards[q], S * 2))
+                        return ZERO_EINVAL;
+            } else {
+                const cudaError_t e = zk::launch_fused_q8(
+                    n, nd, part_pay, master_in + off, m_in + off, v_in + off, master_out + off,
+                    m_out + off, v_out + off, pout, a, nullptr, zk::make_mean(nd), d_status,
+                    (cudaStream_t)stream);
+                if (e != cudaSuccess) return zk::from_cuda(e);
+            }
+            seg += q8_segment_bytes(n);
+        }
+    }
+    return ZERO_OK;
+}
+
 zero_status zero_stage3_step_commit(const zero_plan* plan, const float* master_in, const float* m_in,
                               const float* v_in, float* master_out, float* m_out, float* v_out,
                               uint16_t* const* param_shards, uint32_t* d_status,
