@@ -142,6 +142,9 @@ def workload_config(args) -> dict:
         layers = synth.gpt2_small_layers() if small else synth.gpt_1p3b_layers()
         cfg = {"workload": kind, "psi": sum(numels), "nd": nd, "stage": 3,
                "layers": len(layers), "calls_per_step": None, "tensors": len(numels)}
+        if args.payload == "q8":
+            cfg["payload"] = "int8 records: 128 values and their fp32 scale, one segment per owner part"
+            cfg["workload"] += "_q8"
         return cfg
     elif kind in ("zero2_1p3b", "zero2_gpt2_small"):
         small = kind == "zero2_gpt2_small"
@@ -308,6 +311,8 @@ class Workload:
 
     def inputs(self):
         """The tensors a step consumes that a host would have to upload."""
+        if self.payload == "q8" and self.kind.startswith("zero3"):
+            return [x for pays in self.q3 for x in pays]       # per layer, per rank
         if self.payload == "q8":
             return self.q
         return self.grads
@@ -755,6 +760,16 @@ def _e2e_zero2_fused(self, t0, E, barrier, max_ms):
     return out
 
 
+def _owner_parts(lo: int, hi: int, shard: int):
+    """The owner parts of the flat range [lo, hi), in owner order."""
+    out, a = [], lo
+    while a < hi:
+        b = min(hi, (a // shard + 1) * shard)
+        out.append((a, b))
+        a = b
+    return out
+
+
 def _init_zero3(self, args, dev):
     """Stage 3 on a GPT-shaped list: every rank's full local gradient is resident (as the
     backward pass would leave it layer by layer); the fp16 parameters are Nd partitions of S
@@ -765,9 +780,10 @@ def _init_zero3(self, args, dev):
     zero_stage3_step_commit. Each fused call is timed with its own events in the last step."""
     torch, lz = self.torch, self.lz
     from zero_partitioned_optimizer_plan_b200 import synth
-    if args.payload != "fp16":
-        raise SystemExit("the stage-3 workloads take fp16 payloads")
-    self.payload = "fp16"
+    q8 = args.payload == "q8"
+    if q8 and args.graph:
+        raise SystemExit("the stage-3 graph takes fp16 payloads")
+    self.payload = args.payload
     small = args.workload == "zero3_gpt2_small"
     nd = args.nd or (8 if small else 16)
     numels = synth.gpt2_small_list() if small else synth.gpt_1p3b_list()
@@ -818,8 +834,23 @@ def _init_zero3(self, args, dev):
     self.config["layer_buffers"] = nb
     gather_bytes = 2 * 4 * psi              # two gathers: 2 bytes read + 2 written each
     fused_bytes = (2 * nd + 26) * psi_p
-    self.bytes_per_step = gather_bytes + fused_bytes
     self.dominant = "fused_tma_kernel"
+    self.q3 = None
+    if q8:
+        # every layer's int8 payload of every rank (one segment per owner part), quantized once
+        self.q3, pay_bytes = [], 0
+        for l, (lo, hi) in enumerate(self.layers):
+            ghi = psi_p if l == L - 1 else hi
+            nbytes = lz.zero_stage3_payload_bytes_q8(pl, lo, ghi - lo)
+            pays = [torch.empty(nbytes, dtype=torch.uint8, device=dev) for _ in range(nd)]
+            for r in range(nd):
+                lz.zero_stage3_quantize_q8(pl, lo, ghi - lo, self.grads[r][lo:ghi], pays[r])
+            self.q3.append(pays)
+            pay_bytes += sum(lz.q8_payload_bytes(b - a) for a, b in
+                             _owner_parts(lo, ghi, S)) * nd
+        fused_bytes = pay_bytes + 26 * psi_p
+        self.dominant = "fused_q8_tma_kernel"
+    self.bytes_per_step = gather_bytes + fused_bytes
     self.dominant_bytes = fused_bytes
     self.dominant_calls = n_fused
     self.fused_evs = []
@@ -835,8 +866,12 @@ def _step_zero3(self, t, status, ev=None, grads=None):
     update (disjoint ranges of the partitions); the next step's gathers wait for this step's
     commit (zero_layer_sched_begin_step)."""
     lz, torch = self.lz, self.torch
-    grads = grads or self.grads
     pl, shards, L, sch = self.plan, self.shards, len(self.layers), self.layer_sched
+    if self.q3 is not None:   # int8: the step's inputs are the layers' payloads (inputs())
+        pays = self.q3 if grads is None else \
+            [grads[l * self.nd:(l + 1) * self.nd] for l in range(L)]
+        grads = self.grads    # only the state views of _layer_args are used then
+    grads = grads or self.grads
     main = torch.cuda.current_stream()
     # per-call events only in the step that run_ours marks (the last timed one): recording
     # events around every call of every step doubled the host's work per step, which at
@@ -852,7 +887,7 @@ def _step_zero3(self, t, status, ev=None, grads=None):
     # the layers' updates touch disjoint ranges: one overlap region on the main stream (event
     # waits and records are allowed inside; an event recorded after an update completes only
     # when every update before it has)
-    prepared = self._layer_updates() if grads is self.grads else None
+    prepared = self._layer_updates() if grads is self.grads and self.q3 is None else None
     hp_ref, st_ptr, sh = lz.hparams_ref(self.hp), lz.status_ptr(status), lz.stream_handle(main)
     lz.zero_overlap_begin(main)
     for l in range(L - 1, -1, -1):
@@ -864,6 +899,10 @@ def _step_zero3(self, t, status, ev=None, grads=None):
             e[0].record(main)
         if prepared is not None:
             prepared[l](hp_ref, t, st_ptr, sh)
+        elif self.q3 is not None:          # the owners' update from the int8 payloads
+            n, _, *state = self._layer_args(l, grads)
+            lz.zero_stage3_step_fused_q8(pl, lo, n, pays[l], *state, shards, self.hp, t,
+                                         status, main)
         else:
             lz.zero_stage3_step_fused(pl, lo, *self._layer_args(l, grads), shards, self.hp, t,
                                       status, main)
