@@ -781,8 +781,6 @@ def _init_zero3(self, args, dev):
     torch, lz = self.torch, self.lz
     from zero_partitioned_optimizer_plan_b200 import synth
     q8 = args.payload == "q8"
-    if q8 and args.graph:
-        raise SystemExit("the stage-3 graph takes fp16 payloads")
     self.payload = args.payload
     small = args.workload == "zero3_gpt2_small"
     nd = args.nd or (8 if small else 16)
@@ -940,8 +938,8 @@ def _layer_args(self, l, grads):
 def _enable_graph_zero3(self):
     """Capture the stage-3 step once per ping-pong direction as a CUDA graph on one capture
     stream: the layer scheduler's gathers (on its gather stream), the layers' updates with the
-    step's constants in device memory (zero_stage3_step_fused_dc), the commit. A replay needs no
-    host work but the constants' copy."""
+    step's constants in device memory (zero_stage3_step_fused_dc, or _q8_dc from the int8
+    payloads), the commit. A replay needs no host work but the constants' copy."""
     torch, lz = self.torch, self.lz
     dev = self.cur[0].device
     self.dynamic = False
@@ -966,9 +964,16 @@ def _enable_graph_zero3(self):
             ghi = self.n if l == L - 1 else hi
             lz.zero_layer_sched_acquire(sch, l, l - 1, cap)
             lz.zero_layer_sched_release(sch, l, cap)
-            lz.zero_stage3_step_fused_dc(pl, lo, ghi - lo, [g[lo:ghi] for g in self.grads],
-                                         *[x[lo:ghi] for x in src], *[x[lo:ghi] for x in dst],
-                                         shards, self.d_consts, self.g_status, cap)
+            if self.q3 is not None:
+                lz.zero_stage3_step_fused_q8_dc(pl, lo, ghi - lo, self.q3[l],
+                                                *[x[lo:ghi] for x in src],
+                                                *[x[lo:ghi] for x in dst], shards, self.d_consts,
+                                                self.g_status, cap)
+            else:
+                lz.zero_stage3_step_fused_dc(pl, lo, ghi - lo, [g[lo:ghi] for g in self.grads],
+                                             *[x[lo:ghi] for x in src],
+                                             *[x[lo:ghi] for x in dst], shards, self.d_consts,
+                                             self.g_status, cap)
         lz.zero_overlap_end(cap)
         lz.zero_stage3_step_commit(pl, *src, *dst, shards, self.g_status, cap)
         self.g_flags.bitwise_or_(self.g_status)

@@ -543,6 +543,17 @@ zero_status zero_stage3_step_fused_q8(const zero_plan* plan, uint64_t flat_lo, u
                                       float* m_out, float* v_out, uint16_t* const* param_shards,
                                       const zero_adam_hparams* hp, int64_t step,
                                       uint32_t* d_status, zero_stream_t stream);
+/* zero_stage3_step_fused_q8 with the step's constants read from device memory (d_consts, as
+ * for zero_stage3_step_fused_dc), so that a stage-3 step from int8 payloads is captured once
+ * as a CUDA graph. Errors: as zero_stage3_step_fused_q8, and ZERO_EINVAL / ZERO_EALIGN for
+ * d_consts. */
+zero_status zero_stage3_step_fused_q8_dc(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                                         const uint8_t* const* rank_payload,
+                                         const float* master_in, const float* m_in,
+                                         const float* v_in, float* master_out, float* m_out,
+                                         float* v_out, uint16_t* const* param_shards,
+                                         const zero_adam_consts* d_consts, uint32_t* d_status,
+                                         zero_stream_t stream);
 
 /* The int8 calls of one step over several ranges as one call, as zero_step_fused_ranges is for
  * zero_step_fused: ranges[i] describes what zero_step_fused_q8 takes for range i (rank_payload:

@@ -564,3 +564,104 @@ def test_stage3_q8_steps_vs_oracle(nd):
         for q in range(nd):
             check_f16(f"attempt {i} partition {q}", f16np(shards[q]), p16[q * S:(q + 1) * S],
                       tol=0)
+
+
+def test_stage3_q8_step_captured_in_a_graph():
+    """A stage-3 step from int8 payloads with the constants in device memory
+    (zero_stage3_step_fused_q8_dc), the layer gathers by the layer scheduler and the commit,
+    captured as a CUDA graph per ping-pong direction and replayed at t = 1, 2, 3 (the payloads
+    rewritten in place between replays): state and partitions against the oracle's int8 step
+    per owner part, bit for bit."""
+    numels, split, nd = [40000, 1234, 30000, 777, 5003], [1, 2, 2], 4
+    pl = lz.zero_plan_create(numels, nd, 3, 0)
+    psi, psi_p, S, _ = lz.zero_plan_info(pl)
+    opl = oracle.plan(numels, nd, 0)
+    layers = oracle.layer_ranges(opl, split)
+    gb = oracle.grad_buckets(opl, layers)
+    L = len(layers)
+    bounds = [lo for lo, _ in layers] + [layers[-1][1]]
+    master, m, v = synth.state_warm(psi_p, seed=161)
+    w, mm, vv = master.numpy(), m.numpy(), v.numpy()
+    p16 = oracle.f2h(w)
+    shards = [torch.from_numpy(p16[q * S:(q + 1) * S].view(np.float16)).to(DEV)
+              for q in range(nd)]
+    bufs = [[x.to(DEV) for x in (master, m, v)],
+            [torch.empty(psi_p, dtype=torch.float32, device=DEV) for _ in range(3)]]
+    g_dev = [torch.zeros(psi_p, dtype=torch.float16, device=DEV) for _ in range(nd)]
+    pays = [[torch.empty(lz.zero_stage3_payload_bytes_q8(pl, lo, hi - lo), dtype=torch.uint8,
+                         device=DEV) for _ in range(nd)] for lo, hi in gb]
+    d_consts = torch.empty(lz.ZERO_ADAM_CONSTS_BYTES, dtype=torch.uint8, device=DEV)
+    st = status_word()
+    elems = lz.zero_layer_sched_buf_elems(pl, bounds, 2)
+    pool = torch.empty(elems, dtype=torch.float16, device=DEV)
+    gs, cap = torch.cuda.Stream(), torch.cuda.Stream()
+    sched = lz.zero_layer_sched_create(pl, bounds, shards, pool, elems, 2, gs)
+
+    def body(d):
+        cur, nxt = bufs[d], bufs[1 - d]
+        st.zero_()
+        lz.zero_layer_sched_begin_step(sched, st, cap)
+        for l in range(L):
+            lz.zero_layer_sched_acquire(sched, l, l + 1 if l + 1 < L else -1, cap)
+            lz.zero_layer_sched_release(sched, l, cap)
+        for l in reversed(range(L)):
+            lo, ghi = gb[l]
+            lz.zero_layer_sched_acquire(sched, l, l - 1, cap)
+            lz.zero_layer_sched_release(sched, l, cap)
+            lz.zero_stage3_step_fused_q8_dc(pl, lo, ghi - lo, pays[l], *[x[lo:ghi] for x in cur],
+                                            *[x[lo:ghi] for x in nxt], shards, d_consts, st, cap)
+        lz.zero_stage3_step_commit(pl, *cur, *nxt, shards, st, cap)
+
+    def parts(lo, hi):
+        out, a = [], lo
+        while a < hi:
+            b = min(hi, (a // S + 1) * S)
+            out.append((a, b))
+            a = b
+        return out
+
+    graphs = [None, None]
+    for i, t in enumerate((1, 2, 3)):
+        d = i % 2
+        g = []
+        for r in range(nd):
+            x = torch.zeros(psi_p, dtype=torch.float16)
+            x[:psi] = synth.grad_f16(psi, 1e-3, seed=162, rank=r, step=t)
+            g.append(x)
+        c = lz.zero_adam_consts_for_step(HP, t)
+        with torch.cuda.stream(cap):
+            for gd, x in zip(g_dev, g):
+                gd.copy_(x)
+            for (lo, ghi), pl_pays in zip(gb, pays):
+                for r in range(nd):
+                    lz.zero_stage3_quantize_q8(pl, lo, ghi - lo, g_dev[r][lo:ghi], pl_pays[r], cap)
+            d_consts.copy_(torch.frombuffer(bytearray(bytes(c)), dtype=torch.uint8))
+        if i == 0:                                   # first use outside any capture
+            with torch.cuda.stream(cap):
+                body(d)
+            cap.synchronize()
+            for dd in (1, 0):
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr, stream=cap):
+                    body(dd)
+                graphs[dd] = gr
+        else:
+            with torch.cuda.stream(cap):
+                graphs[d].replay()
+        cap.synchronize()
+        assert lz.zero_step_status(st, cap) == (lz.ZERO_OK, 0)
+        w2, m2, v2, p2 = w.copy(), mm.copy(), vv.copy(), p16.copy()
+        for lo, ghi in gb:
+            for a, b in parts(lo, ghi):
+                qs = [oracle.quant_q8(x.numpy()[a:b]) for x in g]
+                sk, wb, mb, vb, pb = oracle.step_q8([q for q, _ in qs], [s_ for _, s_ in qs],
+                                                    w[a:b], mm[a:b], vv[a:b], ORC_HP, t)
+                assert not sk
+                w2[a:b], m2[a:b], v2[a:b], p2[a:b] = wb, mb, vb, pb
+        w, mm, vv, p16 = w2, m2, v2, p2
+        out = bufs[1 - d]
+        check_f32(f"step {t} master", f32np(out[0]), w, tol=0)
+        check_f32(f"step {t} m", f32np(out[1]), mm, tol=0)
+        check_f32(f"step {t} v", f32np(out[2]), vv, tol=0)
+        for q in range(nd):
+            check_f16(f"step {t} partition {q}", f16np(shards[q]), p16[q * S:(q + 1) * S], tol=0)

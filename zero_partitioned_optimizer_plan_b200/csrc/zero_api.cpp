@@ -656,15 +656,16 @@ zero_status zero_stage3_quantize_q8(const zero_plan* plan, uint64_t flat_lo, uin
     return ZERO_OK;
 }
 
-zero_status zero_stage3_step_fused_q8(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
-                                      const uint8_t* const* rank_payload, const float* master_in,
-                                      const float* m_in, const float* v_in, float* master_out,
-                                      float* m_out, float* v_out, uint16_t* const* param_shards,
-                                      const zero_adam_hparams* hp, int64_t step,
-                                      uint32_t* d_status, zero_stream_t stream) {
+// The owners' int8 update of a stage-3 range with the constants `a` or, when `ad` is not
+// null, from device memory; every part is checked before any is launched.
+static zero_status stage3_fused_q8(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                                   const uint8_t* const* rank_payload, const float* master_in,
+                                   const float* m_in, const float* v_in, float* master_out,
+                                   float* m_out, float* v_out, uint16_t* const* param_shards,
+                                   const zk::AdamConsts& a, const zk::AdamConsts* ad,
+                                   uint32_t* d_status, cudaStream_t stream) {
     int nd = 0;
     uint64_t psi_p = 0, S = 0, q_lo = 0, q_hi = 0;
-    if (!zk::hparams_ok(hp) || step < 1) return ZERO_EINVAL;
     zero_status st = stage3_range(plan, flat_lo, len, &nd, &psi_p, &S, &q_lo, &q_hi);
     if (st != ZERO_OK) return st;
     if (!d_status) return ZERO_EINVAL;
@@ -674,9 +675,7 @@ zero_status zero_stage3_step_fused_q8(const zero_plan* plan, uint64_t flat_lo, u
         return ZERO_EINVAL;
     for (int r = 0; r < nd; ++r)
         if (!rank_payload[r]) return ZERO_EINVAL;
-    // every owner's part is checked before anything is launched
     const uint8_t* part_pay[ZERO_MAX_RANKS];
-    const zk::AdamConsts a = zk::make_adam(hp, step);
     for (int pass = 0; pass < 2; ++pass) {
         uint64_t seg = 0;
         for (uint64_t q = q_lo; q <= q_hi; ++q) {
@@ -696,14 +695,41 @@ zero_status zero_stage3_step_fused_q8(const zero_plan* plan, uint64_t flat_lo, u
             } else {
                 const cudaError_t e = zk::launch_fused_q8(
                     n, nd, part_pay, master_in + off, m_in + off, v_in + off, master_out + off,
-                    m_out + off, v_out + off, pout, a, nullptr, zk::make_mean(nd), d_status,
-                    (cudaStream_t)stream);
+                    m_out + off, v_out + off, pout, a, ad, zk::make_mean(nd), d_status, stream);
                 if (e != cudaSuccess) return zk::from_cuda(e);
             }
             seg += q8_segment_bytes(n);
         }
     }
     return ZERO_OK;
+}
+
+zero_status zero_stage3_step_fused_q8(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                                      const uint8_t* const* rank_payload, const float* master_in,
+                                      const float* m_in, const float* v_in, float* master_out,
+                                      float* m_out, float* v_out, uint16_t* const* param_shards,
+                                      const zero_adam_hparams* hp, int64_t step,
+                                      uint32_t* d_status, zero_stream_t stream) {
+    if (!zk::hparams_ok(hp) || step < 1) return ZERO_EINVAL;
+    return stage3_fused_q8(plan, flat_lo, len, rank_payload, master_in, m_in, v_in, master_out,
+                           m_out, v_out, param_shards, zk::make_adam(hp, step), nullptr,
+                           d_status, (cudaStream_t)stream);
+}
+
+zero_status zero_stage3_step_fused_q8_dc(const zero_plan* plan, uint64_t flat_lo, uint64_t len,
+                                         const uint8_t* const* rank_payload,
+                                         const float* master_in, const float* m_in,
+                                         const float* v_in, float* master_out, float* m_out,
+                                         float* v_out, uint16_t* const* param_shards,
+                                         const zero_adam_consts* d_consts, uint32_t* d_status,
+                                         zero_stream_t stream) {
+    if (!d_consts) return ZERO_EINVAL;
+    if (!zk::aligned(d_consts, 4)) return ZERO_EALIGN;
+    zero_adam_consts unused;
+    memset(&unused, 0, sizeof(unused));
+    return stage3_fused_q8(plan, flat_lo, len, rank_payload, master_in, m_in, v_in, master_out,
+                           m_out, v_out, param_shards, unused, d_consts, d_status,
+                           (cudaStream_t)stream);
 }
 
 zero_status zero_stage3_step_commit(const zero_plan* plan, const float* master_in, const float* m_in,

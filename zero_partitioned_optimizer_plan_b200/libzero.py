@@ -51,7 +51,7 @@ SYMBOLS = (
     "zero_overlap_begin", "zero_overlap_end",
     "zero_gather_params", "zero_stage3_step_fused", "zero_stage3_step_commit",
     "zero_stage3_step_fused_dc", "zero_stage3_payload_bytes_q8", "zero_stage3_quantize_q8",
-    "zero_stage3_step_fused_q8",
+    "zero_stage3_step_fused_q8", "zero_stage3_step_fused_q8_dc",
     "zero_step_fused_ranges", "zero_step_fused_q8_ranges",
     "zero_step_fused_replicas", "zero_step_commit_replicas",
     "zero_sched_slot_elems", "zero_sched_create", "zero_sched_create_fused",
@@ -188,6 +188,8 @@ def _load():
     L.zero_stage3_quantize_q8.argtypes = [vp, u64, u64, vp, vp, vp]
     L.zero_stage3_step_fused_q8.argtypes = [vp, u64, u64, P(vp), vp, vp, vp, vp, vp, vp, P(vp),
                                             P(_HP), i64, vp, vp]
+    L.zero_stage3_step_fused_q8_dc.argtypes = [vp, u64, u64, P(vp), vp, vp, vp, vp, vp, vp,
+                                               P(vp), vp, vp, vp]
     L.zero_overlap_begin.argtypes = [vp]
     L.zero_overlap_end.argtypes = [vp]
     L.zero_sched_slot_elems.argtypes = [vp, i32, P(u64)]
@@ -572,6 +574,18 @@ def zero_stage3_step_fused_q8(plan: Plan, flat_lo: int, length: int, rank_payloa
                                           _ptr_array(param_shards, 2), C.byref(h), step,
                                           _ptr(d_status, 4), _stream(stream)),
            "zero_stage3_step_fused_q8")
+
+
+def zero_stage3_step_fused_q8_dc(plan: Plan, flat_lo: int, length: int, rank_payload,
+                                 master_in, m_in, v_in, master_out, m_out, v_out, param_shards,
+                                 d_consts, d_status, stream=None):
+    _check(_lib.zero_stage3_step_fused_q8_dc(plan.handle, flat_lo, length,
+                                             _ptr_array(rank_payload, 1), _ptr(master_in, 4),
+                                             _ptr(m_in, 4), _ptr(v_in, 4), _ptr(master_out, 4),
+                                             _ptr(m_out, 4), _ptr(v_out, 4),
+                                             _ptr_array(param_shards, 2), _ptr(d_consts),
+                                             _ptr(d_status, 4), _stream(stream)),
+           "zero_stage3_step_fused_q8_dc")
 
 
 class PreparedStage3Update:
