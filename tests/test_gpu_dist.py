@@ -176,7 +176,7 @@ def test_distributed_step_all_gather_in_epilogue_one_rank_nccl(bucket, peer):
     assert int(oracle.ulp_diff_f16(params, ref.params16).max()) == 0
 
 
-def _worker_stage3(port, numels, layer_tensors, out):
+def _worker_stage3(port, numels, layer_tensors, out, payload="fp16"):
     import datetime
     import torch
     import torch.distributed as dist
@@ -197,7 +197,7 @@ def _worker_stage3(port, numels, layer_tensors, out):
         st_in = [x.to(dev) for x in (master, m, v)]
         st_out = [torch.full_like(x, float("nan")) for x in st_in]
         status = torch.zeros(1, dtype=torch.int32, device=dev)
-        step = DistStage3Step(numels, layer_tensors, parts)
+        step = DistStage3Step(numels, layer_tensors, parts, payload=payload)
         layer_buf = torch.zeros(max(hi - lo for lo, hi in step.layers), dtype=torch.float16,
                                 device=dev)
         rec = []
@@ -210,16 +210,18 @@ def _worker_stage3(port, numels, layer_tensors, out):
         dist.destroy_process_group()
 
 
-def test_distributed_stage3_one_rank_nccl():
+@pytest.mark.parametrize("payload", ["fp16", "q8"])
+def test_distributed_stage3_one_rank_nccl(payload):
     """DistStage3Step on one NCCL rank: the partition in torch symmetric memory, each layer
     gathered by the library's gather kernel from the owner's partition address, the layers'
-    gradient buckets exchanged and the owner's update written into its partition; gathered
-    layers, partition and state against the oracle's zero3_step (0 ulp)."""
+    gradient buckets exchanged (fp16, or int8 records quantized by the library) and the owner's
+    update written into its partition; gathered layers, partition and state against the
+    oracle's zero3_step, or its quantizer and int8 step per bucket (0 ulp)."""
     import oracle
     numels, layer_tensors = [1000, 37, 4099, 12345], [1, 2, 1]
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    p = ctx.Process(target=_worker_stage3, args=(_free_port(), numels, layer_tensors, q))
+    p = ctx.Process(target=_worker_stage3, args=(_free_port(), numels, layer_tensors, q, payload))
     p.start()
     try:
         flag, status, shard, part, rec = q.get(timeout=240)
@@ -236,9 +238,19 @@ def test_distributed_stage3_one_rank_nccl():
                             master.numpy(), m.numpy(), v.numpy(),
                             [oracle.f2h(master.numpy())], oracle.AdamHP(), 1)
     assert (flag, status) == (0, 0) and not ref.skipped
-    for name, got, want in zip(("master", "m", "v"), shard, (ref.master, ref.m, ref.v)):
+    want_state, want_part = (ref.master, ref.m, ref.v), ref.param_shards[0]
+    if payload == "q8":                  # one owner: each layer bucket is one int8 part
+        w, mm, vv = master.numpy().copy(), m.numpy().copy(), v.numpy().copy()
+        p16 = oracle.f2h(master.numpy())
+        for lo, hi in buckets:
+            qq, sc = oracle.quant_q8(grad.numpy()[lo:hi])
+            sk, w[lo:hi], mm[lo:hi], vv[lo:hi], p16[lo:hi] = oracle.step_q8(
+                [qq], [sc], w[lo:hi], mm[lo:hi], vv[lo:hi], oracle.AdamHP(), 1)
+            assert not sk
+        want_state, want_part = (w, mm, vv), p16
+    for name, got, want in zip(("master", "m", "v"), shard, want_state):
         assert int(oracle.ulp_diff_f32(got, want).max()) == 0, name
-    assert int(oracle.ulp_diff_f16(part, ref.param_shards[0]).max()) == 0
+    assert int(oracle.ulp_diff_f16(part, want_part).max()) == 0
     L = len(layers)
     for l in range(L):
         assert np.array_equal(rec[l], ref.gathered_fwd[l])

@@ -689,7 +689,7 @@ S3_NUMELS = [1000, 37, 4099, 12345, 6000, 7]
 S3_LAYERS = [1, 2, 1, 2]
 
 
-def _worker_stage3(rank, ws, port, bad_rank, pbufs, gbufs, out):
+def _worker_stage3(rank, ws, port, bad_rank, pbufs, gbufs, out, payload="fp16"):
     import datetime
     import numpy as np
     import torch
@@ -710,13 +710,15 @@ def _worker_stage3(rank, ws, port, bad_rank, pbufs, gbufs, out):
         peers = None
         if gbufs is not None:      # gradients read in place from the peers' buffers
             peers = SharedPeerBuffers(gbufs, rank)
-            peers.local.copy_(grads[rank])
-        step = DistStage3Step(S3_NUMELS, S3_LAYERS, parts, compute=_OracleCompute(), peers=peers)
+            if payload == "fp16":
+                peers.local.copy_(grads[rank])
+        step = DistStage3Step(S3_NUMELS, S3_LAYERS, parts, compute=_OracleCompute(), peers=peers,
+                              payload=payload)
         big = max(hi - lo for lo, hi in step.layers)
         layer_buf = torch.zeros(big, dtype=torch.float16)
         rec = []
-        flag = step.step(peers.local if peers is not None else grads[rank], st_in, st_out,
-                         oracle.AdamHP(), 1, status, layer_buf, rec)
+        local = peers.local if peers is not None and payload == "fp16" else grads[rank]
+        flag = step.step(local, st_in, st_out, oracle.AdamHP(), 1, status, layer_buf, rec)
         dist.barrier()    # every owner's partition is final before it is read back
         out.put((rank, int(flag.item()), int(status.item()), [x.numpy() for x in st_out],
                  [p.numpy().view(np.uint16).copy() for p in parts.tensors],
@@ -778,3 +780,68 @@ def test_distributed_stage3_gloo(ws, bad_rank, peer):
         for l in range(L):
             assert np.array_equal(rec[l], ref.gathered_fwd[l])
             assert np.array_equal(rec[L + (L - 1 - l)], ref.gathered_bwd[l])
+
+
+@pytest.mark.parametrize("peer", [False, True])
+@pytest.mark.parametrize("ws,bad_rank", [(2, -1), (3, 1)])
+def test_distributed_stage3_int8_gloo(ws, bad_rank, peer):
+    """DistStage3Step with the int8 payload on gloo ranks (the layers' gradient buckets
+    exchanged, or read from the peers' buffers, as int8 records): every owner's partition and
+    state shard against the oracle's quantizer and int8 step over the (layer bucket, owner)
+    parts, bit for bit; an inf on one rank skips the step everywhere."""
+    import numpy as np
+    import torch
+    import oracle
+    from zero_partitioned_optimizer_plan_b200.dist import q8_peer_layout
+    psi_p, grads, master, m, v = _dist_case(S3_NUMELS, ws, bad_rank)
+    S = psi_p // ws
+    p16 = oracle.f2h(master.numpy())
+    pbufs = [torch.from_numpy(p16[q * S:(q + 1) * S].copy().view(np.int16)).view(torch.float16)
+             .share_memory_() for q in range(ws)]
+    pl = oracle.plan(S3_NUMELS, ws)
+    layers = oracle.layer_ranges(pl, S3_LAYERS)
+    buckets = oracle.grad_buckets(pl, layers)
+    gbufs = None
+    if peer:
+        _, need = q8_peer_layout(psi_p, 0, ws, buckets[::-1])
+        gbufs = [torch.zeros(need, dtype=torch.uint8).share_memory_() for _ in range(ws)]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_stage3,
+                         args=(r, ws, port, bad_rank, pbufs, gbufs, q, "q8"))
+             for r in range(ws)]
+    for p in procs:
+        p.start()
+    try:
+        res = sorted((q.get(timeout=240) for _ in range(ws)), key=lambda x: x[0])
+    finally:
+        for p in procs:
+            p.join(60)
+            if p.exitcode is None:
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    w, mm, vv = master.numpy().copy(), m.numpy().copy(), v.numpy().copy()
+    pw = p16.copy()
+    skipped = False
+    for lo, hi in buckets:
+        for o in range(ws):
+            a, b = max(lo, o * S), min(hi, (o + 1) * S)
+            if a >= b:
+                continue
+            pay = [oracle.quant_q8(g.numpy()[a:b]) for g in grads]
+            sk, wn, mn, vn, pn = oracle.step_q8([x for x, _ in pay], [c for _, c in pay],
+                                                w[a:b], mm[a:b], vv[a:b], oracle.AdamHP(), 1)
+            skipped |= sk
+            if not sk:
+                w[a:b], mm[a:b], vv[a:b], pw[a:b] = wn, mn, vn, pn
+    if skipped:
+        w, mm, vv, pw = master.numpy(), m.numpy(), v.numpy(), p16
+    assert skipped == (bad_rank >= 0)
+    for rank, flag, status, shard, parts, rec in res:
+        assert flag == (1 if skipped else 0)
+        assert bool(status & 2) == skipped
+        for got, want in zip(shard, (w, mm, vv)):
+            assert np.array_equal(got.view(np.uint32), want[rank * S:(rank + 1) * S].view(np.uint32))
+        for qq in range(ws):
+            assert np.array_equal(parts[qq], pw[qq * S:(qq + 1) * S].view(np.uint16))

@@ -499,10 +499,11 @@ class DistStage3Step:
     exchanges and updates, which touch other layers' ranges); the job-wide verdict;
     nothing is gathered after the step. The gathered layer goes to ``layer_buf`` (the buffer
     the layer's computation would read); ``record`` (a list) receives a copy of each gathered
-    layer, forward then backward, for checking."""
+    layer, forward then backward, for checking. ``payload="q8"``: each layer's gradient bucket
+    travels as int8 records (the exchange or the peer reads of DistZeroStep's int8 forms)."""
 
     def __init__(self, numels: Sequence[int], layer_tensors: Sequence[int], part_peers,
-                 group=None, compute=None, peers=None):
+                 group=None, compute=None, peers=None, payload: str = "fp16"):
         import torch.distributed as dist
         self.dist = dist
         self.numels = list(numels)
@@ -515,7 +516,7 @@ class DistStage3Step:
         grad_buckets[-1] = (grad_buckets[-1][0], self.psi_p)
         self.part_peers = part_peers
         self.compute = compute or LibzeroCompute()
-        self.inner = DistZeroStep(self.psi_p, 0, group, self.compute, peers,
+        self.inner = DistZeroStep(self.psi_p, 0, group, self.compute, peers, payload=payload,
                                   buckets=grad_buckets[::-1], partitioned=True)
 
     def gather(self, l: int, layer_buf, status):
