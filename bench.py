@@ -3,8 +3,10 @@
 the measured HBM roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload zero2_1p3b|gpt2_small|shard_7p5b|flat|zero2_gpt2_small]
-                    [--stage2 fused|unfused] [--nd ND] [--bucket B] [--no-sweep]
+                    [--workload zero2_1p3b|zero2_gpt2_small|zero3_gpt2_small|zero3_1p3b|
+                                gpt2_small|tiny|shard_7p5b|flat]
+                    [--stage2 fused|unfused] [--payload fp16|q8] [--graph] [--nd ND]
+                    [--bucket B] [--layer-buffers L] [--no-sweep]
 
 One step is one pass of the whole hot path over one batch of synthetic input: the
 reduce-scatter of the Nd simulated ranks' fp16 gradients, the unscale, the fp32 Adam update of
@@ -34,6 +36,12 @@ Workloads (synthetic, seeded):
               r*S (r = 31); master U(-0.05, 0.05), m N(0, 1e-4^2), v |N(0, 1e-6^2)|.
   flat        psi = 2^29 flat buffer, one fused call per bucket of B elements in backward
               order, Nd in {2, 4, 8, 16, 64}; state as shard_7p5b.
+  tiny        the 2^20-value stage-1 case (4 tensors, Nd = 4), L2-resident.
+
+--payload q8: the owners reduce int8 records (128 values and their fp32 scale) instead of fp16
+gradients, quantized once before timing (stage 1, flat, the 7.5B view, stage 2 through the
+int8 bucket scheduler, stage 3 per owner part). --graph: each step is one CUDA-graph replay
+(the step's constants read from device memory).
 
 The default line also carries the bucket / Nd sweep ("sweep" in config: the flat workload at
 Nd in {2, 4, 8, 16, 64} with 128 MiB buckets, each point timed the same way; --no-sweep skips
