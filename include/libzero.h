@@ -455,7 +455,9 @@ zero_status zero_stage3_step_commit(const zero_plan* plan, const float* master_i
  * outlive the scheduler; one host thread at a time may use it. A step can be captured into a
  * CUDA graph (with zero_stage3_step_fused_dc for the updates): capture it on one stream, pass
  * that stream to begin_step, acquire and release, so that the gather stream joins the capture
- * through begin_step's event and every wait stays inside the capture. The pages have no
+ * through begin_step's event and every wait stays inside the capture; acquire every layer the
+ * captured step prefetches (an unused prefetch's gather would not be joined back into the
+ * capturing stream, and CUDA refuses to end such a capture). The pages have no
  * scheduler interface; this is the library's runtime for the stage-3 data path.
  * Errors: ZERO_EINVAL (bad plan or bounds, null pointers, an acquire before the first
  * begin_step, a layer out of range or already acquired, release of a layer not acquired,
