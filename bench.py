@@ -1176,19 +1176,38 @@ def host_cpu() -> dict:
     return {"cpu": model, "threads": os.cpu_count()}
 
 
-def cpu_oracle_rate(nd: int, n_sample: int, target_s: float, seed=0):
-    """Time the oracle (single-threaded C, as it stands) on n_sample elements of the workload's
-    distribution; repeat until target_s seconds have passed. Returns (params/s, reps, secs)."""
+def oracle_sample(nd: int, n: int, payload: str = "fp16", seed=0):
+    """The oracle's owner step on n elements of the workload's distribution: a function
+    step(master, m, v, t) -> (master, m, v) and the initial state. With the int8 payload the
+    ranks' records are quantized once here (the senders' part), the step reduces them."""
     import oracle
     from zero_partitioned_optimizer_plan_b200 import synth
-    g = [synth.grad_f16(n_sample, 1e-3, seed=seed, rank=r, step=1, spike_frac=0.01,
+    g = [synth.grad_f16(n, 1e-3, seed=seed, rank=r, step=1, spike_frac=0.01,
                         spike_scale=100.0).numpy() for r in range(nd)]
-    master, m, v = (x.numpy() for x in synth.state_small(n_sample, seed=seed))
+    state = tuple(x.numpy() for x in synth.state_small(n, seed=seed))
     hp = oracle.AdamHP()
+    if payload == "q8":
+        q = [oracle.quant_q8(x) for x in g]
+        qs, scs = [a for a, _ in q], [b for _, b in q]
+
+        def step(w, mm, vv, t):
+            _, w, mm, vv, _ = oracle.step_q8(qs, scs, w, mm, vv, hp, t)
+            return w, mm, vv
+    else:
+        def step(w, mm, vv, t):
+            _, w, mm, vv, _ = oracle.step(g, w, mm, vv, hp, t)
+            return w, mm, vv
+    return step, state
+
+
+def cpu_oracle_rate(nd: int, n_sample: int, target_s: float, seed=0, payload: str = "fp16"):
+    """Time the oracle (single-threaded C, as it stands) on n_sample elements of the workload's
+    distribution; repeat until target_s seconds have passed. Returns (params/s, reps, secs)."""
+    step, (master, m, v) = oracle_sample(nd, n_sample, payload, seed)
     reps, total = 0, 0.0
     while total < target_s and reps < 50:
         t0 = time.perf_counter()
-        skipped, master, m, v, _ = oracle.step(g, master, m, v, hp, reps + 1)
+        master, m, v = step(master, m, v, reps + 1)
         total += time.perf_counter() - t0
         reps += 1
     return n_sample * reps / total, reps, total
@@ -1362,24 +1381,21 @@ def run_reference(args):
     cfg = workload_config(args)
     nd = cfg["nd"]
     # calibrate, then size each step so that the whole run takes about two minutes
-    rate, _, _ = cpu_oracle_rate(nd, 200_000, 0.2)
+    payload = getattr(args, "payload", "fp16")
+    rate, _, _ = cpu_oracle_rate(nd, 200_000, 0.2, payload=payload)
     per_step_s = max(0.05, 120.0 / (args.steps + args.warmup))
     n_sample = int(min(16_000_000, max(100_000, rate * per_step_s)))
-    import oracle
-    from zero_partitioned_optimizer_plan_b200 import synth
-    g = [synth.grad_f16(n_sample, 1e-3, seed=0, rank=r, step=1, spike_frac=0.01,
-                        spike_scale=100.0).numpy() for r in range(nd)]
-    master, m, v = (x.numpy() for x in synth.state_small(n_sample, seed=0))
-    hp = oracle.AdamHP()
+    step, (master, m, v) = oracle_sample(nd, n_sample, payload)
     for t in range(1, args.warmup + 1):
-        _, master, m, v, _ = oracle.step(g, master, m, v, hp, t)
+        master, m, v = step(master, m, v, t)
     t0 = time.perf_counter()
     for t in range(args.warmup + 1, args.warmup + args.steps + 1):
-        _, master, m, v, _ = oracle.step(g, master, m, v, hp, t)
+        master, m, v = step(master, m, v, t)
     dt = time.perf_counter() - t0
     value = n_sample * args.steps / dt
     sample = (f"first {n_sample} elements of the {cfg['workload']} workload's gradient "
-              f"distribution, Nd={nd}, one oracle step per timed step")
+              f"distribution, Nd={nd}, one oracle step per timed step"
+              + (" (int8 records quantized once before timing)" if payload == "q8" else ""))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "params/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -1514,11 +1530,13 @@ def run_ours(args):
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         n_sample = 8_000_000
-        rate, reps, secs = cpu_oracle_rate(wl.nd, n_sample, 10.0)
+        rate, reps, secs = cpu_oracle_rate(wl.nd, n_sample, 10.0, payload=wl.payload)
+        what = ("the oracle's int8 owner step, records quantized once before timing"
+                if wl.payload == "q8" else "the oracle's step is the same element arithmetic "
+                "for every stage and bucketing")
         cpu = {"value": rate, "unit": "params/s", "cores": 1, "kind": "oracle",
                "sample": f"{n_sample} elements with the workload's gradient distribution, "
-                         f"Nd={wl.nd}, {reps} oracle steps, {secs:.1f} s (the oracle's step "
-                         "is the same element arithmetic for every stage and bucketing)",
+                         f"Nd={wl.nd}, {reps} oracle steps, {secs:.1f} s ({what})",
                "host": host_cpu()}
 
     main_line = wl.config["workload"].startswith("zero2_1p3b") and args.stage2 == "fused" and \
